@@ -1,0 +1,357 @@
+/*
+ * ORACLE -- test infrastructure only.
+ *
+ * A plain, slow, obviously-correct CPU restatement of one routed
+ * Mixture-of-Experts layer over a slot-indexed expert cache.  Only the tests,
+ * the smoke check and the CPU-baseline leg of the benchmark load this file; the
+ * product path never does, and it shares no code with the CUDA kernels.
+ *
+ * Sources (FreeToken web pages):
+ *  - chenxutan.com FreeToken article, section "why the bottleneck is bandwidth,
+ *    not capacity": each token activates a few routed experts (6 per token for
+ *    the 284B model); the expert pool stays in host memory and experts are
+ *    pulled into VRAM on demand.
+ *  - same article, section "choosing among the five MoE backends", item
+ *    `offload`: experts in host RAM, a set of LRU slots in VRAM, misses over PCIe.
+ *  - claypier.com "FreeToken MoE edge runtime", first section: only the
+ *    experts needed now are moved into VRAM and a global LRU cache evicts the
+ *    ones unused for a while.
+ *  - pomoai.com FreeToken hub, checkpoint list: MXFP4, NVFP4, FP8 and BF16
+ *    weight formats.
+ * The pages give no formula for the layer; the arithmetic below is the plain
+ * reading of a top-k routed SwiGLU MoE layer (router logits + bias, softmax,
+ * top-k, renormalise over the k picks, SwiGLU experts, gate-weighted sum), with
+ * every silent point resolved as listed in the design notes.
+ *
+ * Precision: products and sums in double, results rounded to float.
+ * Parallelism: OpenMP over independent tokens/rows only (no reordering of any
+ * sum).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+int orc_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/* ---------------------------------------------------------------------------
+ * Number formats (OCP 8-bit floating point spec, E4M3; OCP MX spec, E2M1).
+ * ------------------------------------------------------------------------- */
+
+float orc_bf16_to_f32(uint16_t v) {
+  uint32_t u = (uint32_t)v << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+/* E4M3: 1 sign, 4 exponent bits (bias 7), 3 mantissa bits; exponent 0 is
+ * subnormal (m * 2^-9); S.1111.111 is NaN; no infinities.  Max finite 448. */
+double orc_e4m3_value(uint8_t q) {
+  int sgn = (q >> 7) & 1, e = (q >> 3) & 15, m = q & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0) v = m * pow(2.0, -9);
+  else v = (1.0 + m / 8.0) * pow(2.0, e - 7);
+  return sgn ? -v : v;
+}
+
+/* E2M1: 1 sign, 2 exponent bits (bias 1), 1 mantissa bit; values
+ * {0, 0.5, 1, 1.5, 2, 3, 4, 6}. */
+double orc_e2m1_value(uint8_t nib) {
+  int sgn = (nib >> 3) & 1, e = (nib >> 1) & 3, m = nib & 1;
+  double v = (e == 0) ? 0.5 * m : (1.0 + 0.5 * m) * pow(2.0, e - 1);
+  return sgn ? -v : v;
+}
+
+static double orc_e4m3_table[127];       /* values of codes 0x00 .. 0x7E */
+
+__attribute__((constructor)) static void orc_init_tables(void) {
+  for (int c = 0; c < 127; ++c) orc_e4m3_table[c] = orc_e4m3_value((uint8_t)c);
+}
+
+/* Round to the nearest finite E4M3 value, ties to the code with an even
+ * mantissa, magnitudes beyond 448 saturate to 448.  Done by exhaustive search
+ * over the 127 non-negative finite codes. */
+uint8_t orc_e4m3_encode(float v) {
+  double a = fabs((double)v);
+  int best = 0;
+  double bd = INFINITY;
+  for (int c = 0; c < 127; ++c) {         /* 0x00 .. 0x7E */
+    double dd = fabs(a - orc_e4m3_table[c]);
+    if (dd < bd || (dd == bd && (c & 1) == 0)) { bd = dd; best = c; }
+  }
+  if (best == 0) return 0;
+  return (uint8_t)((v < 0.0f ? 0x80 : 0) | best);
+}
+
+/* Round to the nearest E2M1 value, ties to the even code, saturating at 6. */
+uint8_t orc_e2m1_encode(float v) {
+  double a = fabs((double)v);
+  int best = 0;
+  double bd = INFINITY;
+  for (int c = 0; c < 8; ++c) {
+    double dd = fabs(a - orc_e2m1_value((uint8_t)c));
+    if (dd < bd || (dd == bd && (c & 1) == 0)) { bd = dd; best = c; }
+  }
+  if (best == 0) return 0;
+  return (uint8_t)((v < 0.0f ? 0x8 : 0) | best);
+}
+
+/* ---------------------------------------------------------------------------
+ * Weight dequantisation: the dequantised weight is the layer's ground truth.
+ * ------------------------------------------------------------------------- */
+
+void orc_dequant_bf16(const uint16_t* w, int64_t n, float* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_bf16_to_f32(w[i]);
+}
+
+/* FP8 with one fp32 scale per 128x128 block: w[r][c] = e4m3(q[r][c]) * s[r/128][c/128]. */
+void orc_dequant_fp8_b128(const uint8_t* q, const float* s, int R, int C, float* out) {
+  int CB = C / 128;
+  for (int r = 0; r < R; ++r)
+    for (int c = 0; c < C; ++c)
+      out[(int64_t)r * C + c] =
+          (float)(orc_e4m3_value(q[(int64_t)r * C + c]) * (double)s[(r / 128) * CB + c / 128]);
+}
+
+/* NVFP4: w[r][c] = e2m1(q) * e4m3(s16[r][c/16]) * s_t, two codes per byte
+ * along c, element 2j in the low nibble. */
+void orc_dequant_nvfp4(const uint8_t* qp, const uint8_t* s16, float s_t, int R, int C, float* out) {
+  for (int r = 0; r < R; ++r)
+    for (int c = 0; c < C; ++c) {
+      uint8_t byte = qp[(int64_t)r * (C / 2) + c / 2];
+      uint8_t nib = (c & 1) ? (byte >> 4) : (byte & 15);
+      double sc = orc_e4m3_value(s16[(int64_t)r * (C / 16) + c / 16]);
+      out[(int64_t)r * C + c] = (float)(orc_e2m1_value(nib) * sc * (double)s_t);
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * Activation quantisation (the tensor-core FP8 / NVFP4 paths quantise the
+ * hidden state and the SwiGLU output before their contractions; the oracle
+ * applies the same declared quantiser).  In place: each value is replaced by
+ * its quantised-then-dequantised value.  All scale arithmetic in fp32.
+ * ------------------------------------------------------------------------- */
+
+/* FP8: groups of 128 consecutive elements of a row; s = amax/448;
+ * v <- e4m3(v / s) * s; an all-zero group stays zero. */
+void orc_qa_fp8_g128(float* v, int rows, int K) {
+  for (int r = 0; r < rows; ++r)
+    for (int g = 0; g < K / 128; ++g) {
+      float* p = v + (int64_t)r * K + g * 128;
+      float amax = 0.0f;
+      for (int j = 0; j < 128; ++j) if (fabsf(p[j]) > amax) amax = fabsf(p[j]);
+      float s = amax / 448.0f;
+      for (int j = 0; j < 128; ++j) {
+        if (s == 0.0f) { p[j] = 0.0f; continue; }
+        float qv = p[j] / s;
+        p[j] = (float)(orc_e4m3_value(orc_e4m3_encode(qv)) * (double)s);
+      }
+    }
+}
+
+/* NVFP4 activations: groups of 16 consecutive elements of a row;
+ * s16 = e4m3(amax/6) (per-tensor scale 1); v <- e2m1(v / s16) * s16. */
+void orc_qa_nvfp4_g16(float* v, int rows, int K) {
+  for (int r = 0; r < rows; ++r)
+    for (int g = 0; g < K / 16; ++g) {
+      float* p = v + (int64_t)r * K + g * 16;
+      float amax = 0.0f;
+      for (int j = 0; j < 16; ++j) if (fabsf(p[j]) > amax) amax = fabsf(p[j]);
+      float s = (float)orc_e4m3_value(orc_e4m3_encode(amax / 6.0f));
+      for (int j = 0; j < 16; ++j) {
+        if (s == 0.0f) { p[j] = 0.0f; continue; }
+        float qv = p[j] / s;
+        p[j] = (float)(orc_e2m1_value(orc_e2m1_encode(qv)) * (double)s);
+      }
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * Router: logits, top-k, gates.
+ * ------------------------------------------------------------------------- */
+
+/* logits[t][e] = sum_i x[t][i] * Wr[e][i] + b[e]  (double sum, rounded to float). */
+void orc_router_logits(const float* x, int T, int d, const float* Wr, const float* b, int E, float* logits) {
+#pragma omp parallel for schedule(static)
+  for (int t = 0; t < T; ++t)
+    for (int e = 0; e < E; ++e) {
+      double acc = 0.0;
+      for (int i = 0; i < d; ++i) acc += (double)x[(int64_t)t * d + i] * (double)Wr[(int64_t)e * d + i];
+      if (b) acc += (double)b[e];
+      logits[(int64_t)t * E + e] = (float)acc;
+    }
+}
+
+/* order[0..E) = expert ids sorted by logit descending, equal logits by id ascending. */
+static void orc_sort_desc(const float* l, int E, int* order) {
+  for (int e = 0; e < E; ++e) order[e] = e;
+  for (int i = 1; i < E; ++i) {          /* insertion sort: stable on id */
+    int v = order[i], j = i - 1;
+    while (j >= 0 && l[order[j]] < l[v]) { order[j + 1] = order[j]; --j; }
+    order[j + 1] = v;
+  }
+}
+
+/* ok[t] = 1 iff every gap among the top-(k+1) sorted logits is >= margin
+ * (the synthetic inputs are redrawn until this holds, so the pick set and
+ * pick order are unique). */
+void orc_margin_ok(const float* logits, int T, int E, int k, double margin, uint8_t* ok) {
+  int* order = (int*)malloc(sizeof(int) * E);
+  for (int t = 0; t < T; ++t) {
+    const float* l = logits + (int64_t)t * E;
+    orc_sort_desc(l, E, order);
+    int last = (k < E) ? k : E - 1;
+    ok[t] = 1;
+    for (int r = 0; r < last; ++r)
+      if ((double)l[order[r]] - (double)l[order[r + 1]] < margin) ok[t] = 0;
+  }
+  free(order);
+}
+
+/* ids[t][j] = j-th largest logit's expert; gates: softmax over all E experts,
+ * then renormalised over the k picks: g_j = p[id_j] / sum_j' p[id_j']. */
+void orc_topk_gates(const float* logits, int T, int E, int k, int32_t* ids, float* gates) {
+  int* order = (int*)malloc(sizeof(int) * E);
+  double* p = (double*)malloc(sizeof(double) * E);
+  for (int t = 0; t < T; ++t) {
+    const float* l = logits + (int64_t)t * E;
+    orc_sort_desc(l, E, order);
+    double m = l[order[0]], z = 0.0;
+    for (int e = 0; e < E; ++e) { p[e] = exp((double)l[e] - m); z += p[e]; }
+    for (int e = 0; e < E; ++e) p[e] /= z;
+    double zk = 0.0;
+    for (int j = 0; j < k; ++j) zk += p[order[j]];
+    for (int j = 0; j < k; ++j) {
+      ids[(int64_t)t * k + j] = order[j];
+      gates[(int64_t)t * k + j] = (float)(p[order[j]] / zk);
+    }
+  }
+  free(p);
+  free(order);
+}
+
+/* ---------------------------------------------------------------------------
+ * Permutation of the P = T*k (token, pick) pairs by expert.
+ * counts[e] = #pairs routed to e; offsets[e] = exclusive prefix sum (offsets[E] = P);
+ * pairs are visited in ascending flat index q = t*k + j and placed at
+ * pos = offsets[e] + (number of earlier pairs with the same expert);
+ * perm[pos] = q, inv[q] = pos.
+ * ------------------------------------------------------------------------- */
+void orc_permute(const int32_t* ids, int T, int k, int E, int32_t* counts, int32_t* offsets,
+                 int32_t* perm, int32_t* inv) {
+  int64_t P = (int64_t)T * k;
+  for (int e = 0; e < E; ++e) counts[e] = 0;
+  for (int64_t q = 0; q < P; ++q) counts[ids[q]]++;
+  offsets[0] = 0;
+  for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+  int32_t* run = (int32_t*)calloc((size_t)E, sizeof(int32_t));
+  for (int64_t q = 0; q < P; ++q) {
+    int e = ids[q];
+    int32_t pos = offsets[e] + run[e]++;
+    perm[pos] = (int32_t)q;
+    inv[q] = pos;
+  }
+  free(run);
+}
+
+/* ---------------------------------------------------------------------------
+ * LRU slot cache step.
+ * State: slot_of_expert[E] (-1: not resident), expert_of_slot[S] (-1: empty),
+ * last_use[S] (-1: never).  Step s requests the distinct expert ids in
+ * ids[0..n).  Hits: last_use = s.  Misses, in ascending expert id, each take
+ * the slot with the smallest last_use among slots with last_use < s (ties: the
+ * lowest slot index), unmapping its previous expert.  Returns 0 on success,
+ * -1 (state untouched) when more distinct experts are requested than slots.
+ * miss_expert/miss_slot list the misses in the order they were placed.
+ * ------------------------------------------------------------------------- */
+int orc_lru_step(int E, int S, int32_t* slot_of_expert, int32_t* expert_of_slot, int64_t* last_use,
+                 int64_t s, const int32_t* ids, int n, int32_t* miss_expert, int32_t* miss_slot,
+                 int32_t* n_distinct, int32_t* n_hits, int32_t* n_miss) {
+  uint8_t* want = (uint8_t*)calloc((size_t)E, 1);
+  for (int i = 0; i < n; ++i) want[ids[i]] = 1;
+  int distinct = 0;
+  for (int e = 0; e < E; ++e) distinct += want[e];
+  *n_distinct = distinct;
+  if (distinct > S) { free(want); *n_hits = 0; *n_miss = 0; return -1; }
+  int hits = 0, misses = 0;
+  for (int e = 0; e < E; ++e)
+    if (want[e] && slot_of_expert[e] >= 0) { last_use[slot_of_expert[e]] = s; ++hits; }
+  for (int e = 0; e < E; ++e) {
+    if (!want[e] || slot_of_expert[e] >= 0) continue;
+    int victim = -1;
+    for (int j = 0; j < S; ++j)
+      if (last_use[j] < s && (victim < 0 || last_use[j] < last_use[victim])) victim = j;
+    /* victim >= 0 is guaranteed by distinct <= S */
+    if (expert_of_slot[victim] >= 0) slot_of_expert[expert_of_slot[victim]] = -1;
+    expert_of_slot[victim] = e;
+    slot_of_expert[e] = victim;
+    last_use[victim] = s;
+    miss_expert[misses] = e;
+    miss_slot[misses] = victim;
+    ++misses;
+  }
+  *n_hits = hits;
+  *n_miss = misses;
+  free(want);
+  return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Expert FFN (SwiGLU) over n rows, and the combine.
+ * h[i] = silu(x . Wg[i]) * (x . Wu[i]),  silu(z) = z / (1 + exp(-z));
+ * y[j] = h . Wd[j].
+ * qa = 0: no activation quantisation; 1: FP8 (128-groups) on x and h;
+ * 2: NVFP4 (16-groups) on x and h.
+ * ------------------------------------------------------------------------- */
+void orc_expert_ffn(const float* x, int n, int d, int I, const float* Wg, const float* Wu,
+                    const float* Wd, int qa, float* y) {
+#pragma omp parallel for schedule(dynamic)
+  for (int r = 0; r < n; ++r) {
+    float* xr = (float*)malloc(sizeof(float) * d);
+    float* h = (float*)malloc(sizeof(float) * I);
+    memcpy(xr, x + (int64_t)r * d, sizeof(float) * d);
+    if (qa == 1) orc_qa_fp8_g128(xr, 1, d);
+    if (qa == 2) orc_qa_nvfp4_g16(xr, 1, d);
+    for (int i = 0; i < I; ++i) {
+      double g = 0.0, u = 0.0;
+      for (int c = 0; c < d; ++c) {
+        g += (double)xr[c] * (double)Wg[(int64_t)i * d + c];
+        u += (double)xr[c] * (double)Wu[(int64_t)i * d + c];
+      }
+      h[i] = (float)(g / (1.0 + exp(-g)) * u);
+    }
+    if (qa == 1) orc_qa_fp8_g128(h, 1, I);
+    if (qa == 2) orc_qa_nvfp4_g16(h, 1, I);
+    for (int j = 0; j < d; ++j) {
+      double acc = 0.0;
+      for (int i = 0; i < I; ++i) acc += (double)h[i] * (double)Wd[(int64_t)j * I + i];
+      y[(int64_t)r * d + j] = (float)acc;
+    }
+    free(h);
+    free(xr);
+  }
+}
+
+/* out[t] = sum_{j=0..k-1, ascending} g[t][j] * y[t*k + j]  (+ ysh[t] if given);
+ * y rows here are in pair order q = t*k + j. */
+void orc_combine(const float* y, const float* gates, int T, int k, int d, const float* ysh, float* out) {
+  for (int t = 0; t < T; ++t)
+    for (int c = 0; c < d; ++c) {
+      double acc = 0.0;
+      for (int j = 0; j < k; ++j)
+        acc += (double)gates[(int64_t)t * k + j] * (double)y[((int64_t)t * k + j) * d + c];
+      if (ysh) acc += (double)ysh[(int64_t)t * d + c];
+      out[(int64_t)t * d + c] = (float)acc;
+    }
+}

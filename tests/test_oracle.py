@@ -1,0 +1,370 @@
+"""Pins for the oracle: values fixed by the number-format specs, closed forms,
+invariants, brute force on tiny inputs and an independent LRU replay.  None of
+these re-type the oracle's own formula; each is chosen so a plausible slip in
+the oracle (a dropped term, a wrong sign or index, a transposed operand, a
+wrong tie rule) fails at least one of them."""
+import itertools
+import math
+from collections import OrderedDict
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+
+# ---------------------------------------------------------------------------
+# Number formats
+# ---------------------------------------------------------------------------
+
+def test_e4m3_spec_values():
+    # OCP FP8 E4M3: bias 7, max 448 (S.1111.110), min normal 2^-6, min subnormal 2^-9.
+    assert oracle.e4m3_value(0x7E) == 448.0
+    assert oracle.e4m3_value(0xFE) == -448.0
+    assert oracle.e4m3_value(0x38) == 1.0
+    assert oracle.e4m3_value(0x3C) == 1.5
+    assert oracle.e4m3_value(0x08) == 2.0 ** -6
+    assert oracle.e4m3_value(0x07) == 7 * 2.0 ** -9
+    assert oracle.e4m3_value(0x01) == 2.0 ** -9
+    assert oracle.e4m3_value(0x00) == 0.0
+    assert math.isnan(oracle.e4m3_value(0x7F))
+
+
+def test_e4m3_matches_torch_cast():
+    # torch's float8_e4m3fn cast (round to nearest even) is an independent library routine.
+    vals = sorted({oracle.e4m3_value(c) for c in range(127)})
+    rng = np.random.default_rng(1)
+    xs = np.concatenate([
+        rng.normal(0, 1, 4000), rng.normal(0, 100, 2000), rng.normal(0, 0.01, 2000),
+        np.array(vals), (np.array(vals[:-1]) + np.array(vals[1:])) / 2,  # every midpoint (ties)
+    ]).astype(np.float32)
+    xs = xs[np.abs(xs) <= 448.0]
+    ref = torch.tensor(xs).to(torch.float8_e4m3fn).to(torch.float32).numpy()
+    got = np.array([oracle.e4m3_value(oracle.e4m3_encode(float(v))) for v in xs], dtype=np.float32)
+    assert np.array_equal(np.abs(got), np.abs(ref))
+    assert np.array_equal(np.sign(got[ref != 0]), np.sign(ref[ref != 0]))
+
+
+def test_e4m3_ties_and_saturation():
+    enc = lambda v: oracle.e4m3_value(oracle.e4m3_encode(v))
+    assert enc(1.0625) == 1.0            # tie between 1.0 (m=0) and 1.125 (m=1) -> even
+    assert enc(1.1875) == 1.25           # tie between 1.125 (m=1) and 1.25 (m=2) -> even
+    assert enc(2.0 ** -10) == 0.0        # half the smallest subnormal -> 0
+    assert enc(3 * 2.0 ** -10) == 2.0 ** -8
+    assert enc(460.0) == 448.0
+    assert enc(1e6) == 448.0 and enc(-1e6) == -448.0
+
+
+def test_e2m1_grid_and_ties():
+    grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    for c, v in enumerate(grid):
+        assert oracle.e2m1_value(c) == v
+        assert oracle.e2m1_value(c | 8) == -v
+        assert oracle.e2m1_encode(v) == c
+    enc = lambda v: oracle.e2m1_value(oracle.e2m1_encode(v))
+    for v, want in [(0.25, 0.0), (0.75, 1.0), (1.25, 1.0), (1.75, 2.0), (2.5, 2.0),
+                     (3.5, 4.0), (5.0, 4.0), (7.0, 6.0), (100.0, 6.0), (-2.5, -2.0), (-5.0, -4.0),
+                     (0.3, 0.5), (2.6, 3.0)]:
+        assert enc(v) == want, (v, enc(v), want)
+
+
+def test_bf16_decode():
+    bits = np.array([0x3F80, 0xBF80, 0x4049, 0x0000, 0x7F7F], dtype=np.uint16)
+    f = oracle.bf16_to_f32(bits)
+    assert f[0] == 1.0 and f[1] == -1.0 and f[3] == 0.0
+    assert f[2] == np.float32(3.140625)
+    assert f[4] == np.float32(3.3895313892515355e38)
+
+
+def test_dequant_fp8_block_indexing():
+    # a 256x256 matrix = 2x2 blocks with distinct scales; q=0x38 (1.0) everywhere
+    # except a few probes, so each element must pick its own block's scale.
+    q = np.full((256, 256), 0x38, dtype=np.uint8)
+    q[0, 255] = 0x3C      # 1.5 in block (0, 1)
+    q[200, 3] = 0xB8      # -1.0 in block (1, 0)
+    s = np.array([[1.0, 2.0], [4.0, 8.0]], dtype=np.float32)
+    w = oracle.dequant_fp8_b128(q, s)
+    assert w[0, 0] == 1.0 and w[0, 255] == 3.0 and w[200, 3] == -4.0 and w[255, 255] == 8.0
+    assert w[127, 128] == 2.0 and w[128, 127] == 4.0
+
+
+def test_dequant_nvfp4_nibble_order_and_scales():
+    R, C = 2, 32
+    qp = np.zeros((R, C // 2), dtype=np.uint8)
+    qp[0, 0] = 0x72       # element 0 -> code 2 (1.0), element 1 -> code 7 (6.0)
+    qp[1, 15] = 0xD0      # element 30 -> 0, element 31 -> code 0xD (-3.0)
+    s16 = np.array([[0x38, 0x40], [0x30, 0x48]], dtype=np.uint8)  # 1.0, 2.0, 0.5, 4.0
+    w = oracle.dequant_nvfp4(qp, s16, 0.25)
+    assert w[0, 0] == 0.25 * 1.0 * 1.0 and w[0, 1] == 6.0 * 0.25
+    assert w[1, 31] == -3.0 * 4.0 * 0.25 and w[1, 30] == 0.0
+
+
+def test_generator_quantisers_round_trip_within_format_bound():
+    rng_w = synth.normal(0, 99, 0, 0, 0, 256 * 256, 0.02).reshape(256, 256)
+    q, s = synth.quant_fp8_b128(rng_w)
+    w = oracle.dequant_fp8_b128(q, s)
+    # e4m3 keeps 3 mantissa bits: half-ulp relative error <= 2^-4 in the normal
+    # range; absolute error <= 2^-10 * s in the subnormal range.
+    sb = np.repeat(np.repeat(s, 128, 0), 128, 1)
+    err = np.abs(w - rng_w)
+    assert np.all(err <= np.maximum(np.abs(rng_w) * 2.0 ** -4, sb * 2.0 ** -10) * (1 + 1e-6))
+    # block amax maps exactly to 448 * s
+    assert np.isclose(np.abs(w[:128, :128]).max(), np.abs(rng_w[:128, :128]).max(), rtol=1e-6)
+
+    qp, s16, st = synth.quant_nvfp4(rng_w)
+    w4 = oracle.dequant_nvfp4(qp, s16, st)
+    assert st == np.float32(np.abs(rng_w).max()) / np.float32(2688.0)
+    rel = np.abs(w4 - rng_w).max() / np.abs(rng_w).max()
+    assert rel < 0.25  # e2m1 half-step <= 1/3 of the block amax; coarse bound
+
+
+def test_qa_fp8_exact_on_grid_and_zero_group():
+    s = 0.01
+    grid = np.array([oracle.e4m3_value(c) for c in range(0, 127, 3)] + [448.0], dtype=np.float64)
+    row = np.zeros(128, dtype=np.float32)
+    row[: grid.size] = (grid * s).astype(np.float32)
+    v = np.stack([row, np.zeros(128, np.float32)])
+    out = oracle.qa_fp8(v)
+    # amax = 448*s exactly -> scale s -> on-grid values survive (within fp32 rounding of v/s)
+    assert np.allclose(out[0], row, rtol=2e-7, atol=0)
+    assert np.all(out[1] == 0)
+
+
+def test_qa_nvfp4_group():
+    g = np.array([6, 3, 2.5, -1.75, 0.25, 0.75, 4, 5, 0, 0, 0, 0, 0, 0, 0, 1.25], dtype=np.float32)
+    out = oracle.qa_nvfp4(g[None, :])[0]
+    # amax = 6 -> s16 = e4m3(1.0) = 1 -> plain e2m1 rounding
+    want = [6, 3, 2, -2, 0, 1, 4, 4, 0, 0, 0, 0, 0, 0, 0, 1]
+    assert list(out) == want
+    g2 = g * 0.5  # amax 3 -> s16 = 0.5 -> same codes, halved
+    assert list(oracle.qa_nvfp4(g2[None, :])[0]) == [w * 0.5 for w in want]
+
+
+# ---------------------------------------------------------------------------
+# Router and gating
+# ---------------------------------------------------------------------------
+
+def _rand_router(T=13, d=40, E=11, seed=3, bias=True):
+    rng = np.random.default_rng(seed)
+    x = rng.normal(size=(T, d)).astype(np.float32)
+    W = (rng.normal(size=(E, d)) * 0.3).astype(np.float32)
+    b = rng.uniform(-0.5, 0.5, E).astype(np.float32) if bias else None
+    return x, W, b
+
+
+def test_router_logits_vs_library_matmul():
+    x, W, b = _rand_router()
+    lg = oracle.router_logits(x, W, b)
+    ref = x.astype(np.float64) @ W.astype(np.float64).T + b.astype(np.float64)
+    assert np.allclose(lg, ref, rtol=1e-6, atol=1e-6)
+    lg0 = oracle.router_logits(x, W, None)
+    assert np.allclose(lg - lg0, b[None, :], atol=1e-6)
+
+
+@pytest.mark.parametrize("k", [1, 2, 5, 11])
+def test_topk_brute_force(k):
+    x, W, b = _rand_router()
+    lg = oracle.router_logits(x, W, b)
+    ids, g = oracle.topk_gates(lg, k)
+    T, E = lg.shape
+    for t in range(T):
+        order = sorted(range(E), key=lambda e: (-float(lg[t, e]), e))
+        assert list(ids[t]) == order[:k]
+        p = np.exp(lg[t].astype(np.float64) - lg[t].max())
+        sel = p[order[:k]]
+        assert np.allclose(g[t], sel / sel.sum(), rtol=1e-6)   # softmax restricted to the picks
+        assert abs(float(g[t].sum()) - 1.0) < 1e-6
+    if k == 1:
+        assert np.array_equal(ids[:, 0], lg.argmax(1))
+        assert np.all(g == 1.0)
+    if k == E:
+        assert all(sorted(r) == list(range(E)) for r in ids.tolist())
+
+
+def test_topk_tie_goes_to_lower_id():
+    lg = np.array([[0.5, 1.0, 1.0, -2.0, 1.0]], dtype=np.float32)
+    ids, g = oracle.topk_gates(lg, 3)
+    assert list(ids[0]) == [1, 2, 4]
+    assert np.allclose(g[0], 1 / 3)
+
+
+def test_margin_check_brute_force():
+    rng = np.random.default_rng(5)
+    lg = rng.normal(size=(200, 9)).astype(np.float32)
+    lg[7, 3] = lg[7, 4]  # exact tie somewhere
+    k = 3
+    ok = oracle.margin_ok(lg, k, 0.05)
+    for t in range(200):
+        s = np.sort(lg[t].astype(np.float64))[::-1]
+        want = all(s[r] - s[r + 1] >= 0.05 for r in range(k))
+        assert ok[t] == want
+
+
+# ---------------------------------------------------------------------------
+# Permutation
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,k,E", [(1, 1, 1), (5, 2, 8), (37, 3, 7), (64, 8, 128), (3, 4, 256)])
+def test_permute_invariants(T, k, E):
+    rng = np.random.default_rng(T * 1000 + k)
+    ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    counts, offsets, perm, inv = oracle.permute(ids, E)
+    P = T * k
+    flat = ids.ravel()
+    assert counts.sum() == P and offsets[0] == 0 and offsets[E] == P
+    assert np.array_equal(np.bincount(flat, minlength=E), counts)
+    assert sorted(perm.tolist()) == list(range(P))
+    assert np.array_equal(inv[perm], np.arange(P))
+    assert perm.tolist() == sorted(range(P), key=lambda q: (flat[q], q))   # stable counting sort
+    for e in range(E):
+        seg = perm[offsets[e]:offsets[e + 1]]
+        assert np.all(flat[seg] == e)
+    # every token appears exactly k times
+    assert np.array_equal(np.bincount(perm // k, minlength=T), np.full(T, k))
+
+
+# ---------------------------------------------------------------------------
+# LRU slot cache
+# ---------------------------------------------------------------------------
+
+class ListLRU:
+    """Independent LRU: an eviction list (front = next victim).  Each step takes
+    the touched slots out, fills misses (ascending expert id) from the front and
+    appends every touched slot at the back in ascending slot order."""
+
+    def __init__(self, E, S):
+        self.order = list(range(S))         # empty slots in index order
+        self.expert = [-1] * S
+        self.where = {}
+
+    def step(self, ids):
+        want = sorted(set(int(i) for i in ids))
+        if len(want) > len(self.expert):
+            return None
+        touched = [self.where[e] for e in want if e in self.where]
+        for sl in touched:
+            self.order.remove(sl)
+        misses = []
+        for e in want:
+            if e in self.where:
+                continue
+            sl = self.order.pop(0)
+            if self.expert[sl] >= 0:
+                del self.where[self.expert[sl]]
+            self.expert[sl] = e
+            self.where[e] = sl
+            touched.append(sl)
+            misses.append((e, sl))
+        self.order.extend(sorted(touched))
+        return misses
+
+
+def test_lru_hand_worked_three_slots():
+    st = oracle.LRUState(E=6, S=3)
+    rc, m, nd, nh = st.update(np.array([4, 1]))
+    assert rc == 0 and m == [(1, 0), (4, 1)] and nh == 0          # empty slots in index order
+    rc, m, nd, nh = st.update(np.array([2, 4]))
+    assert m == [(2, 2)] and nh == 1                               # slot 2 still empty
+    rc, m, nd, nh = st.update(np.array([5, 0]))
+    # last_use: slot0 (e1)=0, slot1 (e4)=1, slot2 (e2)=1 -> victims slot0 then slot1
+    assert m == [(0, 0), (5, 1)] and nh == 0
+    assert list(st.expert_of_slot) == [0, 5, 2] and list(st.last_use) == [2, 2, 1]
+    assert st.slot_of_expert.tolist() == [0, -1, 2, -1, -1, 1]
+    rc, m, nd, nh = st.update(np.array([3, 1, 0]))
+    # slot2 (last_use 1) is the only slot older than this step, then slots 0/1 tie
+    # at 2 but slot 0 is requested (hit) -> slot 1
+    assert m == [(1, 2), (3, 1)] and nh == 1
+    before = st.copy()
+    rc, m, nd, nh = st.update(np.array([0, 1, 2, 3]))               # 4 distinct > 3 slots
+    assert rc == -1 and nd == 4
+    assert np.array_equal(st.slot_of_expert, before.slot_of_expert)
+    assert np.array_equal(st.last_use, before.last_use) and st.step == before.step
+
+
+@pytest.mark.parametrize("E,S,n,seed", [(16, 4, 3, 0), (64, 16, 10, 1), (256, 64, 40, 2), (8, 8, 8, 3)])
+def test_lru_matches_list_replay(E, S, n, seed):
+    rng = np.random.default_rng(seed)
+    st = oracle.LRUState(E, S)
+    ref = ListLRU(E, S)
+    zipf = 1.0 / np.arange(1, E + 1) ** 1.1
+    zipf /= zipf.sum()
+    for step in range(200):
+        ids = rng.choice(E, size=n, p=zipf)
+        rc, m, nd, nh = st.update(ids)
+        rm = ref.step(ids)
+        if rm is None:
+            assert rc == -1
+            continue
+        assert rc == 0 and m == rm
+        assert st.expert_of_slot.tolist() == ref.expert
+        assert nh == len(set(ids.tolist())) - len(m)
+
+
+# ---------------------------------------------------------------------------
+# Expert FFN and combine
+# ---------------------------------------------------------------------------
+
+def test_ffn_closed_form_d2_i1():
+    x = np.array([[1.0, 2.0]], dtype=np.float32)
+    Wg = np.array([[0.5, 0.25]], dtype=np.float32)     # g = 1
+    Wu = np.array([[1.0, -1.0]], dtype=np.float32)     # u = -1
+    Wd = np.array([[2.0], [3.0]], dtype=np.float32)
+    y = oracle.expert_ffn(x, Wg, Wu, Wd)
+    h = -1.0 / (1.0 + math.exp(-1.0))
+    assert np.allclose(y[0], [2 * h, 3 * h], rtol=1e-7)
+
+
+def test_ffn_scalar_brute_force():
+    for xv, g, u, dn in itertools.product([-2.0, 0.0, 0.7], [-1.5, 0.3], [2.0, -0.5], [1.0, -3.0]):
+        y = oracle.expert_ffn(np.array([[xv]], np.float32), np.array([[g]], np.float32),
+                              np.array([[u]], np.float32), np.array([[dn]], np.float32))
+        z = xv * g
+        want = z / (1 + math.exp(-z)) * (xv * u) * dn
+        assert abs(float(y[0, 0]) - want) <= 1e-6 * max(1.0, abs(want))
+
+
+def test_ffn_gate_and_up_not_swapped():
+    # silu applies to the gate projection only: swapping Wg/Wu changes the result
+    rng = np.random.default_rng(0)
+    x = rng.normal(size=(3, 8)).astype(np.float32)
+    Wg, Wu = rng.normal(size=(2, 5, 8)).astype(np.float32)
+    Wd = rng.normal(size=(8, 5)).astype(np.float32)
+    a = oracle.expert_ffn(x, Wg, Wu, Wd)
+    b = oracle.expert_ffn(x, Wu, Wg, Wd)
+    assert not np.allclose(a, b)
+    # with Wu = Wg the result is silu(z)*z, which is >= -0.28*|z| ... check one entry
+    c = oracle.expert_ffn(x[:1], Wg, Wg, np.eye(8, 5, dtype=np.float32))
+    z = x[0].astype(np.float64) @ Wg.T.astype(np.float64)
+    assert np.allclose(c[0, :5], z / (1 + np.exp(-z)) * z, rtol=1e-6)
+
+
+def test_combine_hand_example():
+    y = np.array([[1, 2], [3, 4]], dtype=np.float32)
+    g = np.array([[0.25, 0.75]], dtype=np.float32)
+    assert np.allclose(oracle.combine(y, g, None), [[2.5, 3.5]])
+    assert np.allclose(oracle.combine(y, g, np.array([[1, 1]], np.float32)), [[3.5, 4.5]])
+
+
+@pytest.mark.parametrize("shared", [0, 1])
+def test_identical_experts_collapse_to_dense_ffn(shared):
+    cfg = synth.scaled(synth.CONFIGS["tiny"], d=32, I=16, E=5, k=3, has_shared=shared, S=5, T=(6,))
+    layer = synth.Layer(cfg, seed=11)
+    x = layer.hidden_f32(6)
+    Wr = layer.router_f32()
+    ids, g, _ = oracle.route(x, Wr, None, cfg.k)
+    W0 = layer.expert_f32(0)
+    cache = {e: W0 for e in range(cfg.E + 1)}         # every expert (and the shared one) = expert 0
+    out = oracle.moe_rows(layer, x, range(6), ids, g, weight_cache=cache)
+    dense = oracle.expert_ffn(x, *W0)
+    want = dense * (2 if shared else 1)
+    assert np.allclose(out, want, rtol=1e-5, atol=1e-6)
+
+
+def test_generator_philox_known_answers():
+    # Random123 known-answer vectors for Philox4x32-10
+    assert list(synth.philox([0, 0, 0, 0], [0, 0])) == [0x6627E8D5, 0xE169C58D, 0xBC57AC4C, 0x9B00DBD8]
+    assert list(synth.philox([0xFFFFFFFF] * 4, [0xFFFFFFFF] * 2)) == [0x408F276D, 0x41C83B0E, 0xA20BC7C6, 0x6D5451FD]
+    assert list(synth.philox([0x243F6A88, 0x85A308D3, 0x13198A2E, 0x03707344], [0xA4093822, 0x299F31D0])) == \
+        [0xD16CFE09, 0x94FDCCEB, 0x5001E420, 0x24126EA1]
