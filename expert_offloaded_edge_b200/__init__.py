@@ -1,0 +1,35 @@
+"""B200-native routed-MoE layer over a slot-indexed expert cache.
+
+Python binding of the C ABI in ``include/ftm.h`` (argument marshalling only;
+every step runs in the sm_100a kernels of ``libftm.so``).  Function names match
+the C entry points.  Tensors are torch tensors on the CUDA device (or pinned
+host tensors where the header says host); streams default to torch's current
+stream.
+"""
+from .binding import (  # noqa: F401
+    FTM_BF16,
+    FTM_F32,
+    FTM_FP8_E4M3_B128,
+    FTM_NVFP4,
+    BankLayout,
+    FtmError,
+    LayerDesc,
+    LayerWeights,
+    SlotCache,
+    desc_for,
+    ftm_combine,
+    ftm_device_status,
+    ftm_expert_ffn,
+    ftm_ffn_workspace_bytes,
+    ftm_get_bank_layout,
+    ftm_last_error,
+    ftm_moe_layer_forward,
+    ftm_permute,
+    ftm_permute_workspace_bytes,
+    ftm_route,
+    ftm_slot_host_scratch_ints,
+    ftm_slot_lookup_update,
+    ftm_slot_workspace_bytes,
+    ftm_workspace_bytes,
+    library,
+)

@@ -1,0 +1,378 @@
+// C ABI of the routed-MoE layer: argument validation, workspace carving, the
+// miss-copy orchestration of the slot cache, and the whole-layer sequence.
+// Every computation step runs in the kernels of the sibling .cu files.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "ftm_common.cuh"
+
+namespace ftm {
+cudaError_t launch_route(bool f32, const void* x, int T, int d, const void* wr, const float* bias, int E, int k,
+                         int32_t* ids, float* w, cudaStream_t st);
+cudaError_t launch_permute(const int32_t* ids, int P, int E, int32_t* counts, int32_t* offsets, int32_t* perm,
+                           int32_t* inv, void* ws, cudaStream_t st);
+size_t permute_workspace_bytes(int E, int64_t P);
+size_t lru_workspace_bytes(int E, int S);
+cudaError_t launch_lru_step(const int32_t* ids, int P, int E, int S, int64_t step, int32_t* soe, int32_t* eos,
+                            int64_t* lu, int32_t* ws, cudaStream_t st);
+cudaError_t launch_lru_restore(int E, int S, int32_t* soe, int32_t* eos, int64_t* lu, const int32_t* ws,
+                               cudaStream_t st);
+cudaError_t launch_combine(bool f32, const void* y, const int32_t* inv, const float* gw, int T, int k, int d, int P,
+                           int has_shared, void* out, cudaStream_t st);
+const char* launch_expert_ffn(const FfnArgs& a, cudaStream_t st, cudaError_t* cerr);
+}  // namespace ftm
+
+using namespace ftm;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+ftm_status fail(ftm_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+ftm_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(FTM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+ftm_status ok() {
+  g_err[0] = 0;
+  return FTM_OK;
+}
+
+inline cudaStream_t S_(void* s) { return static_cast<cudaStream_t>(s); }
+
+constexpr size_t kAlign = 256;
+inline size_t al(size_t b) { return (b + kAlign - 1) & ~(kAlign - 1); }
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+ftm_status check_desc(const ftm_layer_desc* L) {
+  if (!L) return fail(FTM_ERR_INVALID_ARG, "layer descriptor is NULL");
+  if (L->reserved != 0) return fail(FTM_ERR_INVALID_ARG, "reserved field must be 0");
+  if (L->wdtype < FTM_F32 || L->wdtype > FTM_NVFP4) return fail(FTM_ERR_INVALID_ARG, "unknown wdtype %d", L->wdtype);
+  const int q = L->wdtype == FTM_NVFP4 ? 256 : 128;
+  if (L->d <= 0 || L->d % q) return fail(FTM_ERR_INVALID_ARG, "d=%d must be a positive multiple of %d", L->d, q);
+  if (L->I <= 0 || L->I % q) return fail(FTM_ERR_INVALID_ARG, "I=%d must be a positive multiple of %d", L->I, q);
+  if (L->E < 1 || L->E > 512) return fail(FTM_ERR_INVALID_ARG, "E=%d out of [1, 512]", L->E);
+  if (L->k < 1 || L->k > 16 || L->k > L->E) return fail(FTM_ERR_INVALID_ARG, "k=%d out of [1, min(E,16)]", L->k);
+  if (L->S < 1) return fail(FTM_ERR_INVALID_ARG, "S=%d must be >= 1", L->S);
+  if (L->has_shared != 0 && L->has_shared != 1) return fail(FTM_ERR_INVALID_ARG, "has_shared must be 0 or 1");
+  return FTM_OK;
+}
+
+ftm_status check_T(int32_t T) {
+  if (T < 0) return fail(FTM_ERR_INVALID_ARG, "T=%d is negative", T);
+  if (static_cast<int64_t>(T) * 16 > (1ll << 30)) return fail(FTM_ERR_INVALID_ARG, "T=%d too large", T);
+  return FTM_OK;
+}
+
+void bank_layout(const ftm_layer_desc* L, ftm_bank_layout* b) {
+  memset(b, 0, sizeof(*b));
+  const uint64_t d = L->d, I = L->I;
+  uint64_t wgu = 0, wd = 0, sgu = 0, sd = 0, st = 0;
+  switch (L->wdtype) {
+    case FTM_F32: wgu = 2 * I * d * 4; wd = d * I * 4; break;
+    case FTM_BF16: wgu = 2 * I * d * 2; wd = d * I * 2; break;
+    case FTM_FP8_E4M3_B128:
+      wgu = 2 * I * d; wd = d * I;
+      sgu = (2 * I / 128) * (d / 128) * 4; sd = (d / 128) * (I / 128) * 4;
+      break;
+    case FTM_NVFP4:
+      wgu = 2 * I * d / 2; wd = d * I / 2;
+      sgu = 2 * I * (d / 16); sd = d * (I / 16); st = 16;
+      break;
+  }
+  uint64_t off = 0;
+  b->w_gu_off = off; b->w_gu_bytes = wgu; off = al(off + wgu);
+  b->w_d_off = off; b->w_d_bytes = wd; off = al(off + wd);
+  b->s_gu_off = off; b->s_gu_bytes = sgu; off = al(off + sgu);
+  b->s_d_off = off; b->s_d_bytes = sd; off = al(off + sd);
+  b->s_t_off = off; b->s_t_bytes = st; off = al(off + st);
+  b->bank_bytes = off;
+}
+
+int64_t ffn_rows(const ftm_layer_desc* L, int32_t T) {
+  return static_cast<int64_t>(T) * L->k + (L->has_shared ? T : 0);
+}
+
+size_t act_elt(const ftm_layer_desc* L) { return L->wdtype == FTM_F32 ? 4 : 2; }
+
+size_t ffn_ws_bytes(const ftm_layer_desc* L, int32_t T) {
+  const size_t rows = static_cast<size_t>(ffn_rows(L, T));
+  return al(rows * L->d * act_elt(L)) + al(rows * L->I * act_elt(L));
+}
+
+// Whole-layer workspace carving.
+struct LayerWs {
+  int32_t* ids;
+  float* gates;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* perm;
+  int32_t* inv;
+  void* perm_ws;
+  uint8_t* ffn_ws;
+  void* y;
+  int32_t* lru_ws;
+  size_t total;
+};
+
+LayerWs carve(const ftm_layer_desc* L, int32_t T, uint8_t* base) {
+  LayerWs w;
+  const size_t P = static_cast<size_t>(T) * L->k;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { uint8_t* p = base ? base + off : nullptr; off += al(bytes); return p; };
+  w.ids = reinterpret_cast<int32_t*>(take(P * 4));
+  w.gates = reinterpret_cast<float*>(take(P * 4));
+  w.counts = reinterpret_cast<int32_t*>(take(static_cast<size_t>(L->E) * 4));
+  w.offsets = reinterpret_cast<int32_t*>(take((static_cast<size_t>(L->E) + 1) * 4));
+  w.perm = reinterpret_cast<int32_t*>(take(P * 4));
+  w.inv = reinterpret_cast<int32_t*>(take(P * 4));
+  w.perm_ws = take(permute_workspace_bytes(L->E, static_cast<int64_t>(P)));
+  w.ffn_ws = take(ffn_ws_bytes(L, T));
+  w.y = take(static_cast<size_t>(ffn_rows(L, T)) * L->d * act_elt(L));
+  w.lru_ws = reinterpret_cast<int32_t*>(take(lru_workspace_bytes(L->E, L->S)));
+  w.total = off;
+  return w;
+}
+
+ftm_status check_ws(void* ws, size_t have, size_t need, const char* who) {
+  if (need && !ws) return fail(FTM_ERR_INVALID_ARG, "%s: workspace is NULL (%zu bytes needed)", who, need);
+  if (have < need) return fail(FTM_ERR_INVALID_ARG, "%s: workspace %zu bytes < %zu needed", who, have, need);
+  if (ws && !aligned(ws, kAlign)) return fail(FTM_ERR_INVALID_ARG, "%s: workspace not 256-byte aligned", who);
+  return FTM_OK;
+}
+
+cudaEvent_t copy_event() {
+  static thread_local cudaEvent_t ev = nullptr;
+  static thread_local int dev = -1;
+  int cur = 0;
+  cudaGetDevice(&cur);
+  if (!ev || dev != cur) {
+    if (ev) cudaEventDestroy(ev);
+    ev = nullptr;
+    if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) ev = nullptr;
+    dev = cur;
+  }
+  return ev;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ftm_last_error(void) { return g_err; }
+
+int32_t ftm_device_status(int32_t reset) {
+  cudaDeviceSynchronize();
+  int32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_dev_status, sizeof(v)) != cudaSuccess) return -1;
+  if (reset) {
+    const int32_t z = 0;
+    cudaMemcpyToSymbol(g_dev_status, &z, sizeof(z));
+  }
+  return v;
+}
+
+ftm_status ftm_get_bank_layout(const ftm_layer_desc* L, ftm_bank_layout* out) {
+  ftm_status s = check_desc(L);
+  if (s) return s;
+  if (!out) return fail(FTM_ERR_INVALID_ARG, "out is NULL");
+  bank_layout(L, out);
+  return ok();
+}
+
+ftm_status ftm_route(const ftm_layer_desc* L, const void* x, int32_t T, const void* w_router, const float* bias,
+                     int32_t* topk_ids, float* topk_w, void* stream) {
+  ftm_status s = check_desc(L);
+  if (s || (s = check_T(T))) return s;
+  if (T == 0) return ok();
+  if (!x || !w_router || !topk_ids || !topk_w) return fail(FTM_ERR_INVALID_ARG, "ftm_route: NULL pointer");
+  if (!aligned(x, 16) || !aligned(w_router, 16)) return fail(FTM_ERR_INVALID_ARG, "ftm_route: x/w_router not 16-byte aligned");
+  cudaError_t e = launch_route(L->wdtype == FTM_F32, x, T, L->d, w_router, bias, L->E, L->k, topk_ids, topk_w, S_(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "ftm_route launch");
+  return ok();
+}
+
+size_t ftm_permute_workspace_bytes(const ftm_layer_desc* L, int32_t T) {
+  if (check_desc(L) || T < 0) return 0;
+  return permute_workspace_bytes(L->E, static_cast<int64_t>(T) * L->k);
+}
+
+ftm_status ftm_permute(const ftm_layer_desc* L, const int32_t* topk_ids, int32_t T, int32_t* counts, int32_t* offsets,
+                       int32_t* perm, int32_t* inv, void* workspace, size_t ws_bytes, void* stream) {
+  ftm_status s = check_desc(L);
+  if (s || (s = check_T(T))) return s;
+  if (!counts || !offsets) return fail(FTM_ERR_INVALID_ARG, "ftm_permute: NULL counts/offsets");
+  const int64_t P = static_cast<int64_t>(T) * L->k;
+  if (P > 0 && (!topk_ids || !perm || !inv)) return fail(FTM_ERR_INVALID_ARG, "ftm_permute: NULL pointer");
+  if ((s = check_ws(workspace, ws_bytes, permute_workspace_bytes(L->E, P), "ftm_permute"))) return s;
+  cudaError_t e = launch_permute(topk_ids, static_cast<int>(P), L->E, counts, offsets, perm, inv, workspace, S_(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "ftm_permute launch");
+  return ok();
+}
+
+size_t ftm_slot_host_scratch_ints(const ftm_layer_desc* L) {
+  if (check_desc(L)) return 0;
+  return 4 + 2 * static_cast<size_t>(L->E);
+}
+
+size_t ftm_slot_workspace_bytes(const ftm_layer_desc* L) {
+  if (check_desc(L)) return 0;
+  return lru_workspace_bytes(L->E, L->S);
+}
+
+ftm_status ftm_slot_lookup_update(const ftm_layer_desc* L, ftm_slot_cache* C, const int32_t* topk_ids, int32_t T,
+                                  void* workspace, size_t ws_bytes, void* compute_stream, void* copy_stream) {
+  ftm_status s = check_desc(L);
+  if (s || (s = check_T(T))) return s;
+  if (!C || !C->slot_of_expert || !C->expert_of_slot || !C->last_use || !C->slot_pool || !C->host_pool ||
+      !C->host_scratch)
+    return fail(FTM_ERR_INVALID_ARG, "ftm_slot_lookup_update: cache has a NULL member");
+  if (L->S > 4096) return fail(FTM_ERR_UNSUPPORTED, "LRU cache supports S <= 4096 (S=%d)", L->S);
+  const int64_t P = static_cast<int64_t>(T) * L->k;
+  if (P > 0 && !topk_ids) return fail(FTM_ERR_INVALID_ARG, "ftm_slot_lookup_update: NULL topk_ids");
+  if ((s = check_ws(workspace, ws_bytes, lru_workspace_bytes(L->E, L->S), "ftm_slot_lookup_update"))) return s;
+  cudaPointerAttributes pa;
+  if (cudaPointerGetAttributes(&pa, C->host_pool) != cudaSuccess || pa.type != cudaMemoryTypeHost) {
+    cudaGetLastError();
+    return fail(FTM_ERR_INVALID_ARG, "host_pool is not pinned host memory");
+  }
+  cudaStream_t cs = S_(compute_stream), ps = S_(copy_stream);
+  int32_t* ws = static_cast<int32_t*>(workspace);
+  cudaError_t e = launch_lru_step(topk_ids, static_cast<int>(P), L->E, L->S, C->step, C->slot_of_expert,
+                                  C->expert_of_slot, C->last_use, ws, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "lru step launch");
+  const size_t hdr = sizeof(int32_t) * (4 + 2 * static_cast<size_t>(L->E));
+  if ((e = cudaMemcpyAsync(C->host_scratch, ws, hdr, cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
+    return cuda_fail(e, "miss list copy");
+  if ((e = cudaStreamSynchronize(cs)) != cudaSuccess) return cuda_fail(e, "lru step");
+  const int32_t* h = C->host_scratch;
+  C->last_distinct = h[1];
+  C->last_hits = h[2];
+  C->last_misses = h[3];
+  if (h[0] == FTM_ERR_CAPACITY)
+    return fail(FTM_ERR_CAPACITY, "step %lld requests %d distinct experts > %d slots", static_cast<long long>(C->step),
+                h[1], L->S);
+  ftm_bank_layout bl;
+  bank_layout(L, &bl);
+  const int misses = h[3];
+  bool copy_failed = C->fail_before_copy != 0;
+  const char* why = copy_failed ? "injected copy failure (fail_before_copy)" : nullptr;
+  for (int i = 0; i < misses && !copy_failed; ++i) {
+    const int ex = h[4 + 2 * i], sl = h[4 + 2 * i + 1];
+    e = cudaMemcpyAsync(static_cast<uint8_t*>(C->slot_pool) + static_cast<size_t>(sl) * bl.bank_bytes,
+                        static_cast<const uint8_t*>(C->host_pool) + static_cast<size_t>(ex) * bl.bank_bytes,
+                        bl.bank_bytes, cudaMemcpyHostToDevice, ps);
+    if (e != cudaSuccess) { copy_failed = true; why = cudaGetErrorString(e); }
+  }
+  if (copy_failed) {
+    C->fail_before_copy = 0;
+    cudaError_t e2 = launch_lru_restore(L->E, L->S, C->slot_of_expert, C->expert_of_slot, C->last_use, ws, cs);
+    if (e2 == cudaSuccess) e2 = cudaStreamSynchronize(cs);
+    return fail(FTM_ERR_CUDA, "miss copy failed (%s); slot state rolled back%s", why,
+                e2 == cudaSuccess ? "" : " -- rollback failed too");
+  }
+  if (misses > 0) {
+    cudaEvent_t ev = copy_event();
+    if (!ev) return fail(FTM_ERR_CUDA, "could not create the copy event");
+    if ((e = cudaEventRecord(ev, ps)) != cudaSuccess) return cuda_fail(e, "copy event record");
+    if ((e = cudaStreamWaitEvent(cs, ev, 0)) != cudaSuccess) return cuda_fail(e, "copy event wait");
+  }
+  C->step += 1;
+  return ok();
+}
+
+size_t ftm_ffn_workspace_bytes(const ftm_layer_desc* L, int32_t T) {
+  if (check_desc(L) || T < 0) return 0;
+  return ffn_ws_bytes(L, T);
+}
+
+ftm_status ftm_expert_ffn(const ftm_layer_desc* L, const void* x, int32_t T, const int32_t* offsets,
+                          const int32_t* perm, const int32_t* slot_of_expert, const void* slot_pool,
+                          const void* shared_bank, void* y, void* workspace, size_t ws_bytes, void* stream) {
+  ftm_status s = check_desc(L);
+  if (s || (s = check_T(T))) return s;
+  if (L->wdtype == FTM_FP8_E4M3_B128 || L->wdtype == FTM_NVFP4)
+    return fail(FTM_ERR_UNSUPPORTED, "expert FFN for wdtype %d not built", L->wdtype);
+  if (T == 0) return ok();
+  if (!x || !offsets || !perm || !slot_of_expert || !slot_pool || !y)
+    return fail(FTM_ERR_INVALID_ARG, "ftm_expert_ffn: NULL pointer");
+  if (L->has_shared && !shared_bank) return fail(FTM_ERR_INVALID_ARG, "ftm_expert_ffn: layer has a shared expert but shared_bank is NULL");
+  if (!aligned(slot_pool, 256) || (shared_bank && !aligned(shared_bank, 256)) || !aligned(x, 16) || !aligned(y, 16))
+    return fail(FTM_ERR_INVALID_ARG, "ftm_expert_ffn: misaligned pointer (pool/bank 256 B, x/y 16 B)");
+  if ((s = check_ws(workspace, ws_bytes, ffn_ws_bytes(L, T), "ftm_expert_ffn"))) return s;
+  ftm_bank_layout bl;
+  bank_layout(L, &bl);
+  FfnArgs a;
+  a.d = L->d; a.E = L->E; a.k = L->k; a.I = L->I; a.has_shared = L->has_shared; a.S = L->S;
+  a.f32 = L->wdtype == FTM_F32;
+  a.x = static_cast<const uint8_t*>(x);
+  a.T = T;
+  a.offsets = offsets; a.perm = perm; a.slot_of_expert = slot_of_expert;
+  a.pool = static_cast<const uint8_t*>(slot_pool);
+  a.shared_bank = static_cast<const uint8_t*>(shared_bank);
+  a.bank_bytes = bl.bank_bytes; a.w_gu_off = bl.w_gu_off; a.w_d_off = bl.w_d_off;
+  a.y = y;
+  const size_t rows = static_cast<size_t>(ffn_rows(L, T));
+  a.xp = static_cast<uint8_t*>(workspace);
+  a.h = a.xp + al(rows * L->d * act_elt(L));
+  cudaError_t ce;
+  const char* msg = launch_expert_ffn(a, S_(stream), &ce);
+  if (msg) return ce != cudaSuccess ? cuda_fail(ce, msg) : fail(FTM_ERR_CUDA, "%s", msg);
+  return ok();
+}
+
+ftm_status ftm_combine(const ftm_layer_desc* L, const void* y, const int32_t* inv, const float* topk_w, int32_t T,
+                       void* out, void* stream) {
+  ftm_status s = check_desc(L);
+  if (s || (s = check_T(T))) return s;
+  if (T == 0) return ok();
+  if (!y || !inv || !topk_w || !out) return fail(FTM_ERR_INVALID_ARG, "ftm_combine: NULL pointer");
+  if (!aligned(y, 16) || !aligned(out, 16)) return fail(FTM_ERR_INVALID_ARG, "ftm_combine: y/out not 16-byte aligned");
+  cudaError_t e = launch_combine(L->wdtype == FTM_F32, y, inv, topk_w, T, L->k, L->d, T * L->k, L->has_shared, out,
+                                 S_(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "ftm_combine launch");
+  return ok();
+}
+
+size_t ftm_workspace_bytes(const ftm_layer_desc* L, int32_t T_max) {
+  if (check_desc(L) || T_max < 0) return 0;
+  return carve(L, T_max, nullptr).total;
+}
+
+ftm_status ftm_moe_layer_forward(const ftm_layer_desc* L, const ftm_layer_weights* W, ftm_slot_cache* C,
+                                 const void* x, int32_t T, void* out, void* workspace, size_t ws_bytes, void* stream,
+                                 void* copy_stream) {
+  ftm_status s = check_desc(L);
+  if (s || (s = check_T(T))) return s;
+  if (!W || !W->w_router) return fail(FTM_ERR_INVALID_ARG, "ftm_moe_layer_forward: NULL weights");
+  if (T == 0) return ok();
+  LayerWs w = carve(L, T, static_cast<uint8_t*>(workspace));
+  if ((s = check_ws(workspace, ws_bytes, w.total, "ftm_moe_layer_forward"))) return s;
+  if ((s = ftm_route(L, x, T, W->w_router, W->router_bias, w.ids, w.gates, stream))) return s;
+  if ((s = ftm_permute(L, w.ids, T, w.counts, w.offsets, w.perm, w.inv, w.perm_ws,
+                       permute_workspace_bytes(L->E, static_cast<int64_t>(T) * L->k), stream)))
+    return s;
+  const void* pool = W->slot_pool;
+  const int32_t* soe = W->slot_of_expert;
+  if (C) {
+    if ((s = ftm_slot_lookup_update(L, C, w.ids, T, w.lru_ws, lru_workspace_bytes(L->E, L->S), stream, copy_stream)))
+      return s;
+    pool = C->slot_pool;
+    soe = C->slot_of_expert;
+  }
+  if (!pool || !soe) return fail(FTM_ERR_INVALID_ARG, "ftm_moe_layer_forward: no slot pool / slot table");
+  if ((s = ftm_expert_ffn(L, x, T, w.offsets, w.perm, soe, pool, W->shared_bank, w.y, w.ffn_ws, ffn_ws_bytes(L, T),
+                          stream)))
+    return s;
+  return ftm_combine(L, w.y, w.inv, w.gates, T, out, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,76 @@
+// Weighted un-permute and combine (step a8):
+//   out[t] = sum_{j ascending} g[t][j] * y[inv[t*k + j]]  (+ y[P + t] for the shared expert)
+// fp32 accumulation, fixed summation order (deterministic).  One block per
+// token (grid-strided), 16-byte loads and stores along d.
+#include "ftm_common.cuh"
+
+namespace ftm {
+
+template <bool F32>
+__global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ y, const int32_t* __restrict__ inv,
+                                                      const float* __restrict__ gw, int T, int k, int d, int P,
+                                                      int has_shared, void* __restrict__ out) {
+  constexpr int V = F32 ? 4 : 8;   // elements per 16-byte vector
+  const int nv = d / V;
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    for (int c = threadIdx.x; c < nv; c += blockDim.x) {
+      float acc[V];
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc[i] = 0.f;
+      for (int j = 0; j <= k; ++j) {
+        int row;
+        float g;
+        if (j < k) {
+          row = inv[static_cast<size_t>(t) * k + j];
+          g = gw[static_cast<size_t>(t) * k + j];
+        } else {
+          if (!has_shared) break;
+          row = P + t;
+          g = 1.f;
+        }
+        const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(y) +
+                                                        (static_cast<size_t>(row) * d + static_cast<size_t>(c) * V) *
+                                                            (F32 ? 4 : 2));
+        if constexpr (F32) {
+          const float f[4] = {__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w)};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[i] = fmaf(g, f[i], acc[i]);
+        } else {
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[2 * i] = fmaf(g, __uint_as_float(w[i] << 16), acc[2 * i]);
+            acc[2 * i + 1] = fmaf(g, __uint_as_float(w[i] & 0xFFFF0000u), acc[2 * i + 1]);
+          }
+        }
+      }
+      uint4 o;
+      if constexpr (F32) {
+        o = make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]), __float_as_uint(acc[2]),
+                       __float_as_uint(acc[3]));
+      } else {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+          w[i] = *reinterpret_cast<const uint32_t*>(&b);
+        }
+        o = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      *reinterpret_cast<uint4*>(static_cast<uint8_t*>(out) +
+                                (static_cast<size_t>(t) * d + static_cast<size_t>(c) * V) * (F32 ? 4 : 2)) = o;
+    }
+  }
+}
+
+cudaError_t launch_combine(bool f32, const void* y, const int32_t* inv, const float* gw, int T, int k, int d, int P,
+                           int has_shared, void* out, cudaStream_t st) {
+  const int grid = T < 148 * 16 ? T : 148 * 16;
+  if (f32)
+    combine_kernel<true><<<grid, 256, 0, st>>>(y, inv, gw, T, k, d, P, has_shared, out);
+  else
+    combine_kernel<false><<<grid, 256, 0, st>>>(y, inv, gw, T, k, d, P, has_shared, out);
+  return cudaGetLastError();
+}
+
+}  // namespace ftm

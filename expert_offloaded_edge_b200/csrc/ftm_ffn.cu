@@ -1,0 +1,432 @@
+// Grouped SwiGLU expert FFN over the slot-indexed expert pool (steps a5-a7).
+//
+// Rows of the permuted activation matrix X_p are grouped by expert (group e =
+// rows offsets[e]..offsets[e+1]); the shared expert, when present, is one more
+// group over all T tokens (rows P..P+T-1).  Expert e's weights are the bank
+// slot_pool[slot_of_expert[e]]; the kernel never copies weights.
+//
+//   GEMM1 (+SwiGLU): H[r][i] = silu(X_p[r] . Wg[i]) * (X_p[r] . Wu[i])
+//   GEMM2          : Y[r][j] = H[r] . Wd[j]
+//
+// bf16 layers run the tensor-core kernel below: weights on the MMA M side
+// (128 weight rows per tile), tokens on the N side (BN tokens per tile), so a
+// decode-sized group of a few tokens still streams full 128-row weight tiles
+// (the decode step is bound by the expert weight bytes).  Persistent CTAs walk
+// a (group, weight tile, token tile) list; warp 0 issues TMA loads (weights via
+// a 3-D tensor map whose third coordinate is the slot), warp 1 issues tcgen05
+// MMAs into a double-buffered TMEM accumulator, warps 2-5 drain TMEM, apply
+// SwiGLU and store.  fp32 layers run a plain SIMT kernel.
+#include "ftm_common.cuh"
+
+namespace ftm {
+
+__device__ int32_t g_dev_status = 0;
+
+// ---------------------------------------------------------------------------
+// Gather: X_p[pos] = x[perm[pos] / k] (pos < P); X_p[P + t] = x[t] (shared rows).
+// ---------------------------------------------------------------------------
+__global__ void gather_rows_kernel(const uint8_t* __restrict__ x, const int32_t* __restrict__ perm, int P, int k,
+                                   int T, int has_shared, int row_bytes, uint8_t* __restrict__ xp) {
+  const int rows = P + (has_shared ? T : 0);
+  const int nv = row_bytes / 16;
+  for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+    const int src = r < P ? perm[r] / k : r - P;
+    const uint4* s = reinterpret_cast<const uint4*>(x + static_cast<size_t>(src) * row_bytes);
+    uint4* dd = reinterpret_cast<uint4*>(xp + static_cast<size_t>(r) * row_bytes);
+    for (int c = threadIdx.x; c < nv; c += blockDim.x) dd[c] = s[c];
+  }
+}
+
+// group of row r (binary search over offsets[0..E]); r >= P -> shared group E.
+__device__ __forceinline__ int group_of_row(const int32_t* offsets, int E, int P, int r) {
+  if (r >= P) return E;
+  int lo = 0, hi = E;  // offsets[lo] <= r < offsets[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (offsets[mid] <= r) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+// ---------------------------------------------------------------------------
+// SIMT path (fp32 layers): one warp per output element, lanes split the dot.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float silu(float z) { return z / (1.f + expf(-z)); }
+
+__global__ void __launch_bounds__(256) simt_gemm1_kernel(const float* __restrict__ xp, const int32_t* __restrict__ offsets,
+                                                         const int32_t* __restrict__ slot_of_expert, int E, int P,
+                                                         int d, int I, const uint8_t* __restrict__ pool,
+                                                         const uint8_t* __restrict__ shared_bank, size_t bank_bytes,
+                                                         size_t wgu_off, float* __restrict__ h) {
+  const int r = blockIdx.x;
+  const int g = group_of_row(offsets, E, P, r);
+  const float* W = reinterpret_cast<const float*>(
+      (g < E ? pool + static_cast<size_t>(slot_of_expert[g]) * bank_bytes : shared_bank) + wgu_off);
+  const float* x = xp + static_cast<size_t>(r) * d;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int i = blockIdx.y * 8 + warp; i < I; i += gridDim.y * 8) {
+    const float* wg = W + static_cast<size_t>(i) * d;
+    const float* wu = W + static_cast<size_t>(I + i) * d;
+    float a = 0.f, b = 0.f;
+    for (int c = lane; c < d; c += 32) { a = fmaf(x[c], wg[c], a); b = fmaf(x[c], wu[c], b); }
+    a = warp_sum(a);
+    b = warp_sum(b);
+    if (lane == 0) h[static_cast<size_t>(r) * I + i] = silu(a) * b;
+  }
+}
+
+__global__ void __launch_bounds__(256) simt_gemm2_kernel(const float* __restrict__ h, const int32_t* __restrict__ offsets,
+                                                         const int32_t* __restrict__ slot_of_expert, int E, int P,
+                                                         int d, int I, const uint8_t* __restrict__ pool,
+                                                         const uint8_t* __restrict__ shared_bank, size_t bank_bytes,
+                                                         size_t wd_off, float* __restrict__ y) {
+  const int r = blockIdx.x;
+  const int g = group_of_row(offsets, E, P, r);
+  const float* W = reinterpret_cast<const float*>(
+      (g < E ? pool + static_cast<size_t>(slot_of_expert[g]) * bank_bytes : shared_bank) + wd_off);
+  const float* hr = h + static_cast<size_t>(r) * I;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int j = blockIdx.y * 8 + warp; j < d; j += gridDim.y * 8) {
+    const float* wd = W + static_cast<size_t>(j) * I;
+    float a = 0.f;
+    for (int c = lane; c < I; c += 32) a = fmaf(hr[c], wd[c], a);
+    a = warp_sum(a);
+    if (lane == 0) y[static_cast<size_t>(r) * d + j] = a;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core path (bf16): persistent warp-specialised tcgen05 grouped GEMM.
+// ---------------------------------------------------------------------------
+constexpr int kTcThreads = 192;       // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue
+constexpr int kMaxGroups = 520;
+constexpr int kBK = 64;               // K per stage: 64 bf16 = one 128-byte swizzle row
+constexpr uint32_t kATileBytes = 128 * 128;
+
+struct TileInfo {
+  int g, m, n, rows, row0;
+};
+
+__device__ __forceinline__ TileInfo decode_tile(int t, const int32_t* tile_start, const int32_t* grp_rows,
+                                                const int32_t* grp_row0, int G, int MT, int BN) {
+  int lo = 0, hi = G;  // tile_start[lo] <= t < tile_start[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (tile_start[mid] <= t) lo = mid; else hi = mid;
+  }
+  TileInfo ti;
+  ti.g = lo;
+  ti.rows = grp_rows[lo];
+  ti.row0 = grp_row0[lo];
+  const int ntok = (ti.rows + BN - 1) / BN;
+  const int local = t - tile_start[lo];
+  ti.m = local / ntok;
+  ti.n = local % ntok;
+  (void)MT;
+  return ti;
+}
+
+template <int BN, bool GATED>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAsh,
+                  const __grid_constant__ CUtensorMap tmB, const int32_t* __restrict__ offsets,
+                  const int32_t* __restrict__ slot_of_expert, int E, int has_shared, int T, int P, int K, int Nw,
+                  int up_row0, uint16_t* __restrict__ out, int ld_out, int stages) {
+  constexpr uint32_t kBBytes = ((BN * 128 + 1023) / 1024) * 1024;
+  constexpr uint32_t kStageBytes = kATileBytes * (GATED ? 2 : 1) + kBBytes;
+  constexpr uint32_t kTx = kATileBytes * (GATED ? 2 : 1) + BN * 128;
+  constexpr uint32_t kAccCols = GATED ? 2 * BN : BN;
+  constexpr uint32_t kTmemCols = 2 * kAccCols < 32 ? 32 : 2 * kAccCols;
+  constexpr uint32_t kIdesc = idesc_bf16_f32(128, BN);
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[8], empty_bar[8], tfull_bar[2], tempty_bar[2];
+  __shared__ uint32_t tmem_holder;
+  __shared__ int32_t tile_start[kMaxGroups + 1], grp_rows[kMaxGroups], grp_row0[kMaxGroups];
+
+  const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (smem_base - smem_u32(smem_raw));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int G = E + (has_shared ? 1 : 0);
+  const int MT = Nw / 128;
+  const int KB = K / kBK;
+
+  // per-group rows and the tile prefix
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    const int rows = g < E ? offsets[g + 1] - offsets[g] : T;
+    grp_rows[g] = rows;
+    grp_row0[g] = g < E ? offsets[g] : P;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int per = (G + 31) / 32, b = lane * per, en = min(G, b + per);
+    int s = 0;
+    for (int g = b; g < en; ++g) s += ((grp_rows[g] + BN - 1) / BN) * MT;
+    int incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - s;
+    for (int g = b; g < en; ++g) { tile_start[g] = run; run += ((grp_rows[g] + BN - 1) / BN) * MT; }
+    if (lane == 31) tile_start[G] = incl;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 4); }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_holder, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmAsh);
+    tma_prefetch_desc(&tmB);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_holder;
+  const int total = tile_start[G];
+
+  auto a_tile = [&](int s, int which) -> uint8_t* {
+    return smem + static_cast<size_t>(s) * kStageBytes + which * kATileBytes;
+  };
+  auto b_tile = [&](int s) -> uint8_t* {
+    return smem + static_cast<size_t>(s) * kStageBytes + kATileBytes * (GATED ? 2 : 1);
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, MT, BN);
+        const int slot = ti.g < E ? slot_of_expert[ti.g] : 0;
+        const int brow = ti.row0 + ti.n * BN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full_bar[stage], kTx);
+          if (ti.g < E) {
+            tma_load_3d(a_tile(stage, 0), &tmA, &full_bar[stage], kb * kBK, ti.m * 128, slot);
+            if (GATED) tma_load_3d(a_tile(stage, 1), &tmA, &full_bar[stage], kb * kBK, up_row0 + ti.m * 128, slot);
+          } else {
+            tma_load_2d(a_tile(stage, 0), &tmAsh, &full_bar[stage], kb * kBK, ti.m * 128);
+            if (GATED) tma_load_2d(a_tile(stage, 1), &tmAsh, &full_bar[stage], kb * kBK, up_row0 + ti.m * 128);
+          }
+          tma_load_2d(b_tile(stage), &tmB, &full_bar[stage], kb * kBK, brow);
+          if (++stage == stages) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+        const int ab = it & 1;
+        const uint32_t aphase = (it >> 1) & 1;
+        if (!mbar_wait(&tempty_bar[ab], aphase ^ 1u)) break;
+        tc_fence_after();
+        const uint32_t d_g = tmem_base + ab * kAccCols;
+        const uint32_t d_u = d_g + BN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(a_tile(stage, 0));
+          const uint32_t sb = smem_u32(b_tile(stage));
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t bdesc = smem_desc_sw128(sb + kk * 32);
+            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            umma_f16(d_g, smem_desc_sw128(sa + kk * 32), bdesc, kIdesc, acc);
+            if (GATED) umma_f16(d_u, smem_desc_sw128(sa + kATileBytes + kk * 32), bdesc, kIdesc, acc);
+          }
+          umma_commit(&empty_bar[stage]);
+          if (++stage == stages) { stage = 0; phase ^= 1u; }
+        }
+        if (ok) umma_commit(&tfull_bar[ab]);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int q = warp % 4;  // TMEM lane quadrant this warp may access
+    int it = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+      const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, MT, BN);
+      const int ab = it & 1;
+      const uint32_t aphase = (it >> 1) & 1;
+      if (!mbar_wait(&tfull_bar[ab], aphase)) break;
+      tc_fence_after();
+      const int valid = min(BN, ti.rows - ti.n * BN);
+      const int wrow = ti.m * 128 + q * 32 + lane;
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * kAccCols;
+      uint16_t* obase = out + static_cast<size_t>(ti.row0 + ti.n * BN) * ld_out + wrow;
+      for (int c0 = 0; c0 < valid; c0 += 16) {
+        float a[16], b[16];
+        tmem_ld16(tb + c0, a);
+        if (GATED) tmem_ld16(tb + BN + c0, b);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          if (c0 + j < valid) {
+            const float v = GATED ? silu(a[j]) * b[j] : a[j];
+            const __nv_bfloat16 hv = __float2bfloat16_rn(v);
+            obase[static_cast<size_t>(c0 + j) * ld_out] = *reinterpret_cast<const uint16_t*>(&hv);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty_bar[ab]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 K-major map: dims {K, rows[, slots]}, box {64, box_rows[, 1]}, 128-byte swizzle.
+static bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint64_t row_pitch,
+                          uint64_t slots, uint64_t slot_pitch, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {K, rows, slots};
+  cuuint64_t strides[2] = {row_pitch, slot_pitch};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(kBK), box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  const cuuint32_t rank = slots > 0 ? 3 : 2;
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+
+template <int BN, bool GATED>
+static cudaError_t launch_tc(const CUtensorMap& mA, const CUtensorMap& mAsh, const CUtensorMap& mB,
+                             const FfnArgs& a, int K, int Nw, int up_row0, uint16_t* out, int ld_out,
+                             cudaStream_t st) {
+  constexpr uint32_t kBBytes = ((BN * 128 + 1023) / 1024) * 1024;
+  constexpr uint32_t kStageBytes = kATileBytes * (GATED ? 2 : 1) + kBBytes;
+  const int budget = 200 * 1024;
+  int stages = (budget - 1024) / static_cast<int>(kStageBytes);
+  if (stages > 8) stages = 8;
+  const size_t smem = 1024 + static_cast<size_t>(stages) * kStageBytes;
+  auto kern = ffn_tc_kernel<BN, GATED>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  const int P = a.T * a.k;
+  const int G = a.E + (a.has_shared ? 1 : 0);
+  const long max_tiles = static_cast<long>((P + BN - 1) / BN + G) * (Nw / 128);
+  const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
+  kern<<<grid, kTcThreads, smem, st>>>(mA, mAsh, mB, a.offsets, a.slot_of_expert, a.E, a.has_shared, a.T, P, K, Nw,
+                                       up_row0, out, ld_out, stages);
+  return cudaGetLastError();
+}
+
+template <bool GATED>
+static cudaError_t launch_tc_bn(int bn, const CUtensorMap& mA, const CUtensorMap& mAsh, const CUtensorMap& mB,
+                                const FfnArgs& a, int K, int Nw, int up_row0, uint16_t* out, int ld_out,
+                                cudaStream_t st) {
+  switch (bn) {
+    case 16: return launch_tc<16, GATED>(mA, mAsh, mB, a, K, Nw, up_row0, out, ld_out, st);
+    case 32: return launch_tc<32, GATED>(mA, mAsh, mB, a, K, Nw, up_row0, out, ld_out, st);
+    case 64: return launch_tc<64, GATED>(mA, mAsh, mB, a, K, Nw, up_row0, out, ld_out, st);
+    default: return launch_tc<128, GATED>(mA, mAsh, mB, a, K, Nw, up_row0, out, ld_out, st);
+  }
+}
+
+int ffn_token_tile(int P, int E) {
+  const int per = (P + E - 1) / E;
+  return per <= 16 ? 16 : per <= 32 ? 32 : per <= 64 ? 64 : 128;
+}
+
+// Returns a message on failure, nullptr on success.
+const char* launch_expert_ffn(const FfnArgs& a, cudaStream_t st, cudaError_t* cerr) {
+  const int P = a.T * a.k;
+  const int rows = P + (a.has_shared ? a.T : 0);
+  *cerr = cudaSuccess;
+  if (rows == 0) return nullptr;
+  const int elt = a.f32 ? 4 : 2;
+  {
+    const int grid = rows < 148 * 8 ? rows : 148 * 8;
+    gather_rows_kernel<<<grid, 256, 0, st>>>(a.x, a.perm, P, a.k, a.T, a.has_shared, a.d * elt, a.xp);
+    if ((*cerr = cudaGetLastError()) != cudaSuccess) return "gather launch failed";
+  }
+  if (a.f32) {
+    dim3 g1(rows, (a.I + 63) / 64), g2(rows, (a.d + 63) / 64);
+    simt_gemm1_kernel<<<g1, 256, 0, st>>>(reinterpret_cast<const float*>(a.xp), a.offsets, a.slot_of_expert, a.E, P,
+                                          a.d, a.I, a.pool, a.shared_bank, a.bank_bytes, a.w_gu_off,
+                                          reinterpret_cast<float*>(a.h));
+    if ((*cerr = cudaGetLastError()) != cudaSuccess) return "simt gemm1 launch failed";
+    simt_gemm2_kernel<<<g2, 256, 0, st>>>(reinterpret_cast<const float*>(a.h), a.offsets, a.slot_of_expert, a.E, P,
+                                          a.d, a.I, a.pool, a.shared_bank, a.bank_bytes, a.w_d_off,
+                                          reinterpret_cast<float*>(a.y));
+    if ((*cerr = cudaGetLastError()) != cudaSuccess) return "simt gemm2 launch failed";
+    return nullptr;
+  }
+  // bf16 tensor-core path
+  const int bn = ffn_token_tile(P, a.E);
+  CUtensorMap mA1, mAsh1, mB1, mA2, mAsh2, mB2;
+  const uint64_t S = static_cast<uint64_t>(a.S);
+  bool ok = make_map_bf16(&mA1, a.pool + a.w_gu_off, a.d, 2ull * a.I, 2ull * a.d, S, a.bank_bytes, 128) &&
+            make_map_bf16(&mA2, a.pool + a.w_d_off, a.I, a.d, 2ull * a.I, S, a.bank_bytes, 128) &&
+            make_map_bf16(&mB1, a.xp, a.d, rows, 2ull * a.d, 0, 0, bn) &&
+            make_map_bf16(&mB2, a.h, a.I, rows, 2ull * a.I, 0, 0, bn);
+  if (ok && a.has_shared) {
+    ok = make_map_bf16(&mAsh1, a.shared_bank + a.w_gu_off, a.d, 2ull * a.I, 2ull * a.d, 0, 0, 128) &&
+         make_map_bf16(&mAsh2, a.shared_bank + a.w_d_off, a.I, a.d, 2ull * a.I, 0, 0, 128);
+  } else {
+    mAsh1 = mA1;
+    mAsh2 = mA2;
+  }
+  if (!ok) return "cuTensorMapEncodeTiled failed";
+  if ((*cerr = launch_tc_bn<true>(bn, mA1, mAsh1, mB1, a, a.d, a.I, a.I, reinterpret_cast<uint16_t*>(a.h), a.I,
+                                  st)) != cudaSuccess)
+    return "tensor-core gemm1 launch failed";
+  if ((*cerr = launch_tc_bn<false>(bn, mA2, mAsh2, mB2, a, a.I, a.d, 0, reinterpret_cast<uint16_t*>(a.y), a.d,
+                                   st)) != cudaSuccess)
+    return "tensor-core gemm2 launch failed";
+  return nullptr;
+}
+
+}  // namespace ftm

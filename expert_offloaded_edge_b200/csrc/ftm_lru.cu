@@ -1,0 +1,146 @@
+// LRU slot-table lookup and update (step a4), one block.
+//
+// The pages' `offload` backend keeps a set of LRU slots in VRAM and copies
+// misses over PCIe (chenxutan.com FreeToken article, "choosing among the five
+// MoE backends"); the cache is global and evicts the expert unused for the
+// longest time (claypier.com "FreeToken MoE edge runtime", first section).
+//
+// Step s: mark the distinct requested experts; hits get last_use = s; the
+// misses, in ascending expert id, take the free-for-this-step slots in order
+// of (last_use, slot index).  Because each placement sets last_use = s, the
+// i-th miss simply takes the i-th candidate of that order, so the whole step
+// is a rank computation with no sequential dependence.
+//
+// Workspace (device int32): [0] status, [1] distinct, [2] hits, [3] misses,
+// [4 .. 4+2E) miss list (expert, slot) pairs, then a backup of the state
+// (slot_of_expert[E], expert_of_slot[S], last_use[S] as int64) for rollback.
+#include "ftm_common.cuh"
+
+namespace ftm {
+
+constexpr int kLruThreads = 1024;
+
+size_t lru_workspace_bytes(int E, int S) {
+  size_t b = sizeof(int32_t) * (4 + 2 * static_cast<size_t>(E) + E + S);
+  b = (b + 7) & ~static_cast<size_t>(7);
+  return b + sizeof(int64_t) * S;
+}
+
+__global__ void __launch_bounds__(kLruThreads) lru_step_kernel(const int32_t* __restrict__ ids, int P, int E, int S,
+                                                               int64_t step, int32_t* __restrict__ slot_of_expert,
+                                                               int32_t* __restrict__ expert_of_slot,
+                                                               int64_t* __restrict__ last_use,
+                                                               int32_t* __restrict__ ws) {
+  extern __shared__ int32_t sm[];
+  int32_t* want = sm;              // [E] 0/1
+  int32_t* miss_rank = want + E;   // [E+1] exclusive scan of miss flags
+  int32_t* cand = miss_rank + E + 1;  // [S] candidate flag, later victim_of_rank
+  int32_t* victim = cand + S;      // [S]
+  __shared__ int32_t s_distinct, s_hits;
+
+  for (int e = threadIdx.x; e < E; e += blockDim.x) want[e] = 0;
+  if (threadIdx.x == 0) { s_distinct = 0; s_hits = 0; }
+  __syncthreads();
+  for (int q = threadIdx.x; q < P; q += blockDim.x) want[ids[q]] = 1;
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    if (want[e]) atomicAdd(&s_distinct, 1);
+  __syncthreads();
+  const int distinct = s_distinct;
+  if (distinct > S) {
+    if (threadIdx.x == 0) { ws[0] = FTM_ERR_CAPACITY; ws[1] = distinct; ws[2] = 0; ws[3] = 0; }
+    return;
+  }
+  // backup for rollback
+  int32_t* bk_soe = ws + 4 + 2 * E;
+  int32_t* bk_eos = bk_soe + E;
+  size_t off = sizeof(int32_t) * (4 + 2 * static_cast<size_t>(E) + E + S);
+  off = (off + 7) & ~static_cast<size_t>(7);
+  int64_t* bk_lu = reinterpret_cast<int64_t*>(reinterpret_cast<uint8_t*>(ws) + off);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) bk_soe[e] = slot_of_expert[e];
+  for (int j = threadIdx.x; j < S; j += blockDim.x) { bk_eos[j] = expert_of_slot[j]; bk_lu[j] = last_use[j]; }
+  __syncthreads();
+
+  // hits
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int sl = slot_of_expert[e];
+    const bool miss = want[e] && sl < 0;
+    if (want[e] && sl >= 0) { last_use[sl] = step; atomicAdd(&s_hits, 1); }
+    want[e] = miss ? 1 : 0;   // from here on: miss flag
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    // exclusive scan of miss flags (warp 0)
+    const int lane = threadIdx.x;
+    const int per = (E + 31) / 32, b = lane * per, en = min(E, b + per);
+    int s = 0;
+    for (int e = b; e < en; ++e) s += want[e];
+    int incl = s;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - s;
+    for (int e = b; e < en; ++e) { miss_rank[e] = run; run += want[e]; }
+    if (lane == 31) miss_rank[E] = incl;
+  }
+  for (int j = threadIdx.x; j < S; j += blockDim.x) cand[j] = last_use[j] < step ? 1 : 0;
+  __syncthreads();
+  // rank of each candidate slot in (last_use, index) order
+  for (int j = threadIdx.x; j < S; j += blockDim.x) {
+    if (!cand[j]) continue;
+    const int64_t lj = last_use[j];
+    int r = 0;
+    for (int i = 0; i < S; ++i)
+      if (cand[i]) {
+        const int64_t li = last_use[i];
+        r += (li < lj || (li == lj && i < j)) ? 1 : 0;
+      }
+    victim[r] = j;
+  }
+  __syncthreads();
+  const int misses = miss_rank[E];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    if (!want[e]) continue;
+    const int r = miss_rank[e];
+    const int sl = victim[r];
+    const int old = expert_of_slot[sl];
+    if (old >= 0) slot_of_expert[old] = -1;
+    slot_of_expert[e] = sl;
+    expert_of_slot[sl] = e;
+    last_use[sl] = step;
+    ws[4 + 2 * r] = e;
+    ws[4 + 2 * r + 1] = sl;
+  }
+  if (threadIdx.x == 0) { ws[0] = FTM_OK; ws[1] = distinct; ws[2] = s_hits; ws[3] = misses; }
+}
+
+__global__ void lru_restore_kernel(int E, int S, int32_t* __restrict__ slot_of_expert,
+                                   int32_t* __restrict__ expert_of_slot, int64_t* __restrict__ last_use,
+                                   const int32_t* __restrict__ ws) {
+  const int32_t* bk_soe = ws + 4 + 2 * E;
+  const int32_t* bk_eos = bk_soe + E;
+  size_t off = sizeof(int32_t) * (4 + 2 * static_cast<size_t>(E) + E + S);
+  off = (off + 7) & ~static_cast<size_t>(7);
+  const int64_t* bk_lu = reinterpret_cast<const int64_t*>(reinterpret_cast<const uint8_t*>(ws) + off);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) slot_of_expert[e] = bk_soe[e];
+  for (int j = threadIdx.x; j < S; j += blockDim.x) { expert_of_slot[j] = bk_eos[j]; last_use[j] = bk_lu[j]; }
+}
+
+cudaError_t launch_lru_step(const int32_t* ids, int P, int E, int S, int64_t step, int32_t* soe, int32_t* eos,
+                            int64_t* lu, int32_t* ws, cudaStream_t st) {
+  const size_t smem = sizeof(int32_t) * (2 * static_cast<size_t>(E) + 1 + 2 * S);
+  cudaError_t err =
+      cudaFuncSetAttribute(lru_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  lru_step_kernel<<<1, kLruThreads, smem, st>>>(ids, P, E, S, step, soe, eos, lu, ws);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lru_restore(int E, int S, int32_t* soe, int32_t* eos, int64_t* lu, const int32_t* ws,
+                               cudaStream_t st) {
+  lru_restore_kernel<<<1, kLruThreads, 0, st>>>(E, S, soe, eos, lu, ws);
+  return cudaGetLastError();
+}
+
+}  // namespace ftm

@@ -1,0 +1,216 @@
+/*
+ * ftm.h -- C ABI of a B200 (sm_100a) routed Mixture-of-Experts layer over a
+ * slot-indexed expert cache.
+ *
+ * What the layer computes (FreeToken pages):
+ *  - chenxutan.com FreeToken article, section "why the bottleneck is bandwidth,
+ *    not capacity": every token activates a few routed experts; the full expert
+ *    pool may live in host memory and experts are pulled into VRAM on demand.
+ *  - same article, section "choosing among the five MoE backends", `offload`:
+ *    experts in host RAM, LRU slots in VRAM, misses copied over PCIe.
+ *  - claypier.com "FreeToken MoE edge runtime", first section: a global LRU
+ *    cache evicts the expert weights unused for the longest time.
+ *  - pomoai.com FreeToken hub, checkpoint list: BF16, FP8 and NVFP4 weights.
+ * The pages print no formula; the layer is the plain top-k routed SwiGLU MoE:
+ *   logits = x Wr^T + b;  ids = top-k(logits);  g = softmax(logits) restricted
+ *   to the k picks and renormalised;  h = silu(x Wg_e^T) * (x Wu_e^T);
+ *   y = h Wd_e^T;  out[t] = sum_j g[t][j] y[t,j]  (+ shared expert FFN(x[t])).
+ *
+ * Conventions for every entry point:
+ *  - Pointers marked "device" are CUDA device pointers, "host" are host
+ *    pointers.  The caller owns every buffer; the library never allocates device
+ *    or host memory and keeps no per-call state beyond a thread-local error
+ *    string and one cached CUDA event per thread for the miss-copy ordering.
+ *  - `stream` arguments are cudaStream_t values passed as void* (NULL = the
+ *    legacy default stream).  Work is enqueued asynchronously; the only entry
+ *    point that synchronises the host is ftm_slot_lookup_update on a cache step
+ *    (it must read the miss list before it can issue the copies).
+ *  - Arguments are validated before anything is enqueued; on error nothing is
+ *    launched, the function returns a non-zero ftm_status and ftm_last_error()
+ *    describes it.  No C++ exception crosses this boundary.
+ *  - Device-side faults of the library's own kernels (a bounded wait that timed
+ *    out) are recorded in a device status word read by ftm_device_status().
+ *
+ * Activation dtype: FTM_F32 layers take fp32 x, fp32 router weights and write
+ * fp32 out; every other layer takes bf16 x (raw bits, row-major [T][d]), bf16
+ * router weights and writes bf16 out.  Router bias and gates are fp32.
+ */
+#ifndef FTM_H_
+#define FTM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ftm_status {
+  FTM_OK = 0,
+  FTM_ERR_INVALID_ARG = 1,   /* a size, pointer, alignment or layout is out of contract */
+  FTM_ERR_UNSUPPORTED = 2,   /* valid layer, but no kernel for it (dtype/shape) */
+  FTM_ERR_CAPACITY = 3,      /* more distinct experts in one step than cache slots */
+  FTM_ERR_CUDA = 4           /* a CUDA call failed (message in ftm_last_error) */
+} ftm_status;
+
+typedef enum ftm_wdtype {
+  FTM_F32 = 0,               /* fp32 expert weights */
+  FTM_BF16 = 1,              /* bf16 expert weights */
+  FTM_FP8_E4M3_B128 = 2,     /* e4m3 weights, one fp32 scale per 128x128 block */
+  FTM_NVFP4 = 3              /* e2m1 weights, one e4m3 scale per 16 elements + fp32 per-tensor scale */
+} ftm_wdtype;
+
+/* One layer's shape.  Limits: d, I multiples of 128 (of 256 for NVFP4);
+ * 1 <= k <= min(E, 16); 1 <= E <= 512; 1 <= S. */
+typedef struct ftm_layer_desc {
+  int32_t d;            /* hidden size */
+  int32_t E;            /* routed experts */
+  int32_t k;            /* picks per token */
+  int32_t I;            /* SwiGLU intermediate size */
+  int32_t has_shared;   /* 1: one always-on shared expert (gate weight 1) */
+  int32_t S;            /* expert slots in the HBM pool */
+  int32_t wdtype;       /* ftm_wdtype */
+  int32_t reserved;     /* must be 0 */
+} ftm_layer_desc;
+
+/* Layout of one expert "bank": the contiguous byte range holding all of one
+ * expert's weights, so a cache miss is a single copy.  All offsets are from
+ * the bank start and 256-byte aligned; bank_bytes is a multiple of 256.
+ *   w_gu: [2I][d] row-major, rows 0..I-1 = gate projection, I..2I-1 = up
+ *         (f32 / bf16 / e4m3 elements; NVFP4: [2I][d/2] bytes, two codes per
+ *         byte, element 2j in the low nibble)
+ *   w_d : [d][I] row-major (same element rules)
+ *   s_gu: FP8: fp32 [2I/128][d/128]; NVFP4: e4m3 [2I][d/16]; else empty
+ *   s_d : FP8: fp32 [d/128][I/128];  NVFP4: e4m3 [d][I/16];  else empty
+ *   s_t : NVFP4: fp32[4] = {gate, up, down, 0} per-tensor scales; else empty */
+typedef struct ftm_bank_layout {
+  uint64_t bank_bytes;
+  uint64_t w_gu_off, w_gu_bytes;
+  uint64_t w_d_off, w_d_bytes;
+  uint64_t s_gu_off, s_gu_bytes;
+  uint64_t s_d_off, s_d_bytes;
+  uint64_t s_t_off, s_t_bytes;
+} ftm_bank_layout;
+
+ftm_status ftm_get_bank_layout(const ftm_layer_desc* L, ftm_bank_layout* out);
+
+/* Router + gating (a1, a2).
+ *   x        device [T][d] (fp32 or bf16, see above)
+ *   w_router device [E][d] row-major (same dtype as x)
+ *   bias     device fp32 [E] added to every logit, or NULL
+ *   topk_ids device int32 [T][k]: picks in descending logit order, equal
+ *            logits to the lower expert id
+ *   topk_w   device fp32 [T][k]: softmax over all E logits, renormalised over
+ *            the k picks (= softmax of the k picked logits)
+ * Logits are accumulated in fp32.  T = 0 is a no-op. */
+ftm_status ftm_route(const ftm_layer_desc* L, const void* x, int32_t T, const void* w_router,
+                     const float* bias, int32_t* topk_ids, float* topk_w, void* stream);
+
+/* Permutation of the P = T*k (token, pick) pairs by expert (a3).
+ *   counts  device int32 [E]     pairs per expert
+ *   offsets device int32 [E+1]   exclusive prefix sum, offsets[E] = P
+ *   perm    device int32 [P]     perm[pos] = q = t*k + j, stable: pairs of one
+ *                                expert appear in ascending q
+ *   inv     device int32 [P]     inv[q] = pos
+ *   workspace device, >= ftm_permute_workspace_bytes(L, T) bytes, 256-aligned
+ * Deterministic: identical results run to run. */
+ftm_status ftm_permute(const ftm_layer_desc* L, const int32_t* topk_ids, int32_t T, int32_t* counts,
+                       int32_t* offsets, int32_t* perm, int32_t* inv, void* workspace, size_t ws_bytes,
+                       void* stream);
+size_t ftm_permute_workspace_bytes(const ftm_layer_desc* L, int32_t T);
+
+/* The LRU slot cache (a4).  State lives in caller-owned device arrays:
+ *   slot_of_expert [E] (-1: not resident), expert_of_slot [S] (-1: empty),
+ *   last_use [S] int64 (-1: never).
+ * A step s requests the distinct expert ids routed in that step (the shared
+ * expert is not cached).  Hits set last_use = s.  Misses, in ascending expert
+ * id, each take the slot with the smallest last_use among slots not used in
+ * step s (ties: lowest slot index); the slot's previous expert is unmapped and
+ * the expert's bank is copied host_pool[e] -> slot_pool[slot]. */
+typedef struct ftm_slot_cache {
+  int32_t* slot_of_expert;      /* device [E] */
+  int32_t* expert_of_slot;      /* device [S] */
+  int64_t* last_use;            /* device [S] */
+  int64_t step;                 /* host: index s of the next step; +1 per successful update */
+  void* slot_pool;              /* device: S banks of bank_bytes, slot j at j*bank_bytes */
+  const void* host_pool;        /* host, pinned (cudaHostAlloc/cudaHostRegister): E banks */
+  int32_t* host_scratch;        /* host, pinned, >= ftm_slot_host_scratch_ints(L) int32 */
+  int32_t last_distinct;        /* out: distinct experts requested by the last step */
+  int32_t last_hits;            /* out: of which resident */
+  int32_t last_misses;          /* out: of which copied in */
+  int32_t fail_before_copy;     /* test hook: != 0 makes the next update fail as if its
+                                   first copy had failed; state is rolled back */
+} ftm_slot_cache;
+
+size_t ftm_slot_host_scratch_ints(const ftm_layer_desc* L);
+size_t ftm_slot_workspace_bytes(const ftm_layer_desc* L);
+
+/* One cache step.  Runs the lookup/update kernel on `compute_stream`,
+ * synchronises that stream to read the miss list (the one host sync of the
+ * path), issues one cudaMemcpyAsync per miss on `copy_stream`, and makes
+ * `compute_stream` wait for the copies, so work enqueued afterwards on
+ * `compute_stream` sees the new slots.  Returns FTM_ERR_CAPACITY (state
+ * unchanged) when more than S distinct experts are requested, FTM_ERR_CUDA
+ * (state rolled back to before the call) when a copy cannot be issued.
+ *   workspace device, >= ftm_slot_workspace_bytes(L) bytes */
+ftm_status ftm_slot_lookup_update(const ftm_layer_desc* L, ftm_slot_cache* C, const int32_t* topk_ids,
+                                  int32_t T, void* workspace, size_t ws_bytes, void* compute_stream,
+                                  void* copy_stream);
+
+/* Grouped SwiGLU expert FFN (a5, a6, a7).
+ *   x              device [T][d] activations (token order)
+ *   offsets, perm  from ftm_permute
+ *   slot_of_expert device int32 [E]: bank of expert e is slot_pool[slot_of_expert[e]]
+ *   slot_pool      device, S banks (layout from ftm_get_bank_layout)
+ *   shared_bank    device, one bank, required iff L->has_shared
+ *   y              device [P + (has_shared ? T : 0)][d]: row pos = the FFN output of
+ *                  pair perm[pos] (unweighted); rows P..P+T-1 = shared expert of token t
+ *                  (bf16; fp32 for FTM_F32)
+ *   workspace      device, >= ftm_ffn_workspace_bytes(L, T) bytes, 256-aligned
+ * Every expert that has pairs must be resident (slot_of_expert[e] in [0,S)). */
+ftm_status ftm_expert_ffn(const ftm_layer_desc* L, const void* x, int32_t T, const int32_t* offsets,
+                          const int32_t* perm, const int32_t* slot_of_expert, const void* slot_pool,
+                          const void* shared_bank, void* y, void* workspace, size_t ws_bytes,
+                          void* stream);
+size_t ftm_ffn_workspace_bytes(const ftm_layer_desc* L, int32_t T);
+
+/* Weighted un-permute and combine (a8):
+ *   out[t] = sum_{j=0..k-1 ascending} topk_w[t][j] * y[inv[t*k+j]]  (+ y[P+t] if has_shared),
+ * accumulated in fp32.  y, inv, topk_w device; out device [T][d]. */
+ftm_status ftm_combine(const ftm_layer_desc* L, const void* y, const int32_t* inv, const float* topk_w,
+                       int32_t T, void* out, void* stream);
+
+/* Weights of one layer for ftm_moe_layer_forward. */
+typedef struct ftm_layer_weights {
+  const void* w_router;            /* device [E][d] */
+  const float* router_bias;        /* device [E] or NULL */
+  const void* slot_pool;           /* device, S banks (resident layers; ignored with a cache) */
+  const int32_t* slot_of_expert;   /* device [E] (resident layers; ignored with a cache) */
+  const void* shared_bank;         /* device, one bank, or NULL */
+} ftm_layer_weights;
+
+/* The whole layer: route -> permute -> [cache step] -> expert FFN -> combine.
+ *   C          NULL for a resident layer (every expert in W->slot_pool at
+ *              W->slot_of_expert[e]); otherwise the LRU cache (its slot_pool and
+ *              slot_of_expert are used, and the call synchronises once, see
+ *              ftm_slot_lookup_update)
+ *   x, out     device [T][d]
+ *   workspace  device, >= ftm_workspace_bytes(L, T) bytes, 256-aligned
+ *   copy_stream  stream for the miss copies (only used with a cache) */
+ftm_status ftm_moe_layer_forward(const ftm_layer_desc* L, const ftm_layer_weights* W, ftm_slot_cache* C,
+                                 const void* x, int32_t T, void* out, void* workspace, size_t ws_bytes,
+                                 void* stream, void* copy_stream);
+size_t ftm_workspace_bytes(const ftm_layer_desc* L, int32_t T_max);
+
+/* Thread-local description of the last error returned on this thread. */
+const char* ftm_last_error(void);
+
+/* Reads (and if reset != 0 clears) the device status word the kernels set when
+ * a bounded wait gives up.  Synchronises the device.  0 = no fault. */
+int32_t ftm_device_status(int32_t reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FTM_H_ */

@@ -1,0 +1,78 @@
+"""Helpers of the GPU parity tests: run the C ABI on a staged layer and build the
+oracle's expected values from the same seeded inputs."""
+from __future__ import annotations
+
+from typing import Dict, Optional, Sequence
+
+import numpy as np
+import torch
+
+import expert_offloaded_edge_b200 as ftm
+import oracle
+import synth
+from synth.device import DeviceLayer
+
+TOL = {"f32": 2e-2, "bf16": 2e-2, "fp8": 5e-2, "nvfp4": 5e-2}
+TOL_F32_SIMT = 1e-4
+
+
+def screened_layer(cfg: synth.LayerConfig, T: int, steps: int = 1, seed: int = 0, slot_perm=None) -> DeviceLayer:
+    """A device layer whose hidden rows are screened for the top-k margin by the oracle."""
+    base = synth.Layer(cfg, seed)
+    Wr = base.router_f32()
+    b = base.bias()
+    table = synth.screen_hidden(base, T, steps,
+                                lambda x: oracle.margin_ok(oracle.router_logits(x, Wr, b), cfg.k, synth.MARGIN))
+    return DeviceLayer(cfg, seed, redraws=table, slot_perm=slot_perm)
+
+
+def storage_to_f32(dl: DeviceLayer, arr: np.ndarray) -> np.ndarray:
+    return oracle.bf16_to_f32(arr) if dl.cfg.act_dtype == "bf16" else np.asarray(arr, np.float32)
+
+
+def oracle_route(dl: DeviceLayer, T: int, step: int = 0):
+    x = storage_to_f32(dl, dl.layer.hidden_storage(T, step))
+    Wr = storage_to_f32(dl, dl.layer.router_storage())
+    ids, g, lg = oracle.route(x, Wr, dl.layer.bias(), dl.cfg.k)
+    return x, ids, g
+
+
+def to_np_f32(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy()
+
+
+class Workspace:
+    def __init__(self, nbytes: int, device="cuda"):
+        self.nbytes = max(int(nbytes), 256)
+        self.buf = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device)
+        off = (-self.buf.data_ptr()) % 256
+        self.ptr = self.buf.data_ptr() + off
+
+
+def run_layer(dl: DeviceLayer, x_dev: torch.Tensor, T: int, cache: bool = False) -> torch.Tensor:
+    out = torch.empty((T, dl.cfg.d), dtype=dl.out_dtype(), device=x_dev.device)
+    ws = Workspace(ftm.ftm_workspace_bytes(dl.desc, T))
+    copy_stream = torch.cuda.Stream() if cache else None
+    ftm.ftm_moe_layer_forward(dl.desc, dl.weights(), dl.cache if cache else None, x_dev, T, out, ws.ptr, ws.nbytes,
+                              None, copy_stream)
+    torch.cuda.synchronize()
+    assert ftm.ftm_device_status(True) == 0
+    return out
+
+
+def oracle_rows(dl: DeviceLayer, x: np.ndarray, ids: np.ndarray, g: np.ndarray, rows: Sequence[int],
+                cache: Optional[Dict] = None) -> np.ndarray:
+    return oracle.moe_rows(dl.layer, x, rows, ids, g, weight_cache=cache)
+
+
+def assert_rows_close(got: np.ndarray, want: np.ndarray, frac: float, what: str = ""):
+    """max-abs error per token row <= frac * max |oracle row|."""
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    assert got.shape == want.shape, (got.shape, want.shape)
+    err = np.abs(got - want).max(axis=1)
+    scale = np.abs(want).max(axis=1)
+    bad = np.nonzero(err > frac * scale)[0]
+    worst = float((err / np.maximum(scale, 1e-30)).max()) if len(err) else 0.0
+    assert bad.size == 0, f"{what}: {bad.size} rows exceed {frac} (worst ratio {worst:.3g}, rows {bad[:8]})"
+    return worst

@@ -1,0 +1,77 @@
+"""CPU checks of the C ABI: the library loads, exports every symbol the header
+declares, and rejects out-of-contract arguments before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import expert_offloaded_edge_b200 as ftm
+import synth
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "ftm.h")
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ftm_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert len(names) >= 14
+    lib = ftm.library()
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_bank_layouts():
+    want = {
+        "tiny": 3 * 256 * 512 * 4,
+        "35b_decode": 3 * 2048 * 768 * 2,
+        "284b_trace": 3 * 4096 * 2048 + (2 * 2048 // 128) * (4096 // 128) * 4 + (4096 // 128) * (2048 // 128) * 4,
+        "753b_nvfp4": 3 * 6144 * 2048 // 2 + 3 * 6144 * 2048 // 16 + 256,
+    }
+    for name, nbytes in want.items():
+        bl = ftm.ftm_get_bank_layout(ftm.desc_for(synth.CONFIGS[name]))
+        assert bl.bank_bytes % 256 == 0
+        assert nbytes <= bl.bank_bytes < nbytes + 5 * 256, name
+        assert bl.w_gu_off == 0 and bl.w_d_off >= bl.w_gu_bytes
+    bl = ftm.ftm_get_bank_layout(ftm.desc_for(synth.CONFIGS["284b_trace"]))
+    assert bl.bank_bytes == 25171968           # 25.17 MB per FP8 expert incl. 6,144 B of block scales
+
+
+@pytest.mark.parametrize("field,value", [("d", 100), ("d", 0), ("I", 96), ("k", 0), ("k", 9), ("E", 0),
+                                         ("E", 600), ("S", 0), ("wdtype", 7), ("reserved", 1), ("has_shared", 2)])
+def test_invalid_desc_rejected_without_gpu(field, value):
+    d = ftm.desc_for(synth.CONFIGS["35b_decode"])
+    if field == "k" and value == 9:
+        d.E = 8
+    setattr(d, field, value)
+    with pytest.raises(ftm.FtmError) as ei:
+        ftm.ftm_get_bank_layout(d)
+    assert ei.value.status == 1
+    assert ftm.ftm_last_error()
+
+
+def test_invalid_calls_rejected_without_gpu():
+    d = ftm.desc_for(synth.CONFIGS["35b_decode"])
+    lib = ftm.library()
+    assert lib.ftm_route(None, None, 1, None, None, None, None, None) == 1
+    assert lib.ftm_route(ctypes.byref(d), None, -1, None, None, None, None, None) == 1
+    assert lib.ftm_route(ctypes.byref(d), None, 4, None, None, None, None, None) == 1
+    assert lib.ftm_route(ctypes.byref(d), None, 0, None, None, None, None, None) == 0      # T = 0: no-op
+    # workspace too small / misaligned
+    assert lib.ftm_permute(ctypes.byref(d), 16, 9000, 16, 16, 16, 16, None, 0, None) == 1
+    assert lib.ftm_moe_layer_forward(ctypes.byref(d), None, None, None, 4, None, None, 0, None, None) == 1
+    assert lib.ftm_combine(ctypes.byref(d), None, None, None, 3, None, None) == 1
+    assert "NULL" in ftm.ftm_last_error()
+
+
+def test_workspace_sizes_monotone():
+    for name in synth.CONFIGS:
+        d = ftm.desc_for(synth.CONFIGS[name])
+        sizes = [ftm.ftm_workspace_bytes(d, T) for T in (0, 1, 16, 1024, 16384)]
+        assert sizes == sorted(sizes) and sizes[1] > 0
+        assert ftm.ftm_ffn_workspace_bytes(d, 16) <= ftm.ftm_workspace_bytes(d, 16)
