@@ -1,0 +1,448 @@
+#!/usr/bin/env python
+"""Benchmark of one routed-MoE layer forward pass (route -> permute -> [slot
+cache step] -> grouped SwiGLU FFN -> combine) on B200, through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--T T]
+    python bench.py --impl reference ...      # the CPU oracle on the host cores
+
+One step = one layer pass over one batch of T tokens.  N > 1 (torchrun): every
+rank runs its own replica on its own batch (tokens are independent, no data
+collective); value = all ranks' tokens / max-over-ranks time.  Prints one JSON
+line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import expert_offloaded_edge_b200 as ftm  # noqa: E402
+import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s; decode HBM GB/s & prefill TFLOP/s as % of B200 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", default="ftm", choices=["ftm", "reference"])
+    p.add_argument("--config", default="35b_decode", choices=list(synth.CONFIGS))
+    p.add_argument("--T", type=int, default=None, help="tokens per step (default: the config's largest)")
+    p.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying CUDA graphs")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    return p.parse_args()
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.p = None
+
+    def stop(self) -> dict:
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.count(",") >= 8]
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i] and "Not" not in r[5 + i]})
+        load = [s for s in sm if s > 0.5 * (max(mx) if mx else 1)] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- peaks / traffic
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for n in ("ftm_ffn.cu", "ftm_common.cuh"):
+        with open(os.path.join(ROOT, "expert_offloaded_edge_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str, kernel: str):
+    """dram bytes per launch from the committed ncu summary, or None if absent
+    or taken on a different version of the kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(f"{workload}/{kernel}")
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------------- workload
+def workload_name(cfg, T):
+    return f"{cfg.name} T={T}"
+
+
+class Runner:
+    """Graph-replayed (or eager) layer steps with per-kernel CUDA events."""
+
+    KERNELS = (ftm.binding.FTM_K_ROUTE, ftm.binding.FTM_K_PERMUTE, ftm.binding.FTM_K_GATHER,
+               ftm.binding.FTM_K_GEMM1, ftm.binding.FTM_K_GEMM2, ftm.binding.FTM_K_COMBINE)
+
+    def __init__(self, dl, T, use_graph: bool, chunk: int = 20):
+        from synth.device import Workspace
+        self.dl, self.T = dl, T
+        self.x = dl.hidden(T)
+        self.out = torch.empty((T, dl.cfg.d), dtype=dl.out_dtype(), device="cuda")
+        self.ws = Workspace(ftm.ftm_workspace_bytes(dl.desc, T))
+        self.weights = dl.weights()
+        self.use_graph = use_graph
+        self.chunk = chunk
+        self.graphs = {}
+        self.stream = torch.cuda.Stream()
+
+    def _step(self):
+        ftm.ftm_moe_layer_forward(self.dl.desc, self.weights, None, self.x, self.T, self.out, self.ws.ptr,
+                                  self.ws.nbytes, self.stream)
+
+    def _events(self, n):
+        return [{k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for k in self.KERNELS} for _ in range(n)]
+
+    def _record_steps(self, evs):
+        for ev in evs:
+            for k, (a, b) in ev.items():
+                ftm.ftm_set_profile_events(k, a, b)
+            self._step()
+        for k in self.KERNELS:
+            ftm.ftm_set_profile_events(k, None, None)
+
+    def _graph(self, n, tag):
+        key = (n, tag)
+        if key not in self.graphs:
+            evs = self._events(n)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(self.stream):
+                self._step()          # first launch outside capture (sets kernel attributes)
+                self.stream.synchronize()
+                with torch.cuda.graph(g, stream=self.stream):
+                    self._record_steps(evs)
+            self.graphs[key] = (g, evs)
+        return self.graphs[key]
+
+    def run(self, nsteps: int, collect: dict = None):
+        """Enqueue nsteps steps on self.stream; per-kernel ms appended to collect."""
+        if nsteps <= 0:
+            return
+        if not self.use_graph:
+            evs = self._events(nsteps)
+            with torch.cuda.stream(self.stream):
+                self._record_steps(evs)
+            if collect is not None:
+                self.stream.synchronize()
+                self._collect(evs, collect)
+            return
+        done = 0
+        pending = []
+        tag = 0
+        while done < nsteps:
+            n = min(self.chunk, nsteps - done)
+            g, evs = self._graph(n, tag)
+            if len(pending) == 2:     # the graph about to be replayed last ran two chunks ago
+                pe = pending.pop(0)
+                if collect is not None:
+                    pe[-1][self.KERNELS[-1]][1].synchronize()
+                    self._collect(pe, collect)
+            g.replay()
+            pending.append(evs)
+            tag ^= 1
+            done += n
+        if collect is not None:
+            for pe in pending:
+                pe[-1][self.KERNELS[-1]][1].synchronize()
+                self._collect(pe, collect)
+
+    @staticmethod
+    def _collect(evs, collect):
+        for ev in evs:
+            for k, (a, b) in ev.items():
+                collect.setdefault(k, []).append(a.elapsed_time(b))
+
+
+def routing_stats(dl, T):
+    """Active experts of the benchmarked batch, from the library's own routing."""
+    cfg = dl.cfg
+    x = dl.hidden(T)
+    ids = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
+    gw = torch.empty((T, cfg.k), dtype=torch.float32, device="cuda")
+    ftm.ftm_route(dl.desc, x, T, dl.w_router, dl.bias, ids, gw)
+    torch.cuda.synchronize()
+    counts = np.bincount(ids.cpu().numpy().ravel(), minlength=cfg.E)
+    return counts
+
+
+def algorithmic(dl, T, counts):
+    """Algorithmic bytes and flops of GEMM1 and of the whole step."""
+    cfg = dl.cfg
+    wb = {"f32": 4, "bf16": 2, "fp8": 1, "nvfp4": 0.5}[cfg.wdtype]
+    ab = 4 if cfg.act_dtype == "f32" else 2
+    groups = int((counts > 0).sum()) + (1 if cfg.has_shared else 0)
+    rows = T * cfg.k + (T if cfg.has_shared else 0)
+    g1_bytes = groups * 2 * cfg.I * cfg.d * wb + rows * cfg.d * ab + rows * cfg.I * ab
+    g2_bytes = groups * cfg.d * cfg.I * wb + rows * cfg.I * ab + rows * cfg.d * ab
+    g1_flops = 2.0 * rows * cfg.d * 2 * cfg.I
+    g2_flops = 2.0 * rows * cfg.I * cfg.d
+    return {"groups": groups, "rows": rows, "gemm1_bytes": g1_bytes, "gemm2_bytes": g2_bytes,
+            "gemm1_flops": g1_flops, "gemm2_flops": g2_flops}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def oracle_tokens_per_s(cfg, T, seconds: float, step_tokens: int = 1):
+    """The oracle layer (router for the sampled tokens, their k experts and the
+    shared expert, combine) on the host cores; returns (tokens/s, tokens, cores, s)."""
+    import oracle
+    layer = synth.Layer(cfg, 0, synth.load_redraws(cfg.name, max(cfg.T)) or {})
+    x_all = layer.hidden_f32(T)
+    Wr = layer.router_f32()
+    b = layer.bias()
+    cache = {}
+    done, t_used = 0, 0.0
+    t = 0
+    while t_used < seconds:
+        rows = [(t + i) % T for i in range(step_tokens)]
+        xs = x_all[rows]
+        # dequantised weights are the layer's stored parameters: load them outside the timed part
+        ids, g, _ = oracle.route(xs, Wr, b, cfg.k)
+        for e in set(ids.ravel().tolist()) | ({cfg.E} if cfg.has_shared else set()):
+            if e not in cache:
+                cache[e] = oracle.expert_weights_f32(layer, e)
+        t0 = time.perf_counter()
+        ids, g, _ = oracle.route(xs, Wr, b, cfg.k)
+        oracle.moe_rows(layer, xs, range(len(rows)), ids, g, weight_cache=cache)
+        t_used += time.perf_counter() - t0
+        done += len(rows)
+        t += step_tokens
+        if len(cache) > 48:
+            cache.clear()
+    return done / t_used, done, oracle.threads(), t_used
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return
+    cfg = synth.CONFIGS[args.config]
+    T = args.T or max(cfg.T)
+    import oracle
+    layer = synth.Layer(cfg, 0, synth.load_redraws(cfg.name, max(cfg.T)) or {})
+    x_all = layer.hidden_f32(T)
+    Wr = layer.router_f32()
+    b = layer.bias()
+    cache = {}
+
+    def step(i):
+        rows = [i % T]
+        xs = x_all[rows]
+        ids, g, _ = oracle.route(xs, Wr, b, cfg.k)
+        for e in set(ids.ravel().tolist()) | ({cfg.E} if cfg.has_shared else set()):
+            if e not in cache:
+                cache[e] = oracle.expert_weights_f32(layer, e)
+        t0 = time.perf_counter()
+        ids, g, _ = oracle.route(xs, Wr, b, cfg.k)
+        oracle.moe_rows(layer, xs, range(1), ids, g, weight_cache=cache)
+        dt = time.perf_counter() - t0
+        if len(cache) > 48:
+            cache.clear()
+        return dt
+
+    for i in range(args.warmup):
+        step(i)
+    tot = sum(step(args.warmup + i) for i in range(args.steps))
+    v = args.steps / tot
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64-accumulate/f32",
+            "data": "synthetic", "config": {"workload": workload_name(cfg, T), "d": cfg.d, "E": cfg.E, "k": cfg.k,
+                                            "I": cfg.I, "T": T, "wdtype": cfg.wdtype},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+                             "sample": f"each step = 1 token of the {workload_name(cfg, T)} batch through the full "
+                                       f"oracle layer (router, {cfg.k} experts, combine)"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- main arm
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return reference_arm(args, rank, world)
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    cfg = synth.CONFIGS[args.config]
+    T = args.T or max(cfg.T)
+    if cfg.lru:
+        raise SystemExit("use bench_trace for the slot-cache trace configuration")
+    from synth.device import DeviceLayer
+    dl = DeviceLayer(cfg)
+    counts = routing_stats(dl, T)
+    alg = algorithmic(dl, T, counts)
+    use_graph = not args.no_graph
+    r = Runner(dl, T, use_graph)
+
+    # warm-up (untimed)
+    r.run(args.warmup)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    per_kernel = {}
+    t0.record(r.stream)
+    r.run(args.steps, per_kernel)
+    t1.record(r.stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    clk = clocks.stop()
+    if dist:
+        tt = torch.tensor([ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+        dist.barrier()
+    tokens = args.steps * T * world
+    value = tokens / (ms / 1e3)
+
+    # end to end: host x -> device, forward, device out -> host, every step (eager, public API)
+    x_host = torch.empty_like(r.x, device="cpu").pin_memory()
+    x_host.copy_(r.x)
+    out_host = torch.empty_like(r.out, device="cpu").pin_memory()
+    e_steps = max(1, min(args.steps, 50))
+    s = r.stream
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            r.x.copy_(x_host, non_blocking=True)
+            r._step()
+            out_host.copy_(r.out, non_blocking=True)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    with torch.cuda.stream(s):
+        for _ in range(e_steps):
+            r.x.copy_(x_host, non_blocking=True)
+            r._step()
+            out_host.copy_(r.out, non_blocking=True)
+    e1.record(s)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+    if dist:
+        tt = torch.tensor([e_ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e_ms = float(tt.item())
+    e2e_value = e_steps * T * world / (e_ms / 1e3)
+    status = ftm.ftm_device_status(True)
+
+    if rank == 0:
+        pk, src = peaks()
+        kname = {k: ftm.KERNEL_NAMES[k] for k in Runner.KERNELS}
+        kms = {kname[k]: float(np.mean(v)) for k, v in per_kernel.items()}
+        decode = alg["rows"] / max(1, alg["groups"]) < 64
+        g1 = kms.get("gemm1", float("nan"))
+        if decode:
+            ach = alg["gemm1_bytes"] / (g1 * 1e-3) / 1e9
+            peak = float(pk["hbm_gbs"])
+            roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                    "kernel": "gemm1 (grouped gate/up + SwiGLU)", "algorithmic_bytes": alg["gemm1_bytes"],
+                    "peak_source": f"{src} hbm_gbs"}
+        else:
+            ach = alg["gemm1_flops"] / (g1 * 1e-3) / 1e12
+            peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+            roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                    "kernel": "gemm1 (grouped gate/up + SwiGLU)", "algorithmic_flops": alg["gemm1_flops"],
+                    "peak_source": f"{src} bf16_tflops_sustained"}
+        roof["traffic"] = ncu_traffic(workload_name(cfg, T), "gemm1")
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            v, n, cores, secs = oracle_tokens_per_s(cfg, T, args.cpu_seconds)
+            cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                   "sample": f"{n} tokens of the same batch, one token per oracle call, {secs:.1f} s of CPU work"}
+        step_bytes = alg["gemm1_bytes"] + alg["gemm2_bytes"]
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": cfg.wdtype, "data": "synthetic (seeded generator, weights N(0,0.02^2))",
+            "config": {"workload": workload_name(cfg, T), "d": cfg.d, "E": cfg.E, "k": cfg.k, "I": cfg.I, "T": T,
+                       "wdtype": cfg.wdtype, "active_experts": alg["groups"],
+                       "l2": (f"inputs larger than L2: {step_bytes / 1e9:.2f} GB of expert weights touched per step"
+                              if step_bytes > 4 * L2_BYTES else "working set below 4x L2 (not flushed)"),
+                       "launch": "CUDA graph replay" if use_graph else "eager", "parallelism": f"replicas x{world}"},
+            "roofline": roof,
+            "step_hbm_gbs": step_bytes / (ms / args.steps * 1e-3) / 1e9,
+            "kernels_ms": kms,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": r.x.numel() * r.x.element_size(),
+                    "d2h_bytes_per_step": r.out.numel() * r.out.element_size(), "launch": "eager"},
+            "gpu_launches": (len(Runner.KERNELS) + (2 if T * cfg.k > 4096 else 0)) * args.steps,
+            "clocks": clk,
+            "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        r.graphs.clear()
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

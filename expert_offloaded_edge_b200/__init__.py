@@ -27,6 +27,8 @@ from .binding import (  # noqa: F401
     ftm_permute,
     ftm_permute_workspace_bytes,
     ftm_route,
+    ftm_set_profile_events,
+    KERNEL_NAMES,
     ftm_slot_host_scratch_ints,
     ftm_slot_lookup_update,
     ftm_slot_workspace_bytes,

@@ -10,6 +10,8 @@ SO = os.path.join(PKG, "libftm.so")
 
 FTM_OK, FTM_ERR_INVALID_ARG, FTM_ERR_UNSUPPORTED, FTM_ERR_CAPACITY, FTM_ERR_CUDA = range(5)
 FTM_F32, FTM_BF16, FTM_FP8_E4M3_B128, FTM_NVFP4 = range(4)
+(FTM_K_ROUTE, FTM_K_PERMUTE, FTM_K_LRU, FTM_K_GATHER, FTM_K_GEMM1, FTM_K_GEMM2, FTM_K_COMBINE) = range(7)
+KERNEL_NAMES = ("route", "permute", "lru", "gather", "gemm1", "gemm2", "combine")
 _WDTYPE = {"f32": FTM_F32, "bf16": FTM_BF16, "fp8": FTM_FP8_E4M3_B128, "nvfp4": FTM_NVFP4}
 
 c_i32, c_i64, c_u64, c_p, c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_size_t
@@ -74,6 +76,8 @@ def library() -> ctypes.CDLL:
         L.ftm_combine.argtypes = [P(LayerDesc), c_p, c_p, c_p, c_i32, c_p, c_p]
         L.ftm_moe_layer_forward.argtypes = [P(LayerDesc), P(LayerWeights), P(SlotCache), c_p, c_i32, c_p, c_p, c_sz,
                                             c_p, c_p]
+        L.ftm_set_profile_events.argtypes = [c_i32, c_p, c_p]
+        L.ftm_set_profile_events.restype = c_i32
         L.ftm_workspace_bytes.argtypes = [P(LayerDesc), c_i32]
         L.ftm_workspace_bytes.restype = c_sz
         for name in ("ftm_get_bank_layout", "ftm_route", "ftm_permute", "ftm_slot_lookup_update", "ftm_expert_ffn",
@@ -167,6 +171,13 @@ def ftm_expert_ffn(desc, x, T, offsets, perm, slot_of_expert, slot_pool, shared_
 def ftm_combine(desc, y, inv, topk_w, T, out, stream=None):
     _check(library().ftm_combine(ctypes.byref(desc), _ptr(y), _ptr(inv), _ptr(topk_w), T, _ptr(out),
                                  _stream(stream)))
+
+
+def ftm_set_profile_events(which: int, start_event=None, stop_event=None):
+    """start/stop: torch.cuda.Event(enable_timing=True) (or None to clear)."""
+    sp = None if start_event is None else start_event.cuda_event
+    ep = None if stop_event is None else stop_event.cuda_event
+    _check(library().ftm_set_profile_events(which, sp, ep))
 
 
 def ftm_workspace_bytes(desc, T_max) -> int:

@@ -28,6 +28,7 @@ using namespace ftm;
 namespace {
 
 thread_local char g_err[512] = "";
+thread_local cudaEvent_t g_prof[FTM_K_COUNT][2] = {};
 
 ftm_status fail(ftm_status s, const char* fmt, ...) {
   va_list ap;
@@ -165,9 +166,23 @@ cudaEvent_t copy_event() {
 
 }  // namespace
 
+void ftm::prof_mark(int which, cudaStream_t st, bool stop) {
+  if (which >= 0 && which < FTM_K_COUNT && g_prof[which][stop ? 1 : 0])
+    cudaEventRecord(g_prof[which][stop ? 1 : 0], st);
+}
+
 extern "C" {
 
 const char* ftm_last_error(void) { return g_err; }
+
+ftm_status ftm_set_profile_events(int32_t which, void* start_event, void* stop_event) {
+  if (which < 0 || which >= FTM_K_COUNT) return fail(FTM_ERR_INVALID_ARG, "kernel id %d out of range", which);
+  if ((start_event == nullptr) != (stop_event == nullptr))
+    return fail(FTM_ERR_INVALID_ARG, "start and stop events must both be set or both be NULL");
+  g_prof[which][0] = static_cast<cudaEvent_t>(start_event);
+  g_prof[which][1] = static_cast<cudaEvent_t>(stop_event);
+  return ok();
+}
 
 int32_t ftm_device_status(int32_t reset) {
   cudaDeviceSynchronize();
@@ -195,7 +210,9 @@ ftm_status ftm_route(const ftm_layer_desc* L, const void* x, int32_t T, const vo
   if (T == 0) return ok();
   if (!x || !w_router || !topk_ids || !topk_w) return fail(FTM_ERR_INVALID_ARG, "ftm_route: NULL pointer");
   if (!aligned(x, 16) || !aligned(w_router, 16)) return fail(FTM_ERR_INVALID_ARG, "ftm_route: x/w_router not 16-byte aligned");
+  prof_mark(FTM_K_ROUTE, S_(stream), false);
   cudaError_t e = launch_route(L->wdtype == FTM_F32, x, T, L->d, w_router, bias, L->E, L->k, topk_ids, topk_w, S_(stream));
+  prof_mark(FTM_K_ROUTE, S_(stream), true);
   if (e != cudaSuccess) return cuda_fail(e, "ftm_route launch");
   return ok();
 }
@@ -213,7 +230,9 @@ ftm_status ftm_permute(const ftm_layer_desc* L, const int32_t* topk_ids, int32_t
   const int64_t P = static_cast<int64_t>(T) * L->k;
   if (P > 0 && (!topk_ids || !perm || !inv)) return fail(FTM_ERR_INVALID_ARG, "ftm_permute: NULL pointer");
   if ((s = check_ws(workspace, ws_bytes, permute_workspace_bytes(L->E, P), "ftm_permute"))) return s;
+  prof_mark(FTM_K_PERMUTE, S_(stream), false);
   cudaError_t e = launch_permute(topk_ids, static_cast<int>(P), L->E, counts, offsets, perm, inv, workspace, S_(stream));
+  prof_mark(FTM_K_PERMUTE, S_(stream), true);
   if (e != cudaSuccess) return cuda_fail(e, "ftm_permute launch");
   return ok();
 }
@@ -246,8 +265,10 @@ ftm_status ftm_slot_lookup_update(const ftm_layer_desc* L, ftm_slot_cache* C, co
   }
   cudaStream_t cs = S_(compute_stream), ps = S_(copy_stream);
   int32_t* ws = static_cast<int32_t*>(workspace);
+  prof_mark(FTM_K_LRU, cs, false);
   cudaError_t e = launch_lru_step(topk_ids, static_cast<int>(P), L->E, L->S, C->step, C->slot_of_expert,
                                   C->expert_of_slot, C->last_use, ws, cs);
+  prof_mark(FTM_K_LRU, cs, true);
   if (e != cudaSuccess) return cuda_fail(e, "lru step launch");
   const size_t hdr = sizeof(int32_t) * (4 + 2 * static_cast<size_t>(L->E));
   if ((e = cudaMemcpyAsync(C->host_scratch, ws, hdr, cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
@@ -336,8 +357,10 @@ ftm_status ftm_combine(const ftm_layer_desc* L, const void* y, const int32_t* in
   if (T == 0) return ok();
   if (!y || !inv || !topk_w || !out) return fail(FTM_ERR_INVALID_ARG, "ftm_combine: NULL pointer");
   if (!aligned(y, 16) || !aligned(out, 16)) return fail(FTM_ERR_INVALID_ARG, "ftm_combine: y/out not 16-byte aligned");
+  prof_mark(FTM_K_COMBINE, S_(stream), false);
   cudaError_t e = launch_combine(L->wdtype == FTM_F32, y, inv, topk_w, T, L->k, L->d, T * L->k, L->has_shared, out,
                                  S_(stream));
+  prof_mark(FTM_K_COMBINE, S_(stream), true);
   if (e != cudaSuccess) return cuda_fail(e, "ftm_combine launch");
   return ok();
 }

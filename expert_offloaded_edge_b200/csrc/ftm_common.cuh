@@ -186,6 +186,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Measurement hook (see ftm_set_profile_events): records the caller's events
+// around the launches of kernel `which` on stream `st`.
+void prof_mark(int which, cudaStream_t st, bool stop);
+
 // Arguments of the expert-FFN launcher (shared by the C ABI and the kernels' host code).
 struct FfnArgs {
   int d, E, k, I, has_shared, S, f32;

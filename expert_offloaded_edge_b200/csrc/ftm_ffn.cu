@@ -389,18 +389,24 @@ const char* launch_expert_ffn(const FfnArgs& a, cudaStream_t st, cudaError_t* ce
   const int elt = a.f32 ? 4 : 2;
   {
     const int grid = rows < 148 * 8 ? rows : 148 * 8;
+    prof_mark(FTM_K_GATHER, st, false);
     gather_rows_kernel<<<grid, 256, 0, st>>>(a.x, a.perm, P, a.k, a.T, a.has_shared, a.d * elt, a.xp);
+    prof_mark(FTM_K_GATHER, st, true);
     if ((*cerr = cudaGetLastError()) != cudaSuccess) return "gather launch failed";
   }
   if (a.f32) {
     dim3 g1(rows, (a.I + 63) / 64), g2(rows, (a.d + 63) / 64);
+    prof_mark(FTM_K_GEMM1, st, false);
     simt_gemm1_kernel<<<g1, 256, 0, st>>>(reinterpret_cast<const float*>(a.xp), a.offsets, a.slot_of_expert, a.E, P,
                                           a.d, a.I, a.pool, a.shared_bank, a.bank_bytes, a.w_gu_off,
                                           reinterpret_cast<float*>(a.h));
+    prof_mark(FTM_K_GEMM1, st, true);
     if ((*cerr = cudaGetLastError()) != cudaSuccess) return "simt gemm1 launch failed";
+    prof_mark(FTM_K_GEMM2, st, false);
     simt_gemm2_kernel<<<g2, 256, 0, st>>>(reinterpret_cast<const float*>(a.h), a.offsets, a.slot_of_expert, a.E, P,
                                           a.d, a.I, a.pool, a.shared_bank, a.bank_bytes, a.w_d_off,
                                           reinterpret_cast<float*>(a.y));
+    prof_mark(FTM_K_GEMM2, st, true);
     if ((*cerr = cudaGetLastError()) != cudaSuccess) return "simt gemm2 launch failed";
     return nullptr;
   }
@@ -420,12 +426,14 @@ const char* launch_expert_ffn(const FfnArgs& a, cudaStream_t st, cudaError_t* ce
     mAsh2 = mA2;
   }
   if (!ok) return "cuTensorMapEncodeTiled failed";
-  if ((*cerr = launch_tc_bn<true>(bn, mA1, mAsh1, mB1, a, a.d, a.I, a.I, reinterpret_cast<uint16_t*>(a.h), a.I,
-                                  st)) != cudaSuccess)
-    return "tensor-core gemm1 launch failed";
-  if ((*cerr = launch_tc_bn<false>(bn, mA2, mAsh2, mB2, a, a.I, a.d, 0, reinterpret_cast<uint16_t*>(a.y), a.d,
-                                   st)) != cudaSuccess)
-    return "tensor-core gemm2 launch failed";
+  prof_mark(FTM_K_GEMM1, st, false);
+  *cerr = launch_tc_bn<true>(bn, mA1, mAsh1, mB1, a, a.d, a.I, a.I, reinterpret_cast<uint16_t*>(a.h), a.I, st);
+  prof_mark(FTM_K_GEMM1, st, true);
+  if (*cerr != cudaSuccess) return "tensor-core gemm1 launch failed";
+  prof_mark(FTM_K_GEMM2, st, false);
+  *cerr = launch_tc_bn<false>(bn, mA2, mAsh2, mB2, a, a.I, a.d, 0, reinterpret_cast<uint16_t*>(a.y), a.d, st);
+  prof_mark(FTM_K_GEMM2, st, true);
+  if (*cerr != cudaSuccess) return "tensor-core gemm2 launch failed";
   return nullptr;
 }
 

@@ -202,6 +202,24 @@ ftm_status ftm_moe_layer_forward(const ftm_layer_desc* L, const ftm_layer_weight
                                  void* stream, void* copy_stream);
 size_t ftm_workspace_bytes(const ftm_layer_desc* L, int32_t T_max);
 
+/* Measurement hook.  Kernel ids of the path, in launch order. */
+typedef enum ftm_kernel_id {
+  FTM_K_ROUTE = 0,      /* router + gating */
+  FTM_K_PERMUTE = 1,    /* histogram / scan / scatter (all launches of one call) */
+  FTM_K_LRU = 2,        /* slot lookup/update */
+  FTM_K_GATHER = 3,     /* X_p gather (+ activation quantisation) */
+  FTM_K_GEMM1 = 4,      /* grouped gate/up GEMM + SwiGLU */
+  FTM_K_GEMM2 = 5,      /* grouped down GEMM */
+  FTM_K_COMBINE = 6,    /* weighted un-permute + shared expert */
+  FTM_K_COUNT = 7
+} ftm_kernel_id;
+
+/* While set on the calling thread, every launch of kernel `which` is bracketed
+ * by cudaEventRecord(start) / cudaEventRecord(stop) on the stream it is
+ * launched on (events are cudaEvent_t passed as void*, created by the caller
+ * with timing enabled).  NULL events clear the hook.  Nothing else changes. */
+ftm_status ftm_set_profile_events(int32_t which, void* start_event, void* stop_event);
+
 /* Thread-local description of the last error returned on this thread. */
 const char* ftm_last_error(void);
 

@@ -82,3 +82,13 @@ class DeviceLayer:
 
     def out_dtype(self):
         return torch.float32 if self.cfg.act_dtype == "f32" else torch.bfloat16
+
+
+class Workspace:
+    """A 256-byte aligned device scratch buffer of at least nbytes."""
+
+    def __init__(self, nbytes: int, device="cuda"):
+        self.nbytes = max(int(nbytes), 256)
+        self.buf = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device)
+        off = (-self.buf.data_ptr()) % 256
+        self.ptr = self.buf.data_ptr() + off

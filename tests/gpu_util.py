@@ -10,7 +10,7 @@ import torch
 import expert_offloaded_edge_b200 as ftm
 import oracle
 import synth
-from synth.device import DeviceLayer
+from synth.device import DeviceLayer, Workspace
 
 TOL = {"f32": 2e-2, "bf16": 2e-2, "fp8": 5e-2, "nvfp4": 5e-2}
 TOL_F32_SIMT = 1e-4
@@ -39,14 +39,6 @@ def oracle_route(dl: DeviceLayer, T: int, step: int = 0):
 
 def to_np_f32(t: torch.Tensor) -> np.ndarray:
     return t.float().cpu().numpy()
-
-
-class Workspace:
-    def __init__(self, nbytes: int, device="cuda"):
-        self.nbytes = max(int(nbytes), 256)
-        self.buf = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device)
-        off = (-self.buf.data_ptr()) % 256
-        self.ptr = self.buf.data_ptr() + off
 
 
 def run_layer(dl: DeviceLayer, x_dev: torch.Tensor, T: int, cache: bool = False) -> torch.Tensor:
