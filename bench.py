@@ -149,8 +149,15 @@ class Runner:
                                   self.ws.nbytes, self.stream)
 
     def _events(self, n):
-        return [{k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                 for k in self.KERNELS} for _ in range(n)]
+        evs = [{k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for k in self.KERNELS} for _ in range(n)]
+        # torch creates the CUDA event on its first record(); the library re-records it later
+        for ev in evs:
+            for a, b in ev.values():
+                a.record(self.stream)
+                b.record(self.stream)
+        self.stream.synchronize()
+        return evs
 
     def _record_steps(self, evs):
         for ev in evs:

@@ -166,8 +166,16 @@ cudaEvent_t copy_event() {
 
 }  // namespace
 
+ftm_status ftm::report_error(ftm_status s, const char* msg) { return fail(s, "%s", msg); }
+
 void ftm::prof_mark(int which, cudaStream_t st, bool stop) {
-  if (which >= 0 && which < FTM_K_COUNT && g_prof[which][stop ? 1 : 0])
+  if (which < 0 || which >= FTM_K_COUNT || !g_prof[which][stop ? 1 : 0]) return;
+  // under stream capture the record must become a graph node of its own
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(st, &cs);
+  if (cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(g_prof[which][stop ? 1 : 0], st, cudaEventRecordExternal);
+  else
     cudaEventRecord(g_prof[which][stop ? 1 : 0], st);
 }
 

@@ -190,6 +190,9 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 // around the launches of kernel `which` on stream `st`.
 void prof_mark(int which, cudaStream_t st, bool stop);
 
+// Sets the thread-local error string read by ftm_last_error() and returns s.
+ftm_status report_error(ftm_status s, const char* msg);
+
 // Arguments of the expert-FFN launcher (shared by the C ABI and the kernels' host code).
 struct FfnArgs {
   int d, E, k, I, has_shared, S, f32;

@@ -18,7 +18,7 @@ namespace cg = cooperative_groups;
 namespace ftm {
 
 constexpr int kRouteCluster = 8;
-constexpr int kRouteWarps = 8;
+constexpr int kRouteWarps = 16;
 constexpr int kMaxE = 512;
 constexpr int kMaxK = 16;
 
@@ -85,6 +85,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_topk_kernel(const Tin*
 #pragma unroll
     for (int t = 0; t < TT; ++t) acc[t] = 0.f;
     const Tin* wrow = wr + static_cast<size_t>(e) * d;
+#pragma unroll 4
     for (int c = lane * V; c < d; c += 32 * V) {
       float w[V];
       IO::load(wrow + c, w);
