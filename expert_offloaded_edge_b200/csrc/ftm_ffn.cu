@@ -15,8 +15,9 @@
 // a (group, weight tile, token tile) list; warp 0 issues TMA loads (weights via
 // a 3-D tensor map whose third coordinate is the slot), warp 1 issues tcgen05
 // MMAs into a double-buffered TMEM accumulator, warps 2-5 drain TMEM, apply
-// SwiGLU and store.  fp32 layers run a plain SIMT kernel.
-#include "ftm_common.cuh"
+// SwiGLU and store.  fp32 layers run a plain SIMT kernel; FP8 layers run the
+// block-scaled kernel in ftm_ffn_fp8.cu.
+#include "ftm_gemm.cuh"
 
 namespace ftm {
 
@@ -51,8 +52,6 @@ __device__ __forceinline__ int group_of_row(const int32_t* offsets, int E, int P
 // ---------------------------------------------------------------------------
 // SIMT path (fp32 layers): one warp per output element, lanes split the dot.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float silu(float z) { return z / (1.f + expf(-z)); }
-
 __global__ void __launch_bounds__(256) simt_gemm1_kernel(const float* __restrict__ xp, const int32_t* __restrict__ offsets,
                                                          const int32_t* __restrict__ slot_of_expert, int E, int P,
                                                          int d, int I, const uint8_t* __restrict__ pool,
@@ -98,33 +97,7 @@ __global__ void __launch_bounds__(256) simt_gemm2_kernel(const float* __restrict
 // ---------------------------------------------------------------------------
 // Tensor-core path (bf16): persistent warp-specialised tcgen05 grouped GEMM.
 // ---------------------------------------------------------------------------
-constexpr int kTcThreads = 192;       // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue
-constexpr int kMaxGroups = 520;
 constexpr int kBK = 64;               // K per stage: 64 bf16 = one 128-byte swizzle row
-constexpr uint32_t kATileBytes = 128 * 128;
-
-struct TileInfo {
-  int g, m, n, rows, row0;
-};
-
-__device__ __forceinline__ TileInfo decode_tile(int t, const int32_t* tile_start, const int32_t* grp_rows,
-                                                const int32_t* grp_row0, int G, int MT, int BN) {
-  int lo = 0, hi = G;  // tile_start[lo] <= t < tile_start[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (tile_start[mid] <= t) lo = mid; else hi = mid;
-  }
-  TileInfo ti;
-  ti.g = lo;
-  ti.rows = grp_rows[lo];
-  ti.row0 = grp_row0[lo];
-  const int ntok = (ti.rows + BN - 1) / BN;
-  const int local = t - tile_start[lo];
-  ti.m = local / ntok;
-  ti.n = local % ntok;
-  (void)MT;
-  return ti;
-}
 
 template <int BN, bool GATED>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -151,27 +124,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int MT = Nw / 128;
   const int KB = K / kBK;
 
-  // per-group rows and the tile prefix
-  for (int g = threadIdx.x; g < G; g += blockDim.x) {
-    const int rows = g < E ? offsets[g + 1] - offsets[g] : T;
-    grp_rows[g] = rows;
-    grp_row0[g] = g < E ? offsets[g] : P;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const int per = (G + 31) / 32, b = lane * per, en = min(G, b + per);
-    int s = 0;
-    for (int g = b; g < en; ++g) s += ((grp_rows[g] + BN - 1) / BN) * MT;
-    int incl = s;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    int run = incl - s;
-    for (int g = b; g < en; ++g) { tile_start[g] = run; run += ((grp_rows[g] + BN - 1) / BN) * MT; }
-    if (lane == 31) tile_start[G] = incl;
-  }
+  build_tile_table(offsets, E, has_shared, T, P, MT, BN, tile_start, grp_rows, grp_row0);
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 4); }
@@ -205,7 +158,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, MT, BN);
+        const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, BN);
         const int slot = ti.g < E ? slot_of_expert[ti.g] : 0;
         const int brow = ti.row0 + ti.n * BN;
         for (int kb = 0; kb < KB; ++kb) {
@@ -260,7 +213,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int q = warp % 4;  // TMEM lane quadrant this warp may access
     int it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-      const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, MT, BN);
+      const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, BN);
       const int ab = it & 1;
       const uint32_t aphase = (it >> 1) & 1;
       if (!mbar_wait(&tfull_bar[ab], aphase)) break;
@@ -297,49 +250,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
 // bf16 K-major map: dims {K, rows[, slots]}, box {64, box_rows[, 1]}, 128-byte swizzle.
 static bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint64_t row_pitch,
                           uint64_t slots, uint64_t slot_pitch, uint32_t box_rows) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {K, rows, slots};
-  cuuint64_t strides[2] = {row_pitch, slot_pitch};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(kBK), box_rows, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  const cuuint32_t rank = slots > 0 ? 3 : 2;
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, es,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return make_map_sw128(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, K, rows, row_pitch, slots, slot_pitch,
+                        box_rows);
 }
-
-static int num_sms() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
-
 
 template <int BN, bool GATED>
 static cudaError_t launch_tc(const CUtensorMap& mA, const CUtensorMap& mAsh, const CUtensorMap& mB,
