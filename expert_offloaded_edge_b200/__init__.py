@@ -24,6 +24,7 @@ from .binding import (  # noqa: F401
     ftm_get_bank_layout,
     ftm_last_error,
     ftm_moe_layer_forward,
+    ftm_moe_layer_forward_noalloc,
     ftm_permute,
     ftm_permute_workspace_bytes,
     ftm_route,

@@ -76,6 +76,8 @@ def library() -> ctypes.CDLL:
         L.ftm_combine.argtypes = [P(LayerDesc), c_p, c_p, c_p, c_i32, c_p, c_p]
         L.ftm_moe_layer_forward.argtypes = [P(LayerDesc), P(LayerWeights), P(SlotCache), c_p, c_i32, c_p, c_p, c_sz,
                                             c_p, c_p]
+        L.ftm_moe_layer_forward_noalloc.argtypes = [P(LayerDesc), P(LayerWeights), c_p, c_i32, c_p, c_p]
+        L.ftm_moe_layer_forward_noalloc.restype = c_i32
         L.ftm_set_profile_events.argtypes = [c_i32, c_p, c_p]
         L.ftm_set_profile_events.restype = c_i32
         L.ftm_workspace_bytes.argtypes = [P(LayerDesc), c_i32]
@@ -190,3 +192,10 @@ def ftm_moe_layer_forward(desc, weights: LayerWeights, cache: Optional[SlotCache
                                            ctypes.byref(cache) if cache is not None else None, _ptr(x), T, _ptr(out),
                                            _ptr(workspace), ws_bytes, _stream(stream),
                                            _stream(copy_stream) if cache is not None else None))
+
+
+def ftm_moe_layer_forward_noalloc(desc, weights: LayerWeights, x, T, out, stream=None):
+    """Resident layer forward whose scratch is the library's static device array
+    (for callers that cannot allocate device memory; see include/ftm.h)."""
+    _check(library().ftm_moe_layer_forward_noalloc(ctypes.byref(desc), ctypes.byref(weights), _ptr(x), T, _ptr(out),
+                                                   _stream(stream)))

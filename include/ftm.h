@@ -202,6 +202,23 @@ ftm_status ftm_moe_layer_forward(const ftm_layer_desc* L, const ftm_layer_weight
                                  void* stream, void* copy_stream);
 size_t ftm_workspace_bytes(const ftm_layer_desc* L, int32_t T_max);
 
+/* The whole resident layer, for callers that cannot allocate device memory
+ * (code running while a CUDA graph is being captured, allocator-free embedded
+ * runtimes, engines whose memory is reserved up front).  The pages have no
+ * counterpart of this entry point.
+ *   Same computation and arguments as ftm_moe_layer_forward with C = NULL, but
+ *   no workspace argument: the scratch is a static 16 MiB device array inside
+ *   the library, which every GPU that loads the library keeps until exit.
+ *   Calls whose ftm_workspace_bytes(L, T) exceeds 16 MiB are rejected with
+ *   FTM_ERR_INVALID_ARG (decode-sized batches fit; large prefills do not).
+ *   The first call on a device looks up the array's device address (with that
+ *   device current); make that first call before any stream capture.
+ *   All calls share the one array: calls that overlap on the GPU (on different
+ *   streams, or from different host threads, without ordering) race on it.
+ *   Nothing is allocated: no cudaMalloc/cudaFree and no allocating library call. */
+ftm_status ftm_moe_layer_forward_noalloc(const ftm_layer_desc* L, const ftm_layer_weights* W, const void* x,
+                                         int32_t T, void* out, void* stream);
+
 /* Measurement hook.  Kernel ids of the path, in launch order. */
 typedef enum ftm_kernel_id {
   FTM_K_ROUTE = 0,      /* router + gating */
