@@ -21,6 +21,9 @@ cudaError_t launch_lru_restore(int E, int S, int32_t* soe, int32_t* eos, int64_t
 cudaError_t launch_combine(bool f32, const void* y, const int32_t* inv, const float* gw, int T, int k, int d, int P,
                            int has_shared, void* out, cudaStream_t st);
 const char* launch_expert_ffn(const FfnArgs& a, cudaStream_t st, cudaError_t* cerr);
+size_t fp8_ffn_workspace_bytes(int64_t rows, int d, int I);
+const char* launch_expert_ffn_fp8(const FfnArgs& a, size_t s_gu_off, size_t s_d_off, uint8_t* ws, cudaStream_t st,
+                                  cudaError_t* cerr);
 }  // namespace ftm
 
 using namespace ftm;
@@ -106,6 +109,7 @@ size_t act_elt(const ftm_layer_desc* L) { return L->wdtype == FTM_F32 ? 4 : 2; }
 
 size_t ffn_ws_bytes(const ftm_layer_desc* L, int32_t T) {
   const size_t rows = static_cast<size_t>(ffn_rows(L, T));
+  if (L->wdtype == FTM_FP8_E4M3_B128) return fp8_ffn_workspace_bytes(static_cast<int64_t>(rows), L->d, L->I);
   return al(rows * L->d * act_elt(L)) + al(rows * L->I * act_elt(L));
 }
 
@@ -328,8 +332,7 @@ ftm_status ftm_expert_ffn(const ftm_layer_desc* L, const void* x, int32_t T, con
                           const void* shared_bank, void* y, void* workspace, size_t ws_bytes, void* stream) {
   ftm_status s = check_desc(L);
   if (s || (s = check_T(T))) return s;
-  if (L->wdtype == FTM_FP8_E4M3_B128 || L->wdtype == FTM_NVFP4)
-    return fail(FTM_ERR_UNSUPPORTED, "expert FFN for wdtype %d not built", L->wdtype);
+  if (L->wdtype == FTM_NVFP4) return fail(FTM_ERR_UNSUPPORTED, "expert FFN for wdtype %d not built", L->wdtype);
   if (T == 0) return ok();
   if (!x || !offsets || !perm || !slot_of_expert || !slot_pool || !y)
     return fail(FTM_ERR_INVALID_ARG, "ftm_expert_ffn: NULL pointer");
@@ -353,7 +356,10 @@ ftm_status ftm_expert_ffn(const ftm_layer_desc* L, const void* x, int32_t T, con
   a.xp = static_cast<uint8_t*>(workspace);
   a.h = a.xp + al(rows * L->d * act_elt(L));
   cudaError_t ce;
-  const char* msg = launch_expert_ffn(a, S_(stream), &ce);
+  const char* msg = L->wdtype == FTM_FP8_E4M3_B128
+                        ? launch_expert_ffn_fp8(a, bl.s_gu_off, bl.s_d_off, static_cast<uint8_t*>(workspace),
+                                                S_(stream), &ce)
+                        : launch_expert_ffn(a, S_(stream), &ce);
   if (msg) return ce != cudaSuccess ? cuda_fail(ce, msg) : fail(FTM_ERR_CUDA, "%s", msg);
   return ok();
 }

@@ -71,6 +71,22 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const int32_t* tile_start
 // Named barrier over the four epilogue warps (warps 2-5).
 __device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// Named-barrier AND over the four epilogue warps: every epilogue warp gets the
+// same answer, so they leave their loop together (no warp is left waiting at a
+// later named barrier for one that gave up).
+__device__ __forceinline__ bool epilogue_all(bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, 1, 128, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(p))
+      : "memory");
+  return r != 0;
+}
+
 // ---- host -------------------------------------------------------------------
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
