@@ -74,9 +74,13 @@ double orc_e2m1_value(uint8_t nib) {
 }
 
 static double orc_e4m3_table[127];       /* values of codes 0x00 .. 0x7E */
+static double orc_e4m3_all[256];         /* value of every code (decode lookup) */
+static double orc_e2m1_all[16];
 
 __attribute__((constructor)) static void orc_init_tables(void) {
   for (int c = 0; c < 127; ++c) orc_e4m3_table[c] = orc_e4m3_value((uint8_t)c);
+  for (int c = 0; c < 256; ++c) orc_e4m3_all[c] = orc_e4m3_value((uint8_t)c);
+  for (int c = 0; c < 16; ++c) orc_e2m1_all[c] = orc_e2m1_value((uint8_t)c);
 }
 
 /* Round to the nearest finite E4M3 value, ties to the code with an even
@@ -118,21 +122,23 @@ void orc_dequant_bf16(const uint16_t* w, int64_t n, float* out) {
 /* FP8 with one fp32 scale per 128x128 block: w[r][c] = e4m3(q[r][c]) * s[r/128][c/128]. */
 void orc_dequant_fp8_b128(const uint8_t* q, const float* s, int R, int C, float* out) {
   int CB = C / 128;
+#pragma omp parallel for schedule(static)
   for (int r = 0; r < R; ++r)
     for (int c = 0; c < C; ++c)
       out[(int64_t)r * C + c] =
-          (float)(orc_e4m3_value(q[(int64_t)r * C + c]) * (double)s[(r / 128) * CB + c / 128]);
+          (float)(orc_e4m3_all[q[(int64_t)r * C + c]] * (double)s[(r / 128) * CB + c / 128]);
 }
 
 /* NVFP4: w[r][c] = e2m1(q) * e4m3(s16[r][c/16]) * s_t, two codes per byte
  * along c, element 2j in the low nibble. */
 void orc_dequant_nvfp4(const uint8_t* qp, const uint8_t* s16, float s_t, int R, int C, float* out) {
+#pragma omp parallel for schedule(static)
   for (int r = 0; r < R; ++r)
     for (int c = 0; c < C; ++c) {
       uint8_t byte = qp[(int64_t)r * (C / 2) + c / 2];
       uint8_t nib = (c & 1) ? (byte >> 4) : (byte & 15);
-      double sc = orc_e4m3_value(s16[(int64_t)r * (C / 16) + c / 16]);
-      out[(int64_t)r * C + c] = (float)(orc_e2m1_value(nib) * sc * (double)s_t);
+      double sc = orc_e4m3_all[s16[(int64_t)r * (C / 16) + c / 16]];
+      out[(int64_t)r * C + c] = (float)(orc_e2m1_all[nib] * sc * (double)s_t);
     }
 }
 
