@@ -22,6 +22,9 @@ cudaError_t launch_combine(bool f32, const void* y, const int32_t* inv, const fl
                            int has_shared, void* out, cudaStream_t st);
 const char* launch_expert_ffn(const FfnArgs& a, cudaStream_t st, cudaError_t* cerr);
 size_t fp8_ffn_workspace_bytes(int64_t rows, int d, int I);
+size_t nvfp4_ffn_workspace_bytes(int64_t P, int T, int E, int has_shared, int d, int I);
+const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_d_off, size_t s_t_off, uint8_t* ws,
+                                    cudaStream_t st, cudaError_t* cerr);
 const char* launch_expert_ffn_fp8(const FfnArgs& a, size_t s_gu_off, size_t s_d_off, uint8_t* ws, cudaStream_t st,
                                   cudaError_t* cerr);
 }  // namespace ftm
@@ -110,6 +113,8 @@ size_t act_elt(const ftm_layer_desc* L) { return L->wdtype == FTM_F32 ? 4 : 2; }
 size_t ffn_ws_bytes(const ftm_layer_desc* L, int32_t T) {
   const size_t rows = static_cast<size_t>(ffn_rows(L, T));
   if (L->wdtype == FTM_FP8_E4M3_B128) return fp8_ffn_workspace_bytes(static_cast<int64_t>(rows), L->d, L->I);
+  if (L->wdtype == FTM_NVFP4)
+    return nvfp4_ffn_workspace_bytes(static_cast<int64_t>(T) * L->k, T, L->E, L->has_shared, L->d, L->I);
   return al(rows * L->d * act_elt(L)) + al(rows * L->I * act_elt(L));
 }
 
@@ -332,7 +337,6 @@ ftm_status ftm_expert_ffn(const ftm_layer_desc* L, const void* x, int32_t T, con
                           const void* shared_bank, void* y, void* workspace, size_t ws_bytes, void* stream) {
   ftm_status s = check_desc(L);
   if (s || (s = check_T(T))) return s;
-  if (L->wdtype == FTM_NVFP4) return fail(FTM_ERR_UNSUPPORTED, "expert FFN for wdtype %d not built", L->wdtype);
   if (T == 0) return ok();
   if (!x || !offsets || !perm || !slot_of_expert || !slot_pool || !y)
     return fail(FTM_ERR_INVALID_ARG, "ftm_expert_ffn: NULL pointer");
@@ -356,10 +360,14 @@ ftm_status ftm_expert_ffn(const ftm_layer_desc* L, const void* x, int32_t T, con
   a.xp = static_cast<uint8_t*>(workspace);
   a.h = a.xp + al(rows * L->d * act_elt(L));
   cudaError_t ce;
-  const char* msg = L->wdtype == FTM_FP8_E4M3_B128
-                        ? launch_expert_ffn_fp8(a, bl.s_gu_off, bl.s_d_off, static_cast<uint8_t*>(workspace),
-                                                S_(stream), &ce)
-                        : launch_expert_ffn(a, S_(stream), &ce);
+  const char* msg;
+  if (L->wdtype == FTM_FP8_E4M3_B128)
+    msg = launch_expert_ffn_fp8(a, bl.s_gu_off, bl.s_d_off, static_cast<uint8_t*>(workspace), S_(stream), &ce);
+  else if (L->wdtype == FTM_NVFP4)
+    msg = launch_expert_ffn_nvfp4(a, bl.s_gu_off, bl.s_d_off, bl.s_t_off, static_cast<uint8_t*>(workspace),
+                                  S_(stream), &ce);
+  else
+    msg = launch_expert_ffn(a, S_(stream), &ce);
   if (msg) return ce != cudaSuccess ? cuda_fail(ce, msg) : fail(FTM_ERR_CUDA, "%s", msg);
   return ok();
 }

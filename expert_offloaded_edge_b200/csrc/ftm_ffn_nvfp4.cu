@@ -1,0 +1,495 @@
+// NVFP4 grouped SwiGLU FFN: e2m1 weights with one e4m3 scale per 16 elements
+// and one fp32 scale per tensor; activations quantised to e2m1 with one e4m3
+// scale per 16 elements (per-tensor activation scale 1).
+//
+// The contraction is tcgen05.mma kind::mxf4nvf4 with hardware block scaling:
+// each MMA (K = 64) takes the four scales of every A row and every B row from
+// TMEM.  The scales travel global -> shared memory by bulk copy (512-byte
+// chunks in the layout the MMA expects) and shared -> TMEM by tcgen05.cp
+// (32x128b, replicated to the four lane quadrants), issued by the MMA thread
+// right before the MMAs that use them.
+//
+// Scale-chunk layout (weights and activations alike): one 512-byte chunk per
+// (block of rows, 64 elements of K); the scale of local row r (< 128) for the
+// j-th 16-element group of the chunk is byte (r % 32) * 16 + (r / 32) * 4 + j.
+// Weight chunks cover 128-row blocks; activation chunks cover BN-row blocks,
+// and every expert group of activation rows is padded to a multiple of BN rows
+// so each token tile is exactly one block.
+#include "ftm_gemm.cuh"
+
+namespace ftm {
+
+constexpr int kF4StageK = 256;         // K per stage: 128 bytes of packed e2m1 = one swizzle row
+constexpr uint32_t kSfChunk = 512;     // bytes of one scale chunk (64 K x 128 rows)
+constexpr uint32_t kSfStage = 4 * kSfChunk;
+
+// ---- conversions ---------------------------------------------------------------
+__device__ __forceinline__ uint8_t f32_to_e4m3_sat(float v) {
+  uint16_t r;
+  asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\tmov.b16 %0, t;\n\t}" : "=h"(r) : "f"(0.f), "f"(v));
+  return static_cast<uint8_t>(r & 0xFF);
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint8_t q) {
+  uint32_t h2;
+  const uint16_t in = q;
+  asm("{\n\t.reg .b16 t;\n\tmov.b16 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h2) : "h"(in));
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFF)));
+}
+
+// byte = e2m1(hi) << 4 | e2m1(lo), round to nearest even, saturating at 6.
+__device__ __forceinline__ uint8_t f32x2_to_e2m1x2(float hi, float lo) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u16.u8 %0, t;\n\t}"
+      : "=h"(r)
+      : "f"(hi), "f"(lo));
+  return static_cast<uint8_t>(r & 0xFF);
+}
+
+__host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
+  // a/b format E2M1 (1) at bits 7 and 10; scale format UE4M3 (0) at bit 23; K = 64
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// shared -> TMEM copy of one 512-byte scale chunk: 32 rows x 16 bytes,
+// replicated into the four 32-lane quadrants (4 columns each).
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Descriptor of a 512-byte chunk: no swizzle, 8-row core matrices of 16-byte
+// rows stored contiguously (stride between 8-row groups 128 bytes).
+__device__ __forceinline__ uint64_t smem_desc_sf(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(16u >> 4) << 16;      // leading byte offset (one 16-byte column only)
+  d |= static_cast<uint64_t>(128u >> 4) << 32;     // stride byte offset: 8 rows x 16 bytes
+  d |= static_cast<uint64_t>(1u) << 46;            // version
+  return d;                                         // layout type 0: no swizzle
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ uint32_t sf_byte(int r, int j) { return (r % 32) * 16 + (r / 32) * 4 + j; }
+
+// ---------------------------------------------------------------------------
+// Padded row offsets: prow0[g] = sum_{g' < g} roundup(rows_g', BN), g = 0..G.
+// ---------------------------------------------------------------------------
+__global__ void pad_offsets_kernel(const int32_t* __restrict__ offsets, int E, int has_shared, int T, int BN,
+                                   int32_t* __restrict__ prow0) {
+  __shared__ int32_t rows[kMaxGroups];
+  const int G = E + (has_shared ? 1 : 0);
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    const int r = g < E ? offsets[g + 1] - offsets[g] : T;
+    rows[g] = (r + BN - 1) / BN * BN;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int per = (G + 31) / 32, b = lane * per, en = min(G, b + per);
+    int s = 0;
+    for (int g = b; g < en; ++g) s += rows[g];
+    int incl = s;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - s;
+    for (int g = b; g < en; ++g) { prow0[g] = run; run += rows[g]; }
+    if (lane == 31) prow0[G] = incl;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Gather + NVFP4 quantisation of x into the padded activation rows.
+// One warp per (padded row, 64-element K block); lane l holds elements 2l, 2l+1.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) gather_quant_nvfp4_kernel(const uint16_t* __restrict__ x,
+                                                                const int32_t* __restrict__ perm,
+                                                                const int32_t* __restrict__ offsets,
+                                                                const int32_t* __restrict__ prow0, int E,
+                                                                int has_shared, int T, int k, int d, int BN,
+                                                                int rows_pad_max, uint8_t* __restrict__ xq,
+                                                                uint8_t* __restrict__ sfx) {
+  const int G = E + (has_shared ? 1 : 0);
+  const int rows_pad = prow0[G];
+  const int kb64 = d / 64;
+  const int lane = threadIdx.x % 32;
+  const long total = static_cast<long>(rows_pad) * kb64;
+  (void)rows_pad_max;
+  for (long w = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32; w < total;
+       w += static_cast<long>(gridDim.x) * blockDim.x / 32) {
+    const int pr = static_cast<int>(w / kb64), kb = static_cast<int>(w % kb64);
+    int lo = 0, hi = G;  // prow0[lo] <= pr < prow0[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (prow0[mid] <= pr) lo = mid; else hi = mid;
+    }
+    const int g = lo;
+    const int local = pr - prow0[g];
+    const int rows = g < E ? offsets[g + 1] - offsets[g] : T;
+    float v0 = 0.f, v1 = 0.f;
+    if (local < rows) {
+      const int src = g < E ? perm[offsets[g] + local] / k : local;
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(x + static_cast<size_t>(src) * d + kb * 64 + 2 * lane);
+      v0 = bf16_bits_to_f32(u & 0xFFFF);
+      v1 = bf16_bits_to_f32(u >> 16);
+    }
+    float amax = fmaxf(fabsf(v0), fabsf(v1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    const uint8_t sq = f32_to_e4m3_sat(amax / 6.0f);
+    const float s = e4m3_to_f32(sq);
+    const uint8_t byte = s == 0.f ? 0 : f32x2_to_e2m1x2(v1 / s, v0 / s);
+    xq[static_cast<size_t>(pr) * (d / 2) + kb * 32 + lane] = byte;
+    if ((lane & 7) == 0) {
+      const int blk = pr / BN, r = pr % BN;
+      sfx[(static_cast<size_t>(blk) * kb64 + kb) * kSfChunk + sf_byte(r, lane / 8)] = sq;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The grouped GEMM.
+//   A: packed e2m1 weights via a 3-D map {K bytes, rows, slot} (shared: 2-D)
+//   weight scale chunks at bank + wsf_off; per-tensor scales at bank + st_off
+//   B: packed e2m1 activations {K bytes, rows_pad}, scale chunks act_sf
+//   GATED: out_q (e2m1 H [rows_pad][Nw/2]) + out_sf (chunks); else out_bf16 [rows][Nw]
+// ---------------------------------------------------------------------------
+template <int BN, bool GATED>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    ffn_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAsh,
+                     const __grid_constant__ CUtensorMap tmB, const int32_t* __restrict__ offsets,
+                     const int32_t* __restrict__ prow0, const int32_t* __restrict__ slot_of_expert, int E,
+                     int has_shared, int T, int P, int K, int Nw, int up_row0, const uint8_t* __restrict__ pool,
+                     const uint8_t* __restrict__ shared_bank, size_t bank_bytes, size_t wsf_off, size_t st_off,
+                     int st_idx, const uint8_t* __restrict__ act_sf, uint8_t* __restrict__ out_q,
+                     uint8_t* __restrict__ out_sf, uint16_t* __restrict__ out_bf16, int stages) {
+  constexpr uint32_t kBBytes = ((BN * 128 + 1023) / 1024) * 1024;
+  constexpr uint32_t kNA = GATED ? 2 : 1;
+  constexpr uint32_t kStageBytes = kATileBytes * kNA + kBBytes + kSfStage * (kNA + 1);
+  constexpr uint32_t kTx = kATileBytes * kNA + BN * 128 + kSfStage * (kNA + 1);
+  constexpr uint32_t kAccCols = GATED ? 2 * BN : BN;
+  constexpr uint32_t kSfCols = 16 * (kNA + 1);                 // 4 chunks x 4 columns per operand
+  constexpr uint32_t kUsedCols = 2 * kAccCols + kSfCols;
+  constexpr uint32_t kTmemCols = kUsedCols <= 32 ? 32 : kUsedCols <= 64 ? 64 : kUsedCols <= 128 ? 128
+                                 : kUsedCols <= 256 ? 256 : 512;
+  static_assert(kUsedCols <= 512, "TMEM budget");
+  constexpr uint32_t kIdesc = idesc_nvf4(128, BN);
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[8], empty_bar[8], tfull_bar[2], tempty_bar[2];
+  __shared__ uint32_t tmem_holder;
+  __shared__ int32_t tile_start[kMaxGroups + 1], grp_rows[kMaxGroups], grp_row0[kMaxGroups];
+
+  const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (smem_base - smem_u32(smem_raw));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int G = E + (has_shared ? 1 : 0);
+  const int MT = Nw / 128;
+  const int KB = K / kF4StageK;
+  const int K64 = K / 64;
+
+  build_tile_table(offsets, E, has_shared, T, P, MT, BN, tile_start, grp_rows, grp_row0);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 4); }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_holder, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmAsh);
+    tma_prefetch_desc(&tmB);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_holder;
+  const uint32_t tmem_sf = tmem_base + 2 * kAccCols;   // SFA gate | SFA up | SFB, 16 columns each
+  const int total = tile_start[G];
+
+  auto a_tile = [&](int s, int which) -> uint8_t* {
+    return smem + static_cast<size_t>(s) * kStageBytes + which * kATileBytes;
+  };
+  auto b_tile = [&](int s) -> uint8_t* { return smem + static_cast<size_t>(s) * kStageBytes + kATileBytes * kNA; };
+  auto sf_tile = [&](int s, int which) -> uint8_t* {   // which: 0 gate, 1 up, kNA = activations
+    return smem + static_cast<size_t>(s) * kStageBytes + kATileBytes * kNA + kBBytes + which * kSfStage;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, BN);
+        const int slot = ti.g < E ? slot_of_expert[ti.g] : 0;
+        const uint8_t* bank = ti.g < E ? pool + static_cast<size_t>(slot) * bank_bytes : shared_bank;
+        const uint8_t* wsf = bank + wsf_off;
+        const int prow = prow0[ti.g] + ti.n * BN;
+        const uint8_t* asf = act_sf + static_cast<size_t>(prow / BN) * K64 * kSfChunk;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full_bar[stage], kTx);
+          const int kc = kb * (kF4StageK / 2);   // byte coordinate along K
+          if (ti.g < E) {
+            tma_load_3d(a_tile(stage, 0), &tmA, &full_bar[stage], kc, ti.m * 128, slot);
+            if (GATED) tma_load_3d(a_tile(stage, 1), &tmA, &full_bar[stage], kc, up_row0 + ti.m * 128, slot);
+          } else {
+            tma_load_2d(a_tile(stage, 0), &tmAsh, &full_bar[stage], kc, ti.m * 128);
+            if (GATED) tma_load_2d(a_tile(stage, 1), &tmAsh, &full_bar[stage], kc, up_row0 + ti.m * 128);
+          }
+          tma_load_2d(b_tile(stage), &tmB, &full_bar[stage], kc, prow);
+          bulk_load(sf_tile(stage, 0), wsf + (static_cast<size_t>(ti.m) * K64 + 4 * kb) * kSfChunk, kSfStage,
+                    &full_bar[stage]);
+          if (GATED)
+            bulk_load(sf_tile(stage, 1), wsf + (static_cast<size_t>(up_row0 / 128 + ti.m) * K64 + 4 * kb) * kSfChunk,
+                      kSfStage, &full_bar[stage]);
+          bulk_load(sf_tile(stage, kNA), asf + static_cast<size_t>(4 * kb) * kSfChunk, kSfStage, &full_bar[stage]);
+          if (++stage == stages) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+        const int ab = it & 1;
+        const uint32_t aphase = (it >> 1) & 1;
+        if (!mbar_wait(&tempty_bar[ab], aphase ^ 1u)) break;
+        tc_fence_after();
+        const uint32_t d_g = tmem_base + ab * kAccCols;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(a_tile(stage, 0));
+          const uint32_t sb = smem_u32(b_tile(stage));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            tmem_cp_sf(tmem_sf + 4 * kk, smem_desc_sf(smem_u32(sf_tile(stage, 0)) + kk * kSfChunk));
+            if (GATED) tmem_cp_sf(tmem_sf + 16 + 4 * kk, smem_desc_sf(smem_u32(sf_tile(stage, 1)) + kk * kSfChunk));
+            tmem_cp_sf(tmem_sf + 16 * kNA + 4 * kk, smem_desc_sf(smem_u32(sf_tile(stage, kNA)) + kk * kSfChunk));
+          }
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bdesc = smem_desc_sw128(sb + kk * 32);
+            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            umma_nvf4(d_g, smem_desc_sw128(sa + kk * 32), bdesc, kIdesc, tmem_sf + 4 * kk,
+                      tmem_sf + 16 * kNA + 4 * kk, acc);
+            if (GATED)
+              umma_nvf4(d_g + BN, smem_desc_sw128(sa + kATileBytes + kk * 32), bdesc, kIdesc, tmem_sf + 16 + 4 * kk,
+                        tmem_sf + 16 * kNA + 4 * kk, acc);
+          }
+          umma_commit(&empty_bar[stage]);
+          if (++stage == stages) { stage = 0; phase ^= 1u; }
+        }
+        if (ok) umma_commit(&tfull_bar[ab]);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int q = warp % 4;
+    int it = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+      const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, BN);
+      const int ab = it & 1;
+      const uint32_t aphase = (it >> 1) & 1;
+      if (!mbar_wait(&tfull_bar[ab], aphase)) break;
+      tc_fence_after();
+      const int valid = min(BN, ti.rows - ti.n * BN);
+      const uint8_t* bank = ti.g < E ? pool + static_cast<size_t>(slot_of_expert[ti.g]) * bank_bytes : shared_bank;
+      const float* st = reinterpret_cast<const float*>(bank + st_off);
+      const float s_a = st[st_idx];
+      const float s_u = GATED ? st[st_idx + 1] : 0.f;
+      const int wrow = ti.m * 128 + q * 32 + lane;
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * kAccCols;
+      if (GATED) {
+        const int prow = prow0[ti.g] + ti.n * BN;
+        const int blk = prow / BN;
+        const int gidx = wrow / 16;               // 16-group along the intermediate dim
+        const int kb64 = gidx / 4, j = gidx % 4;
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          float a[16], b[16];
+          tmem_ld16(tb + c0, a);
+          tmem_ld16(tb + BN + c0, b);
+          tmem_ld_wait();
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int c = c0 + jj;
+            // padding columns are quantised too (their rows are never read back)
+            const float h = silu(a[jj] * s_a) * (b[jj] * s_u);
+            float amax = fabsf(h);
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 8));
+            const uint8_t sq = f32_to_e4m3_sat(amax / 6.0f);
+            const float s = e4m3_to_f32(sq);
+            const float hv = s == 0.f ? 0.f : h / s;
+            const float hodd = __shfl_down_sync(0xffffffffu, hv, 1);
+            if ((lane & 1) == 0)
+              out_q[static_cast<size_t>(prow + c) * (Nw / 2) + wrow / 2] = s == 0.f ? 0 : f32x2_to_e2m1x2(hodd, hv);
+            if ((lane & 15) == 0)
+              out_sf[(static_cast<size_t>(blk) * (Nw / 64) + kb64) * kSfChunk + sf_byte(c, j)] = sq;
+          }
+        }
+      } else {
+        uint16_t* obase = out_bf16 + static_cast<size_t>(ti.row0 + ti.n * BN) * Nw + wrow;
+        for (int c0 = 0; c0 < valid; c0 += 16) {
+          float a[16];
+          tmem_ld16(tb + c0, a);
+          tmem_ld_wait();
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            if (c0 + jj < valid) {
+              const __nv_bfloat16 hb = __float2bfloat16_rn(a[jj] * s_a);
+              obase[static_cast<size_t>(c0 + jj) * Nw] = *reinterpret_cast<const uint16_t*>(&hb);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty_bar[ab]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// Host
+// ---------------------------------------------------------------------------
+static bool make_map_f4(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint64_t slots,
+                        uint64_t slot_pitch, uint32_t box_rows) {
+  // packed e2m1: K/2 bytes per row, addressed as bytes
+  return make_map_sw128(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, K / 2, rows, K / 2, slots, slot_pitch, box_rows);
+}
+
+int nvfp4_token_tile(int P, int E) { return (P + E - 1) / E <= 32 ? 32 : 64; }
+
+static size_t al256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+// Upper bound of the padded activation rows for token tile BN.
+static int64_t nvfp4_rows_pad(int64_t P, int T, int G, int has_shared, int BN) {
+  return P + (has_shared ? T : 0) + static_cast<int64_t>(G) * (BN - 1);
+}
+
+// Workspace: prow0 | Xq [rows_pad][d/2] | SFx chunks | Hq [rows_pad][I/2] | SFh chunks
+size_t nvfp4_ffn_workspace_bytes(int64_t P, int T, int E, int has_shared, int d, int I) {
+  const int G = E + (has_shared ? 1 : 0);
+  const int BN = 64;   // the larger tile bounds both
+  const int64_t rp = nvfp4_rows_pad(P, T, G, has_shared, BN);
+  const int64_t blocks = rp / 32 + G + 1;   // chunks are per BN-row block; BN >= 32
+  return al256(sizeof(int32_t) * (G + 1)) + al256(rp * (d / 2)) + al256(blocks * (d / 64) * kSfChunk) +
+         al256(rp * (I / 2)) + al256(blocks * (I / 64) * kSfChunk);
+}
+
+template <int BN, bool GATED>
+static cudaError_t launch_nvfp4(const CUtensorMap& mA, const CUtensorMap& mAsh, const CUtensorMap& mB,
+                                const FfnArgs& a, const int32_t* prow0, int K, int Nw, int up_row0, size_t wsf_off,
+                                size_t st_off, int st_idx, const uint8_t* act_sf, uint8_t* out_q, uint8_t* out_sf,
+                                uint16_t* out_bf16, cudaStream_t st) {
+  constexpr uint32_t kBBytes = ((BN * 128 + 1023) / 1024) * 1024;
+  constexpr uint32_t kNA = GATED ? 2 : 1;
+  constexpr uint32_t kStageBytes = kATileBytes * kNA + kBBytes + kSfStage * (kNA + 1);
+  int stages = (200 * 1024 - 1024) / static_cast<int>(kStageBytes);
+  if (stages > 8) stages = 8;
+  const size_t smem = 1024 + static_cast<size_t>(stages) * kStageBytes;
+  auto kern = ffn_nvfp4_kernel<BN, GATED>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  const int P = a.T * a.k;
+  const int G = a.E + (a.has_shared ? 1 : 0);
+  const long max_tiles = static_cast<long>((P + BN - 1) / BN + G) * (Nw / 128);
+  const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
+  kern<<<grid, kTcThreads, smem, st>>>(mA, mAsh, mB, a.offsets, prow0, a.slot_of_expert, a.E, a.has_shared, a.T, P,
+                                       K, Nw, up_row0, a.pool, a.shared_bank, a.bank_bytes, wsf_off, st_off, st_idx,
+                                       act_sf, out_q, out_sf, out_bf16, stages);
+  return cudaGetLastError();
+}
+
+const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_d_off, size_t s_t_off, uint8_t* ws,
+                                    cudaStream_t st, cudaError_t* cerr) {
+  const int P = a.T * a.k;
+  const int G = a.E + (a.has_shared ? 1 : 0);
+  *cerr = cudaSuccess;
+  if (P + (a.has_shared ? a.T : 0) == 0) return nullptr;
+  const int BN = nvfp4_token_tile(P, a.E);
+  const int64_t rp = nvfp4_rows_pad(P, a.T, G, a.has_shared, 64);
+  const int64_t blocks = rp / 32 + G + 1;
+  int32_t* prow0 = reinterpret_cast<int32_t*>(ws);
+  uint8_t* xq = ws + al256(sizeof(int32_t) * (G + 1));
+  uint8_t* sfx = xq + al256(rp * (a.d / 2));
+  uint8_t* hq = sfx + al256(blocks * (a.d / 64) * kSfChunk);
+  uint8_t* sfh = hq + al256(rp * (a.I / 2));
+  prof_mark(FTM_K_GATHER, st, false);
+  pad_offsets_kernel<<<1, 512, 0, st>>>(a.offsets, a.E, a.has_shared, a.T, BN, prow0);
+  {
+    const long warps = rp * (a.d / 64);
+    const int grid = static_cast<int>(warps / 8 + 1 < 148 * 16 ? warps / 8 + 1 : 148 * 16);
+    gather_quant_nvfp4_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint16_t*>(a.x), a.perm, a.offsets, prow0,
+                                                    a.E, a.has_shared, a.T, a.k, a.d, BN, static_cast<int>(rp), xq,
+                                                    sfx);
+  }
+  prof_mark(FTM_K_GATHER, st, true);
+  if ((*cerr = cudaGetLastError()) != cudaSuccess) return "nvfp4 gather launch failed";
+  CUtensorMap mA1, mAsh1, mB1, mA2, mAsh2, mB2;
+  const uint64_t S = static_cast<uint64_t>(a.S);
+  bool ok = make_map_f4(&mA1, a.pool + a.w_gu_off, a.d, 2ull * a.I, S, a.bank_bytes, 128) &&
+            make_map_f4(&mA2, a.pool + a.w_d_off, a.I, a.d, S, a.bank_bytes, 128) &&
+            make_map_f4(&mB1, xq, a.d, static_cast<uint64_t>(rp), 0, 0, BN) &&
+            make_map_f4(&mB2, hq, a.I, static_cast<uint64_t>(rp), 0, 0, BN);
+  if (ok && a.has_shared) {
+    ok = make_map_f4(&mAsh1, a.shared_bank + a.w_gu_off, a.d, 2ull * a.I, 0, 0, 128) &&
+         make_map_f4(&mAsh2, a.shared_bank + a.w_d_off, a.I, a.d, 0, 0, 128);
+  } else {
+    mAsh1 = mA1;
+    mAsh2 = mA2;
+  }
+  if (!ok) return "cuTensorMapEncodeTiled failed";
+  prof_mark(FTM_K_GEMM1, st, false);
+  *cerr = BN == 32 ? launch_nvfp4<32, true>(mA1, mAsh1, mB1, a, prow0, a.d, a.I, a.I, s_gu_off, s_t_off, 0, sfx, hq,
+                                            sfh, nullptr, st)
+                   : launch_nvfp4<64, true>(mA1, mAsh1, mB1, a, prow0, a.d, a.I, a.I, s_gu_off, s_t_off, 0, sfx, hq,
+                                            sfh, nullptr, st);
+  prof_mark(FTM_K_GEMM1, st, true);
+  if (*cerr != cudaSuccess) return "nvfp4 gemm1 launch failed";
+  prof_mark(FTM_K_GEMM2, st, false);
+  *cerr = BN == 32 ? launch_nvfp4<32, false>(mA2, mAsh2, mB2, a, prow0, a.I, a.d, 0, s_d_off, s_t_off, 2, sfh,
+                                             nullptr, nullptr, reinterpret_cast<uint16_t*>(a.y), st)
+                   : launch_nvfp4<64, false>(mA2, mAsh2, mB2, a, prow0, a.I, a.d, 0, s_d_off, s_t_off, 2, sfh,
+                                             nullptr, nullptr, reinterpret_cast<uint16_t*>(a.y), st);
+  prof_mark(FTM_K_GEMM2, st, true);
+  if (*cerr != cudaSuccess) return "nvfp4 gemm2 launch failed";
+  return nullptr;
+}
+
+}  // namespace ftm

@@ -67,13 +67,23 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_topk_kernel(const Tin*
   const int nt = min(TT, T - t0);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  // token tile -> shared memory (rows beyond T are zero)
+  // token tile -> shared memory (rows beyond T are zero); 8 loads in flight per thread
   const int vec_per_row = d / V;
-  for (int i = threadIdx.x; i < TT * vec_per_row; i += blockDim.x) {
-    const int r = i / vec_per_row, c = i % vec_per_row;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r < nt) v = *reinterpret_cast<const uint4*>(x + static_cast<size_t>(t0 + r) * d + c * V);
-    *reinterpret_cast<uint4*>(xs + static_cast<size_t>(r) * d + c * V) = v;
+  const int nvec = TT * vec_per_row;
+  for (int base = threadIdx.x; base < nvec; base += 8 * blockDim.x) {
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + u * blockDim.x;
+      const int r = i / vec_per_row, c = i % vec_per_row;
+      v[u] = make_uint4(0, 0, 0, 0);
+      if (i < nvec && r < nt) v[u] = *reinterpret_cast<const uint4*>(x + static_cast<size_t>(t0 + r) * d + c * V);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + u * blockDim.x;
+      if (i < nvec) *reinterpret_cast<uint4*>(xs + static_cast<size_t>(i) * V) = v[u];
+    }
   }
   __syncthreads();
 
@@ -85,7 +95,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_topk_kernel(const Tin*
 #pragma unroll
     for (int t = 0; t < TT; ++t) acc[t] = 0.f;
     const Tin* wrow = wr + static_cast<size_t>(e) * d;
-#pragma unroll 4
+#pragma unroll 8
     for (int c = lane * V; c < d; c += 32 * V) {
       float w[V];
       IO::load(wrow + c, w);
@@ -175,9 +185,15 @@ static cudaError_t launch_route_tt(const void* x, int T, int d, const void* wr, 
                             ids, w);
 }
 
-// Token-tile size: the x tile must fit next to the logits buffer.
+bool route_tc_applicable(bool f32, int T, int E, int k);
+cudaError_t launch_route_tc(const void* x, int T, int d, const void* wr, const float* bias, int E, int k,
+                            int32_t* ids, float* w, cudaStream_t st);
+
+// Large bf16 batches go to the tensor-core router; otherwise the token-tile
+// size is chosen so the x tile fits next to the logits buffer.
 cudaError_t launch_route(bool f32, const void* x, int T, int d, const void* wr, const float* bias, int E, int k,
                          int32_t* ids, float* w, cudaStream_t st) {
+  if (route_tc_applicable(f32, T, E, k)) return launch_route_tc(x, T, d, wr, bias, E, k, ids, w, st);
   const size_t elt = f32 ? 4 : 2;
   const size_t budget = 160 * 1024 - sizeof(float) * 16 * kMaxE;
   if (16 * d * elt <= budget && T >= 16) {

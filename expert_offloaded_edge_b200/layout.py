@@ -11,6 +11,16 @@ import numpy as np
 from .binding import FTM_BF16, FTM_F32, FTM_FP8_E4M3_B128, FTM_NVFP4, BankLayout, LayerDesc, ftm_get_bank_layout
 
 
+def nvfp4_scale_chunks(s16: np.ndarray) -> np.ndarray:
+    """e4m3 scales [R][C/16] -> the MMA chunk layout: one 512-byte chunk per
+    (128-row block rb, 64-column block kb), chunks ordered [rb][kb]; inside a
+    chunk the scale of local row r and 16-group j is byte (r%32)*16 + (r//32)*4 + j."""
+    R, G16 = s16.shape
+    assert R % 128 == 0 and G16 % 4 == 0
+    a = np.ascontiguousarray(s16, dtype=np.uint8).reshape(R // 128, 4, 32, G16 // 4, 4)
+    return np.ascontiguousarray(a.transpose(0, 3, 2, 1, 4)).ravel()
+
+
 def _put(bank: np.ndarray, off: int, arr: np.ndarray, nbytes: int):
     b = np.ascontiguousarray(arr).view(np.uint8).ravel()
     assert b.size == nbytes, (b.size, nbytes)
@@ -36,8 +46,8 @@ def pack_bank(desc: LayerDesc, ew, bl: BankLayout = None, out: np.ndarray = None
     elif w == FTM_NVFP4:
         _put(bank, bl.w_gu_off, np.concatenate([ew.gate[0], ew.up[0]], axis=0), bl.w_gu_bytes)
         _put(bank, bl.w_d_off, ew.down[0], bl.w_d_bytes)
-        _put(bank, bl.s_gu_off, np.concatenate([ew.gate[1], ew.up[1]], axis=0), bl.s_gu_bytes)
-        _put(bank, bl.s_d_off, ew.down[1], bl.s_d_bytes)
+        _put(bank, bl.s_gu_off, nvfp4_scale_chunks(np.concatenate([ew.gate[1], ew.up[1]], axis=0)), bl.s_gu_bytes)
+        _put(bank, bl.s_d_off, nvfp4_scale_chunks(ew.down[1]), bl.s_d_bytes)
         _put(bank, bl.s_t_off, np.array([ew.gate[2], ew.up[2], ew.down[2], 0.0], dtype=np.float32), bl.s_t_bytes)
     else:
         raise ValueError(w)

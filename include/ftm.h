@@ -80,9 +80,13 @@ typedef struct ftm_layer_desc {
  *         (f32 / bf16 / e4m3 elements; NVFP4: [2I][d/2] bytes, two codes per
  *         byte, element 2j in the low nibble)
  *   w_d : [d][I] row-major (same element rules)
- *   s_gu: FP8: fp32 [2I/128][d/128]; NVFP4: e4m3 [2I][d/16]; else empty
- *   s_d : FP8: fp32 [d/128][I/128];  NVFP4: e4m3 [d][I/16];  else empty
- *   s_t : NVFP4: fp32[4] = {gate, up, down, 0} per-tensor scales; else empty */
+ *   s_gu: FP8: fp32 [2I/128][d/128]; NVFP4: the 2I x d/16 e4m3 scales in chunks (below)
+ *   s_d : FP8: fp32 [d/128][I/128];  NVFP4: the d x I/16 e4m3 scales in chunks
+ *   s_t : NVFP4: fp32[4] = {gate, up, down, 0} per-tensor scales; else empty
+ * NVFP4 scale chunks (the layout the block-scaled MMA reads): one 512-byte
+ * chunk per (128-row block rb, 64-column block kb), ordered [rb][kb]; in a
+ * chunk the scale of local row r (0..127) for its j-th 16-column group of the
+ * block (0..3) is byte (r % 32) * 16 + (r / 32) * 4 + j. */
 typedef struct ftm_bank_layout {
   uint64_t bank_bytes;
   uint64_t w_gu_off, w_gu_bytes;

@@ -4,6 +4,8 @@ import ctypes
 import os
 import re
 
+import numpy as np
+
 import pytest
 
 import expert_offloaded_edge_b200 as ftm
@@ -75,3 +77,17 @@ def test_workspace_sizes_monotone():
         sizes = [ftm.ftm_workspace_bytes(d, T) for T in (0, 1, 16, 1024, 16384)]
         assert sizes == sorted(sizes) and sizes[1] > 0
         assert ftm.ftm_ffn_workspace_bytes(d, 16) <= ftm.ftm_workspace_bytes(d, 16)
+
+
+def test_nvfp4_scale_chunk_packing_brute_force():
+    from expert_offloaded_edge_b200.layout import nvfp4_scale_chunks
+    rng = np.random.default_rng(0)
+    R, G16 = 256, 24
+    s16 = rng.integers(0, 256, size=(R, G16), dtype=np.uint8)
+    packed = nvfp4_scale_chunks(s16)
+    assert packed.size == s16.size
+    for r in range(R):
+        for g in range(G16):
+            rb, kb, rl, j = r // 128, g // 4, r % 128, g % 4
+            off = (rb * (G16 // 4) + kb) * 512 + (rl % 32) * 16 + (rl // 32) * 4 + j
+            assert packed[off] == s16[r, g]
