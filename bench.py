@@ -99,24 +99,28 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def kernel_source_hash() -> str:
+KERNEL_FILES = {"bf16": "ftm_ffn.cu", "f32": "ftm_ffn.cu", "fp8": "ftm_ffn_fp8.cu", "nvfp4": "ftm_ffn_nvfp4.cu"}
+
+
+def kernel_source_hash(wdtype: str) -> str:
+    """Hash of the sources the dominant kernel of a dtype is built from."""
     h = hashlib.sha256()
-    for n in ("ftm_ffn.cu", "ftm_common.cuh"):
+    for n in (KERNEL_FILES[wdtype], "ftm_gemm.cuh", "ftm_common.cuh"):
         with open(os.path.join(ROOT, "expert_offloaded_edge_b200", "csrc", n), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload: str, kernel: str):
-    """dram bytes per launch from the committed ncu summary, or None if absent
-    or taken on a different version of the kernel source."""
+def ncu_traffic(workload: str, kernel: str, wdtype: str):
+    """dram bytes per launch from the committed ncu summary (profiles/traffic.json),
+    or None if absent or taken on a different version of the kernel source."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(f"{workload}/{kernel}")
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(wdtype):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -403,7 +407,7 @@ def trace_main(args, cfg, T, rank, world, local, dist):
         "roofline": {"bound": "hbm", "achieved": ach, "peak": float(pk["hbm_gbs"]), "unit": "GB/s",
                      "frac": ach / float(pk["hbm_gbs"]), "kernel": "gemm1 (fp8 grouped gate/up + SwiGLU)",
                      "algorithmic_bytes": alg_g1, "peak_source": f"{src} hbm_gbs",
-                     "traffic": ncu_traffic(workload_name(cfg, T), "gemm1")},
+                     "traffic": ncu_traffic(workload_name(cfg, T), "gemm1", cfg.wdtype)},
         "cache": {"hit_rate": hits / max(1, distinct), "misses_per_step": misses / K,
                   "h2d_gb_per_step": misses / K * bl.bank_bytes / 1e9,
                   "h2d_gbs_effective": misses * bl.bank_bytes / (ms * 1e-3) / 1e9},
@@ -531,11 +535,16 @@ def main():
                     "peak_source": f"{src} hbm_gbs"}
         else:
             ach = alg["gemm1_flops"] / (g1 * 1e-3) / 1e12
-            peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+            bf16 = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+            # a contraction takes its own dtype's peak: the measured bf16 figure times the
+            # nominal dense ratio (fp8 4.5/2.25 = 2, fp4 9/2.25 = 4), labelled as derived
+            ratio = {"f32": 1.0, "bf16": 1.0, "fp8": 2.0, "nvfp4": 4.0}[cfg.wdtype]
+            peak = bf16 * ratio
             roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
                     "kernel": "gemm1 (grouped gate/up + SwiGLU)", "algorithmic_flops": alg["gemm1_flops"],
-                    "peak_source": f"{src} bf16_tflops_sustained"}
-        roof["traffic"] = ncu_traffic(workload_name(cfg, T), "gemm1")
+                    "peak_source": (f"{src} bf16_tflops_sustained" if ratio == 1.0 else
+                                    f"derived: {ratio:g} x {src} bf16_tflops_sustained (nominal dense ratio)")}
+        roof["traffic"] = ncu_traffic(workload_name(cfg, T), "gemm1", cfg.wdtype)
         cpu = None
         if not args.no_cpu_baseline and world == 1:
             v, n, cores, secs = oracle_tokens_per_s(cfg, T, args.cpu_seconds)

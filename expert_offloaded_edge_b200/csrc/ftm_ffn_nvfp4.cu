@@ -118,35 +118,39 @@ __global__ void pad_offsets_kernel(const int32_t* __restrict__ offsets, int E, i
 
 // ---------------------------------------------------------------------------
 // Gather + NVFP4 quantisation of x into the padded activation rows.
-// One warp per (padded row, 64-element K block); lane l holds elements 2l, 2l+1.
+// One block per padded row (grid-strided): the row's source token is found once
+// (thread 0 searches the padded group offsets), then each warp takes 64-element
+// K blocks; lane l holds elements 2l, 2l+1.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) gather_quant_nvfp4_kernel(const uint16_t* __restrict__ x,
                                                                 const int32_t* __restrict__ perm,
                                                                 const int32_t* __restrict__ offsets,
                                                                 const int32_t* __restrict__ prow0, int E,
                                                                 int has_shared, int T, int k, int d, int BN,
-                                                                int rows_pad_max, uint8_t* __restrict__ xq,
+                                                                uint8_t* __restrict__ xq,
                                                                 uint8_t* __restrict__ sfx) {
+  __shared__ int s_src;
   const int G = E + (has_shared ? 1 : 0);
   const int rows_pad = prow0[G];
   const int kb64 = d / 64;
-  const int lane = threadIdx.x % 32;
-  const long total = static_cast<long>(rows_pad) * kb64;
-  (void)rows_pad_max;
-  for (long w = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32; w < total;
-       w += static_cast<long>(gridDim.x) * blockDim.x / 32) {
-    const int pr = static_cast<int>(w / kb64), kb = static_cast<int>(w % kb64);
-    int lo = 0, hi = G;  // prow0[lo] <= pr < prow0[hi]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (prow0[mid] <= pr) lo = mid; else hi = mid;
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nwarps = blockDim.x / 32;
+  for (int pr = blockIdx.x; pr < rows_pad; pr += gridDim.x) {
+    if (threadIdx.x == 0) {
+      int lo = 0, hi = G;  // prow0[lo] <= pr < prow0[hi]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (prow0[mid] <= pr) lo = mid; else hi = mid;
+      }
+      const int local = pr - prow0[lo];
+      const int rows = lo < E ? offsets[lo + 1] - offsets[lo] : T;
+      s_src = local >= rows ? -1 : (lo < E ? perm[offsets[lo] + local] / k : local);
     }
-    const int g = lo;
-    const int local = pr - prow0[g];
-    const int rows = g < E ? offsets[g + 1] - offsets[g] : T;
+    __syncthreads();
+    const int src = s_src;
+    __syncthreads();
+    for (int kb = warp; kb < kb64; kb += nwarps) {
     float v0 = 0.f, v1 = 0.f;
-    if (local < rows) {
-      const int src = g < E ? perm[offsets[g] + local] / k : local;
+    if (src >= 0) {
       const uint32_t u = *reinterpret_cast<const uint32_t*>(x + static_cast<size_t>(src) * d + kb * 64 + 2 * lane);
       v0 = bf16_bits_to_f32(u & 0xFFFF);
       v1 = bf16_bits_to_f32(u >> 16);
@@ -162,6 +166,7 @@ __global__ void __launch_bounds__(256) gather_quant_nvfp4_kernel(const uint16_t*
     if ((lane & 7) == 0) {
       const int blk = pr / BN, r = pr % BN;
       sfx[(static_cast<size_t>(blk) * kb64 + kb) * kSfChunk + sf_byte(r, lane / 8)] = sq;
+    }
     }
   }
 }
@@ -453,11 +458,9 @@ const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_
   prof_mark(FTM_K_GATHER, st, false);
   pad_offsets_kernel<<<1, 512, 0, st>>>(a.offsets, a.E, a.has_shared, a.T, BN, prow0);
   {
-    const long warps = rp * (a.d / 64);
-    const int grid = static_cast<int>(warps / 8 + 1 < 148 * 16 ? warps / 8 + 1 : 148 * 16);
+    const int grid = static_cast<int>(rp < 148 * 16 ? rp : 148 * 16);
     gather_quant_nvfp4_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint16_t*>(a.x), a.perm, a.offsets, prow0,
-                                                    a.E, a.has_shared, a.T, a.k, a.d, BN, static_cast<int>(rp), xq,
-                                                    sfx);
+                                                    a.E, a.has_shared, a.T, a.k, a.d, BN, xq, sfx);
   }
   prof_mark(FTM_K_GATHER, st, true);
   if ((*cerr = cudaGetLastError()) != cudaSuccess) return "nvfp4 gather launch failed";
