@@ -125,6 +125,20 @@ def ncu_traffic(workload: str, kernel: str, wdtype: str):
     return e.get("dram_bytes_per_launch")
 
 
+# --------------------------------------------------------------------------- ranks
+def job_throughput(local_ms: float, units_per_rank: int, dist, device) -> tuple:
+    """Whole-job throughput of N independent replicas: the slowest rank's time
+    (max over ranks) and all ranks' units divided by it.  dist=None: one rank."""
+    world = 1
+    ms = float(local_ms)
+    if dist is not None:
+        world = dist.get_world_size()
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms, units_per_rank * world / (ms / 1e3)
+
+
 # --------------------------------------------------------------------------- workload
 def workload_name(cfg, T):
     return f"{cfg.name} T={T}"
@@ -382,11 +396,7 @@ def trace_main(args, cfg, T, rank, world, local, dist):
     ms = t0.elapsed_time(t1)
     clk = clocks.stop()
     g1 = [a.elapsed_time(b) for a, b in evs]
-    if dist:
-        tt = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
-    value = K * T * world / (ms / 1e3)
+    ms, value = job_throughput(ms, K * T, dist, "cuda")
     status = ftm.ftm_device_status(True)
     if rank != 0:
         return
@@ -476,13 +486,9 @@ def main():
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1)
     clk = clocks.stop()
+    ms, value = job_throughput(ms, args.steps * T, dist, "cuda")
     if dist:
-        tt = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
         dist.barrier()
-    tokens = args.steps * T * world
-    value = tokens / (ms / 1e3)
 
     # per-kernel breakdown (after the timed region; every kernel bracketed by events)
     r.KERNELS = Runner.ALL
@@ -513,12 +519,7 @@ def main():
             out_host.copy_(r.out, non_blocking=True)
     e1.record(s)
     torch.cuda.synchronize()
-    e_ms = e0.elapsed_time(e1)
-    if dist:
-        tt = torch.tensor([e_ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e_ms = float(tt.item())
-    e2e_value = e_steps * T * world / (e_ms / 1e3)
+    e_ms, e2e_value = job_throughput(e0.elapsed_time(e1), e_steps * T, dist, "cuda")
     status = ftm.ftm_device_status(True)
 
     if rank == 0:

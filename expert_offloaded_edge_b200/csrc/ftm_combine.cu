@@ -12,6 +12,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ y
                                                       int has_shared, void* __restrict__ out) {
   constexpr int V = F32 ? 4 : 8;   // elements per 16-byte vector
   const int nv = d / V;
+  pdl_wait();
+  pdl_trigger();
   for (int t = blockIdx.x; t < T; t += gridDim.x) {
     for (int c = threadIdx.x; c < nv; c += blockDim.x) {
       float acc[V];
@@ -67,9 +69,9 @@ cudaError_t launch_combine(bool f32, const void* y, const int32_t* inv, const fl
                            int has_shared, void* out, cudaStream_t st) {
   const int grid = T < 148 * 16 ? T : 148 * 16;
   if (f32)
-    combine_kernel<true><<<grid, 256, 0, st>>>(y, inv, gw, T, k, d, P, has_shared, out);
+    return launch_pdl(combine_kernel<true>, dim3(grid), dim3(256), 0, st, y, inv, gw, T, k, d, P, has_shared, out);
   else
-    combine_kernel<false><<<grid, 256, 0, st>>>(y, inv, gw, T, k, d, P, has_shared, out);
+    return launch_pdl(combine_kernel<false>, dim3(grid), dim3(256), 0, st, y, inv, gw, T, k, d, P, has_shared, out);
   return cudaGetLastError();
 }
 

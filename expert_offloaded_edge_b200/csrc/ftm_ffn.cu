@@ -28,6 +28,8 @@ __device__ int32_t g_dev_status = 0;
 // ---------------------------------------------------------------------------
 __global__ void gather_rows_kernel(const uint8_t* __restrict__ x, const int32_t* __restrict__ perm, int P, int k,
                                    int T, int has_shared, int row_bytes, uint8_t* __restrict__ xp) {
+  pdl_wait();
+  pdl_trigger();
   const int rows = P + (has_shared ? T : 0);
   const int nv = row_bytes / 16;
   for (int r = blockIdx.x; r < rows; r += gridDim.x) {
@@ -57,6 +59,8 @@ __global__ void __launch_bounds__(256) simt_gemm1_kernel(const float* __restrict
                                                          int d, int I, const uint8_t* __restrict__ pool,
                                                          const uint8_t* __restrict__ shared_bank, size_t bank_bytes,
                                                          size_t wgu_off, float* __restrict__ h) {
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   const int g = group_of_row(offsets, E, P, r);
   const float* W = reinterpret_cast<const float*>(
@@ -79,6 +83,8 @@ __global__ void __launch_bounds__(256) simt_gemm2_kernel(const float* __restrict
                                                          int d, int I, const uint8_t* __restrict__ pool,
                                                          const uint8_t* __restrict__ shared_bank, size_t bank_bytes,
                                                          size_t wd_off, float* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   const int g = group_of_row(offsets, E, P, r);
   const float* W = reinterpret_cast<const float*>(
@@ -124,7 +130,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int MT = Nw / 128;
   const int KB = K / kBK;
 
-  build_tile_table(offsets, E, has_shared, T, P, MT, BN, tile_start, grp_rows, grp_row0);
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 4); }
@@ -139,6 +144,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tma_prefetch_desc(&tmAsh);
     tma_prefetch_desc(&tmB);
   }
+  pdl_wait();      // the group offsets come from earlier kernels
+  pdl_trigger();
+  build_tile_table(offsets, E, has_shared, T, P, MT, BN, tile_start, grp_rows, grp_row0);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -274,9 +282,8 @@ static cudaError_t launch_tc(const CUtensorMap& mA, const CUtensorMap& mAsh, con
   const int G = a.E + (a.has_shared ? 1 : 0);
   const long max_tiles = static_cast<long>((P + BN - 1) / BN + G) * (Nw / 128);
   const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
-  kern<<<grid, kTcThreads, smem, st>>>(mA, mAsh, mB, a.offsets, a.slot_of_expert, a.E, a.has_shared, a.T, P, K, Nw,
-                                       up_row0, out, ld_out, stages);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st, mA, mAsh, mB, a.offsets, a.slot_of_expert, a.E,
+                    a.has_shared, a.T, P, K, Nw, up_row0, out, ld_out, stages);
 }
 
 template <bool GATED>
@@ -287,7 +294,11 @@ static cudaError_t launch_tc_bn(int bn, const CUtensorMap& mA, const CUtensorMap
     case 16: return launch_tc<16, GATED>(mA, mAsh, mB, a, K, Nw, up_row0, out, ld_out, st);
     case 32: return launch_tc<32, GATED>(mA, mAsh, mB, a, K, Nw, up_row0, out, ld_out, st);
     case 64: return launch_tc<64, GATED>(mA, mAsh, mB, a, K, Nw, up_row0, out, ld_out, st);
-    default: return launch_tc<128, GATED>(mA, mAsh, mB, a, K, Nw, up_row0, out, ld_out, st);
+    case 128: return launch_tc<128, GATED>(mA, mAsh, mB, a, K, Nw, up_row0, out, ld_out, st);
+    default:
+      // 256-token tiles only without the gate/up pair (TMEM holds 2 x 256 fp32 columns)
+      if (GATED) return launch_tc<128, GATED>(mA, mAsh, mB, a, K, Nw, up_row0, out, ld_out, st);
+      return launch_tc<256, false>(mA, mAsh, mB, a, K, Nw, up_row0, out, ld_out, st);
   }
 }
 
@@ -306,34 +317,36 @@ const char* launch_expert_ffn(const FfnArgs& a, cudaStream_t st, cudaError_t* ce
   {
     const int grid = rows < 148 * 8 ? rows : 148 * 8;
     prof_mark(FTM_K_GATHER, st, false);
-    gather_rows_kernel<<<grid, 256, 0, st>>>(a.x, a.perm, P, a.k, a.T, a.has_shared, a.d * elt, a.xp);
+    *cerr = launch_pdl(gather_rows_kernel, dim3(grid), dim3(256), 0, st, a.x, a.perm, P, a.k, a.T, a.has_shared,
+                       a.d * elt, a.xp);
     prof_mark(FTM_K_GATHER, st, true);
-    if ((*cerr = cudaGetLastError()) != cudaSuccess) return "gather launch failed";
+    if (*cerr != cudaSuccess) return "gather launch failed";
   }
   if (a.f32) {
     dim3 g1(rows, (a.I + 63) / 64), g2(rows, (a.d + 63) / 64);
     prof_mark(FTM_K_GEMM1, st, false);
-    simt_gemm1_kernel<<<g1, 256, 0, st>>>(reinterpret_cast<const float*>(a.xp), a.offsets, a.slot_of_expert, a.E, P,
-                                          a.d, a.I, a.pool, a.shared_bank, a.bank_bytes, a.w_gu_off,
-                                          reinterpret_cast<float*>(a.h));
+    *cerr = launch_pdl(simt_gemm1_kernel, g1, dim3(256), 0, st, reinterpret_cast<const float*>(a.xp), a.offsets,
+                       a.slot_of_expert, a.E, P, a.d, a.I, a.pool, a.shared_bank, a.bank_bytes, a.w_gu_off,
+                       reinterpret_cast<float*>(a.h));
     prof_mark(FTM_K_GEMM1, st, true);
-    if ((*cerr = cudaGetLastError()) != cudaSuccess) return "simt gemm1 launch failed";
+    if (*cerr != cudaSuccess) return "simt gemm1 launch failed";
     prof_mark(FTM_K_GEMM2, st, false);
-    simt_gemm2_kernel<<<g2, 256, 0, st>>>(reinterpret_cast<const float*>(a.h), a.offsets, a.slot_of_expert, a.E, P,
-                                          a.d, a.I, a.pool, a.shared_bank, a.bank_bytes, a.w_d_off,
-                                          reinterpret_cast<float*>(a.y));
+    *cerr = launch_pdl(simt_gemm2_kernel, g2, dim3(256), 0, st, reinterpret_cast<const float*>(a.h), a.offsets,
+                       a.slot_of_expert, a.E, P, a.d, a.I, a.pool, a.shared_bank, a.bank_bytes, a.w_d_off,
+                       reinterpret_cast<float*>(a.y));
     prof_mark(FTM_K_GEMM2, st, true);
-    if ((*cerr = cudaGetLastError()) != cudaSuccess) return "simt gemm2 launch failed";
+    if (*cerr != cudaSuccess) return "simt gemm2 launch failed";
     return nullptr;
   }
-  // bf16 tensor-core path
+  // bf16 tensor-core path; the down projection takes 256-token tiles when groups are large
   const int bn = ffn_token_tile(P, a.E);
+  const int bn2 = (P + a.E - 1) / a.E >= 192 ? 256 : bn;
   CUtensorMap mA1, mAsh1, mB1, mA2, mAsh2, mB2;
   const uint64_t S = static_cast<uint64_t>(a.S);
   bool ok = make_map_bf16(&mA1, a.pool + a.w_gu_off, a.d, 2ull * a.I, 2ull * a.d, S, a.bank_bytes, 128) &&
             make_map_bf16(&mA2, a.pool + a.w_d_off, a.I, a.d, 2ull * a.I, S, a.bank_bytes, 128) &&
             make_map_bf16(&mB1, a.xp, a.d, rows, 2ull * a.d, 0, 0, bn) &&
-            make_map_bf16(&mB2, a.h, a.I, rows, 2ull * a.I, 0, 0, bn);
+            make_map_bf16(&mB2, a.h, a.I, rows, 2ull * a.I, 0, 0, bn2);
   if (ok && a.has_shared) {
     ok = make_map_bf16(&mAsh1, a.shared_bank + a.w_gu_off, a.d, 2ull * a.I, 2ull * a.d, 0, 0, 128) &&
          make_map_bf16(&mAsh2, a.shared_bank + a.w_d_off, a.I, a.d, 2ull * a.I, 0, 0, 128);
@@ -347,7 +360,7 @@ const char* launch_expert_ffn(const FfnArgs& a, cudaStream_t st, cudaError_t* ce
   prof_mark(FTM_K_GEMM1, st, true);
   if (*cerr != cudaSuccess) return "tensor-core gemm1 launch failed";
   prof_mark(FTM_K_GEMM2, st, false);
-  *cerr = launch_tc_bn<false>(bn, mA2, mAsh2, mB2, a, a.I, a.d, 0, reinterpret_cast<uint16_t*>(a.y), a.d, st);
+  *cerr = launch_tc_bn<false>(bn2, mA2, mAsh2, mB2, a, a.I, a.d, 0, reinterpret_cast<uint16_t*>(a.y), a.d, st);
   prof_mark(FTM_K_GEMM2, st, true);
   if (*cerr != cudaSuccess) return "tensor-core gemm2 launch failed";
   return nullptr;

@@ -17,6 +17,7 @@
 namespace ftm {
 
 constexpr uint32_t kF8StageK = 128;          // K per stage = one scale block = one 128-byte swizzle row
+constexpr int kF8MaxKB = 64;                  // K <= 8192 (scales of a tile staged in shared memory)
 
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
   // c_format F32 (bit 4); a/b format E4M3 = 0; K-major; N>>3 at 17; M>>4 at 24
@@ -48,6 +49,8 @@ __global__ void __launch_bounds__(256) gather_quant_fp8_kernel(const uint16_t* _
                                                               const int32_t* __restrict__ perm, int P, int k, int T,
                                                               int has_shared, int d, uint8_t* __restrict__ xq,
                                                               float* __restrict__ sx) {
+  pdl_wait();
+  pdl_trigger();
   const int rows = P + (has_shared ? T : 0);
   const int groups = d / 128;
   const int lane = threadIdx.x % 32;
@@ -101,6 +104,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ uint32_t tmem_holder;
   __shared__ int32_t tile_start[kMaxGroups + 1], grp_rows[kMaxGroups], grp_row0[kMaxGroups];
   __shared__ float red[4][BN];
+  __shared__ float s_sact[BN * kF8MaxKB], s_wsc[2][kF8MaxKB];
 
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (smem_base - smem_u32(smem_raw));
@@ -109,7 +113,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int MT = Nw / 128;
   const int KB = K / kF8StageK;
 
-  build_tile_table(offsets, E, has_shared, T, P, MT, BN, tile_start, grp_rows, grp_row0);
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(&pfull_bar[a], 1); mbar_init(&pempty_bar[a], 4); }
@@ -124,6 +127,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tma_prefetch_desc(&tmAsh);
     tma_prefetch_desc(&tmB);
   }
+  pdl_wait();      // the group offsets come from earlier kernels
+  pdl_trigger();
+  build_tile_table(offsets, E, has_shared, T, P, MT, BN, tile_start, grp_rows, grp_row0);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -203,6 +209,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int rowbase = ti.row0 + ti.n * BN;
       const uint8_t* bank = ti.g < E ? pool + static_cast<size_t>(slot_of_expert[ti.g]) * bank_bytes : shared_bank;
       const float* wsc = reinterpret_cast<const float*>(bank + wscale_off);
+      // the tile's scales, staged once so the per-K-block promotion reads shared memory only
+      epilogue_bar();   // readers of the previous tile are done
+      for (int i = et; i < BN * KB; i += 128) {
+        const int c = i / KB, kb = i % KB;
+        s_sact[i] = c < valid ? sact[static_cast<size_t>(rowbase + c) * KB + kb] : 0.f;
+      }
+      for (int i = et; i < KB; i += 128) {
+        s_wsc[0][i] = wsc[static_cast<size_t>(ti.m) * KB + i];
+        if (GATED) s_wsc[1][i] = wsc[static_cast<size_t>(up_row0 / 128 + ti.m) * KB + i];
+      }
+      epilogue_bar();
       float acc_g[BN], acc_u[GATED ? BN : 1];
 #pragma unroll
       for (int c = 0; c < BN; ++c) acc_g[c] = 0.f;
@@ -210,12 +227,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int c = 0; c < (GATED ? BN : 1); ++c) acc_u[c] = 0.f;
       for (int kb = 0; kb < KB; ++kb, ++kcount) {
         const uint32_t pb = kcount & 1u, pph = (kcount >> 1) & 1u;
-        // scales first (independent of the MMA)
-        const float sa_g = wsc[static_cast<size_t>(ti.m) * KB + kb];
-        const float sa_u = GATED ? wsc[static_cast<size_t>(up_row0 / 128 + ti.m) * KB + kb] : 0.f;
+        const float sa_g = s_wsc[0][kb];
+        const float sa_u = GATED ? s_wsc[1][kb] : 0.f;
         float sb[BN];
 #pragma unroll
-        for (int c = 0; c < BN; ++c) sb[c] = c < valid ? sact[static_cast<size_t>(rowbase + c) * KB + kb] : 0.f;
+        for (int c = 0; c < BN; ++c) sb[c] = s_sact[c * KB + kb];
         if (!epilogue_all(mbar_wait(&pfull_bar[pb], pph))) { ok = false; break; }
         tc_fence_after();
         const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + pb * kAccCols;
@@ -308,10 +324,9 @@ static cudaError_t launch_fp8(const CUtensorMap& mA, const CUtensorMap& mAsh, co
   const int G = a.E + (a.has_shared ? 1 : 0);
   const long max_tiles = static_cast<long>((P + BN - 1) / BN + G) * (Nw / 128);
   const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
-  kern<<<grid, kTcThreads, smem, st>>>(mA, mAsh, mB, a.offsets, a.slot_of_expert, a.E, a.has_shared, a.T, P, K, Nw,
-                                       up_row0, a.pool, a.shared_bank, a.bank_bytes, wscale_off, sact, out_q, out_s,
-                                       out_bf16, stages);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st, mA, mAsh, mB, a.offsets, a.slot_of_expert, a.E,
+                    a.has_shared, a.T, P, K, Nw, up_row0, a.pool, a.shared_bank, a.bank_bytes, wscale_off, sact, out_q,
+                    out_s, out_bf16, stages);
 }
 
 template <bool GATED>
@@ -336,6 +351,7 @@ const char* launch_expert_ffn_fp8(const FfnArgs& a, size_t s_gu_off, size_t s_d_
   const int rows = P + (a.has_shared ? a.T : 0);
   *cerr = cudaSuccess;
   if (rows == 0) return nullptr;
+  if (a.d / 128 > kF8MaxKB || a.I / 128 > kF8MaxKB) return "FP8 FFN supports d, I <= 8192";
   uint8_t* xq = ws;
   float* sx = reinterpret_cast<float*>(xq + al(static_cast<size_t>(rows) * a.d));
   uint8_t* hq = reinterpret_cast<uint8_t*>(sx) + al(static_cast<size_t>(rows) * (a.d / 128) * 4);
@@ -344,10 +360,10 @@ const char* launch_expert_ffn_fp8(const FfnArgs& a, size_t s_gu_off, size_t s_d_
     const long warps = static_cast<long>(rows) * (a.d / 128);
     const int grid = static_cast<int>(warps / 8 + 1 < 148 * 16 ? warps / 8 + 1 : 148 * 16);
     prof_mark(FTM_K_GATHER, st, false);
-    gather_quant_fp8_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint16_t*>(a.x), a.perm, P, a.k, a.T,
-                                                  a.has_shared, a.d, xq, sx);
+    *cerr = launch_pdl(gather_quant_fp8_kernel, dim3(grid), dim3(256), 0, st, reinterpret_cast<const uint16_t*>(a.x),
+                       a.perm, P, a.k, a.T, a.has_shared, a.d, xq, sx);
     prof_mark(FTM_K_GATHER, st, true);
-    if ((*cerr = cudaGetLastError()) != cudaSuccess) return "fp8 gather launch failed";
+    if (*cerr != cudaSuccess) return "fp8 gather launch failed";
   }
   const int per = (P + a.E - 1) / a.E;
   const int bn = per <= 16 ? 16 : 32;

@@ -94,6 +94,9 @@ __device__ __forceinline__ uint32_t sf_byte(int r, int j) { return (r % 32) * 16
 __global__ void pad_offsets_kernel(const int32_t* __restrict__ offsets, int E, int has_shared, int T, int BN,
                                    int32_t* __restrict__ prow0) {
   __shared__ int32_t rows[kMaxGroups];
+  pdl_wait();
+  pdl_trigger();
+
   const int G = E + (has_shared ? 1 : 0);
   for (int g = threadIdx.x; g < G; g += blockDim.x) {
     const int r = g < E ? offsets[g + 1] - offsets[g] : T;
@@ -118,9 +121,9 @@ __global__ void pad_offsets_kernel(const int32_t* __restrict__ offsets, int E, i
 
 // ---------------------------------------------------------------------------
 // Gather + NVFP4 quantisation of x into the padded activation rows.
-// One block per padded row (grid-strided): the row's source token is found once
-// (thread 0 searches the padded group offsets), then each warp takes 64-element
-// K blocks; lane l holds elements 2l, 2l+1.
+// One warp per padded row (grid-strided); the padded group offsets sit in
+// shared memory, lane 0 finds the row's source token, and each lane quantises
+// whole 16-element groups (two 16-byte loads -> 8 packed bytes + one scale).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) gather_quant_nvfp4_kernel(const uint16_t* __restrict__ x,
                                                                 const int32_t* __restrict__ perm,
@@ -129,44 +132,57 @@ __global__ void __launch_bounds__(256) gather_quant_nvfp4_kernel(const uint16_t*
                                                                 int has_shared, int T, int k, int d, int BN,
                                                                 uint8_t* __restrict__ xq,
                                                                 uint8_t* __restrict__ sfx) {
-  __shared__ int s_src;
+  __shared__ int32_t s_prow0[kMaxGroups + 1];
+  pdl_wait();
+  pdl_trigger();
   const int G = E + (has_shared ? 1 : 0);
-  const int rows_pad = prow0[G];
-  const int kb64 = d / 64;
+  for (int i = threadIdx.x; i <= G; i += blockDim.x) s_prow0[i] = prow0[i];
+  __syncthreads();
+  const int rows_pad = s_prow0[G];
+  const int kb64 = d / 64, ng = d / 16;
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nwarps = blockDim.x / 32;
-  for (int pr = blockIdx.x; pr < rows_pad; pr += gridDim.x) {
-    if (threadIdx.x == 0) {
-      int lo = 0, hi = G;  // prow0[lo] <= pr < prow0[hi]
+  for (int pr = blockIdx.x * nwarps + warp; pr < rows_pad; pr += gridDim.x * nwarps) {
+    int src = -1;
+    if (lane == 0) {
+      int lo = 0, hi = G;  // s_prow0[lo] <= pr < s_prow0[hi]
       while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (prow0[mid] <= pr) lo = mid; else hi = mid;
+        if (s_prow0[mid] <= pr) lo = mid; else hi = mid;
       }
-      const int local = pr - prow0[lo];
+      const int local = pr - s_prow0[lo];
       const int rows = lo < E ? offsets[lo + 1] - offsets[lo] : T;
-      s_src = local >= rows ? -1 : (lo < E ? perm[offsets[lo] + local] / k : local);
+      src = local >= rows ? -1 : (lo < E ? perm[offsets[lo] + local] / k : local);
     }
-    __syncthreads();
-    const int src = s_src;
-    __syncthreads();
-    for (int kb = warp; kb < kb64; kb += nwarps) {
-    float v0 = 0.f, v1 = 0.f;
-    if (src >= 0) {
-      const uint32_t u = *reinterpret_cast<const uint32_t*>(x + static_cast<size_t>(src) * d + kb * 64 + 2 * lane);
-      v0 = bf16_bits_to_f32(u & 0xFFFF);
-      v1 = bf16_bits_to_f32(u >> 16);
-    }
-    float amax = fmaxf(fabsf(v0), fabsf(v1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-    const uint8_t sq = f32_to_e4m3_sat(amax / 6.0f);
-    const float s = e4m3_to_f32(sq);
-    const uint8_t byte = s == 0.f ? 0 : f32x2_to_e2m1x2(v1 / s, v0 / s);
-    xq[static_cast<size_t>(pr) * (d / 2) + kb * 32 + lane] = byte;
-    if ((lane & 7) == 0) {
-      const int blk = pr / BN, r = pr % BN;
-      sfx[(static_cast<size_t>(blk) * kb64 + kb) * kSfChunk + sf_byte(r, lane / 8)] = sq;
-    }
+    src = __shfl_sync(0xffffffffu, src, 0);
+    const int blk = pr / BN, r = pr % BN;
+    for (int g16 = lane; g16 < ng; g16 += 32) {
+      float v[16];
+      if (src >= 0) {
+        const uint4* p = reinterpret_cast<const uint4*>(x + static_cast<size_t>(src) * d + g16 * 16);
+        const uint4 u0 = p[0], u1 = p[1];
+        const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          v[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFF);
+          v[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = 0.f;
+      }
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      const uint8_t sq = f32_to_e4m3_sat(amax / 6.0f);
+      const float s = e4m3_to_f32(sq);
+      uint32_t packed[2] = {0, 0};
+      if (s != 0.f) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          packed[i / 4] |= static_cast<uint32_t>(f32x2_to_e2m1x2(v[2 * i + 1] / s, v[2 * i] / s)) << (8 * (i % 4));
+      }
+      *reinterpret_cast<uint2*>(xq + static_cast<size_t>(pr) * (d / 2) + g16 * 8) = make_uint2(packed[0], packed[1]);
+      sfx[(static_cast<size_t>(blk) * kb64 + g16 / 4) * kSfChunk + sf_byte(r, g16 % 4)] = sq;
     }
   }
 }
@@ -212,7 +228,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int KB = K / kF4StageK;
   const int K64 = K / 64;
 
-  build_tile_table(offsets, E, has_shared, T, P, MT, BN, tile_start, grp_rows, grp_row0);
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 4); }
@@ -227,6 +242,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tma_prefetch_desc(&tmAsh);
     tma_prefetch_desc(&tmB);
   }
+  pdl_wait();      // the group offsets come from earlier kernels
+  pdl_trigger();
+  build_tile_table(offsets, E, has_shared, T, P, MT, BN, tile_start, grp_rows, grp_row0);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -435,10 +453,9 @@ static cudaError_t launch_nvfp4(const CUtensorMap& mA, const CUtensorMap& mAsh, 
   const int G = a.E + (a.has_shared ? 1 : 0);
   const long max_tiles = static_cast<long>((P + BN - 1) / BN + G) * (Nw / 128);
   const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
-  kern<<<grid, kTcThreads, smem, st>>>(mA, mAsh, mB, a.offsets, prow0, a.slot_of_expert, a.E, a.has_shared, a.T, P,
-                                       K, Nw, up_row0, a.pool, a.shared_bank, a.bank_bytes, wsf_off, st_off, st_idx,
-                                       act_sf, out_q, out_sf, out_bf16, stages);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st, mA, mAsh, mB, a.offsets, prow0, a.slot_of_expert,
+                    a.E, a.has_shared, a.T, P, K, Nw, up_row0, a.pool, a.shared_bank, a.bank_bytes, wsf_off, st_off,
+                    st_idx, act_sf, out_q, out_sf, out_bf16, stages);
 }
 
 const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_d_off, size_t s_t_off, uint8_t* ws,
@@ -456,14 +473,15 @@ const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_
   uint8_t* hq = sfx + al256(blocks * (a.d / 64) * kSfChunk);
   uint8_t* sfh = hq + al256(rp * (a.I / 2));
   prof_mark(FTM_K_GATHER, st, false);
-  pad_offsets_kernel<<<1, 512, 0, st>>>(a.offsets, a.E, a.has_shared, a.T, BN, prow0);
-  {
-    const int grid = static_cast<int>(rp < 148 * 16 ? rp : 148 * 16);
-    gather_quant_nvfp4_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint16_t*>(a.x), a.perm, a.offsets, prow0,
-                                                    a.E, a.has_shared, a.T, a.k, a.d, BN, xq, sfx);
+  *cerr = launch_pdl(pad_offsets_kernel, dim3(1), dim3(512), 0, st, a.offsets, a.E, a.has_shared, a.T, BN, prow0);
+  if (*cerr == cudaSuccess) {
+    const int grid = static_cast<int>(rp / 8 + 1 < 148 * 8 ? rp / 8 + 1 : 148 * 8);
+    *cerr = launch_pdl(gather_quant_nvfp4_kernel, dim3(grid), dim3(256), 0, st,
+                       reinterpret_cast<const uint16_t*>(a.x), a.perm, a.offsets, prow0, a.E, a.has_shared, a.T,
+                       a.k, a.d, BN, xq, sfx);
   }
   prof_mark(FTM_K_GATHER, st, true);
-  if ((*cerr = cudaGetLastError()) != cudaSuccess) return "nvfp4 gather launch failed";
+  if (*cerr != cudaSuccess) return "nvfp4 gather launch failed";
   CUtensorMap mA1, mAsh1, mB1, mA2, mAsh2, mB2;
   const uint64_t S = static_cast<uint64_t>(a.S);
   bool ok = make_map_f4(&mA1, a.pool + a.w_gu_off, a.d, 2ull * a.I, S, a.bank_bytes, 128) &&

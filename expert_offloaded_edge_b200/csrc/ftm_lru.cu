@@ -37,6 +37,8 @@ __global__ void __launch_bounds__(kLruThreads) lru_step_kernel(const int32_t* __
   int32_t* cand = miss_rank + E + 1;  // [S] candidate flag, later victim_of_rank
   int32_t* victim = cand + S;      // [S]
   __shared__ int32_t s_distinct, s_hits;
+  pdl_wait();
+  pdl_trigger();
 
   for (int e = threadIdx.x; e < E; e += blockDim.x) want[e] = 0;
   if (threadIdx.x == 0) { s_distinct = 0; s_hits = 0; }
@@ -133,8 +135,7 @@ cudaError_t launch_lru_step(const int32_t* ids, int P, int E, int S, int64_t ste
   cudaError_t err =
       cudaFuncSetAttribute(lru_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  lru_step_kernel<<<1, kLruThreads, smem, st>>>(ids, P, E, S, step, soe, eos, lu, ws);
-  return cudaGetLastError();
+  return launch_pdl(lru_step_kernel, dim3(1), dim3(kLruThreads), smem, st, ids, P, E, S, step, soe, eos, lu, ws);
 }
 
 cudaError_t launch_lru_restore(int E, int S, int32_t* soe, int32_t* eos, int64_t* lu, const int32_t* ws,

@@ -70,6 +70,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_single_kernel(const int3
                                                                       int32_t* __restrict__ offsets,
                                                                       int32_t* __restrict__ perm,
                                                                       int32_t* __restrict__ inv) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int32_t sm[];
   int32_t* cnt = sm;                 // [E]
   int32_t* base = cnt + E;           // [E+1]
@@ -90,6 +92,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_single_kernel(const int3
 // Large P, pass 1: per-chunk histogram hist[c][e].
 __global__ void __launch_bounds__(kPermThreads) permute_hist_kernel(const int32_t* __restrict__ ids, int P, int E,
                                                                     int32_t* __restrict__ hist) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int32_t sm[];
   for (int i = threadIdx.x; i < E; i += blockDim.x) sm[i] = 0;
   __syncthreads();
@@ -103,6 +107,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_hist_kernel(const int32_
 __global__ void __launch_bounds__(kPermThreads) permute_scan_kernel(int nchunks, int E, int32_t* __restrict__ hist,
                                                                     int32_t* __restrict__ counts,
                                                                     int32_t* __restrict__ offsets) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int32_t sm[];
   int32_t* tot = sm;          // [E]
   int32_t* off = sm + E;      // [E+1]
@@ -132,6 +138,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(const int
                                                                        const int32_t* __restrict__ hist,
                                                                        int32_t* __restrict__ perm,
                                                                        int32_t* __restrict__ inv) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int32_t sm[];
   int32_t* base = sm;            // [E]
   int32_t* wcnt = sm + E;        // [warps][E]
@@ -154,18 +162,20 @@ cudaError_t launch_permute(const int32_t* ids, int P, int E, int32_t* counts, in
     cudaError_t err = cudaFuncSetAttribute(permute_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(wsm));
     if (err != cudaSuccess) return err;
-    permute_single_kernel<<<1, kPermThreads, wsm, st>>>(ids, P, E, counts, offsets, perm, inv);
-    return cudaGetLastError();
+    return launch_pdl(permute_single_kernel, dim3(1), dim3(kPermThreads), wsm, st, ids, P, E, counts, offsets, perm,
+                      inv);
   }
   const int nchunks = (P + kChunk - 1) / kChunk;
   int32_t* hist = static_cast<int32_t*>(ws);
   cudaError_t err = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(wsm));
   if (err != cudaSuccess) return err;
-  permute_hist_kernel<<<nchunks, kPermThreads, sizeof(int32_t) * E, st>>>(ids, P, E, hist);
-  permute_scan_kernel<<<1, kPermThreads, sizeof(int32_t) * (2 * E + 1), st>>>(nchunks, E, hist, counts, offsets);
-  permute_scatter_kernel<<<nchunks, kPermThreads, wsm, st>>>(ids, P, E, hist, perm, inv);
-  return cudaGetLastError();
+  err = launch_pdl(permute_hist_kernel, dim3(nchunks), dim3(kPermThreads), sizeof(int32_t) * E, st, ids, P, E, hist);
+  if (err != cudaSuccess) return err;
+  err = launch_pdl(permute_scan_kernel, dim3(1), dim3(kPermThreads), sizeof(int32_t) * (2 * E + 1), st, nchunks, E,
+                   hist, counts, offsets);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(permute_scatter_kernel, dim3(nchunks), dim3(kPermThreads), wsm, st, ids, P, E, hist, perm, inv);
 }
 
 }  // namespace ftm

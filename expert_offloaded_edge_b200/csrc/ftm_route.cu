@@ -66,6 +66,8 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_topk_kernel(const Tin*
   const int t0 = tile * TT;
   const int nt = min(TT, T - t0);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  pdl_wait();
+  pdl_trigger();
 
   // token tile -> shared memory (rows beyond T are zero); 8 loads in flight per thread
   const int vec_per_row = d / V;
@@ -174,13 +176,15 @@ static cudaError_t launch_route_tt(const void* x, int T, int d, const void* wr, 
   cfg.blockDim = dim3(kRouteWarps * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = kRouteCluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<const Tin*>(x), T, d, static_cast<const Tin*>(wr), bias, E, k,
                             ids, w);
 }

@@ -50,6 +50,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_alloc(&tmem_holder, kTmemCols);
     tmem_relinquish();
   }
+  pdl_wait();
+  pdl_trigger();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -211,14 +213,16 @@ cudaError_t launch_route_tc(const void* x, int T, int d, const void* wr, const f
     auto kern = route_tc_kernel<1, 4>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid, kTcThreads, smem, st>>>(mW, mX, T, d, bias, E, k, ids, w);
+    e = launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st, mW, mX, T, d, bias, E, k, ids, w);
+    if (e != cudaSuccess) return e;
   } else {
     constexpr uint32_t stage = 2 * 128 * 128 + kRtBN * 128;
     const size_t smem = 1024 + 3 * stage + sizeof(float) * kRtBN * (2 * 128 + 1);
     auto kern = route_tc_kernel<2, 3>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid, kTcThreads, smem, st>>>(mW, mX, T, d, bias, E, k, ids, w);
+    e = launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st, mW, mX, T, d, bias, E, k, ids, w);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

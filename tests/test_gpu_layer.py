@@ -34,7 +34,7 @@ def test_tiny_fp32_layer():
 SMALL = synth.scaled(synth.CONFIGS["35b_decode"], name="small_bf16", d=256, I=256, E=16, k=4, S=16, T=(700,))
 
 
-@pytest.mark.parametrize("T", [1, 7, 64, 700])
+@pytest.mark.parametrize("T", [1, 7, 64, 700, 1000])
 def test_small_bf16_layer(T):
     dl = screened_layer(SMALL, T)
     _check_layer(dl, T)
