@@ -11,25 +11,28 @@ __global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ y
                                                       const float* __restrict__ gw, int T, int k, int d, int P,
                                                       int has_shared, void* __restrict__ out) {
   constexpr int V = F32 ? 4 : 8;   // elements per 16-byte vector
+  __shared__ int32_t s_row[17];
+  __shared__ float s_g[17];
   const int nv = d / V;
+  const int nterms = k + (has_shared ? 1 : 0);
   pdl_wait();
   pdl_trigger();
   for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    // the token's rows and weights first, so the row loads below are independent
+    if (threadIdx.x < nterms) {
+      const int j = threadIdx.x;
+      s_row[j] = j < k ? inv[static_cast<size_t>(t) * k + j] : P + t;
+      s_g[j] = j < k ? gw[static_cast<size_t>(t) * k + j] : 1.f;
+    }
+    __syncthreads();
     for (int c = threadIdx.x; c < nv; c += blockDim.x) {
       float acc[V];
 #pragma unroll
       for (int i = 0; i < V; ++i) acc[i] = 0.f;
-      for (int j = 0; j <= k; ++j) {
-        int row;
-        float g;
-        if (j < k) {
-          row = inv[static_cast<size_t>(t) * k + j];
-          g = gw[static_cast<size_t>(t) * k + j];
-        } else {
-          if (!has_shared) break;
-          row = P + t;
-          g = 1.f;
-        }
+#pragma unroll 4
+      for (int j = 0; j < nterms; ++j) {
+        const int row = s_row[j];
+        const float g = s_g[j];
         const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(y) +
                                                         (static_cast<size_t>(row) * d + static_cast<size_t>(c) * V) *
                                                             (F32 ? 4 : 2));
@@ -62,6 +65,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ y
       *reinterpret_cast<uint4*>(static_cast<uint8_t*>(out) +
                                 (static_cast<size_t>(t) * d + static_cast<size_t>(c) * V) * (F32 ? 4 : 2)) = o;
     }
+    __syncthreads();   // s_row / s_g are rewritten for the next token
   }
 }
 

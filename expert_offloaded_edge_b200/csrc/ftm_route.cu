@@ -193,13 +193,23 @@ bool route_tc_applicable(bool f32, int T, int E, int k);
 cudaError_t launch_route_tc(const void* x, int T, int d, const void* wr, const float* bias, int E, int k,
                             int32_t* ids, float* w, cudaStream_t st);
 
-// Large bf16 batches go to the tensor-core router; otherwise the token-tile
-// size is chosen so the x tile fits next to the logits buffer.
+// Large bf16 batches go to the tensor-core router.  Otherwise the token tile
+// is small enough that the batch spreads over ~16 clusters (each thread's dot
+// products are the latency of the kernel) and the x tile fits next to the
+// logits buffer.
 cudaError_t launch_route(bool f32, const void* x, int T, int d, const void* wr, const float* bias, int E, int k,
                          int32_t* ids, float* w, cudaStream_t st) {
   if (route_tc_applicable(f32, T, E, k)) return launch_route_tc(x, T, d, wr, bias, E, k, ids, w, st);
   const size_t elt = f32 ? 4 : 2;
   const size_t budget = 160 * 1024 - sizeof(float) * 16 * kMaxE;
+  if (T <= 32) {
+    return f32 ? launch_route_tt<float, 1>(x, T, d, wr, bias, E, k, ids, w, st)
+               : launch_route_tt<uint16_t, 1>(x, T, d, wr, bias, E, k, ids, w, st);
+  }
+  if (T <= 128 && 4 * d * elt <= budget) {
+    return f32 ? launch_route_tt<float, 4>(x, T, d, wr, bias, E, k, ids, w, st)
+               : launch_route_tt<uint16_t, 4>(x, T, d, wr, bias, E, k, ids, w, st);
+  }
   if (16 * d * elt <= budget && T >= 16) {
     return f32 ? launch_route_tt<float, 16>(x, T, d, wr, bias, E, k, ids, w, st)
                : launch_route_tt<uint16_t, 16>(x, T, d, wr, bias, E, k, ids, w, st);
