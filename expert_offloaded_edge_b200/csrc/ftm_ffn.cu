@@ -302,6 +302,9 @@ static cudaError_t launch_tc_bn(int bn, const CUtensorMap& mA, const CUtensorMap
   }
 }
 
+bool tc2_applicable(int P, int E, int I, int d);
+const char* launch_ffn_gemms_tc2(const FfnArgs& a, int rows, cudaStream_t st, cudaError_t* cerr);
+
 int ffn_token_tile(int P, int E) {
   const int per = (P + E - 1) / E;
   return per <= 16 ? 16 : per <= 32 ? 32 : per <= 64 ? 64 : 128;
@@ -338,7 +341,8 @@ const char* launch_expert_ffn(const FfnArgs& a, cudaStream_t st, cudaError_t* ce
     if (*cerr != cudaSuccess) return "simt gemm2 launch failed";
     return nullptr;
   }
-  // bf16 tensor-core path; the down projection takes 256-token tiles when groups are large
+  // bf16 tensor-core path: CTA pairs for prefill-size groups, single CTAs otherwise
+  if (tc2_applicable(P, a.E, a.I, a.d)) return launch_ffn_gemms_tc2(a, rows, st, cerr);
   const int bn = ffn_token_tile(P, a.E);
   const int bn2 = (P + a.E - 1) / a.E >= 192 ? 256 : bn;
   CUtensorMap mA1, mAsh1, mB1, mA2, mAsh2, mB2;

@@ -47,6 +47,15 @@ def test_small_bf16_layer_shared_expert_ragged_E(T):
     _check_layer(dl, T)
 
 
+@pytest.mark.parametrize("T", [900, 1537])
+def test_small_bf16_layer_pair_tiles(T):
+    # >= 192 rows per expert on average: both GEMMs run on CTA pairs (256 x 256
+    # tiles), with ragged groups, a shared expert and a partial last token tile
+    cfg = synth.scaled(SMALL, name="small_bf16_pairs", E=20, k=5, S=24, has_shared=1, I=384, d=512)
+    dl = screened_layer(cfg, T)
+    _check_layer(dl, T)
+
+
 @pytest.mark.parametrize("T", [1, 8, 32, 64])
 def test_35b_decode_layer(T):
     dl = DeviceLayer(synth.CONFIGS["35b_decode"])
