@@ -99,13 +99,14 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-KERNEL_FILES = {"bf16": "ftm_ffn.cu", "f32": "ftm_ffn.cu", "fp8": "ftm_ffn_fp8.cu", "nvfp4": "ftm_ffn_nvfp4.cu"}
+KERNEL_FILES = {"bf16": ("ftm_ffn.cu", "ftm_ffn_tc2.cu"), "f32": ("ftm_ffn.cu",), "fp8": ("ftm_ffn_fp8.cu",),
+                "nvfp4": ("ftm_ffn_nvfp4.cu",)}
 
 
 def kernel_source_hash(wdtype: str) -> str:
     """Hash of the sources the dominant kernel of a dtype is built from."""
     h = hashlib.sha256()
-    for n in (KERNEL_FILES[wdtype], "ftm_gemm.cuh", "ftm_common.cuh"):
+    for n in KERNEL_FILES[wdtype] + ("ftm_gemm.cuh", "ftm_common.cuh"):
         with open(os.path.join(ROOT, "expert_offloaded_edge_b200", "csrc", n), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

@@ -117,9 +117,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr uint32_t kAccCols = GATED ? 2 * BN : BN;
   constexpr uint32_t kTmemCols = 2 * kAccCols < 32 ? 32 : 2 * kAccCols;
   constexpr uint32_t kIdesc = idesc_bf16_f32(128, BN);
+  constexpr int kRedStride = GATED ? 36 : 20;     // floats per thread row of a split-K partial chunk
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[8], empty_bar[8], tfull_bar[2], tempty_bar[2];
+  __shared__ __align__(8) uint64_t full_bar[8], empty_bar[8], tfull_bar[2], tempty_bar[2], red_full, red_empty;
   __shared__ uint32_t tmem_holder;
   __shared__ int32_t tile_start[kMaxGroups + 1], grp_rows[kMaxGroups], grp_row0[kMaxGroups];
 
@@ -129,10 +130,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int G = E + (has_shared ? 1 : 0);
   const int MT = Nw / 128;
   const int KB = K / kBK;
+  // Split-K: a cluster of ks CTAs shares each tile, rank kr accumulating
+  // k-blocks [kb0, kb1); the other ranks hand their partial sums to rank 0
+  // through its shared memory, and rank 0 adds them in rank order (so the
+  // result does not depend on timing) and runs the epilogue.
+  const int ks = static_cast<int>(cluster_nranks());
+  const int kr = static_cast<int>(cluster_rank());
+  const int kb0 = kr * KB / ks, kb1 = (kr + 1) * KB / ks;
+  const int cl = blockIdx.x / ks, ncl = gridDim.x / ks;
+  float* red = reinterpret_cast<float*>(smem + static_cast<size_t>(stages) * kStageBytes);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 4); }
+    mbar_init(&red_full, 128 * (ks - 1 > 0 ? ks - 1 : 1));
+    mbar_init(&red_empty, 128);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -148,7 +160,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   pdl_trigger();
   build_tile_table(offsets, E, has_shared, T, P, MT, BN, tile_start, grp_rows, grp_row0);
   tc_fence_before();
-  __syncthreads();
+  if (ks > 1) cluster_sync_all();   // every rank's barriers exist before any remote arrival
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_holder;
   const int total = tile_start[G];
@@ -165,11 +178,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int t = cl; t < total && ok; t += ncl) {
         const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, BN);
         const int slot = ti.g < E ? slot_of_expert[ti.g] : 0;
         const int brow = ti.row0 + ti.n * BN;
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], kTx);
           if (ti.g < E) {
@@ -191,14 +204,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+      for (int t = cl; t < total && ok; t += ncl, ++it) {
         const int ab = it & 1;
         const uint32_t aphase = (it >> 1) & 1;
         if (!mbar_wait(&tempty_bar[ab], aphase ^ 1u)) break;
         tc_fence_after();
         const uint32_t d_g = tmem_base + ab * kAccCols;
         const uint32_t d_u = d_g + BN;
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(a_tile(stage, 0));
@@ -206,7 +219,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t bdesc = smem_desc_sw128(sb + kk * 32);
-            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            const uint32_t acc = (kb != kb0 || kk != 0) ? 1u : 0u;
             umma_f16(d_g, smem_desc_sw128(sa + kk * 32), bdesc, kIdesc, acc);
             if (GATED) umma_f16(d_u, smem_desc_sw128(sa + kATileBytes + kk * 32), bdesc, kIdesc, acc);
           }
@@ -219,22 +232,55 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else {
     const int q = warp % 4;  // TMEM lane quadrant this warp may access
+    const int er = q * 32 + lane;  // accumulator row (TMEM lane) of this thread
+    // split-K exchange: rank r > 0 writes its chunk into slot r - 1 of rank 0's buffer
+    const uint32_t red_slot = kr > 0 ? mapa_rank(smem_u32(red + ((kr - 1) * 128 + er) * kRedStride), 0) : 0u;
+    uint32_t chunk = 0;  // partial-sum chunks exchanged so far (parity of red_full / red_empty)
+    bool ok = true;
     int it = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+    for (int t = cl; t < total && ok; t += ncl, ++it) {
       const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, BN);
       const int ab = it & 1;
       const uint32_t aphase = (it >> 1) & 1;
-      if (!mbar_wait(&tfull_bar[ab], aphase)) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull_bar[ab], aphase))) break;
       tc_fence_after();
       const int valid = min(BN, ti.rows - ti.n * BN);
-      const int wrow = ti.m * 128 + q * 32 + lane;
+      const int wrow = ti.m * 128 + er;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * kAccCols;
       uint16_t* obase = out + static_cast<size_t>(ti.row0 + ti.n * BN) * ld_out + wrow;
-      for (int c0 = 0; c0 < valid; c0 += 16) {
+      for (int c0 = 0; c0 < valid; c0 += 16, ++chunk) {
         float a[16], b[16];
         tmem_ld16(tb + c0, a);
         if (GATED) tmem_ld16(tb + BN + c0, b);
         tmem_ld_wait();
+        if (ks > 1) {
+          const uint32_t ph = chunk & 1u;
+          if (kr > 0) {
+            // hand the partial chunk to rank 0 once it has consumed the previous one
+            if (!__all_sync(0xffffffffu, mbar_wait_cl(&red_empty, ph ^ 1u))) { ok = false; break; }
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) {
+              st_cluster_v4(red_slot + 4u * j, a[j], a[j + 1], a[j + 2], a[j + 3]);
+              if (GATED) st_cluster_v4(red_slot + 4u * (16 + j), b[j], b[j + 1], b[j + 2], b[j + 3]);
+            }
+            mbar_arrive_remote(mapa_rank(smem_u32(&red_full), 0));
+            continue;
+          }
+          if (!__all_sync(0xffffffffu, mbar_wait_cl(&red_full, ph))) { ok = false; break; }
+          for (int r = 1; r < ks; ++r) {
+            const float4* pr = reinterpret_cast<const float4*>(red + ((r - 1) * 128 + er) * kRedStride);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float4 u = pr[j];
+              a[4 * j] += u.x; a[4 * j + 1] += u.y; a[4 * j + 2] += u.z; a[4 * j + 3] += u.w;
+              if (GATED) {
+                const float4 w = pr[4 + j];
+                b[4 * j] += w.x; b[4 * j + 1] += w.y; b[4 * j + 2] += w.z; b[4 * j + 3] += w.w;
+              }
+            }
+          }
+          for (int r = 1; r < ks; ++r) mbar_arrive_remote(mapa_rank(smem_u32(&red_empty), static_cast<uint32_t>(r)));
+        }
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           if (c0 + j < valid) {
@@ -250,7 +296,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   }
   tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  if (ks > 1) cluster_sync_all();   // no rank leaves while another may still write to or signal it
+  else __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
 }
@@ -265,25 +313,78 @@ static bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t K, uint64_t
                         box_rows);
 }
 
+// Upper bound on the tiles of a launch, from sizes alone: at most min(E, P)
+// routed groups are non-empty and their token tiles number at most
+// min(P, ceil(P / BN) + groups); the shared expert adds ceil(T / BN).
+static long tile_bound(int P, int T, int E, int has_shared, int BN, int MT) {
+  const long groups = E < P ? E : P;
+  long routed = (P + BN - 1) / BN + groups;
+  if (routed > P) routed = P;
+  return (routed + (has_shared ? (T + BN - 1) / BN : 0)) * MT;
+}
+
+// Split-K ranks for a launch whose tiles cannot fill the GPU: the largest ks
+// <= 4 (and <= the k-blocks) with ks x tiles <= SMs.  1 = no split.
+static int split_k_ranks(long tiles, int KB) {
+  const long sms = num_sms();
+  if (tiles <= 0 || 2 * tiles > sms) return 1;
+  long ks = sms / tiles;
+  if (ks > 4) ks = 4;
+  if (ks > KB) ks = KB;
+  return ks < 1 ? 1 : static_cast<int>(ks);
+}
+
 template <int BN, bool GATED>
 static cudaError_t launch_tc(const CUtensorMap& mA, const CUtensorMap& mAsh, const CUtensorMap& mB,
                              const FfnArgs& a, int K, int Nw, int up_row0, uint16_t* out, int ld_out,
                              cudaStream_t st) {
   constexpr uint32_t kBBytes = ((BN * 128 + 1023) / 1024) * 1024;
   constexpr uint32_t kStageBytes = kATileBytes * (GATED ? 2 : 1) + kBBytes;
+  constexpr int kRedStride = GATED ? 36 : 20;
+  const int P = a.T * a.k;
+  const long tiles = tile_bound(P, a.T, a.E, a.has_shared, BN, Nw / 128);
+  const int ks = split_k_ranks(tiles, K / kBK);
+  const int red_bytes = (ks - 1) * 128 * kRedStride * 4;
   const int budget = 200 * 1024;
-  int stages = (budget - 1024) / static_cast<int>(kStageBytes);
+  int stages = (budget - 1024 - red_bytes) / static_cast<int>(kStageBytes);
   if (stages > 8) stages = 8;
-  const size_t smem = 1024 + static_cast<size_t>(stages) * kStageBytes;
+  const size_t smem = 1024 + static_cast<size_t>(stages) * kStageBytes + red_bytes;
   auto kern = ffn_tc_kernel<BN, GATED>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  const int P = a.T * a.k;
-  const int G = a.E + (a.has_shared ? 1 : 0);
-  const long max_tiles = static_cast<long>((P + BN - 1) / BN + G) * (Nw / 128);
-  const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
-  return launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st, mA, mAsh, mB, a.offsets, a.slot_of_expert, a.E,
-                    a.has_shared, a.T, P, K, Nw, up_row0, out, ld_out, stages);
+  if (ks == 1) {
+    const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
+    return launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st, mA, mAsh, mB, a.offsets, a.slot_of_expert, a.E,
+                      a.has_shared, a.T, P, K, Nw, up_row0, out, ld_out, stages);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = ks;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static int max_clusters[5] = {0, 0, 0, 0, 0};   // co-resident clusters of ks CTAs, per ks
+  if (!max_clusters[ks]) {
+    cfg.gridDim = dim3(num_sms() / ks * ks);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+      (void)cudaGetLastError();
+      n = num_sms() / ks;
+    }
+    max_clusters[ks] = n;
+  }
+  const long ncl = tiles < max_clusters[ks] ? tiles : max_clusters[ks];
+  cfg.gridDim = dim3(static_cast<unsigned>(ncl * ks));
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, mA, mAsh, mB, a.offsets, a.slot_of_expert, a.E, a.has_shared, a.T, P, K, Nw,
+                            up_row0, out, ld_out, stages);
 }
 
 template <bool GATED>
