@@ -209,7 +209,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr uint32_t kTx = kATileBytes * kNA + BN * 128 + kSfStage * (kNA + 1);
   constexpr uint32_t kAccCols = GATED ? 2 * BN : BN;
   constexpr uint32_t kSfCols = 16 * (kNA + 1);                 // 4 chunks x 4 columns per operand
-  constexpr uint32_t kUsedCols = 2 * kAccCols + kSfCols;
+  // Ring of scale-factor column sets, one per stage in flight: the copies for
+  // stage s + 1 never overwrite columns the MMAs of stage s still read, so the
+  // tensor pipe can overlap them.
+  constexpr uint32_t kSfSets = (512 - 2 * kAccCols) / kSfCols >= 4 ? 4 : (512 - 2 * kAccCols) / kSfCols;
+  static_assert(kSfSets >= 1, "TMEM budget");
+  constexpr uint32_t kUsedCols = 2 * kAccCols + kSfSets * kSfCols;
   constexpr uint32_t kTmemCols = kUsedCols <= 32 ? 32 : kUsedCols <= 64 ? 64 : kUsedCols <= 128 ? 128
                                  : kUsedCols <= 256 ? 256 : 512;
   static_assert(kUsedCols <= 512, "TMEM budget");
@@ -219,6 +224,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ __align__(8) uint64_t full_bar[8], empty_bar[8], tfull_bar[2], tempty_bar[2];
   __shared__ uint32_t tmem_holder;
   __shared__ int32_t tile_start[kMaxGroups + 1], grp_rows[kMaxGroups], grp_row0[kMaxGroups];
+  // gate/up epilogue: per warp, a 16-token x 32-row block of H transposed so a
+  // thread holds one token's 16 consecutive intermediate values (one e2m1 group)
+  __shared__ float hbuf[GATED ? 4 * 16 * 33 : 1];
 
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (smem_base - smem_u32(smem_raw));
@@ -249,7 +257,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_holder;
-  const uint32_t tmem_sf = tmem_base + 2 * kAccCols;   // SFA gate | SFA up | SFB, 16 columns each
+  const uint32_t tmem_sf0 = tmem_base + 2 * kAccCols;  // set i: SFA gate | SFA up | SFB, 16 columns each
   const int total = tile_start[G];
 
   auto a_tile = [&](int s, int which) -> uint8_t* {
@@ -301,6 +309,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
+      uint32_t sf_set = 0;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
         const int ab = it & 1;
         const uint32_t aphase = (it >> 1) & 1;
@@ -310,6 +319,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase)) { ok = false; break; }
           tc_fence_after();
+          const uint32_t tmem_sf = tmem_sf0 + sf_set * kSfCols;
+          if (++sf_set == kSfSets) sf_set = 0;
           const uint32_t sa = smem_u32(a_tile(stage, 0));
           const uint32_t sb = smem_u32(b_tile(stage));
 #pragma unroll
@@ -352,34 +363,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int wrow = ti.m * 128 + q * 32 + lane;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * kAccCols;
       if (GATED) {
+        // H = silu(gate) * up in fp32, then one e4m3 scale per 16 consecutive
+        // intermediate values of a token (amax / 6) and e2m1 codes of H / scale.
         const int prow = prow0[ti.g] + ti.n * BN;
         const int blk = prow / BN;
-        const int gidx = wrow / 16;               // 16-group along the intermediate dim
-        const int kb64 = gidx / 4, j = gidx % 4;
+        const int c = lane % 16, hh = lane / 16;          // token column and row half after the transpose
+        const int i0 = ti.m * 128 + q * 32 + hh * 16;     // first intermediate index of this thread's group
+        const int gidx = i0 / 16, kb64 = gidx / 4, j = gidx % 4;
+        float* hw = hbuf + q * (16 * 33);
         for (int c0 = 0; c0 < BN; c0 += 16) {
           float a[16], b[16];
           tmem_ld16(tb + c0, a);
           tmem_ld16(tb + BN + c0, b);
           tmem_ld_wait();
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const int c = c0 + jj;
-            // padding columns are quantised too (their rows are never read back)
-            const float h = silu(a[jj] * s_a) * (b[jj] * s_u);
-            float amax = fabsf(h);
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 8));
-            const uint8_t sq = f32_to_e4m3_sat(amax / 6.0f);
-            const float s = e4m3_to_f32(sq);
-            const float hv = s == 0.f ? 0.f : h / s;
-            const float hodd = __shfl_down_sync(0xffffffffu, hv, 1);
-            if ((lane & 1) == 0)
-              out_q[static_cast<size_t>(prow + c) * (Nw / 2) + wrow / 2] = s == 0.f ? 0 : f32x2_to_e2m1x2(hodd, hv);
-            if ((lane & 15) == 0)
-              out_sf[(static_cast<size_t>(blk) * (Nw / 64) + kb64) * kSfChunk + sf_byte(c, j)] = sq;
+          for (int jj = 0; jj < 16; ++jj) hw[jj * 33 + lane] = silu(a[jj] * s_a) * (b[jj] * s_u);
+          __syncwarp();
+          float v[16];
+          float amax = 0.f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            v[i] = hw[c * 33 + hh * 16 + i];
+            amax = fmaxf(amax, fabsf(v[i]));
           }
+          __syncwarp();   // hbuf is rewritten by the next chunk
+          // padding columns are quantised too (their rows are never read back)
+          const uint8_t sq = f32_to_e4m3_sat(amax / 6.0f);
+          const float sc = e4m3_to_f32(sq);
+          uint32_t packed[2] = {0u, 0u};
+          if (sc != 0.f) {
+#pragma unroll
+            for (int i = 0; i < 16; i += 2)
+              packed[i / 8] |= static_cast<uint32_t>(f32x2_to_e2m1x2(v[i + 1] / sc, v[i] / sc)) << (4 * (i % 8));
+          }
+          *reinterpret_cast<uint2*>(out_q + static_cast<size_t>(prow + c0 + c) * (Nw / 2) + i0 / 2) =
+              make_uint2(packed[0], packed[1]);
+          out_sf[(static_cast<size_t>(blk) * (Nw / 64) + kb64) * kSfChunk + sf_byte(c0 + c, j)] = sq;
         }
       } else {
         uint16_t* obase = out_bf16 + static_cast<size_t>(ti.row0 + ti.n * BN) * Nw + wrow;
