@@ -88,6 +88,11 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 
 __device__ __forceinline__ uint32_t sf_byte(int r, int j) { return (r % 32) * 16 + (r / 32) * 4 + j; }
 
+// 128-row A tiles per stage: narrow gate/up token tiles take two paired blocks
+// (128 intermediate indices) so a stage still streams 32 KB of weights per
+// 4 KB of activations; 128-token tiles take one (the TMEM budget).
+__host__ __device__ constexpr int nvfp4_a_tiles(int BN, bool gated) { return gated && BN <= 64 ? 2 : 1; }
+
 // ---------------------------------------------------------------------------
 // Padded row offsets: prow0[g] = sum_{g' < g} roundup(rows_g', BN), g = 0..G.
 // ---------------------------------------------------------------------------
@@ -193,6 +198,14 @@ __global__ void __launch_bounds__(256) gather_quant_nvfp4_kernel(const uint16_t*
 //   weight scale chunks at bank + wsf_off; per-tensor scales at bank + st_off
 //   B: packed e2m1 activations {K bytes, rows_pad}, scale chunks act_sf
 //   GATED: out_q (e2m1 H [rows_pad][Nw/2]) + out_sf (chunks); else out_bf16 [rows][Nw]
+//
+// Every stage holds NP 128-row A tiles (nvfp4_a_tiles), so each 64-deep K step
+// is NP MMAs of M = 128 x N = BN.  Gate/up GEMM: an A tile is 64 gate rows and the same 64
+// up rows (two 64-row boxes), matching the paired order of the gate/up scale
+// chunks, so the accumulator's lane i and lane i + 64 hold gate and up of one
+// intermediate index; the epilogue pairs them across warps through shared
+// memory, applies the per-tensor scales and SwiGLU, then transposes H so each
+// thread quantises one token's 16 consecutive intermediate values.
 // ---------------------------------------------------------------------------
 template <int BN, bool GATED>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -204,35 +217,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                      int st_idx, const uint8_t* __restrict__ act_sf, uint8_t* __restrict__ out_q,
                      uint8_t* __restrict__ out_sf, uint16_t* __restrict__ out_bf16, int stages) {
   constexpr uint32_t kBBytes = ((BN * 128 + 1023) / 1024) * 1024;
-  constexpr uint32_t kNA = GATED ? 2 : 1;
-  constexpr uint32_t kStageBytes = kATileBytes * kNA + kBBytes + kSfStage * (kNA + 1);
-  constexpr uint32_t kTx = kATileBytes * kNA + BN * 128 + kSfStage * (kNA + 1);
-  constexpr uint32_t kAccCols = GATED ? 2 * BN : BN;
-  constexpr uint32_t kSfCols = 16 * (kNA + 1);                 // 4 chunks x 4 columns per operand
+  constexpr int NP = nvfp4_a_tiles(BN, GATED);     // 128-row A tiles per stage, one accumulator each
+  constexpr uint32_t kStageBytes = NP * kATileBytes + kBBytes + (NP + 1) * kSfStage;
+  constexpr uint32_t kTx = NP * kATileBytes + BN * 128 + (NP + 1) * kSfStage;
+  constexpr uint32_t kAccCols = NP * BN;
+  constexpr uint32_t kSfCols = 16 * (NP + 1);      // SFA per A tile | SFB: 4 chunks x 4 columns each
   // Ring of scale-factor column sets, one per stage in flight: the copies for
-  // stage s + 1 never overwrite columns the MMAs of stage s still read, so the
-  // tensor pipe can overlap them.
-  constexpr uint32_t kSfSets = (512 - 2 * kAccCols) / kSfCols >= 4 ? 4 : (512 - 2 * kAccCols) / kSfCols;
-  static_assert(kSfSets >= 1, "TMEM budget");
+  // stage s + 1 never overwrite columns the MMAs of stage s still read.
+  constexpr uint32_t kSfSets = 4;
   constexpr uint32_t kUsedCols = 2 * kAccCols + kSfSets * kSfCols;
-  constexpr uint32_t kTmemCols = kUsedCols <= 32 ? 32 : kUsedCols <= 64 ? 64 : kUsedCols <= 128 ? 128
-                                 : kUsedCols <= 256 ? 256 : 512;
   static_assert(kUsedCols <= 512, "TMEM budget");
+  constexpr uint32_t kTmemCols = kUsedCols <= 256 ? 256 : 512;
   constexpr uint32_t kIdesc = idesc_nvf4(128, BN);
+  constexpr int kRowsPerTile = (GATED ? 64 : 128) * NP;   // output rows (intermediate / hidden) per tile
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[8], empty_bar[8], tfull_bar[2], tempty_bar[2];
   __shared__ uint32_t tmem_holder;
   __shared__ int32_t tile_start[kMaxGroups + 1], grp_rows[kMaxGroups], grp_row0[kMaxGroups];
-  // gate/up epilogue: per warp, a 16-token x 32-row block of H transposed so a
-  // thread holds one token's 16 consecutive intermediate values (one e2m1 group)
-  __shared__ float hbuf[GATED ? 4 * 16 * 33 : 1];
+  // gate/up epilogue: half-chunks crossing between gate and up warps, and a
+  // 32-token x 64-intermediate block of H (16-groups padded to 17 floats)
+  __shared__ float xbuf[GATED ? 128 * 17 : 1];
+  __shared__ float tbuf[GATED ? 32 * 68 : 1];
 
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (smem_base - smem_u32(smem_raw));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int G = E + (has_shared ? 1 : 0);
-  const int MT = Nw / 128;
+  const int MT = Nw / kRowsPerTile;
   const int KB = K / kF4StageK;
   const int K64 = K / 64;
 
@@ -257,15 +269,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_holder;
-  const uint32_t tmem_sf0 = tmem_base + 2 * kAccCols;  // set i: SFA gate | SFA up | SFB, 16 columns each
+  const uint32_t tmem_sf0 = tmem_base + 2 * kAccCols;
   const int total = tile_start[G];
 
-  auto a_tile = [&](int s, int which) -> uint8_t* {
-    return smem + static_cast<size_t>(s) * kStageBytes + which * kATileBytes;
+  auto a_tile = [&](int s, int p) -> uint8_t* {
+    return smem + static_cast<size_t>(s) * kStageBytes + p * kATileBytes;
   };
-  auto b_tile = [&](int s) -> uint8_t* { return smem + static_cast<size_t>(s) * kStageBytes + kATileBytes * kNA; };
-  auto sf_tile = [&](int s, int which) -> uint8_t* {   // which: 0 gate, 1 up, kNA = activations
-    return smem + static_cast<size_t>(s) * kStageBytes + kATileBytes * kNA + kBBytes + which * kSfStage;
+  auto b_tile = [&](int s) -> uint8_t* { return smem + static_cast<size_t>(s) * kStageBytes + NP * kATileBytes; };
+  auto sf_tile = [&](int s, int which) -> uint8_t* {   // which: p < NP weights of A tile p, NP activations
+    return smem + static_cast<size_t>(s) * kStageBytes + NP * kATileBytes + kBBytes + which * kSfStage;
   };
 
   if (warp == 0) {
@@ -277,27 +289,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, BN);
         const int slot = ti.g < E ? slot_of_expert[ti.g] : 0;
         const uint8_t* bank = ti.g < E ? pool + static_cast<size_t>(slot) * bank_bytes : shared_bank;
-        const uint8_t* wsf = bank + wsf_off;
+        const uint8_t* wsf = bank + wsf_off + static_cast<size_t>(ti.m) * NP * K64 * kSfChunk;
         const int prow = prow0[ti.g] + ti.n * BN;
         const uint8_t* asf = act_sf + static_cast<size_t>(prow / BN) * K64 * kSfChunk;
+        const int r0 = ti.m * kRowsPerTile;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], kTx);
           const int kc = kb * (kF4StageK / 2);   // byte coordinate along K
-          if (ti.g < E) {
-            tma_load_3d(a_tile(stage, 0), &tmA, &full_bar[stage], kc, ti.m * 128, slot);
-            if (GATED) tma_load_3d(a_tile(stage, 1), &tmA, &full_bar[stage], kc, up_row0 + ti.m * 128, slot);
-          } else {
-            tma_load_2d(a_tile(stage, 0), &tmAsh, &full_bar[stage], kc, ti.m * 128);
-            if (GATED) tma_load_2d(a_tile(stage, 1), &tmAsh, &full_bar[stage], kc, up_row0 + ti.m * 128);
+#pragma unroll
+          for (int p = 0; p < NP; ++p) {
+            // gate/up: tile p is the paired block of 64 gate rows and the same 64 up rows
+            const int rp = r0 + p * (GATED ? 64 : 128);
+            if (ti.g < E) {
+              tma_load_3d(a_tile(stage, p), &tmA, &full_bar[stage], kc, rp, slot);
+              if (GATED)
+                tma_load_3d(a_tile(stage, p) + kATileBytes / 2, &tmA, &full_bar[stage], kc, up_row0 + rp, slot);
+            } else {
+              tma_load_2d(a_tile(stage, p), &tmAsh, &full_bar[stage], kc, rp);
+              if (GATED) tma_load_2d(a_tile(stage, p) + kATileBytes / 2, &tmAsh, &full_bar[stage], kc, up_row0 + rp);
+            }
+            bulk_load(sf_tile(stage, p), wsf + (static_cast<size_t>(p) * K64 + 4 * kb) * kSfChunk, kSfStage,
+                      &full_bar[stage]);
           }
           tma_load_2d(b_tile(stage), &tmB, &full_bar[stage], kc, prow);
-          bulk_load(sf_tile(stage, 0), wsf + (static_cast<size_t>(ti.m) * K64 + 4 * kb) * kSfChunk, kSfStage,
-                    &full_bar[stage]);
-          if (GATED)
-            bulk_load(sf_tile(stage, 1), wsf + (static_cast<size_t>(up_row0 / 128 + ti.m) * K64 + 4 * kb) * kSfChunk,
-                      kSfStage, &full_bar[stage]);
-          bulk_load(sf_tile(stage, kNA), asf + static_cast<size_t>(4 * kb) * kSfChunk, kSfStage, &full_bar[stage]);
+          bulk_load(sf_tile(stage, NP), asf + static_cast<size_t>(4 * kb) * kSfChunk, kSfStage, &full_bar[stage]);
           if (++stage == stages) { stage = 0; phase ^= 1u; }
         }
       }
@@ -315,29 +331,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t aphase = (it >> 1) & 1;
         if (!mbar_wait(&tempty_bar[ab], aphase ^ 1u)) break;
         tc_fence_after();
-        const uint32_t d_g = tmem_base + ab * kAccCols;
+        const uint32_t d = tmem_base + ab * kAccCols;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase)) { ok = false; break; }
           tc_fence_after();
           const uint32_t tmem_sf = tmem_sf0 + sf_set * kSfCols;
           if (++sf_set == kSfSets) sf_set = 0;
-          const uint32_t sa = smem_u32(a_tile(stage, 0));
           const uint32_t sb = smem_u32(b_tile(stage));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            tmem_cp_sf(tmem_sf + 4 * kk, smem_desc_sf(smem_u32(sf_tile(stage, 0)) + kk * kSfChunk));
-            if (GATED) tmem_cp_sf(tmem_sf + 16 + 4 * kk, smem_desc_sf(smem_u32(sf_tile(stage, 1)) + kk * kSfChunk));
-            tmem_cp_sf(tmem_sf + 16 * kNA + 4 * kk, smem_desc_sf(smem_u32(sf_tile(stage, kNA)) + kk * kSfChunk));
+#pragma unroll
+            for (int p = 0; p <= NP; ++p)
+              tmem_cp_sf(tmem_sf + 16 * p + 4 * kk, smem_desc_sf(smem_u32(sf_tile(stage, p)) + kk * kSfChunk));
           }
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bdesc = smem_desc_sw128(sb + kk * 32);
-            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
-            umma_nvf4(d_g, smem_desc_sw128(sa + kk * 32), bdesc, kIdesc, tmem_sf + 4 * kk,
-                      tmem_sf + 16 * kNA + 4 * kk, acc);
-            if (GATED)
-              umma_nvf4(d_g + BN, smem_desc_sw128(sa + kATileBytes + kk * 32), bdesc, kIdesc, tmem_sf + 16 + 4 * kk,
-                        tmem_sf + 16 * kNA + 4 * kk, acc);
+#pragma unroll
+            for (int p = 0; p < NP; ++p)
+              umma_nvf4(d + p * BN, smem_desc_sw128(smem_u32(a_tile(stage, p)) + kk * 32), smem_desc_sw128(sb + kk * 32),
+                        kIdesc, tmem_sf + 16 * p + 4 * kk, tmem_sf + 16 * NP + 4 * kk, (kb | kk) != 0 ? 1u : 0u);
           }
           umma_commit(&empty_bar[stage]);
           if (++stage == stages) { stage = 0; phase ^= 1u; }
@@ -353,54 +365,68 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, BN);
       const int ab = it & 1;
       const uint32_t aphase = (it >> 1) & 1;
-      if (!mbar_wait(&tfull_bar[ab], aphase)) break;
+      if (!epilogue_all(mbar_wait(&tfull_bar[ab], aphase))) break;
       tc_fence_after();
       const int valid = min(BN, ti.rows - ti.n * BN);
       const uint8_t* bank = ti.g < E ? pool + static_cast<size_t>(slot_of_expert[ti.g]) * bank_bytes : shared_bank;
       const float* st = reinterpret_cast<const float*>(bank + st_off);
-      const float s_a = st[st_idx];
-      const float s_u = GATED ? st[st_idx + 1] : 0.f;
-      const int wrow = ti.m * 128 + q * 32 + lane;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * kAccCols;
       if (GATED) {
-        // H = silu(gate) * up in fp32, then one e4m3 scale per 16 consecutive
-        // intermediate values of a token (amax / 6) and e2m1 codes of H / scale.
+        // H = silu(s_gate * gate) * (s_up * up) in fp32, then per token one e4m3
+        // scale per 16 consecutive intermediate values (amax / 6) and e2m1
+        // codes of H / scale.  Padding columns are quantised too (their rows
+        // are never read back).
+        const bool gate_warp = q < 2;
+        const float s_row = st[st_idx + (gate_warp ? 0 : 1)];
+        const int me = q * 32 + lane, partner = (q ^ 2) * 32 + lane;
+        const int il = (q % 2) * 32 + lane;               // intermediate index within the tile
+        const int col_off = gate_warp ? 0 : 16;           // the 16 columns of a chunk this warp evaluates
+        const int tslot = (il / 16) * 17 + il % 16;
         const int prow = prow0[ti.g] + ti.n * BN;
         const int blk = prow / BN;
-        const int c = lane % 16, hh = lane / 16;          // token column and row half after the transpose
-        const int i0 = ti.m * 128 + q * 32 + hh * 16;     // first intermediate index of this thread's group
-        const int gidx = i0 / 16, kb64 = gidx / 4, j = gidx % 4;
-        float* hw = hbuf + q * (16 * 33);
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          float a[16], b[16];
-          tmem_ld16(tb + c0, a);
-          tmem_ld16(tb + BN + c0, b);
-          tmem_ld_wait();
+        const int tok = me >> 2, grp = me & 3;            // quantisation: one (token, 16-group) per thread
+        for (int p = 0; p < NP; ++p) {   // accumulator p = paired block mb of 64 intermediate indices
+          const int mb = ti.m * NP + p;
+          for (int c0 = 0; c0 < BN; c0 += 32) {
+            float v[32];
+            tmem_ld16(tb + p * BN + c0, v);
+            tmem_ld16(tb + p * BN + c0 + 16, v + 16);
+            tmem_ld_wait();
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) hw[jj * 33 + lane] = silu(a[jj] * s_a) * (b[jj] * s_u);
-          __syncwarp();
-          float v[16];
-          float amax = 0.f;
+            for (int j = 0; j < 32; ++j) v[j] *= s_row;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            v[i] = hw[c * 33 + hh * 16 + i];
-            amax = fmaxf(amax, fabsf(v[i]));
+            for (int j = 0; j < 16; ++j) xbuf[me * 17 + j] = gate_warp ? v[16 + j] : v[j];
+            epilogue_bar();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float other = xbuf[partner * 17 + j];
+              tbuf[(col_off + j) * 68 + tslot] = gate_warp ? silu(v[j]) * other : silu(other) * v[16 + j];
+            }
+            epilogue_bar();
+            float h[16];
+            float amax = 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              h[i] = tbuf[tok * 68 + grp * 17 + i];
+              amax = fmaxf(amax, fabsf(h[i]));
+            }
+            const uint8_t sq = f32_to_e4m3_sat(amax / 6.0f);
+            const float sc = e4m3_to_f32(sq);
+            uint32_t packed[2] = {0u, 0u};
+            if (sc != 0.f) {
+#pragma unroll
+              for (int i = 0; i < 16; i += 2)
+                packed[i / 8] |= static_cast<uint32_t>(f32x2_to_e2m1x2(h[i + 1] / sc, h[i] / sc)) << (4 * (i % 8));
+            }
+            const int i0 = mb * 64 + grp * 16;
+            *reinterpret_cast<uint2*>(out_q + static_cast<size_t>(prow + c0 + tok) * (Nw / 2) + i0 / 2) =
+                make_uint2(packed[0], packed[1]);
+            out_sf[(static_cast<size_t>(blk) * (Nw / 64) + mb) * kSfChunk + sf_byte(c0 + tok, grp)] = sq;
           }
-          __syncwarp();   // hbuf is rewritten by the next chunk
-          // padding columns are quantised too (their rows are never read back)
-          const uint8_t sq = f32_to_e4m3_sat(amax / 6.0f);
-          const float sc = e4m3_to_f32(sq);
-          uint32_t packed[2] = {0u, 0u};
-          if (sc != 0.f) {
-#pragma unroll
-            for (int i = 0; i < 16; i += 2)
-              packed[i / 8] |= static_cast<uint32_t>(f32x2_to_e2m1x2(v[i + 1] / sc, v[i] / sc)) << (4 * (i % 8));
-          }
-          *reinterpret_cast<uint2*>(out_q + static_cast<size_t>(prow + c0 + c) * (Nw / 2) + i0 / 2) =
-              make_uint2(packed[0], packed[1]);
-          out_sf[(static_cast<size_t>(blk) * (Nw / 64) + kb64) * kSfChunk + sf_byte(c0 + c, j)] = sq;
         }
       } else {
+        const float s_a = st[st_idx];
+        const int wrow = ti.m * 128 + q * 32 + lane;
         uint16_t* obase = out_bf16 + static_cast<size_t>(ti.row0 + ti.n * BN) * Nw + wrow;
         for (int c0 = 0; c0 < valid; c0 += 16) {
           float a[16];
@@ -435,7 +461,12 @@ static bool make_map_f4(CUtensorMap* m, const void* base, uint64_t K, uint64_t r
   return make_map_sw128(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, K / 2, rows, K / 2, slots, slot_pitch, box_rows);
 }
 
-int nvfp4_token_tile(int P, int E) { return (P + E - 1) / E <= 32 ? 32 : 64; }
+// Token tile: the smallest of 32 / 64 / 128 that holds an average group, so
+// decode batches pad little and prefill batches get wide MMAs.
+int nvfp4_token_tile(int P, int E) {
+  const int avg = (P + E - 1) / E;
+  return avg <= 32 ? 32 : avg <= 96 ? 64 : 128;
+}
 
 static size_t al256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 
@@ -447,7 +478,7 @@ static int64_t nvfp4_rows_pad(int64_t P, int T, int G, int has_shared, int BN) {
 // Workspace: prow0 | Xq [rows_pad][d/2] | SFx chunks | Hq [rows_pad][I/2] | SFh chunks
 size_t nvfp4_ffn_workspace_bytes(int64_t P, int T, int E, int has_shared, int d, int I) {
   const int G = E + (has_shared ? 1 : 0);
-  const int BN = 64;   // the larger tile bounds both
+  const int BN = 128;   // the largest tile bounds all
   const int64_t rp = nvfp4_rows_pad(P, T, G, has_shared, BN);
   const int64_t blocks = rp / 32 + G + 1;   // chunks are per BN-row block; BN >= 32
   return al256(sizeof(int32_t) * (G + 1)) + al256(rp * (d / 2)) + al256(blocks * (d / 64) * kSfChunk) +
@@ -460,8 +491,8 @@ static cudaError_t launch_nvfp4(const CUtensorMap& mA, const CUtensorMap& mAsh, 
                                 size_t st_off, int st_idx, const uint8_t* act_sf, uint8_t* out_q, uint8_t* out_sf,
                                 uint16_t* out_bf16, cudaStream_t st) {
   constexpr uint32_t kBBytes = ((BN * 128 + 1023) / 1024) * 1024;
-  constexpr uint32_t kNA = GATED ? 2 : 1;
-  constexpr uint32_t kStageBytes = kATileBytes * kNA + kBBytes + kSfStage * (kNA + 1);
+  constexpr int NP = nvfp4_a_tiles(BN, GATED);
+  constexpr uint32_t kStageBytes = NP * kATileBytes + kBBytes + (NP + 1) * kSfStage;
   int stages = (200 * 1024 - 1024) / static_cast<int>(kStageBytes);
   if (stages > 8) stages = 8;
   const size_t smem = 1024 + static_cast<size_t>(stages) * kStageBytes;
@@ -470,7 +501,7 @@ static cudaError_t launch_nvfp4(const CUtensorMap& mA, const CUtensorMap& mAsh, 
   if (err != cudaSuccess) return err;
   const int P = a.T * a.k;
   const int G = a.E + (a.has_shared ? 1 : 0);
-  const long max_tiles = static_cast<long>((P + BN - 1) / BN + G) * (Nw / 128);
+  const long max_tiles = static_cast<long>((P + BN - 1) / BN + G) * (Nw / ((GATED ? 64 : 128) * NP));
   const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
   return launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st, mA, mAsh, mB, a.offsets, prow0, a.slot_of_expert,
                     a.E, a.has_shared, a.T, P, K, Nw, up_row0, a.pool, a.shared_bank, a.bank_bytes, wsf_off, st_off,
@@ -484,7 +515,7 @@ const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_
   *cerr = cudaSuccess;
   if (P + (a.has_shared ? a.T : 0) == 0) return nullptr;
   const int BN = nvfp4_token_tile(P, a.E);
-  const int64_t rp = nvfp4_rows_pad(P, a.T, G, a.has_shared, 64);
+  const int64_t rp = nvfp4_rows_pad(P, a.T, G, a.has_shared, 128);
   const int64_t blocks = rp / 32 + G + 1;
   int32_t* prow0 = reinterpret_cast<int32_t*>(ws);
   uint8_t* xq = ws + al256(sizeof(int32_t) * (G + 1));
@@ -503,12 +534,13 @@ const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_
   if (*cerr != cudaSuccess) return "nvfp4 gather launch failed";
   CUtensorMap mA1, mAsh1, mB1, mA2, mAsh2, mB2;
   const uint64_t S = static_cast<uint64_t>(a.S);
-  bool ok = make_map_f4(&mA1, a.pool + a.w_gu_off, a.d, 2ull * a.I, S, a.bank_bytes, 128) &&
+  // gate/up boxes are 64 rows: a tile stages 64 gate rows and the same 64 up rows
+  bool ok = make_map_f4(&mA1, a.pool + a.w_gu_off, a.d, 2ull * a.I, S, a.bank_bytes, 64) &&
             make_map_f4(&mA2, a.pool + a.w_d_off, a.I, a.d, S, a.bank_bytes, 128) &&
             make_map_f4(&mB1, xq, a.d, static_cast<uint64_t>(rp), 0, 0, BN) &&
             make_map_f4(&mB2, hq, a.I, static_cast<uint64_t>(rp), 0, 0, BN);
   if (ok && a.has_shared) {
-    ok = make_map_f4(&mAsh1, a.shared_bank + a.w_gu_off, a.d, 2ull * a.I, 0, 0, 128) &&
+    ok = make_map_f4(&mAsh1, a.shared_bank + a.w_gu_off, a.d, 2ull * a.I, 0, 0, 64) &&
          make_map_f4(&mAsh2, a.shared_bank + a.w_d_off, a.I, a.d, 0, 0, 128);
   } else {
     mAsh1 = mA1;
@@ -518,15 +550,20 @@ const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_
   prof_mark(FTM_K_GEMM1, st, false);
   *cerr = BN == 32 ? launch_nvfp4<32, true>(mA1, mAsh1, mB1, a, prow0, a.d, a.I, a.I, s_gu_off, s_t_off, 0, sfx, hq,
                                             sfh, nullptr, st)
-                   : launch_nvfp4<64, true>(mA1, mAsh1, mB1, a, prow0, a.d, a.I, a.I, s_gu_off, s_t_off, 0, sfx, hq,
-                                            sfh, nullptr, st);
+          : BN == 64 ? launch_nvfp4<64, true>(mA1, mAsh1, mB1, a, prow0, a.d, a.I, a.I, s_gu_off, s_t_off, 0, sfx, hq,
+                                              sfh, nullptr, st)
+                     : launch_nvfp4<128, true>(mA1, mAsh1, mB1, a, prow0, a.d, a.I, a.I, s_gu_off, s_t_off, 0, sfx,
+                                               hq, sfh, nullptr, st);
   prof_mark(FTM_K_GEMM1, st, true);
   if (*cerr != cudaSuccess) return "nvfp4 gemm1 launch failed";
   prof_mark(FTM_K_GEMM2, st, false);
+  uint16_t* y = reinterpret_cast<uint16_t*>(a.y);
   *cerr = BN == 32 ? launch_nvfp4<32, false>(mA2, mAsh2, mB2, a, prow0, a.I, a.d, 0, s_d_off, s_t_off, 2, sfh,
-                                             nullptr, nullptr, reinterpret_cast<uint16_t*>(a.y), st)
-                   : launch_nvfp4<64, false>(mA2, mAsh2, mB2, a, prow0, a.I, a.d, 0, s_d_off, s_t_off, 2, sfh,
-                                             nullptr, nullptr, reinterpret_cast<uint16_t*>(a.y), st);
+                                             nullptr, nullptr, y, st)
+          : BN == 64 ? launch_nvfp4<64, false>(mA2, mAsh2, mB2, a, prow0, a.I, a.d, 0, s_d_off, s_t_off, 2, sfh,
+                                               nullptr, nullptr, y, st)
+                     : launch_nvfp4<128, false>(mA2, mAsh2, mB2, a, prow0, a.I, a.d, 0, s_d_off, s_t_off, 2, sfh,
+                                                nullptr, nullptr, y, st);
   prof_mark(FTM_K_GEMM2, st, true);
   if (*cerr != cudaSuccess) return "nvfp4 gemm2 launch failed";
   return nullptr;

@@ -21,6 +21,16 @@ def nvfp4_scale_chunks(s16: np.ndarray) -> np.ndarray:
     return np.ascontiguousarray(a.transpose(0, 3, 2, 1, 4)).ravel()
 
 
+def gate_up_paired_rows(gate: np.ndarray, up: np.ndarray) -> np.ndarray:
+    """[I][C] gate and up rows -> [2I][C] in paired order: 64 gate rows, then
+    the same 64 up rows, and so on (the row order of the NVFP4 gate/up scale
+    chunks, so one 128-row chunk covers the gate and up rows of 64 intermediate
+    indices)."""
+    I, C = gate.shape
+    assert up.shape == (I, C) and I % 64 == 0
+    return np.stack([gate.reshape(I // 64, 64, C), up.reshape(I // 64, 64, C)], axis=1).reshape(2 * I, C)
+
+
 def _put(bank: np.ndarray, off: int, arr: np.ndarray, nbytes: int):
     b = np.ascontiguousarray(arr).view(np.uint8).ravel()
     assert b.size == nbytes, (b.size, nbytes)
@@ -46,7 +56,7 @@ def pack_bank(desc: LayerDesc, ew, bl: BankLayout = None, out: np.ndarray = None
     elif w == FTM_NVFP4:
         _put(bank, bl.w_gu_off, np.concatenate([ew.gate[0], ew.up[0]], axis=0), bl.w_gu_bytes)
         _put(bank, bl.w_d_off, ew.down[0], bl.w_d_bytes)
-        _put(bank, bl.s_gu_off, nvfp4_scale_chunks(np.concatenate([ew.gate[1], ew.up[1]], axis=0)), bl.s_gu_bytes)
+        _put(bank, bl.s_gu_off, nvfp4_scale_chunks(gate_up_paired_rows(ew.gate[1], ew.up[1])), bl.s_gu_bytes)
         _put(bank, bl.s_d_off, nvfp4_scale_chunks(ew.down[1]), bl.s_d_bytes)
         _put(bank, bl.s_t_off, np.array([ew.gate[2], ew.up[2], ew.down[2], 0.0], dtype=np.float32), bl.s_t_bytes)
     else:

@@ -80,7 +80,9 @@ typedef struct ftm_layer_desc {
  *         (f32 / bf16 / e4m3 elements; NVFP4: [2I][d/2] bytes, two codes per
  *         byte, element 2j in the low nibble)
  *   w_d : [d][I] row-major (same element rules)
- *   s_gu: FP8: fp32 [2I/128][d/128]; NVFP4: the 2I x d/16 e4m3 scales in chunks (below)
+ *   s_gu: FP8: fp32 [2I/128][d/128]; NVFP4: the 2I x d/16 e4m3 scales in chunks (below),
+ *         rows taken in paired order: gate rows 64b..64b+63 then up rows
+ *         64b..64b+63 for b = 0..I/64-1 (chunk row block rb = b)
  *   s_d : FP8: fp32 [d/128][I/128];  NVFP4: the d x I/16 e4m3 scales in chunks
  *   s_t : NVFP4: fp32[4] = {gate, up, down, 0} per-tensor scales; else empty
  * NVFP4 scale chunks (the layout the block-scaled MMA reads): one 512-byte

@@ -91,3 +91,17 @@ def test_nvfp4_scale_chunk_packing_brute_force():
             rb, kb, rl, j = r // 128, g // 4, r % 128, g % 4
             off = (rb * (G16 // 4) + kb) * 512 + (rl % 32) * 16 + (rl // 32) * 4 + j
             assert packed[off] == s16[r, g]
+
+
+def test_gate_up_paired_rows_brute_force():
+    from expert_offloaded_edge_b200.layout import gate_up_paired_rows
+    rng = np.random.default_rng(1)
+    I, C = 192, 5
+    gate = rng.integers(0, 256, size=(I, C), dtype=np.uint8)
+    up = rng.integers(0, 256, size=(I, C), dtype=np.uint8)
+    paired = gate_up_paired_rows(gate, up)
+    assert paired.shape == (2 * I, C)
+    for r in range(2 * I):
+        b, rl = r // 128, r % 128
+        want = gate[64 * b + rl] if rl < 64 else up[64 * b + rl - 64]
+        assert (paired[r] == want).all()

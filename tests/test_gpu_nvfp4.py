@@ -25,7 +25,7 @@ def _check(dl, T, rows=None):
     return out, x, ids, g, rows, worst
 
 
-@pytest.mark.parametrize("T", [1, 20, 300])
+@pytest.mark.parametrize("T", [1, 20, 300, 700])   # token tiles of 32, 32, 64 and 128 rows
 def test_small_nvfp4_layer(T):
     dl = screened_layer(SMALL_FP4, T)
     out, x, ids, g, rows, worst = _check(dl, T)
