@@ -159,6 +159,7 @@ __global__ void __launch_bounds__(256) gather_quant_nvfp4_kernel(const uint16_t*
       src = local >= rows ? -1 : (lo < E ? perm[offsets[lo] + local] / k : local);
     }
     src = __shfl_sync(0xffffffffu, src, 0);
+    const int nsub = (BN + 127) / 128;   // 128-row scale chunks per BN-row block
     const int blk = pr / BN, r = pr % BN;
     for (int g16 = lane; g16 < ng; g16 += 32) {
       float v[16];
@@ -187,7 +188,7 @@ __global__ void __launch_bounds__(256) gather_quant_nvfp4_kernel(const uint16_t*
           packed[i / 4] |= static_cast<uint32_t>(f32x2_to_e2m1x2(v[2 * i + 1] / s, v[2 * i] / s)) << (8 * (i % 4));
       }
       *reinterpret_cast<uint2*>(xq + static_cast<size_t>(pr) * (d / 2) + g16 * 8) = make_uint2(packed[0], packed[1]);
-      sfx[(static_cast<size_t>(blk) * kb64 + g16 / 4) * kSfChunk + sf_byte(r, g16 % 4)] = sq;
+      sfx[((static_cast<size_t>(blk) * nsub + r / 128) * kb64 + g16 / 4) * kSfChunk + sf_byte(r % 128, g16 % 4)] = sq;
     }
   }
 }
@@ -453,6 +454,294 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Prefill-size NVFP4 GEMMs on CTA pairs (tcgen05 cta_group::2).
+//
+// A pair tile is M = 256 weight rows (128 staged by each CTA) by N <= 224
+// tokens (N/2 staged by each CTA), K = 256 per stage: four block-scaled MMAs
+// of K = 64, issued by the even CTA.  Every load of a stage -- weights, tokens
+// and both kinds of scale chunks -- is a TMA copy with .cta_group::2 whose
+// bytes count on the even CTA's full barrier.  The scale chunks are viewed as
+// rows of 256 bytes (a 2 KB stage slice = 8 rows).  Each CTA's TMEM holds its
+// 128 rows for all N columns (two 224-column accumulators), the weight scales
+// of its own rows and the token scales of all N tokens (two 128-row chunks),
+// copied smem -> TMEM by one tcgen05.cp.cta_group::2 per chunk.
+// Tokens are padded per expert group to 224-row blocks; the activation scale
+// chunks of a block are its two 128-row halves.  A group's last tile runs the
+// MMA at N = the next multiple of 32 above its token count.
+// No TMA multicast: every CTA loads its own tiles.
+// ---------------------------------------------------------------------------
+constexpr int kQN = 224;                        // tokens per pair tile (padded block)
+constexpr int kQH = kQN / 2;                    // token rows staged per CTA
+constexpr uint32_t kQABytes = 128 * 128;        // 128 weight rows x 256 e2m1
+constexpr uint32_t kQBBytes = kQH * 128;        // 112 token rows x 256 e2m1
+constexpr uint32_t kQSfaBytes = 4 * kSfChunk;   // 4 K64 chunks of this CTA's 128 weight rows
+constexpr uint32_t kQSfbBytes = 8 * kSfChunk;   // 4 K64 chunks x 2 halves of the token block
+constexpr uint32_t kQStage = kQABytes + kQBBytes + kQSfaBytes + kQSfbBytes;
+constexpr int kQStages = 5;
+constexpr uint32_t kQSfCol = 2 * kQN;           // TMEM: accumulators [0, 448), scales [448, 496)
+
+__device__ __forceinline__ int quad_tile_n(int valid) { return min(kQN, (valid + 31) & ~31); }
+
+__device__ __forceinline__ void umma2_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Both CTAs of the pair: copy one 512-byte scale chunk from this offset of
+// each CTA's shared memory into the same columns of its own TMEM.
+__device__ __forceinline__ void tmem_cp_sf2(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+template <bool GATED>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    ffn_nvfp4_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAsh,
+                         const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmSfa,
+                         const __grid_constant__ CUtensorMap tmSfaSh, const __grid_constant__ CUtensorMap tmSfb,
+                         const int32_t* __restrict__ offsets, const int32_t* __restrict__ prow0,
+                         const int32_t* __restrict__ slot_of_expert, int E, int has_shared, int T, int P, int K,
+                         int Nw, int up_row0, const uint8_t* __restrict__ pool,
+                         const uint8_t* __restrict__ shared_bank, size_t bank_bytes, size_t st_off, int st_idx,
+                         uint8_t* __restrict__ out_q, uint8_t* __restrict__ out_sf, uint16_t* __restrict__ out_bf16) {
+  constexpr uint32_t kTmemCols = 512;
+  constexpr int kRowsPerPair = GATED ? 128 : 256;   // output rows (intermediate / hidden) per pair tile
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kQStages], empty_bar[kQStages], tfull_bar[2], tempty_bar[2];
+  __shared__ uint32_t tmem_holder;
+  __shared__ int32_t tile_start[kMaxGroups + 1], grp_rows[kMaxGroups], grp_row0[kMaxGroups];
+  __shared__ float xbuf[GATED ? 128 * 17 : 1];
+  __shared__ float tbuf[GATED ? 32 * 68 : 1];
+
+  const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (smem_base - smem_u32(smem_raw));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int npairs = gridDim.x / 2;
+  const int pair = blockIdx.x / 2;
+  const int G = E + (has_shared ? 1 : 0);
+  const int MT = Nw / kRowsPerPair;
+  const int KB = K / kF4StageK;
+  const int K64 = K / 64;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kQStages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 8); }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_holder)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmAsh);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmSfa);
+    tma_prefetch_desc(&tmSfaSh);
+    tma_prefetch_desc(&tmSfb);
+  }
+  pdl_wait();
+  pdl_trigger();
+  build_tile_table(offsets, E, has_shared, T, P, MT, kQN, tile_start, grp_rows, grp_row0);
+  tc_fence_before();
+  cluster_sync_all();     // barriers initialised and TMEM allocated in both CTAs
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_holder;
+  const int total = tile_start[G];
+
+  auto a_tile = [&](int s) -> uint8_t* { return smem + static_cast<size_t>(s) * kQStage; };
+  auto b_tile = [&](int s) -> uint8_t* { return a_tile(s) + kQABytes; };
+  auto sfa_tile = [&](int s) -> uint8_t* { return a_tile(s) + kQABytes + kQBBytes; };
+  auto sfb_tile = [&](int s) -> uint8_t* { return a_tile(s) + kQABytes + kQBBytes + kQSfaBytes; };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += npairs) {
+        const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, kQN);
+        const int ntile = quad_tile_n(min(kQN, ti.rows - ti.n * kQN));
+        const bool routed = ti.g < E;
+        const int slot = routed ? slot_of_expert[ti.g] : 0;
+        const int prow = prow0[ti.g] + ti.n * kQN;
+        const int blk = prow / kQN;
+        const int brow = prow + static_cast<int>(rank) * (ntile / 2);
+        const int wb = ti.m * 2 + static_cast<int>(rank);   // this CTA's 128-row weight block (paired for gate/up)
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_cl(&empty_bar[stage], phase ^ 1u)) { ok = false; break; }
+          if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * kQStage);
+          const uint32_t lbar = mapa_rank(smem_u32(&full_bar[stage]), 0);   // the even CTA's barrier
+          const int kc = kb * (kF4StageK / 2);                              // byte coordinate along K
+          const int sfa_row = (wb * K64 + 4 * kb) * 2;                       // 256-byte rows of the chunks
+          if (GATED) {
+            if (routed) {
+              tma2_load_3d(a_tile(stage), &tmA, lbar, kc, wb * 64, slot);
+              tma2_load_3d(a_tile(stage) + kQABytes / 2, &tmA, lbar, kc, up_row0 + wb * 64, slot);
+            } else {
+              tma2_load_2d(a_tile(stage), &tmAsh, lbar, kc, wb * 64);
+              tma2_load_2d(a_tile(stage) + kQABytes / 2, &tmAsh, lbar, kc, up_row0 + wb * 64);
+            }
+          } else {
+            if (routed) tma2_load_3d(a_tile(stage), &tmA, lbar, kc, wb * 128, slot);
+            else tma2_load_2d(a_tile(stage), &tmAsh, lbar, kc, wb * 128);
+          }
+          if (routed) tma2_load_3d(sfa_tile(stage), &tmSfa, lbar, 0, sfa_row, slot);
+          else tma2_load_2d(sfa_tile(stage), &tmSfaSh, lbar, 0, sfa_row);
+          tma2_load_2d(b_tile(stage), &tmB, lbar, kc, brow);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            tma2_load_2d(sfb_tile(stage) + h * (4 * kSfChunk), &tmSfb, lbar, 0, ((blk * 2 + h) * K64 + 4 * kb) * 2);
+          if (++stage == kQStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      const uint32_t sfa_t = tmem_base + kQSfCol, sfb_t = tmem_base + kQSfCol + 16;
+      for (int t = pair; t < total && ok; t += npairs, ++it) {
+        const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, kQN);
+        const uint32_t idesc = idesc_nvf4(256, quad_tile_n(min(kQN, ti.rows - ti.n * kQN)));
+        const int ab = it & 1;
+        const uint32_t aphase = (it >> 1) & 1;
+        if (!mbar_wait_cl(&tempty_bar[ab], aphase ^ 1u)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + ab * kQN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_cl(&full_bar[stage], phase)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(a_tile(stage)), sb = smem_u32(b_tile(stage));
+          const uint32_t ssa = smem_u32(sfa_tile(stage)), ssb = smem_u32(sfb_tile(stage));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            tmem_cp_sf2(sfa_t + 4 * kk, smem_desc_sf(ssa + kk * kSfChunk));
+            tmem_cp_sf2(sfb_t + 8 * kk, smem_desc_sf(ssb + kk * kSfChunk));
+            tmem_cp_sf2(sfb_t + 8 * kk + 4, smem_desc_sf(ssb + 4 * kSfChunk + kk * kSfChunk));
+          }
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma2_nvf4(d, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32), idesc, sfa_t + 4 * kk,
+                       sfb_t + 8 * kk, (kb | kk) != 0 ? 1u : 0u);
+          umma2_commit_both(&empty_bar[stage]);
+          if (++stage == kQStages) { stage = 0; phase ^= 1u; }
+        }
+        if (ok) umma2_commit_both(&tfull_bar[ab]);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int q = warp % 4;           // TMEM lane quadrant
+    const uint32_t tempty0 = mapa_rank(smem_u32(&tempty_bar[0]), 0);
+    const uint32_t tempty1 = mapa_rank(smem_u32(&tempty_bar[1]), 0);
+    int it = 0;
+    for (int t = pair; t < total; t += npairs, ++it) {
+      const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, kQN);
+      const int valid = min(kQN, ti.rows - ti.n * kQN);
+      const int ntile = quad_tile_n(valid);
+      const int ab = it & 1;
+      const uint32_t aphase = (it >> 1) & 1;
+      if (!epilogue_all(mbar_wait_cl(&tfull_bar[ab], aphase))) break;
+      tc_fence_after();
+      const uint8_t* bank = ti.g < E ? pool + static_cast<size_t>(slot_of_expert[ti.g]) * bank_bytes : shared_bank;
+      const float* st = reinterpret_cast<const float*>(bank + st_off);
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * kQN;
+      if (GATED) {
+        // this CTA's rows: 64 gate + the same 64 up rows of paired block pb
+        const int pb = ti.m * 2 + static_cast<int>(rank);
+        const bool gate_warp = q < 2;
+        const float s_row = st[st_idx + (gate_warp ? 0 : 1)];
+        const int me = q * 32 + lane, partner = (q ^ 2) * 32 + lane;
+        const int il = (q % 2) * 32 + lane;
+        const int col_off = gate_warp ? 0 : 16;
+        const int tslot = (il / 16) * 17 + il % 16;
+        const int prow = prow0[ti.g] + ti.n * kQN;
+        const int blk = prow / kQN;
+        const int tok = me >> 2, grp = me & 3;
+        for (int c0 = 0; c0 < ntile; c0 += 32) {
+          float v[32];
+          tmem_ld16(tb + c0, v);
+          tmem_ld16(tb + c0 + 16, v + 16);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] *= s_row;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) xbuf[me * 17 + j] = gate_warp ? v[16 + j] : v[j];
+          epilogue_bar();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float other = xbuf[partner * 17 + j];
+            tbuf[(col_off + j) * 68 + tslot] = gate_warp ? silu(v[j]) * other : silu(other) * v[16 + j];
+          }
+          epilogue_bar();
+          float h[16];
+          float amax = 0.f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            h[i] = tbuf[tok * 68 + grp * 17 + i];
+            amax = fmaxf(amax, fabsf(h[i]));
+          }
+          const uint8_t sq = f32_to_e4m3_sat(amax / 6.0f);
+          const float sc = e4m3_to_f32(sq);
+          uint32_t packed[2] = {0u, 0u};
+          if (sc != 0.f) {
+#pragma unroll
+            for (int i = 0; i < 16; i += 2)
+              packed[i / 8] |= static_cast<uint32_t>(f32x2_to_e2m1x2(h[i + 1] / sc, h[i] / sc)) << (4 * (i % 8));
+          }
+          const int tr = c0 + tok;   // token row within the 224-row block
+          *reinterpret_cast<uint2*>(out_q + static_cast<size_t>(prow + tr) * (Nw / 2) + (pb * 64 + grp * 16) / 2) =
+              make_uint2(packed[0], packed[1]);
+          out_sf[(static_cast<size_t>(blk * 2 + tr / 128) * (Nw / 64) + pb) * kSfChunk + sf_byte(tr % 128, grp)] = sq;
+        }
+      } else {
+        const float s_a = st[st_idx];
+        const int wrow = ti.m * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
+        uint16_t* o = out_bf16 + static_cast<size_t>(ti.row0 + ti.n * kQN) * Nw + wrow;
+        for (int c0 = 0; c0 < valid; c0 += 16) {
+          float a[16];
+          tmem_ld16(tb + c0, a);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (c0 + j < valid) {
+              const __nv_bfloat16 hb = __float2bfloat16_rn(a[j] * s_a);
+              o[static_cast<size_t>(c0 + j) * Nw] = *reinterpret_cast<const uint16_t*>(&hb);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(&tempty_bar[ab]);
+        else mbar_arrive_remote(ab ? tempty1 : tempty0);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync_all();     // no CTA leaves while its pair may still signal it
+  tc_fence_after();
+  if (warp == 1)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols) : "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Host
 // ---------------------------------------------------------------------------
 static bool make_map_f4(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint64_t slots,
@@ -478,9 +767,8 @@ static int64_t nvfp4_rows_pad(int64_t P, int T, int G, int has_shared, int BN) {
 // Workspace: prow0 | Xq [rows_pad][d/2] | SFx chunks | Hq [rows_pad][I/2] | SFh chunks
 size_t nvfp4_ffn_workspace_bytes(int64_t P, int T, int E, int has_shared, int d, int I) {
   const int G = E + (has_shared ? 1 : 0);
-  const int BN = 128;   // the largest tile bounds all
-  const int64_t rp = nvfp4_rows_pad(P, T, G, has_shared, BN);
-  const int64_t blocks = rp / 32 + G + 1;   // chunks are per BN-row block; BN >= 32
+  const int64_t rp = nvfp4_rows_pad(P, T, G, has_shared, kQN);   // the largest tile bounds all
+  const int64_t blocks = rp / 32 + G + 1;   // 128-row scale chunks: at most rows_pad / 32 + one partial per group
   return al256(sizeof(int32_t) * (G + 1)) + al256(rp * (d / 2)) + al256(blocks * (d / 64) * kSfChunk) +
          al256(rp * (I / 2)) + al256(blocks * (I / 64) * kSfChunk);
 }
@@ -508,14 +796,118 @@ static cudaError_t launch_nvfp4(const CUtensorMap& mA, const CUtensorMap& mAsh, 
                     st_idx, act_sf, out_q, out_sf, out_bf16, stages);
 }
 
+// ---- CTA-pair launch (prefill-size groups) -----------------------------------
+// Groups averaging >= 192 rows run on CTA pairs with 224-token tiles.
+static bool nvfp4_pair_applicable(int P, int E) { return (P + E - 1) / E >= 192; }
+
+// Scale chunks as rows of 256 bytes (a stage's 4 chunks = 8 rows), no swizzle:
+// dims {256, rows[, slots]}, box {256, 8[, 1]}.
+static bool make_map_rows256(CUtensorMap* m, const void* base, uint64_t bytes, uint64_t slots, uint64_t slot_pitch) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {256, bytes / 256, slots};
+  cuuint64_t strides[2] = {256, slot_pitch};
+  cuuint32_t box[3] = {256, 8, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  const cuuint32_t rank = slots > 0 ? 3 : 2;
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <bool GATED>
+static cudaError_t launch_nvfp4_tc2_one(const CUtensorMap* maps, const FfnArgs& a, const int32_t* prow0, int K,
+                                        int Nw, int up_row0, size_t st_off, int st_idx, uint8_t* out_q,
+                                        uint8_t* out_sf, uint16_t* out_bf16, cudaStream_t st) {
+  const size_t smem = 1024 + static_cast<size_t>(kQStages) * kQStage;
+  auto kern = ffn_nvfp4_tc2_kernel<GATED>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  const int P = a.T * a.k;
+  const int G = a.E + (a.has_shared ? 1 : 0);
+  const long tiles = static_cast<long>((P + kQN - 1) / kQN + G) * (Nw / (GATED ? 128 : 256));
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static int pairs_max[2] = {0, 0};   // co-resident pairs (not every SM may find a partner)
+  if (!pairs_max[GATED]) {
+    cfg.gridDim = dim3(num_sms());
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+      (void)cudaGetLastError();
+      n = num_sms() / 2;
+    }
+    pairs_max[GATED] = n < num_sms() / 2 ? n : num_sms() / 2;
+  }
+  const int pairs = static_cast<int>(tiles < pairs_max[GATED] ? tiles : pairs_max[GATED]);
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], a.offsets, prow0,
+                            a.slot_of_expert, a.E, a.has_shared, a.T, P, K, Nw, up_row0, a.pool, a.shared_bank,
+                            a.bank_bytes, st_off, st_idx, out_q, out_sf, out_bf16);
+}
+
+// Both GEMMs on CTA pairs; xq/sfx (gathered, padded to 224-row blocks) are ready.
+static const char* launch_nvfp4_gemms_tc2(const FfnArgs& a, const int32_t* prow0, size_t s_gu_off, size_t s_d_off,
+                                          size_t s_t_off, int64_t rp, uint8_t* xq, uint8_t* sfx, size_t sfx_bytes,
+                                          uint8_t* hq, uint8_t* sfh, size_t sfh_bytes, cudaStream_t st,
+                                          cudaError_t* cerr) {
+  const uint64_t S = static_cast<uint64_t>(a.S);
+  const uint64_t s_gu_bytes = 2ull * a.I * (a.d / 16), s_d_bytes = static_cast<uint64_t>(a.d) * (a.I / 16);
+  // maps per GEMM: A, A (shared expert), B, A scales, A scales (shared expert), B scales
+  CUtensorMap m1[6], m2[6];
+  bool ok = make_map_f4(&m1[0], a.pool + a.w_gu_off, a.d, 2ull * a.I, S, a.bank_bytes, 64) &&
+            make_map_f4(&m1[2], xq, a.d, static_cast<uint64_t>(rp), 0, 0, kQH) &&
+            make_map_rows256(&m1[3], a.pool + s_gu_off, s_gu_bytes, S, a.bank_bytes) &&
+            make_map_rows256(&m1[5], sfx, sfx_bytes, 0, 0) &&
+            make_map_f4(&m2[0], a.pool + a.w_d_off, a.I, a.d, S, a.bank_bytes, 128) &&
+            make_map_f4(&m2[2], hq, a.I, static_cast<uint64_t>(rp), 0, 0, kQH) &&
+            make_map_rows256(&m2[3], a.pool + s_d_off, s_d_bytes, S, a.bank_bytes) &&
+            make_map_rows256(&m2[5], sfh, sfh_bytes, 0, 0);
+  if (ok && a.has_shared) {
+    ok = make_map_f4(&m1[1], a.shared_bank + a.w_gu_off, a.d, 2ull * a.I, 0, 0, 64) &&
+         make_map_rows256(&m1[4], a.shared_bank + s_gu_off, s_gu_bytes, 0, 0) &&
+         make_map_f4(&m2[1], a.shared_bank + a.w_d_off, a.I, a.d, 0, 0, 128) &&
+         make_map_rows256(&m2[4], a.shared_bank + s_d_off, s_d_bytes, 0, 0);
+  } else {
+    m1[1] = m1[0];
+    m1[4] = m1[3];
+    m2[1] = m2[0];
+    m2[4] = m2[3];
+  }
+  if (!ok) return "cuTensorMapEncodeTiled failed";
+  prof_mark(FTM_K_GEMM1, st, false);
+  *cerr = launch_nvfp4_tc2_one<true>(m1, a, prow0, a.d, a.I, a.I, s_t_off, 0, hq, sfh, nullptr, st);
+  prof_mark(FTM_K_GEMM1, st, true);
+  if (*cerr != cudaSuccess) return "nvfp4 pair gemm1 launch failed";
+  prof_mark(FTM_K_GEMM2, st, false);
+  *cerr = launch_nvfp4_tc2_one<false>(m2, a, prow0, a.I, a.d, 0, s_t_off, 2, nullptr, nullptr,
+                                      reinterpret_cast<uint16_t*>(a.y), st);
+  prof_mark(FTM_K_GEMM2, st, true);
+  if (*cerr != cudaSuccess) return "nvfp4 pair gemm2 launch failed";
+  return nullptr;
+}
+
 const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_d_off, size_t s_t_off, uint8_t* ws,
                                     cudaStream_t st, cudaError_t* cerr) {
   const int P = a.T * a.k;
   const int G = a.E + (a.has_shared ? 1 : 0);
   *cerr = cudaSuccess;
   if (P + (a.has_shared ? a.T : 0) == 0) return nullptr;
-  const int BN = nvfp4_token_tile(P, a.E);
-  const int64_t rp = nvfp4_rows_pad(P, a.T, G, a.has_shared, 128);
+  const bool pair = nvfp4_pair_applicable(P, a.E);
+  const int BN = pair ? kQN : nvfp4_token_tile(P, a.E);
+  const int64_t rp = nvfp4_rows_pad(P, a.T, G, a.has_shared, kQN);
   const int64_t blocks = rp / 32 + G + 1;
   int32_t* prow0 = reinterpret_cast<int32_t*>(ws);
   uint8_t* xq = ws + al256(sizeof(int32_t) * (G + 1));
@@ -532,6 +924,9 @@ const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_
   }
   prof_mark(FTM_K_GATHER, st, true);
   if (*cerr != cudaSuccess) return "nvfp4 gather launch failed";
+  if (pair)
+    return launch_nvfp4_gemms_tc2(a, prow0, s_gu_off, s_d_off, s_t_off, rp, xq, sfx, blocks * (a.d / 64) * kSfChunk,
+                                  hq, sfh, blocks * (a.I / 64) * kSfChunk, st, cerr);
   CUtensorMap mA1, mAsh1, mB1, mA2, mAsh2, mB2;
   const uint64_t S = static_cast<uint64_t>(a.S);
   // gate/up boxes are 64 rows: a tile stages 64 gate rows and the same 64 up rows

@@ -25,13 +25,21 @@ def _check(dl, T, rows=None):
     return out, x, ids, g, rows, worst
 
 
-@pytest.mark.parametrize("T", [1, 20, 300, 700])   # token tiles of 32, 32, 64 and 128 rows
+@pytest.mark.parametrize("T", [1, 20, 300, 700, 1100])   # token tiles of 32, 32, 64, 128 rows; CTA pairs
 def test_small_nvfp4_layer(T):
     dl = screened_layer(SMALL_FP4, T)
     out, x, ids, g, rows, worst = _check(dl, T)
     # against the oracle without activation quantisation (W4A4 error is expected to be larger)
     plain = oracle.moe_rows(dl.layer, x, rows, ids, g, qa=oracle.QA_NONE)
     assert_rows_close(out[rows], plain, 0.35, "nvfp4 vs unquantised activations")
+
+
+def test_nvfp4_pair_tiles_multi_stage():
+    # >= 192 rows per expert on average: both GEMMs on CTA pairs (224-token
+    # tiles), several K stages in each GEMM, ragged groups and a shared expert
+    cfg = synth.scaled(SMALL_FP4, name="small_nvfp4_pairs", d=768, I=512, E=12, k=4, S=12)
+    dl = screened_layer(cfg, 900)
+    _check(dl, 900)
 
 
 def test_small_nvfp4_no_shared_expert():
