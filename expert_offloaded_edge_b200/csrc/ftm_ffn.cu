@@ -323,17 +323,6 @@ static long tile_bound(int P, int T, int E, int has_shared, int BN, int MT) {
   return (routed + (has_shared ? (T + BN - 1) / BN : 0)) * MT;
 }
 
-// Split-K ranks for a launch whose tiles cannot fill the GPU: the largest ks
-// <= 4 (and <= the k-blocks) with ks x tiles <= SMs.  1 = no split.
-static int split_k_ranks(long tiles, int KB) {
-  const long sms = num_sms();
-  if (tiles <= 0 || 2 * tiles > sms) return 1;
-  long ks = sms / tiles;
-  if (ks > 4) ks = 4;
-  if (ks > KB) ks = KB;
-  return ks < 1 ? 1 : static_cast<int>(ks);
-}
-
 template <int BN, bool GATED>
 static cudaError_t launch_tc(const CUtensorMap& mA, const CUtensorMap& mAsh, const CUtensorMap& mB,
                              const FfnArgs& a, int K, int Nw, int up_row0, uint16_t* out, int ld_out,
@@ -343,13 +332,53 @@ static cudaError_t launch_tc(const CUtensorMap& mA, const CUtensorMap& mAsh, con
   constexpr int kRedStride = GATED ? 36 : 20;
   const int P = a.T * a.k;
   const long tiles = tile_bound(P, a.T, a.E, a.has_shared, BN, Nw / 128);
-  const int ks = split_k_ranks(tiles, K / kBK);
-  const int red_bytes = (ks - 1) * 128 * kRedStride * 4;
-  const int budget = 200 * 1024;
-  int stages = (budget - 1024 - red_bytes) / static_cast<int>(kStageBytes);
-  if (stages > 8) stages = 8;
-  const size_t smem = 1024 + static_cast<size_t>(stages) * kStageBytes + red_bytes;
+  const int KB = K / kBK;
   auto kern = ffn_tc_kernel<BN, GATED>;
+  auto stages_for = [](int ks) {
+    const int red_bytes = (ks - 1) * 128 * kRedStride * 4;
+    const int s = (200 * 1024 - 1024 - red_bytes) / static_cast<int>(kStageBytes);
+    return s > 8 ? 8 : s;
+  };
+  auto smem_for = [&](int ks) {
+    return 1024 + static_cast<size_t>(stages_for(ks)) * kStageBytes + static_cast<size_t>(ks - 1) * 128 * kRedStride * 4;
+  };
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  // Split-K when the tiles cannot fill the GPU: a cluster of ks CTAs per tile,
+  // the largest ks <= 4 (and <= the k-blocks) whose clusters all fit at once
+  // (one wave: a second wave of clusters would double the kernel time).
+  static int max_clusters[5] = {0, 0, 0, 0, 0};   // co-resident clusters of ks CTAs, per ks
+  int ks = 1;
+  if (tiles > 0 && 2 * tiles <= num_sms()) {
+    for (int c = 4; c >= 2; --c) {
+      if (c > KB || c * tiles > num_sms()) continue;
+      if (!max_clusters[c]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_for(c)));
+        if (e != cudaSuccess) return e;
+        attr[0].val.clusterDim.x = c;
+        cfg.numAttrs = 1;
+        cfg.dynamicSmemBytes = smem_for(c);
+        cfg.gridDim = dim3(num_sms() / c * c);
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+          (void)cudaGetLastError();
+          n = 0;
+        }
+        max_clusters[c] = n > 0 ? n : -1;
+      }
+      if (tiles <= max_clusters[c]) { ks = c; break; }
+    }
+  }
+  const int stages = stages_for(ks);
+  const size_t smem = smem_for(ks);
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   if (ks == 1) {
@@ -357,31 +386,9 @@ static cudaError_t launch_tc(const CUtensorMap& mA, const CUtensorMap& mAsh, con
     return launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st, mA, mAsh, mB, a.offsets, a.slot_of_expert, a.E,
                       a.has_shared, a.T, P, K, Nw, up_row0, out, ld_out, stages);
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kTcThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = ks;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  static int max_clusters[5] = {0, 0, 0, 0, 0};   // co-resident clusters of ks CTAs, per ks
-  if (!max_clusters[ks]) {
-    cfg.gridDim = dim3(num_sms() / ks * ks);
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
-      (void)cudaGetLastError();
-      n = num_sms() / ks;
-    }
-    max_clusters[ks] = n;
-  }
-  const long ncl = tiles < max_clusters[ks] ? tiles : max_clusters[ks];
-  cfg.gridDim = dim3(static_cast<unsigned>(ncl * ks));
+  cfg.dynamicSmemBytes = smem;
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles * ks));
   cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, mA, mAsh, mB, a.offsets, a.slot_of_expert, a.E, a.has_shared, a.T, P, K, Nw,
                             up_row0, out, ld_out, stages);
