@@ -125,18 +125,61 @@ __global__ void pad_offsets_kernel(const int32_t* __restrict__ offsets, int E, i
 }
 
 // ---------------------------------------------------------------------------
-// Gather + NVFP4 quantisation of x into the padded activation rows.
-// One warp per padded row (grid-strided); the padded group offsets sit in
-// shared memory, lane 0 finds the row's source token, and each lane quantises
-// whole 16-element groups (two 16-byte loads -> 8 packed bytes + one scale).
+// NVFP4 quantisation of x, once per token: xq_tok [T][d/2] packed e2m1 and
+// sw_tok [T][d/64] words holding the four e4m3 scales of each 64-element
+// block (the 4 bytes a scale chunk keeps together for one row).  One warp per
+// token; each lane quantises whole 16-element groups (two 16-byte loads ->
+// 8 packed bytes + one scale).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) gather_quant_nvfp4_kernel(const uint16_t* __restrict__ x,
-                                                                const int32_t* __restrict__ perm,
-                                                                const int32_t* __restrict__ offsets,
-                                                                const int32_t* __restrict__ prow0, int E,
-                                                                int has_shared, int T, int k, int d, int BN,
-                                                                uint8_t* __restrict__ xq,
-                                                                uint8_t* __restrict__ sfx) {
+__global__ void __launch_bounds__(256) quant_tokens_nvfp4_kernel(const uint16_t* __restrict__ x, int T, int d,
+                                                                 uint8_t* __restrict__ xq_tok,
+                                                                 uint8_t* __restrict__ s_tok) {
+  pdl_wait();
+  pdl_trigger();
+  const int ng = d / 16;
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nwarps = blockDim.x / 32;
+  for (int t = blockIdx.x * nwarps + warp; t < T; t += gridDim.x * nwarps) {
+    for (int g16 = lane; g16 < ng; g16 += 32) {
+      float v[16];
+      const uint4* p = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d + g16 * 16);
+      const uint4 u0 = p[0], u1 = p[1];
+      const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFF);
+        v[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
+      }
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      const uint8_t sq = f32_to_e4m3_sat(amax / 6.0f);
+      const float sc = e4m3_to_f32(sq);
+      uint32_t packed[2] = {0, 0};
+      if (sc != 0.f) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          packed[i / 4] |= static_cast<uint32_t>(f32x2_to_e2m1x2(v[2 * i + 1] / sc, v[2 * i] / sc)) << (8 * (i % 4));
+      }
+      *reinterpret_cast<uint2*>(xq_tok + static_cast<size_t>(t) * (d / 2) + g16 * 8) = make_uint2(packed[0], packed[1]);
+      s_tok[static_cast<size_t>(t) * (d / 16) + g16] = sq;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Gather of the quantised tokens into the padded activation rows: one warp
+// per padded row copies its token's d/2 packed bytes (16-byte vectors) and
+// scatters its d/64 scale words into the row's place in the scale chunks
+// (rows past a group's end are zeros).  The padded group offsets sit in
+// shared memory; lane 0 finds the row's source token.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) gather_nvfp4_kernel(const uint8_t* __restrict__ xq_tok,
+                                                          const uint8_t* __restrict__ s_tok,
+                                                          const int32_t* __restrict__ perm,
+                                                          const int32_t* __restrict__ offsets,
+                                                          const int32_t* __restrict__ prow0, int E, int has_shared,
+                                                          int T, int k, int d, int BN, uint8_t* __restrict__ xq,
+                                                          uint8_t* __restrict__ sfx) {
   __shared__ int32_t s_prow0[kMaxGroups + 1];
   pdl_wait();
   pdl_trigger();
@@ -144,7 +187,8 @@ __global__ void __launch_bounds__(256) gather_quant_nvfp4_kernel(const uint16_t*
   for (int i = threadIdx.x; i <= G; i += blockDim.x) s_prow0[i] = prow0[i];
   __syncthreads();
   const int rows_pad = s_prow0[G];
-  const int kb64 = d / 64, ng = d / 16;
+  const int kb64 = d / 64, nvec = d / 32;          // 16-byte vectors per packed row
+  const int nsub = (BN + 127) / 128;               // 128-row scale chunks per BN-row block
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nwarps = blockDim.x / 32;
   for (int pr = blockIdx.x * nwarps + warp; pr < rows_pad; pr += gridDim.x * nwarps) {
     int src = -1;
@@ -159,37 +203,14 @@ __global__ void __launch_bounds__(256) gather_quant_nvfp4_kernel(const uint16_t*
       src = local >= rows ? -1 : (lo < E ? perm[offsets[lo] + local] / k : local);
     }
     src = __shfl_sync(0xffffffffu, src, 0);
-    const int nsub = (BN + 127) / 128;   // 128-row scale chunks per BN-row block
+    const uint4* s = reinterpret_cast<const uint4*>(xq_tok + static_cast<size_t>(src < 0 ? 0 : src) * (d / 2));
+    uint4* dst = reinterpret_cast<uint4*>(xq + static_cast<size_t>(pr) * (d / 2));
+    for (int c = lane; c < nvec; c += 32) dst[c] = src >= 0 ? s[c] : make_uint4(0, 0, 0, 0);
     const int blk = pr / BN, r = pr % BN;
-    for (int g16 = lane; g16 < ng; g16 += 32) {
-      float v[16];
-      if (src >= 0) {
-        const uint4* p = reinterpret_cast<const uint4*>(x + static_cast<size_t>(src) * d + g16 * 16);
-        const uint4 u0 = p[0], u1 = p[1];
-        const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          v[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFF);
-          v[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = 0.f;
-      }
-      float amax = 0.f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-      const uint8_t sq = f32_to_e4m3_sat(amax / 6.0f);
-      const float s = e4m3_to_f32(sq);
-      uint32_t packed[2] = {0, 0};
-      if (s != 0.f) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          packed[i / 4] |= static_cast<uint32_t>(f32x2_to_e2m1x2(v[2 * i + 1] / s, v[2 * i] / s)) << (8 * (i % 4));
-      }
-      *reinterpret_cast<uint2*>(xq + static_cast<size_t>(pr) * (d / 2) + g16 * 8) = make_uint2(packed[0], packed[1]);
-      sfx[((static_cast<size_t>(blk) * nsub + r / 128) * kb64 + g16 / 4) * kSfChunk + sf_byte(r % 128, g16 % 4)] = sq;
-    }
+    const uint32_t* sw = reinterpret_cast<const uint32_t*>(s_tok + static_cast<size_t>(src < 0 ? 0 : src) * (d / 16));
+    uint8_t* chunk0 = sfx + (static_cast<size_t>(blk) * nsub + r / 128) * kb64 * kSfChunk + sf_byte(r % 128, 0);
+    for (int kb = lane; kb < kb64; kb += 32)
+      *reinterpret_cast<uint32_t*>(chunk0 + static_cast<size_t>(kb) * kSfChunk) = src >= 0 ? sw[kb] : 0u;
   }
 }
 
@@ -764,13 +785,15 @@ static int64_t nvfp4_rows_pad(int64_t P, int T, int G, int has_shared, int BN) {
   return P + (has_shared ? T : 0) + static_cast<int64_t>(G) * (BN - 1);
 }
 
-// Workspace: prow0 | Xq [rows_pad][d/2] | SFx chunks | Hq [rows_pad][I/2] | SFh chunks
+// Workspace: prow0 | Xq [rows_pad][d/2] | SFx chunks | Hq [rows_pad][I/2] | SFh chunks |
+//            per-token Xq [T][d/2] | per-token scales [T][d/16]
 size_t nvfp4_ffn_workspace_bytes(int64_t P, int T, int E, int has_shared, int d, int I) {
   const int G = E + (has_shared ? 1 : 0);
   const int64_t rp = nvfp4_rows_pad(P, T, G, has_shared, kQN);   // the largest tile bounds all
   const int64_t blocks = rp / 32 + G + 1;   // 128-row scale chunks: at most rows_pad / 32 + one partial per group
   return al256(sizeof(int32_t) * (G + 1)) + al256(rp * (d / 2)) + al256(blocks * (d / 64) * kSfChunk) +
-         al256(rp * (I / 2)) + al256(blocks * (I / 64) * kSfChunk);
+         al256(rp * (I / 2)) + al256(blocks * (I / 64) * kSfChunk) + al256(static_cast<int64_t>(T) * (d / 2)) +
+         al256(static_cast<int64_t>(T) * (d / 16));
 }
 
 template <int BN, bool GATED>
@@ -914,13 +937,21 @@ const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_
   uint8_t* sfx = xq + al256(rp * (a.d / 2));
   uint8_t* hq = sfx + al256(blocks * (a.d / 64) * kSfChunk);
   uint8_t* sfh = hq + al256(rp * (a.I / 2));
+  uint8_t* xq_tok = sfh + al256(blocks * (a.I / 64) * kSfChunk);
+  uint8_t* s_tok = xq_tok + al256(static_cast<int64_t>(a.T) * (a.d / 2));
   prof_mark(FTM_K_GATHER, st, false);
+  // each token is quantised once, then its packed row is copied into every
+  // padded row that uses it (k routed picks + the shared expert)
   *cerr = launch_pdl(pad_offsets_kernel, dim3(1), dim3(512), 0, st, a.offsets, a.E, a.has_shared, a.T, BN, prow0);
   if (*cerr == cudaSuccess) {
+    const int grid = a.T / 8 + 1 < 148 * 8 ? a.T / 8 + 1 : 148 * 8;
+    *cerr = launch_pdl(quant_tokens_nvfp4_kernel, dim3(grid), dim3(256), 0, st,
+                       reinterpret_cast<const uint16_t*>(a.x), a.T, a.d, xq_tok, s_tok);
+  }
+  if (*cerr == cudaSuccess) {
     const int grid = static_cast<int>(rp / 8 + 1 < 148 * 8 ? rp / 8 + 1 : 148 * 8);
-    *cerr = launch_pdl(gather_quant_nvfp4_kernel, dim3(grid), dim3(256), 0, st,
-                       reinterpret_cast<const uint16_t*>(a.x), a.perm, a.offsets, prow0, a.E, a.has_shared, a.T,
-                       a.k, a.d, BN, xq, sfx);
+    *cerr = launch_pdl(gather_nvfp4_kernel, dim3(grid), dim3(256), 0, st, xq_tok, s_tok, a.perm, a.offsets, prow0,
+                       a.E, a.has_shared, a.T, a.k, a.d, BN, xq, sfx);
   }
   prof_mark(FTM_K_GATHER, st, true);
   if (*cerr != cudaSuccess) return "nvfp4 gather launch failed";
