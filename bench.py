@@ -350,14 +350,18 @@ def reference_arm(args, rank, world):
 def trace_main(args, cfg, T, rank, world, local, dist):
     """The decode trace over the LRU slot cache: one step = route, permute, cache
     update with miss copies (host sync), FFN, combine.  Warm-up = the first W
-    steps of the trace, timed = the next K (K + W <= trace length)."""
+    steps of the trace, timed = the next K with the tokens resident in HBM,
+    then end to end = the K2 steps after those, each step copying its tokens
+    from pinned host memory and its output back (K + K2 + W <= trace length)."""
     from synth.device import DeviceLayer, Workspace
     dl = DeviceLayer(cfg)
     W = args.warmup
-    K = args.steps if args.steps is not None else cfg.trace_steps - W
-    K = max(1, min(K, cfg.trace_steps - W))
+    K = args.steps if args.steps is not None else (cfg.trace_steps - W) // 2
+    K = max(1, min(K, cfg.trace_steps - W - 1))
+    K2 = max(1, min(K, cfg.trace_steps - W - K))
     args.steps = K
     xs = [dl.hidden(T, step=s) for s in range(W + K)]
+    xs_host = [dl.hidden(T, step=s).cpu().pin_memory() for s in range(W + K, W + K + K2)]
     ws = Workspace(ftm.ftm_workspace_bytes(dl.desc, T))
     out = torch.empty((T, cfg.d), dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.Stream()
@@ -398,6 +402,21 @@ def trace_main(args, cfg, T, rank, world, local, dist):
     clk = clocks.stop()
     g1 = [a.elapsed_time(b) for a, b in evs]
     ms, value = job_throughput(ms, K * T, dist, "cuda")
+    # end to end: the next K2 steps through the public call with host tokens in and out
+    x_dev = torch.empty_like(xs[0])
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(K2):
+        with torch.cuda.stream(stream):
+            x_dev.copy_(xs_host[i], non_blocking=True)
+        ftm.ftm_moe_layer_forward(dl.desc, w, dl.cache, x_dev, T, out, ws.ptr, ws.nbytes, stream, copy_stream)
+        with torch.cuda.stream(stream):
+            out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms, e2e_value = job_throughput(e0.elapsed_time(e1), K2 * T, dist, "cuda")
     status = ftm.ftm_device_status(True)
     if rank != 0:
         return
@@ -423,8 +442,12 @@ def trace_main(args, cfg, T, rank, world, local, dist):
                   "h2d_gb_per_step": misses / K * bl.bank_bytes / 1e9,
                   "h2d_gbs_effective": misses * bl.bank_bytes / (ms * 1e-3) / 1e9},
         "cpu_baseline": None,
-        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": int(misses / K * bl.bank_bytes),
-                "d2h_bytes_per_step": 0, "launch": "eager; the step already includes the host miss-copy path"},
+        "e2e": {"value": e2e_value, "unit": "tokens/s",
+                "h2d_bytes_per_step": int(xs_host[0].numel() * xs_host[0].element_size()),
+                "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size()),
+                "steps": K2, "trace_steps": f"{W + K}..{W + K + K2 - 1}",
+                "launch": "eager; tokens copied in from pinned host memory and the output copied out every step, "
+                          "on top of the miss copies the step already makes"},
         "gpu_launches": 7 * K,
         "clocks": clk,
         "device_status": status,
