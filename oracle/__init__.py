@@ -59,6 +59,8 @@ def lib():
         L.orc_permute.argtypes = [p, i32, i32, i32, p, p, p, p]
         L.orc_lru_step.argtypes = [i32, i32, p, p, p, i64, p, i32, p, p, p, p, p]
         L.orc_lru_step.restype = i32
+        L.orc_lru_resize.argtypes = [i32, i32, p, p, p, i32, p, p, p, p]
+        L.orc_lru_resize.restype = i32
         L.orc_expert_ffn.argtypes = [p, i32, i32, i32, p, p, p, i32, p]
         L.orc_combine.argtypes = [p, p, i32, i32, i32, p, p]
         _lib = L
@@ -216,6 +218,18 @@ class LRUState:
             self.step += 1
         misses = [(int(me[i]), int(ms[i])) for i in range(int(nm[0]))]
         return rc, misses, int(nd[0]), int(nh[0])
+
+    def resize(self, S_new: int):
+        """Elastic resize to S_new slots (see orc_lru_resize).  Returns the new
+        state and move_from: slot i of the new pool holds the bank of old slot
+        move_from[i]."""
+        n = LRUState(self.E, S_new)
+        n.step = self.step
+        mf = np.empty(max(1, min(self.S, S_new)), dtype=np.int32)
+        kept = lib().orc_lru_resize(self.E, self.S, _p(self.slot_of_expert), _p(self.expert_of_slot),
+                                    _p(self.last_use), S_new, _p(n.slot_of_expert), _p(n.expert_of_slot),
+                                    _p(n.last_use), _p(mf))
+        return n, mf[:kept].copy()
 
 
 # ---- expert FFN / combine -----------------------------------------------------------

@@ -314,6 +314,46 @@ int orc_lru_step(int E, int S, int32_t* slot_of_expert, int32_t* expert_of_slot,
 }
 
 /* ---------------------------------------------------------------------------
+ * Elastic slot-pool resize.  The pages let the expert cache's share of VRAM
+ * change at run time without restarting the engine or reloading weights
+ * (pomoai.com FreeToken hub, the two-level expert memory paragraph; freelamp.com
+ * FreeToken article, section 2.3 "elastic memory management": `ftctl cache
+ * --moe <slots>`).  Reading taken here: the min(S_new, resident)
+ * most recently used resident experts stay (largest last_use first, ties to the
+ * lower old slot), in their old slot order, in slots 0..; the rest are evicted;
+ * each kept expert keeps its last_use; the step counter does not move.
+ * Written as the definition: S_new rounds of "take the most recent resident
+ * slot not yet taken".  Returns the number of kept experts; move_from[i] ->
+ * i is the bank move of the i-th kept expert.
+ * ------------------------------------------------------------------------- */
+int orc_lru_resize(int E, int S_old, const int32_t* slot_of_expert, const int32_t* expert_of_slot,
+                   const int64_t* last_use, int S_new, int32_t* soe_new, int32_t* eos_new, int64_t* lu_new,
+                   int32_t* move_from) {
+  (void)slot_of_expert;
+  uint8_t* kept = (uint8_t*)calloc((size_t)(S_old > 0 ? S_old : 1), 1);
+  for (int r = 0; r < S_new; ++r) {
+    int best = -1;
+    for (int j = 0; j < S_old; ++j)
+      if (expert_of_slot[j] >= 0 && !kept[j] && (best < 0 || last_use[j] > last_use[best])) best = j;
+    if (best < 0) break;
+    kept[best] = 1;
+  }
+  for (int e = 0; e < E; ++e) soe_new[e] = -1;
+  for (int j = 0; j < S_new; ++j) { eos_new[j] = -1; lu_new[j] = -1; }
+  int n = 0;
+  for (int j = 0; j < S_old; ++j) {
+    if (!kept[j]) continue;
+    eos_new[n] = expert_of_slot[j];
+    lu_new[n] = last_use[j];
+    soe_new[expert_of_slot[j]] = n;
+    move_from[n] = j;
+    ++n;
+  }
+  free(kept);
+  return n;
+}
+
+/* ---------------------------------------------------------------------------
  * Expert FFN (SwiGLU) over n rows, and the combine.
  * h[i] = silu(x . Wg[i]) * (x . Wu[i]),  silu(z) = z / (1 + exp(-z));
  * y[j] = h . Wd[j].

@@ -302,6 +302,87 @@ def test_lru_matches_list_replay(E, S, n, seed):
         assert nh == len(set(ids.tolist())) - len(m)
 
 
+def test_lru_resize_hand_worked():
+    st = oracle.LRUState(E=10, S=4)
+    st.expert_of_slot[:] = [5, -1, 2, 7]
+    st.last_use[:] = [3, -1, 9, 3]
+    st.slot_of_expert[:] = -1
+    st.slot_of_expert[[5, 2, 7]] = [0, 2, 3]
+    st.step = 10
+    # shrink to 2: keep slot 2 (last_use 9) and slot 0 (3; ties with slot 3 -> the lower slot), in old order
+    n, mf = st.resize(2)
+    assert mf.tolist() == [0, 2]
+    assert n.expert_of_slot.tolist() == [5, 2] and n.last_use.tolist() == [3, 9]
+    assert n.slot_of_expert[5] == 0 and n.slot_of_expert[2] == 1 and n.slot_of_expert[7] == -1
+    assert n.step == 10 and n.S == 2
+    # grow to 6: every resident expert stays, compacted; the new slots are empty
+    g, mf = st.resize(6)
+    assert mf.tolist() == [0, 2, 3]
+    assert g.expert_of_slot.tolist() == [5, 2, 7, -1, -1, -1] and g.last_use.tolist() == [3, 9, 3, -1, -1, -1]
+    # shrink to 1: only the most recent
+    o, mf = st.resize(1)
+    assert mf.tolist() == [2] and o.expert_of_slot.tolist() == [2]
+
+
+def _resize_by_sort(st, S_new):
+    """The resize written another way: sort the residents by (-last_use, slot)."""
+    res = [j for j in range(st.S) if st.expert_of_slot[j] >= 0]
+    keep = sorted(sorted(res, key=lambda j: (-int(st.last_use[j]), j))[:S_new])
+    eos = [int(st.expert_of_slot[j]) for j in keep] + [-1] * (S_new - len(keep))
+    lu = [int(st.last_use[j]) for j in keep] + [-1] * (S_new - len(keep))
+    return keep, eos, lu
+
+
+@pytest.mark.parametrize("E,S,n,seed", [(16, 4, 3, 0), (64, 16, 10, 1), (256, 64, 40, 2)])
+def test_lru_resize_matches_sort_and_invariants(E, S, n, seed):
+    rng = np.random.default_rng(seed)
+    st = oracle.LRUState(E, S)
+    zipf = 1.0 / np.arange(1, E + 1) ** 1.1
+    zipf /= zipf.sum()
+    for step in range(30):
+        st.update(rng.choice(E, size=n, p=zipf))
+        for S_new in sorted({1, max(1, S // 2), S - 1, S, S + 3, 2 * S} - {0}):
+            new, mf = st.resize(S_new)
+            keep, eos, lu = _resize_by_sort(st, S_new)
+            assert mf.tolist() == keep
+            assert new.expert_of_slot.tolist() == eos and new.last_use.tolist() == lu
+            # slot table and reverse table agree; evicted experts are unmapped
+            for j, e in enumerate(eos):
+                if e >= 0:
+                    assert new.slot_of_expert[e] == j
+            assert int((new.slot_of_expert >= 0).sum()) == len(keep)
+            # nothing kept is older than anything evicted
+            ev = [int(st.last_use[j]) for j in range(S) if st.expert_of_slot[j] >= 0 and j not in keep]
+            if ev and keep:
+                assert min(int(st.last_use[j]) for j in keep) >= max(ev)
+
+
+def test_lru_resize_then_steps_match_list_replay():
+    """After a resize the cache keeps following the LRU rule: an eviction-list
+    LRU seeded with the kept experts (in last-use order) replays the same misses."""
+    E, S, n = 64, 16, 10
+    rng = np.random.default_rng(5)
+    st = oracle.LRUState(E, S)
+    zipf = 1.0 / np.arange(1, E + 1) ** 1.1
+    zipf /= zipf.sum()
+    for _ in range(20):
+        st.update(rng.choice(E, size=n, p=zipf))
+    st, _ = st.resize(12)
+    ref = ListLRU(E, 12)
+    ref.expert = st.expert_of_slot.tolist()
+    ref.where = {e: j for j, e in enumerate(ref.expert) if e >= 0}
+    # eviction order: empty slots by index, then by (last_use, slot)
+    ref.order = sorted(range(12), key=lambda j: (int(st.last_use[j]), j))
+    for _ in range(100):
+        ids = rng.choice(E, size=n, p=zipf)
+        rc, m, nd, nh = st.update(ids)
+        rm = ref.step(ids)
+        if rm is None:
+            assert rc == -1
+            continue
+        assert rc == 0 and m == rm
+
+
 # ---------------------------------------------------------------------------
 # Expert FFN and combine
 # ---------------------------------------------------------------------------
