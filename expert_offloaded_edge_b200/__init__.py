@@ -32,6 +32,7 @@ from .binding import (  # noqa: F401
     KERNEL_NAMES,
     ftm_slot_host_scratch_ints,
     ftm_slot_lookup_update,
+    ftm_slot_resize,
     ftm_slot_workspace_bytes,
     ftm_workspace_bytes,
     library,

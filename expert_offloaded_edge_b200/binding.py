@@ -70,6 +70,7 @@ def library() -> ctypes.CDLL:
         L.ftm_slot_workspace_bytes.argtypes = [P(LayerDesc)]
         L.ftm_slot_workspace_bytes.restype = c_sz
         L.ftm_slot_lookup_update.argtypes = [P(LayerDesc), P(SlotCache), c_p, c_i32, c_p, c_sz, c_p, c_p]
+        L.ftm_slot_resize.argtypes = [P(LayerDesc), P(SlotCache), c_i32, P(SlotCache), c_p, c_sz, c_p]
         L.ftm_expert_ffn.argtypes = [P(LayerDesc), c_p, c_i32, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_sz, c_p]
         L.ftm_ffn_workspace_bytes.argtypes = [P(LayerDesc), c_i32]
         L.ftm_ffn_workspace_bytes.restype = c_sz
@@ -82,8 +83,8 @@ def library() -> ctypes.CDLL:
         L.ftm_set_profile_events.restype = c_i32
         L.ftm_workspace_bytes.argtypes = [P(LayerDesc), c_i32]
         L.ftm_workspace_bytes.restype = c_sz
-        for name in ("ftm_get_bank_layout", "ftm_route", "ftm_permute", "ftm_slot_lookup_update", "ftm_expert_ffn",
-                     "ftm_combine", "ftm_moe_layer_forward"):
+        for name in ("ftm_get_bank_layout", "ftm_route", "ftm_permute", "ftm_slot_lookup_update", "ftm_slot_resize",
+                     "ftm_expert_ffn", "ftm_combine", "ftm_moe_layer_forward"):
             getattr(L, name).restype = c_i32
         _lib = L
     return _lib
@@ -157,6 +158,11 @@ def ftm_slot_lookup_update(desc, cache: SlotCache, topk_ids, T, workspace, ws_by
     _check(library().ftm_slot_lookup_update(ctypes.byref(desc), ctypes.byref(cache), _ptr(topk_ids), T,
                                             _ptr(workspace), ws_bytes, _stream(compute_stream),
                                             _stream(copy_stream)))
+
+
+def ftm_slot_resize(desc, cache: SlotCache, S_new: int, new_cache: SlotCache, workspace, ws_bytes, stream=None):
+    _check(library().ftm_slot_resize(ctypes.byref(desc), ctypes.byref(cache), S_new, ctypes.byref(new_cache),
+                                     _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def ftm_ffn_workspace_bytes(desc, T) -> int:

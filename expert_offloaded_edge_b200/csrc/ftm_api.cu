@@ -18,6 +18,9 @@ cudaError_t launch_lru_step(const int32_t* ids, int P, int E, int S, int64_t ste
                             int64_t* lu, int32_t* ws, cudaStream_t st);
 cudaError_t launch_lru_restore(int E, int S, int32_t* soe, int32_t* eos, int64_t* lu, const int32_t* ws,
                                cudaStream_t st);
+cudaError_t launch_slot_resize(int E, int S_old, const int32_t* eos_old, const int64_t* lu_old, int S_new,
+                               int32_t* soe_new, int32_t* eos_new, int64_t* lu_new, const void* old_pool,
+                               void* new_pool, size_t bank_bytes, int32_t* ws, cudaStream_t st);
 cudaError_t launch_combine(bool f32, const void* y, const int32_t* inv, const float* gw, int T, int k, int d, int P,
                            int has_shared, void* out, cudaStream_t st);
 const char* launch_expert_ffn(const FfnArgs& a, cudaStream_t st, cudaError_t* cerr);
@@ -262,6 +265,36 @@ size_t ftm_slot_host_scratch_ints(const ftm_layer_desc* L) {
 size_t ftm_slot_workspace_bytes(const ftm_layer_desc* L) {
   if (check_desc(L)) return 0;
   return lru_workspace_bytes(L->E, L->S);
+}
+
+ftm_status ftm_slot_resize(const ftm_layer_desc* L, const ftm_slot_cache* C, int32_t S_new, ftm_slot_cache* C_new,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  ftm_status s = check_desc(L);
+  if (s) return s;
+  if (!C || !C->slot_of_expert || !C->expert_of_slot || !C->last_use || !C->slot_pool)
+    return fail(FTM_ERR_INVALID_ARG, "ftm_slot_resize: cache has a NULL member");
+  if (!C_new || !C_new->slot_of_expert || !C_new->expert_of_slot || !C_new->last_use || !C_new->slot_pool)
+    return fail(FTM_ERR_INVALID_ARG, "ftm_slot_resize: new cache has a NULL member");
+  if (S_new < 1) return fail(FTM_ERR_INVALID_ARG, "ftm_slot_resize: S_new=%d < 1", S_new);
+  if (L->S > 4096 || S_new > 4096)
+    return fail(FTM_ERR_UNSUPPORTED, "LRU cache supports S <= 4096 (S=%d, S_new=%d)", L->S, S_new);
+  ftm_bank_layout bl;
+  if ((s = ftm_get_bank_layout(L, &bl))) return s;
+  // the new pool and state must not overlap the old ones (the moves read the old pool while writing the new)
+  const uintptr_t o0 = reinterpret_cast<uintptr_t>(C->slot_pool), o1 = o0 + bl.bank_bytes * L->S;
+  const uintptr_t n0 = reinterpret_cast<uintptr_t>(C_new->slot_pool), n1 = n0 + bl.bank_bytes * S_new;
+  if (n0 < o1 && o0 < n1) return fail(FTM_ERR_INVALID_ARG, "ftm_slot_resize: new slot pool overlaps the old one");
+  if (C_new->slot_of_expert == C->slot_of_expert || C_new->expert_of_slot == C->expert_of_slot ||
+      C_new->last_use == C->last_use)
+    return fail(FTM_ERR_INVALID_ARG, "ftm_slot_resize: new state arrays must be distinct from the old ones");
+  if ((s = check_ws(workspace, ws_bytes, lru_workspace_bytes(L->E, L->S), "ftm_slot_resize"))) return s;
+  cudaError_t e = launch_slot_resize(L->E, L->S, C->expert_of_slot, C->last_use, S_new, C_new->slot_of_expert,
+                                     C_new->expert_of_slot, C_new->last_use, C->slot_pool, C_new->slot_pool,
+                                     bl.bank_bytes, static_cast<int32_t*>(workspace), S_(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "slot resize launch");
+  C_new->step = C->step;
+  C_new->last_distinct = C_new->last_hits = C_new->last_misses = 0;
+  return FTM_OK;
 }
 
 ftm_status ftm_slot_lookup_update(const ftm_layer_desc* L, ftm_slot_cache* C, const int32_t* topk_ids, int32_t T,

@@ -144,4 +144,110 @@ cudaError_t launch_lru_restore(int E, int S, int32_t* soe, int32_t* eos, int64_t
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Elastic slot-pool resize (the pages: the expert cache's share of VRAM can be
+// changed at run time without restarting or reloading weights; pomoai.com
+// FreeToken hub, two-level expert memory; freelamp.com FreeToken article,
+// section 2.3 "elastic memory management", `ftctl cache --moe <slots>`).
+// The min(S_new, resident) most recently used resident experts stay (largest
+// last_use first, ties to the lower old slot), compacted into slots 0.. in
+// their old slot order, keeping their last_use; the rest are evicted.
+//
+// One block: each resident slot's rank in keep order is a count over the other
+// slots (no sort); warp 0 scans the keep flags into new slot indices.  The
+// move list goes to the workspace: ws[0] = kept, ws[1 + i] = old slot of new
+// slot i; the bank copies then run on the device from that list.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kLruThreads) slot_resize_kernel(int E, int S_old,
+                                                                  const int32_t* __restrict__ eos_old,
+                                                                  const int64_t* __restrict__ lu_old, int S_new,
+                                                                  int32_t* __restrict__ soe_new,
+                                                                  int32_t* __restrict__ eos_new,
+                                                                  int64_t* __restrict__ lu_new,
+                                                                  int32_t* __restrict__ ws) {
+  extern __shared__ __align__(8) uint8_t sm_raw[];
+  int64_t* s_lu = reinterpret_cast<int64_t*>(sm_raw);            // [S_old]
+  int32_t* s_eos = reinterpret_cast<int32_t*>(s_lu + S_old);     // [S_old]
+  int32_t* s_pos = s_eos + S_old;                                 // [S_old] keep flag, then new slot (or -1)
+  pdl_wait();
+  pdl_trigger();
+  for (int j = threadIdx.x; j < S_old; j += blockDim.x) { s_lu[j] = lu_old[j]; s_eos[j] = eos_old[j]; }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) soe_new[e] = -1;
+  for (int j = threadIdx.x; j < S_new; j += blockDim.x) { eos_new[j] = -1; lu_new[j] = -1; }
+  __syncthreads();
+  for (int j = threadIdx.x; j < S_old; j += blockDim.x) {
+    int keep = 0;
+    if (s_eos[j] >= 0) {
+      int before = 0;   // resident slots that come earlier in keep order
+      for (int i = 0; i < S_old; ++i)
+        before += (s_eos[i] >= 0 && (s_lu[i] > s_lu[j] || (s_lu[i] == s_lu[j] && i < j))) ? 1 : 0;
+      keep = before < S_new;
+    }
+    s_pos[j] = keep;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int per = (S_old + 31) / 32, b = lane * per, en = min(S_old, b + per);
+    int cnt = 0;
+    for (int j = b; j < en; ++j) cnt += s_pos[j];
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - cnt;
+    for (int j = b; j < en; ++j) {
+      const int k = s_pos[j];
+      s_pos[j] = k ? run : -1;
+      run += k;
+    }
+    if (lane == 31) ws[0] = incl;
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < S_old; j += blockDim.x) {
+    const int n = s_pos[j];
+    if (n < 0) continue;
+    eos_new[n] = s_eos[j];
+    lu_new[n] = s_lu[j];
+    soe_new[s_eos[j]] = n;
+    ws[1 + n] = j;
+  }
+}
+
+// Bank moves of a resize: new slot y <- old slot ws[1 + y] for y < ws[0];
+// blockIdx.y = new slot, blocks along x stride over the bank in 16-byte vectors.
+__global__ void bank_move_kernel(const uint8_t* __restrict__ old_pool, uint8_t* __restrict__ new_pool,
+                                 size_t bank_bytes, const int32_t* __restrict__ ws) {
+  pdl_wait();
+  pdl_trigger();
+  const int y = blockIdx.y;
+  if (y >= ws[0]) return;
+  const uint4* src = reinterpret_cast<const uint4*>(old_pool + static_cast<size_t>(ws[1 + y]) * bank_bytes);
+  uint4* dst = reinterpret_cast<uint4*>(new_pool + static_cast<size_t>(y) * bank_bytes);
+  const size_t n = bank_bytes / 16;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    dst[i] = src[i];
+}
+
+cudaError_t launch_slot_resize(int E, int S_old, const int32_t* eos_old, const int64_t* lu_old, int S_new,
+                               int32_t* soe_new, int32_t* eos_new, int64_t* lu_new, const void* old_pool,
+                               void* new_pool, size_t bank_bytes, int32_t* ws, cudaStream_t st) {
+  const size_t smem = (sizeof(int64_t) + 2 * sizeof(int32_t)) * static_cast<size_t>(S_old);
+  cudaError_t err =
+      cudaFuncSetAttribute(slot_resize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  err = launch_pdl(slot_resize_kernel, dim3(1), dim3(kLruThreads), smem, st, E, S_old, eos_old, lu_old, S_new,
+                   soe_new, eos_new, lu_new, ws);
+  if (err != cudaSuccess) return err;
+  const int moves = S_old < S_new ? S_old : S_new;
+  const size_t vec = bank_bytes / 16;
+  const int bx = static_cast<int>((vec + 256 * 16 - 1) / (256 * 16) < 64 ? (vec + 256 * 16 - 1) / (256 * 16) : 64);
+  return launch_pdl(bank_move_kernel, dim3(bx > 0 ? bx : 1, moves), dim3(256), 0, st,
+                    static_cast<const uint8_t*>(old_pool), static_cast<uint8_t*>(new_pool), bank_bytes,
+                    static_cast<const int32_t*>(ws));
+}
+
 }  // namespace ftm

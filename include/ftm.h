@@ -163,6 +163,29 @@ ftm_status ftm_slot_lookup_update(const ftm_layer_desc* L, ftm_slot_cache* C, co
                                   int32_t T, void* workspace, size_t ws_bytes, void* compute_stream,
                                   void* copy_stream);
 
+/* Elastic slot-pool resize: move the cache to S_new slots at run time without
+ * reloading weights from the host (pomoai.com FreeToken hub, two-level expert
+ * memory: the expert cache's VRAM share changes while the engine runs;
+ * freelamp.com FreeToken article, section 2.3 "elastic memory management",
+ * `ftctl cache --moe <slots>`).  The pages give no rule for which experts stay;
+ * this library keeps the min(S_new, resident) most recently used resident
+ * experts (largest last_use first, ties to the lower old slot), compacted into
+ * slots 0.. in their old slot order with their last_use, and evicts the rest.
+ *   L          the layer with the OLD slot count (L->S = S_old)
+ *   C          the current cache (read: state arrays and slot_pool)
+ *   S_new      1 <= S_new <= 4096
+ *   C_new      caller-owned new state: slot_of_expert [E], expert_of_slot
+ *              [S_new], last_use [S_new] (device) and slot_pool (S_new banks),
+ *              none overlapping C's; host_pool / host_scratch may be C's.  On
+ *              success C_new->step = C->step and its counters are zeroed.
+ *   workspace  device, >= ftm_slot_workspace_bytes(L) bytes, 256-aligned
+ * Enqueues on `stream`, with no host synchronisation, one kernel that writes
+ * the new state and the move list and one that copies the kept banks
+ * device-to-device.  Afterwards use C_new with a layer desc whose S = S_new;
+ * C's arrays and pool may be released once the stream has passed this call. */
+ftm_status ftm_slot_resize(const ftm_layer_desc* L, const ftm_slot_cache* C, int32_t S_new, ftm_slot_cache* C_new,
+                           void* workspace, size_t ws_bytes, void* stream);
+
 /* Grouped SwiGLU expert FFN (a5, a6, a7).
  *   x              device [T][d] activations (token order)
  *   offsets, perm  from ftm_permute

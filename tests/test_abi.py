@@ -105,3 +105,26 @@ def test_gate_up_paired_rows_brute_force():
         b, rl = r // 128, r % 128
         want = gate[64 * b + rl] if rl < 64 else up[64 * b + rl - 64]
         assert (paired[r] == want).all()
+
+
+def test_slot_resize_rejected_without_gpu():
+    cfg = synth.CONFIGS["284b_trace"]
+    d = ftm.desc_for(cfg)
+    bb = ftm.ftm_get_bank_layout(d).bank_bytes
+    lib = ftm.library()
+    # fake, never dereferenced device addresses: the checks fail before any launch
+    old = ftm.SlotCache(0x100000, 0x200000, 0x300000, 7, 0x10_0000_0000, 0x4000_0000, 0x5000_0000, 0, 0, 0, 0)
+    new_pool = 0x10_0000_0000 + bb * cfg.S          # right after the old pool: no overlap
+    new = ftm.SlotCache(0x600000, 0x700000, 0x800000, 0, new_pool, 0x4000_0000, 0x5000_0000, 0, 0, 0, 0)
+    ws = 0x9000_0000
+    nbytes = ftm.ftm_slot_workspace_bytes(d)
+    assert lib.ftm_slot_resize(None, ctypes.byref(old), 8, ctypes.byref(new), ws, nbytes, None) == 1
+    assert lib.ftm_slot_resize(ctypes.byref(d), ctypes.byref(old), 0, ctypes.byref(new), ws, nbytes, None) == 1
+    assert lib.ftm_slot_resize(ctypes.byref(d), ctypes.byref(old), 5000, ctypes.byref(new), ws, nbytes, None) == 2
+    bad = ftm.SlotCache(0x600000, 0x700000, 0x800000, 0, 0x10_0000_0000 + bb, 0, 0, 0, 0, 0, 0)  # overlaps
+    assert lib.ftm_slot_resize(ctypes.byref(d), ctypes.byref(old), 8, ctypes.byref(bad), ws, nbytes, None) == 1
+    assert "overlap" in ftm.ftm_last_error()
+    same = ftm.SlotCache(0x100000, 0x700000, 0x800000, 0, new_pool, 0, 0, 0, 0, 0, 0)            # shared state array
+    assert lib.ftm_slot_resize(ctypes.byref(d), ctypes.byref(old), 8, ctypes.byref(same), ws, nbytes, None) == 1
+    assert lib.ftm_slot_resize(ctypes.byref(d), ctypes.byref(old), 8, ctypes.byref(new), ws, nbytes - 8, None) == 1
+    assert lib.ftm_slot_resize(ctypes.byref(d), ctypes.byref(old), 8, ctypes.byref(new), None, nbytes, None) == 1
