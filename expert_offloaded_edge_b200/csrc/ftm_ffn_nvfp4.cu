@@ -491,7 +491,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // MMA at N = the next multiple of 32 above its token count.
 // No TMA multicast: every CTA loads its own tiles.
 // ---------------------------------------------------------------------------
-constexpr int kQN = 224;                        // tokens per pair tile (padded block)
+constexpr int kQN = 224;                        // tokens per pair tile (padded block; a multiple of the 32-row scale groups)
 constexpr int kQH = kQN / 2;                    // token rows staged per CTA
 constexpr uint32_t kQABytes = 128 * 128;        // 128 weight rows x 256 e2m1
 constexpr uint32_t kQBBytes = kQH * 128;        // 112 token rows x 256 e2m1
@@ -499,7 +499,9 @@ constexpr uint32_t kQSfaBytes = 4 * kSfChunk;   // 4 K64 chunks of this CTA's 12
 constexpr uint32_t kQSfbBytes = 8 * kSfChunk;   // 4 K64 chunks x 2 halves of the token block
 constexpr uint32_t kQStage = kQABytes + kQBBytes + kQSfaBytes + kQSfbBytes;
 constexpr int kQStages = 5;
-constexpr uint32_t kQSfCol = 2 * kQN;           // TMEM: accumulators [0, 448), scales [448, 496)
+constexpr uint32_t kQSfCol = 2 * kQN;           // TMEM: accumulators [0, 448), two half-stage scale slots [448, 496)
+constexpr uint32_t kQSfHalfCols = 24;           // one half stage (2 K steps): SFA 2 x 4 columns + SFB 2 x 8 columns
+constexpr int kQThreads = 224;                  // warps 0 TMA, 1 MMA, 2-5 epilogue, 6 scale copies
 
 __device__ __forceinline__ int quad_tile_n(int valid) { return min(kQN, (valid + 31) & ~31); }
 
@@ -520,8 +522,14 @@ __device__ __forceinline__ void tmem_cp_sf2(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
+// Arrive on this CTA's barrier once the executing thread's pair operations complete.
+__device__ __forceinline__ void umma2_commit_local(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
 template <bool GATED>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kQThreads, 1)
     ffn_nvfp4_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAsh,
                          const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmSfa,
                          const __grid_constant__ CUtensorMap tmSfaSh, const __grid_constant__ CUtensorMap tmSfb,
@@ -535,6 +543,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kQStages], empty_bar[kQStages], tfull_bar[2], tempty_bar[2];
+  // Scale copies and MMAs run from different threads.  Half h of a stage (K steps 2h, 2h + 1) always uses
+  // scale slot h: sf_ready[h * kQStages + stage] = that half's scales are in TMEM, sf_free[h] = the MMAs that
+  // read slot h are done, so the copies of one half overlap the MMAs of the other.
+  __shared__ __align__(8) uint64_t sf_ready[2 * kQStages], sf_free[2];
   __shared__ uint32_t tmem_holder;
   __shared__ int32_t tile_start[kMaxGroups + 1], grp_rows[kMaxGroups], grp_row0[kMaxGroups];
   __shared__ float xbuf[GATED ? 128 * 17 : 1];
@@ -553,8 +565,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int K64 = K / 64;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kQStages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 8); }
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+      mbar_init(&sf_ready[s], 1);
+      mbar_init(&sf_ready[kQStages + s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 8);
+      mbar_init(&sf_free[a], 1);
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -634,7 +655,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
-      const uint32_t sfa_t = tmem_base + kQSfCol, sfb_t = tmem_base + kQSfCol + 16;
+      int g = 0;   // stages consumed so far (the scale set of stage g is g % 2)
       for (int t = pair; t < total && ok; t += npairs, ++it) {
         const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, kQN);
         const uint32_t idesc = idesc_nvf4(256, quad_tile_n(min(kQN, ti.rows - ti.n * kQN)));
@@ -643,25 +664,59 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!mbar_wait_cl(&tempty_bar[ab], aphase ^ 1u)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + ab * kQN;
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = 0; kb < KB; ++kb, ++g) {
           if (!mbar_wait_cl(&full_bar[stage], phase)) { ok = false; break; }
-          tc_fence_after();
           const uint32_t sa = smem_u32(a_tile(stage)), sb = smem_u32(b_tile(stage));
-          const uint32_t ssa = smem_u32(sfa_tile(stage)), ssb = smem_u32(sfb_tile(stage));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            tmem_cp_sf2(sfa_t + 4 * kk, smem_desc_sf(ssa + kk * kSfChunk));
-            tmem_cp_sf2(sfb_t + 8 * kk, smem_desc_sf(ssb + kk * kSfChunk));
-            tmem_cp_sf2(sfb_t + 8 * kk + 4, smem_desc_sf(ssb + 4 * kSfChunk + kk * kSfChunk));
+          for (int h = 0; h < 2; ++h) {
+            if (!mbar_wait_cl(&sf_ready[h * kQStages + stage], phase)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sf = tmem_base + kQSfCol + h * kQSfHalfCols;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int kk = 2 * h + j;
+              umma2_nvf4(d, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32), idesc, sf + 4 * j,
+                         sf + 8 + 8 * j, (kb | kk) != 0 ? 1u : 0u);
+            }
+            umma2_commit_local(&sf_free[h]);
           }
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma2_nvf4(d, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32), idesc, sfa_t + 4 * kk,
-                       sfb_t + 8 * kk, (kb | kk) != 0 ? 1u : 0u);
+          if (!ok) break;
           umma2_commit_both(&empty_bar[stage]);
           if (++stage == kQStages) { stage = 0; phase ^= 1u; }
         }
         if (ok) umma2_commit_both(&tfull_bar[ab]);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 6) {
+    // the even CTA copies each stage's scales into TMEM (both CTAs) ahead of the MMA thread
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int g = 0;
+      for (int t = pair; t < total && ok; t += npairs) {
+        for (int kb = 0; kb < KB; ++kb, ++g) {
+          if (!mbar_wait_cl(&full_bar[stage], phase)) { ok = false; break; }
+          const uint32_t ssa = smem_u32(sfa_tile(stage)), ssb = smem_u32(sfb_tile(stage));
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            // slot h is free once the MMAs of the previous stage's half h are done
+            if (g >= 1 && !mbar_wait_cl(&sf_free[h], static_cast<uint32_t>(g - 1) & 1u)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sf = tmem_base + kQSfCol + h * kQSfHalfCols;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int kk = 2 * h + j;
+              tmem_cp_sf2(sf + 4 * j, smem_desc_sf(ssa + kk * kSfChunk));
+              tmem_cp_sf2(sf + 8 + 8 * j, smem_desc_sf(ssb + kk * kSfChunk));
+              tmem_cp_sf2(sf + 8 + 8 * j + 4, smem_desc_sf(ssb + 4 * kSfChunk + kk * kSfChunk));
+            }
+            umma2_commit_local(&sf_ready[h * kQStages + stage]);
+          }
+          if (!ok) break;
+          if (++stage == kQStages) { stage = 0; phase ^= 1u; }
+        }
       }
     }
     __syncwarp();
@@ -851,7 +906,7 @@ static cudaError_t launch_nvfp4_tc2_one(const CUtensorMap* maps, const FfnArgs& 
   const int G = a.E + (a.has_shared ? 1 : 0);
   const long tiles = static_cast<long>((P + kQN - 1) / kQN + G) * (Nw / (GATED ? 128 : 256));
   cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kTcThreads);
+  cfg.blockDim = dim3(kQThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
