@@ -53,6 +53,13 @@ def lib():
         L.orc_dequant_nvfp4.argtypes = [p, p, ctypes.c_float, i32, i32, p]
         L.orc_qa_fp8_g128.argtypes = [p, i32, i32]
         L.orc_qa_nvfp4_g16.argtypes = [p, i32, i32]
+        L.orc_e8m0_value.argtypes = [ctypes.c_uint8]
+        L.orc_e8m0_value.restype = ctypes.c_double
+        L.orc_mx_scale_code.argtypes = [p, i32]
+        L.orc_mx_scale_code.restype = ctypes.c_uint8
+        L.orc_quant_mxfp4.argtypes = [p, i32, i32, p, p]
+        L.orc_dequant_mxfp4.argtypes = [p, p, i32, i32, p]
+        L.orc_qa_mxfp4_g32.argtypes = [p, i32, i32]
         L.orc_router_logits.argtypes = [p, i32, i32, p, p, i32, p]
         L.orc_margin_ok.argtypes = [p, i32, i32, i32, ctypes.c_double, p]
         L.orc_topk_gates.argtypes = [p, i32, i32, i32, p, p]
@@ -136,6 +143,41 @@ def qa_nvfp4(v: np.ndarray) -> np.ndarray:
     v = _f32(v).copy()
     rows, K = v.reshape(-1, v.shape[-1]).shape
     lib().orc_qa_nvfp4_g16(_p(v), rows, K)
+    return v
+
+
+def e8m0_value(c: int) -> float:
+    return float(lib().orc_e8m0_value(c))
+
+
+def mx_scale_code(v: np.ndarray) -> int:
+    v = _f32(v).ravel().copy()
+    return int(lib().orc_mx_scale_code(_p(v), v.size))
+
+
+def quant_mxfp4(w: np.ndarray):
+    """w [R][C] (C a multiple of 32) -> (packed e2m1 [R][C/2], E8M0 scale codes [R][C/32])."""
+    w = _f32(w)
+    R, C = w.shape
+    q = np.empty((R, C // 2), dtype=np.uint8)
+    s = np.empty((R, C // 32), dtype=np.uint8)
+    lib().orc_quant_mxfp4(_p(w), R, C, _p(q), _p(s))
+    return q, s
+
+
+def dequant_mxfp4(qp: np.ndarray, s: np.ndarray) -> np.ndarray:
+    qp = np.ascontiguousarray(qp, dtype=np.uint8)
+    s = np.ascontiguousarray(s, dtype=np.uint8)
+    R, C = qp.shape[0], qp.shape[1] * 2
+    out = np.empty((R, C), dtype=np.float32)
+    lib().orc_dequant_mxfp4(_p(qp), _p(s), R, C, _p(out))
+    return out
+
+
+def qa_mxfp4(v: np.ndarray) -> np.ndarray:
+    v = _f32(v).copy()
+    rows, K = v.reshape(-1, v.shape[-1]).shape
+    lib().orc_qa_mxfp4_g32(_p(v), rows, K)
     return v
 
 

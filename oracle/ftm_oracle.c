@@ -184,6 +184,70 @@ void orc_qa_nvfp4_g16(float* v, int rows, int K) {
 }
 
 /* ---------------------------------------------------------------------------
+ * MXFP4 (pomoai.com FreeToken hub, checkpoint list: the engine loads MXFP4,
+ * NVFP4, FP8 and BF16 checkpoints).  The format is the OCP Microscaling (MX)
+ * v1.0 one: blocks of 32 consecutive elements along a row share one E8M0
+ * scale X = 2^(e - 127) (code 255 is NaN) and each element is E2M1.
+ * Quantisation of a block (the specification's conversion rule): the shared
+ * exponent is floor(log2(max |v|)) minus the largest E2M1 exponent (2),
+ * clamped to the E8M0 range [-127, 127]; each element is v / X rounded to
+ * the nearest E2M1 value, ties to even, saturating at 6.  Reading for an
+ * all-zero block (the specification leaves the exponent of zero open):
+ * scale code 127 (X = 1) and zero elements.
+ * ------------------------------------------------------------------------- */
+
+double orc_e8m0_value(uint8_t c) { return c == 255 ? NAN : ldexp(1.0, (int)c - 127); }
+
+/* Shared-scale code of one block of n values. */
+uint8_t orc_mx_scale_code(const float* v, int n) {
+  float amax = 0.0f;
+  for (int j = 0; j < n; ++j) if (fabsf(v[j]) > amax) amax = fabsf(v[j]);
+  if (amax == 0.0f) return 127;
+  int e = (int)floor(log2((double)amax)) - 2;
+  if (e < -127) e = -127;
+  if (e > 127) e = 127;
+  return (uint8_t)(e + 127);
+}
+
+/* w [R][C] -> packed codes q [R][C/2] (element 2j in the low nibble) and
+ * scale codes s [R][C/32]. */
+void orc_quant_mxfp4(const float* w, int R, int C, uint8_t* q, uint8_t* s) {
+  for (int r = 0; r < R; ++r)
+    for (int b = 0; b < C / 32; ++b) {
+      const float* p = w + (int64_t)r * C + b * 32;
+      uint8_t sc = orc_mx_scale_code(p, 32);
+      s[(int64_t)r * (C / 32) + b] = sc;
+      double X = orc_e8m0_value(sc);
+      for (int j = 0; j < 32; j += 2) {
+        uint8_t lo = orc_e2m1_encode((float)(p[j] / X)), hi = orc_e2m1_encode((float)(p[j + 1] / X));
+        q[(int64_t)r * (C / 2) + (b * 32 + j) / 2] = (uint8_t)(lo | (hi << 4));
+      }
+    }
+}
+
+/* w[r][c] = e2m1(q) * 2^(s[r][c/32] - 127). */
+void orc_dequant_mxfp4(const uint8_t* qp, const uint8_t* s, int R, int C, float* out) {
+#pragma omp parallel for schedule(static)
+  for (int r = 0; r < R; ++r)
+    for (int c = 0; c < C; ++c) {
+      uint8_t byte = qp[(int64_t)r * (C / 2) + c / 2];
+      uint8_t nib = (c & 1) ? (byte >> 4) : (byte & 15);
+      out[(int64_t)r * C + c] = (float)(orc_e2m1_all[nib] * orc_e8m0_value(s[(int64_t)r * (C / 32) + c / 32]));
+    }
+}
+
+/* MXFP4 activations, in place: each 32-group of a row is replaced by its
+ * quantised-then-dequantised values. */
+void orc_qa_mxfp4_g32(float* v, int rows, int K) {
+  for (int r = 0; r < rows; ++r)
+    for (int b = 0; b < K / 32; ++b) {
+      float* p = v + (int64_t)r * K + b * 32;
+      double X = orc_e8m0_value(orc_mx_scale_code(p, 32));
+      for (int j = 0; j < 32; ++j) p[j] = (float)(orc_e2m1_value(orc_e2m1_encode((float)(p[j] / X))) * X);
+    }
+}
+
+/* ---------------------------------------------------------------------------
  * Router: logits, top-k, gates.
  * ------------------------------------------------------------------------- */
 

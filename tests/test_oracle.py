@@ -383,6 +383,58 @@ def test_lru_resize_then_steps_match_list_replay():
         assert rc == 0 and m == rm
 
 
+def test_e8m0_decode():
+    assert oracle.e8m0_value(127) == 1.0
+    assert oracle.e8m0_value(0) == 2.0 ** -127 and oracle.e8m0_value(254) == 2.0 ** 127
+    assert oracle.e8m0_value(130) == 8.0
+    assert math.isnan(oracle.e8m0_value(255))
+
+
+def test_mxfp4_hand_worked_block():
+    v = np.zeros(32, dtype=np.float32)
+    v[:6] = [3.0, 1.0, 0.3, -1.25, 2.5 * 0.5, 5.0 * 0.5]
+    # amax 3: shared exponent floor(log2 3) - 2 = -1, X = 0.5; v/X = 6, 2, 0.6, -2.5, 2.5, 5
+    assert oracle.mx_scale_code(v) == 126
+    q, s = oracle.quant_mxfp4(v.reshape(1, 32))
+    w = oracle.dequant_mxfp4(q, s)[0]
+    # 0.6 -> 0.5; -2.5 and 2.5 tie between 2 and 3 -> 2 (even code); 5 ties between 4 and 6 -> 4
+    assert w[:6].tolist() == [3.0, 1.0, 0.25, -1.0, 1.0, 2.0]
+    assert not w[6:].any()
+    # saturation: amax 7.5 -> X = 1, 7.5 -> 6
+    v2 = np.zeros((1, 32), dtype=np.float32)
+    v2[0, 0] = 7.5
+    q, s = oracle.quant_mxfp4(v2)
+    assert s[0, 0] == 127 and oracle.dequant_mxfp4(q, s)[0, 0] == 6.0
+    # an all-zero block: scale code 127, zero codes
+    q, s = oracle.quant_mxfp4(np.zeros((1, 32), dtype=np.float32))
+    assert s[0, 0] == 127 and not q.any()
+    # the scale exponent clamps to the E8M0 range
+    assert oracle.mx_scale_code(np.full(32, 1e-40, np.float32)) == 0
+
+
+def test_mxfp4_invariants_and_brute_force_elements():
+    rng = np.random.default_rng(7)
+    grid = np.array([oracle.e2m1_value(c) for c in range(16)])
+    for scale in (1e-3, 0.02, 1.0, 300.0):
+        v = (rng.standard_normal((4, 96)) * scale).astype(np.float32)
+        q, s = oracle.quant_mxfp4(v)
+        w = oracle.dequant_mxfp4(q, s)
+        for r in range(4):
+            for b in range(3):
+                blk = v[r, b * 32:(b + 1) * 32].astype(np.float64)
+                X = oracle.e8m0_value(int(s[r, b]))
+                assert math.log2(X) == int(math.log2(X))
+                # normalisation: the largest magnitude lands on 4 or 6 in units of X
+                assert np.abs(w[r, b * 32:(b + 1) * 32]).max() / X in (4.0, 6.0)
+                for j in range(32):
+                    t = blk[j] / X
+                    d = np.abs(grid - t)
+                    cands = [c for c in range(16) if d[c] == d.min()]
+                    want = grid[min(cands, key=lambda c: (c & 7) & 1)] if abs(t) <= 6 else math.copysign(6.0, t)
+                    assert w[r, b * 32 + j] == np.float32(want * X), (scale, r, b, j, t)
+    assert np.array_equal(oracle.qa_mxfp4(v), w)
+
+
 # ---------------------------------------------------------------------------
 # Expert FFN and combine
 # ---------------------------------------------------------------------------
