@@ -20,8 +20,12 @@
  *    weight formats.
  * The pages give no formula for the layer; the arithmetic below is the plain
  * reading of a top-k routed SwiGLU MoE layer (router logits + bias, softmax,
- * top-k, renormalise over the k picks, SwiGLU experts, gate-weighted sum), with
- * every silent point resolved as listed in the design notes.
+ * top-k, renormalise over the k picks, SwiGLU experts, gate-weighted sum).
+ * Where the pages are silent, the reading taken is stated in the comment of
+ * the function concerned: bias added to the logit before selection and
+ * gating; picks in descending logit order with ties to the lower id; a stable
+ * permutation by flat pair index; silu on the gate projection; the routing
+ * gate applied after the down projection; the shared expert with weight 1.
  *
  * Precision: products and sums in double, results rounded to float.
  * Parallelism: OpenMP over independent tokens/rows only (no reordering of any

@@ -473,6 +473,107 @@ def test_ffn_gate_and_up_not_swapped():
     assert np.allclose(c[0, :5], z / (1 + np.exp(-z)) * z, rtol=1e-6)
 
 
+def _silu(z):
+    return z / (1.0 + math.exp(-z))
+
+
+def test_ffn_fp8_activation_quantisation_hand_worked():
+    # FP8 mode (qa = 1): x is quantised per 128-group before the gate/up
+    # contraction and h = silu(g) * u per 128-group before the down
+    # contraction; the down output is not quantised.
+    d = I = 128
+    x = np.zeros((1, d), np.float32)
+    x[0, :4] = [448.0, 1.0625, 17.0, -0.3]
+    # group amax 448 -> s = 1; e4m3 RNE: 1.0625 -> 1.0 (tie, even mantissa),
+    # 17 -> 16 (tie, even), -0.3 -> -0.3125 (nearest in steps of 2^-5)
+    Wg = np.zeros((I, d), np.float32)
+    Wu = np.zeros((I, d), np.float32)
+    Wg[0, 1] = 1.0          # g0 = q(x1) = 1
+    Wu[0, 2] = 0.125        # u0 = q(x2) / 8 = 2
+    Wg[1, 3] = 1.0          # g1 = q(x3) = -0.3125
+    Wu[1, 0] = 2.0 ** -8    # u1 = 448 / 256 = 1.75
+    Wd = np.zeros((d, I), np.float32)
+    Wd[0, 0] = 1.0
+    Wd[1, 1] = 1.0
+    Wd[2, 0], Wd[2, 1] = 0.3, 1.0
+    y = oracle.expert_ffn(x, Wg, Wu, Wd, oracle.QA_FP8)[0].astype(np.float64)
+    h0 = _silu(1.0) * 2.0
+    h1 = _silu(-0.3125) * 1.75
+    # h's 128-group: amax h0 -> s = h0/448; h0 -> 448 s; h1/s = -70.8 -> -72 (e4m3 step 8 in [64, 128))
+    s = float(np.float32(np.float32(h0) / np.float32(448.0)))
+    want = np.zeros(d)
+    want[0] = 448.0 * s
+    want[1] = -72.0 * s
+    want[2] = 0.3 * 448.0 * s - 72.0 * s
+    assert np.allclose(y, want, rtol=1e-6, atol=1e-7)
+    # plausible slips each move an entry well beyond that tolerance:
+    no_qx = _silu(1.0625) * 2.125                           # x not quantised
+    assert abs(y[0] - no_qx) > 0.1
+    assert abs(y[1] - h1) > 1e-3                             # h not quantised
+    g1_q = -144.0 / 448.0                                    # g, u quantised (before SiLU) instead of h
+    assert abs(y[1] - _silu(g1_q) * 1.75) > 1e-3
+    assert abs(y[2] - 64.0 * s) > 1e-3                       # down output quantised too (62.4 -> 64)
+
+
+def test_ffn_nvfp4_activation_quantisation_hand_worked():
+    # NVFP4 mode (qa = 2): 16-groups with an e4m3 group scale e4m3(amax/6) and
+    # e2m1 elements, on x and on h; exact dyadic results.
+    d, I = 32, 16
+    x = np.zeros((1, d), np.float32)
+    x[0, :3] = [6.0, 2.5, 0.75]       # amax 6 -> s16 = 1: 2.5 -> 2, 0.75 -> 1 (ties to even codes)
+    x[0, 16:19] = [3.0, 1.3, -0.4]    # amax 3 -> s16 = 0.5: 1.3 -> 1.5, -0.4 -> -0.5
+    Wg = np.zeros((I, d), np.float32)
+    Wu = np.zeros((I, d), np.float32)
+    Wg[0, 1], Wu[0, 17] = 1.0, 1.0    # g0 = 2, u0 = 1.5
+    Wg[1, 2], Wu[1, 18] = 1.0, 1.0    # g1 = 1, u1 = -0.5
+    Wd = np.zeros((d, I), np.float32)
+    Wd[0, 0] = 1.0
+    Wd[1, 1] = 1.0
+    Wd[2, 0], Wd[2, 1] = 1.0, 1.0
+    y = oracle.expert_ffn(x, Wg, Wu, Wd, oracle.QA_NVFP4)[0]
+    # h = (silu(2) * 1.5, silu(1) * -0.5) = (2.6424, -0.3655): amax/6 = 0.4404 -> s16 = 0.4375;
+    # 6.04 -> 6 and -0.835 -> -1 in units of s16
+    want = np.zeros(d, np.float32)
+    want[:3] = [2.625, -0.4375, 2.1875]
+    assert np.array_equal(y, want)
+    assert abs(y[0] - 3.0) > 0.1                 # x not quantised gives h0 -> 3.0 after quantising h
+    assert abs(y[0] - _silu(2.0) * 1.5) > 1e-2   # h not quantised
+    # down output quantised too: 2.1875 / 0.4375 = 5 -> 4 (tie to even) -> 1.75
+    assert abs(y[2] - 1.75) > 0.1
+
+
+@pytest.mark.parametrize("qa,d,I", [(1, 256, 128), (2, 64, 48)])
+def test_ffn_activation_quantised_composes_pinned_pieces(qa, d, I):
+    # The quantised FFN equals the composition of the separately pinned
+    # quantisers with an fp64 library matmul: qa(x) -> gate/up -> silu(g)*u ->
+    # qa(h) -> down.  Swapping the order of any stage breaks it.
+    rng = np.random.default_rng(7 + qa)
+    n = 5
+    x = rng.normal(size=(n, d)).astype(np.float32)
+    Wg, Wu = (rng.normal(0, 0.05, size=(I, d)).astype(np.float32) for _ in range(2))
+    Wd = rng.normal(0, 0.05, size=(d, I)).astype(np.float32)
+    q = oracle.qa_fp8 if qa == 1 else oracle.qa_nvfp4
+    y = oracle.expert_ffn(x, Wg, Wu, Wd, qa).astype(np.float64)
+    xq = q(x).astype(np.float64)
+    g = xq @ Wg.T.astype(np.float64)
+    u = xq @ Wu.T.astype(np.float64)
+    h = (g / (1.0 + np.exp(-g)) * u).astype(np.float32)
+    want = q(h).astype(np.float64) @ Wd.T.astype(np.float64)
+    assert np.allclose(y, want, rtol=1e-5, atol=1e-6)
+    scale = np.abs(want).max()
+    # x skipped
+    g0, u0 = x.astype(np.float64) @ Wg.T.astype(np.float64), x.astype(np.float64) @ Wu.T.astype(np.float64)
+    alt = q((g0 / (1 + np.exp(-g0)) * u0).astype(np.float32)).astype(np.float64) @ Wd.T.astype(np.float64)
+    assert np.abs(y - alt).max() > 1e-3 * scale
+    # quantising g and u before SiLU instead of h
+    gq, uq = q(g.astype(np.float32)).astype(np.float64), q(u.astype(np.float32)).astype(np.float64)
+    alt = (gq / (1 + np.exp(-gq)) * uq) @ Wd.T.astype(np.float64)
+    assert np.abs(y - alt).max() > 1e-3 * scale
+    # quantising the down output as well
+    alt = q(want.astype(np.float32)).astype(np.float64)
+    assert np.abs(y - alt).max() > 1e-3 * scale
+
+
 def test_combine_hand_example():
     y = np.array([[1, 2], [3, 4]], dtype=np.float32)
     g = np.array([[0.25, 0.75]], dtype=np.float32)
