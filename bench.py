@@ -2,24 +2,36 @@
 """Benchmark of one routed-MoE layer forward pass (route -> permute -> [slot
 cache step] -> grouped SwiGLU FFN -> combine) on B200, through the C ABI.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--T T]
-    python bench.py --impl reference ...      # the CPU oracle on the host cores
+    python bench.py [--gpus N] [--steps K] [--warmup W]          # headline + every workload (N = 1)
+    python bench.py --config NAME [--T T] ...                    # one workload only
+    python bench.py --impl reference ...                         # the CPU oracle on the host cores
 
-One step = one layer pass over one batch of T tokens.  N > 1 (torchrun): every
-rank runs its own replica on its own batch (tokens are independent, no data
-collective); value = all ranks' tokens / max-over-ranks time.  Prints one JSON
-line on rank 0.
+One step = one layer pass over one batch of T tokens.  The headline is the
+largest layer, the 753B-class NVFP4 layer at T = 16384; at N = 1 the line also
+carries one record per other workload (35B decode T = 1/8/32/64, 35B prefill,
+the 284B FP8 slot-cache trace, 753B NVFP4 decode), each timed the same way.
+N > 1 (torchrun): every rank runs its own replica of the headline on its own
+batch (tokens are independent, no data collective); value = all ranks' tokens
+/ max-over-ranks time.  Prints one JSON line on rank 0.
+
+Timing: W untimed warm-up steps, every CUDA graph captured, then exactly K
+steps between CUDA events on the launching stream, synchronised on both sides
+(barrier + max over ranks for N > 1).  Workloads whose expert bytes per step
+are below 3x the L2 size rotate over that many copies of the slot pool, so
+no step finds its weights in L2.
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 import numpy as np
@@ -34,19 +46,25 @@ import synth  # noqa: E402
 METRIC = "MoE-layer tokens/s; decode HBM GB/s & prefill TFLOP/s as % of B200 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
+HEADLINE = ("753b_nvfp4", 16384)
+SUITE = (("35b_decode", (1, 8, 32, 64)), ("35b_prefill", (8192,)), ("284b_trace", (32,)), ("753b_nvfp4", (16,)))
+K_BREAKDOWN = 40
 
 
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=None, help="timed steps (default: ~1.5 s worth)")
-    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--steps", type=int, default=20, help="timed steps per workload")
+    p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="ftm", choices=["ftm", "reference"])
-    p.add_argument("--config", default="35b_decode", choices=list(synth.CONFIGS))
-    p.add_argument("--T", type=int, default=None, help="tokens per step (default: the config's largest)")
+    p.add_argument("--config", default=None, choices=list(synth.CONFIGS),
+                   help="run this workload only (default: the headline and, at N = 1, every workload)")
+    p.add_argument("--T", type=int, default=None, help="tokens per step with --config (default: its largest)")
     p.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying CUDA graphs")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--cpu-seconds", type=float, default=6.0, help="per CPU-baseline mode")
+    p.add_argument("--bank-cache", default=os.path.join(tempfile.gettempdir(), "ftm_bench_banks"),
+                   help="directory for packed expert banks reused across runs ('' = off)")
     return p.parse_args()
 
 
@@ -56,19 +74,20 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, interval_ms: int = 50):
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         try:
             self.p = subprocess.Popen(["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.FIELDS}",
-                                       "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                                       "--format=csv,noheader,nounits", "-lms", str(interval_ms)], stdout=self.f,
                                       stderr=subprocess.DEVNULL)
         except (OSError, ValueError):
             self.p = None
+        time.sleep(0.3)     # let the first sample land before the timed region starts
 
     def stop(self) -> dict:
         if self.p is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.25)
+        time.sleep(0.1)
         self.p.terminate()
         try:
             self.p.wait(timeout=5)
@@ -126,6 +145,16 @@ def ncu_traffic(workload: str, kernel: str, wdtype: str):
     return e.get("dram_bytes_per_launch")
 
 
+def dtype_peak(pk: dict, src: str, wdtype: str):
+    """Dense tensor peak of a dtype (TFLOP/s) and where it comes from: the measured
+    sustained bf16 figure times the nominal dense ratio for fp8 (2) and fp4 (4)."""
+    bf16 = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+    ratio = {"f32": 1.0, "bf16": 1.0, "fp8": 2.0, "nvfp4": 4.0}[wdtype]
+    where = (f"{src} bf16_tflops_sustained" if ratio == 1.0 else
+             f"derived: {ratio:g} x {src} bf16_tflops_sustained (nominal dense ratio)")
+    return bf16 * ratio, where
+
+
 # --------------------------------------------------------------------------- ranks
 def job_throughput(local_ms: float, units_per_rank: int, dist, device) -> tuple:
     """Whole-job throughput of N independent replicas: the slowest rank's time
@@ -140,9 +169,104 @@ def job_throughput(local_ms: float, units_per_rank: int, dist, device) -> tuple:
     return ms, units_per_rank * world / (ms / 1e3)
 
 
-# --------------------------------------------------------------------------- workload
+# --------------------------------------------------------------------------- layers
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in ("synth/gen.c", "synth/__init__.py", "expert_offloaded_edge_b200/layout.py"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def packed_banks(cfg, cache_dir: str, local_rank: int, dist):
+    """The layer's packed banks, drawn once and kept on the host's disk so later
+    runs (and the other ranks of this one) read them instead of drawing again."""
+    from synth.device import pack_banks
+    if not cache_dir:
+        return None
+    path = os.path.join(cache_dir, f"{cfg.name}_{source_hash()}_{hashlib.sha1(repr(cfg).encode()).hexdigest()[:8]}.npy")
+    if local_rank == 0 and not os.path.exists(path):
+        try:
+            os.makedirs(cache_dir, exist_ok=True)
+            banks = pack_banks(cfg)
+            tmp = path + f".tmp{os.getpid()}"
+            np.save(tmp, banks)
+            os.replace(tmp, path)
+        except OSError:
+            pass
+    if dist is not None:
+        dist.barrier()
+    if os.path.exists(path):
+        return np.load(path, mmap_mode="r")
+    return None
+
+
+def device_layer(cfg, args, local, dist):
+    from synth.device import DeviceLayer
+    return DeviceLayer(cfg, banks=packed_banks(cfg, args.bank_cache, local, dist))
+
+
 def workload_name(cfg, T):
     return f"{cfg.name} T={T}"
+
+
+def workload_config(cfg, T, world):
+    """The config block of a line: the same for this arm and the reference arm."""
+    return {"workload": workload_name(cfg, T), "d": cfg.d, "E": cfg.E, "k": cfg.k, "I": cfg.I, "T": T,
+            "has_shared": cfg.has_shared, "S": cfg.S, "wdtype": cfg.wdtype, "seed": 0,
+            "parallelism": f"replicas x{world}"}
+
+
+def routing_stats(dl, T, x):
+    """Per-expert load of the benchmarked batch, from the library's own routing."""
+    cfg = dl.cfg
+    ids = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
+    gw = torch.empty((T, cfg.k), dtype=torch.float32, device="cuda")
+    ftm.ftm_route(dl.desc, x, T, dl.w_router, dl.bias, ids, gw)
+    torch.cuda.synchronize()
+    return np.bincount(ids.cpu().numpy().ravel(), minlength=cfg.E)
+
+
+def algorithmic(cfg, bl, T, counts):
+    """Algorithmic bytes and flops of GEMM1 and of the whole layer step.  Bytes:
+    the weight bytes of every expert touched (gate/up, down and their scales,
+    i.e. its bank) plus the activations each GEMM reads and writes once."""
+    wb = {"f32": 4, "bf16": 2, "fp8": 1, "nvfp4": 0.5}[cfg.wdtype]
+    ab = 4 if cfg.act_dtype == "f32" else 2
+    groups = int((counts > 0).sum()) + (1 if cfg.has_shared else 0)
+    rows = T * cfg.k + (T if cfg.has_shared else 0)
+    g1_w = 2 * cfg.I * cfg.d * wb + bl.s_gu_bytes + bl.s_t_bytes
+    g2_w = cfg.d * cfg.I * wb + bl.s_d_bytes
+    g1_bytes = groups * g1_w + rows * cfg.d * ab + rows * cfg.I * ab
+    g2_bytes = groups * g2_w + rows * cfg.I * ab + rows * cfg.d * ab
+    router_bytes = cfg.E * cfg.d * ab
+    g1_flops = 2.0 * rows * cfg.d * 2 * cfg.I
+    g2_flops = 2.0 * rows * cfg.I * cfg.d
+    return {"groups": groups, "rows": rows, "gemm1_bytes": g1_bytes, "gemm2_bytes": g2_bytes,
+            "layer_bytes": g1_bytes + g2_bytes + router_bytes + T * cfg.d * ab * 2,
+            "weight_bytes": groups * (g1_w + g2_w), "gemm1_flops": g1_flops, "gemm2_flops": g2_flops,
+            "layer_flops": g1_flops + g2_flops + 2.0 * T * cfg.E * cfg.d}
+
+
+def rooflines(cfg, alg, g1_ms, step_ms, decode: bool):
+    pk, src = peaks()
+    if decode:
+        peak = float(pk["hbm_gbs"])
+        ach = alg["gemm1_bytes"] / (g1_ms * 1e-3) / 1e9
+        lay = alg["layer_bytes"] / (step_ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                "kernel": "gemm1 (grouped gate/up + SwiGLU)", "algorithmic_bytes": alg["gemm1_bytes"],
+                "peak_source": f"{src} hbm_gbs (of {src})",
+                "layer": {"achieved": lay, "frac": lay / peak, "algorithmic_bytes": alg["layer_bytes"],
+                          "what": "expert banks touched + router + activations, per step, over ms_per_step"}}
+    peak, where = dtype_peak(pk, src, cfg.wdtype)
+    ach = alg["gemm1_flops"] / (g1_ms * 1e-3) / 1e12
+    lay = alg["layer_flops"] / (step_ms * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+            "kernel": "gemm1 (grouped gate/up + SwiGLU)", "algorithmic_flops": alg["gemm1_flops"],
+            "peak_source": where,
+            "layer": {"achieved": lay, "frac": lay / peak, "algorithmic_flops": alg["layer_flops"],
+                      "what": "router + gate/up + down flops per step, over ms_per_step"}}
 
 
 class Runner:
@@ -150,31 +274,45 @@ class Runner:
 
     `kernels` are the kernel ids whose launches are bracketed by events; the
     timed region instruments only the dominant kernel (each event is one more
-    graph node), a separate pass after it instruments all of them."""
+    graph node), a separate pass after it instruments all of them.  Steps
+    rotate over `replicas` copies of the slot pool."""
 
     ALL = (ftm.binding.FTM_K_ROUTE, ftm.binding.FTM_K_PERMUTE, ftm.binding.FTM_K_GATHER,
            ftm.binding.FTM_K_GEMM1, ftm.binding.FTM_K_GEMM2, ftm.binding.FTM_K_COMBINE)
 
-    def __init__(self, dl, T, use_graph: bool, chunk: int = 20):
+    def __init__(self, dl, T, x, use_graph: bool, replicas: int = 1, chunk: int = 20):
         from synth.device import Workspace
         self.dl, self.T = dl, T
-        self.x = dl.hidden(T)
+        self.x = x
         self.out = torch.empty((T, dl.cfg.d), dtype=dl.out_dtype(), device="cuda")
         self.ws = Workspace(ftm.ftm_workspace_bytes(dl.desc, T))
-        self.weights = dl.weights()
+        self.pools = [dl.pool] + [dl.pool.clone() for _ in range(replicas - 1)]
+        bias = None if dl.bias is None else dl.bias.data_ptr()
+        shared = None if dl.shared_bank is None else dl.shared_bank.data_ptr()
+        self.weights = [ftm.LayerWeights(dl.w_router.data_ptr(), bias, p.data_ptr(), dl.slot_of_expert.data_ptr(),
+                                         shared) for p in self.pools]
         self.use_graph = use_graph
         self.chunk = chunk
         self.graphs = {}
         self.stream = torch.cuda.Stream()
-        self.KERNELS = (ftm.binding.FTM_K_GEMM1,)
+        self.kernels = (ftm.binding.FTM_K_GEMM1,)
 
-    def _step(self):
-        ftm.ftm_moe_layer_forward(self.dl.desc, self.weights, None, self.x, self.T, self.out, self.ws.ptr,
-                                  self.ws.nbytes, self.stream)
+    def step(self, i, x=None, out=None, stream=None):
+        ftm.ftm_moe_layer_forward(self.dl.desc, self.weights[i % len(self.weights)], None,
+                                  self.x if x is None else x, self.T, self.out if out is None else out,
+                                  self.ws.ptr, self.ws.nbytes, self.stream if stream is None else stream)
+
+    def launches_per_step(self) -> int:
+        torch.cuda.synchronize()
+        n0 = ftm.ftm_kernel_launches()
+        self.step(0)
+        n1 = ftm.ftm_kernel_launches()
+        torch.cuda.synchronize()
+        return n1 - n0
 
     def _events(self, n):
         evs = [{k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for k in self.KERNELS} for _ in range(n)]
+                for k in self.kernels} for _ in range(n)]
         # torch creates the CUDA event on its first record(); the library re-records it later
         for ev in evs:
             for a, b in ev.values():
@@ -184,25 +322,39 @@ class Runner:
         return evs
 
     def _record_steps(self, evs):
-        for ev in evs:
+        for i, ev in enumerate(evs):
             for k, (a, b) in ev.items():
                 ftm.ftm_set_profile_events(k, a, b)
-            self._step()
-        for k in self.KERNELS:
+            self.step(i)
+        for k in self.kernels:
             ftm.ftm_set_profile_events(k, None, None)
 
-    def _graph(self, n, tag):
-        key = (n, tag, self.KERNELS)
-        if key not in self.graphs:
+    def _plan(self, nsteps):
+        out, done, tag = [], 0, 0
+        while done < nsteps:
+            n = min(self.chunk, nsteps - done)
+            out.append((n, tag))
+            tag ^= 1
+            done += n
+        return out
+
+    def prepare(self, nsteps):
+        """Capture every graph run(nsteps) replays (before any timed region)."""
+        if not self.use_graph:
+            return
+        for n, tag in self._plan(nsteps):
+            key = (n, tag, self.kernels)
+            if key in self.graphs:
+                continue
             evs = self._events(n)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.stream(self.stream):
-                self._step()          # first launch outside capture (sets kernel attributes)
+                self.step(0)          # one launch outside capture (sets kernel attributes)
                 self.stream.synchronize()
                 with torch.cuda.graph(g, stream=self.stream):
                     self._record_steps(evs)
             self.graphs[key] = (g, evs)
-        return self.graphs[key]
+        torch.cuda.synchronize()
 
     def run(self, nsteps: int, collect: dict = None):
         """Enqueue nsteps steps on self.stream; per-kernel ms appended to collect."""
@@ -216,24 +368,19 @@ class Runner:
                 self.stream.synchronize()
                 self._collect(evs, collect)
             return
-        done = 0
         pending = []
-        tag = 0
-        while done < nsteps:
-            n = min(self.chunk, nsteps - done)
-            g, evs = self._graph(n, tag)
+        for n, tag in self._plan(nsteps):
+            g, evs = self.graphs[(n, tag, self.kernels)]     # captured by prepare()
             if len(pending) == 2:     # the graph about to be replayed last ran two chunks ago
                 pe = pending.pop(0)
                 if collect is not None:
-                    pe[-1][self.KERNELS[-1]][1].synchronize()
+                    pe[-1][self.kernels[-1]][1].synchronize()
                     self._collect(pe, collect)
             g.replay()
             pending.append(evs)
-            tag ^= 1
-            done += n
         if collect is not None:
             for pe in pending:
-                pe[-1][self.KERNELS[-1]][1].synchronize()
+                pe[-1][self.kernels[-1]][1].synchronize()
                 self._collect(pe, collect)
 
     @staticmethod
@@ -243,123 +390,132 @@ class Runner:
                 collect.setdefault(k, []).append(a.elapsed_time(b))
 
 
-def routing_stats(dl, T):
-    """Active experts of the benchmarked batch, from the library's own routing."""
-    cfg = dl.cfg
-    x = dl.hidden(T)
-    ids = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
-    gw = torch.empty((T, cfg.k), dtype=torch.float32, device="cuda")
-    ftm.ftm_route(dl.desc, x, T, dl.w_router, dl.bias, ids, gw)
+def e2e_pipelined(r: Runner, steps: int, dist):
+    """End to end through the public call, every step: its tokens copied in from
+    pinned host memory, the layer, its output copied back to pinned host
+    memory.  Two buffer sets and separate copy streams let step i's copies run
+    while step i +- 1 computes (PCIe is full duplex)."""
+    T = r.T
+    xs_h = [torch.empty_like(r.x, device="cpu").pin_memory() for _ in range(2)]
+    for xh in xs_h:
+        xh.copy_(r.x)
+    outs_h = [torch.empty_like(r.out, device="cpu").pin_memory() for _ in range(2)]
+    xs_d = [r.x, torch.empty_like(r.x)]
+    outs_d = [r.out, torch.empty_like(r.out)]
+    h2d, d2h, comp = torch.cuda.Stream(), torch.cuda.Stream(), r.stream
+    ev_h = [torch.cuda.Event() for _ in range(2)]
+    ev_c = [torch.cuda.Event() for _ in range(2)]
+    ev_d = [torch.cuda.Event() for _ in range(2)]
+
+    def run(n):
+        for i in range(n):
+            b = i % 2
+            if i >= 2:
+                h2d.wait_event(ev_c[b])           # step i-2 has read xs_d[b]
+            with torch.cuda.stream(h2d):
+                xs_d[b].copy_(xs_h[b], non_blocking=True)
+            ev_h[b].record(h2d)
+            comp.wait_event(ev_h[b])
+            if i >= 2:
+                comp.wait_event(ev_d[b])          # step i-2's output has left outs_d[b]
+            r.step(i, x=xs_d[b], out=outs_d[b], stream=comp)
+            ev_c[b].record(comp)
+            d2h.wait_event(ev_c[b])
+            with torch.cuda.stream(d2h):
+                outs_h[b].copy_(outs_d[b], non_blocking=True)
+            ev_d[b].record(d2h)
+
+    run(3)
     torch.cuda.synchronize()
-    counts = np.bincount(ids.cpu().numpy().ravel(), minlength=cfg.E)
-    return counts
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(h2d)
+    run(steps)
+    t1.record(d2h)
+    torch.cuda.synchronize()
+    ms, value = job_throughput(t0.elapsed_time(t1), steps * T, dist, "cuda")
+    nb_in = r.x.numel() * r.x.element_size()
+    nb_out = r.out.numel() * r.out.element_size()
+    return {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": nb_in, "d2h_bytes_per_step": nb_out,
+            "steps": steps, "ms_per_step": ms / steps,
+            "launch": "eager ftm_moe_layer_forward; tokens in and outputs out through pinned host memory every "
+                      "step, copies on their own streams overlapping the neighbouring steps' compute"}
 
 
-def algorithmic(dl, T, counts):
-    """Algorithmic bytes and flops of GEMM1 and of the whole step."""
+def run_resident(dl, T, args, dist, local):
+    """One resident-layer workload: warm-up, graphs captured, K timed steps, a
+    per-kernel breakdown pass and the end-to-end pass."""
     cfg = dl.cfg
-    wb = {"f32": 4, "bf16": 2, "fp8": 1, "nvfp4": 0.5}[cfg.wdtype]
-    ab = 4 if cfg.act_dtype == "f32" else 2
-    groups = int((counts > 0).sum()) + (1 if cfg.has_shared else 0)
-    rows = T * cfg.k + (T if cfg.has_shared else 0)
-    g1_bytes = groups * 2 * cfg.I * cfg.d * wb + rows * cfg.d * ab + rows * cfg.I * ab
-    g2_bytes = groups * cfg.d * cfg.I * wb + rows * cfg.I * ab + rows * cfg.d * ab
-    g1_flops = 2.0 * rows * cfg.d * 2 * cfg.I
-    g2_flops = 2.0 * rows * cfg.I * cfg.d
-    return {"groups": groups, "rows": rows, "gemm1_bytes": g1_bytes, "gemm2_bytes": g2_bytes,
-            "gemm1_flops": g1_flops, "gemm2_flops": g2_flops}
+    K, W = args.steps, args.warmup
+    x = dl.hidden(T)
+    counts = routing_stats(dl, T, x)
+    alg = algorithmic(cfg, dl.bl, T, counts)
+    replicas = max(1, min(8, math.ceil(3 * L2_BYTES / max(1, alg["weight_bytes"]))))
+    r = Runner(dl, T, x, not args.no_graph, replicas=replicas)
+    per_step_launches = r.launches_per_step()
+    with torch.cuda.stream(r.stream):
+        for i in range(W):
+            r.step(i)
+    r.prepare(K)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    per_kernel = {}
+    t0.record(r.stream)
+    r.run(K, per_kernel)
+    t1.record(r.stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    clk = clocks.stop()
+    ms, value = job_throughput(ms, K * T, dist, "cuda")
+    # per-kernel breakdown, after the timed region (every kernel bracketed by events)
+    r.kernels = Runner.ALL
+    r.prepare(K_BREAKDOWN)
+    breakdown = {}
+    r.run(K_BREAKDOWN, breakdown)
+    torch.cuda.synchronize()
+    e2e = e2e_pipelined(r, K, dist)
+    status = ftm.ftm_device_status(True)
+    kms = {ftm.KERNEL_NAMES[k]: float(np.mean(v)) for k, v in per_kernel.items()}
+    kbreak = {ftm.KERNEL_NAMES[k]: float(np.mean(v)) for k, v in breakdown.items()}
+    decode = alg["rows"] / max(1, alg["groups"]) < 64
+    roof = rooflines(cfg, alg, kms.get("gemm1", float("nan")), ms / K, decode)
+    roof["traffic"] = ncu_traffic(workload_name(cfg, T), "gemm1", cfg.wdtype)
+    step_bytes = alg["weight_bytes"] * replicas
+    rec = {
+        "workload": workload_name(cfg, T), "value": value, "unit": "tokens/s", "ms_per_step": ms / K, "steps": K,
+        "warmup": W, "dtype": cfg.wdtype, "config": workload_config(cfg, T, dist.get_world_size() if dist else 1),
+        "l2": (f"inputs larger than L2: {alg['weight_bytes'] / 1e9:.3f} GB of expert banks per step"
+               + (f", rotating over {replicas} copies of the slot pool ({step_bytes / 1e9:.2f} GB per cycle)"
+                  if replicas > 1 else "")),
+        "launch": "CUDA graph replay (graphs captured before the timed region)" if r.use_graph else "eager",
+        "routing": {"active_experts": int((counts > 0).sum()), "rows": alg["rows"],
+                    "max_rows_per_expert": int(counts.max()), "min_rows_active": int(counts[counts > 0].min())},
+        "roofline": roof, "kernels_ms": kms, "kernels_ms_breakdown": kbreak, "e2e": e2e,
+        "gpu_launches": per_step_launches * K, "launches_per_step": per_step_launches, "clocks": clk,
+        "device_status": status,
+    }
+    if cfg.name == "35b_prefill":
+        rec["routing"]["per_expert_rows"] = counts.tolist()
+    return rec
 
 
-# --------------------------------------------------------------------------- CPU oracle
-def oracle_tokens_per_s(cfg, T, seconds: float, step_tokens: int = 1):
-    """The oracle layer (router for the sampled tokens, their k experts and the
-    shared expert, combine) on the host cores; returns (tokens/s, tokens, cores, s)."""
-    import oracle
-    layer = synth.Layer(cfg, 0, synth.load_redraws(cfg.name, max(cfg.T)) or {})
-    x_all = layer.hidden_f32(T)
-    Wr = layer.router_f32()
-    b = layer.bias()
-    cache = {}
-    done, t_used = 0, 0.0
-    t = 0
-    while t_used < seconds:
-        rows = [(t + i) % T for i in range(step_tokens)]
-        xs = x_all[rows]
-        # dequantised weights are the layer's stored parameters: load them outside the timed part
-        ids, g, _ = oracle.route(xs, Wr, b, cfg.k)
-        for e in set(ids.ravel().tolist()) | ({cfg.E} if cfg.has_shared else set()):
-            if e not in cache:
-                cache[e] = oracle.expert_weights_f32(layer, e)
-        t0 = time.perf_counter()
-        ids, g, _ = oracle.route(xs, Wr, b, cfg.k)
-        oracle.moe_rows(layer, xs, range(len(rows)), ids, g, weight_cache=cache)
-        t_used += time.perf_counter() - t0
-        done += len(rows)
-        t += step_tokens
-        if len(cache) > 48:
-            cache.clear()
-    return done / t_used, done, oracle.threads(), t_used
-
-
-def reference_arm(args, rank, world):
-    if rank != 0:
-        return
-    if args.steps is None:
-        args.steps = 20
-    cfg = synth.CONFIGS[args.config]
-    T = args.T or max(cfg.T)
-    import oracle
-    layer = synth.Layer(cfg, 0, synth.load_redraws(cfg.name, max(cfg.T)) or {})
-    x_all = layer.hidden_f32(T)
-    Wr = layer.router_f32()
-    b = layer.bias()
-    cache = {}
-
-    def step(i):
-        rows = [i % T]
-        xs = x_all[rows]
-        ids, g, _ = oracle.route(xs, Wr, b, cfg.k)
-        for e in set(ids.ravel().tolist()) | ({cfg.E} if cfg.has_shared else set()):
-            if e not in cache:
-                cache[e] = oracle.expert_weights_f32(layer, e)
-        t0 = time.perf_counter()
-        ids, g, _ = oracle.route(xs, Wr, b, cfg.k)
-        oracle.moe_rows(layer, xs, range(1), ids, g, weight_cache=cache)
-        dt = time.perf_counter() - t0
-        if len(cache) > 48:
-            cache.clear()
-        return dt
-
-    for i in range(args.warmup):
-        step(i)
-    tot = sum(step(args.warmup + i) for i in range(args.steps))
-    v = args.steps / tot
-    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64-accumulate/f32",
-            "data": "synthetic", "config": {"workload": workload_name(cfg, T), "d": cfg.d, "E": cfg.E, "k": cfg.k,
-                                            "I": cfg.I, "T": T, "wdtype": cfg.wdtype},
-            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
-                             "sample": f"each step = 1 token of the {workload_name(cfg, T)} batch through the full "
-                                       f"oracle layer (router, {cfg.k} experts, combine)"},
-            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-    print(json.dumps(line), flush=True)
-
-
-# --------------------------------------------------------------------------- slot-cache trace
-def trace_main(args, cfg, T, rank, world, local, dist):
+def run_trace(cfg, T, args, dist, local):
     """The decode trace over the LRU slot cache: one step = route, permute, cache
     update with miss copies (host sync), FFN, combine.  Warm-up = the first W
     steps of the trace, timed = the next K with the tokens resident in HBM,
-    then end to end = the K2 steps after those, each step copying its tokens
-    from pinned host memory and its output back (K + K2 + W <= trace length)."""
-    from synth.device import DeviceLayer, Workspace
-    dl = DeviceLayer(cfg)
-    W = args.warmup
-    K = args.steps if args.steps is not None else (cfg.trace_steps - W) // 2
-    K = max(1, min(K, cfg.trace_steps - W - 1))
-    K2 = max(1, min(K, cfg.trace_steps - W - K))
-    args.steps = K
+    then end to end = the K steps after those, each step copying its tokens
+    from pinned host memory and its output back (2K + W <= trace length)."""
+    from synth.device import Workspace
+    dl = device_layer(cfg, args, local, dist)
+    W = min(args.warmup, cfg.trace_steps - 2)
+    K = max(1, min(args.steps, (cfg.trace_steps - W) // 2))
+    K2 = K
     xs = [dl.hidden(T, step=s) for s in range(W + K)]
     xs_host = [dl.hidden(T, step=s).cpu().pin_memory() for s in range(W + K, W + K + K2)]
     ws = Workspace(ftm.ftm_workspace_bytes(dl.desc, T))
@@ -377,12 +533,11 @@ def trace_main(args, cfg, T, rank, world, local, dist):
             ftm.ftm_set_profile_events(ftm.binding.FTM_K_GEMM1, None, None)
         return dl.cache.last_hits, dl.cache.last_misses, dl.cache.last_distinct
 
+    n0 = ftm.ftm_kernel_launches()
     for s in range(W):
         step(s)
+    launches_warm = (ftm.ftm_kernel_launches() - n0) / max(1, W)
     torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    clocks = ClockSampler(local)
     evs = []
     for _ in range(K):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -390,19 +545,23 @@ def trace_main(args, cfg, T, rank, world, local, dist):
         b.record(stream)
         evs.append((a, b))
     torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = ClockSampler(local)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     hits = misses = distinct = 0
+    n0 = ftm.ftm_kernel_launches()
     t0.record(stream)
     for i in range(K):
         h, m, dct = step(W + i, evs[i])
         hits, misses, distinct = hits + h, misses + m, distinct + dct
     t1.record(stream)
     torch.cuda.synchronize()
+    launches = ftm.ftm_kernel_launches() - n0
     ms = t0.elapsed_time(t1)
     clk = clocks.stop()
     g1 = [a.elapsed_time(b) for a, b in evs]
     ms, value = job_throughput(ms, K * T, dist, "cuda")
-    # end to end: the next K2 steps through the public call with host tokens in and out
     x_dev = torch.empty_like(xs[0])
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -418,40 +577,157 @@ def trace_main(args, cfg, T, rank, world, local, dist):
     torch.cuda.synchronize()
     e2e_ms, e2e_value = job_throughput(e0.elapsed_time(e1), K2 * T, dist, "cuda")
     status = ftm.ftm_device_status(True)
-    if rank != 0:
-        return
     pk, src = peaks()
-    # GEMM1 bytes of one step: (distinct routed experts + the shared expert) x gate/up bytes
-    alg_g1 = (distinct / K + 1) * 2 * cfg.I * cfg.d * 1 + (T * cfg.k + T) * (cfg.d + cfg.I)
+    # GEMM1 bytes of one step: (distinct routed experts + the shared expert) x gate/up bytes (+ scales)
+    g1_w = 2 * cfg.I * cfg.d + bl.s_gu_bytes
+    g2_w = cfg.d * cfg.I + bl.s_d_bytes
+    groups = distinct / K + 1
+    rows = T * cfg.k + T
+    alg_g1 = groups * g1_w + rows * (cfg.d + cfg.I) * 2
+    layer_bytes = groups * (g1_w + g2_w) + rows * (cfg.d + cfg.I) * 4 + cfg.E * cfg.d * 2 + 2 * T * cfg.d * 2
     g1_ms = float(np.mean(g1))
     ach = alg_g1 / (g1_ms * 1e-3) / 1e9
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
-        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.wdtype,
-        "data": "synthetic decode trace (seeded generator, Zipf(1.1) router bias)",
-        "config": {"workload": workload_name(cfg, T) + f" trace steps {W}..{W + K - 1}", "d": cfg.d, "E": cfg.E,
-                   "k": cfg.k, "I": cfg.I, "T": T, "S": cfg.S, "wdtype": cfg.wdtype,
-                   "l2": "inputs larger than L2: ~1.1 GB of FP8 expert weights touched per step",
-                   "launch": "eager (one host sync per step to read the miss list)",
-                   "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "achieved": ach, "peak": float(pk["hbm_gbs"]), "unit": "GB/s",
-                     "frac": ach / float(pk["hbm_gbs"]), "kernel": "gemm1 (fp8 grouped gate/up + SwiGLU)",
-                     "algorithmic_bytes": alg_g1, "peak_source": f"{src} hbm_gbs",
-                     "traffic": ncu_traffic(workload_name(cfg, T), "gemm1", cfg.wdtype)},
+    peak = float(pk["hbm_gbs"])
+    return {
+        "workload": workload_name(cfg, T) + f" trace steps {W}..{W + K - 1}", "value": value, "unit": "tokens/s",
+        "ms_per_step": ms / K, "steps": K, "warmup": W, "dtype": cfg.wdtype,
+        "config": workload_config(cfg, T, dist.get_world_size() if dist else 1),
+        "l2": "inputs larger than L2: ~1.1 GB of FP8 expert banks touched per step",
+        "launch": "eager (one host sync per step to read the miss list)",
+        "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                     "kernel": "gemm1 (fp8 grouped gate/up + SwiGLU)", "algorithmic_bytes": alg_g1,
+                     "peak_source": f"{src} hbm_gbs (of {src})",
+                     "traffic": ncu_traffic(workload_name(cfg, T), "gemm1", cfg.wdtype),
+                     "layer": {"achieved": layer_bytes / (ms / K * 1e-3) / 1e9,
+                               "frac": layer_bytes / (ms / K * 1e-3) / 1e9 / peak, "algorithmic_bytes": layer_bytes,
+                               "what": "expert banks touched per step over the step time, which includes the "
+                                       "PCIe miss copies the step waits for"}},
         "cache": {"hit_rate": hits / max(1, distinct), "misses_per_step": misses / K,
                   "h2d_gb_per_step": misses / K * bl.bank_bytes / 1e9,
                   "h2d_gbs_effective": misses * bl.bank_bytes / (ms * 1e-3) / 1e9},
-        "cpu_baseline": None,
         "e2e": {"value": e2e_value, "unit": "tokens/s",
                 "h2d_bytes_per_step": int(xs_host[0].numel() * xs_host[0].element_size()),
                 "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size()),
                 "steps": K2, "trace_steps": f"{W + K}..{W + K + K2 - 1}",
                 "launch": "eager; tokens copied in from pinned host memory and the output copied out every step, "
                           "on top of the miss copies the step already makes"},
-        "gpu_launches": 7 * K,
-        "clocks": clk,
-        "device_status": status,
+        "gpu_launches": int(launches), "launches_per_step": launches / K, "launches_per_warmup_step": launches_warm,
+        "clocks": clk, "device_status": status,
     }
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+class OracleTokens:
+    """The oracle layer on one token at a time (router, its k experts, the shared
+    expert, combine), on the first `ntok` tokens of the batch.  Their experts'
+    weights are dequantised once, outside any timing: they are the layer's
+    stored parameters."""
+
+    def __init__(self, cfg, ntok: int = 2):
+        import oracle
+        self.oracle = oracle
+        self.cfg = cfg
+        self.layer = synth.Layer(cfg, 0, synth.load_redraws(cfg.name, max(cfg.T)) or {})
+        self.x = self.layer.hidden_f32(ntok)
+        self.Wr = self.layer.router_f32()
+        self.b = self.layer.bias()
+        ids, _, _ = oracle.route(self.x, self.Wr, self.b, cfg.k)
+        want = set(ids.ravel().tolist()) | ({cfg.E} if cfg.has_shared else set())
+        self.cache = {e: oracle.expert_weights_f32(self.layer, e) for e in sorted(want)}
+
+    def token(self, t: int):
+        o = self.oracle
+        xs = self.x[t % len(self.x)][None, :]
+        ids, g, _ = o.route(xs, self.Wr, self.b, self.cfg.k)
+        o.moe_rows(self.layer, xs, [0], ids, g, weight_cache=self.cache)
+
+    def timed(self, threads: int, seconds: float = None, per_thread: int = None):
+        """Tokens processed by `threads` host threads (one oracle thread each), for
+        `seconds` of wall time or `per_thread` tokens each; returns (tokens, s)."""
+        done = [0] * threads
+
+        def work(j):
+            self.oracle.set_threads(1)
+            n = 0
+            while True:
+                if per_thread is not None and n >= per_thread:
+                    break
+                if seconds is not None and time.perf_counter() - t0 >= seconds:
+                    break
+                self.token(j + n * threads)
+                n += 1
+            done[j] = n
+
+        th = [threading.Thread(target=work, args=(j,)) for j in range(threads)]
+        t0 = time.perf_counter()
+        for t in th:
+            t.start()
+        for t in th:
+            t.join()
+        return sum(done), time.perf_counter() - t0
+
+
+def cpu_baseline(cfg, T, seconds: float):
+    ot = OracleTokens(cfg)
+    ot.timed(1, per_thread=1)                     # warm
+    n1, s1 = ot.timed(1, seconds=seconds)
+    cores = host_cores()
+    nc, sc = ot.timed(cores, seconds=seconds)
+    return {"value": nc / sc, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "single_thread": {"value": n1 / s1, "unit": "tokens/s", "tokens": n1, "seconds": s1},
+            "all_cores": {"value": nc / sc, "unit": "tokens/s", "tokens": nc, "seconds": sc, "threads": cores},
+            "cpu_model": cpu_model(),
+            "sample": (f"tokens 0..{len(ot.x) - 1} of the {workload_name(cfg, T)} batch, one token per oracle layer "
+                       f"call (router, {cfg.k} experts{', shared expert' if cfg.has_shared else ''}, combine), "
+                       f"{seconds:g} s on 1 thread, then {seconds:g} s on {cores} threads; expert weights "
+                       f"dequantised beforehand")}
+
+
+def reference_arm(args, rank, world):
+    """The oracle as it stands, timed on the host cores on the same workload:
+    each step = one token per host core, all cores at once."""
+    if rank != 0:
+        return
+    name, T = (args.config, args.T or max(synth.CONFIGS[args.config].T)) if args.config else HEADLINE
+    cfg = synth.CONFIGS[name]
+    ot = OracleTokens(cfg)
+    cores = host_cores()
+    for _ in range(args.warmup):
+        ot.timed(cores, per_thread=1)
+    tot = 0.0
+    for _ in range(args.steps):
+        tot += ot.timed(cores, per_thread=1)[1]
+    v = args.steps * cores / tot
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64-accumulate/f32",
+            "data": "synthetic (seeded generator, weights N(0,0.02^2))",
+            "config": workload_config(cfg, T, world),
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "cpu_model": cpu_model(),
+                             "sample": f"each step = {cores} tokens of the {workload_name(cfg, T)} batch (tokens "
+                                       f"0..{len(ot.x) - 1} in turn), one per host thread, each through the full "
+                                       f"oracle layer (router, {cfg.k} experts"
+                                       f"{', shared expert' if cfg.has_shared else ''}, combine)"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
@@ -463,142 +739,65 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return reference_arm(args, rank, world)
+    args.warmup = max(args.warmup, 3)
     torch.cuda.set_device(local)
     dist = None
     if world > 1:
         import datetime
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    cfg = synth.CONFIGS[args.config]
-    T = args.T or max(cfg.T)
-    if cfg.lru:
-        return trace_main(args, cfg, T, rank, world, local, dist)
-    from synth.device import DeviceLayer
-    dl = DeviceLayer(cfg)
-    counts = routing_stats(dl, T)
-    alg = algorithmic(dl, T, counts)
-    use_graph = not args.no_graph
-    r = Runner(dl, T, use_graph)
-
-    # warm-up (untimed)
-    r.run(args.warmup)
-    torch.cuda.synchronize()
-    if args.steps is None:
-        # enough steps for ~1.5 s of timed work, so the clock sampler sees the load
-        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        p0.record(r.stream)
-        r.run(20)
-        p1.record(r.stream)
-        torch.cuda.synchronize()
-        est = p0.elapsed_time(p1) / 20
-        steps = int(min(20000, max(50, 1500.0 / max(est, 1e-3))))
-        if dist:
-            tt = torch.tensor([steps], device="cuda")
-            dist.all_reduce(tt, op=dist.ReduceOp.MIN)
-            steps = int(tt.item())
-        args.steps = steps
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    clocks = ClockSampler(local)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    per_kernel = {}
-    t0.record(r.stream)
-    r.run(args.steps, per_kernel)
-    t1.record(r.stream)
-    torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1)
-    clk = clocks.stop()
-    ms, value = job_throughput(ms, args.steps * T, dist, "cuda")
-    if dist:
-        dist.barrier()
-
-    # per-kernel breakdown (after the timed region; every kernel bracketed by events)
-    r.KERNELS = Runner.ALL
-    breakdown = {}
-    r.run(40, breakdown)
-    torch.cuda.synchronize()
-
-    # end to end: host x -> device, forward, device out -> host, every step (eager, public API)
-    x_host = torch.empty_like(r.x, device="cpu").pin_memory()
-    x_host.copy_(r.x)
-    out_host = torch.empty_like(r.out, device="cpu").pin_memory()
-    e_steps = max(1, min(args.steps, 50))
-    s = r.stream
-    with torch.cuda.stream(s):
-        for _ in range(3):
-            r.x.copy_(x_host, non_blocking=True)
-            r._step()
-            out_host.copy_(r.out, non_blocking=True)
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s)
-    with torch.cuda.stream(s):
-        for _ in range(e_steps):
-            r.x.copy_(x_host, non_blocking=True)
-            r._step()
-            out_host.copy_(r.out, non_blocking=True)
-    e1.record(s)
-    torch.cuda.synchronize()
-    e_ms, e2e_value = job_throughput(e0.elapsed_time(e1), e_steps * T, dist, "cuda")
-    status = ftm.ftm_device_status(True)
-
-    if rank == 0:
-        pk, src = peaks()
-        kms = {ftm.KERNEL_NAMES[k]: float(np.mean(v)) for k, v in per_kernel.items()}
-        kbreak = {ftm.KERNEL_NAMES[k]: float(np.mean(v)) for k, v in breakdown.items()}
-        decode = alg["rows"] / max(1, alg["groups"]) < 64
-        g1 = kms.get("gemm1", float("nan"))
-        if decode:
-            ach = alg["gemm1_bytes"] / (g1 * 1e-3) / 1e9
-            peak = float(pk["hbm_gbs"])
-            roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-                    "kernel": "gemm1 (grouped gate/up + SwiGLU)", "algorithmic_bytes": alg["gemm1_bytes"],
-                    "peak_source": f"{src} hbm_gbs"}
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    if args.config:
+        head = (args.config, args.T or max(synth.CONFIGS[args.config].T))
+        suite = ()
+    else:
+        head = HEADLINE
+        suite = SUITE if world == 1 else ()
+    records = []
+    head_rec = None
+    head_cfg = synth.CONFIGS[head[0]]
+    for name, Ts in suite:
+        cfg = synth.CONFIGS[name]
+        if cfg.lru:
+            for T in Ts:
+                records.append(run_trace(cfg, T, args, dist, local))
+            continue
+        dl = device_layer(cfg, args, local, dist)
+        for T in Ts:
+            records.append(run_resident(dl, T, args, dist, local))
+        if name == head[0]:
+            head_rec = run_resident(dl, head[1], args, dist, local)
+        del dl
+        torch.cuda.empty_cache()
+    if head_rec is None:
+        if head_cfg.lru:
+            head_rec = run_trace(head_cfg, head[1], args, dist, local)
         else:
-            ach = alg["gemm1_flops"] / (g1 * 1e-3) / 1e12
-            bf16 = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
-            # a contraction takes its own dtype's peak: the measured bf16 figure times the
-            # nominal dense ratio (fp8 4.5/2.25 = 2, fp4 9/2.25 = 4), labelled as derived
-            ratio = {"f32": 1.0, "bf16": 1.0, "fp8": 2.0, "nvfp4": 4.0}[cfg.wdtype]
-            peak = bf16 * ratio
-            roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
-                    "kernel": "gemm1 (grouped gate/up + SwiGLU)", "algorithmic_flops": alg["gemm1_flops"],
-                    "peak_source": (f"{src} bf16_tflops_sustained" if ratio == 1.0 else
-                                    f"derived: {ratio:g} x {src} bf16_tflops_sustained (nominal dense ratio)")}
-        roof["traffic"] = ncu_traffic(workload_name(cfg, T), "gemm1", cfg.wdtype)
+            dl = device_layer(head_cfg, args, local, dist)
+            head_rec = run_resident(dl, head[1], args, dist, local)
+            del dl
+    if rank == 0:
         cpu = None
         if not args.no_cpu_baseline and world == 1:
-            v, n, cores, secs = oracle_tokens_per_s(cfg, T, args.cpu_seconds)
-            cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                   "sample": f"{n} tokens of the same batch, one token per oracle call, {secs:.1f} s of CPU work"}
-        step_bytes = alg["gemm1_bytes"] + alg["gemm2_bytes"]
+            cpu = cpu_baseline(head_cfg, head[1], args.cpu_seconds)
         line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": cfg.wdtype, "data": "synthetic (seeded generator, weights N(0,0.02^2))",
-            "config": {"workload": workload_name(cfg, T), "d": cfg.d, "E": cfg.E, "k": cfg.k, "I": cfg.I, "T": T,
-                       "wdtype": cfg.wdtype, "active_experts": alg["groups"],
-                       "l2": (f"inputs larger than L2: {step_bytes / 1e9:.2f} GB of expert weights touched per step"
-                              if step_bytes > 4 * L2_BYTES else "working set below 4x L2 (not flushed)"),
-                       "launch": "CUDA graph replay" if use_graph else "eager", "parallelism": f"replicas x{world}"},
-            "roofline": roof,
-            "step_hbm_gbs": step_bytes / (ms / args.steps * 1e-3) / 1e9,
-            "kernels_ms": kms,
-            "kernels_ms_breakdown": kbreak,
+            "metric": METRIC, "value": head_rec["value"], "unit": "tokens/s", "n_gpus": world,
+            "steps": head_rec["steps"], "warmup": head_rec["warmup"], "ms_per_step": head_rec["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": head_rec["dtype"],
+            "data": "synthetic (seeded generator, weights N(0,0.02^2), hidden N(0,1))",
+            "config": dict(head_rec["config"], l2=head_rec["l2"], launch=head_rec["launch"]),
+            "roofline": head_rec["roofline"],
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": r.x.numel() * r.x.element_size(),
-                    "d2h_bytes_per_step": r.out.numel() * r.out.element_size(), "launch": "eager"},
-            "gpu_launches": (len(Runner.ALL) + (2 if T * cfg.k > 4096 else 0)) * args.steps,
-            "clocks": clk,
-            "device_status": status,
+            "e2e": head_rec["e2e"],
+            "gpu_launches": head_rec["gpu_launches"],
+            "clocks": head_rec["clocks"],
+            "routing": head_rec.get("routing"),
+            "kernels_ms": head_rec.get("kernels_ms"),
+            "kernels_ms_breakdown": head_rec.get("kernels_ms_breakdown"),
+            "device_status": head_rec["device_status"],
+            "workloads": records,
         }
         print(json.dumps(line), flush=True)
     if dist:
-        r.graphs.clear()
         dist.barrier()
         dist.destroy_process_group()
 

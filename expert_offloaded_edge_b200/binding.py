@@ -81,6 +81,8 @@ def library() -> ctypes.CDLL:
         L.ftm_moe_layer_forward_noalloc.restype = c_i32
         L.ftm_set_profile_events.argtypes = [c_i32, c_p, c_p]
         L.ftm_set_profile_events.restype = c_i32
+        L.ftm_kernel_launches.argtypes = []
+        L.ftm_kernel_launches.restype = c_u64
         L.ftm_workspace_bytes.argtypes = [P(LayerDesc), c_i32]
         L.ftm_workspace_bytes.restype = c_sz
         for name in ("ftm_get_bank_layout", "ftm_route", "ftm_permute", "ftm_slot_lookup_update", "ftm_slot_resize",
@@ -186,6 +188,10 @@ def ftm_set_profile_events(which: int, start_event=None, stop_event=None):
     sp = None if start_event is None else start_event.cuda_event
     ep = None if stop_event is None else stop_event.cuda_event
     _check(library().ftm_set_profile_events(which, sp, ep))
+
+
+def ftm_kernel_launches() -> int:
+    return int(library().ftm_kernel_launches())
 
 
 def ftm_workspace_bytes(desc, T_max) -> int:

@@ -2,6 +2,7 @@
 // miss-copy orchestration of the slot cache, and the whole-layer sequence.
 // Every computation step runs in the kernels of the sibling .cu files.
 #include <stdarg.h>
+#include <atomic>
 #include <stdio.h>
 #include <string.h>
 
@@ -17,7 +18,7 @@ size_t lru_workspace_bytes(int E, int S);
 cudaError_t launch_lru_step(const int32_t* ids, int P, int E, int S, int64_t step, int32_t* soe, int32_t* eos,
                             int64_t* lu, int32_t* ws, cudaStream_t st);
 cudaError_t launch_lru_restore(int E, int S, int32_t* soe, int32_t* eos, int64_t* lu, const int32_t* ws,
-                               cudaStream_t st);
+                               int n_dirty, cudaStream_t st);
 cudaError_t launch_slot_resize(int E, int S_old, const int32_t* eos_old, const int64_t* lu_old, int S_new,
                                int32_t* soe_new, int32_t* eos_new, int64_t* lu_new, const void* old_pool,
                                void* new_pool, size_t bank_bytes, int32_t* ws, cudaStream_t st);
@@ -180,6 +181,15 @@ cudaEvent_t copy_event() {
 
 ftm_status ftm::report_error(ftm_status s, const char* msg) { return fail(s, "%s", msg); }
 
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}
+
+cudaError_t ftm::count_launch(cudaError_t e) {
+  if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+  return e;
+}
+
 void ftm::prof_mark(int which, cudaStream_t st, bool stop) {
   if (which < 0 || which >= FTM_K_COUNT || !g_prof[which][stop ? 1 : 0]) return;
   // under stream capture the record must become a graph node of its own
@@ -194,6 +204,8 @@ void ftm::prof_mark(int which, cudaStream_t st, bool stop) {
 extern "C" {
 
 const char* ftm_last_error(void) { return g_err; }
+
+uint64_t ftm_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 ftm_status ftm_set_profile_events(int32_t which, void* start_event, void* stop_event) {
   if (which < 0 || which >= FTM_K_COUNT) return fail(FTM_ERR_INVALID_ARG, "kernel id %d out of range", which);
@@ -328,26 +340,38 @@ ftm_status ftm_slot_lookup_update(const ftm_layer_desc* L, ftm_slot_cache* C, co
   C->last_distinct = h[1];
   C->last_hits = h[2];
   C->last_misses = h[3];
+  if (h[0] == FTM_ERR_INVALID_ARG)
+    return fail(FTM_ERR_INVALID_ARG, "step %lld: topk_ids holds an expert id outside [0, %d); state unchanged",
+                static_cast<long long>(C->step), L->E);
   if (h[0] == FTM_ERR_CAPACITY)
     return fail(FTM_ERR_CAPACITY, "step %lld requests %d distinct experts > %d slots", static_cast<long long>(C->step),
                 h[1], L->S);
   ftm_bank_layout bl;
   bank_layout(L, &bl);
   const int misses = h[3];
-  bool copy_failed = C->fail_before_copy != 0;
-  const char* why = copy_failed ? "injected copy failure (fail_before_copy)" : nullptr;
+  bool copy_failed = false;
+  const char* why = nullptr;
+  int n_dirty = 0;     // miss-list slots a copy may have written
   for (int i = 0; i < misses && !copy_failed; ++i) {
+    if (C->fail_before_copy > 0 && i + 1 == C->fail_before_copy) {
+      copy_failed = true;
+      why = "injected copy failure (fail_before_copy)";
+      break;
+    }
     const int ex = h[4 + 2 * i], sl = h[4 + 2 * i + 1];
     e = cudaMemcpyAsync(static_cast<uint8_t*>(C->slot_pool) + static_cast<size_t>(sl) * bl.bank_bytes,
                         static_cast<const uint8_t*>(C->host_pool) + static_cast<size_t>(ex) * bl.bank_bytes,
                         bl.bank_bytes, cudaMemcpyHostToDevice, ps);
+    n_dirty = i + 1;     // a copy that failed to issue may still have started
     if (e != cudaSuccess) { copy_failed = true; why = cudaGetErrorString(e); }
   }
   if (copy_failed) {
     C->fail_before_copy = 0;
-    cudaError_t e2 = launch_lru_restore(L->E, L->S, C->slot_of_expert, C->expert_of_slot, C->last_use, ws, cs);
+    cudaError_t e2 = launch_lru_restore(L->E, L->S, C->slot_of_expert, C->expert_of_slot, C->last_use, ws, n_dirty,
+                                        cs);
     if (e2 == cudaSuccess) e2 = cudaStreamSynchronize(cs);
-    return fail(FTM_ERR_CUDA, "miss copy failed (%s); slot state rolled back%s", why,
+    return fail(FTM_ERR_CUDA, "a miss copy failed (%s) with %d of %d copies issued; slot state rolled back, the "
+                "%d slot(s) a copy may have written left empty%s", why, n_dirty, misses, n_dirty,
                 e2 == cudaSuccess ? "" : " -- rollback failed too");
   }
   if (misses > 0) {

@@ -21,7 +21,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ y
     // the token's rows and weights first, so the row loads below are independent
     if (threadIdx.x < nterms) {
       const int j = threadIdx.x;
-      s_row[j] = j < k ? inv[static_cast<size_t>(t) * k + j] : P + t;
+      int row = j < k ? inv[static_cast<size_t>(t) * k + j] : P + t;
+      if (j < k && (row < 0 || row >= P)) {   // a pair the permutation skipped (id out of range)
+        report_bad_index();
+        row = -1;
+      }
+      s_row[j] = row;
       s_g[j] = j < k ? gw[static_cast<size_t>(t) * k + j] : 1.f;
     }
     __syncthreads();
@@ -32,6 +37,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ y
 #pragma unroll 4
       for (int j = 0; j < nterms; ++j) {
         const int row = s_row[j];
+        if (row < 0) continue;
         const float g = s_g[j];
         const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(y) +
                                                         (static_cast<size_t>(row) * d + static_cast<size_t>(c) * V) *

@@ -11,9 +11,14 @@
 
 namespace ftm {
 
-// Device status word (set by a bounded wait that gives up).
+// Device status word: set by a bounded wait that gives up, or by a kernel
+// that met an index out of its range (the access is skipped).
 constexpr int32_t kDevErrTimeout = 1;
+constexpr int32_t kDevErrBadIndex = 2;
 extern __device__ int32_t g_dev_status;
+
+// Records an out-of-range index (first error wins; never overwrites a timeout).
+__device__ __forceinline__ void report_bad_index() { atomicCAS(&g_dev_status, 0, kDevErrBadIndex); }
 
 // A wait on an mbarrier gives up after this much wall time (ns) and reports
 // kDevErrTimeout; the kernel then unwinds (frees TMEM) instead of hanging.
@@ -33,6 +38,10 @@ __device__ __forceinline__ uint64_t globaltimer() {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// Host count of kernel launches enqueued by the library (read by
+// ftm_kernel_launches); every launch site passes its result through here.
+cudaError_t count_launch(cudaError_t e);
+
 // Launch with programmatic stream serialisation (host).
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
@@ -47,7 +56,7 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  return count_launch(cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...));
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {

@@ -33,7 +33,9 @@ __global__ void gather_rows_kernel(const uint8_t* __restrict__ x, const int32_t*
   const int rows = P + (has_shared ? T : 0);
   const int nv = row_bytes / 16;
   for (int r = blockIdx.x; r < rows; r += gridDim.x) {
-    const int src = r < P ? perm[r] / k : r - P;
+    const int q = r < P ? perm[r] : 0;
+    if (q < 0) continue;     // no pair placed here (ids out of range); no group reads this row
+    const int src = r < P ? q / k : r - P;
     const uint4* s = reinterpret_cast<const uint4*>(x + static_cast<size_t>(src) * row_bytes);
     uint4* dd = reinterpret_cast<uint4*>(xp + static_cast<size_t>(r) * row_bytes);
     for (int c = threadIdx.x; c < nv; c += blockDim.x) dd[c] = s[c];
@@ -390,8 +392,8 @@ static cudaError_t launch_tc(const CUtensorMap& mA, const CUtensorMap& mAsh, con
   cfg.dynamicSmemBytes = smem;
   cfg.gridDim = dim3(static_cast<unsigned>(tiles * ks));
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, mA, mAsh, mB, a.offsets, a.slot_of_expert, a.E, a.has_shared, a.T, P, K, Nw,
-                            up_row0, out, ld_out, stages);
+  return count_launch(cudaLaunchKernelEx(&cfg, kern, mA, mAsh, mB, a.offsets, a.slot_of_expert, a.E, a.has_shared, a.T, P, K, Nw,
+                            up_row0, out, ld_out, stages));
 }
 
 template <bool GATED>

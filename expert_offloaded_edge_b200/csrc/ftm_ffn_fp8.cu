@@ -58,7 +58,9 @@ __global__ void __launch_bounds__(256) gather_quant_fp8_kernel(const uint16_t* _
   for (long w = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32; w < total;
        w += static_cast<long>(gridDim.x) * blockDim.x / 32) {
     const int r = static_cast<int>(w / groups), g = static_cast<int>(w % groups);
-    const int src = r < P ? perm[r] / k : r - P;
+    const int q = r < P ? perm[r] : 0;
+    if (q < 0) continue;     // no pair placed here (ids out of range); warp-uniform
+    const int src = r < P ? q / k : r - P;
     const uint2 u = *reinterpret_cast<const uint2*>(x + static_cast<size_t>(src) * d + g * 128 + lane * 4);
     float v[4] = {bf16_bits_to_f32(u.x & 0xFFFF), bf16_bits_to_f32(u.x >> 16), bf16_bits_to_f32(u.y & 0xFFFF),
                   bf16_bits_to_f32(u.y >> 16)};

@@ -931,9 +931,9 @@ static cudaError_t launch_nvfp4_tc2_one(const CUtensorMap* maps, const FfnArgs& 
   const int pairs = static_cast<int>(tiles < pairs_max[GATED] ? tiles : pairs_max[GATED]);
   cfg.gridDim = dim3(2 * pairs);
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], a.offsets, prow0,
+  return count_launch(cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], a.offsets, prow0,
                             a.slot_of_expert, a.E, a.has_shared, a.T, P, K, Nw, up_row0, a.pool, a.shared_bank,
-                            a.bank_bytes, st_off, st_idx, out_q, out_sf, out_bf16);
+                            a.bank_bytes, st_off, st_idx, out_q, out_sf, out_bf16));
 }
 
 // Both GEMMs on CTA pairs; xq/sfx (gathered, padded to 224-row blocks) are ready.

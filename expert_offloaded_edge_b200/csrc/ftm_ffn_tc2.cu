@@ -287,8 +287,8 @@ static cudaError_t launch_tc2_one(const CUtensorMap& mA, const CUtensorMap& mAsh
   const int pairs = static_cast<int>(tiles < pairs_max[GATED] ? tiles : pairs_max[GATED]);
   cfg.gridDim = dim3(2 * pairs);
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, mA, mAsh, mB, a.offsets, a.slot_of_expert, a.E, a.has_shared, a.T, P, K, Nw,
-                            up_row0, out, ld_out);
+  return count_launch(cudaLaunchKernelEx(&cfg, kern, mA, mAsh, mB, a.offsets, a.slot_of_expert, a.E, a.has_shared, a.T, P, K, Nw,
+                            up_row0, out, ld_out));
 }
 
 static bool map_bf16(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint64_t row_pitch, uint64_t slots,

@@ -36,15 +36,26 @@ __global__ void __launch_bounds__(kLruThreads) lru_step_kernel(const int32_t* __
   int32_t* miss_rank = want + E;   // [E+1] exclusive scan of miss flags
   int32_t* cand = miss_rank + E + 1;  // [S] candidate flag, later victim_of_rank
   int32_t* victim = cand + S;      // [S]
-  __shared__ int32_t s_distinct, s_hits;
+  __shared__ int32_t s_distinct, s_hits, s_bad;
   pdl_wait();
   pdl_trigger();
 
   for (int e = threadIdx.x; e < E; e += blockDim.x) want[e] = 0;
-  if (threadIdx.x == 0) { s_distinct = 0; s_hits = 0; }
+  if (threadIdx.x == 0) { s_distinct = 0; s_hits = 0; s_bad = 0; }
   __syncthreads();
-  for (int q = threadIdx.x; q < P; q += blockDim.x) want[ids[q]] = 1;
+  for (int q = threadIdx.x; q < P; q += blockDim.x) {
+    const int e = ids[q];
+    if (e >= 0 && e < E) want[e] = 1;
+    else s_bad = 1;
+  }
   __syncthreads();
+  if (s_bad) {   // an id outside [0, E): the state is left untouched
+    if (threadIdx.x == 0) {
+      report_bad_index();
+      ws[0] = FTM_ERR_INVALID_ARG; ws[1] = 0; ws[2] = 0; ws[3] = 0;
+    }
+    return;
+  }
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     if (want[e]) atomicAdd(&s_distinct, 1);
   __syncthreads();
@@ -117,9 +128,13 @@ __global__ void __launch_bounds__(kLruThreads) lru_step_kernel(const int32_t* __
   if (threadIdx.x == 0) { ws[0] = FTM_OK; ws[1] = distinct; ws[2] = s_hits; ws[3] = misses; }
 }
 
+// Rollback of a step whose miss copies could not all be issued: the state
+// before the step comes back from the backup, except that the first n_dirty
+// slots of the miss list (whose banks a copy may already have overwritten)
+// are left empty and their previous experts unmapped.
 __global__ void lru_restore_kernel(int E, int S, int32_t* __restrict__ slot_of_expert,
                                    int32_t* __restrict__ expert_of_slot, int64_t* __restrict__ last_use,
-                                   const int32_t* __restrict__ ws) {
+                                   const int32_t* __restrict__ ws, int n_dirty) {
   const int32_t* bk_soe = ws + 4 + 2 * E;
   const int32_t* bk_eos = bk_soe + E;
   size_t off = sizeof(int32_t) * (4 + 2 * static_cast<size_t>(E) + E + S);
@@ -127,6 +142,14 @@ __global__ void lru_restore_kernel(int E, int S, int32_t* __restrict__ slot_of_e
   const int64_t* bk_lu = reinterpret_cast<const int64_t*>(reinterpret_cast<const uint8_t*>(ws) + off);
   for (int e = threadIdx.x; e < E; e += blockDim.x) slot_of_expert[e] = bk_soe[e];
   for (int j = threadIdx.x; j < S; j += blockDim.x) { expert_of_slot[j] = bk_eos[j]; last_use[j] = bk_lu[j]; }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_dirty; i += blockDim.x) {
+    const int sl = ws[4 + 2 * i + 1];
+    const int old = bk_eos[sl];
+    if (old >= 0) slot_of_expert[old] = -1;
+    expert_of_slot[sl] = -1;
+    last_use[sl] = -1;
+  }
 }
 
 cudaError_t launch_lru_step(const int32_t* ids, int P, int E, int S, int64_t step, int32_t* soe, int32_t* eos,
@@ -139,9 +162,9 @@ cudaError_t launch_lru_step(const int32_t* ids, int P, int E, int S, int64_t ste
 }
 
 cudaError_t launch_lru_restore(int E, int S, int32_t* soe, int32_t* eos, int64_t* lu, const int32_t* ws,
-                               cudaStream_t st) {
-  lru_restore_kernel<<<1, kLruThreads, 0, st>>>(E, S, soe, eos, lu, ws);
-  return cudaGetLastError();
+                               int n_dirty, cudaStream_t st) {
+  lru_restore_kernel<<<1, kLruThreads, 0, st>>>(E, S, soe, eos, lu, ws, n_dirty);
+  return count_launch(cudaGetLastError());
 }
 
 // ---------------------------------------------------------------------------

@@ -33,6 +33,16 @@ __device__ void warp0_exclusive_scan(const int32_t* in, int32_t* out, int E) {
   if (lane == 31) out[E] = incl;
 }
 
+// cnt[e] += number of pairs in [q0, q1) routed to e (shared memory).  An id
+// outside [0, E) is not counted and is reported in the device status word.
+__device__ __forceinline__ void count_ids(const int32_t* __restrict__ ids, int q0, int q1, int E, int32_t* cnt) {
+  for (int q = q0 + threadIdx.x; q < q1; q += blockDim.x) {
+    const int e = ids[q];
+    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+    else report_bad_index();
+  }
+}
+
 // Place pairs [q_begin, q_end) in order; base[e] (shared) is the next free
 // position of expert e and is advanced.  wcnt (shared, [warps][E]) must be zero.
 __device__ void stable_scatter(const int32_t* __restrict__ ids, int q_begin, int q_end, int32_t* base,
@@ -41,12 +51,14 @@ __device__ void stable_scatter(const int32_t* __restrict__ ids, int q_begin, int
   const unsigned lt_mask = (1u << lane) - 1u;
   for (int r0 = q_begin; r0 < q_end; r0 += blockDim.x) {
     const int q = r0 + threadIdx.x;
-    const bool valid = q < q_end;
-    const int e = valid ? ids[q] : E;
+    const int e_in = q < q_end ? ids[q] : E;
+    const bool valid = q < q_end && e_in >= 0 && e_in < E;   // an id outside [0, E) is skipped
+    const int e = valid ? e_in : E;
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int rank_w = __popc(peers & lt_mask);
     if (valid && rank_w == 0) wcnt[warp * E + e] = __popc(peers);
     __syncthreads();
+    if (q < q_end && !valid) inv[q] = -1;
     if (valid) {
       int before = 0;
       for (int w = 0; w < warp; ++w) before += wcnt[w * E + e];
@@ -79,7 +91,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_single_kernel(const int3
   for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
   for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) wcnt[i] = 0;
   __syncthreads();
-  for (int q = threadIdx.x; q < P; q += blockDim.x) atomicAdd(&cnt[ids[q]], 1);
+  count_ids(ids, 0, P, E, cnt);
   __syncthreads();
   if (threadIdx.x < 32) warp0_exclusive_scan(cnt, base, E);
   __syncthreads();
@@ -87,6 +99,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_single_kernel(const int3
   for (int i = threadIdx.x; i < E; i += blockDim.x) counts[i] = cnt[i];
   __syncthreads();
   stable_scatter(ids, 0, P, base, wcnt, E, perm, inv);
+  // positions past the last placed pair (only when ids held out-of-range values)
+  for (int pos = base[E] + threadIdx.x; pos < P; pos += blockDim.x) perm[pos] = -1;
 }
 
 // Large P, pass 1: per-chunk histogram hist[c][e].
@@ -98,15 +112,17 @@ __global__ void __launch_bounds__(kPermThreads) permute_hist_kernel(const int32_
   for (int i = threadIdx.x; i < E; i += blockDim.x) sm[i] = 0;
   __syncthreads();
   const int q0 = blockIdx.x * kChunk, q1 = min(P, q0 + kChunk);
-  for (int q = q0 + threadIdx.x; q < q1; q += blockDim.x) atomicAdd(&sm[ids[q]], 1);
+  count_ids(ids, q0, q1, E, sm);
   __syncthreads();
   for (int i = threadIdx.x; i < E; i += blockDim.x) hist[static_cast<size_t>(blockIdx.x) * E + i] = sm[i];
 }
 
 // Large P, pass 2 (one block): counts, offsets, and hist[c][e] <- start of chunk c's run of expert e.
-__global__ void __launch_bounds__(kPermThreads) permute_scan_kernel(int nchunks, int E, int32_t* __restrict__ hist,
+__global__ void __launch_bounds__(kPermThreads) permute_scan_kernel(int nchunks, int E, int P,
+                                                                    int32_t* __restrict__ hist,
                                                                     int32_t* __restrict__ counts,
-                                                                    int32_t* __restrict__ offsets) {
+                                                                    int32_t* __restrict__ offsets,
+                                                                    int32_t* __restrict__ perm) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ int32_t sm[];
@@ -131,6 +147,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_scan_kernel(int nchunks,
     }
   }
   for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets[e] = off[e];
+  // positions past the last placed pair (only when ids held out-of-range values)
+  for (int pos = off[E] + threadIdx.x; pos < P; pos += blockDim.x) perm[pos] = -1;
 }
 
 // Large P, pass 3: each chunk places its pairs in order from its bases.
@@ -173,7 +191,7 @@ cudaError_t launch_permute(const int32_t* ids, int P, int E, int32_t* counts, in
   err = launch_pdl(permute_hist_kernel, dim3(nchunks), dim3(kPermThreads), sizeof(int32_t) * E, st, ids, P, E, hist);
   if (err != cudaSuccess) return err;
   err = launch_pdl(permute_scan_kernel, dim3(1), dim3(kPermThreads), sizeof(int32_t) * (2 * E + 1), st, nchunks, E,
-                   hist, counts, offsets);
+                   P, hist, counts, offsets, perm);
   if (err != cudaSuccess) return err;
   return launch_pdl(permute_scatter_kernel, dim3(nchunks), dim3(kPermThreads), wsm, st, ids, P, E, hist, perm, inv);
 }

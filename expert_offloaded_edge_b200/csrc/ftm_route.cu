@@ -185,8 +185,8 @@ static cudaError_t launch_route_tt(const void* x, int T, int d, const void* wr, 
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<const Tin*>(x), T, d, static_cast<const Tin*>(wr), bias, E, k,
-                            ids, w);
+  return count_launch(cudaLaunchKernelEx(&cfg, kern, static_cast<const Tin*>(x), T, d, static_cast<const Tin*>(wr), bias, E, k,
+                            ids, w));
 }
 
 bool route_tc_applicable(bool f32, int T, int E, int k);

@@ -100,7 +100,11 @@ typedef struct ftm_bank_layout {
 
 ftm_status ftm_get_bank_layout(const ftm_layer_desc* L, ftm_bank_layout* out);
 
-/* Router + gating (a1, a2).
+/* Router + gating (a1, a2).  chenxutan.com FreeToken article, section "why
+ * the bottleneck is bandwidth, not capacity": each token activates only a few
+ * of the routed experts (6 of them for the 284B model), picked per token by
+ * the router; the gate reading (softmax over all E logits, then renormalised
+ * over the k picks) is the plain top-k routed MoE.
  *   x        device [T][d] (fp32 or bf16, see above)
  *   w_router device [E][d] row-major (same dtype as x)
  *   bias     device fp32 [E] added to every logit, or NULL
@@ -112,14 +116,23 @@ ftm_status ftm_get_bank_layout(const ftm_layer_desc* L, ftm_bank_layout* out);
 ftm_status ftm_route(const ftm_layer_desc* L, const void* x, int32_t T, const void* w_router,
                      const float* bias, int32_t* topk_ids, float* topk_w, void* stream);
 
-/* Permutation of the P = T*k (token, pick) pairs by expert (a3).
+/* Permutation of the P = T*k (token, pick) pairs by expert (a3).  chenxutan.com
+ * FreeToken article, same section: in prefill a large batch routes to nearly
+ * every expert at once, so the batch's pairs are grouped per expert and each
+ * expert's weights are read once for all of its rows (the grouping a fused
+ * MoE kernel performs; pomoai.com FreeToken hub, install paragraph, [accel]
+ * fused kernels).
  *   counts  device int32 [E]     pairs per expert
  *   offsets device int32 [E+1]   exclusive prefix sum, offsets[E] = P
  *   perm    device int32 [P]     perm[pos] = q = t*k + j, stable: pairs of one
  *                                expert appear in ascending q
  *   inv     device int32 [P]     inv[q] = pos
  *   workspace device, >= ftm_permute_workspace_bytes(L, T) bytes, 256-aligned
- * Deterministic: identical results run to run. */
+ * Deterministic: identical results run to run.  Ids are range-checked on the
+ * device: a pair whose id is outside [0, E) is not counted or placed, its
+ * inv entry is -1, perm positions from offsets[E] to P-1 hold -1, and the
+ * device status word (ftm_device_status) reads 2; no out-of-range access is
+ * made. */
 ftm_status ftm_permute(const ftm_layer_desc* L, const int32_t* topk_ids, int32_t T, int32_t* counts,
                        int32_t* offsets, int32_t* perm, int32_t* inv, void* workspace, size_t ws_bytes,
                        void* stream);
@@ -144,8 +157,10 @@ typedef struct ftm_slot_cache {
   int32_t last_distinct;        /* out: distinct experts requested by the last step */
   int32_t last_hits;            /* out: of which resident */
   int32_t last_misses;          /* out: of which copied in */
-  int32_t fail_before_copy;     /* test hook: != 0 makes the next update fail as if its
-                                   first copy had failed; state is rolled back */
+  int32_t fail_before_copy;     /* test hook: n >= 1 makes the next update with at least n
+                                   misses fail as if its n-th copy could not be issued
+                                   (copies 1..n-1 are issued); see the rollback rule of
+                                   ftm_slot_lookup_update.  Cleared when it fires. */
 } ftm_slot_cache;
 
 size_t ftm_slot_host_scratch_ints(const ftm_layer_desc* L);
@@ -155,9 +170,16 @@ size_t ftm_slot_workspace_bytes(const ftm_layer_desc* L);
  * synchronises that stream to read the miss list (the one host sync of the
  * path), issues one cudaMemcpyAsync per miss on `copy_stream`, and makes
  * `compute_stream` wait for the copies, so work enqueued afterwards on
- * `compute_stream` sees the new slots.  Returns FTM_ERR_CAPACITY (state
- * unchanged) when more than S distinct experts are requested, FTM_ERR_CUDA
- * (state rolled back to before the call) when a copy cannot be issued.
+ * `compute_stream` sees the new slots.  Returns
+ *   FTM_ERR_CAPACITY (state unchanged) when more than S distinct experts are
+ *     requested;
+ *   FTM_ERR_INVALID_ARG (state unchanged) when topk_ids holds an id outside
+ *     [0, E) (found on the device, which also sets the device status word to 2);
+ *   FTM_ERR_CUDA when a copy cannot be issued: the state is rolled back to
+ *     before the call, except that every slot whose copy was already issued
+ *     (it may hold part of the new bank) is left empty (expert_of_slot -1,
+ *     last_use -1) with its previous expert unmapped, so no partly
+ *     overwritten bank is ever taken for a hit.
  *   workspace device, >= ftm_slot_workspace_bytes(L) bytes */
 ftm_status ftm_slot_lookup_update(const ftm_layer_desc* L, ftm_slot_cache* C, const int32_t* topk_ids,
                                   int32_t T, void* workspace, size_t ws_bytes, void* compute_stream,
@@ -186,7 +208,12 @@ ftm_status ftm_slot_lookup_update(const ftm_layer_desc* L, ftm_slot_cache* C, co
 ftm_status ftm_slot_resize(const ftm_layer_desc* L, const ftm_slot_cache* C, int32_t S_new, ftm_slot_cache* C_new,
                            void* workspace, size_t ws_bytes, void* stream);
 
-/* Grouped SwiGLU expert FFN (a5, a6, a7).
+/* Grouped SwiGLU expert FFN (a5, a6, a7).  chenxutan.com FreeToken article,
+ * section "choosing among the five MoE backends": `fused` (every expert resident
+ * in VRAM) and `offload` (experts computed on the GPU from LRU slots in VRAM);
+ * pomoai.com FreeToken hub, checkpoint list: BF16, FP8 and NVFP4 expert weights.
+ * The SwiGLU form and the shared expert (weight 1, configs with one) are the
+ * plain reading of the DeepSeek/GLM/Qwen MoE layers the pages run.
  *   x              device [T][d] activations (token order)
  *   offsets, perm  from ftm_permute
  *   slot_of_expert device int32 [E]: bank of expert e is slot_pool[slot_of_expert[e]]
@@ -203,9 +230,14 @@ ftm_status ftm_expert_ffn(const ftm_layer_desc* L, const void* x, int32_t T, con
                           void* stream);
 size_t ftm_ffn_workspace_bytes(const ftm_layer_desc* L, int32_t T);
 
-/* Weighted un-permute and combine (a8):
+/* Weighted un-permute and combine (a8).  chenxutan.com FreeToken article,
+ * section "why the bottleneck is bandwidth, not capacity": a token's output is
+ * made from the few routed experts it activated; the gate-weighted sum (plus
+ * the shared expert) is the plain reading:
  *   out[t] = sum_{j=0..k-1 ascending} topk_w[t][j] * y[inv[t*k+j]]  (+ y[P+t] if has_shared),
- * accumulated in fp32.  y, inv, topk_w device; out device [T][d]. */
+ * accumulated in fp32.  y, inv, topk_w device; out device [T][d].  A pair
+ * whose inv entry is outside [0, P) (one ftm_permute skipped) is left out of
+ * the sum and sets the device status word to 2. */
 ftm_status ftm_combine(const ftm_layer_desc* L, const void* y, const int32_t* inv, const float* topk_w,
                        int32_t T, void* out, void* stream);
 
@@ -219,6 +251,9 @@ typedef struct ftm_layer_weights {
 } ftm_layer_weights;
 
 /* The whole layer: route -> permute -> [cache step] -> expert FFN -> combine.
+ * chenxutan.com FreeToken article, section "choosing among the five MoE
+ * backends": `fused` (C = NULL, every expert resident) and `offload` (C set:
+ * experts in host RAM, LRU slots in VRAM, misses copied over PCIe).
  *   C          NULL for a resident layer (every expert in W->slot_pool at
  *              W->slot_of_expert[e]); otherwise the LRU cache (its slot_pool and
  *              slot_of_expert are used, and the call synchronises once, see
@@ -266,11 +301,19 @@ typedef enum ftm_kernel_id {
  * with timing enabled).  NULL events clear the hook.  Nothing else changes. */
 ftm_status ftm_set_profile_events(int32_t which, void* start_event, void* stop_event);
 
+/* Number of kernel launches the library has enqueued in this process so far
+ * (all threads and devices; launches recorded into a CUDA graph under stream
+ * capture count once, at capture).  A measurement hook: the difference across
+ * one eager layer call is the number of kernels that call launches. */
+uint64_t ftm_kernel_launches(void);
+
 /* Thread-local description of the last error returned on this thread. */
 const char* ftm_last_error(void);
 
-/* Reads (and if reset != 0 clears) the device status word the kernels set when
- * a bounded wait gives up.  Synchronises the device.  0 = no fault. */
+/* Reads (and if reset != 0 clears) the device status word.  Synchronises the
+ * device.  0 = no fault; 1 = a bounded wait of a tensor-core kernel gave up
+ * (the kernel unwound and freed its tensor memory); 2 = a kernel met an index
+ * outside its range (an expert id outside [0, E)) and skipped the access. */
 int32_t ftm_device_status(int32_t reset);
 
 #ifdef __cplusplus

@@ -38,6 +38,7 @@ def lib():
         L = ctypes.CDLL(build())
         p, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
         L.orc_threads.restype = i32
+        L.orc_set_threads.argtypes = [i32]
         L.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
         L.orc_bf16_to_f32.restype = ctypes.c_float
         L.orc_e4m3_value.argtypes = [ctypes.c_uint8]
@@ -87,6 +88,11 @@ def _f32(a) -> np.ndarray:
 
 def threads() -> int:
     return int(lib().orc_threads())
+
+
+def set_threads(n: int) -> None:
+    """OpenMP threads for the oracle calls of the calling thread."""
+    lib().orc_set_threads(int(n))
 
 
 # ---- formats -----------------------------------------------------------------
@@ -327,6 +333,7 @@ def moe_rows(layer, x: np.ndarray, rows: Sequence[int], ids: np.ndarray, gates: 
     qa = qa_mode(cfg.wdtype) if qa is None else qa
     rows = list(rows)
     k = cfg.k
+    keep = weight_cache is not None      # without a cache, each expert's weights are dropped after use
     cache = {} if weight_cache is None else weight_cache
     y_pairs = np.zeros((len(rows) * k, cfg.d), dtype=np.float32)
     # group (row, pick) by expert so each expert's weights are dequantised once
@@ -342,6 +349,8 @@ def moe_rows(layer, x: np.ndarray, rows: Sequence[int], ids: np.ndarray, gates: 
         ys = expert_ffn(xs, Wg, Wu, Wd, qa)
         for (ri, j), yv in zip(lst, ys):
             y_pairs[ri * k + j] = yv
+        if not keep:
+            del cache[e]
     ysh = None
     if cfg.has_shared:
         if cfg.E not in cache:

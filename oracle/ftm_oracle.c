@@ -47,6 +47,16 @@ int orc_threads(void) {
 #endif
 }
 
+/* Threads the calling thread's OpenMP regions use from now on (the setting
+ * belongs to the calling thread). */
+void orc_set_threads(int n) {
+#ifdef _OPENMP
+  omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 /* ---------------------------------------------------------------------------
  * Number formats (OCP 8-bit floating point spec, E4M3; OCP MX spec, E2M1).
  * ------------------------------------------------------------------------- */

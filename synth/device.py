@@ -30,7 +30,10 @@ class DeviceLayer:
     pinned host pool and the device pool of S slots starts empty."""
 
     def __init__(self, cfg: LayerConfig, seed: int = 0, device: str = "cuda", T_redraw: Optional[int] = None,
-                 redraws=None, slot_perm: Optional[np.ndarray] = None):
+                 redraws=None, slot_perm: Optional[np.ndarray] = None, banks: Optional[np.ndarray] = None):
+        """banks: optional [E + has_shared][bank_bytes] uint8, the packed banks of
+        this layer (row E = the shared expert), e.g. from pack_banks() saved
+        earlier; when absent they are drawn and packed here."""
         self.cfg = cfg
         self.device = device
         if redraws is None:
@@ -40,17 +43,26 @@ class DeviceLayer:
         self.bl = ftm.ftm_get_bank_layout(self.desc)
         bb = self.bl.bank_bytes
         L = self.layer
+        if banks is not None:
+            assert banks.shape == (cfg.E + cfg.has_shared, bb), banks.shape
+
+        def bank(e):
+            return banks[e] if banks is not None else pack_bank(self.desc, L.expert(e), self.bl)
+
         self.w_router = to_device_storage(L.router_storage(), cfg.act_dtype, device)
         b = L.bias()
         self.bias = None if b is None else torch.from_numpy(b).to(device)
         self.shared_bank = None
         if cfg.has_shared:
-            self.shared_bank = torch.from_numpy(pack_bank(self.desc, L.expert(cfg.E), self.bl)).to(device)
+            self.shared_bank = torch.from_numpy(np.ascontiguousarray(bank(cfg.E))).to(device)
         if cfg.lru:
             self.host_pool = torch.empty(cfg.E * bb, dtype=torch.uint8, pin_memory=True)
             hp = self.host_pool.numpy()
             for e in range(cfg.E):
-                pack_bank(self.desc, L.expert(e), self.bl, out=hp[e * bb:(e + 1) * bb])
+                if banks is not None:
+                    hp[e * bb:(e + 1) * bb] = banks[e]
+                else:
+                    pack_bank(self.desc, L.expert(e), self.bl, out=hp[e * bb:(e + 1) * bb])
             self.pool = torch.zeros(cfg.S * bb, dtype=torch.uint8, device=device)
             self.slot_of_expert_np = None
             self.slot_of_expert = torch.full((cfg.E,), -1, dtype=torch.int32, device=device)
@@ -69,7 +81,7 @@ class DeviceLayer:
             self.pool = torch.zeros(cfg.S * bb, dtype=torch.uint8, device=device)
             for e in range(cfg.E):
                 s = int(soe[e])
-                self.pool[s * bb:(s + 1) * bb].copy_(torch.from_numpy(pack_bank(self.desc, L.expert(e), self.bl)))
+                self.pool[s * bb:(s + 1) * bb].copy_(torch.from_numpy(np.ascontiguousarray(bank(e))))
             self.cache = None
 
     def weights(self) -> ftm.LayerWeights:
@@ -82,6 +94,17 @@ class DeviceLayer:
 
     def out_dtype(self):
         return torch.float32 if self.cfg.act_dtype == "f32" else torch.bfloat16
+
+
+def pack_banks(cfg: LayerConfig, seed: int = 0) -> np.ndarray:
+    """All banks of a layer, [E + has_shared][bank_bytes] uint8 (row E = shared)."""
+    layer = Layer(cfg, seed)
+    desc = ftm.desc_for(cfg)
+    bl = ftm.ftm_get_bank_layout(desc)
+    out = np.zeros((cfg.E + cfg.has_shared, bl.bank_bytes), dtype=np.uint8)
+    for e in range(cfg.E + cfg.has_shared):
+        pack_bank(desc, layer.expert(e), bl, out=out[e])
+    return out
 
 
 class Workspace:

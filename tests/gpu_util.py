@@ -68,3 +68,20 @@ def assert_rows_close(got: np.ndarray, want: np.ndarray, frac: float, what: str 
     worst = float((err / np.maximum(scale, 1e-30)).max()) if len(err) else 0.0
     assert bad.size == 0, f"{what}: {bad.size} rows exceed {frac} (worst ratio {worst:.3g}, rows {bad[:8]})"
     return worst
+
+
+def group_edge_rows(ids: np.ndarray, E: int, T: int, n: int = 512, seed: int = 0):
+    """Token rows to check on a large batch: the tokens of the first and the
+    last pair of every expert group (the ragged edges of the GEMM tiles), the
+    first and last token, and seeded random tokens up to n rows."""
+    counts, offsets, perm, _ = oracle.permute(ids, E)
+    k = ids.shape[1]
+    rows = {0, T - 1}
+    for e in range(E):
+        if counts[e]:
+            rows.add(int(perm[offsets[e]]) // k)
+            rows.add(int(perm[offsets[e + 1] - 1]) // k)
+    rng = np.random.default_rng(seed)
+    while len(rows) < min(n, T):
+        rows.add(int(rng.integers(T)))
+    return sorted(rows)

@@ -10,8 +10,8 @@ import expert_offloaded_edge_b200 as ftm
 import oracle
 import synth
 from synth.device import DeviceLayer
-from tests.gpu_util import (TOL, TOL_F32_SIMT, Workspace, assert_rows_close, oracle_route, oracle_rows, run_layer,
-                            screened_layer, to_np_f32)
+from tests.gpu_util import (TOL, TOL_F32_SIMT, Workspace, assert_rows_close, group_edge_rows, oracle_route, oracle_rows,
+                            run_layer, screened_layer, to_np_f32)
 
 pytestmark = pytest.mark.gpu
 
@@ -62,11 +62,14 @@ def test_35b_decode_layer(T):
     _check_layer(dl, T)
 
 
-def test_35b_prefill_layer_sampled():
+def test_35b_prefill_layer_512_rows():
+    """512 token rows of the 8192-token prefill, including the tokens of the
+    first and last pair of every expert group (the ragged tile edges)."""
     dl = DeviceLayer(synth.CONFIGS["35b_prefill"])
     T = 8192
-    rng = np.random.default_rng(0)
-    rows = sorted(set([0, 1, T - 1] + rng.choice(T, 29, replace=False).tolist()))
+    _, ids, _ = oracle_route(dl, T)
+    rows = group_edge_rows(ids, dl.cfg.E, T, 512)
+    assert len(rows) >= 512
     _check_layer(dl, T, rows=rows)
 
 

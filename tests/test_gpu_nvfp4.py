@@ -7,7 +7,8 @@ import pytest
 import oracle
 import synth
 from synth.device import DeviceLayer
-from tests.gpu_util import TOL, assert_rows_close, oracle_route, oracle_rows, run_layer, screened_layer, to_np_f32
+from tests.gpu_util import (TOL, assert_rows_close, group_edge_rows, oracle_route, oracle_rows, run_layer,
+                            screened_layer, to_np_f32)
 
 pytestmark = pytest.mark.gpu
 
@@ -48,14 +49,20 @@ def test_small_nvfp4_no_shared_expert():
     _check(dl, 45)
 
 
-def test_753b_nvfp4_decode_layer():
-    dl = DeviceLayer(synth.CONFIGS["753b_nvfp4"])
-    _check(dl, 16)
+@pytest.fixture(scope="module")
+def dl_753b():
+    return DeviceLayer(synth.CONFIGS["753b_nvfp4"])
 
 
-def test_753b_nvfp4_prefill_layer_sampled():
-    dl = DeviceLayer(synth.CONFIGS["753b_nvfp4"])
+def test_753b_nvfp4_decode_layer(dl_753b):
+    _check(dl_753b, 16)
+
+
+def test_753b_nvfp4_prefill_layer_512_rows(dl_753b):
+    """512 token rows of the 16384-token prefill, including the tokens of the
+    first and last pair of every expert group (the ragged 224-token tile edges)."""
     T = 16384
-    rng = np.random.default_rng(1)
-    rows = sorted(set([0, T - 1] + rng.choice(T, 10, replace=False).tolist()))
-    _check(dl, T, rows)
+    _, ids, _ = oracle_route(dl_753b, T)
+    rows = group_edge_rows(ids, dl_753b.cfg.E, T, 512, seed=1)
+    assert len(rows) >= 512
+    _check(dl_753b, T, rows)

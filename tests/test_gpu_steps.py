@@ -163,3 +163,116 @@ def test_combine_hand_example():
     yc = y.cpu().numpy().astype(np.float64)
     want = np.stack([0.25 * yc[3] + 0.75 * yc[0] + yc[4], 0.5 * yc[1] + 0.5 * yc[2] + yc[5]])
     assert np.allclose(out.cpu().numpy(), want, rtol=1e-6)
+
+
+def test_lru_rollback_after_partial_copies():
+    """A copy failure after some copies were issued: slots whose copy was issued
+    come back empty with their old experts unmapped; everything else is rolled
+    back; the cache keeps working from that state like the oracle's LRU."""
+    E, S = 16, 4
+    desc, bl, cache, (soe, eos, lu, pool), ws = _lru_setup(E, S)
+    copy_stream = torch.cuda.Stream()
+
+    def step(ids):
+        t = torch.tensor([ids], dtype=torch.int32, device="cuda")
+        ftm.ftm_slot_lookup_update(desc, cache, t, 1, ws.ptr, ws.nbytes, None, copy_stream)
+
+    desc.k = 2
+    step([0, 1])
+    step([2, 3])           # slots 0..3 hold experts 0..3, last_use 0, 0, 1, 1
+    step([0, 1])           # slots 0, 1 used again at step 2
+    torch.cuda.synchronize()
+    assert eos.cpu().tolist() == [0, 1, 2, 3] and lu.cpu().tolist() == [2, 2, 1, 1]
+    # step 3 misses 7 and 8: victims in (last_use, slot) order are slots 2 and 3;
+    # the second copy fails, after the first (7 -> slot 2) was issued
+    cache.fail_before_copy = 2
+    with pytest.raises(ftm.FtmError) as ei:
+        step([7, 8])
+    assert ei.value.status == 4 and cache.fail_before_copy == 0
+    torch.cuda.synchronize()
+    assert cache.step == 3
+    assert eos.cpu().tolist() == [0, 1, -1, 3]             # slot 2 may hold part of bank 7: empty
+    assert lu.cpu().tolist() == [2, 2, -1, 1]
+    want_soe = [-1] * E
+    want_soe[0], want_soe[1], want_soe[3] = 0, 1, 3         # expert 2 unmapped; 7 never mapped
+    assert soe.cpu().tolist() == want_soe
+    banks = pool.view(S, -1)[:, :4].contiguous().view(torch.int32).cpu().numpy()[:, 0]
+    assert banks[0] == 0 and banks[1] == 1 and banks[3] == 3  # untouched slots keep their banks
+    # later steps behave like the oracle's LRU started from the rolled-back state
+    ref = oracle.LRUState(E, S)
+    ref.slot_of_expert[:] = want_soe
+    ref.expert_of_slot[:] = [0, 1, -1, 3]
+    ref.last_use[:] = [2, 2, -1, 1]
+    ref.step = 3
+    for ids in ([7, 8], [2, 7], [9, 0], [3, 2]):
+        ref.update(np.array(ids, np.int32))
+        step(ids)
+        torch.cuda.synchronize()
+        assert soe.cpu().tolist() == ref.slot_of_expert.tolist()
+        assert eos.cpu().tolist() == ref.expert_of_slot.tolist()
+        assert lu.cpu().tolist() == ref.last_use.tolist()
+    banks = pool.view(S, -1)[:, :4].contiguous().view(torch.int32).cpu().numpy()[:, 0]
+    for s, e in enumerate(eos.cpu().tolist()):
+        if e >= 0:
+            assert banks[s] == e
+
+
+def test_lru_rejects_out_of_range_ids():
+    E, S = 16, 4
+    desc, bl, cache, (soe, eos, lu, pool), ws = _lru_setup(E, S)
+    desc.k = 2
+    copy_stream = torch.cuda.Stream()
+    assert ftm.ftm_device_status(True) == 0
+    before = (soe.clone(), eos.clone(), lu.clone())
+    for bad in (E, -1):
+        t = torch.tensor([[1, bad]], dtype=torch.int32, device="cuda")
+        with pytest.raises(ftm.FtmError) as ei:
+            ftm.ftm_slot_lookup_update(desc, cache, t, 1, ws.ptr, ws.nbytes, None, copy_stream)
+        assert ei.value.status == 1 and cache.step == 0
+        assert all(torch.equal(a, b) for a, b in zip(before, (soe, eos, lu)))
+        assert ftm.ftm_device_status(True) == 2
+
+
+@pytest.mark.parametrize("T", [40, 700])     # one-block and three-pass permutation
+def test_permute_skips_out_of_range_ids(T):
+    E, k = 12, 3
+    rng = np.random.default_rng(T)
+    ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    ids[3, 1] = E
+    ids[T - 1, 0] = -5
+    desc = ftm.LayerDesc(128, E, k, 128, 0, E, ftm.FTM_BF16, 0)
+    P = T * k
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.full((P,), 123, dtype=torch.int32, device="cuda")
+    inv = torch.full((P,), 123, dtype=torch.int32, device="cuda")
+    ws = Workspace(ftm.ftm_permute_workspace_bytes(desc, T))
+    assert ftm.ftm_device_status(True) == 0
+    ftm.ftm_permute(desc, torch.from_numpy(ids).cuda(), T, counts, offsets, perm, inv, ws.ptr, ws.nbytes)
+    torch.cuda.synchronize()
+    assert ftm.ftm_device_status(True) == 2
+    flat = ids.ravel()
+    ok = (flat >= 0) & (flat < E)
+    want_counts = np.bincount(flat[ok], minlength=E)
+    assert np.array_equal(counts.cpu().numpy(), want_counts)
+    assert np.array_equal(offsets.cpu().numpy(), np.concatenate([[0], np.cumsum(want_counts)]))
+    order = sorted(np.nonzero(ok)[0].tolist(), key=lambda q: (flat[q], q))
+    pm, iv = perm.cpu().numpy(), inv.cpu().numpy()
+    assert pm[:len(order)].tolist() == order and (pm[len(order):] == -1).all()
+    assert (iv[~ok] == -1).all() and all(iv[q] == pos for pos, q in enumerate(order))
+
+
+def test_combine_skips_unplaced_pairs():
+    desc = ftm.LayerDesc(128, 4, 2, 128, 0, 4, ftm.FTM_F32, 0)
+    T, k, d = 2, 2, 128
+    y = torch.arange(T * k * d, dtype=torch.float32, device="cuda").view(T * k, d) / 100
+    inv = torch.tensor([3, -1, 1, 2], dtype=torch.int32, device="cuda")
+    gw = torch.tensor([[0.25, 0.75], [0.5, 0.5]], dtype=torch.float32, device="cuda")
+    out = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    assert ftm.ftm_device_status(True) == 0
+    ftm.ftm_combine(desc, y, inv, gw, T, out)
+    torch.cuda.synchronize()
+    assert ftm.ftm_device_status(True) == 2
+    yc = y.cpu().numpy().astype(np.float64)
+    want = np.stack([0.25 * yc[3], 0.5 * yc[1] + 0.5 * yc[2]])
+    assert np.allclose(out.cpu().numpy(), want, rtol=1e-6)
