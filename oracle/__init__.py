@@ -67,6 +67,8 @@ def lib():
         L.orc_permute.argtypes = [p, i32, i32, i32, p, p, p, p]
         L.orc_lru_step.argtypes = [i32, i32, p, p, p, i64, p, i32, p, p, p, p, p]
         L.orc_lru_step.restype = i32
+        L.orc_lru_step_reserve.argtypes = [i32, i32, p, p, p, i64, i64, p, i32, p, p, p, p, p]
+        L.orc_lru_step_reserve.restype = i32
         L.orc_lru_resize.argtypes = [i32, i32, p, p, p, i32, p, p, p, p]
         L.orc_lru_resize.restype = i32
         L.orc_expert_ffn.argtypes = [p, i32, i32, i32, p, p, p, i32, p]
@@ -266,6 +268,29 @@ class LRUState:
             self.step += 1
         misses = [(int(me[i]), int(ms[i])) for i in range(int(nm[0]))]
         return rc, misses, int(nd[0]), int(nh[0])
+
+    def update_reserve(self, keys: np.ndarray, reserve: int):
+        """One step whose misses may only take slots with last_use < reserve
+        (see orc_lru_step_reserve).  Returns (status, misses, distinct, hits)."""
+        keys = np.ascontiguousarray(keys, dtype=np.int32).ravel()
+        mk = np.empty(max(1, self.E), dtype=np.int32)
+        ms = np.empty(max(1, self.E), dtype=np.int32)
+        nd, nh, nm = (np.zeros(1, dtype=np.int32) for _ in range(3))
+        rc = lib().orc_lru_step_reserve(self.E, self.S, _p(self.slot_of_expert), _p(self.expert_of_slot),
+                                        _p(self.last_use), self.step, int(reserve), _p(keys), keys.size, _p(mk),
+                                        _p(ms), _p(nd), _p(nh), _p(nm))
+        if rc == 0:
+            self.step += 1
+        misses = [(int(mk[i]), int(ms[i])) for i in range(int(nm[0]))]
+        return rc, misses, int(nd[0]), int(nh[0])
+
+    def stage_layer(self, layer: int, E: int, overlap: bool):
+        """One staging step of a cache shared by layers of E experts (this
+        state's E is then n_layers * E): all E experts of `layer` become
+        resident.  overlap: the step runs while the previous step's layer
+        computes, so that step's slots are kept (reserve = step - 1)."""
+        keys = np.arange(layer * E, (layer + 1) * E, dtype=np.int32)
+        return self.update_reserve(keys, self.step - 1 if overlap else self.step)
 
     def resize(self, S_new: int):
         """Elastic resize to S_new slots (see orc_lru_resize).  Returns the new

@@ -392,6 +392,60 @@ int orc_lru_step(int E, int S, int32_t* slot_of_expert, int32_t* expert_of_slot,
 }
 
 /* ---------------------------------------------------------------------------
+ * Cache step of a cache shared by several layers, with slots held back.
+ * Keys: the cache holds n_keys entries; in a cache shared by several layers of
+ * E experts each, layer l's expert e is key l*E + e.  Step s requests the
+ * distinct keys in keys[0..n).  As in orc_lru_step, hits set last_use = s and
+ * misses, in ascending key, each take the slot with the smallest last_use
+ * (ties: lowest slot index) -- but only among slots with last_use < reserve
+ * (reserve <= s): slots used in steps reserve..s-1 keep their experts, because
+ * the compute of those steps may still be reading them while this step's
+ * copies run (pomoai.com FreeToken hub, prefill-overlap paragraph: layer n+1's
+ * experts are copied while layer n computes, which needs room for two whole
+ * layers).  With reserve = s this is orc_lru_step.  Returns -1 with the state
+ * untouched when the misses outnumber the slots they may take.
+ * ------------------------------------------------------------------------- */
+int orc_lru_step_reserve(int n_keys, int S, int32_t* slot_of_key, int32_t* key_of_slot, int64_t* last_use,
+                         int64_t s, int64_t reserve, const int32_t* keys, int n, int32_t* miss_key,
+                         int32_t* miss_slot, int32_t* n_distinct, int32_t* n_hits, int32_t* n_miss) {
+  uint8_t* want = (uint8_t*)calloc((size_t)n_keys, 1);
+  for (int i = 0; i < n; ++i) want[keys[i]] = 1;
+  int distinct = 0, hits = 0, misses = 0, free_slots = 0;
+  for (int key = 0; key < n_keys; ++key) {
+    if (!want[key]) continue;
+    ++distinct;
+    if (slot_of_key[key] >= 0) ++hits; else ++misses;
+  }
+  /* slots a miss may take: not used since `reserve`, and not hit by this step */
+  for (int j = 0; j < S; ++j) {
+    int hit = key_of_slot[j] >= 0 && want[key_of_slot[j]];
+    if (last_use[j] < reserve && !hit) ++free_slots;
+  }
+  *n_distinct = distinct;
+  if (misses > free_slots) { free(want); *n_hits = 0; *n_miss = 0; return -1; }
+  for (int key = 0; key < n_keys; ++key)
+    if (want[key] && slot_of_key[key] >= 0) last_use[slot_of_key[key]] = s;
+  int placed = 0;
+  for (int key = 0; key < n_keys; ++key) {
+    if (!want[key] || slot_of_key[key] >= 0) continue;
+    int victim = -1;
+    for (int j = 0; j < S; ++j)
+      if (last_use[j] < reserve && (victim < 0 || last_use[j] < last_use[victim])) victim = j;
+    if (key_of_slot[victim] >= 0) slot_of_key[key_of_slot[victim]] = -1;
+    key_of_slot[victim] = key;
+    slot_of_key[key] = victim;
+    last_use[victim] = s;
+    miss_key[placed] = key;
+    miss_slot[placed] = victim;
+    ++placed;
+  }
+  *n_hits = hits;
+  *n_miss = placed;
+  free(want);
+  return 0;
+}
+
+/* ---------------------------------------------------------------------------
  * Elastic slot-pool resize.  The pages let the expert cache's share of VRAM
  * change at run time without restarting the engine or reloading weights
  * (pomoai.com FreeToken hub, the two-level expert memory paragraph; freelamp.com

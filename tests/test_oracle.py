@@ -302,6 +302,121 @@ def test_lru_matches_list_replay(E, S, n, seed):
         assert nh == len(set(ids.tolist())) - len(m)
 
 
+class ListLRUReserve:
+    """Independent model of a step whose misses may only take slots not used
+    since step `reserve`: an eviction list (front = least recently used, a
+    step's touched slots appended in slot order) plus the step each slot was
+    last touched; a miss takes the first slot of the list touched before
+    `reserve`."""
+
+    def __init__(self, n_keys, S):
+        self.order = list(range(S))
+        self.key = [-1] * S
+        self.touched_at = [-1] * S
+        self.where = {}
+
+    def step(self, keys, s, reserve):
+        want = sorted(set(int(k) for k in keys))
+        hits = [self.where[k] for k in want if k in self.where]
+        misses_needed = sum(1 for k in want if k not in self.where)
+        free = [sl for sl in self.order if self.touched_at[sl] < reserve and sl not in hits]
+        if misses_needed > len(free):
+            return None
+        for sl in hits:
+            self.order.remove(sl)
+        touched = list(hits)
+        misses = []
+        for k in want:
+            if k in self.where:
+                continue
+            sl = next(x for x in self.order if self.touched_at[x] < reserve)
+            self.order.remove(sl)
+            if self.key[sl] >= 0:
+                del self.where[self.key[sl]]
+            self.key[sl] = k
+            self.where[k] = sl
+            touched.append(sl)
+            misses.append((k, sl))
+        for sl in touched:
+            self.touched_at[sl] = s
+        self.order.extend(sorted(touched))
+        return misses
+
+
+def test_lru_reserve_hand_worked():
+    st = oracle.LRUState(E=8, S=4)
+    assert st.update_reserve(np.array([0, 1]), 0)[1] == [(0, 0), (1, 1)]     # empty slots in index order
+    assert st.update_reserve(np.array([2, 3]), 0)[1] == [(2, 2), (3, 3)]     # step 0's slots kept
+    assert st.update_reserve(np.array([4, 5]), 1)[1] == [(4, 0), (5, 1)]     # step 1's slots kept
+    assert st.last_use.tolist() == [2, 2, 1, 1]
+    before = st.copy()
+    # step 3 keeps steps 2's slots: key 2 is a hit (slot 2), only slot 3 may be
+    # taken, but 6 and 7 both miss -> refused, state untouched
+    rc, m, nd, nh = st.update_reserve(np.array([6, 7, 2]), 2)
+    assert rc == -1 and nd == 3
+    assert np.array_equal(st.last_use, before.last_use) and st.step == 3
+    assert np.array_equal(st.slot_of_expert, before.slot_of_expert)
+    # without holding step 2 back: slot 3 (last_use 1), then slot 0 (2, lower index than 1)
+    rc, m, nd, nh = st.update_reserve(np.array([6, 7, 2]), 3)
+    assert rc == 0 and m == [(6, 3), (7, 0)] and nh == 1
+    assert st.expert_of_slot.tolist() == [7, 5, 2, 6] and st.last_use.tolist() == [3, 2, 3, 3]
+    assert st.slot_of_expert.tolist() == [-1, -1, 2, -1, -1, 1, 3, 0]
+
+
+@pytest.mark.parametrize("E,S,n,seed", [(16, 4, 3, 0), (64, 16, 10, 1), (256, 64, 40, 2)])
+def test_lru_reserve_equal_to_step_is_the_plain_lru(E, S, n, seed):
+    rng = np.random.default_rng(seed)
+    a, b = oracle.LRUState(E, S), oracle.LRUState(E, S)
+    zipf = 1.0 / np.arange(1, E + 1) ** 1.1
+    zipf /= zipf.sum()
+    for step in range(200):
+        ids = rng.choice(E, size=n, p=zipf)
+        ra = a.update(ids)
+        rb = b.update_reserve(ids, b.step)
+        assert ra == rb
+        assert np.array_equal(a.slot_of_expert, b.slot_of_expert)
+        assert np.array_equal(a.expert_of_slot, b.expert_of_slot) and np.array_equal(a.last_use, b.last_use)
+
+
+@pytest.mark.parametrize("layers,E,S,seed", [(5, 8, 16, 0), (4, 8, 20, 1), (6, 16, 40, 2), (4, 8, 12, 3)])
+def test_lru_reserve_matches_list_replay(layers, E, S, seed):
+    """Whole-layer staging with the previous step held back, mixed with routed
+    steps of random keys and random hold-back windows, against the list model."""
+    rng = np.random.default_rng(seed)
+    st = oracle.LRUState(layers * E, S)
+    ref = ListLRUReserve(layers * E, S)
+    for it in range(120):
+        s = st.step
+        if rng.random() < 0.5:
+            layer = int(rng.integers(layers))
+            keys = np.arange(layer * E, (layer + 1) * E)
+        else:
+            keys = rng.choice(layers * E, size=int(rng.integers(1, E + 1)))
+        reserve = s - int(rng.integers(0, 3))
+        rc, m, nd, nh = st.update_reserve(keys, reserve)
+        rm = ref.step(keys, s, reserve)
+        if rm is None:
+            assert rc == -1 and st.step == s
+            continue
+        assert rc == 0 and m == rm, it
+        assert st.expert_of_slot.tolist() == ref.key
+        for k, sl in ref.where.items():
+            assert st.slot_of_expert[k] == sl
+        assert (st.slot_of_expert >= 0).sum() == len(ref.where)
+
+
+def test_stage_overlap_needs_two_whole_layers():
+    # staging layer l+1 while layer l computes keeps layer l's E slots: it fits
+    # exactly when the cache holds two whole layers (S >= 2E)
+    for S, ok in ((16, True), (15, False), (24, True)):
+        st = oracle.LRUState(4 * 8, S)
+        assert st.stage_layer(0, 8, overlap=False)[0] == 0
+        rcs = [st.stage_layer(l, 8, overlap=True)[0] for l in range(1, 4)]
+        assert all(rc == 0 for rc in rcs) == ok
+        if not ok:
+            assert rcs[0] == -1
+
+
 def test_lru_resize_hand_worked():
     st = oracle.LRUState(E=10, S=4)
     st.expert_of_slot[:] = [5, -1, 2, 7]
