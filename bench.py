@@ -178,17 +178,18 @@ def source_hash() -> str:
     return h.hexdigest()[:12]
 
 
-def packed_banks(cfg, cache_dir: str, local_rank: int, dist):
+def packed_banks(cfg, cache_dir: str, local_rank: int, dist, seed: int = 0):
     """The layer's packed banks, drawn once and kept on the host's disk so later
     runs (and the other ranks of this one) read them instead of drawing again."""
     from synth.device import pack_banks
     if not cache_dir:
-        return None
-    path = os.path.join(cache_dir, f"{cfg.name}_{source_hash()}_{hashlib.sha1(repr(cfg).encode()).hexdigest()[:8]}.npy")
+        return None if seed == 0 else pack_banks(cfg, seed)
+    tag = hashlib.sha1(repr(cfg).encode()).hexdigest()[:8]
+    path = os.path.join(cache_dir, f"{cfg.name}_{source_hash()}_{tag}_s{seed}.npy")
     if local_rank == 0 and not os.path.exists(path):
         try:
             os.makedirs(cache_dir, exist_ok=True)
-            banks = pack_banks(cfg)
+            banks = pack_banks(cfg, seed)
             tmp = path + f".tmp{os.getpid()}"
             np.save(tmp, banks)
             os.replace(tmp, path)
@@ -198,7 +199,7 @@ def packed_banks(cfg, cache_dir: str, local_rank: int, dist):
         dist.barrier()
     if os.path.exists(path):
         return np.load(path, mmap_mode="r")
-    return None
+    return None if seed == 0 else pack_banks(cfg, seed)
 
 
 def device_layer(cfg, args, local, dist):
@@ -616,6 +617,72 @@ def run_trace(cfg, T, args, dist, local):
     }
 
 
+def run_layers_pipeline(cfg, T, n_layers, args, local):
+    """Prefill of n_layers layers of one shape (each with its own seed) through
+    one slot cache of two layers' size (S = 2E), every layer's experts staged
+    from pinned host memory: layer l+1's copies overlapped with layer l's
+    compute, against staging then computing each layer.  One step = one pass
+    over the stack, the output of layer l feeding layer l+1."""
+    from synth.device import Workspace, to_device_storage
+    E = cfg.E
+    S = 2 * E
+    desc = ftm.desc_for(synth.scaled(cfg, S=S))
+    bl = ftm.ftm_get_bank_layout(desc)
+    bb = bl.bank_bytes
+    host_pool = torch.empty(n_layers * E * bb, dtype=torch.uint8, pin_memory=True)
+    hp = host_pool.numpy()
+    weights, keep = [], []
+    for l in range(n_layers):
+        banks = packed_banks(cfg, args.bank_cache, local, None, seed=l)
+        hp[l * E * bb:(l + 1) * E * bb] = np.asarray(banks[:E]).reshape(-1)
+        layer = synth.Layer(cfg, seed=l)
+        wr = to_device_storage(layer.router_storage(), cfg.act_dtype)
+        b = layer.bias()
+        bias = None if b is None else torch.from_numpy(b).cuda()
+        keep += [wr, bias]
+        weights.append(ftm.LayerWeights(wr.data_ptr(), None if bias is None else bias.data_ptr(), None, None, None))
+    pool = torch.zeros(S * bb, dtype=torch.uint8, device="cuda")
+    soe = torch.full((n_layers * E,), -1, dtype=torch.int32, device="cuda")
+    eos = torch.full((S,), -1, dtype=torch.int32, device="cuda")
+    lu = torch.full((S,), -1, dtype=torch.int64, device="cuda")
+    scratch = torch.zeros(ftm.ftm_slot_host_scratch_ints(desc), dtype=torch.int32, pin_memory=True)
+    cache = ftm.SlotCache(soe.data_ptr(), eos.data_ptr(), lu.data_ptr(), 0, pool.data_ptr(), host_pool.data_ptr(),
+                          scratch.data_ptr(), 0, 0, 0, 0, n_layers * E, 0)
+    x0 = to_device_storage(synth.Layer(cfg, 0).hidden_storage(T), cfg.act_dtype)
+    acts = [x0] + [torch.empty((T, cfg.d), dtype=torch.bfloat16, device="cuda") for _ in range(n_layers)]
+    ws = Workspace(ftm.ftm_workspace_bytes(desc, T))
+    stream, copy_stream = torch.cuda.Stream(), torch.cuda.Stream()
+    passes = max(1, min(args.steps, 10))
+    out = {}
+    for mode in ("overlap", "serial"):
+        used = None
+        for _ in range(2):                            # warm-up passes
+            used = ftm.ftm_moe_layers_forward(desc, weights, cache, acts[:-1], T, acts[1:], mode == "overlap",
+                                              ws.ptr, ws.nbytes, stream, copy_stream)
+        torch.cuda.synchronize()
+        misses0 = 0
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(passes):
+            ftm.ftm_moe_layers_forward(desc, weights, cache, acts[:-1], T, acts[1:], mode == "overlap", ws.ptr,
+                                       ws.nbytes, stream, copy_stream)
+            misses0 += cache.last_misses
+        t1.record(stream)
+        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1)
+        out[mode] = {"ms_per_pass": ms / passes, "ms_per_layer": ms / passes / n_layers, "overlap_ran": bool(used),
+                     "last_layer_misses_per_pass": misses0 / passes,
+                     # every layer misses like the last one: the cache holds two of the four layers
+                     "h2d_gbs": misses0 * n_layers * bb / (ms * 1e-3) / 1e9 if misses0 else None}
+    status = ftm.ftm_device_status(True)
+    return {"workload": f"{cfg.name} x{n_layers} layers staged through one cache (S = 2E = {S}) T={T}",
+            "value": T * n_layers / (out["overlap"]["ms_per_pass"] * 1e-3), "unit": "layer-tokens/s",
+            "passes": passes, "overlap": out["overlap"], "serial": out["serial"],
+            "speedup_overlap": out["serial"]["ms_per_pass"] / out["overlap"]["ms_per_pass"],
+            "bank_bytes_per_layer": E * bb, "bound": "pcie (host-to-device expert copies)",
+            "launch": "eager ftm_moe_layers_forward; layer l's output feeds layer l+1", "device_status": status}
+
+
 # --------------------------------------------------------------------------- CPU oracle
 def cpu_model() -> str:
     try:
@@ -757,6 +824,8 @@ def main():
     head_cfg = synth.CONFIGS[head[0]]
     for name, Ts in suite:
         cfg = synth.CONFIGS[name]
+        if name == "35b_prefill":
+            records.append(run_layers_pipeline(cfg, Ts[0], 4, args, local))
         if cfg.lru:
             for T in Ts:
                 records.append(run_trace(cfg, T, args, dist, local))

@@ -26,6 +26,8 @@ from .binding import (  # noqa: F401
     ftm_last_error,
     ftm_moe_layer_forward,
     ftm_moe_layer_forward_noalloc,
+    ftm_moe_layers_forward,
+    ftm_last_warning,
     ftm_permute,
     ftm_permute_workspace_bytes,
     ftm_route,
@@ -34,6 +36,7 @@ from .binding import (  # noqa: F401
     ftm_slot_host_scratch_ints,
     ftm_slot_lookup_update,
     ftm_slot_resize,
+    ftm_slot_stage_layer,
     ftm_slot_workspace_bytes,
     ftm_workspace_bytes,
     library,

@@ -31,12 +31,13 @@ class BankLayout(ctypes.Structure):
 class SlotCache(ctypes.Structure):
     _fields_ = [("slot_of_expert", c_p), ("expert_of_slot", c_p), ("last_use", c_p), ("step", c_i64),
                 ("slot_pool", c_p), ("host_pool", c_p), ("host_scratch", c_p), ("last_distinct", c_i32),
-                ("last_hits", c_i32), ("last_misses", c_i32), ("fail_before_copy", c_i32)]
+                ("last_hits", c_i32), ("last_misses", c_i32), ("fail_before_copy", c_i32), ("n_keys", c_i32),
+                ("key_base", c_i32)]
 
 
 class LayerWeights(ctypes.Structure):
     _fields_ = [("w_router", c_p), ("router_bias", c_p), ("slot_pool", c_p), ("slot_of_expert", c_p),
-                ("shared_bank", c_p)]
+                ("shared_bank", c_p), ("act_scale", c_p)]
 
 
 class FtmError(RuntimeError):
@@ -71,7 +72,11 @@ def library() -> ctypes.CDLL:
         L.ftm_slot_workspace_bytes.restype = c_sz
         L.ftm_slot_lookup_update.argtypes = [P(LayerDesc), P(SlotCache), c_p, c_i32, c_p, c_sz, c_p, c_p]
         L.ftm_slot_resize.argtypes = [P(LayerDesc), P(SlotCache), c_i32, P(SlotCache), c_p, c_sz, c_p]
-        L.ftm_expert_ffn.argtypes = [P(LayerDesc), c_p, c_i32, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_sz, c_p]
+        L.ftm_slot_stage_layer.argtypes = [P(LayerDesc), P(SlotCache), c_i32, c_i32, c_p, c_p, c_sz, c_p, c_p]
+        L.ftm_moe_layers_forward.argtypes = [P(LayerDesc), c_i32, P(LayerWeights), P(SlotCache), P(c_p), c_i32,
+                                             P(c_p), c_i32, P(c_i32), c_p, c_sz, c_p, c_p]
+        L.ftm_last_warning.restype = ctypes.c_char_p
+        L.ftm_expert_ffn.argtypes = [P(LayerDesc), c_p, c_i32, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_sz, c_p]
         L.ftm_ffn_workspace_bytes.argtypes = [P(LayerDesc), c_i32]
         L.ftm_ffn_workspace_bytes.restype = c_sz
         L.ftm_combine.argtypes = [P(LayerDesc), c_p, c_p, c_p, c_i32, c_p, c_p]
@@ -86,7 +91,8 @@ def library() -> ctypes.CDLL:
         L.ftm_workspace_bytes.argtypes = [P(LayerDesc), c_i32]
         L.ftm_workspace_bytes.restype = c_sz
         for name in ("ftm_get_bank_layout", "ftm_route", "ftm_permute", "ftm_slot_lookup_update", "ftm_slot_resize",
-                     "ftm_expert_ffn", "ftm_combine", "ftm_moe_layer_forward"):
+                     "ftm_slot_stage_layer", "ftm_expert_ffn", "ftm_combine", "ftm_moe_layer_forward",
+                     "ftm_moe_layers_forward"):
             getattr(L, name).restype = c_i32
         _lib = L
     return _lib
@@ -167,15 +173,44 @@ def ftm_slot_resize(desc, cache: SlotCache, S_new: int, new_cache: SlotCache, wo
                                      _ptr(workspace), ws_bytes, _stream(stream)))
 
 
+def ftm_slot_stage_layer(desc, cache: SlotCache, layer: int, hold_previous: bool, after_event, workspace, ws_bytes,
+                         copy_stream=None, ready_event=None):
+    """after_event / ready_event: torch.cuda.Event (or None)."""
+    _check(library().ftm_slot_stage_layer(ctypes.byref(desc), ctypes.byref(cache), layer, 1 if hold_previous else 0,
+                                          None if after_event is None else after_event.cuda_event, _ptr(workspace),
+                                          ws_bytes, _stream(copy_stream),
+                                          None if ready_event is None else ready_event.cuda_event))
+
+
+def ftm_moe_layers_forward(desc, weights, cache: SlotCache, xs, T, outs, overlap: bool, workspace, ws_bytes,
+                           stream=None, copy_stream=None) -> bool:
+    """weights: sequence of LayerWeights; xs / outs: sequences of device tensors.
+    Returns whether the copy/compute overlap ran."""
+    n = len(weights)
+    W = (LayerWeights * n)(*weights)
+    X = (c_p * n)(*[_ptr(t) for t in xs])
+    O = (c_p * n)(*[_ptr(t) for t in outs])
+    used = c_i32(0)
+    _check(library().ftm_moe_layers_forward(ctypes.byref(desc), n, W, ctypes.byref(cache), X, T, O,
+                                            1 if overlap else 0, ctypes.byref(used), _ptr(workspace), ws_bytes,
+                                            _stream(stream), _stream(copy_stream)))
+    return bool(used.value)
+
+
+def ftm_last_warning() -> str:
+    return library().ftm_last_warning().decode()
+
+
 def ftm_ffn_workspace_bytes(desc, T) -> int:
     return int(library().ftm_ffn_workspace_bytes(ctypes.byref(desc), T))
 
 
 def ftm_expert_ffn(desc, x, T, offsets, perm, slot_of_expert, slot_pool, shared_bank, y, workspace, ws_bytes,
-                   stream=None):
+                   stream=None, act_scale=None):
+    """act_scale: device fp32[2] (NVFP4 activation global scales of x and h) or None."""
     _check(library().ftm_expert_ffn(ctypes.byref(desc), _ptr(x), T, _ptr(offsets), _ptr(perm), _ptr(slot_of_expert),
-                                    _ptr(slot_pool), _ptr(shared_bank), _ptr(y), _ptr(workspace), ws_bytes,
-                                    _stream(stream)))
+                                    _ptr(slot_pool), _ptr(shared_bank), _ptr(act_scale), _ptr(y), _ptr(workspace),
+                                    ws_bytes, _stream(stream)))
 
 
 def ftm_combine(desc, y, inv, topk_w, T, out, stream=None):

@@ -15,9 +15,9 @@ cudaError_t launch_permute(const int32_t* ids, int P, int E, int32_t* counts, in
                            int32_t* inv, void* ws, cudaStream_t st);
 size_t permute_workspace_bytes(int E, int64_t P);
 size_t lru_workspace_bytes(int E, int S);
-cudaError_t launch_lru_step(const int32_t* ids, int P, int E, int S, int64_t step, int32_t* soe, int32_t* eos,
-                            int64_t* lu, int32_t* ws, cudaStream_t st);
-cudaError_t launch_lru_restore(int E, int S, int32_t* soe, int32_t* eos, int64_t* lu, const int32_t* ws,
+cudaError_t launch_lru_step(const int32_t* ids, int P, int E, int S, int64_t step, int64_t reserve, int key_base,
+                            int32_t* soe, int32_t* eos, int64_t* lu, int32_t* ws, cudaStream_t st);
+cudaError_t launch_lru_restore(int E, int S, int key_base, int32_t* soe, int32_t* eos, int64_t* lu, int32_t* ws,
                                int n_dirty, cudaStream_t st);
 cudaError_t launch_slot_resize(int E, int S_old, const int32_t* eos_old, const int64_t* lu_old, int S_new,
                                int32_t* soe_new, int32_t* eos_new, int64_t* lu_new, const void* old_pool,
@@ -177,6 +177,131 @@ cudaEvent_t copy_event() {
   return ev;
 }
 
+// Cache arguments shared by the lookup and the staging calls.
+ftm_status check_cache(const ftm_layer_desc* L, const ftm_slot_cache* C, const char* who) {
+  if (!C || !C->slot_of_expert || !C->expert_of_slot || !C->last_use || !C->slot_pool || !C->host_pool ||
+      !C->host_scratch)
+    return fail(FTM_ERR_INVALID_ARG, "%s: cache has a NULL member", who);
+  if (L->S > 4096) return fail(FTM_ERR_UNSUPPORTED, "LRU cache supports S <= 4096 (S=%d)", L->S);
+  const int n_keys = C->n_keys ? C->n_keys : L->E;
+  if (n_keys < L->E || C->key_base < 0 || static_cast<int64_t>(C->key_base) + L->E > n_keys)
+    return fail(FTM_ERR_INVALID_ARG, "%s: key_base=%d + E=%d outside the cache's %d keys", who, C->key_base, L->E,
+                n_keys);
+  cudaPointerAttributes pa;
+  if (cudaPointerGetAttributes(&pa, C->host_pool) != cudaSuccess || pa.type != cudaMemoryTypeHost) {
+    cudaGetLastError();
+    return fail(FTM_ERR_INVALID_ARG, "%s: host_pool is not pinned host memory", who);
+  }
+  return FTM_OK;
+}
+
+cudaEvent_t list_event() {
+  static thread_local cudaEvent_t ev = nullptr;
+  static thread_local int dev = -1;
+  int cur = 0;
+  cudaGetDevice(&cur);
+  if (!ev || dev != cur) {
+    if (ev) cudaEventDestroy(ev);
+    ev = nullptr;
+    if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) ev = nullptr;
+    dev = cur;
+  }
+  return ev;
+}
+
+// One cache step of the layer at C->key_base: the lookup/update kernel on
+// `lru_stream` (ids == nullptr: all E experts of the layer), after `after`
+// when given, the miss list read back (the host waits for that kernel only),
+// then one bank copy per miss on `copy_stream` (also after `after`).  Victims
+// are the slots with last_use < reserve.  On a copy failure the state is
+// rolled back (slots a copy may have written left empty).
+ftm_status cache_step(const ftm_layer_desc* L, ftm_slot_cache* C, const int32_t* ids, int P, int64_t reserve,
+                      int32_t* ws, cudaStream_t lru_stream, cudaStream_t copy_stream, cudaEvent_t after,
+                      int* misses_out) {
+  *misses_out = 0;
+  cudaError_t e;
+  // the step rewrites the entries of the keys it evicts: the compute that
+  // reads them (done when `after` completes) must be over first
+  if (after && (e = cudaStreamWaitEvent(lru_stream, after, 0)) != cudaSuccess) return cuda_fail(e, "lru stream wait");
+  prof_mark(FTM_K_LRU, lru_stream, false);
+  e = launch_lru_step(ids, P, L->E, L->S, C->step, reserve, C->key_base, C->slot_of_expert,
+                                  C->expert_of_slot, C->last_use, ws, lru_stream);
+  prof_mark(FTM_K_LRU, lru_stream, true);
+  if (e != cudaSuccess) return cuda_fail(e, "lru step launch");
+  const size_t hdr = sizeof(int32_t) * (4 + 2 * static_cast<size_t>(L->E));
+  if ((e = cudaMemcpyAsync(C->host_scratch, ws, hdr, cudaMemcpyDeviceToHost, lru_stream)) != cudaSuccess)
+    return cuda_fail(e, "miss list copy");
+  cudaEvent_t lev = list_event();
+  if (!lev) return fail(FTM_ERR_CUDA, "could not create the miss-list event");
+  if ((e = cudaEventRecord(lev, lru_stream)) != cudaSuccess) return cuda_fail(e, "miss list event record");
+  if ((e = cudaEventSynchronize(lev)) != cudaSuccess) return cuda_fail(e, "lru step");
+  const int32_t* h = C->host_scratch;
+  C->last_distinct = h[1];
+  C->last_hits = h[2];
+  C->last_misses = h[3];
+  if (h[0] == FTM_ERR_INVALID_ARG)
+    return fail(FTM_ERR_INVALID_ARG, "step %lld: topk_ids holds an expert id outside [0, %d); state unchanged",
+                static_cast<long long>(C->step), L->E);
+  if (h[0] == FTM_ERR_CAPACITY)
+    return fail(FTM_ERR_CAPACITY, "step %lld requests %d distinct experts, more than the %d slots it may fill",
+                static_cast<long long>(C->step), h[1], L->S);
+  ftm_bank_layout bl;
+  bank_layout(L, &bl);
+  const int misses = h[3];
+  if (misses > 0 && after && copy_stream != lru_stream &&
+      (e = cudaStreamWaitEvent(copy_stream, after, 0)) != cudaSuccess)
+    return cuda_fail(e, "copy stream wait");
+  bool copy_failed = false;
+  const char* why = nullptr;
+  int n_dirty = 0;     // miss-list slots a copy may have written
+  for (int i = 0; i < misses && !copy_failed; ++i) {
+    if (C->fail_before_copy > 0 && i + 1 == C->fail_before_copy) {
+      copy_failed = true;
+      why = "injected copy failure (fail_before_copy)";
+      break;
+    }
+    const int key = h[4 + 2 * i], sl = h[4 + 2 * i + 1];
+    e = cudaMemcpyAsync(static_cast<uint8_t*>(C->slot_pool) + static_cast<size_t>(sl) * bl.bank_bytes,
+                        static_cast<const uint8_t*>(C->host_pool) + static_cast<size_t>(key) * bl.bank_bytes,
+                        bl.bank_bytes, cudaMemcpyHostToDevice, copy_stream);
+    n_dirty = i + 1;     // a copy that failed to issue may still have started
+    if (e != cudaSuccess) { copy_failed = true; why = cudaGetErrorString(e); }
+  }
+  if (copy_failed) {
+    C->fail_before_copy = 0;
+    cudaError_t e2 = launch_lru_restore(L->E, L->S, C->key_base, C->slot_of_expert, C->expert_of_slot, C->last_use,
+                                        ws, n_dirty, lru_stream);
+    if (e2 == cudaSuccess) e2 = cudaStreamSynchronize(lru_stream);
+    return fail(FTM_ERR_CUDA, "a miss copy failed (%s) with %d of %d copies issued; slot state rolled back, the "
+                "%d slot(s) a copy may have written left empty%s", why, n_dirty, misses, n_dirty,
+                e2 == cudaSuccess ? "" : " -- rollback failed too");
+  }
+  C->step += 1;
+  *misses_out = misses;
+  return FTM_OK;
+}
+
+thread_local char g_warn[256] = "";
+
+// Events of the multi-layer pipeline, per thread and device: [0, 1] a layer's
+// experts are in their slots (by layer parity), [2, 3] a layer's compute is
+// done, [4] the work enqueued before the call.
+cudaEvent_t pipe_event(int i) {
+  static thread_local cudaEvent_t ev[5] = {};
+  static thread_local int dev = -1;
+  int cur = 0;
+  cudaGetDevice(&cur);
+  if (dev != cur) {
+    for (auto& x : ev) {
+      if (x) cudaEventDestroy(x);
+      x = nullptr;
+    }
+    dev = cur;
+  }
+  if (!ev[i] && cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess) ev[i] = nullptr;
+  return ev[i];
+}
+
 }  // namespace
 
 ftm_status ftm::report_error(ftm_status s, const char* msg) { return fail(s, "%s", msg); }
@@ -300,11 +425,14 @@ ftm_status ftm_slot_resize(const ftm_layer_desc* L, const ftm_slot_cache* C, int
       C_new->last_use == C->last_use)
     return fail(FTM_ERR_INVALID_ARG, "ftm_slot_resize: new state arrays must be distinct from the old ones");
   if ((s = check_ws(workspace, ws_bytes, lru_workspace_bytes(L->E, L->S), "ftm_slot_resize"))) return s;
-  cudaError_t e = launch_slot_resize(L->E, L->S, C->expert_of_slot, C->last_use, S_new, C_new->slot_of_expert,
+  const int n_keys = C->n_keys ? C->n_keys : L->E;
+  cudaError_t e = launch_slot_resize(n_keys, L->S, C->expert_of_slot, C->last_use, S_new, C_new->slot_of_expert,
                                      C_new->expert_of_slot, C_new->last_use, C->slot_pool, C_new->slot_pool,
                                      bl.bank_bytes, static_cast<int32_t*>(workspace), S_(stream));
   if (e != cudaSuccess) return cuda_fail(e, "slot resize launch");
   C_new->step = C->step;
+  C_new->n_keys = C->n_keys;
+  C_new->key_base = C->key_base;
   C_new->last_distinct = C_new->last_hits = C_new->last_misses = 0;
   return FTM_OK;
 }
@@ -313,74 +441,51 @@ ftm_status ftm_slot_lookup_update(const ftm_layer_desc* L, ftm_slot_cache* C, co
                                   void* workspace, size_t ws_bytes, void* compute_stream, void* copy_stream) {
   ftm_status s = check_desc(L);
   if (s || (s = check_T(T))) return s;
-  if (!C || !C->slot_of_expert || !C->expert_of_slot || !C->last_use || !C->slot_pool || !C->host_pool ||
-      !C->host_scratch)
-    return fail(FTM_ERR_INVALID_ARG, "ftm_slot_lookup_update: cache has a NULL member");
-  if (L->S > 4096) return fail(FTM_ERR_UNSUPPORTED, "LRU cache supports S <= 4096 (S=%d)", L->S);
   const int64_t P = static_cast<int64_t>(T) * L->k;
   if (P > 0 && !topk_ids) return fail(FTM_ERR_INVALID_ARG, "ftm_slot_lookup_update: NULL topk_ids");
+  if ((s = check_cache(L, C, "ftm_slot_lookup_update"))) return s;
   if ((s = check_ws(workspace, ws_bytes, lru_workspace_bytes(L->E, L->S), "ftm_slot_lookup_update"))) return s;
-  cudaPointerAttributes pa;
-  if (cudaPointerGetAttributes(&pa, C->host_pool) != cudaSuccess || pa.type != cudaMemoryTypeHost) {
-    cudaGetLastError();
-    return fail(FTM_ERR_INVALID_ARG, "host_pool is not pinned host memory");
-  }
   cudaStream_t cs = S_(compute_stream), ps = S_(copy_stream);
-  int32_t* ws = static_cast<int32_t*>(workspace);
-  prof_mark(FTM_K_LRU, cs, false);
-  cudaError_t e = launch_lru_step(topk_ids, static_cast<int>(P), L->E, L->S, C->step, C->slot_of_expert,
-                                  C->expert_of_slot, C->last_use, ws, cs);
-  prof_mark(FTM_K_LRU, cs, true);
-  if (e != cudaSuccess) return cuda_fail(e, "lru step launch");
-  const size_t hdr = sizeof(int32_t) * (4 + 2 * static_cast<size_t>(L->E));
-  if ((e = cudaMemcpyAsync(C->host_scratch, ws, hdr, cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
-    return cuda_fail(e, "miss list copy");
-  if ((e = cudaStreamSynchronize(cs)) != cudaSuccess) return cuda_fail(e, "lru step");
-  const int32_t* h = C->host_scratch;
-  C->last_distinct = h[1];
-  C->last_hits = h[2];
-  C->last_misses = h[3];
-  if (h[0] == FTM_ERR_INVALID_ARG)
-    return fail(FTM_ERR_INVALID_ARG, "step %lld: topk_ids holds an expert id outside [0, %d); state unchanged",
-                static_cast<long long>(C->step), L->E);
-  if (h[0] == FTM_ERR_CAPACITY)
-    return fail(FTM_ERR_CAPACITY, "step %lld requests %d distinct experts > %d slots", static_cast<long long>(C->step),
-                h[1], L->S);
-  ftm_bank_layout bl;
-  bank_layout(L, &bl);
-  const int misses = h[3];
-  bool copy_failed = false;
-  const char* why = nullptr;
-  int n_dirty = 0;     // miss-list slots a copy may have written
-  for (int i = 0; i < misses && !copy_failed; ++i) {
-    if (C->fail_before_copy > 0 && i + 1 == C->fail_before_copy) {
-      copy_failed = true;
-      why = "injected copy failure (fail_before_copy)";
-      break;
-    }
-    const int ex = h[4 + 2 * i], sl = h[4 + 2 * i + 1];
-    e = cudaMemcpyAsync(static_cast<uint8_t*>(C->slot_pool) + static_cast<size_t>(sl) * bl.bank_bytes,
-                        static_cast<const uint8_t*>(C->host_pool) + static_cast<size_t>(ex) * bl.bank_bytes,
-                        bl.bank_bytes, cudaMemcpyHostToDevice, ps);
-    n_dirty = i + 1;     // a copy that failed to issue may still have started
-    if (e != cudaSuccess) { copy_failed = true; why = cudaGetErrorString(e); }
-  }
-  if (copy_failed) {
-    C->fail_before_copy = 0;
-    cudaError_t e2 = launch_lru_restore(L->E, L->S, C->slot_of_expert, C->expert_of_slot, C->last_use, ws, n_dirty,
-                                        cs);
-    if (e2 == cudaSuccess) e2 = cudaStreamSynchronize(cs);
-    return fail(FTM_ERR_CUDA, "a miss copy failed (%s) with %d of %d copies issued; slot state rolled back, the "
-                "%d slot(s) a copy may have written left empty%s", why, n_dirty, misses, n_dirty,
-                e2 == cudaSuccess ? "" : " -- rollback failed too");
-  }
+  // the victims were last used by steps whose compute is ahead of the lookup
+  // kernel on the compute stream, and the host waits for that kernel before
+  // it issues any copy: no copy can overwrite a bank still being read
+  int misses = 0;
+  if ((s = cache_step(L, C, topk_ids, static_cast<int>(P), C->step, static_cast<int32_t*>(workspace), cs, ps, nullptr,
+                      &misses)))
+    return s;
   if (misses > 0) {
     cudaEvent_t ev = copy_event();
+    cudaError_t e;
     if (!ev) return fail(FTM_ERR_CUDA, "could not create the copy event");
     if ((e = cudaEventRecord(ev, ps)) != cudaSuccess) return cuda_fail(e, "copy event record");
     if ((e = cudaStreamWaitEvent(cs, ev, 0)) != cudaSuccess) return cuda_fail(e, "copy event wait");
   }
-  C->step += 1;
+  return ok();
+}
+
+ftm_status ftm_slot_stage_layer(const ftm_layer_desc* L, ftm_slot_cache* C, int32_t layer, int32_t hold_previous,
+                                void* after_event, void* workspace, size_t ws_bytes, void* copy_stream,
+                                void* ready_event) {
+  ftm_status s = check_desc(L);
+  if (s) return s;
+  if (!C) return fail(FTM_ERR_INVALID_ARG, "ftm_slot_stage_layer: cache is NULL");
+  const int n_keys = C->n_keys ? C->n_keys : L->E;
+  if (layer < 0 || static_cast<int64_t>(layer + 1) * L->E > n_keys)
+    return fail(FTM_ERR_INVALID_ARG, "ftm_slot_stage_layer: layer %d outside the cache's %d keys", layer, n_keys);
+  const int32_t base_saved = C->key_base;
+  C->key_base = layer * L->E;
+  s = check_cache(L, C, "ftm_slot_stage_layer");
+  if (!s) s = check_ws(workspace, ws_bytes, lru_workspace_bytes(L->E, L->S), "ftm_slot_stage_layer");
+  if (s) { C->key_base = base_saved; return s; }
+  cudaStream_t ps = S_(copy_stream);
+  int misses = 0;
+  const int64_t reserve = hold_previous ? C->step - 1 : C->step;
+  s = cache_step(L, C, nullptr, 0, reserve, static_cast<int32_t*>(workspace), ps, ps,
+                 static_cast<cudaEvent_t>(after_event), &misses);
+  if (s) { C->key_base = base_saved; return s; }
+  cudaError_t e;
+  if (ready_event && (e = cudaEventRecord(static_cast<cudaEvent_t>(ready_event), ps)) != cudaSuccess)
+    return cuda_fail(e, "ready event record");
   return ok();
 }
 
@@ -391,7 +496,8 @@ size_t ftm_ffn_workspace_bytes(const ftm_layer_desc* L, int32_t T) {
 
 ftm_status ftm_expert_ffn(const ftm_layer_desc* L, const void* x, int32_t T, const int32_t* offsets,
                           const int32_t* perm, const int32_t* slot_of_expert, const void* slot_pool,
-                          const void* shared_bank, void* y, void* workspace, size_t ws_bytes, void* stream) {
+                          const void* shared_bank, const float* act_scale, void* y, void* workspace, size_t ws_bytes,
+                          void* stream) {
   ftm_status s = check_desc(L);
   if (s || (s = check_T(T))) return s;
   if (T == 0) return ok();
@@ -413,6 +519,7 @@ ftm_status ftm_expert_ffn(const ftm_layer_desc* L, const void* x, int32_t T, con
   a.shared_bank = static_cast<const uint8_t*>(shared_bank);
   a.bank_bytes = bl.bank_bytes; a.w_gu_off = bl.w_gu_off; a.w_d_off = bl.w_d_off;
   a.y = y;
+  a.act_scale = act_scale;
   const size_t rows = static_cast<size_t>(ffn_rows(L, T));
   a.xp = static_cast<uint8_t*>(workspace);
   a.h = a.xp + al(rows * L->d * act_elt(L));
@@ -468,13 +575,80 @@ ftm_status ftm_moe_layer_forward(const ftm_layer_desc* L, const ftm_layer_weight
     if ((s = ftm_slot_lookup_update(L, C, w.ids, T, w.lru_ws, lru_workspace_bytes(L->E, L->S), stream, copy_stream)))
       return s;
     pool = C->slot_pool;
-    soe = C->slot_of_expert;
+    soe = C->slot_of_expert + C->key_base;
   }
   if (!pool || !soe) return fail(FTM_ERR_INVALID_ARG, "ftm_moe_layer_forward: no slot pool / slot table");
-  if ((s = ftm_expert_ffn(L, x, T, w.offsets, w.perm, soe, pool, W->shared_bank, w.y, w.ffn_ws, ffn_ws_bytes(L, T),
+  if ((s = ftm_expert_ffn(L, x, T, w.offsets, w.perm, soe, pool, W->shared_bank, W->act_scale, w.y, w.ffn_ws,
+                          ffn_ws_bytes(L, T),
                           stream)))
     return s;
   return ftm_combine(L, w.y, w.inv, w.gates, T, out, stream);
 }
+
+ftm_status ftm_moe_layers_forward(const ftm_layer_desc* L, int32_t n_layers, const ftm_layer_weights* W,
+                                  ftm_slot_cache* C, const void* const* x, int32_t T, void* const* out,
+                                  int32_t overlap, int32_t* overlapped, void* workspace, size_t ws_bytes,
+                                  void* stream, void* copy_stream) {
+  ftm_status s = check_desc(L);
+  if (s || (s = check_T(T))) return s;
+  if (n_layers < 1 || !W || !x || !out || !C) return fail(FTM_ERR_INVALID_ARG, "ftm_moe_layers_forward: NULL array");
+  const int E = L->E;
+  const int n_keys = C->n_keys ? C->n_keys : E;
+  if (static_cast<int64_t>(n_layers) * E > n_keys)
+    return fail(FTM_ERR_INVALID_ARG, "ftm_moe_layers_forward: %d layers of %d experts need %lld keys, the cache has %d",
+                n_layers, E, static_cast<long long>(n_layers) * E, n_keys);
+  for (int l = 0; l < n_layers; ++l)
+    if (!W[l].w_router || (T > 0 && (!x[l] || !out[l])))
+      return fail(FTM_ERR_INVALID_ARG, "ftm_moe_layers_forward: layer %d has a NULL router, input or output", l);
+  LayerWs w = carve(L, T, static_cast<uint8_t*>(workspace));
+  if ((s = check_ws(workspace, ws_bytes, w.total, "ftm_moe_layers_forward"))) return s;
+  const bool on = overlap != 0 && L->S >= 2 * E;
+  if (overlapped) *overlapped = on ? 1 : 0;
+  g_warn[0] = 0;
+  if (overlap && !on) {
+    snprintf(g_warn, sizeof(g_warn),
+             "WARNING Disabling MoE prefill overlap: the slot cache (%d slots) cannot hold two whole layers of "
+             "experts (2 x %d); each layer's experts are copied before its compute",
+             L->S, E);
+    static std::atomic<bool> printed{false};
+    if (!printed.exchange(true)) fprintf(stderr, "%s\n", g_warn);
+  }
+  if (T == 0) return ok();
+  cudaStream_t cs = S_(stream);
+  cudaEvent_t ev[5];
+  for (int i = 0; i < 5; ++i)
+    if (!(ev[i] = pipe_event(i))) return fail(FTM_ERR_CUDA, "could not create the pipeline events");
+  cudaError_t e;
+  if ((e = cudaEventRecord(ev[4], cs)) != cudaSuccess) return cuda_fail(e, "event record");
+  const size_t lru_bytes = lru_workspace_bytes(E, L->S);
+  // staging of layer l on the copy stream: a cache step for all its experts,
+  // after `after` (the compute that reads the slots it may take); the copies
+  // complete on ready[l % 2]
+  auto stage = [&](int l, bool hold_previous, cudaEvent_t after) {
+    return ftm_slot_stage_layer(L, C, l, hold_previous ? 1 : 0, after, w.lru_ws, lru_bytes, copy_stream, ev[l % 2]);
+  };
+  auto compute = [&](int l) -> ftm_status {
+    cudaError_t ce;
+    if ((ce = cudaStreamWaitEvent(cs, ev[l % 2], 0)) != cudaSuccess) return cuda_fail(ce, "ready event wait");
+    ftm_layer_weights wl = W[l];
+    wl.slot_pool = C->slot_pool;
+    wl.slot_of_expert = C->slot_of_expert + static_cast<size_t>(l) * E;
+    ftm_status st = ftm_moe_layer_forward(L, &wl, nullptr, x[l], T, out[l], workspace, ws_bytes, stream, nullptr);
+    if (st) return st;
+    if ((ce = cudaEventRecord(ev[2 + l % 2], cs)) != cudaSuccess) return cuda_fail(ce, "done event record");
+    return FTM_OK;
+  };
+  if ((s = stage(0, false, ev[4]))) return s;
+  for (int l = 0; l < n_layers; ++l) {
+    if (!on && l > 0 && (s = stage(l, false, ev[2 + (l - 1) % 2]))) return s;
+    if ((s = compute(l))) return s;
+    // layer l+1's copies run while layer l computes; they may take the slots
+    // of layer l-1 once its compute is over, never those of layer l
+    if (on && l + 1 < n_layers && (s = stage(l + 1, true, l >= 1 ? ev[2 + (l - 1) % 2] : ev[4]))) return s;
+  }
+  return ok();
+}
+
+const char* ftm_last_warning(void) { return g_warn; }
 
 }  // extern "C"

@@ -239,6 +239,7 @@ struct FfnArgs {
   const uint8_t* shared_bank;
   size_t bank_bytes, w_gu_off, w_d_off;
   void* y;
+  const float* act_scale;   // NVFP4: device fp32[2] activation global scales (x, h), or nullptr (1, 1)
   uint8_t* xp;   // workspace [rows][d]
   uint8_t* h;    // workspace [rows][I]
 };

@@ -1,6 +1,9 @@
 // NVFP4 grouped SwiGLU FFN: e2m1 weights with one e4m3 scale per 16 elements
 // and one fp32 scale per tensor; activations quantised to e2m1 with one e4m3
-// scale per 16 elements (per-tensor activation scale 1).
+// scale per 16 elements and a per-tensor fp32 global scale (x: gx, the SwiGLU
+// output h: gh; static values supplied with the layer, 1 when absent):
+// s16 = e4m3(amax / (6 g)), codes = e2m1(v / (s16 g)).  The accumulators are
+// scaled by (weight tensor scale) x (activation global scale).
 //
 // The contraction is tcgen05.mma kind::mxf4nvf4 with hardware block scaling:
 // each MMA (K = 64) takes the four scales of every A row and every B row from
@@ -132,10 +135,13 @@ __global__ void pad_offsets_kernel(const int32_t* __restrict__ offsets, int E, i
 // 8 packed bytes + one scale).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) quant_tokens_nvfp4_kernel(const uint16_t* __restrict__ x, int T, int d,
+                                                                 const float* __restrict__ act_scale,
                                                                  uint8_t* __restrict__ xq_tok,
                                                                  uint8_t* __restrict__ s_tok) {
   pdl_wait();
   pdl_trigger();
+  const float gx = act_scale ? act_scale[0] : 1.f;
+  const float six_gx = 6.0f * gx;
   const int ng = d / 16;
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nwarps = blockDim.x / 32;
   for (int t = blockIdx.x * nwarps + warp; t < T; t += gridDim.x * nwarps) {
@@ -152,8 +158,8 @@ __global__ void __launch_bounds__(256) quant_tokens_nvfp4_kernel(const uint16_t*
       float amax = 0.f;
 #pragma unroll
       for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-      const uint8_t sq = f32_to_e4m3_sat(amax / 6.0f);
-      const float sc = e4m3_to_f32(sq);
+      const uint8_t sq = f32_to_e4m3_sat(amax / six_gx);
+      const float sc = e4m3_to_f32(sq) * gx;
       uint32_t packed[2] = {0, 0};
       if (sc != 0.f) {
 #pragma unroll
@@ -237,7 +243,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                      int has_shared, int T, int P, int K, int Nw, int up_row0, const uint8_t* __restrict__ pool,
                      const uint8_t* __restrict__ shared_bank, size_t bank_bytes, size_t wsf_off, size_t st_off,
                      int st_idx, const uint8_t* __restrict__ act_sf, uint8_t* __restrict__ out_q,
-                     uint8_t* __restrict__ out_sf, uint16_t* __restrict__ out_bf16, int stages) {
+                     uint8_t* __restrict__ out_sf, uint16_t* __restrict__ out_bf16,
+                     const float* __restrict__ act_scale, int stages) {
   constexpr uint32_t kBBytes = ((BN * 128 + 1023) / 1024) * 1024;
   constexpr int NP = nvfp4_a_tiles(BN, GATED);     // 128-row A tiles per stage, one accumulator each
   constexpr uint32_t kStageBytes = NP * kATileBytes + kBBytes + (NP + 1) * kSfStage;
@@ -399,7 +406,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // codes of H / scale.  Padding columns are quantised too (their rows
         // are never read back).
         const bool gate_warp = q < 2;
-        const float s_row = st[st_idx + (gate_warp ? 0 : 1)];
+        const float gx = act_scale ? act_scale[0] : 1.f, gh = act_scale ? act_scale[1] : 1.f;
+        const float six_gh = 6.0f * gh;
+        const float s_row = st[st_idx + (gate_warp ? 0 : 1)] * gx;
         const int me = q * 32 + lane, partner = (q ^ 2) * 32 + lane;
         const int il = (q % 2) * 32 + lane;               // intermediate index within the tile
         const int col_off = gate_warp ? 0 : 16;           // the 16 columns of a chunk this warp evaluates
@@ -432,8 +441,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               h[i] = tbuf[tok * 68 + grp * 17 + i];
               amax = fmaxf(amax, fabsf(h[i]));
             }
-            const uint8_t sq = f32_to_e4m3_sat(amax / 6.0f);
-            const float sc = e4m3_to_f32(sq);
+            const uint8_t sq = f32_to_e4m3_sat(amax / six_gh);
+            const float sc = e4m3_to_f32(sq) * gh;
             uint32_t packed[2] = {0u, 0u};
             if (sc != 0.f) {
 #pragma unroll
@@ -447,7 +456,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       } else {
-        const float s_a = st[st_idx];
+        const float s_a = st[st_idx] * (act_scale ? act_scale[1] : 1.f);
         const int wrow = ti.m * 128 + q * 32 + lane;
         uint16_t* obase = out_bf16 + static_cast<size_t>(ti.row0 + ti.n * BN) * Nw + wrow;
         for (int c0 = 0; c0 < valid; c0 += 16) {
@@ -537,7 +546,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
                          const int32_t* __restrict__ slot_of_expert, int E, int has_shared, int T, int P, int K,
                          int Nw, int up_row0, const uint8_t* __restrict__ pool,
                          const uint8_t* __restrict__ shared_bank, size_t bank_bytes, size_t st_off, int st_idx,
-                         uint8_t* __restrict__ out_q, uint8_t* __restrict__ out_sf, uint16_t* __restrict__ out_bf16) {
+                         uint8_t* __restrict__ out_q, uint8_t* __restrict__ out_sf, uint16_t* __restrict__ out_bf16,
+                         const float* __restrict__ act_scale) {
   constexpr uint32_t kTmemCols = 512;
   constexpr int kRowsPerPair = GATED ? 128 : 256;   // output rows (intermediate / hidden) per pair tile
 
@@ -740,7 +750,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
         // this CTA's rows: 64 gate + the same 64 up rows of paired block pb
         const int pb = ti.m * 2 + static_cast<int>(rank);
         const bool gate_warp = q < 2;
-        const float s_row = st[st_idx + (gate_warp ? 0 : 1)];
+        const float gx = act_scale ? act_scale[0] : 1.f, gh = act_scale ? act_scale[1] : 1.f;
+        const float six_gh = 6.0f * gh;
+        const float s_row = st[st_idx + (gate_warp ? 0 : 1)] * gx;
         const int me = q * 32 + lane, partner = (q ^ 2) * 32 + lane;
         const int il = (q % 2) * 32 + lane;
         const int col_off = gate_warp ? 0 : 16;
@@ -771,8 +783,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
             h[i] = tbuf[tok * 68 + grp * 17 + i];
             amax = fmaxf(amax, fabsf(h[i]));
           }
-          const uint8_t sq = f32_to_e4m3_sat(amax / 6.0f);
-          const float sc = e4m3_to_f32(sq);
+          const uint8_t sq = f32_to_e4m3_sat(amax / six_gh);
+          const float sc = e4m3_to_f32(sq) * gh;
           uint32_t packed[2] = {0u, 0u};
           if (sc != 0.f) {
 #pragma unroll
@@ -785,7 +797,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
           out_sf[(static_cast<size_t>(blk * 2 + tr / 128) * (Nw / 64) + pb) * kSfChunk + sf_byte(tr % 128, grp)] = sq;
         }
       } else {
-        const float s_a = st[st_idx];
+        const float s_a = st[st_idx] * (act_scale ? act_scale[1] : 1.f);
         const int wrow = ti.m * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
         uint16_t* o = out_bf16 + static_cast<size_t>(ti.row0 + ti.n * kQN) * Nw + wrow;
         for (int c0 = 0; c0 < valid; c0 += 16) {
@@ -871,7 +883,7 @@ static cudaError_t launch_nvfp4(const CUtensorMap& mA, const CUtensorMap& mAsh, 
   const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
   return launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st, mA, mAsh, mB, a.offsets, prow0, a.slot_of_expert,
                     a.E, a.has_shared, a.T, P, K, Nw, up_row0, a.pool, a.shared_bank, a.bank_bytes, wsf_off, st_off,
-                    st_idx, act_sf, out_q, out_sf, out_bf16, stages);
+                    st_idx, act_sf, out_q, out_sf, out_bf16, a.act_scale, stages);
 }
 
 // ---- CTA-pair launch (prefill-size groups) -----------------------------------
@@ -933,7 +945,7 @@ static cudaError_t launch_nvfp4_tc2_one(const CUtensorMap* maps, const FfnArgs& 
   cfg.numAttrs = 2;
   return count_launch(cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], a.offsets, prow0,
                             a.slot_of_expert, a.E, a.has_shared, a.T, P, K, Nw, up_row0, a.pool, a.shared_bank,
-                            a.bank_bytes, st_off, st_idx, out_q, out_sf, out_bf16));
+                            a.bank_bytes, st_off, st_idx, out_q, out_sf, out_bf16, a.act_scale));
 }
 
 // Both GEMMs on CTA pairs; xq/sfx (gathered, padded to 224-row blocks) are ready.
@@ -1001,7 +1013,7 @@ const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_
   if (*cerr == cudaSuccess) {
     const int grid = a.T / 8 + 1 < 148 * 8 ? a.T / 8 + 1 : 148 * 8;
     *cerr = launch_pdl(quant_tokens_nvfp4_kernel, dim3(grid), dim3(256), 0, st,
-                       reinterpret_cast<const uint16_t*>(a.x), a.T, a.d, xq_tok, s_tok);
+                       reinterpret_cast<const uint16_t*>(a.x), a.T, a.d, a.act_scale, xq_tok, s_tok);
   }
   if (*cerr == cudaSuccess) {
     const int grid = static_cast<int>(rp / 8 + 1 < 148 * 8 ? rp / 8 + 1 : 148 * 8);

@@ -5,15 +5,21 @@
 // MoE backends"); the cache is global and evicts the expert unused for the
 // longest time (claypier.com "FreeToken MoE edge runtime", first section).
 //
-// Step s: mark the distinct requested experts; hits get last_use = s; the
-// misses, in ascending expert id, take the free-for-this-step slots in order
-// of (last_use, slot index).  Because each placement sets last_use = s, the
-// i-th miss simply takes the i-th candidate of that order, so the whole step
-// is a rank computation with no sequential dependence.
+// The cache may be shared by several layers: its entries are keys, layer l's
+// expert e being key l*E + e (key_base = l*E for the layer looked up).
+// Step s: mark the distinct requested experts of the layer (all E of them for
+// whole-layer staging, ids == nullptr); hits get last_use = s; the misses, in
+// ascending key, take the slots with last_use < reserve (reserve <= s; slots
+// used since `reserve` are held back for compute still in flight) in order of
+// (last_use, slot index).  Because each placement sets last_use = s >=
+// reserve, the i-th miss simply takes the i-th candidate of that order, so
+// the whole step is a rank computation with no sequential dependence.  When
+// the misses outnumber the candidates the step is refused before any write.
 //
 // Workspace (device int32): [0] status, [1] distinct, [2] hits, [3] misses,
-// [4 .. 4+2E) miss list (expert, slot) pairs, then a backup of the state
-// (slot_of_expert[E], expert_of_slot[S], last_use[S] as int64) for rollback.
+// [4 .. 4+2E) miss list (key, slot) pairs, then a backup for rollback: the
+// layer's slot_of_key[key_base .. key_base+E), key_of_slot[S], last_use[S]
+// (int64).
 #include "ftm_common.cuh"
 
 namespace ftm {
@@ -26,27 +32,37 @@ size_t lru_workspace_bytes(int E, int S) {
   return b + sizeof(int64_t) * S;
 }
 
+__device__ __forceinline__ int64_t* lru_backup_lu(int32_t* ws, int E, int S) {
+  size_t off = sizeof(int32_t) * (4 + 2 * static_cast<size_t>(E) + E + S);
+  off = (off + 7) & ~static_cast<size_t>(7);
+  return reinterpret_cast<int64_t*>(reinterpret_cast<uint8_t*>(ws) + off);
+}
+
 __global__ void __launch_bounds__(kLruThreads) lru_step_kernel(const int32_t* __restrict__ ids, int P, int E, int S,
-                                                               int64_t step, int32_t* __restrict__ slot_of_expert,
-                                                               int32_t* __restrict__ expert_of_slot,
+                                                               int64_t step, int64_t reserve, int key_base,
+                                                               int32_t* __restrict__ slot_of_key,
+                                                               int32_t* __restrict__ key_of_slot,
                                                                int64_t* __restrict__ last_use,
                                                                int32_t* __restrict__ ws) {
   extern __shared__ int32_t sm[];
   int32_t* want = sm;              // [E] 0/1
   int32_t* miss_rank = want + E;   // [E+1] exclusive scan of miss flags
-  int32_t* cand = miss_rank + E + 1;  // [S] candidate flag, later victim_of_rank
-  int32_t* victim = cand + S;      // [S]
-  __shared__ int32_t s_distinct, s_hits, s_bad;
+  int32_t* cand = miss_rank + E + 1;  // [S] candidate flag
+  int32_t* victim = cand + S;      // [S] candidate of each rank
+  __shared__ int32_t s_distinct, s_hits, s_misses, s_free, s_bad;
   pdl_wait();
   pdl_trigger();
+  int32_t* soe = slot_of_key + key_base;   // this layer's entries
 
-  for (int e = threadIdx.x; e < E; e += blockDim.x) want[e] = 0;
-  if (threadIdx.x == 0) { s_distinct = 0; s_hits = 0; s_bad = 0; }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) want[e] = ids ? 0 : 1;
+  if (threadIdx.x == 0) { s_distinct = 0; s_hits = 0; s_misses = 0; s_free = 0; s_bad = 0; }
   __syncthreads();
-  for (int q = threadIdx.x; q < P; q += blockDim.x) {
-    const int e = ids[q];
-    if (e >= 0 && e < E) want[e] = 1;
-    else s_bad = 1;
+  if (ids) {
+    for (int q = threadIdx.x; q < P; q += blockDim.x) {
+      const int e = ids[q];
+      if (e >= 0 && e < E) want[e] = 1;
+      else s_bad = 1;
+    }
   }
   __syncthreads();
   if (s_bad) {   // an id outside [0, E): the state is left untouched
@@ -56,27 +72,34 @@ __global__ void __launch_bounds__(kLruThreads) lru_step_kernel(const int32_t* __
     }
     return;
   }
+  // capacity: the misses must not outnumber the slots they may take
   for (int e = threadIdx.x; e < E; e += blockDim.x)
-    if (want[e]) atomicAdd(&s_distinct, 1);
+    if (want[e]) {
+      atomicAdd(&s_distinct, 1);
+      if (soe[e] < 0) atomicAdd(&s_misses, 1);
+    }
+  for (int j = threadIdx.x; j < S; j += blockDim.x) {
+    const int k = key_of_slot[j] - key_base;
+    const bool hit = k >= 0 && k < E && want[k];
+    if (last_use[j] < reserve && !hit) atomicAdd(&s_free, 1);
+  }
   __syncthreads();
   const int distinct = s_distinct;
-  if (distinct > S) {
+  if (s_misses > s_free) {
     if (threadIdx.x == 0) { ws[0] = FTM_ERR_CAPACITY; ws[1] = distinct; ws[2] = 0; ws[3] = 0; }
     return;
   }
   // backup for rollback
   int32_t* bk_soe = ws + 4 + 2 * E;
   int32_t* bk_eos = bk_soe + E;
-  size_t off = sizeof(int32_t) * (4 + 2 * static_cast<size_t>(E) + E + S);
-  off = (off + 7) & ~static_cast<size_t>(7);
-  int64_t* bk_lu = reinterpret_cast<int64_t*>(reinterpret_cast<uint8_t*>(ws) + off);
-  for (int e = threadIdx.x; e < E; e += blockDim.x) bk_soe[e] = slot_of_expert[e];
-  for (int j = threadIdx.x; j < S; j += blockDim.x) { bk_eos[j] = expert_of_slot[j]; bk_lu[j] = last_use[j]; }
+  int64_t* bk_lu = lru_backup_lu(ws, E, S);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) bk_soe[e] = soe[e];
+  for (int j = threadIdx.x; j < S; j += blockDim.x) { bk_eos[j] = key_of_slot[j]; bk_lu[j] = last_use[j]; }
   __syncthreads();
 
   // hits
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    const int sl = slot_of_expert[e];
+    const int sl = soe[e];
     const bool miss = want[e] && sl < 0;
     if (want[e] && sl >= 0) { last_use[sl] = step; atomicAdd(&s_hits, 1); }
     want[e] = miss ? 1 : 0;   // from here on: miss flag
@@ -97,7 +120,7 @@ __global__ void __launch_bounds__(kLruThreads) lru_step_kernel(const int32_t* __
     for (int e = b; e < en; ++e) { miss_rank[e] = run; run += want[e]; }
     if (lane == 31) miss_rank[E] = incl;
   }
-  for (int j = threadIdx.x; j < S; j += blockDim.x) cand[j] = last_use[j] < step ? 1 : 0;
+  for (int j = threadIdx.x; j < S; j += blockDim.x) cand[j] = last_use[j] < reserve ? 1 : 0;
   __syncthreads();
   // rank of each candidate slot in (last_use, index) order
   for (int j = threadIdx.x; j < S; j += blockDim.x) {
@@ -117,53 +140,59 @@ __global__ void __launch_bounds__(kLruThreads) lru_step_kernel(const int32_t* __
     if (!want[e]) continue;
     const int r = miss_rank[e];
     const int sl = victim[r];
-    const int old = expert_of_slot[sl];
-    if (old >= 0) slot_of_expert[old] = -1;
-    slot_of_expert[e] = sl;
-    expert_of_slot[sl] = e;
+    const int old = key_of_slot[sl];
+    if (old >= 0) slot_of_key[old] = -1;
+    soe[e] = sl;
+    key_of_slot[sl] = key_base + e;
     last_use[sl] = step;
-    ws[4 + 2 * r] = e;
+    ws[4 + 2 * r] = key_base + e;
     ws[4 + 2 * r + 1] = sl;
   }
   if (threadIdx.x == 0) { ws[0] = FTM_OK; ws[1] = distinct; ws[2] = s_hits; ws[3] = misses; }
 }
 
-// Rollback of a step whose miss copies could not all be issued: the state
-// before the step comes back from the backup, except that the first n_dirty
-// slots of the miss list (whose banks a copy may already have overwritten)
-// are left empty and their previous experts unmapped.
-__global__ void lru_restore_kernel(int E, int S, int32_t* __restrict__ slot_of_expert,
-                                   int32_t* __restrict__ expert_of_slot, int64_t* __restrict__ last_use,
-                                   const int32_t* __restrict__ ws, int n_dirty) {
-  const int32_t* bk_soe = ws + 4 + 2 * E;
-  const int32_t* bk_eos = bk_soe + E;
-  size_t off = sizeof(int32_t) * (4 + 2 * static_cast<size_t>(E) + E + S);
-  off = (off + 7) & ~static_cast<size_t>(7);
-  const int64_t* bk_lu = reinterpret_cast<const int64_t*>(reinterpret_cast<const uint8_t*>(ws) + off);
-  for (int e = threadIdx.x; e < E; e += blockDim.x) slot_of_expert[e] = bk_soe[e];
-  for (int j = threadIdx.x; j < S; j += blockDim.x) { expert_of_slot[j] = bk_eos[j]; last_use[j] = bk_lu[j]; }
-  __syncthreads();
-  for (int i = threadIdx.x; i < n_dirty; i += blockDim.x) {
-    const int sl = ws[4 + 2 * i + 1];
-    const int old = bk_eos[sl];
-    if (old >= 0) slot_of_expert[old] = -1;
-    expert_of_slot[sl] = -1;
-    last_use[sl] = -1;
-  }
-}
-
-cudaError_t launch_lru_step(const int32_t* ids, int P, int E, int S, int64_t step, int32_t* soe, int32_t* eos,
-                            int64_t* lu, int32_t* ws, cudaStream_t st) {
+cudaError_t launch_lru_step(const int32_t* ids, int P, int E, int S, int64_t step, int64_t reserve, int key_base,
+                            int32_t* soe, int32_t* eos, int64_t* lu, int32_t* ws, cudaStream_t st) {
   const size_t smem = sizeof(int32_t) * (2 * static_cast<size_t>(E) + 1 + 2 * S);
   cudaError_t err =
       cudaFuncSetAttribute(lru_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  return launch_pdl(lru_step_kernel, dim3(1), dim3(kLruThreads), smem, st, ids, P, E, S, step, soe, eos, lu, ws);
+  return launch_pdl(lru_step_kernel, dim3(1), dim3(kLruThreads), smem, st, ids, P, E, S, step, reserve, key_base,
+                    soe, eos, lu, ws);
 }
 
-cudaError_t launch_lru_restore(int E, int S, int32_t* soe, int32_t* eos, int64_t* lu, const int32_t* ws,
+// Rollback of a step whose miss copies could not all be issued: the state
+// before the step comes back from the backup (the layer's entries, every
+// slot's key and last_use, and -- through the slots' old keys -- the entries
+// of the keys the step evicted), except that the first n_dirty slots of the
+// miss list (whose banks a copy may already have overwritten) are left empty
+// and their previous keys unmapped.
+__global__ void lru_restore_kernel(int E, int S, int key_base, int32_t* __restrict__ slot_of_key,
+                                   int32_t* __restrict__ key_of_slot, int64_t* __restrict__ last_use,
+                                   int32_t* __restrict__ ws, int n_dirty) {
+  const int32_t* bk_soe = ws + 4 + 2 * E;
+  const int32_t* bk_eos = bk_soe + E;
+  const int64_t* bk_lu = lru_backup_lu(ws, E, S);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) slot_of_key[key_base + e] = bk_soe[e];
+  __syncthreads();
+  for (int j = threadIdx.x; j < S; j += blockDim.x) {
+    key_of_slot[j] = bk_eos[j];
+    last_use[j] = bk_lu[j];
+    if (bk_eos[j] >= 0) slot_of_key[bk_eos[j]] = j;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_dirty; i += blockDim.x) {
+    const int sl = ws[4 + 2 * i + 1];
+    const int old = bk_eos[sl];
+    if (old >= 0) slot_of_key[old] = -1;
+    key_of_slot[sl] = -1;
+    last_use[sl] = -1;
+  }
+}
+
+cudaError_t launch_lru_restore(int E, int S, int key_base, int32_t* soe, int32_t* eos, int64_t* lu, int32_t* ws,
                                int n_dirty, cudaStream_t st) {
-  lru_restore_kernel<<<1, kLruThreads, 0, st>>>(E, S, soe, eos, lu, ws, n_dirty);
+  lru_restore_kernel<<<1, kLruThreads, 0, st>>>(E, S, key_base, soe, eos, lu, ws, n_dirty);
   return count_launch(cudaGetLastError());
 }
 

@@ -22,9 +22,11 @@
  *    or host memory and keeps no per-call state beyond a thread-local error
  *    string and one cached CUDA event per thread for the miss-copy ordering.
  *  - `stream` arguments are cudaStream_t values passed as void* (NULL = the
- *    legacy default stream).  Work is enqueued asynchronously; the only entry
- *    point that synchronises the host is ftm_slot_lookup_update on a cache step
- *    (it must read the miss list before it can issue the copies).
+ *    legacy default stream).  Work is enqueued asynchronously; the entry
+ *    points that synchronise the host are the cache steps
+ *    (ftm_slot_lookup_update, ftm_slot_stage_layer, ftm_moe_layers_forward,
+ *    and ftm_moe_layer_forward with a cache): each must read its miss list
+ *    before it can issue the copies, and waits for that kernel alone.
  *  - Arguments are validated before anything is enqueued; on error nothing is
  *    launched, the function returns a non-zero ftm_status and ftm_last_error()
  *    describes it.  No C++ exception crosses this boundary.
@@ -139,13 +141,14 @@ ftm_status ftm_permute(const ftm_layer_desc* L, const int32_t* topk_ids, int32_t
 size_t ftm_permute_workspace_bytes(const ftm_layer_desc* L, int32_t T);
 
 /* The LRU slot cache (a4).  State lives in caller-owned device arrays:
- *   slot_of_expert [E] (-1: not resident), expert_of_slot [S] (-1: empty),
- *   last_use [S] int64 (-1: never).
+ *   slot_of_expert [n_keys] (-1: not resident), expert_of_slot [S] (the key
+ *   held, -1: empty), last_use [S] int64 (-1: never).
  * A step s requests the distinct expert ids routed in that step (the shared
- * expert is not cached).  Hits set last_use = s.  Misses, in ascending expert
- * id, each take the slot with the smallest last_use among slots not used in
- * step s (ties: lowest slot index); the slot's previous expert is unmapped and
- * the expert's bank is copied host_pool[e] -> slot_pool[slot]. */
+ * expert is not cached), as keys key_base + id.  Hits set last_use = s.
+ * Misses, in ascending key, each take the slot with the smallest last_use
+ * among slots not used in step s (ties: lowest slot index); the slot's
+ * previous key is unmapped and the bank is copied host_pool[key] ->
+ * slot_pool[slot]. */
 typedef struct ftm_slot_cache {
   int32_t* slot_of_expert;      /* device [E] */
   int32_t* expert_of_slot;      /* device [S] */
@@ -161,6 +164,12 @@ typedef struct ftm_slot_cache {
                                    misses fail as if its n-th copy could not be issued
                                    (copies 1..n-1 are issued); see the rollback rule of
                                    ftm_slot_lookup_update.  Cleared when it fires. */
+  int32_t n_keys;               /* entries of slot_of_expert and banks of host_pool; 0 means E.
+                                   A cache shared by several layers of E experts each (the
+                                   pages' global LRU expert cache) has n_layers * E keys,
+                                   layer l's expert e being key l*E + e */
+  int32_t key_base;             /* first key of the layer a lookup serves (l*E; 0 for a cache
+                                   of one layer); ftm_slot_stage_layer sets it */
 } ftm_slot_cache;
 
 size_t ftm_slot_host_scratch_ints(const ftm_layer_desc* L);
@@ -184,6 +193,29 @@ size_t ftm_slot_workspace_bytes(const ftm_layer_desc* L);
 ftm_status ftm_slot_lookup_update(const ftm_layer_desc* L, ftm_slot_cache* C, const int32_t* topk_ids,
                                   int32_t T, void* workspace, size_t ws_bytes, void* compute_stream,
                                   void* copy_stream);
+
+/* Whole-layer staging (prefill double buffering).  pomoai.com FreeToken hub,
+ * prefill-overlap paragraph: in prefill every MoE layer moves its experts from
+ * host memory to the GPU; with overlap, layer n+1's copies run while layer n
+ * computes, so a layer costs about max(copy, compute) instead of their sum,
+ * which needs a cache that holds two whole layers (refft.com FreeToken guide:
+ * full-layer double-buffered prefill over a global LRU expert cache).
+ * One cache step that makes all E experts of `layer` resident (keys
+ * layer*E .. layer*E+E-1; C->key_base is set to layer*E).  Everything runs on
+ * `copy_stream`: after `after_event` (cudaEvent_t or NULL) the lookup/update
+ * kernel, the miss-list read (the host waits for this kernel), then one copy
+ * per miss; `ready_event` (cudaEvent_t or NULL) is recorded after the copies,
+ * so compute that waits for it sees the layer in its slots.  hold_previous =
+ * 1: the slots used by the previous step are kept (their layer may still be
+ * computing): misses take only slots with last_use < step - 1, and more
+ * misses than such slots gives FTM_ERR_CAPACITY (state unchanged).  The step
+ * rewrites the entries of the keys it evicts, so `after_event` must mark the
+ * end of every compute that reads those keys' slots.  Other errors as
+ * ftm_slot_lookup_update.
+ *   workspace device, >= ftm_slot_workspace_bytes(L) bytes */
+ftm_status ftm_slot_stage_layer(const ftm_layer_desc* L, ftm_slot_cache* C, int32_t layer, int32_t hold_previous,
+                                void* after_event, void* workspace, size_t ws_bytes, void* copy_stream,
+                                void* ready_event);
 
 /* Elastic slot-pool resize: move the cache to S_new slots at run time without
  * reloading weights from the host (pomoai.com FreeToken hub, two-level expert
@@ -219,6 +251,15 @@ ftm_status ftm_slot_resize(const ftm_layer_desc* L, const ftm_slot_cache* C, int
  *   slot_of_expert device int32 [E]: bank of expert e is slot_pool[slot_of_expert[e]]
  *   slot_pool      device, S banks (layout from ftm_get_bank_layout)
  *   shared_bank    device, one bank, required iff L->has_shared
+ *   act_scale      device fp32[2] or NULL (= {1, 1}); NVFP4 layers only (ignored
+ *                  otherwise): the per-tensor global scales of the activations,
+ *                  gx for x and gh for the SwiGLU output h, static values that
+ *                  come with an NVFP4 checkpoint's calibration.  An activation
+ *                  v is quantised per 16 consecutive elements as
+ *                  s16 = e4m3(amax / (6 g)), code = e2m1(v / (s16 g)).  With
+ *                  g = 1 a group whose amax / 6 is below 2^-10 (half the smallest
+ *                  e4m3 subnormal) quantises to zero, so small activations need
+ *                  a g near amax / (6 * 448) of their tensor.
  *   y              device [P + (has_shared ? T : 0)][d]: row pos = the FFN output of
  *                  pair perm[pos] (unweighted); rows P..P+T-1 = shared expert of token t
  *                  (bf16; fp32 for FTM_F32)
@@ -226,8 +267,8 @@ ftm_status ftm_slot_resize(const ftm_layer_desc* L, const ftm_slot_cache* C, int
  * Every expert that has pairs must be resident (slot_of_expert[e] in [0,S)). */
 ftm_status ftm_expert_ffn(const ftm_layer_desc* L, const void* x, int32_t T, const int32_t* offsets,
                           const int32_t* perm, const int32_t* slot_of_expert, const void* slot_pool,
-                          const void* shared_bank, void* y, void* workspace, size_t ws_bytes,
-                          void* stream);
+                          const void* shared_bank, const float* act_scale, void* y, void* workspace,
+                          size_t ws_bytes, void* stream);
 size_t ftm_ffn_workspace_bytes(const ftm_layer_desc* L, int32_t T);
 
 /* Weighted un-permute and combine (a8).  chenxutan.com FreeToken article,
@@ -248,6 +289,8 @@ typedef struct ftm_layer_weights {
   const void* slot_pool;           /* device, S banks (resident layers; ignored with a cache) */
   const int32_t* slot_of_expert;   /* device [E] (resident layers; ignored with a cache) */
   const void* shared_bank;         /* device, one bank, or NULL */
+  const float* act_scale;          /* device fp32[2] or NULL: NVFP4 activation global scales (see
+                                      ftm_expert_ffn) */
 } ftm_layer_weights;
 
 /* The whole layer: route -> permute -> [cache step] -> expert FFN -> combine.
@@ -265,6 +308,36 @@ ftm_status ftm_moe_layer_forward(const ftm_layer_desc* L, const ftm_layer_weight
                                  const void* x, int32_t T, void* out, void* workspace, size_t ws_bytes,
                                  void* stream, void* copy_stream);
 size_t ftm_workspace_bytes(const ftm_layer_desc* L, int32_t T_max);
+
+/* Several MoE layers in sequence over one slot cache shared by all of them,
+ * with full-layer double buffering (see ftm_slot_stage_layer for the pages'
+ * passages).  Layer l's experts are staged into the cache (one cache step per
+ * layer, all E experts), then layer l runs as a resident layer on the staged
+ * slots: route, permute, expert FFN, combine.
+ *   L          one layer's shape (every layer has it); L->S = slots of C
+ *   n_layers   >= 1; C->n_keys must be >= n_layers * E, host_pool holding
+ *              layer l's expert banks at keys l*E ..
+ *   W          host array [n_layers]: w_router, router_bias, shared_bank of
+ *              each layer (slot_pool and slot_of_expert are ignored)
+ *   x, out     host arrays [n_layers] of device pointers: layer l reads x[l]
+ *              ([T][d]) and writes out[l]; x[l+1] may be out[l]
+ *   overlap    1: stage layer l+1 on copy_stream while layer l computes on
+ *              `stream` (the staging holds layer l's slots back, and may take
+ *              layer l-1's once its compute is over); needs S >= 2E, else the
+ *              overlap is switched off with a warning (ftm_last_warning, and
+ *              once per process on stderr).  0: stage each layer after the
+ *              previous layer's compute, then compute it.
+ *   overlapped host, nullable: set to 1 when the overlap ran
+ *   workspace  device, >= ftm_workspace_bytes(L, T) bytes, 256-aligned
+ * The host waits once per layer for a staging kernel (its miss list).
+ * C->step advances by n_layers. */
+ftm_status ftm_moe_layers_forward(const ftm_layer_desc* L, int32_t n_layers, const ftm_layer_weights* W,
+                                  ftm_slot_cache* C, const void* const* x, int32_t T, void* const* out,
+                                  int32_t overlap, int32_t* overlapped, void* workspace, size_t ws_bytes,
+                                  void* stream, void* copy_stream);
+
+/* Thread-local warning of the last ftm_moe_layers_forward call ("" if none). */
+const char* ftm_last_warning(void);
 
 /* The whole resident layer, for callers that cannot allocate device memory
  * (code running while a CUDA graph is being captured, allocator-free embedded

@@ -54,6 +54,8 @@ def lib():
         L.orc_dequant_nvfp4.argtypes = [p, p, ctypes.c_float, i32, i32, p]
         L.orc_qa_fp8_g128.argtypes = [p, i32, i32]
         L.orc_qa_nvfp4_g16.argtypes = [p, i32, i32]
+        L.orc_qa_nvfp4_g16_gs.argtypes = [p, i32, i32, ctypes.c_float]
+        L.orc_expert_ffn_gs.argtypes = [p, i32, i32, i32, p, p, p, i32, ctypes.c_float, ctypes.c_float, p]
         L.orc_e8m0_value.argtypes = [ctypes.c_uint8]
         L.orc_e8m0_value.restype = ctypes.c_double
         L.orc_mx_scale_code.argtypes = [p, i32]
@@ -147,10 +149,14 @@ def qa_fp8(v: np.ndarray) -> np.ndarray:
     return v
 
 
-def qa_nvfp4(v: np.ndarray) -> np.ndarray:
+def qa_nvfp4(v: np.ndarray, gs: Optional[float] = None) -> np.ndarray:
+    """gs: the per-tensor global scale (None: the scale-1 quantiser)."""
     v = _f32(v).copy()
     rows, K = v.reshape(-1, v.shape[-1]).shape
-    lib().orc_qa_nvfp4_g16(_p(v), rows, K)
+    if gs is None:
+        lib().orc_qa_nvfp4_g16(_p(v), rows, K)
+    else:
+        lib().orc_qa_nvfp4_g16_gs(_p(v), rows, K, ctypes.c_float(gs))
     return v
 
 
@@ -310,12 +316,18 @@ class LRUState:
 QA_NONE, QA_FP8, QA_NVFP4 = 0, 1, 2
 
 
-def expert_ffn(x: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndarray, qa: int = QA_NONE) -> np.ndarray:
+def expert_ffn(x: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndarray, qa: int = QA_NONE,
+               act_scale: Optional[Tuple[float, float]] = None) -> np.ndarray:
+    """act_scale: NVFP4 activation global scales (of x, of h); None: 1, 1."""
     x, Wg, Wu, Wd = _f32(x), _f32(Wg), _f32(Wu), _f32(Wd)
     n, d = x.shape
     I = Wg.shape[0]
     y = np.empty((n, d), dtype=np.float32)
-    lib().orc_expert_ffn(_p(x), n, d, I, _p(Wg), _p(Wu), _p(Wd), qa, _p(y))
+    if act_scale is None:
+        lib().orc_expert_ffn(_p(x), n, d, I, _p(Wg), _p(Wu), _p(Wd), qa, _p(y))
+    else:
+        lib().orc_expert_ffn_gs(_p(x), n, d, I, _p(Wg), _p(Wu), _p(Wd), qa, ctypes.c_float(act_scale[0]),
+                                ctypes.c_float(act_scale[1]), _p(y))
     return y
 
 
@@ -351,7 +363,8 @@ def qa_mode(wdtype: str) -> int:
 
 
 def moe_rows(layer, x: np.ndarray, rows: Sequence[int], ids: np.ndarray, gates: np.ndarray,
-             qa: Optional[int] = None, weight_cache: Optional[Dict[int, tuple]] = None) -> np.ndarray:
+             qa: Optional[int] = None, weight_cache: Optional[Dict[int, tuple]] = None,
+             act_scale: Optional[Tuple[float, float]] = None) -> np.ndarray:
     """Layer output for the selected token rows (routing given by the oracle's
     own ids/gates for all tokens).  Returns [len(rows), d] float32."""
     cfg = layer.cfg
@@ -371,7 +384,7 @@ def moe_rows(layer, x: np.ndarray, rows: Sequence[int], ids: np.ndarray, gates: 
             cache[e] = expert_weights_f32(layer, e)
         Wg, Wu, Wd = cache[e]
         xs = np.stack([x[rows[ri]] for ri, _ in lst])
-        ys = expert_ffn(xs, Wg, Wu, Wd, qa)
+        ys = expert_ffn(xs, Wg, Wu, Wd, qa, act_scale)
         for (ri, j), yv in zip(lst, ys):
             y_pairs[ri * k + j] = yv
         if not keep:
@@ -381,6 +394,6 @@ def moe_rows(layer, x: np.ndarray, rows: Sequence[int], ids: np.ndarray, gates: 
         if cfg.E not in cache:
             cache[cfg.E] = expert_weights_f32(layer, cfg.E)
         Wg, Wu, Wd = cache[cfg.E]
-        ysh = expert_ffn(np.stack([x[t] for t in rows]), Wg, Wu, Wd, qa)
+        ysh = expert_ffn(np.stack([x[t] for t in rows]), Wg, Wu, Wd, qa, act_scale)
     g = np.stack([gates[t] for t in rows])
     return combine(y_pairs, g, ysh)

@@ -197,6 +197,29 @@ void orc_qa_nvfp4_g16(float* v, int rows, int K) {
     }
 }
 
+/* NVFP4 activations with a per-tensor global scale gs (fp32), the NVFP4
+ * checkpoint convention of a static calibrated activation scale: groups of 16
+ * consecutive elements of a row; s16 = e4m3(amax / (6 gs)); with
+ * u = s16 * gs, v <- e2m1(v / u) * u.  gs = 1 is orc_qa_nvfp4_g16.  The global
+ * scale keeps small activations in the e4m3 scale range (with gs = 1 a group
+ * whose amax/6 is below half the smallest e4m3 subnormal, 2^-10, quantises to
+ * zero). */
+void orc_qa_nvfp4_g16_gs(float* v, int rows, int K, float gs) {
+  const float six_gs = 6.0f * gs;
+  for (int r = 0; r < rows; ++r)
+    for (int g = 0; g < K / 16; ++g) {
+      float* p = v + (int64_t)r * K + g * 16;
+      float amax = 0.0f;
+      for (int j = 0; j < 16; ++j) if (fabsf(p[j]) > amax) amax = fabsf(p[j]);
+      float u = (float)orc_e4m3_value(orc_e4m3_encode(amax / six_gs)) * gs;
+      for (int j = 0; j < 16; ++j) {
+        if (u == 0.0f) { p[j] = 0.0f; continue; }
+        float qv = p[j] / u;
+        p[j] = (float)(orc_e2m1_value(orc_e2m1_encode(qv)) * (double)u);
+      }
+    }
+}
+
 /* ---------------------------------------------------------------------------
  * MXFP4 (pomoai.com FreeToken hub, checkpoint list: the engine loads MXFP4,
  * NVFP4, FP8 and BF16 checkpoints).  The format is the OCP Microscaling (MX)
@@ -492,15 +515,25 @@ int orc_lru_resize(int E, int S_old, const int32_t* slot_of_expert, const int32_
  * qa = 0: no activation quantisation; 1: FP8 (128-groups) on x and h;
  * 2: NVFP4 (16-groups) on x and h.
  * ------------------------------------------------------------------------- */
+void orc_expert_ffn_gs(const float* x, int n, int d, int I, const float* Wg, const float* Wu,
+                       const float* Wd, int qa, float gx, float gh, float* y);
+
 void orc_expert_ffn(const float* x, int n, int d, int I, const float* Wg, const float* Wu,
                     const float* Wd, int qa, float* y) {
+  orc_expert_ffn_gs(x, n, d, I, Wg, Wu, Wd, qa, 1.0f, 1.0f, y);
+}
+
+/* As orc_expert_ffn; in NVFP4 mode (qa = 2) x is quantised with the global
+ * scale gx and h with gh (orc_qa_nvfp4_g16_gs); other modes ignore them. */
+void orc_expert_ffn_gs(const float* x, int n, int d, int I, const float* Wg, const float* Wu,
+                       const float* Wd, int qa, float gx, float gh, float* y) {
 #pragma omp parallel for schedule(dynamic)
   for (int r = 0; r < n; ++r) {
     float* xr = (float*)malloc(sizeof(float) * d);
     float* h = (float*)malloc(sizeof(float) * I);
     memcpy(xr, x + (int64_t)r * d, sizeof(float) * d);
     if (qa == 1) orc_qa_fp8_g128(xr, 1, d);
-    if (qa == 2) orc_qa_nvfp4_g16(xr, 1, d);
+    if (qa == 2) orc_qa_nvfp4_g16_gs(xr, 1, d, gx);
     for (int i = 0; i < I; ++i) {
       double g = 0.0, u = 0.0;
       for (int c = 0; c < d; ++c) {
@@ -510,7 +543,7 @@ void orc_expert_ffn(const float* x, int n, int d, int I, const float* Wg, const 
       h[i] = (float)(g / (1.0 + exp(-g)) * u);
     }
     if (qa == 1) orc_qa_fp8_g128(h, 1, I);
-    if (qa == 2) orc_qa_nvfp4_g16(h, 1, I);
+    if (qa == 2) orc_qa_nvfp4_g16_gs(h, 1, I, gh);
     for (int j = 0; j < d; ++j) {
       double acc = 0.0;
       for (int i = 0; i < I; ++i) acc += (double)h[i] * (double)Wd[(int64_t)j * I + i];

@@ -16,6 +16,18 @@ TOL = {"f32": 2e-2, "bf16": 2e-2, "fp8": 5e-2, "nvfp4": 5e-2}
 TOL_F32_SIMT = 1e-4
 
 
+def gate_rtol(d: int, sigma_x: float = 1.0, sigma_w: float = 0.02) -> float:
+    """Relative tolerance of the gates against the oracle, from the arithmetic.
+    A logit is d exact products accumulated in fp32 (unit roundoff u = 2^-24);
+    its partial sums random-walk with step sigma_x * sigma_w, so the rounding
+    error has standard deviation about u * sigma_x * sigma_w * d / sqrt(2).  A
+    gate is the softmax of the k picked logits: its relative error is at most
+    twice the largest logit error.  Six standard deviations, and never below
+    1e-5 (the bar for the widths where fp32 rounding is far smaller)."""
+    u = 2.0 ** -24
+    return max(1e-5, 2 * 6 * u * sigma_x * sigma_w * d / np.sqrt(2.0))
+
+
 def screened_layer(cfg: synth.LayerConfig, T: int, steps: int = 1, seed: int = 0, slot_perm=None) -> DeviceLayer:
     """A device layer whose hidden rows are screened for the top-k margin by the oracle."""
     base = synth.Layer(cfg, seed)

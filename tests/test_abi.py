@@ -128,3 +128,42 @@ def test_slot_resize_rejected_without_gpu():
     assert lib.ftm_slot_resize(ctypes.byref(d), ctypes.byref(old), 8, ctypes.byref(same), ws, nbytes, None) == 1
     assert lib.ftm_slot_resize(ctypes.byref(d), ctypes.byref(old), 8, ctypes.byref(new), ws, nbytes - 8, None) == 1
     assert lib.ftm_slot_resize(ctypes.byref(d), ctypes.byref(old), 8, ctypes.byref(new), None, nbytes, None) == 1
+
+
+def _layers_call(S, overlap, n_layers=3, n_keys=None, T=0):
+    """ftm_moe_layers_forward on fake, never dereferenced addresses: at T = 0 the
+    call validates, settles the overlap rule and returns before any launch."""
+    cfg = synth.scaled(synth.CONFIGS["35b_decode"], S=S, E=8, k=2, d=256, I=256)
+    d = ftm.desc_for(cfg)
+    lib = ftm.library()
+    cache = ftm.SlotCache(0x100000, 0x200000, 0x300000, 0, 0x10_0000_0000, 0x4000_0000, 0x5000_0000, 0, 0, 0, 0,
+                          n_layers * cfg.E if n_keys is None else n_keys, 0)
+    W = (ftm.LayerWeights * n_layers)(*[ftm.LayerWeights(0x7000_0000, None, None, None, None)
+                                        for _ in range(n_layers)])
+    X = (ctypes.c_void_p * n_layers)(*[0x8000_0000] * n_layers)
+    O = (ctypes.c_void_p * n_layers)(*[0x9000_0000] * n_layers)
+    used = ctypes.c_int32(-1)
+    ws = np.zeros(ftm.ftm_workspace_bytes(d, T) + 512, dtype=np.uint8)
+    wp = ws.ctypes.data + (-ws.ctypes.data) % 256
+    st = lib.ftm_moe_layers_forward(ctypes.byref(d), n_layers, W, ctypes.byref(cache), X, T, O, int(overlap),
+                                    ctypes.byref(used), wp, ws.nbytes - 256, None, None)
+    return st, used.value
+
+
+def test_layers_overlap_rule_without_gpu():
+    # the copy/compute overlap needs room for two whole layers of experts (S >= 2E)
+    st, used = _layers_call(S=16, overlap=True)
+    assert st == 0 and used == 1 and ftm.ftm_last_warning() == ""
+    st, used = _layers_call(S=15, overlap=True)
+    assert st == 0 and used == 0
+    w = ftm.ftm_last_warning()
+    assert w.startswith("WARNING Disabling MoE prefill overlap") and "two whole layers" in w
+    st, used = _layers_call(S=40, overlap=False)
+    assert st == 0 and used == 0 and ftm.ftm_last_warning() == ""
+
+
+def test_layers_rejected_without_gpu():
+    st, _ = _layers_call(S=16, overlap=True, n_keys=8)             # 3 layers x 8 experts need 24 keys
+    assert st == 1 and "keys" in ftm.ftm_last_error()
+    st, _ = _layers_call(S=16, overlap=True, n_layers=0)
+    assert st == 1

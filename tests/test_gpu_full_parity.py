@@ -10,6 +10,7 @@ import expert_offloaded_edge_b200 as ftm
 import oracle
 import synth
 from synth.device import Workspace, to_device_storage
+from tests.gpu_util import gate_rtol
 
 pytestmark = pytest.mark.gpu
 
@@ -38,7 +39,9 @@ def _route_permute_case(cfg, T, step=0):
     to32 = oracle.bf16_to_f32 if cfg.act_dtype == "bf16" else (lambda a: np.asarray(a, np.float32))
     rid, rg, _ = oracle.route(to32(x_st), to32(wr_st), b, cfg.k)
     assert np.array_equal(ids.cpu().numpy(), rid), f"{cfg.name} T={T} step {step}: routing ids differ"
-    assert np.allclose(gw.cpu().numpy(), rg, rtol=1e-5, atol=1e-6)
+    g = gw.cpu().numpy()
+    rel = float((np.abs(g - rg) / np.abs(rg)).max())
+    assert np.allclose(g, rg, rtol=gate_rtol(cfg.d), atol=1e-6), f"worst gate relative error {rel:.3g}"
     rc, ro, rp, ri = oracle.permute(rid, cfg.E)
     assert np.array_equal(counts.cpu().numpy(), rc)
     assert np.array_equal(offsets.cpu().numpy(), ro)

@@ -588,6 +588,67 @@ def test_ffn_gate_and_up_not_swapped():
     assert np.allclose(c[0, :5], z / (1 + np.exp(-z)) * z, rtol=1e-6)
 
 
+def test_qa_nvfp4_global_scale_one_is_the_plain_quantiser():
+    rng = np.random.default_rng(5)
+    v = rng.normal(size=(7, 64)).astype(np.float32)
+    assert np.array_equal(oracle.qa_nvfp4(v, 1.0), oracle.qa_nvfp4(v))
+
+
+def test_qa_nvfp4_global_scale_hand_worked():
+    g = np.zeros(16, np.float32)
+    g[:4] = [3.0, 1.25, 0.375, -1.1]
+    # gs = 0.5: amax / (6 gs) = 1 -> s16 = 1, u = 0.5: v/u = 6, 2.5, 0.75, -2.2 -> 6, 2, 1, -2 (ties to even)
+    assert oracle.qa_nvfp4(g[None], 0.5)[0][:4].tolist() == [3.0, 1.0, 0.5, -1.0]
+    h = np.zeros(16, np.float32)
+    h[:2] = [12.0, 3.0]
+    # gs = 3: 12 / 18 = 0.667 -> e4m3 0.6875 (step 1/16), u = 2.0625: 5.82 -> 6, 1.45 -> 1.5
+    assert oracle.qa_nvfp4(h[None], 3.0)[0][:2].tolist() == [6 * 2.0625, 1.5 * 2.0625]
+
+
+@pytest.mark.parametrize("k", [-7, -1, 3])
+def test_qa_nvfp4_global_scale_commutes_with_powers_of_two(k):
+    rng = np.random.default_rng(20 + k)
+    v = rng.normal(size=(5, 48)).astype(np.float32)
+    gs = 0.37
+    a = oracle.qa_nvfp4(v * np.float32(2.0 ** k), np.float32(gs * 2.0 ** k))
+    b = oracle.qa_nvfp4(v, gs) * np.float32(2.0 ** k)
+    assert np.array_equal(a, b)
+
+
+def test_qa_nvfp4_small_activations_need_the_global_scale():
+    # amax/6 of every group below 2^-10 (half the smallest e4m3 subnormal): with
+    # global scale 1 every group rounds to zero; a calibrated global scale
+    # (amax / (6 * 448)) keeps each value within the e2m1/e4m3 rounding bound
+    rng = np.random.default_rng(7)
+    v = (rng.normal(size=(6, 256)) * 1e-3).astype(np.float32)
+    v = np.clip(v, -5.5e-3, 5.5e-3)
+    assert (np.abs(v).reshape(6, 16, 16).max(-1) / 6 < 2.0 ** -10).all()
+    assert (oracle.qa_nvfp4(v) == 0).all()
+    gs = float(np.abs(v).max()) / (6 * 448)
+    q = oracle.qa_nvfp4(v, gs)
+    amax = np.abs(v).reshape(6, 16, 16).max(-1, keepdims=True)
+    err = np.abs(q - v).reshape(6, 16, 16)
+    assert (err <= 0.25 * amax).all() and (q != 0).any()
+
+
+def test_ffn_nvfp4_global_scales_compose_pinned_pieces():
+    rng = np.random.default_rng(8)
+    d, I, n = 64, 32, 4
+    x = (rng.normal(size=(n, d)) * 1e-2).astype(np.float32)
+    Wg, Wu = (rng.normal(0, 0.05, size=(I, d)).astype(np.float32) for _ in range(2))
+    Wd = rng.normal(0, 0.05, size=(d, I)).astype(np.float32)
+    gx, gh = 3.1e-6, 7.3e-9
+    y = oracle.expert_ffn(x, Wg, Wu, Wd, oracle.QA_NVFP4, (gx, gh)).astype(np.float64)
+    xq = oracle.qa_nvfp4(x, gx).astype(np.float64)
+    g, u = xq @ Wg.T.astype(np.float64), xq @ Wu.T.astype(np.float64)
+    h = (g / (1.0 + np.exp(-g)) * u).astype(np.float32)
+    want = oracle.qa_nvfp4(h, gh).astype(np.float64) @ Wd.T.astype(np.float64)
+    assert np.allclose(y, want, rtol=1e-5, atol=1e-12)
+    assert np.abs(want).max() > 0
+    assert np.array_equal(oracle.expert_ffn(x, Wg, Wu, Wd, oracle.QA_NVFP4, (1.0, 1.0)),
+                          oracle.expert_ffn(x, Wg, Wu, Wd, oracle.QA_NVFP4))
+
+
 def _silu(z):
     return z / (1.0 + math.exp(-z))
 
