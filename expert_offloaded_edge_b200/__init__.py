@@ -10,6 +10,7 @@ from .binding import (  # noqa: F401
     FTM_BF16,
     FTM_F32,
     FTM_FP8_E4M3_B128,
+    FTM_MXFP4,
     FTM_NVFP4,
     BankLayout,
     FtmError,

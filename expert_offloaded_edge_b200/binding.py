@@ -9,10 +9,10 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 SO = os.path.join(PKG, "libftm.so")
 
 FTM_OK, FTM_ERR_INVALID_ARG, FTM_ERR_UNSUPPORTED, FTM_ERR_CAPACITY, FTM_ERR_CUDA = range(5)
-FTM_F32, FTM_BF16, FTM_FP8_E4M3_B128, FTM_NVFP4 = range(4)
+FTM_F32, FTM_BF16, FTM_FP8_E4M3_B128, FTM_NVFP4, FTM_MXFP4 = range(5)
 (FTM_K_ROUTE, FTM_K_PERMUTE, FTM_K_LRU, FTM_K_GATHER, FTM_K_GEMM1, FTM_K_GEMM2, FTM_K_COMBINE) = range(7)
 KERNEL_NAMES = ("route", "permute", "lru", "gather", "gemm1", "gemm2", "combine")
-_WDTYPE = {"f32": FTM_F32, "bf16": FTM_BF16, "fp8": FTM_FP8_E4M3_B128, "nvfp4": FTM_NVFP4}
+_WDTYPE = {"f32": FTM_F32, "bf16": FTM_BF16, "fp8": FTM_FP8_E4M3_B128, "nvfp4": FTM_NVFP4, "mxfp4": FTM_MXFP4}
 
 c_i32, c_i64, c_u64, c_p, c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_size_t
 

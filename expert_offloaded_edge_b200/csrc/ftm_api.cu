@@ -66,8 +66,8 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 ftm_status check_desc(const ftm_layer_desc* L) {
   if (!L) return fail(FTM_ERR_INVALID_ARG, "layer descriptor is NULL");
   if (L->reserved != 0) return fail(FTM_ERR_INVALID_ARG, "reserved field must be 0");
-  if (L->wdtype < FTM_F32 || L->wdtype > FTM_NVFP4) return fail(FTM_ERR_INVALID_ARG, "unknown wdtype %d", L->wdtype);
-  const int q = L->wdtype == FTM_NVFP4 ? 256 : 128;
+  if (L->wdtype < FTM_F32 || L->wdtype > FTM_MXFP4) return fail(FTM_ERR_INVALID_ARG, "unknown wdtype %d", L->wdtype);
+  const int q = (L->wdtype == FTM_NVFP4 || L->wdtype == FTM_MXFP4) ? 256 : 128;
   if (L->d <= 0 || L->d % q) return fail(FTM_ERR_INVALID_ARG, "d=%d must be a positive multiple of %d", L->d, q);
   if (L->I <= 0 || L->I % q) return fail(FTM_ERR_INVALID_ARG, "I=%d must be a positive multiple of %d", L->I, q);
   if (L->E < 1 || L->E > 512) return fail(FTM_ERR_INVALID_ARG, "E=%d out of [1, 512]", L->E);
@@ -97,6 +97,10 @@ void bank_layout(const ftm_layer_desc* L, ftm_bank_layout* b) {
     case FTM_NVFP4:
       wgu = 2 * I * d / 2; wd = d * I / 2;
       sgu = 2 * I * (d / 16); sd = d * (I / 16); st = 16;
+      break;
+    case FTM_MXFP4:
+      wgu = 2 * I * d / 2; wd = d * I / 2;
+      sgu = 2 * I * (d / 32); sd = d * (I / 32);
       break;
   }
   uint64_t off = 0;

@@ -8,13 +8,14 @@ from __future__ import annotations
 
 import numpy as np
 
-from .binding import FTM_BF16, FTM_F32, FTM_FP8_E4M3_B128, FTM_NVFP4, BankLayout, LayerDesc, ftm_get_bank_layout
+from .binding import FTM_BF16, FTM_F32, FTM_FP8_E4M3_B128, FTM_MXFP4, FTM_NVFP4, BankLayout, LayerDesc, ftm_get_bank_layout
 
 
 def nvfp4_scale_chunks(s16: np.ndarray) -> np.ndarray:
-    """e4m3 scales [R][C/16] -> the MMA chunk layout: one 512-byte chunk per
-    (128-row block rb, 64-column block kb), chunks ordered [rb][kb]; inside a
-    chunk the scale of local row r and 16-group j is byte (r%32)*16 + (r//32)*4 + j."""
+    """Block scales [R][G] (G groups per row: C/16 for NVFP4, C/32 for MXFP4)
+    -> the MMA chunk layout: one 512-byte chunk per (128-row block rb, block
+    kb of four groups), chunks ordered [rb][kb]; inside a chunk the scale of
+    local row r and group j of the block is byte (r%32)*16 + (r//32)*4 + j."""
     R, G16 = s16.shape
     assert R % 128 == 0 and G16 % 4 == 0
     a = np.ascontiguousarray(s16, dtype=np.uint8).reshape(R // 128, 4, 32, G16 // 4, 4)
@@ -41,7 +42,8 @@ def pack_bank(desc: LayerDesc, ew, bl: BankLayout = None, out: np.ndarray = None
     """ew: an expert in storage form with .gate/.up/.down
     f32/bf16: arrays [I][d], [I][d], [d][I] (float32 or bf16 bits as uint16);
     fp8: (q uint8, s float32 [R/128][C/128]) per matrix;
-    nvfp4: (q packed uint8 [R][C/2], s16 uint8 [R][C/16], s_t float) per matrix."""
+    nvfp4: (q packed uint8 [R][C/2], s16 uint8 [R][C/16], s_t float) per matrix;
+    mxfp4: (q packed uint8 [R][C/2], s32 E8M0 codes uint8 [R][C/32]) per matrix."""
     bl = bl or ftm_get_bank_layout(desc)
     bank = out if out is not None else np.zeros(bl.bank_bytes, dtype=np.uint8)
     w = desc.wdtype
@@ -59,6 +61,11 @@ def pack_bank(desc: LayerDesc, ew, bl: BankLayout = None, out: np.ndarray = None
         _put(bank, bl.s_gu_off, nvfp4_scale_chunks(gate_up_paired_rows(ew.gate[1], ew.up[1])), bl.s_gu_bytes)
         _put(bank, bl.s_d_off, nvfp4_scale_chunks(ew.down[1]), bl.s_d_bytes)
         _put(bank, bl.s_t_off, np.array([ew.gate[2], ew.up[2], ew.down[2], 0.0], dtype=np.float32), bl.s_t_bytes)
+    elif w == FTM_MXFP4:
+        _put(bank, bl.w_gu_off, np.concatenate([ew.gate[0], ew.up[0]], axis=0), bl.w_gu_bytes)
+        _put(bank, bl.w_d_off, ew.down[0], bl.w_d_bytes)
+        _put(bank, bl.s_gu_off, nvfp4_scale_chunks(gate_up_paired_rows(ew.gate[1], ew.up[1])), bl.s_gu_bytes)
+        _put(bank, bl.s_d_off, nvfp4_scale_chunks(ew.down[1]), bl.s_d_bytes)
     else:
         raise ValueError(w)
     return bank

@@ -59,10 +59,11 @@ typedef enum ftm_wdtype {
   FTM_F32 = 0,               /* fp32 expert weights */
   FTM_BF16 = 1,              /* bf16 expert weights */
   FTM_FP8_E4M3_B128 = 2,     /* e4m3 weights, one fp32 scale per 128x128 block */
-  FTM_NVFP4 = 3              /* e2m1 weights, one e4m3 scale per 16 elements + fp32 per-tensor scale */
+  FTM_NVFP4 = 3,             /* e2m1 weights, one e4m3 scale per 16 elements + fp32 per-tensor scale */
+  FTM_MXFP4 = 4              /* e2m1 weights, one E8M0 scale (power of two) per 32 elements (OCP MX) */
 } ftm_wdtype;
 
-/* One layer's shape.  Limits: d, I multiples of 128 (of 256 for NVFP4);
+/* One layer's shape.  Limits: d, I multiples of 128 (of 256 for NVFP4 and MXFP4);
  * 1 <= k <= min(E, 16); 1 <= E <= 512; 1 <= S. */
 typedef struct ftm_layer_desc {
   int32_t d;            /* hidden size */
@@ -87,10 +88,14 @@ typedef struct ftm_layer_desc {
  *         64b..64b+63 for b = 0..I/64-1 (chunk row block rb = b)
  *   s_d : FP8: fp32 [d/128][I/128];  NVFP4: the d x I/16 e4m3 scales in chunks
  *   s_t : NVFP4: fp32[4] = {gate, up, down, 0} per-tensor scales; else empty
- * NVFP4 scale chunks (the layout the block-scaled MMA reads): one 512-byte
- * chunk per (128-row block rb, 64-column block kb), ordered [rb][kb]; in a
- * chunk the scale of local row r (0..127) for its j-th 16-column group of the
- * block (0..3) is byte (r % 32) * 16 + (r / 32) * 4 + j. */
+ *   MXFP4: w_gu, w_d packed as NVFP4; s_gu: the 2I x d/32 E8M0 codes in chunks
+ *          (rows in the paired order above), s_d: the d x I/32 codes in chunks;
+ *          no s_t.
+ * Scale chunks (the layout the block-scaled MMA reads): one 512-byte chunk per
+ * (128-row block rb, column block kb of four scale groups: 64 columns for
+ * NVFP4's 16-groups, 128 for MXFP4's 32-groups), ordered [rb][kb]; in a chunk
+ * the scale of local row r (0..127) for its j-th group of the block (0..3) is
+ * byte (r % 32) * 16 + (r / 32) * 4 + j. */
 typedef struct ftm_bank_layout {
   uint64_t bank_bytes;
   uint64_t w_gu_off, w_gu_bytes;

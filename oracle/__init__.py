@@ -313,7 +313,7 @@ class LRUState:
 
 # ---- expert FFN / combine -----------------------------------------------------------
 
-QA_NONE, QA_FP8, QA_NVFP4 = 0, 1, 2
+QA_NONE, QA_FP8, QA_NVFP4, QA_MXFP4 = 0, 1, 2, 3
 
 
 def expert_ffn(x: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndarray, qa: int = QA_NONE,
@@ -355,11 +355,13 @@ def expert_weights_f32(layer, e: int) -> Tuple[np.ndarray, np.ndarray, np.ndarra
         return tuple(dequant_fp8_b128(q, s) for (q, s) in (ew.gate, ew.up, ew.down))
     if w == "nvfp4":
         return tuple(dequant_nvfp4(q, s16, st) for (q, s16, st) in (ew.gate, ew.up, ew.down))
+    if w == "mxfp4":
+        return tuple(dequant_mxfp4(q, s) for (q, s) in (ew.gate, ew.up, ew.down))
     raise ValueError(w)
 
 
 def qa_mode(wdtype: str) -> int:
-    return {"f32": QA_NONE, "bf16": QA_NONE, "fp8": QA_FP8, "nvfp4": QA_NVFP4}[wdtype]
+    return {"f32": QA_NONE, "bf16": QA_NONE, "fp8": QA_FP8, "nvfp4": QA_NVFP4, "mxfp4": QA_MXFP4}[wdtype]
 
 
 def moe_rows(layer, x: np.ndarray, rows: Sequence[int], ids: np.ndarray, gates: np.ndarray,

@@ -513,7 +513,8 @@ int orc_lru_resize(int E, int S_old, const int32_t* slot_of_expert, const int32_
  * h[i] = silu(x . Wg[i]) * (x . Wu[i]),  silu(z) = z / (1 + exp(-z));
  * y[j] = h . Wd[j].
  * qa = 0: no activation quantisation; 1: FP8 (128-groups) on x and h;
- * 2: NVFP4 (16-groups) on x and h.
+ * 2: NVFP4 (16-groups) on x and h; 3: MXFP4 (32-groups, E8M0 scales) on x
+ * and h -- the same activation reading as NVFP4, with MX's own block format.
  * ------------------------------------------------------------------------- */
 void orc_expert_ffn_gs(const float* x, int n, int d, int I, const float* Wg, const float* Wu,
                        const float* Wd, int qa, float gx, float gh, float* y);
@@ -534,6 +535,7 @@ void orc_expert_ffn_gs(const float* x, int n, int d, int I, const float* Wg, con
     memcpy(xr, x + (int64_t)r * d, sizeof(float) * d);
     if (qa == 1) orc_qa_fp8_g128(xr, 1, d);
     if (qa == 2) orc_qa_nvfp4_g16_gs(xr, 1, d, gx);
+    if (qa == 3) orc_qa_mxfp4_g32(xr, 1, d);
     for (int i = 0; i < I; ++i) {
       double g = 0.0, u = 0.0;
       for (int c = 0; c < d; ++c) {
@@ -544,6 +546,7 @@ void orc_expert_ffn_gs(const float* x, int n, int d, int I, const float* Wg, con
     }
     if (qa == 1) orc_qa_fp8_g128(h, 1, I);
     if (qa == 2) orc_qa_nvfp4_g16_gs(h, 1, I, gh);
+    if (qa == 3) orc_qa_mxfp4_g32(h, 1, I);
     for (int j = 0; j < d; ++j) {
       double acc = 0.0;
       for (int i = 0; i < I; ++i) acc += (double)h[i] * (double)Wd[(int64_t)j * I + i];

@@ -59,6 +59,7 @@ def lib():
         _lib.synth_bf16_from_f32.argtypes = [p, i64, p]
         _lib.synth_quant_fp8_b128.argtypes = [p, i32, i32, p, p]
         _lib.synth_quant_nvfp4.argtypes = [p, i32, i32, p, p, p]
+        _lib.synth_quant_mxfp4.argtypes = [p, i32, i32, p, p]
     return _lib
 
 
@@ -125,6 +126,17 @@ def quant_nvfp4(W: np.ndarray) -> Tuple[np.ndarray, np.ndarray, float]:
     return q, s16, float(st[0])
 
 
+def quant_mxfp4(W: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """W [R][C] -> (packed e2m1 [R][C/2], E8M0 scale codes [R][C/32])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    R, C = W.shape
+    assert C % 32 == 0
+    q = np.empty((R, C // 2), dtype=np.uint8)
+    s = np.empty((R, C // 32), dtype=np.uint8)
+    lib().synth_quant_mxfp4(_ptr(W), R, C, _ptr(q), _ptr(s))
+    return q, s
+
+
 # --------------------------------------------------------------------------
 # Layer configurations (the five synthetic workloads).
 # --------------------------------------------------------------------------
@@ -137,7 +149,7 @@ class LayerConfig:
     E: int
     k: int
     I: int
-    wdtype: str           # "f32" | "bf16" | "fp8" | "nvfp4"
+    wdtype: str           # "f32" | "bf16" | "fp8" | "nvfp4" | "mxfp4"
     has_shared: int
     S: int                # slots in the HBM pool
     bias: str             # "none" | "uniform" | "zero" | "zipf"
@@ -161,7 +173,15 @@ CONFIGS: Dict[str, LayerConfig] = {
                               S=64, bias="zipf", T=(32,), trace_steps=256, lru=True),
     "753b_nvfp4": LayerConfig("753b_nvfp4", d=6144, E=160, k=8, I=2048, wdtype="nvfp4", has_shared=1,
                               S=160, bias="zero", T=(16, 16384)),
+    # the same layer with MXFP4 weights (pomoai.com FreeToken hub, checkpoint
+    # list: MXFP4 next to NVFP4, FP8 and BF16); router, bias and hidden states
+    # are those of the NVFP4 layer
+    "753b_mxfp4": LayerConfig("753b_mxfp4", d=6144, E=160, k=8, I=2048, wdtype="mxfp4", has_shared=1,
+                              S=160, bias="zero", T=(16, 16384)),
 }
+
+# configurations whose router and hidden states (hence redraw tables) are another's
+REDRAWS_OF = {"753b_mxfp4": "753b_nvfp4"}
 
 
 def scaled(cfg: LayerConfig, **kw) -> LayerConfig:
@@ -174,7 +194,8 @@ def scaled(cfg: LayerConfig, **kw) -> LayerConfig:
 @dataclass
 class ExpertWeights:
     """One expert in storage form.  For f32/bf16: gate/up [I][d], down [d][I]
-    (float32 or bf16 bits).  fp8: (q, s) per matrix.  nvfp4: (q_packed, s16, s_t)."""
+    (float32 or bf16 bits).  fp8: (q, s) per matrix.  nvfp4: (q_packed, s16, s_t).
+    mxfp4: (q_packed, s32) per matrix (E8M0 codes, one per 32 elements)."""
     gate: object
     up: object
     down: object
@@ -244,6 +265,8 @@ class Layer:
             ew = ExpertWeights(quant_fp8_b128(g), quant_fp8_b128(u), quant_fp8_b128(dn))
         elif w == "nvfp4":
             ew = ExpertWeights(quant_nvfp4(g), quant_nvfp4(u), quant_nvfp4(dn))
+        elif w == "mxfp4":
+            ew = ExpertWeights(quant_mxfp4(g), quant_mxfp4(u), quant_mxfp4(dn))
         else:
             raise ValueError(w)
         if cache:
@@ -285,7 +308,7 @@ def redraw_path(name: str, T: int) -> str:
 
 
 def load_redraws(name: str, T: int) -> Optional[Dict[Tuple[int, int], int]]:
-    p = redraw_path(name, T)
+    p = redraw_path(REDRAWS_OF.get(name, name), T)
     if not os.path.exists(p):
         return None
     with open(p) as f:

@@ -199,3 +199,35 @@ void synth_quant_nvfp4(const float* W, int32_t R, int32_t C, uint8_t* qp, uint8_
     }
   }
 }
+
+/* W [R][C] fp32 -> MXFP4 (OCP Microscaling v1.0): per 32 consecutive elements
+ * of a row one E8M0 scale code e (value 2^(e-127)) with e - 127 =
+ * floor(log2(block amax)) - 2 clamped to [-127, 127] (an all-zero block gets
+ * e = 127), and E2M1 codes of w / 2^(e-127), nearest with ties to even,
+ * saturating at 6.  q packed two per byte along C, element 2j in the low
+ * nibble; s [R][C/32]. */
+void synth_quant_mxfp4(const float* W, int32_t R, int32_t C, uint8_t* qp, uint8_t* s32) {
+  int32_t CB = C / 32;
+#pragma omp parallel for schedule(static)
+  for (int32_t r = 0; r < R; ++r) {
+    for (int32_t cb = 0; cb < CB; ++cb) {
+      const float* w = W + (int64_t)r * C + cb * 32;
+      float ab = 0.0f;
+      for (int j = 0; j < 32; ++j) { float a = fabsf(w[j]); if (a > ab) ab = a; }
+      int e = 0;
+      if (ab > 0.0f) {
+        int ex;
+        frexp((double)ab, &ex);             /* ab = m * 2^ex, m in [0.5, 1): floor(log2 ab) = ex - 1 */
+        e = ex - 1 - 2;
+        if (e < -127) e = -127;
+        if (e > 127) e = 127;
+      }
+      s32[(int64_t)r * CB + cb] = (uint8_t)(e + 127);
+      double X = ldexp(1.0, e);
+      for (int j = 0; j < 32; j += 2) {
+        uint8_t lo = gen_e2m1((float)(w[j] / X)), hi = gen_e2m1((float)(w[j + 1] / X));
+        qp[(int64_t)r * (C / 2) + cb * 16 + j / 2] = (uint8_t)(lo | (hi << 4));
+      }
+    }
+  }
+}

@@ -718,7 +718,45 @@ def test_ffn_nvfp4_activation_quantisation_hand_worked():
     assert abs(y[2] - 1.75) > 0.1
 
 
-@pytest.mark.parametrize("qa,d,I", [(1, 256, 128), (2, 64, 48)])
+def test_ffn_mxfp4_activation_quantisation_hand_worked():
+    # MXFP4 mode (qa = 3): 32-groups with an E8M0 scale 2^(floor(log2 amax) - 2)
+    # and e2m1 elements, on x and on h; exact dyadic results.
+    d, I = 64, 32
+    x = np.zeros((1, d), np.float32)
+    x[0, :3] = [6.0, 2.5, 0.75]        # amax 6 -> X = 1: 2.5 -> 2, 0.75 -> 1 (ties to even codes)
+    x[0, 32:35] = [3.0, 1.2, -0.4]     # amax 3 -> X = 0.5: 1.2 -> 1.0, -0.4 -> -0.5
+    Wg = np.zeros((I, d), np.float32)
+    Wu = np.zeros((I, d), np.float32)
+    Wg[0, 1], Wu[0, 33] = 1.0, 1.0     # g0 = 2, u0 = 1
+    Wg[1, 2], Wu[1, 34] = 1.0, 1.0     # g1 = 1, u1 = -0.5
+    Wd = np.zeros((d, I), np.float32)
+    Wd[0, 0] = 1.0
+    Wd[1, 1] = 1.0
+    Wd[2, 0], Wd[2, 1] = 1.0, 1.0
+    y = oracle.expert_ffn(x, Wg, Wu, Wd, oracle.QA_MXFP4)[0]
+    # h = (silu(2), -silu(1)/2) = (1.7616, -0.3655): amax in [1, 2) -> X = 2^-2;
+    # 7.05 -> 6 (saturation), -1.46 -> -1.5
+    want = np.zeros(d, np.float32)
+    want[:3] = [1.5, -0.375, 1.125]
+    assert np.array_equal(y, want)
+    assert abs(y[0] - 3.0) > 0.1                 # x not quantised: h0 = 2.77 -> X = 0.5 -> 3.0
+    assert abs(y[0] - _silu(2.0)) > 0.1          # h not quantised
+    assert abs(y[2] - 1.0) > 0.1                 # down output quantised too: 4.5 -> 4 (tie to even) -> 1.0
+
+
+def test_generator_mxfp4_quantiser_agrees_with_the_oracle():
+    # two independent implementations of the OCP MX conversion (the input
+    # generator's and the oracle's) give the same codes
+    w = synth.normal(0, 97, 0, 0, 0, 256 * 256, 0.02).reshape(256, 256)
+    w[3, 64:96] = 0.0                            # an all-zero block
+    w[5, :32] *= 1e-30                           # a block at the bottom of the E8M0 range
+    qg, sg = synth.quant_mxfp4(w)
+    qo, so = oracle.quant_mxfp4(w)
+    assert np.array_equal(sg, so) and np.array_equal(qg, qo)
+    assert sg[3, 2] == 127                       # zero block: scale 1
+
+
+@pytest.mark.parametrize("qa,d,I", [(1, 256, 128), (2, 64, 48), (3, 128, 64)])
 def test_ffn_activation_quantised_composes_pinned_pieces(qa, d, I):
     # The quantised FFN equals the composition of the separately pinned
     # quantisers with an fp64 library matmul: qa(x) -> gate/up -> silu(g)*u ->
@@ -728,7 +766,7 @@ def test_ffn_activation_quantised_composes_pinned_pieces(qa, d, I):
     x = rng.normal(size=(n, d)).astype(np.float32)
     Wg, Wu = (rng.normal(0, 0.05, size=(I, d)).astype(np.float32) for _ in range(2))
     Wd = rng.normal(0, 0.05, size=(d, I)).astype(np.float32)
-    q = oracle.qa_fp8 if qa == 1 else oracle.qa_nvfp4
+    q = {1: oracle.qa_fp8, 2: oracle.qa_nvfp4, 3: oracle.qa_mxfp4}[qa]
     y = oracle.expert_ffn(x, Wg, Wu, Wd, qa).astype(np.float64)
     xq = q(x).astype(np.float64)
     g = xq @ Wg.T.astype(np.float64)
