@@ -47,7 +47,8 @@ METRIC = "MoE-layer tokens/s; decode HBM GB/s & prefill TFLOP/s as % of B200 pea
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
 HEADLINE = ("753b_nvfp4", 16384)
-SUITE = (("35b_decode", (1, 8, 32, 64)), ("35b_prefill", (8192,)), ("284b_trace", (32,)), ("753b_nvfp4", (16,)))
+SUITE = (("35b_decode", (1, 8, 32, 64)), ("35b_prefill", (8192,)), ("284b_trace", (32,)), ("753b_mxfp4", (16, 16384)),
+         ("753b_nvfp4", (16,)))
 K_BREAKDOWN = 40
 
 
@@ -183,23 +184,27 @@ def packed_banks(cfg, cache_dir: str, local_rank: int, dist, seed: int = 0):
     runs (and the other ranks of this one) read them instead of drawing again."""
     from synth.device import pack_banks
     if not cache_dir:
-        return None if seed == 0 else pack_banks(cfg, seed)
+        return pack_banks(cfg, seed)
     tag = hashlib.sha1(repr(cfg).encode()).hexdigest()[:8]
     path = os.path.join(cache_dir, f"{cfg.name}_{source_hash()}_{tag}_s{seed}.npy")
+    banks = None
     if local_rank == 0 and not os.path.exists(path):
+        banks = pack_banks(cfg, seed)
         try:
             os.makedirs(cache_dir, exist_ok=True)
-            banks = pack_banks(cfg, seed)
             tmp = path + f".tmp{os.getpid()}"
-            np.save(tmp, banks)
+            with open(tmp, "wb") as f:
+                np.save(f, banks)
             os.replace(tmp, path)
         except OSError:
             pass
     if dist is not None:
         dist.barrier()
+    if banks is not None:
+        return banks
     if os.path.exists(path):
         return np.load(path, mmap_mode="r")
-    return None if seed == 0 else pack_banks(cfg, seed)
+    return pack_banks(cfg, seed)
 
 
 def device_layer(cfg, args, local, dist):
@@ -832,7 +837,12 @@ def main():
             continue
         dl = device_layer(cfg, args, local, dist)
         for T in Ts:
-            records.append(run_resident(dl, T, args, dist, local))
+            try:
+                records.append(run_resident(dl, T, args, dist, local))
+            except ftm.FtmError as e:     # a workload this build has no kernel for
+                if e.status != ftm.binding.FTM_ERR_UNSUPPORTED:
+                    raise
+                records.append({"workload": workload_name(cfg, T), "unsupported": str(e)})
         if name == head[0]:
             head_rec = run_resident(dl, head[1], args, dist, local)
         del dl

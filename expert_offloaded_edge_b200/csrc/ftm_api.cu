@@ -529,6 +529,7 @@ ftm_status ftm_expert_ffn(const ftm_layer_desc* L, const void* x, int32_t T, con
   a.h = a.xp + al(rows * L->d * act_elt(L));
   cudaError_t ce;
   const char* msg;
+  if (L->wdtype == FTM_MXFP4) return fail(FTM_ERR_UNSUPPORTED, "ftm_expert_ffn: no MXFP4 kernel in this build");
   if (L->wdtype == FTM_FP8_E4M3_B128)
     msg = launch_expert_ffn_fp8(a, bl.s_gu_off, bl.s_d_off, static_cast<uint8_t*>(workspace), S_(stream), &ce);
   else if (L->wdtype == FTM_NVFP4)
