@@ -31,6 +31,8 @@ const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_
                                     cudaStream_t st, cudaError_t* cerr);
 const char* launch_expert_ffn_fp8(const FfnArgs& a, size_t s_gu_off, size_t s_d_off, uint8_t* ws, cudaStream_t st,
                                   cudaError_t* cerr);
+const char* launch_expert_ffn_mxfp4(const FfnArgs& a, size_t s_gu_off, size_t s_d_off, uint8_t* ws, cudaStream_t st,
+                                    cudaError_t* cerr);
 }  // namespace ftm
 
 using namespace ftm;
@@ -121,7 +123,7 @@ size_t act_elt(const ftm_layer_desc* L) { return L->wdtype == FTM_F32 ? 4 : 2; }
 size_t ffn_ws_bytes(const ftm_layer_desc* L, int32_t T) {
   const size_t rows = static_cast<size_t>(ffn_rows(L, T));
   if (L->wdtype == FTM_FP8_E4M3_B128) return fp8_ffn_workspace_bytes(static_cast<int64_t>(rows), L->d, L->I);
-  if (L->wdtype == FTM_NVFP4)
+  if (L->wdtype == FTM_NVFP4 || L->wdtype == FTM_MXFP4)   // MXFP4 needs at most NVFP4's scratch
     return nvfp4_ffn_workspace_bytes(static_cast<int64_t>(T) * L->k, T, L->E, L->has_shared, L->d, L->I);
   return al(rows * L->d * act_elt(L)) + al(rows * L->I * act_elt(L));
 }
@@ -529,8 +531,9 @@ ftm_status ftm_expert_ffn(const ftm_layer_desc* L, const void* x, int32_t T, con
   a.h = a.xp + al(rows * L->d * act_elt(L));
   cudaError_t ce;
   const char* msg;
-  if (L->wdtype == FTM_MXFP4) return fail(FTM_ERR_UNSUPPORTED, "ftm_expert_ffn: no MXFP4 kernel in this build");
-  if (L->wdtype == FTM_FP8_E4M3_B128)
+  if (L->wdtype == FTM_MXFP4)
+    msg = launch_expert_ffn_mxfp4(a, bl.s_gu_off, bl.s_d_off, static_cast<uint8_t*>(workspace), S_(stream), &ce);
+  else if (L->wdtype == FTM_FP8_E4M3_B128)
     msg = launch_expert_ffn_fp8(a, bl.s_gu_off, bl.s_d_off, static_cast<uint8_t*>(workspace), S_(stream), &ce);
   else if (L->wdtype == FTM_NVFP4)
     msg = launch_expert_ffn_nvfp4(a, bl.s_gu_off, bl.s_d_off, bl.s_t_off, static_cast<uint8_t*>(workspace),

@@ -23,8 +23,20 @@
 namespace ftm {
 
 constexpr int kF4StageK = 256;         // K per stage: 128 bytes of packed e2m1 = one swizzle row
-constexpr uint32_t kSfChunk = 512;     // bytes of one scale chunk (64 K x 128 rows)
-constexpr uint32_t kSfStage = 4 * kSfChunk;
+constexpr uint32_t kSfChunk = 512;     // bytes of one scale chunk (128 rows x four scale groups)
+
+// The two block-scale formats of the e2m1 kernels.  NVFP4 (MX = false): one
+// e4m3 scale per 16 elements, a chunk covers K = 64, one MMA (K = 64) reads
+// all four bytes of a row's 32-bit scale column.  MXFP4 (MX = true, OCP MX):
+// one E8M0 scale per 32 elements, a chunk covers K = 128, and the two MMAs of
+// a chunk read bytes 0-1 and 2-3 of the column (scale-factor ids 0 and 2).
+template <bool MX>
+struct F4Fmt {
+  static constexpr int kGroup = MX ? 32 : 16;             // elements per scale
+  static constexpr int kChunkK = 4 * kGroup;              // K covered by one chunk
+  static constexpr int kChunks = kF4StageK / kChunkK;     // chunks per stage (per 128-row operand tile)
+  static constexpr uint32_t kSfStage = kChunks * kSfChunk;
+};
 
 // ---- conversions ---------------------------------------------------------------
 __device__ __forceinline__ uint8_t f32_to_e4m3_sat(float v) {
@@ -54,6 +66,16 @@ __host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
   return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// MXFP4: scale format UE8M0 (bit 23); sf_id (0 or 2) = the byte of the 32-bit
+// scale column this MMA starts at, for A (bits 29-30) and B (bits 4-5).
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N, uint32_t sf_id) {
+  return idesc_nvf4(M, N) | (1u << 23) | (sf_id << 29) | (sf_id << 4);
+}
+
+// The block scale of a tile's TMEM scale address for sf_id (its top two bits
+// carry the byte offset, as the instruction descriptor does).
+__device__ __forceinline__ uint32_t sf_addr(uint32_t taddr, uint32_t sf_id) { return taddr | (sf_id << 30); }
+
 __device__ __forceinline__ void umma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                           uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
   asm volatile(
@@ -64,6 +86,32 @@ __device__ __forceinline__ void umma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
       : "memory");
 }
+
+__device__ __forceinline__ void umma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// E8M0 code of a 32-group (OCP MX): 2^(code - 127) with code - 127 =
+// floor(log2 amax) - 2, clamped to [-127, 127]; an all-zero group gets 127.
+// Exponent read from the bits: a subnormal amax (< 2^-126) clamps to -127.
+__device__ __forceinline__ int mx_scale_code(float amax) {
+  if (amax == 0.f) return 127;
+  const int be = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF);
+  int e = be - 127 - 2;
+  if (be == 0) e = -127;
+  return e < -127 ? 0 : e + 127;
+}
+
+// 2^(127 - code): the exact power of two that divides a group by its scale
+// (always a normal float for the codes mx_scale_code returns from finite input).
+__device__ __forceinline__ float mx_inv_scale(int code) { return __uint_as_float(static_cast<uint32_t>(254 - code) << 23); }
 
 // shared -> TMEM copy of one 512-byte scale chunk: 32 rows x 16 bytes,
 // replicated into the four 32-lane quadrants (4 columns each).
@@ -128,46 +176,65 @@ __global__ void pad_offsets_kernel(const int32_t* __restrict__ offsets, int E, i
 }
 
 // ---------------------------------------------------------------------------
-// NVFP4 quantisation of x, once per token: xq_tok [T][d/2] packed e2m1 and
-// sw_tok [T][d/64] words holding the four e4m3 scales of each 64-element
-// block (the 4 bytes a scale chunk keeps together for one row).  One warp per
-// token; each lane quantises whole 16-element groups (two 16-byte loads ->
-// 8 packed bytes + one scale).
+// Quantisation of x, once per token: xq_tok [T][d/2] packed e2m1 and s_tok
+// [T][d/G] scale bytes (G = 16 e4m3 scales for NVFP4, 32 E8M0 codes for
+// MXFP4); every four consecutive scale bytes of a token are the 32-bit word a
+// scale chunk keeps together for one row.  One warp per token; each lane
+// quantises whole groups (NVFP4: two 16-byte loads -> 8 packed bytes + one
+// scale; MXFP4: four loads -> 16 packed bytes + one code).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) quant_tokens_nvfp4_kernel(const uint16_t* __restrict__ x, int T, int d,
-                                                                 const float* __restrict__ act_scale,
-                                                                 uint8_t* __restrict__ xq_tok,
-                                                                 uint8_t* __restrict__ s_tok) {
+template <bool MX>
+__global__ void __launch_bounds__(256) quant_tokens_f4_kernel(const uint16_t* __restrict__ x, int T, int d,
+                                                              const float* __restrict__ act_scale,
+                                                              uint8_t* __restrict__ xq_tok,
+                                                              uint8_t* __restrict__ s_tok) {
+  constexpr int G = F4Fmt<MX>::kGroup;
   pdl_wait();
   pdl_trigger();
-  const float gx = act_scale ? act_scale[0] : 1.f;
+  const float gx = (!MX && act_scale) ? act_scale[0] : 1.f;
   const float six_gx = 6.0f * gx;
-  const int ng = d / 16;
+  const int ng = d / G;
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nwarps = blockDim.x / 32;
   for (int t = blockIdx.x * nwarps + warp; t < T; t += gridDim.x * nwarps) {
-    for (int g16 = lane; g16 < ng; g16 += 32) {
-      float v[16];
-      const uint4* p = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d + g16 * 16);
-      const uint4 u0 = p[0], u1 = p[1];
-      const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    for (int g = lane; g < ng; g += 32) {
+      float v[G];
+      const uint4* p = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d + g * G);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        v[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFF);
-        v[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
+      for (int u = 0; u < G / 8; ++u) {
+        const uint4 w4 = p[u];
+        const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v[8 * u + 2 * i] = bf16_bits_to_f32(w[i] & 0xFFFF);
+          v[8 * u + 2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
+        }
       }
       float amax = 0.f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-      const uint8_t sq = f32_to_e4m3_sat(amax / six_gx);
-      const float sc = e4m3_to_f32(sq) * gx;
-      uint32_t packed[2] = {0, 0};
-      if (sc != 0.f) {
+      for (int i = 0; i < G; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      uint8_t sq;
+      if constexpr (MX) {
+        const int code = mx_scale_code(amax);
+        const float mul = mx_inv_scale(code);      // exact: v * 2^-e == v / 2^e
+        sq = static_cast<uint8_t>(code);
+        uint32_t packed[4] = {0, 0, 0, 0};
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          packed[i / 4] |= static_cast<uint32_t>(f32x2_to_e2m1x2(v[2 * i + 1] / sc, v[2 * i] / sc)) << (8 * (i % 4));
+        for (int i = 0; i < 16; ++i)
+          packed[i / 4] |= static_cast<uint32_t>(f32x2_to_e2m1x2(v[2 * i + 1] * mul, v[2 * i] * mul)) << (8 * (i % 4));
+        *reinterpret_cast<uint4*>(xq_tok + static_cast<size_t>(t) * (d / 2) + g * 16) =
+            make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      } else {
+        sq = f32_to_e4m3_sat(amax / six_gx);
+        const float sc = e4m3_to_f32(sq) * gx;
+        uint32_t packed[2] = {0, 0};
+        if (sc != 0.f) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            packed[i / 4] |= static_cast<uint32_t>(f32x2_to_e2m1x2(v[2 * i + 1] / sc, v[2 * i] / sc)) << (8 * (i % 4));
+        }
+        *reinterpret_cast<uint2*>(xq_tok + static_cast<size_t>(t) * (d / 2) + g * 8) = make_uint2(packed[0], packed[1]);
       }
-      *reinterpret_cast<uint2*>(xq_tok + static_cast<size_t>(t) * (d / 2) + g16 * 8) = make_uint2(packed[0], packed[1]);
-      s_tok[static_cast<size_t>(t) * (d / 16) + g16] = sq;
+      s_tok[static_cast<size_t>(t) * ng + g] = sq;
     }
   }
 }
@@ -175,11 +242,13 @@ __global__ void __launch_bounds__(256) quant_tokens_nvfp4_kernel(const uint16_t*
 // ---------------------------------------------------------------------------
 // Gather of the quantised tokens into the padded activation rows: one warp
 // per padded row copies its token's d/2 packed bytes (16-byte vectors) and
-// scatters its d/64 scale words into the row's place in the scale chunks
-// (rows past a group's end are zeros).  The padded group offsets sit in
+// scatters its scale words (one per chunk of four groups: d/64 for NVFP4,
+// d/128 for MXFP4) into the row's place in the scale chunks (rows past a
+// group's end are zeros).  The padded group offsets sit in
 // shared memory; lane 0 finds the row's source token.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) gather_nvfp4_kernel(const uint8_t* __restrict__ xq_tok,
+template <bool MX>
+__global__ void __launch_bounds__(256) gather_f4_kernel(const uint8_t* __restrict__ xq_tok,
                                                           const uint8_t* __restrict__ s_tok,
                                                           const int32_t* __restrict__ perm,
                                                           const int32_t* __restrict__ offsets,
@@ -193,7 +262,7 @@ __global__ void __launch_bounds__(256) gather_nvfp4_kernel(const uint8_t* __rest
   for (int i = threadIdx.x; i <= G; i += blockDim.x) s_prow0[i] = prow0[i];
   __syncthreads();
   const int rows_pad = s_prow0[G];
-  const int kb64 = d / 64, nvec = d / 32;          // 16-byte vectors per packed row
+  const int nkc = d / F4Fmt<MX>::kChunkK, nvec = d / 32;    // scale words, 16-byte vectors per packed row
   const int nsub = (BN + 127) / 128;               // 128-row scale chunks per BN-row block
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nwarps = blockDim.x / 32;
   for (int pr = blockIdx.x * nwarps + warp; pr < rows_pad; pr += gridDim.x * nwarps) {
@@ -213,10 +282,49 @@ __global__ void __launch_bounds__(256) gather_nvfp4_kernel(const uint8_t* __rest
     uint4* dst = reinterpret_cast<uint4*>(xq + static_cast<size_t>(pr) * (d / 2));
     for (int c = lane; c < nvec; c += 32) dst[c] = src >= 0 ? s[c] : make_uint4(0, 0, 0, 0);
     const int blk = pr / BN, r = pr % BN;
-    const uint32_t* sw = reinterpret_cast<const uint32_t*>(s_tok + static_cast<size_t>(src < 0 ? 0 : src) * (d / 16));
-    uint8_t* chunk0 = sfx + (static_cast<size_t>(blk) * nsub + r / 128) * kb64 * kSfChunk + sf_byte(r % 128, 0);
-    for (int kb = lane; kb < kb64; kb += 32)
+    const uint32_t* sw = reinterpret_cast<const uint32_t*>(s_tok + static_cast<size_t>(src < 0 ? 0 : src) * (4 * nkc));
+    uint8_t* chunk0 = sfx + (static_cast<size_t>(blk) * nsub + r / 128) * nkc * kSfChunk + sf_byte(r % 128, 0);
+    for (int kb = lane; kb < nkc; kb += 32)
       *reinterpret_cast<uint32_t*>(chunk0 + static_cast<size_t>(kb) * kSfChunk) = src >= 0 ? sw[kb] : 0u;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// GEMM1 epilogue: quantise one thread's 16 consecutive intermediate values
+// (16-group `grp` of the 64-wide paired block mb, for one token row) and store
+// the packed codes (q_dst, 8 bytes) and the scale into out_sf: chunk row
+// block rb, row rr of the chunk, Nw intermediate columns.  NVFP4: e4m3 scale
+// of amax / (6 gh) times gh.  MXFP4: the 32-group is this thread's 16 values
+// and those of lane ^ 1 (all 32 lanes must call); the even lane stores the
+// code.  Padding rows are quantised too (never read back).
+// ---------------------------------------------------------------------------
+template <bool MX>
+__device__ __forceinline__ void quant_store_h(const float (&h)[16], float gh, float six_gh, uint8_t* q_dst,
+                                              uint8_t* out_sf, size_t rb, int rr, int mb, int grp, int Nw) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(h[i]));
+  uint32_t packed[2] = {0u, 0u};
+  if constexpr (MX) {
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    const int code = mx_scale_code(amax);
+    const float mul = mx_inv_scale(code);
+#pragma unroll
+    for (int i = 0; i < 16; i += 2)
+      packed[i / 8] |= static_cast<uint32_t>(f32x2_to_e2m1x2(h[i + 1] * mul, h[i] * mul)) << (4 * (i % 8));
+    *reinterpret_cast<uint2*>(q_dst) = make_uint2(packed[0], packed[1]);
+    if ((grp & 1) == 0)
+      out_sf[(rb * (Nw / 128) + mb / 2) * kSfChunk + sf_byte(rr, (mb & 1) * 2 + grp / 2)] = static_cast<uint8_t>(code);
+  } else {
+    const uint8_t sq = f32_to_e4m3_sat(amax / six_gh);
+    const float sc = e4m3_to_f32(sq) * gh;
+    if (sc != 0.f) {
+#pragma unroll
+      for (int i = 0; i < 16; i += 2)
+        packed[i / 8] |= static_cast<uint32_t>(f32x2_to_e2m1x2(h[i + 1] / sc, h[i] / sc)) << (4 * (i % 8));
+    }
+    *reinterpret_cast<uint2*>(q_dst) = make_uint2(packed[0], packed[1]);
+    out_sf[(rb * (Nw / 64) + mb) * kSfChunk + sf_byte(rr, grp)] = sq;
   }
 }
 
@@ -235,7 +343,7 @@ __global__ void __launch_bounds__(256) gather_nvfp4_kernel(const uint8_t* __rest
 // memory, applies the per-tensor scales and SwiGLU, then transposes H so each
 // thread quantises one token's 16 consecutive intermediate values.
 // ---------------------------------------------------------------------------
-template <int BN, bool GATED>
+template <int BN, bool GATED, bool MX>
 __global__ void __launch_bounds__(kTcThreads, 1)
     ffn_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAsh,
                      const __grid_constant__ CUtensorMap tmB, const int32_t* __restrict__ offsets,
@@ -245,12 +353,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                      int st_idx, const uint8_t* __restrict__ act_sf, uint8_t* __restrict__ out_q,
                      uint8_t* __restrict__ out_sf, uint16_t* __restrict__ out_bf16,
                      const float* __restrict__ act_scale, int stages) {
+  using Fmt = F4Fmt<MX>;
+  constexpr uint32_t kSfStage = Fmt::kSfStage;
+  constexpr int kCh = Fmt::kChunks;                 // scale chunks per stage and operand tile
   constexpr uint32_t kBBytes = ((BN * 128 + 1023) / 1024) * 1024;
   constexpr int NP = nvfp4_a_tiles(BN, GATED);     // 128-row A tiles per stage, one accumulator each
   constexpr uint32_t kStageBytes = NP * kATileBytes + kBBytes + (NP + 1) * kSfStage;
   constexpr uint32_t kTx = NP * kATileBytes + BN * 128 + (NP + 1) * kSfStage;
   constexpr uint32_t kAccCols = NP * BN;
-  constexpr uint32_t kSfCols = 16 * (NP + 1);      // SFA per A tile | SFB: 4 chunks x 4 columns each
+  constexpr uint32_t kSfCols = 4 * kCh * (NP + 1); // SFA per A tile | SFB: kCh chunks x 4 columns each
   // Ring of scale-factor column sets, one per stage in flight: the copies for
   // stage s + 1 never overwrite columns the MMAs of stage s still read.
   constexpr uint32_t kSfSets = 4;
@@ -275,7 +386,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int G = E + (has_shared ? 1 : 0);
   const int MT = Nw / kRowsPerTile;
   const int KB = K / kF4StageK;
-  const int K64 = K / 64;
+  const int Kc = K / Fmt::kChunkK;                  // scale chunks along K of one 128-row block
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
@@ -318,9 +429,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, BN);
         const int slot = ti.g < E ? slot_of_expert[ti.g] : 0;
         const uint8_t* bank = ti.g < E ? pool + static_cast<size_t>(slot) * bank_bytes : shared_bank;
-        const uint8_t* wsf = bank + wsf_off + static_cast<size_t>(ti.m) * NP * K64 * kSfChunk;
+        const uint8_t* wsf = bank + wsf_off + static_cast<size_t>(ti.m) * NP * Kc * kSfChunk;
         const int prow = prow0[ti.g] + ti.n * BN;
-        const uint8_t* asf = act_sf + static_cast<size_t>(prow / BN) * K64 * kSfChunk;
+        const uint8_t* asf = act_sf + static_cast<size_t>(prow / BN) * Kc * kSfChunk;
         const int r0 = ti.m * kRowsPerTile;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) { ok = false; break; }
@@ -338,11 +449,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               tma_load_2d(a_tile(stage, p), &tmAsh, &full_bar[stage], kc, rp);
               if (GATED) tma_load_2d(a_tile(stage, p) + kATileBytes / 2, &tmAsh, &full_bar[stage], kc, up_row0 + rp);
             }
-            bulk_load(sf_tile(stage, p), wsf + (static_cast<size_t>(p) * K64 + 4 * kb) * kSfChunk, kSfStage,
+            bulk_load(sf_tile(stage, p), wsf + (static_cast<size_t>(p) * Kc + kCh * kb) * kSfChunk, kSfStage,
                       &full_bar[stage]);
           }
           tma_load_2d(b_tile(stage), &tmB, &full_bar[stage], kc, prow);
-          bulk_load(sf_tile(stage, NP), asf + static_cast<size_t>(4 * kb) * kSfChunk, kSfStage, &full_bar[stage]);
+          bulk_load(sf_tile(stage, NP), asf + static_cast<size_t>(kCh * kb) * kSfChunk, kSfStage, &full_bar[stage]);
           if (++stage == stages) { stage = 0; phase ^= 1u; }
         }
       }
@@ -368,17 +479,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (++sf_set == kSfSets) sf_set = 0;
           const uint32_t sb = smem_u32(b_tile(stage));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
+          for (int c = 0; c < kCh; ++c) {
 #pragma unroll
             for (int p = 0; p <= NP; ++p)
-              tmem_cp_sf(tmem_sf + 16 * p + 4 * kk, smem_desc_sf(smem_u32(sf_tile(stage, p)) + kk * kSfChunk));
+              tmem_cp_sf(tmem_sf + 4 * kCh * p + 4 * c, smem_desc_sf(smem_u32(sf_tile(stage, p)) + c * kSfChunk));
           }
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
+            const int c = kk * kCh / 4;                    // the chunk of this K step
 #pragma unroll
-            for (int p = 0; p < NP; ++p)
-              umma_nvf4(d + p * BN, smem_desc_sw128(smem_u32(a_tile(stage, p)) + kk * 32), smem_desc_sw128(sb + kk * 32),
-                        kIdesc, tmem_sf + 16 * p + 4 * kk, tmem_sf + 16 * NP + 4 * kk, (kb | kk) != 0 ? 1u : 0u);
+            for (int p = 0; p < NP; ++p) {
+              const uint32_t sfa = tmem_sf + 4 * kCh * p + 4 * c, sfb = tmem_sf + 4 * kCh * NP + 4 * c;
+              const uint64_t ad = smem_desc_sw128(smem_u32(a_tile(stage, p)) + kk * 32);
+              const uint64_t bd = smem_desc_sw128(sb + kk * 32);
+              const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+              if constexpr (MX) {
+                const uint32_t sf_id = 2u * (kk & 1);      // bytes 0-1 or 2-3 of the chunk's columns
+                umma_mxf4(d + p * BN, ad, bd, idesc_mxf4(128, BN, sf_id), sf_addr(sfa, sf_id), sf_addr(sfb, sf_id),
+                          acc);
+              } else {
+                umma_nvf4(d + p * BN, ad, bd, kIdesc, sfa, sfb, acc);
+              }
+            }
           }
           umma_commit(&empty_bar[stage]);
           if (++stage == stages) { stage = 0; phase ^= 1u; }
@@ -398,17 +520,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_after();
       const int valid = min(BN, ti.rows - ti.n * BN);
       const uint8_t* bank = ti.g < E ? pool + static_cast<size_t>(slot_of_expert[ti.g]) * bank_bytes : shared_bank;
-      const float* st = reinterpret_cast<const float*>(bank + st_off);
+      const float* st = reinterpret_cast<const float*>(bank + st_off);   // NVFP4 only
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * kAccCols;
       if (GATED) {
-        // H = silu(s_gate * gate) * (s_up * up) in fp32, then per token one e4m3
-        // scale per 16 consecutive intermediate values (amax / 6) and e2m1
-        // codes of H / scale.  Padding columns are quantised too (their rows
-        // are never read back).
+        // H = silu(s_gate * gate) * (s_up * up) in fp32 (NVFP4: weight tensor
+        // scale x activation global scale; MXFP4: no tensor scale), then the
+        // e2m1 codes and block scales of H (quant_store_h).
         const bool gate_warp = q < 2;
-        const float gx = act_scale ? act_scale[0] : 1.f, gh = act_scale ? act_scale[1] : 1.f;
+        const float gx = (!MX && act_scale) ? act_scale[0] : 1.f, gh = (!MX && act_scale) ? act_scale[1] : 1.f;
         const float six_gh = 6.0f * gh;
-        const float s_row = st[st_idx + (gate_warp ? 0 : 1)] * gx;
+        const float s_row = MX ? 1.f : st[st_idx + (gate_warp ? 0 : 1)] * gx;
         const int me = q * 32 + lane, partner = (q ^ 2) * 32 + lane;
         const int il = (q % 2) * 32 + lane;               // intermediate index within the tile
         const int col_off = gate_warp ? 0 : 16;           // the 16 columns of a chunk this warp evaluates
@@ -435,28 +556,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             epilogue_bar();
             float h[16];
-            float amax = 0.f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              h[i] = tbuf[tok * 68 + grp * 17 + i];
-              amax = fmaxf(amax, fabsf(h[i]));
-            }
-            const uint8_t sq = f32_to_e4m3_sat(amax / six_gh);
-            const float sc = e4m3_to_f32(sq) * gh;
-            uint32_t packed[2] = {0u, 0u};
-            if (sc != 0.f) {
-#pragma unroll
-              for (int i = 0; i < 16; i += 2)
-                packed[i / 8] |= static_cast<uint32_t>(f32x2_to_e2m1x2(h[i + 1] / sc, h[i] / sc)) << (4 * (i % 8));
-            }
+            for (int i = 0; i < 16; ++i) h[i] = tbuf[tok * 68 + grp * 17 + i];
             const int i0 = mb * 64 + grp * 16;
-            *reinterpret_cast<uint2*>(out_q + static_cast<size_t>(prow + c0 + tok) * (Nw / 2) + i0 / 2) =
-                make_uint2(packed[0], packed[1]);
-            out_sf[(static_cast<size_t>(blk) * (Nw / 64) + mb) * kSfChunk + sf_byte(c0 + tok, grp)] = sq;
+            quant_store_h<MX>(h, gh, six_gh, out_q + static_cast<size_t>(prow + c0 + tok) * (Nw / 2) + i0 / 2, out_sf,
+                              static_cast<size_t>(blk), c0 + tok, mb, grp, Nw);
           }
         }
       } else {
-        const float s_a = st[st_idx] * (act_scale ? act_scale[1] : 1.f);
+        const float s_a = MX ? 1.f : st[st_idx] * (act_scale ? act_scale[1] : 1.f);
         const int wrow = ti.m * 128 + q * 32 + lane;
         uint16_t* obase = out_bf16 + static_cast<size_t>(ti.row0 + ti.n * BN) * Nw + wrow;
         for (int c0 = 0; c0 < valid; c0 += 16) {
@@ -504,13 +612,24 @@ constexpr int kQN = 224;                        // tokens per pair tile (padded 
 constexpr int kQH = kQN / 2;                    // token rows staged per CTA
 constexpr uint32_t kQABytes = 128 * 128;        // 128 weight rows x 256 e2m1
 constexpr uint32_t kQBBytes = kQH * 128;        // 112 token rows x 256 e2m1
-constexpr uint32_t kQSfaBytes = 4 * kSfChunk;   // 4 K64 chunks of this CTA's 128 weight rows
-constexpr uint32_t kQSfbBytes = 8 * kSfChunk;   // 4 K64 chunks x 2 halves of the token block
-constexpr uint32_t kQStage = kQABytes + kQBBytes + kQSfaBytes + kQSfbBytes;
 constexpr int kQStages = 5;
-constexpr uint32_t kQSfCol = 2 * kQN;           // TMEM: accumulators [0, 448), two half-stage scale slots [448, 496)
-constexpr uint32_t kQSfHalfCols = 24;           // one half stage (2 K steps): SFA 2 x 4 columns + SFB 2 x 8 columns
+constexpr uint32_t kQSfCol = 2 * kQN;           // TMEM: accumulators [0, 448), then two half-stage scale slots
 constexpr int kQThreads = 224;                  // warps 0 TMA, 1 MMA, 2-5 epilogue, 6 scale copies
+
+// Stage layout of the pair kernel per scale format: A tile | B tile | the
+// stage's scale chunks of this CTA's 128 weight rows | of the token block's
+// two 128-row halves.  A half stage (2 K steps) of scales in TMEM: NVFP4 2 x 4
+// columns SFA + 2 x 8 SFB (one chunk per K step); MXFP4 4 SFA + 8 SFB (both K
+// steps share one chunk).
+template <bool MX>
+struct Q2Fmt {
+  static constexpr uint32_t kSfa = F4Fmt<MX>::kSfStage;
+  static constexpr uint32_t kSfb = 2 * F4Fmt<MX>::kSfStage;
+  static constexpr uint32_t kStage = kQABytes + kQBBytes + kSfa + kSfb;
+  static constexpr uint32_t kHalfCols = MX ? 12 : 24;
+  static_assert(kStage % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled tiles");
+  static_assert(kQSfCol + 2 * kHalfCols <= 512, "TMEM budget");
+};
 
 __device__ __forceinline__ int quad_tile_n(int valid) { return min(kQN, (valid + 31) & ~31); }
 
@@ -520,6 +639,17 @@ __device__ __forceinline__ void umma2_nvf4(uint32_t d_tmem, uint64_t a_desc, uin
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma2_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
           d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
       : "memory");
@@ -537,7 +667,7 @@ __device__ __forceinline__ void umma2_commit_local(uint64_t* bar) {
                : "memory");
 }
 
-template <bool GATED>
+template <bool GATED, bool MX>
 __global__ void __launch_bounds__(kQThreads, 1)
     ffn_nvfp4_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAsh,
                          const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmSfa,
@@ -550,6 +680,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
                          const float* __restrict__ act_scale) {
   constexpr uint32_t kTmemCols = 512;
   constexpr int kRowsPerPair = GATED ? 128 : 256;   // output rows (intermediate / hidden) per pair tile
+  using Q = Q2Fmt<MX>;
+  constexpr int kCh = F4Fmt<MX>::kChunks;
+  constexpr uint32_t kQStage = Q::kStage;
+  constexpr uint32_t kQSfHalfCols = Q::kHalfCols;
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kQStages], empty_bar[kQStages], tfull_bar[2], tempty_bar[2];
@@ -572,7 +706,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   const int G = E + (has_shared ? 1 : 0);
   const int MT = Nw / kRowsPerPair;
   const int KB = K / kF4StageK;
-  const int K64 = K / 64;
+  const int Kc = K / F4Fmt<MX>::kChunkK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kQStages; ++s) {
@@ -614,7 +748,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   auto a_tile = [&](int s) -> uint8_t* { return smem + static_cast<size_t>(s) * kQStage; };
   auto b_tile = [&](int s) -> uint8_t* { return a_tile(s) + kQABytes; };
   auto sfa_tile = [&](int s) -> uint8_t* { return a_tile(s) + kQABytes + kQBBytes; };
-  auto sfb_tile = [&](int s) -> uint8_t* { return a_tile(s) + kQABytes + kQBBytes + kQSfaBytes; };
+  auto sfb_tile = [&](int s) -> uint8_t* { return a_tile(s) + kQABytes + kQBBytes + Q::kSfa; };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -635,7 +769,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * kQStage);
           const uint32_t lbar = mapa_rank(smem_u32(&full_bar[stage]), 0);   // the even CTA's barrier
           const int kc = kb * (kF4StageK / 2);                              // byte coordinate along K
-          const int sfa_row = (wb * K64 + 4 * kb) * 2;                       // 256-byte rows of the chunks
+          const int sfa_row = (wb * Kc + kCh * kb) * 2;                      // 256-byte rows of the chunks
           if (GATED) {
             if (routed) {
               tma2_load_3d(a_tile(stage), &tmA, lbar, kc, wb * 64, slot);
@@ -653,7 +787,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
           tma2_load_2d(b_tile(stage), &tmB, lbar, kc, brow);
 #pragma unroll
           for (int h = 0; h < 2; ++h)
-            tma2_load_2d(sfb_tile(stage) + h * (4 * kSfChunk), &tmSfb, lbar, 0, ((blk * 2 + h) * K64 + 4 * kb) * 2);
+            tma2_load_2d(sfb_tile(stage) + h * Q::kSfa, &tmSfb, lbar, 0, ((blk * 2 + h) * Kc + kCh * kb) * 2);
           if (++stage == kQStages) { stage = 0; phase ^= 1u; }
         }
       }
@@ -668,7 +802,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
       int g = 0;   // stages consumed so far (the scale set of stage g is g % 2)
       for (int t = pair; t < total && ok; t += npairs, ++it) {
         const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, kQN);
-        const uint32_t idesc = idesc_nvf4(256, quad_tile_n(min(kQN, ti.rows - ti.n * kQN)));
+        const int ntile = quad_tile_n(min(kQN, ti.rows - ti.n * kQN));
+        const uint32_t idesc = MX ? idesc_mxf4(256, ntile, 0) : idesc_nvf4(256, ntile);
         const int ab = it & 1;
         const uint32_t aphase = (it >> 1) & 1;
         if (!mbar_wait_cl(&tempty_bar[ab], aphase ^ 1u)) break;
@@ -685,8 +820,15 @@ __global__ void __launch_bounds__(kQThreads, 1)
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
               const int kk = 2 * h + j;
-              umma2_nvf4(d, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32), idesc, sf + 4 * j,
-                         sf + 8 + 8 * j, (kb | kk) != 0 ? 1u : 0u);
+              const uint64_t ad = smem_desc_sw128(sa + kk * 32), bd = smem_desc_sw128(sb + kk * 32);
+              const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+              if constexpr (MX) {
+                const uint32_t sf_id = 2u * j;             // both K steps of a half share one chunk
+                umma2_mxf4(d, ad, bd, idesc | (sf_id << 29) | (sf_id << 4), sf_addr(sf, sf_id),
+                           sf_addr(sf + 4, sf_id), acc);
+              } else {
+                umma2_nvf4(d, ad, bd, idesc, sf + 4 * j, sf + 8 + 8 * j, acc);
+              }
             }
             umma2_commit_local(&sf_free[h]);
           }
@@ -715,12 +857,18 @@ __global__ void __launch_bounds__(kQThreads, 1)
             if (g >= 1 && !mbar_wait_cl(&sf_free[h], static_cast<uint32_t>(g - 1) & 1u)) { ok = false; break; }
             tc_fence_after();
             const uint32_t sf = tmem_base + kQSfCol + h * kQSfHalfCols;
+            if constexpr (MX) {       // one chunk holds both K steps of the half
+              tmem_cp_sf2(sf, smem_desc_sf(ssa + h * kSfChunk));
+              tmem_cp_sf2(sf + 4, smem_desc_sf(ssb + h * kSfChunk));
+              tmem_cp_sf2(sf + 8, smem_desc_sf(ssb + Q::kSfa + h * kSfChunk));
+            } else {
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const int kk = 2 * h + j;
-              tmem_cp_sf2(sf + 4 * j, smem_desc_sf(ssa + kk * kSfChunk));
-              tmem_cp_sf2(sf + 8 + 8 * j, smem_desc_sf(ssb + kk * kSfChunk));
-              tmem_cp_sf2(sf + 8 + 8 * j + 4, smem_desc_sf(ssb + 4 * kSfChunk + kk * kSfChunk));
+              for (int j = 0; j < 2; ++j) {
+                const int kk = 2 * h + j;
+                tmem_cp_sf2(sf + 4 * j, smem_desc_sf(ssa + kk * kSfChunk));
+                tmem_cp_sf2(sf + 8 + 8 * j, smem_desc_sf(ssb + kk * kSfChunk));
+                tmem_cp_sf2(sf + 8 + 8 * j + 4, smem_desc_sf(ssb + Q::kSfa + kk * kSfChunk));
+              }
             }
             umma2_commit_local(&sf_ready[h * kQStages + stage]);
           }
@@ -750,9 +898,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
         // this CTA's rows: 64 gate + the same 64 up rows of paired block pb
         const int pb = ti.m * 2 + static_cast<int>(rank);
         const bool gate_warp = q < 2;
-        const float gx = act_scale ? act_scale[0] : 1.f, gh = act_scale ? act_scale[1] : 1.f;
+        const float gx = (!MX && act_scale) ? act_scale[0] : 1.f, gh = (!MX && act_scale) ? act_scale[1] : 1.f;
         const float six_gh = 6.0f * gh;
-        const float s_row = st[st_idx + (gate_warp ? 0 : 1)] * gx;
+        const float s_row = MX ? 1.f : st[st_idx + (gate_warp ? 0 : 1)] * gx;
         const int me = q * 32 + lane, partner = (q ^ 2) * 32 + lane;
         const int il = (q % 2) * 32 + lane;
         const int col_off = gate_warp ? 0 : 16;
@@ -777,27 +925,14 @@ __global__ void __launch_bounds__(kQThreads, 1)
           }
           epilogue_bar();
           float h[16];
-          float amax = 0.f;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            h[i] = tbuf[tok * 68 + grp * 17 + i];
-            amax = fmaxf(amax, fabsf(h[i]));
-          }
-          const uint8_t sq = f32_to_e4m3_sat(amax / six_gh);
-          const float sc = e4m3_to_f32(sq) * gh;
-          uint32_t packed[2] = {0u, 0u};
-          if (sc != 0.f) {
-#pragma unroll
-            for (int i = 0; i < 16; i += 2)
-              packed[i / 8] |= static_cast<uint32_t>(f32x2_to_e2m1x2(h[i + 1] / sc, h[i] / sc)) << (4 * (i % 8));
-          }
+          for (int i = 0; i < 16; ++i) h[i] = tbuf[tok * 68 + grp * 17 + i];
           const int tr = c0 + tok;   // token row within the 224-row block
-          *reinterpret_cast<uint2*>(out_q + static_cast<size_t>(prow + tr) * (Nw / 2) + (pb * 64 + grp * 16) / 2) =
-              make_uint2(packed[0], packed[1]);
-          out_sf[(static_cast<size_t>(blk * 2 + tr / 128) * (Nw / 64) + pb) * kSfChunk + sf_byte(tr % 128, grp)] = sq;
+          quant_store_h<MX>(h, gh, six_gh, out_q + static_cast<size_t>(prow + tr) * (Nw / 2) + (pb * 64 + grp * 16) / 2,
+                            out_sf, static_cast<size_t>(blk * 2 + tr / 128), tr % 128, pb, grp, Nw);
         }
       } else {
-        const float s_a = st[st_idx] * (act_scale ? act_scale[1] : 1.f);
+        const float s_a = MX ? 1.f : st[st_idx] * (act_scale ? act_scale[1] : 1.f);
         const int wrow = ti.m * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
         uint16_t* o = out_bf16 + static_cast<size_t>(ti.row0 + ti.n * kQN) * Nw + wrow;
         for (int c0 = 0; c0 < valid; c0 += 16) {
@@ -863,18 +998,18 @@ size_t nvfp4_ffn_workspace_bytes(int64_t P, int T, int E, int has_shared, int d,
          al256(static_cast<int64_t>(T) * (d / 16));
 }
 
-template <int BN, bool GATED>
+template <int BN, bool GATED, bool MX>
 static cudaError_t launch_nvfp4(const CUtensorMap& mA, const CUtensorMap& mAsh, const CUtensorMap& mB,
                                 const FfnArgs& a, const int32_t* prow0, int K, int Nw, int up_row0, size_t wsf_off,
                                 size_t st_off, int st_idx, const uint8_t* act_sf, uint8_t* out_q, uint8_t* out_sf,
                                 uint16_t* out_bf16, cudaStream_t st) {
   constexpr uint32_t kBBytes = ((BN * 128 + 1023) / 1024) * 1024;
   constexpr int NP = nvfp4_a_tiles(BN, GATED);
-  constexpr uint32_t kStageBytes = NP * kATileBytes + kBBytes + (NP + 1) * kSfStage;
+  constexpr uint32_t kStageBytes = NP * kATileBytes + kBBytes + (NP + 1) * F4Fmt<MX>::kSfStage;
   int stages = (200 * 1024 - 1024) / static_cast<int>(kStageBytes);
   if (stages > 8) stages = 8;
   const size_t smem = 1024 + static_cast<size_t>(stages) * kStageBytes;
-  auto kern = ffn_nvfp4_kernel<BN, GATED>;
+  auto kern = ffn_nvfp4_kernel<BN, GATED, MX>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   const int P = a.T * a.k;
@@ -890,14 +1025,16 @@ static cudaError_t launch_nvfp4(const CUtensorMap& mA, const CUtensorMap& mAsh, 
 // Groups averaging >= 192 rows run on CTA pairs with 224-token tiles.
 static bool nvfp4_pair_applicable(int P, int E) { return (P + E - 1) / E >= 192; }
 
-// Scale chunks as rows of 256 bytes (a stage's 4 chunks = 8 rows), no swizzle:
-// dims {256, rows[, slots]}, box {256, 8[, 1]}.
-static bool make_map_rows256(CUtensorMap* m, const void* base, uint64_t bytes, uint64_t slots, uint64_t slot_pitch) {
+// Scale chunks as rows of 256 bytes (a stage's chunks = box_rows rows: 8 for
+// NVFP4's four chunks, 4 for MXFP4's two), no swizzle:
+// dims {256, rows[, slots]}, box {256, box_rows[, 1]}.
+static bool make_map_rows256(CUtensorMap* m, const void* base, uint64_t bytes, uint64_t slots, uint64_t slot_pitch,
+                             uint32_t box_rows) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {256, bytes / 256, slots};
   cuuint64_t strides[2] = {256, slot_pitch};
-  cuuint32_t box[3] = {256, 8, 1};
+  cuuint32_t box[3] = {256, box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
   const cuuint32_t rank = slots > 0 ? 3 : 2;
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), dims, strides, box, es,
@@ -906,12 +1043,12 @@ static bool make_map_rows256(CUtensorMap* m, const void* base, uint64_t bytes, u
   return r == CUDA_SUCCESS;
 }
 
-template <bool GATED>
+template <bool GATED, bool MX>
 static cudaError_t launch_nvfp4_tc2_one(const CUtensorMap* maps, const FfnArgs& a, const int32_t* prow0, int K,
                                         int Nw, int up_row0, size_t st_off, int st_idx, uint8_t* out_q,
                                         uint8_t* out_sf, uint16_t* out_bf16, cudaStream_t st) {
-  const size_t smem = 1024 + static_cast<size_t>(kQStages) * kQStage;
-  auto kern = ffn_nvfp4_tc2_kernel<GATED>;
+  const size_t smem = 1024 + static_cast<size_t>(kQStages) * Q2Fmt<MX>::kStage;
+  auto kern = ffn_nvfp4_tc2_kernel<GATED, MX>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   const int P = a.T * a.k;
@@ -930,17 +1067,17 @@ static cudaError_t launch_nvfp4_tc2_one(const CUtensorMap* maps, const FfnArgs& 
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  static int pairs_max[2] = {0, 0};   // co-resident pairs (not every SM may find a partner)
-  if (!pairs_max[GATED]) {
+  static int pairs_max = 0;   // co-resident pairs of this instantiation (not every SM may find a partner)
+  if (!pairs_max) {
     cfg.gridDim = dim3(num_sms());
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
       (void)cudaGetLastError();
       n = num_sms() / 2;
     }
-    pairs_max[GATED] = n < num_sms() / 2 ? n : num_sms() / 2;
+    pairs_max = n < num_sms() / 2 ? n : num_sms() / 2;
   }
-  const int pairs = static_cast<int>(tiles < pairs_max[GATED] ? tiles : pairs_max[GATED]);
+  const int pairs = static_cast<int>(tiles < pairs_max ? tiles : pairs_max);
   cfg.gridDim = dim3(2 * pairs);
   cfg.numAttrs = 2;
   return count_launch(cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], a.offsets, prow0,
@@ -949,27 +1086,30 @@ static cudaError_t launch_nvfp4_tc2_one(const CUtensorMap* maps, const FfnArgs& 
 }
 
 // Both GEMMs on CTA pairs; xq/sfx (gathered, padded to 224-row blocks) are ready.
+template <bool MX>
 static const char* launch_nvfp4_gemms_tc2(const FfnArgs& a, const int32_t* prow0, size_t s_gu_off, size_t s_d_off,
                                           size_t s_t_off, int64_t rp, uint8_t* xq, uint8_t* sfx, size_t sfx_bytes,
                                           uint8_t* hq, uint8_t* sfh, size_t sfh_bytes, cudaStream_t st,
                                           cudaError_t* cerr) {
+  constexpr int G = F4Fmt<MX>::kGroup;
+  constexpr uint32_t kBox = 2 * F4Fmt<MX>::kChunks;   // 256-byte rows of a stage's chunks
   const uint64_t S = static_cast<uint64_t>(a.S);
-  const uint64_t s_gu_bytes = 2ull * a.I * (a.d / 16), s_d_bytes = static_cast<uint64_t>(a.d) * (a.I / 16);
+  const uint64_t s_gu_bytes = 2ull * a.I * (a.d / G), s_d_bytes = static_cast<uint64_t>(a.d) * (a.I / G);
   // maps per GEMM: A, A (shared expert), B, A scales, A scales (shared expert), B scales
   CUtensorMap m1[6], m2[6];
   bool ok = make_map_f4(&m1[0], a.pool + a.w_gu_off, a.d, 2ull * a.I, S, a.bank_bytes, 64) &&
             make_map_f4(&m1[2], xq, a.d, static_cast<uint64_t>(rp), 0, 0, kQH) &&
-            make_map_rows256(&m1[3], a.pool + s_gu_off, s_gu_bytes, S, a.bank_bytes) &&
-            make_map_rows256(&m1[5], sfx, sfx_bytes, 0, 0) &&
+            make_map_rows256(&m1[3], a.pool + s_gu_off, s_gu_bytes, S, a.bank_bytes, kBox) &&
+            make_map_rows256(&m1[5], sfx, sfx_bytes, 0, 0, kBox) &&
             make_map_f4(&m2[0], a.pool + a.w_d_off, a.I, a.d, S, a.bank_bytes, 128) &&
             make_map_f4(&m2[2], hq, a.I, static_cast<uint64_t>(rp), 0, 0, kQH) &&
-            make_map_rows256(&m2[3], a.pool + s_d_off, s_d_bytes, S, a.bank_bytes) &&
-            make_map_rows256(&m2[5], sfh, sfh_bytes, 0, 0);
+            make_map_rows256(&m2[3], a.pool + s_d_off, s_d_bytes, S, a.bank_bytes, kBox) &&
+            make_map_rows256(&m2[5], sfh, sfh_bytes, 0, 0, kBox);
   if (ok && a.has_shared) {
     ok = make_map_f4(&m1[1], a.shared_bank + a.w_gu_off, a.d, 2ull * a.I, 0, 0, 64) &&
-         make_map_rows256(&m1[4], a.shared_bank + s_gu_off, s_gu_bytes, 0, 0) &&
+         make_map_rows256(&m1[4], a.shared_bank + s_gu_off, s_gu_bytes, 0, 0, kBox) &&
          make_map_f4(&m2[1], a.shared_bank + a.w_d_off, a.I, a.d, 0, 0, 128) &&
-         make_map_rows256(&m2[4], a.shared_bank + s_d_off, s_d_bytes, 0, 0);
+         make_map_rows256(&m2[4], a.shared_bank + s_d_off, s_d_bytes, 0, 0, kBox);
   } else {
     m1[1] = m1[0];
     m1[4] = m1[3];
@@ -978,19 +1118,21 @@ static const char* launch_nvfp4_gemms_tc2(const FfnArgs& a, const int32_t* prow0
   }
   if (!ok) return "cuTensorMapEncodeTiled failed";
   prof_mark(FTM_K_GEMM1, st, false);
-  *cerr = launch_nvfp4_tc2_one<true>(m1, a, prow0, a.d, a.I, a.I, s_t_off, 0, hq, sfh, nullptr, st);
+  *cerr = launch_nvfp4_tc2_one<true, MX>(m1, a, prow0, a.d, a.I, a.I, s_t_off, 0, hq, sfh, nullptr, st);
   prof_mark(FTM_K_GEMM1, st, true);
   if (*cerr != cudaSuccess) return "nvfp4 pair gemm1 launch failed";
   prof_mark(FTM_K_GEMM2, st, false);
-  *cerr = launch_nvfp4_tc2_one<false>(m2, a, prow0, a.I, a.d, 0, s_t_off, 2, nullptr, nullptr,
-                                      reinterpret_cast<uint16_t*>(a.y), st);
+  *cerr = launch_nvfp4_tc2_one<false, MX>(m2, a, prow0, a.I, a.d, 0, s_t_off, 2, nullptr, nullptr,
+                                          reinterpret_cast<uint16_t*>(a.y), st);
   prof_mark(FTM_K_GEMM2, st, true);
   if (*cerr != cudaSuccess) return "nvfp4 pair gemm2 launch failed";
   return nullptr;
 }
 
-const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_d_off, size_t s_t_off, uint8_t* ws,
-                                    cudaStream_t st, cudaError_t* cerr) {
+template <bool MX>
+static const char* launch_f4(const FfnArgs& a, size_t s_gu_off, size_t s_d_off, size_t s_t_off, uint8_t* ws,
+                             cudaStream_t st, cudaError_t* cerr) {
+  constexpr int kCK = F4Fmt<MX>::kChunkK;
   const int P = a.T * a.k;
   const int G = a.E + (a.has_shared ? 1 : 0);
   *cerr = cudaSuccess;
@@ -1002,6 +1144,7 @@ const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_
   int32_t* prow0 = reinterpret_cast<int32_t*>(ws);
   uint8_t* xq = ws + al256(sizeof(int32_t) * (G + 1));
   uint8_t* sfx = xq + al256(rp * (a.d / 2));
+  // regions sized for NVFP4's chunks (MXFP4 uses half of each scale region)
   uint8_t* hq = sfx + al256(blocks * (a.d / 64) * kSfChunk);
   uint8_t* sfh = hq + al256(rp * (a.I / 2));
   uint8_t* xq_tok = sfh + al256(blocks * (a.I / 64) * kSfChunk);
@@ -1012,19 +1155,19 @@ const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_
   *cerr = launch_pdl(pad_offsets_kernel, dim3(1), dim3(512), 0, st, a.offsets, a.E, a.has_shared, a.T, BN, prow0);
   if (*cerr == cudaSuccess) {
     const int grid = a.T / 8 + 1 < 148 * 8 ? a.T / 8 + 1 : 148 * 8;
-    *cerr = launch_pdl(quant_tokens_nvfp4_kernel, dim3(grid), dim3(256), 0, st,
+    *cerr = launch_pdl(quant_tokens_f4_kernel<MX>, dim3(grid), dim3(256), 0, st,
                        reinterpret_cast<const uint16_t*>(a.x), a.T, a.d, a.act_scale, xq_tok, s_tok);
   }
   if (*cerr == cudaSuccess) {
     const int grid = static_cast<int>(rp / 8 + 1 < 148 * 8 ? rp / 8 + 1 : 148 * 8);
-    *cerr = launch_pdl(gather_nvfp4_kernel, dim3(grid), dim3(256), 0, st, xq_tok, s_tok, a.perm, a.offsets, prow0,
+    *cerr = launch_pdl(gather_f4_kernel<MX>, dim3(grid), dim3(256), 0, st, xq_tok, s_tok, a.perm, a.offsets, prow0,
                        a.E, a.has_shared, a.T, a.k, a.d, BN, xq, sfx);
   }
   prof_mark(FTM_K_GATHER, st, true);
   if (*cerr != cudaSuccess) return "nvfp4 gather launch failed";
   if (pair)
-    return launch_nvfp4_gemms_tc2(a, prow0, s_gu_off, s_d_off, s_t_off, rp, xq, sfx, blocks * (a.d / 64) * kSfChunk,
-                                  hq, sfh, blocks * (a.I / 64) * kSfChunk, st, cerr);
+    return launch_nvfp4_gemms_tc2<MX>(a, prow0, s_gu_off, s_d_off, s_t_off, rp, xq, sfx,
+                                      blocks * (a.d / kCK) * kSfChunk, hq, sfh, blocks * (a.I / kCK) * kSfChunk, st, cerr);
   CUtensorMap mA1, mAsh1, mB1, mA2, mAsh2, mB2;
   const uint64_t S = static_cast<uint64_t>(a.S);
   // gate/up boxes are 64 rows: a tile stages 64 gate rows and the same 64 up rows
@@ -1041,25 +1184,36 @@ const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_
   }
   if (!ok) return "cuTensorMapEncodeTiled failed";
   prof_mark(FTM_K_GEMM1, st, false);
-  *cerr = BN == 32 ? launch_nvfp4<32, true>(mA1, mAsh1, mB1, a, prow0, a.d, a.I, a.I, s_gu_off, s_t_off, 0, sfx, hq,
+  *cerr = BN == 32 ? launch_nvfp4<32, true, MX>(mA1, mAsh1, mB1, a, prow0, a.d, a.I, a.I, s_gu_off, s_t_off, 0, sfx, hq,
                                             sfh, nullptr, st)
-          : BN == 64 ? launch_nvfp4<64, true>(mA1, mAsh1, mB1, a, prow0, a.d, a.I, a.I, s_gu_off, s_t_off, 0, sfx, hq,
+          : BN == 64 ? launch_nvfp4<64, true, MX>(mA1, mAsh1, mB1, a, prow0, a.d, a.I, a.I, s_gu_off, s_t_off, 0, sfx, hq,
                                               sfh, nullptr, st)
-                     : launch_nvfp4<128, true>(mA1, mAsh1, mB1, a, prow0, a.d, a.I, a.I, s_gu_off, s_t_off, 0, sfx,
+                     : launch_nvfp4<128, true, MX>(mA1, mAsh1, mB1, a, prow0, a.d, a.I, a.I, s_gu_off, s_t_off, 0, sfx,
                                                hq, sfh, nullptr, st);
   prof_mark(FTM_K_GEMM1, st, true);
   if (*cerr != cudaSuccess) return "nvfp4 gemm1 launch failed";
   prof_mark(FTM_K_GEMM2, st, false);
   uint16_t* y = reinterpret_cast<uint16_t*>(a.y);
-  *cerr = BN == 32 ? launch_nvfp4<32, false>(mA2, mAsh2, mB2, a, prow0, a.I, a.d, 0, s_d_off, s_t_off, 2, sfh,
+  *cerr = BN == 32 ? launch_nvfp4<32, false, MX>(mA2, mAsh2, mB2, a, prow0, a.I, a.d, 0, s_d_off, s_t_off, 2, sfh,
                                              nullptr, nullptr, y, st)
-          : BN == 64 ? launch_nvfp4<64, false>(mA2, mAsh2, mB2, a, prow0, a.I, a.d, 0, s_d_off, s_t_off, 2, sfh,
+          : BN == 64 ? launch_nvfp4<64, false, MX>(mA2, mAsh2, mB2, a, prow0, a.I, a.d, 0, s_d_off, s_t_off, 2, sfh,
                                                nullptr, nullptr, y, st)
-                     : launch_nvfp4<128, false>(mA2, mAsh2, mB2, a, prow0, a.I, a.d, 0, s_d_off, s_t_off, 2, sfh,
+                     : launch_nvfp4<128, false, MX>(mA2, mAsh2, mB2, a, prow0, a.I, a.d, 0, s_d_off, s_t_off, 2, sfh,
                                                 nullptr, nullptr, y, st);
   prof_mark(FTM_K_GEMM2, st, true);
   if (*cerr != cudaSuccess) return "nvfp4 gemm2 launch failed";
   return nullptr;
+}
+
+const char* launch_expert_ffn_nvfp4(const FfnArgs& a, size_t s_gu_off, size_t s_d_off, size_t s_t_off, uint8_t* ws,
+                                    cudaStream_t st, cudaError_t* cerr) {
+  return launch_f4<false>(a, s_gu_off, s_d_off, s_t_off, ws, st, cerr);
+}
+
+// MXFP4: the same kernels with E8M0 scales per 32 elements; no tensor scale.
+const char* launch_expert_ffn_mxfp4(const FfnArgs& a, size_t s_gu_off, size_t s_d_off, uint8_t* ws, cudaStream_t st,
+                                    cudaError_t* cerr) {
+  return launch_f4<true>(a, s_gu_off, s_d_off, 0, ws, st, cerr);
 }
 
 }  // namespace ftm

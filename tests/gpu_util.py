@@ -12,7 +12,7 @@ import oracle
 import synth
 from synth.device import DeviceLayer, Workspace
 
-TOL = {"f32": 2e-2, "bf16": 2e-2, "fp8": 5e-2, "nvfp4": 5e-2}
+TOL = {"f32": 2e-2, "bf16": 2e-2, "fp8": 5e-2, "nvfp4": 5e-2, "mxfp4": 5e-2}
 TOL_F32_SIMT = 1e-4
 
 

@@ -42,6 +42,10 @@ def test_bank_layouts():
         assert bl.w_gu_off == 0 and bl.w_d_off >= bl.w_gu_bytes
     bl = ftm.ftm_get_bank_layout(ftm.desc_for(synth.CONFIGS["284b_trace"]))
     assert bl.bank_bytes == 25171968           # 25.17 MB per FP8 expert incl. 6,144 B of block scales
+    mx = ftm.ftm_get_bank_layout(ftm.desc_for(synth.CONFIGS["753b_mxfp4"]))
+    d, I = 6144, 2048
+    assert (mx.w_gu_bytes, mx.w_d_bytes, mx.s_gu_bytes, mx.s_d_bytes, mx.s_t_bytes) == \
+        (2 * I * d // 2, d * I // 2, 2 * I * d // 32, d * I // 32, 0)
 
 
 @pytest.mark.parametrize("field,value", [("d", 100), ("d", 0), ("I", 96), ("k", 0), ("k", 9), ("E", 0),
