@@ -61,6 +61,9 @@ def parse():
     p.add_argument("--config", default=None, choices=list(synth.CONFIGS),
                    help="run this workload only (default: the headline and, at N = 1, every workload)")
     p.add_argument("--T", type=int, default=None, help="tokens per step with --config (default: its largest)")
+    p.add_argument("--experts", type=int, default=None,
+                   help="with --config: the same layer with this many routed experts (and slots), e.g. a small "
+                        "case of the same shape for a profiler capture")
     p.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying CUDA graphs")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=6.0, help="per CPU-baseline mode")
@@ -120,7 +123,7 @@ def peaks():
 
 
 KERNEL_FILES = {"bf16": ("ftm_ffn.cu", "ftm_ffn_tc2.cu"), "f32": ("ftm_ffn.cu",), "fp8": ("ftm_ffn_fp8.cu",),
-                "nvfp4": ("ftm_ffn_nvfp4.cu",)}
+                "nvfp4": ("ftm_ffn_nvfp4.cu",), "mxfp4": ("ftm_ffn_nvfp4.cu",)}
 
 
 def kernel_source_hash(wdtype: str) -> str:
@@ -150,7 +153,7 @@ def dtype_peak(pk: dict, src: str, wdtype: str):
     """Dense tensor peak of a dtype (TFLOP/s) and where it comes from: the measured
     sustained bf16 figure times the nominal dense ratio for fp8 (2) and fp4 (4)."""
     bf16 = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
-    ratio = {"f32": 1.0, "bf16": 1.0, "fp8": 2.0, "nvfp4": 4.0}[wdtype]
+    ratio = {"f32": 1.0, "bf16": 1.0, "fp8": 2.0, "nvfp4": 4.0, "mxfp4": 4.0}[wdtype]
     where = (f"{src} bf16_tflops_sustained" if ratio == 1.0 else
              f"derived: {ratio:g} x {src} bf16_tflops_sustained (nominal dense ratio)")
     return bf16 * ratio, where
@@ -237,7 +240,7 @@ def algorithmic(cfg, bl, T, counts):
     """Algorithmic bytes and flops of GEMM1 and of the whole layer step.  Bytes:
     the weight bytes of every expert touched (gate/up, down and their scales,
     i.e. its bank) plus the activations each GEMM reads and writes once."""
-    wb = {"f32": 4, "bf16": 2, "fp8": 1, "nvfp4": 0.5}[cfg.wdtype]
+    wb = {"f32": 4, "bf16": 2, "fp8": 1, "nvfp4": 0.5, "mxfp4": 0.5}[cfg.wdtype]
     ab = 4 if cfg.act_dtype == "f32" else 2
     groups = int((counts > 0).sum()) + (1 if cfg.has_shared else 0)
     rows = T * cfg.k + (T if cfg.has_shared else 0)
@@ -821,6 +824,10 @@ def main():
     if args.config:
         head = (args.config, args.T or max(synth.CONFIGS[args.config].T))
         suite = ()
+        if args.experts:
+            c = synth.CONFIGS[args.config]
+            synth.CONFIGS[args.config] = synth.scaled(c, E=args.experts, S=min(c.S, args.experts),
+                                                      k=min(c.k, args.experts))
     else:
         head = HEADLINE
         suite = SUITE if world == 1 else ()

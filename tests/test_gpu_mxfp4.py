@@ -30,8 +30,11 @@ def _check(dl, T, rows=None):
 def test_small_mxfp4_layer(T):
     dl = screened_layer(SMALL_MX, T)
     out, x, ids, g, rows = _check(dl, T)
+    # against the oracle without activation quantisation: the W4A4 error itself.
+    # E8M0 scales put a block's amax between 4 and 8 units of its scale, so
+    # values above 6 saturate: a looser bound than NVFP4's e4m3 scales need
     plain = oracle.moe_rows(dl.layer, x, rows, ids, g, qa=oracle.QA_NONE)
-    assert_rows_close(out[rows], plain, 0.35, "mxfp4 vs unquantised activations")
+    assert_rows_close(out[rows], plain, 0.5, "mxfp4 vs unquantised activations")
 
 
 def test_mxfp4_pair_tiles_multi_stage():
