@@ -210,9 +210,12 @@ def packed_banks(cfg, cache_dir: str, local_rank: int, dist, seed: int = 0):
     return pack_banks(cfg, seed)
 
 
-def device_layer(cfg, args, local, dist):
+def device_layer(cfg, args, local, dist, cache: bool = False):
+    """The layer on this device.  cache: draw its banks once per host and keep
+    them on disk (the headline layer, which every rank of a multi-GPU run and
+    later runs on the same host stage again); the other layers are drawn here."""
     from synth.device import DeviceLayer
-    return DeviceLayer(cfg, banks=packed_banks(cfg, args.bank_cache, local, dist))
+    return DeviceLayer(cfg, banks=packed_banks(cfg, args.bank_cache if cache else "", local, dist))
 
 
 def workload_name(cfg, T):
@@ -641,7 +644,7 @@ def run_layers_pipeline(cfg, T, n_layers, args, local):
     hp = host_pool.numpy()
     weights, keep = [], []
     for l in range(n_layers):
-        banks = packed_banks(cfg, args.bank_cache, local, None, seed=l)
+        banks = packed_banks(cfg, "", local, None, seed=l)
         hp[l * E * bb:(l + 1) * E * bb] = np.asarray(banks[:E]).reshape(-1)
         layer = synth.Layer(cfg, seed=l)
         wr = to_device_storage(layer.router_storage(), cfg.act_dtype)
@@ -842,7 +845,7 @@ def main():
             for T in Ts:
                 records.append(run_trace(cfg, T, args, dist, local))
             continue
-        dl = device_layer(cfg, args, local, dist)
+        dl = device_layer(cfg, args, local, dist, cache=name == head[0])
         for T in Ts:
             try:
                 records.append(run_resident(dl, T, args, dist, local))
@@ -858,7 +861,7 @@ def main():
         if head_cfg.lru:
             head_rec = run_trace(head_cfg, head[1], args, dist, local)
         else:
-            dl = device_layer(head_cfg, args, local, dist)
+            dl = device_layer(head_cfg, args, local, dist, cache=True)
             head_rec = run_resident(dl, head[1], args, dist, local)
             del dl
     if rank == 0:

@@ -341,9 +341,6 @@ static cudaError_t launch_tc(const CUtensorMap& mA, const CUtensorMap& mAsh, con
     const int s = (200 * 1024 - 1024 - red_bytes) / static_cast<int>(kStageBytes);
     return s > 8 ? 8 : s;
   };
-  auto smem_for = [&](int ks) {
-    return 1024 + static_cast<size_t>(stages_for(ks)) * kStageBytes + static_cast<size_t>(ks - 1) * 128 * kRedStride * 4;
-  };
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kTcThreads);
   cfg.stream = st;
@@ -356,31 +353,53 @@ static cudaError_t launch_tc(const CUtensorMap& mA, const CUtensorMap& mAsh, con
   cfg.attrs = attr;
   // Split-K when the tiles cannot fill the GPU: a cluster of ks CTAs per tile,
   // the largest ks <= 4 (and <= the k-blocks) whose clusters all fit at once
-  // (one wave: a second wave of clusters would double the kernel time).
-  static int max_clusters[5] = {0, 0, 0, 0, 0};   // co-resident clusters of ks CTAs, per ks
-  int ks = 1;
-  if (tiles > 0 && 2 * tiles <= num_sms()) {
-    for (int c = 4; c >= 2; --c) {
-      if (c > KB || c * tiles > num_sms()) continue;
-      if (!max_clusters[c]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_for(c)));
-        if (e != cudaSuccess) return e;
+  // (one wave: a second wave of clusters would double the kernel time).  When
+  // one CTA per SM leaves too few clusters, a configuration with fewer stages
+  // lets two CTAs share an SM (only when twice their tensor memory fits).
+  constexpr uint32_t kAccCols = GATED ? 2 * BN : BN;
+  constexpr uint32_t kTmemCols = 2 * kAccCols < 32 ? 32 : 2 * kAccCols;
+  auto smem_of = [&](int ks, int st) {
+    return 1024 + static_cast<size_t>(st) * kStageBytes + static_cast<size_t>(ks - 1) * 128 * kRedStride * 4;
+  };
+  auto stages_two_per_sm = [&](int ks) {       // stages that fit half an SM's shared memory
+    const int budget = 113 * 1024 - 1024 - (ks - 1) * 128 * kRedStride * 4;
+    const int st = budget / static_cast<int>(kStageBytes);
+    return st < stages_for(ks) ? st : stages_for(ks);
+  };
+  static int max_clusters[5][2] = {};   // co-resident clusters of ks CTAs, per ks and config (1 or 2 CTAs per SM)
+  auto clusters = [&](int c, int two) -> int {
+    if (!max_clusters[c][two]) {
+      const int st = two ? stages_two_per_sm(c) : stages_for(c);
+      const size_t sm = smem_of(c, st);
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
+      int n = 0;
+      if (e == cudaSuccess) {
         attr[0].val.clusterDim.x = c;
         cfg.numAttrs = 1;
-        cfg.dynamicSmemBytes = smem_for(c);
+        cfg.dynamicSmemBytes = sm;
         cfg.gridDim = dim3(num_sms() / c * c);
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
-          (void)cudaGetLastError();
-          n = 0;
-        }
-        max_clusters[c] = n > 0 ? n : -1;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = 0;
       }
-      if (tiles <= max_clusters[c]) { ks = c; break; }
+      (void)cudaGetLastError();
+      max_clusters[c][two] = n > 0 ? n : -1;
+    }
+    return max_clusters[c][two];
+  };
+  int ks = 1, stages = stages_for(1);
+  if (tiles > 0 && tiles < num_sms()) {
+    for (int c = 4; c >= 2 && ks == 1; --c) {
+      if (c > KB) continue;
+      if (2 * tiles <= num_sms() && c * tiles <= num_sms() && tiles <= clusters(c, 0)) {
+        ks = c;
+        stages = stages_for(c);
+      } else if (2 * kTmemCols <= 512 && stages_two_per_sm(c) >= 3 && c * tiles <= 2 * num_sms() &&
+                 tiles <= clusters(c, 1)) {
+        ks = c;
+        stages = stages_two_per_sm(c);
+      }
     }
   }
-  const int stages = stages_for(ks);
-  const size_t smem = smem_for(ks);
+  const size_t smem = smem_of(ks, stages);
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   if (ks == 1) {
