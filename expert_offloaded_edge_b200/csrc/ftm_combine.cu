@@ -1,53 +1,73 @@
 // Weighted un-permute and combine (step a8):
 //   out[t] = sum_{j ascending} g[t][j] * y[inv[t*k + j]]  (+ y[P + t] for the shared expert)
-// fp32 accumulation, fixed summation order (deterministic).  One block per
+// fp32 accumulation, fixed summation order (deterministic).  One warp per
 // token (grid-strided), 16-byte loads and stores along d.
 #include "ftm_common.cuh"
 
 namespace ftm {
 
+constexpr int kMaxTerms = 17;   // k <= 16 routed picks + the shared expert
+
+// One warp per token: lane j < k fetches the token's j-th row index and gate
+// (lane k: the shared expert's row, gate 1), the warp shares them by shuffles,
+// then every lane walks its 16-byte vectors of d, issuing all of the token's
+// row loads before the fused multiply-adds.  The terms are added in ascending
+// j, so the result does not depend on the schedule.
 template <bool F32>
-__global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ y, const int32_t* __restrict__ inv,
+__global__ void __launch_bounds__(256, 2) combine_kernel(const void* __restrict__ y, const int32_t* __restrict__ inv,
                                                       const float* __restrict__ gw, int T, int k, int d, int P,
                                                       int has_shared, void* __restrict__ out) {
   constexpr int V = F32 ? 4 : 8;   // elements per 16-byte vector
-  __shared__ int32_t s_row[17];
-  __shared__ float s_g[17];
+  constexpr int EB = F32 ? 4 : 2;  // bytes per element
   const int nv = d / V;
   const int nterms = k + (has_shared ? 1 : 0);
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  __shared__ int s_rows[8][kMaxTerms];
+  __shared__ float s_gs[8][kMaxTerms];
   pdl_wait();
   pdl_trigger();
-  for (int t = blockIdx.x; t < T; t += gridDim.x) {
-    // the token's rows and weights first, so the row loads below are independent
-    if (threadIdx.x < nterms) {
-      const int j = threadIdx.x;
-      int row = j < k ? inv[static_cast<size_t>(t) * k + j] : P + t;
-      if (j < k && (row < 0 || row >= P)) {   // a pair the permutation skipped (id out of range)
+  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
+    int my_row = -1;
+    float my_g = 0.f;
+    if (lane < nterms) {
+      int row = lane < k ? inv[static_cast<size_t>(t) * k + lane] : P + t;
+      if (lane < k && (row < 0 || row >= P)) {   // a pair the permutation skipped (id out of range)
         report_bad_index();
         row = -1;
       }
-      s_row[j] = row;
-      s_g[j] = j < k ? gw[static_cast<size_t>(t) * k + j] : 1.f;
+      my_row = row;
+      my_g = lane < k ? gw[static_cast<size_t>(t) * k + lane] : 1.f;
     }
-    __syncthreads();
-    for (int c = threadIdx.x; c < nv; c += blockDim.x) {
+    // the warp's copy of the token's rows and gates
+    int* rows = s_rows[threadIdx.x >> 5];
+    float* gs = s_gs[threadIdx.x >> 5];
+    if (lane < kMaxTerms) {
+      rows[lane] = lane < nterms ? my_row : -1;
+      gs[lane] = my_g;
+    }
+    __syncwarp();
+    for (int c = lane; c < nv; c += 32) {
+      uint4 u[kMaxTerms];
+#pragma unroll
+      for (int j = 0; j < kMaxTerms; ++j)
+        if (j < nterms && rows[j] >= 0)
+          u[j] = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(y) +
+                                                 (static_cast<size_t>(rows[j]) * d + static_cast<size_t>(c) * V) * EB);
       float acc[V];
 #pragma unroll
       for (int i = 0; i < V; ++i) acc[i] = 0.f;
-#pragma unroll 4
-      for (int j = 0; j < nterms; ++j) {
-        const int row = s_row[j];
-        if (row < 0) continue;
-        const float g = s_g[j];
-        const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(y) +
-                                                        (static_cast<size_t>(row) * d + static_cast<size_t>(c) * V) *
-                                                            (F32 ? 4 : 2));
+#pragma unroll
+      for (int j = 0; j < kMaxTerms; ++j) {
+        if (j >= nterms || rows[j] < 0) continue;
+        const float g = gs[j];
         if constexpr (F32) {
-          const float f[4] = {__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w)};
+          const float f[4] = {__uint_as_float(u[j].x), __uint_as_float(u[j].y), __uint_as_float(u[j].z),
+                              __uint_as_float(u[j].w)};
 #pragma unroll
           for (int i = 0; i < 4; ++i) acc[i] = fmaf(g, f[i], acc[i]);
         } else {
-          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+          const uint32_t w[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             acc[2 * i] = fmaf(g, __uint_as_float(w[i] << 16), acc[2 * i]);
@@ -69,15 +89,16 @@ __global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ y
         o = make_uint4(w[0], w[1], w[2], w[3]);
       }
       *reinterpret_cast<uint4*>(static_cast<uint8_t*>(out) +
-                                (static_cast<size_t>(t) * d + static_cast<size_t>(c) * V) * (F32 ? 4 : 2)) = o;
+                                (static_cast<size_t>(t) * d + static_cast<size_t>(c) * V) * EB) = o;
     }
-    __syncthreads();   // s_row / s_g are rewritten for the next token
+    __syncwarp();   // the warp's rows and gates are rewritten for its next token
   }
 }
 
 cudaError_t launch_combine(bool f32, const void* y, const int32_t* inv, const float* gw, int T, int k, int d, int P,
                            int has_shared, void* out, cudaStream_t st) {
-  const int grid = T < 148 * 16 ? T : 148 * 16;
+  const int blocks = (T + 7) / 8;   // 8 tokens (warps) per block
+  const int grid = blocks < 148 * 8 ? blocks : 148 * 8;
   if (f32)
     return launch_pdl(combine_kernel<true>, dim3(grid), dim3(256), 0, st, y, inv, gw, T, k, d, P, has_shared, out);
   else

@@ -25,20 +25,36 @@ __device__ int32_t g_dev_status = 0;
 
 // ---------------------------------------------------------------------------
 // Gather: X_p[pos] = x[perm[pos] / k] (pos < P); X_p[P + t] = x[t] (shared rows).
-// ---------------------------------------------------------------------------
-__global__ void gather_rows_kernel(const uint8_t* __restrict__ x, const int32_t* __restrict__ perm, int P, int k,
-                                   int T, int has_shared, int row_bytes, uint8_t* __restrict__ xp) {
+// One warp per row (grid-strided); each lane moves up to 8 of the row's
+// 16-byte vectors per round, all loads of a round issued before its stores.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint8_t* __restrict__ x,
+                                                          const int32_t* __restrict__ perm, int P, int k, int T,
+                                                          int has_shared, int row_bytes, uint8_t* __restrict__ xp) {
   pdl_wait();
   pdl_trigger();
   const int rows = P + (has_shared ? T : 0);
   const int nv = row_bytes / 16;
-  for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < rows; r += gridDim.x * wpb) {
     const int q = r < P ? perm[r] : 0;
     if (q < 0) continue;     // no pair placed here (ids out of range); no group reads this row
     const int src = r < P ? q / k : r - P;
     const uint4* s = reinterpret_cast<const uint4*>(x + static_cast<size_t>(src) * row_bytes);
     uint4* dd = reinterpret_cast<uint4*>(xp + static_cast<size_t>(r) * row_bytes);
-    for (int c = threadIdx.x; c < nv; c += blockDim.x) dd[c] = s[c];
+    for (int c0 = 0; c0 < nv; c0 += 32 * 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < nv) v[u] = s[c];
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < nv) dd[c] = v[u];
+      }
+    }
   }
 }
 
@@ -447,7 +463,8 @@ const char* launch_expert_ffn(const FfnArgs& a, cudaStream_t st, cudaError_t* ce
   if (rows == 0) return nullptr;
   const int elt = a.f32 ? 4 : 2;
   {
-    const int grid = rows < 148 * 8 ? rows : 148 * 8;
+    const int blocks = (rows + 7) / 8;   // 8 rows (warps) per block
+    const int grid = blocks < 148 * 16 ? blocks : 148 * 16;
     prof_mark(FTM_K_GATHER, st, false);
     *cerr = launch_pdl(gather_rows_kernel, dim3(grid), dim3(256), 0, st, a.x, a.perm, P, a.k, a.T, a.has_shared,
                        a.d * elt, a.xp);

@@ -280,7 +280,19 @@ __global__ void __launch_bounds__(256) gather_f4_kernel(const uint8_t* __restric
     src = __shfl_sync(0xffffffffu, src, 0);
     const uint4* s = reinterpret_cast<const uint4*>(xq_tok + static_cast<size_t>(src < 0 ? 0 : src) * (d / 2));
     uint4* dst = reinterpret_cast<uint4*>(xq + static_cast<size_t>(pr) * (d / 2));
-    for (int c = lane; c < nvec; c += 32) dst[c] = src >= 0 ? s[c] : make_uint4(0, 0, 0, 0);
+    for (int c0 = 0; c0 < nvec; c0 += 32 * 8) {     // up to 8 loads in flight per lane, then the stores
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int c = c0 + u * 32 + lane;
+        v[u] = (c < nvec && src >= 0) ? s[c] : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < nvec) dst[c] = v[u];
+      }
+    }
     const int blk = pr / BN, r = pr % BN;
     const uint32_t* sw = reinterpret_cast<const uint32_t*>(s_tok + static_cast<size_t>(src < 0 ? 0 : src) * (4 * nkc));
     uint8_t* chunk0 = sfx + (static_cast<size_t>(blk) * nsub + r / 128) * nkc * kSfChunk + sf_byte(r % 128, 0);

@@ -6,14 +6,15 @@
 // lanes, ranks across warps from per-warp per-expert counts in shared memory,
 // ranks across blocks from per-chunk histograms and a column scan.  Small P
 // runs as one block in one launch; large P as histogram / scan / scatter over
-// chunks of kChunk pairs.
+// chunks of kChunk pairs (larger P).
 #include "ftm_common.cuh"
 
 namespace ftm {
 
 constexpr int kPermThreads = 1024;
 constexpr int kPermWarps = kPermThreads / 32;
-constexpr int kChunk = 4096;
+constexpr int kSingleMax = 4096;   // pairs one block sorts in one launch
+constexpr int kChunk = 1024;       // pairs per block of the three-pass sort (one round of the block's threads)
 
 // Warp 0 only: out[e] = sum_{e' < e} in[e'] for e in [0, E); returns the total in out[E].
 __device__ void warp0_exclusive_scan(const int32_t* in, int32_t* out, int E) {
@@ -76,7 +77,7 @@ __device__ void stable_scatter(const int32_t* __restrict__ ids, int q_begin, int
   }
 }
 
-// One block does everything (P <= kChunk).
+// One block does everything (P <= kSingleMax).
 __global__ void __launch_bounds__(kPermThreads) permute_single_kernel(const int32_t* __restrict__ ids, int P, int E,
                                                                       int32_t* __restrict__ counts,
                                                                       int32_t* __restrict__ offsets,
@@ -169,14 +170,15 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(const int
 }
 
 size_t permute_workspace_bytes(int E, int64_t P) {
+  if (P <= kSingleMax) return 0;
   const int64_t nchunks = (P + kChunk - 1) / kChunk;
-  return nchunks > 1 ? static_cast<size_t>(nchunks * E) * sizeof(int32_t) : 0;
+  return static_cast<size_t>(nchunks * E) * sizeof(int32_t);
 }
 
 cudaError_t launch_permute(const int32_t* ids, int P, int E, int32_t* counts, int32_t* offsets, int32_t* perm,
                            int32_t* inv, void* ws, cudaStream_t st) {
   const size_t wsm = sizeof(int32_t) * (static_cast<size_t>(kPermWarps) * E + 2 * E + 1);
-  if (P <= kChunk) {
+  if (P <= kSingleMax) {
     cudaError_t err = cudaFuncSetAttribute(permute_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(wsm));
     if (err != cudaSuccess) return err;

@@ -32,9 +32,12 @@ def test_route_configs(name, T):
 
 @pytest.mark.parametrize("E,k,d,T,dt", [(37, 1, 128, 5, "bf16"), (16, 16, 128, 3, "bf16"), (300, 7, 256, 33, "bf16"),
                                         (8, 8, 128, 9, "f32"), (512, 16, 128, 17, "bf16"), (1, 1, 128, 4, "f32"),
-                                        # tensor-core router: 64-token tiles (one and two 128-row router
-                                        # tiles) and 128-token tiles (one and two), ragged last tile
+                                        # cluster router at medium batches
                                         (120, 4, 256, 300, "bf16"), (200, 6, 128, 333, "bf16"),
+                                        # tensor-core router (T >= 2048): 128-token tiles, experts on the
+                                        # MMA N side padded to 16 (N = 48 .. 256), ragged last tiles, k = 16
+                                        (37, 3, 128, 2049, "bf16"), (120, 4, 256, 2100, "bf16"),
+                                        (200, 6, 128, 2500, "bf16"), (256, 16, 256, 3000, "bf16"),
                                         (128, 8, 256, 10000, "bf16"), (160, 8, 256, 9601, "bf16")])
 def test_route_shapes(E, k, d, T, dt):
     cfg = synth.LayerConfig("route_case", d=d, E=E, k=k, I=128, wdtype=dt, has_shared=0, S=E, bias="uniform", T=(T,))
