@@ -625,22 +625,27 @@ constexpr int kQH = kQN / 2;                    // token rows staged per CTA
 constexpr uint32_t kQABytes = 128 * 128;        // 128 weight rows x 256 e2m1
 constexpr uint32_t kQBBytes = kQH * 128;        // 112 token rows x 256 e2m1
 constexpr int kQStages = 5;
-constexpr uint32_t kQSfCol = 2 * kQN;           // TMEM: accumulators [0, 448), then two half-stage scale slots
+constexpr uint32_t kQSfCol = 2 * kQN;           // TMEM: accumulators [0, 448), then the ring of scale units
 constexpr int kQThreads = 224;                  // warps 0 TMA, 1 MMA, 2-5 epilogue, 6 scale copies
 
 // Stage layout of the pair kernel per scale format: A tile | B tile | the
 // stage's scale chunks of this CTA's 128 weight rows | of the token block's
-// two 128-row halves.  A half stage (2 K steps) of scales in TMEM: NVFP4 2 x 4
-// columns SFA + 2 x 8 SFB (one chunk per K step); MXFP4 4 SFA + 8 SFB (both K
-// steps share one chunk).
+// two 128-row halves.  In TMEM the scales travel in units of one chunk per
+// operand: 4 columns of weight scales + 2 x 4 of token scales (the block's two
+// 128-row halves), 12 columns per unit.  A unit serves one K step (NVFP4) or
+// two (MXFP4, through scale-factor ids 0 and 2); units cycle through a ring
+// of kUnitRing slots so the copies can run several units ahead of the MMAs.
+constexpr uint32_t kUnitCols = 12;
+constexpr int kUnitRing = 5;
+static_assert(kQSfCol + kUnitRing * kUnitCols <= 512, "TMEM budget");
+
 template <bool MX>
 struct Q2Fmt {
   static constexpr uint32_t kSfa = F4Fmt<MX>::kSfStage;
   static constexpr uint32_t kSfb = 2 * F4Fmt<MX>::kSfStage;
   static constexpr uint32_t kStage = kQABytes + kQBBytes + kSfa + kSfb;
-  static constexpr uint32_t kHalfCols = MX ? 12 : 24;
+  static constexpr int kUnits = F4Fmt<MX>::kChunks;     // scale units per stage
   static_assert(kStage % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled tiles");
-  static_assert(kQSfCol + 2 * kHalfCols <= 512, "TMEM budget");
 };
 
 __device__ __forceinline__ int quad_tile_n(int valid) { return min(kQN, (valid + 31) & ~31); }
@@ -695,14 +700,13 @@ __global__ void __launch_bounds__(kQThreads, 1)
   using Q = Q2Fmt<MX>;
   constexpr int kCh = F4Fmt<MX>::kChunks;
   constexpr uint32_t kQStage = Q::kStage;
-  constexpr uint32_t kQSfHalfCols = Q::kHalfCols;
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kQStages], empty_bar[kQStages], tfull_bar[2], tempty_bar[2];
-  // Scale copies and MMAs run from different threads.  Half h of a stage (K steps 2h, 2h + 1) always uses
-  // scale slot h: sf_ready[h * kQStages + stage] = that half's scales are in TMEM, sf_free[h] = the MMAs that
-  // read slot h are done, so the copies of one half overlap the MMAs of the other.
-  __shared__ __align__(8) uint64_t sf_ready[2 * kQStages], sf_free[2];
+  // Scale copies and MMAs run from different threads.  Scale unit u (counted over the whole kernel) uses
+  // TMEM slot u % kUnitRing: sf_ready[slot] = its scales are in TMEM, sf_free[slot] = the MMAs that read it
+  // are done, so the copies run up to kUnitRing - 1 units ahead of the MMAs.
+  __shared__ __align__(8) uint64_t sf_ready[kUnitRing], sf_free[kUnitRing];
   __shared__ uint32_t tmem_holder;
   __shared__ int32_t tile_start[kMaxGroups + 1], grp_rows[kMaxGroups], grp_row0[kMaxGroups];
   __shared__ float xbuf[GATED ? 128 * 17 : 1];
@@ -724,13 +728,14 @@ __global__ void __launch_bounds__(kQThreads, 1)
     for (int s = 0; s < kQStages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
-      mbar_init(&sf_ready[s], 1);
-      mbar_init(&sf_ready[kQStages + s], 1);
+    }
+    for (int r = 0; r < kUnitRing; ++r) {
+      mbar_init(&sf_ready[r], 1);
+      mbar_init(&sf_free[r], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
       mbar_init(&tempty_bar[a], 8);
-      mbar_init(&sf_free[a], 1);
     }
     fence_mbar_init();
   }
@@ -811,7 +816,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
-      int g = 0;   // stages consumed so far (the scale set of stage g is g % 2)
+      int u = 0;   // scale units consumed so far
       for (int t = pair; t < total && ok; t += npairs, ++it) {
         const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, kQN);
         const int ntile = quad_tile_n(min(kQN, ti.rows - ti.n * kQN));
@@ -821,28 +826,29 @@ __global__ void __launch_bounds__(kQThreads, 1)
         if (!mbar_wait_cl(&tempty_bar[ab], aphase ^ 1u)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + ab * kQN;
-        for (int kb = 0; kb < KB; ++kb, ++g) {
+        for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_cl(&full_bar[stage], phase)) { ok = false; break; }
           const uint32_t sa = smem_u32(a_tile(stage)), sb = smem_u32(b_tile(stage));
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            if (!mbar_wait_cl(&sf_ready[h * kQStages + stage], phase)) { ok = false; break; }
+          for (int j = 0; j < Q::kUnits; ++j, ++u) {
+            const int slot = u % kUnitRing;
+            if (!mbar_wait_cl(&sf_ready[slot], static_cast<uint32_t>(u / kUnitRing) & 1u)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t sf = tmem_base + kQSfCol + h * kQSfHalfCols;
+            const uint32_t sf = tmem_base + kQSfCol + kUnitCols * slot;
+            if constexpr (MX) {
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const int kk = 2 * h + j;
-              const uint64_t ad = smem_desc_sw128(sa + kk * 32), bd = smem_desc_sw128(sb + kk * 32);
-              const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
-              if constexpr (MX) {
-                const uint32_t sf_id = 2u * j;             // both K steps of a half share one chunk
-                umma2_mxf4(d, ad, bd, idesc | (sf_id << 29) | (sf_id << 4), sf_addr(sf, sf_id),
-                           sf_addr(sf + 4, sf_id), acc);
-              } else {
-                umma2_nvf4(d, ad, bd, idesc, sf + 4 * j, sf + 8 + 8 * j, acc);
+              for (int jj = 0; jj < 2; ++jj) {                 // the unit's two K steps
+                const int kk = 2 * j + jj;
+                const uint32_t sf_id = 2u * jj;
+                umma2_mxf4(d, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32),
+                           idesc | (sf_id << 29) | (sf_id << 4), sf_addr(sf, sf_id), sf_addr(sf + 4, sf_id),
+                           (kb | kk) != 0 ? 1u : 0u);
               }
+            } else {
+              umma2_nvf4(d, smem_desc_sw128(sa + j * 32), smem_desc_sw128(sb + j * 32), idesc, sf, sf + 4,
+                         (kb | j) != 0 ? 1u : 0u);
             }
-            umma2_commit_local(&sf_free[h]);
+            umma2_commit_local(&sf_free[slot]);
           }
           if (!ok) break;
           umma2_commit_both(&empty_bar[stage]);
@@ -858,31 +864,23 @@ __global__ void __launch_bounds__(kQThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int g = 0;
+      int u = 0;   // scale units copied so far
       for (int t = pair; t < total && ok; t += npairs) {
-        for (int kb = 0; kb < KB; ++kb, ++g) {
+        for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_cl(&full_bar[stage], phase)) { ok = false; break; }
           const uint32_t ssa = smem_u32(sfa_tile(stage)), ssb = smem_u32(sfb_tile(stage));
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            // slot h is free once the MMAs of the previous stage's half h are done
-            if (g >= 1 && !mbar_wait_cl(&sf_free[h], static_cast<uint32_t>(g - 1) & 1u)) { ok = false; break; }
+          for (int j = 0; j < Q::kUnits; ++j, ++u) {
+            // the slot is free once the MMAs of the unit kUnitRing earlier are done
+            const int slot = u % kUnitRing;
+            if (u >= kUnitRing &&
+                !mbar_wait_cl(&sf_free[slot], static_cast<uint32_t>(u / kUnitRing - 1) & 1u)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t sf = tmem_base + kQSfCol + h * kQSfHalfCols;
-            if constexpr (MX) {       // one chunk holds both K steps of the half
-              tmem_cp_sf2(sf, smem_desc_sf(ssa + h * kSfChunk));
-              tmem_cp_sf2(sf + 4, smem_desc_sf(ssb + h * kSfChunk));
-              tmem_cp_sf2(sf + 8, smem_desc_sf(ssb + Q::kSfa + h * kSfChunk));
-            } else {
-#pragma unroll
-              for (int j = 0; j < 2; ++j) {
-                const int kk = 2 * h + j;
-                tmem_cp_sf2(sf + 4 * j, smem_desc_sf(ssa + kk * kSfChunk));
-                tmem_cp_sf2(sf + 8 + 8 * j, smem_desc_sf(ssb + kk * kSfChunk));
-                tmem_cp_sf2(sf + 8 + 8 * j + 4, smem_desc_sf(ssb + Q::kSfa + kk * kSfChunk));
-              }
-            }
-            umma2_commit_local(&sf_ready[h * kQStages + stage]);
+            const uint32_t sf = tmem_base + kQSfCol + kUnitCols * slot;
+            tmem_cp_sf2(sf, smem_desc_sf(ssa + j * kSfChunk));                  // weight rows of this CTA
+            tmem_cp_sf2(sf + 4, smem_desc_sf(ssb + j * kSfChunk));              // tokens 0-127 of the block
+            tmem_cp_sf2(sf + 8, smem_desc_sf(ssb + Q::kSfa + j * kSfChunk));    // tokens 128-223
+            umma2_commit_local(&sf_ready[slot]);
           }
           if (!ok) break;
           if (++stage == kQStages) { stage = 0; phase ^= 1u; }
