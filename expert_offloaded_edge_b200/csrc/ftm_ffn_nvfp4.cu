@@ -630,22 +630,25 @@ constexpr int kQThreads = 224;                  // warps 0 TMA, 1 MMA, 2-5 epilo
 
 // Stage layout of the pair kernel per scale format: A tile | B tile | the
 // stage's scale chunks of this CTA's 128 weight rows | of the token block's
-// two 128-row halves.  In TMEM the scales travel in units of one chunk per
-// operand: 4 columns of weight scales + 2 x 4 of token scales (the block's two
-// 128-row halves), 12 columns per unit.  A unit serves one K step (NVFP4) or
-// two (MXFP4, through scale-factor ids 0 and 2); units cycle through a ring
-// of kUnitRing slots so the copies can run several units ahead of the MMAs.
-constexpr uint32_t kUnitCols = 12;
-constexpr int kUnitRing = 5;
-static_assert(kQSfCol + kUnitRing * kUnitCols <= 512, "TMEM budget");
-
+// two 128-row halves.  In TMEM a chunk per operand takes 12 columns: 4 of
+// weight scales + 2 x 4 of token scales.  The scales travel in units of two K
+// steps, 24 columns for NVFP4 (a chunk per K step) and 12 for MXFP4 (one chunk
+// read through scale-factor ids 0 and 2), cycling through a ring of kRing unit
+// slots in the columns left after the accumulators, so the copies of a unit
+// overlap the MMAs of the ones before.
 template <bool MX>
 struct Q2Fmt {
   static constexpr uint32_t kSfa = F4Fmt<MX>::kSfStage;
   static constexpr uint32_t kSfb = 2 * F4Fmt<MX>::kSfStage;
   static constexpr uint32_t kStage = kQABytes + kQBBytes + kSfa + kSfb;
-  static constexpr int kUnits = F4Fmt<MX>::kChunks;     // scale units per stage
+  static constexpr int kUnitK = MX ? 4 : 2;               // K steps per scale unit
+  static constexpr int kUnits = 4 / kUnitK;               // scale units per stage (4 K steps)
+  static constexpr int kUnitChunks = MX ? kUnitK / 2 : kUnitK;
+  static constexpr uint32_t kUnitCols = 12 * kUnitChunks;
+  static constexpr uint32_t kRing = (512 - kQSfCol) / kUnitCols < 5 ? (512 - kQSfCol) / kUnitCols : 5;
+  static_assert(kRing >= 2, "scale copies overlap MMAs");
   static_assert(kStage % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled tiles");
+  static_assert(kQSfCol + kRing * kUnitCols <= 512, "TMEM budget");
 };
 
 __device__ __forceinline__ int quad_tile_n(int valid) { return min(kQN, (valid + 31) & ~31); }
@@ -704,9 +707,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kQStages], empty_bar[kQStages], tfull_bar[2], tempty_bar[2];
   // Scale copies and MMAs run from different threads.  Scale unit u (counted over the whole kernel) uses
-  // TMEM slot u % kUnitRing: sf_ready[slot] = its scales are in TMEM, sf_free[slot] = the MMAs that read it
-  // are done, so the copies run up to kUnitRing - 1 units ahead of the MMAs.
-  __shared__ __align__(8) uint64_t sf_ready[kUnitRing], sf_free[kUnitRing];
+  // TMEM slot u % kRing.  sf_ready[stage * kUnits + j] = unit j of the stage in that smem slot is in TMEM
+  // (one barrier per stage slot and unit, so a barrier is reused only once per trip round the stages);
+  // sf_free[slot] = the MMAs that read the TMEM slot are done.  The copies run up to kRing - 1 units ahead.
+  __shared__ __align__(8) uint64_t sf_ready[kQStages * Q::kUnits], sf_free[Q::kRing];
   __shared__ uint32_t tmem_holder;
   __shared__ int32_t tile_start[kMaxGroups + 1], grp_rows[kMaxGroups], grp_row0[kMaxGroups];
   __shared__ float xbuf[GATED ? 128 * 17 : 1];
@@ -729,10 +733,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    for (int r = 0; r < kUnitRing; ++r) {
-      mbar_init(&sf_ready[r], 1);
-      mbar_init(&sf_free[r], 1);
-    }
+    for (int r = 0; r < kQStages * Q::kUnits; ++r) mbar_init(&sf_ready[r], 1);
+    for (int r = 0; r < Q::kRing; ++r) mbar_init(&sf_free[r], 1);
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
       mbar_init(&tempty_bar[a], 8);
@@ -816,7 +818,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
-      int u = 0;   // scale units consumed so far
+      uint32_t u = 0;   // scale units consumed so far (unsigned: the ring index is a mask or a shift)
       for (int t = pair; t < total && ok; t += npairs, ++it) {
         const TileInfo ti = decode_tile(t, tile_start, grp_rows, grp_row0, G, kQN);
         const int ntile = quad_tile_n(min(kQN, ti.rows - ti.n * kQN));
@@ -831,22 +833,24 @@ __global__ void __launch_bounds__(kQThreads, 1)
           const uint32_t sa = smem_u32(a_tile(stage)), sb = smem_u32(b_tile(stage));
 #pragma unroll
           for (int j = 0; j < Q::kUnits; ++j, ++u) {
-            const int slot = u % kUnitRing;
-            if (!mbar_wait_cl(&sf_ready[slot], static_cast<uint32_t>(u / kUnitRing) & 1u)) { ok = false; break; }
+            const uint32_t slot = u % Q::kRing;
+            if (!mbar_wait_cl(&sf_ready[stage * Q::kUnits + j], phase)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t sf = tmem_base + kQSfCol + kUnitCols * slot;
-            if constexpr (MX) {
+            const uint32_t sf = tmem_base + kQSfCol + Q::kUnitCols * slot;
 #pragma unroll
-              for (int jj = 0; jj < 2; ++jj) {                 // the unit's two K steps
-                const int kk = 2 * j + jj;
-                const uint32_t sf_id = 2u * jj;
-                umma2_mxf4(d, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32),
-                           idesc | (sf_id << 29) | (sf_id << 4), sf_addr(sf, sf_id), sf_addr(sf + 4, sf_id),
-                           (kb | kk) != 0 ? 1u : 0u);
+            for (int jj = 0; jj < Q::kUnitK; ++jj) {          // the unit's K steps
+              const int kk = Q::kUnitK * j + jj;
+              const uint64_t ad = smem_desc_sw128(sa + kk * 32), bd = smem_desc_sw128(sb + kk * 32);
+              const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+              const uint32_t c = MX ? jj / 2 : jj;                 // the K step's chunk within the unit
+              const uint32_t sfa = sf + 4 * c, sfb = sf + 4 * Q::kUnitChunks + 8 * c;
+              if constexpr (MX) {                                   // bytes 0-1 or 2-3 of the chunk's columns
+                const uint32_t sf_id = 2u * (jj & 1);
+                umma2_mxf4(d, ad, bd, idesc | (sf_id << 29) | (sf_id << 4), sf_addr(sfa, sf_id),
+                           sf_addr(sfb, sf_id), acc);
+              } else {
+                umma2_nvf4(d, ad, bd, idesc, sfa, sfb, acc);
               }
-            } else {
-              umma2_nvf4(d, smem_desc_sw128(sa + j * 32), smem_desc_sw128(sb + j * 32), idesc, sf, sf + 4,
-                         (kb | j) != 0 ? 1u : 0u);
             }
             umma2_commit_local(&sf_free[slot]);
           }
@@ -864,23 +868,26 @@ __global__ void __launch_bounds__(kQThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int u = 0;   // scale units copied so far
+      uint32_t u = 0;   // scale units copied so far
       for (int t = pair; t < total && ok; t += npairs) {
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_cl(&full_bar[stage], phase)) { ok = false; break; }
           const uint32_t ssa = smem_u32(sfa_tile(stage)), ssb = smem_u32(sfb_tile(stage));
 #pragma unroll
           for (int j = 0; j < Q::kUnits; ++j, ++u) {
-            // the slot is free once the MMAs of the unit kUnitRing earlier are done
-            const int slot = u % kUnitRing;
-            if (u >= kUnitRing &&
-                !mbar_wait_cl(&sf_free[slot], static_cast<uint32_t>(u / kUnitRing - 1) & 1u)) { ok = false; break; }
+            // the slot is free once the MMAs of the unit kRing earlier are done
+            const uint32_t slot = u % Q::kRing;
+            if (u >= Q::kRing && !mbar_wait_cl(&sf_free[slot], (u / Q::kRing - 1) & 1u)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t sf = tmem_base + kQSfCol + kUnitCols * slot;
-            tmem_cp_sf2(sf, smem_desc_sf(ssa + j * kSfChunk));                  // weight rows of this CTA
-            tmem_cp_sf2(sf + 4, smem_desc_sf(ssb + j * kSfChunk));              // tokens 0-127 of the block
-            tmem_cp_sf2(sf + 8, smem_desc_sf(ssb + Q::kSfa + j * kSfChunk));    // tokens 128-223
-            umma2_commit_local(&sf_ready[slot]);
+            const uint32_t sf = tmem_base + kQSfCol + Q::kUnitCols * slot;
+#pragma unroll
+            for (int c = 0; c < Q::kUnitChunks; ++c) {   // NVFP4 one chunk per K step, MXFP4 one per two
+              const uint32_t off = (j * Q::kUnitChunks + c) * kSfChunk;
+              tmem_cp_sf2(sf + 4 * c, smem_desc_sf(ssa + off));                          // this CTA's weight rows
+              tmem_cp_sf2(sf + 4 * Q::kUnitChunks + 8 * c, smem_desc_sf(ssb + off));     // tokens 0-127
+              tmem_cp_sf2(sf + 4 * Q::kUnitChunks + 8 * c + 4, smem_desc_sf(ssb + Q::kSfa + off));  // 128-223
+            }
+            umma2_commit_local(&sf_ready[stage * Q::kUnits + j]);
           }
           if (!ok) break;
           if (++stage == kQStages) { stage = 0; phase ^= 1u; }
