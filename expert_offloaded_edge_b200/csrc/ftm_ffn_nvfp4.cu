@@ -715,6 +715,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
   __shared__ int32_t tile_start[kMaxGroups + 1], grp_rows[kMaxGroups], grp_row0[kMaxGroups];
   __shared__ float xbuf[GATED ? 128 * 17 : 1];
   __shared__ float tbuf[GATED ? 32 * 68 : 1];
+  constexpr int kYPitch = 40;   // bf16 per staging row: 32 columns + 16 bytes, rows stay 16-byte aligned
+  __shared__ __align__(16) uint16_t ybuf[GATED ? 8 : 4 * 32 * kYPitch];
 
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (smem_base - smem_u32(smem_raw));
@@ -949,20 +951,31 @@ __global__ void __launch_bounds__(kQThreads, 1)
                             out_sf, static_cast<size_t>(blk * 2 + tr / 128), tr % 128, pb, grp, Nw);
         }
       } else {
+        // lane = output column, TMEM column = token: 32 tokens at a time go through the warp's staging
+        // rows so that each store is 16 bytes of one token's row
         const float s_a = MX ? 1.f : st[st_idx] * (act_scale ? act_scale[1] : 1.f);
-        const int wrow = ti.m * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
-        uint16_t* o = out_bf16 + static_cast<size_t>(ti.row0 + ti.n * kQN) * Nw + wrow;
-        for (int c0 = 0; c0 < valid; c0 += 16) {
-          float a[16];
+        const int w0 = ti.m * 256 + static_cast<int>(rank) * 128 + q * 32;
+        uint16_t* o = out_bf16 + static_cast<size_t>(ti.row0 + ti.n * kQN) * Nw + w0;
+        uint16_t* yb = ybuf + (warp - 2) * (32 * kYPitch);
+        for (int c0 = 0; c0 < valid; c0 += 32) {
+          float a[32];
           tmem_ld16(tb + c0, a);
+          tmem_ld16(tb + c0 + 16, a + 16);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (c0 + j < valid) {
-              const __nv_bfloat16 hb = __float2bfloat16_rn(a[j] * s_a);
-              o[static_cast<size_t>(c0 + j) * Nw] = *reinterpret_cast<const uint16_t*>(&hb);
-            }
+          for (int j = 0; j < 32; ++j) {
+            const __nv_bfloat16 hb = __float2bfloat16_rn(a[j] * s_a);
+            yb[j * kYPitch + lane] = *reinterpret_cast<const uint16_t*>(&hb);
           }
+          __syncwarp();
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int j = r * 8 + lane / 4, part = lane % 4;
+            if (c0 + j < valid)
+              *reinterpret_cast<uint4*>(o + static_cast<size_t>(c0 + j) * Nw + part * 8) =
+                  *reinterpret_cast<const uint4*>(yb + j * kYPitch + part * 8);
+          }
+          __syncwarp();
         }
       }
       tc_fence_before();

@@ -60,6 +60,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ int32_t tile_start[kMaxGroups + 1], grp_rows[kMaxGroups], grp_row0[kMaxGroups];
   // half-chunks crossing between the gate and up warps, double-buffered
   __shared__ float xbuf[GATED ? 2 * 128 * 17 : 1];
+  constexpr int kYPitch = 40;   // bf16 per staging row: 32 columns + 16 bytes, rows stay 16-byte aligned
+  __shared__ __align__(16) uint16_t ybuf[GATED ? 8 : 4 * 32 * kYPitch];
 
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (smem_base - smem_u32(smem_raw));
@@ -214,19 +216,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       } else {
-        const int wrow = ti.m * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
-        uint16_t* o = out + rowbase * ld_out + wrow;
-        for (int c0 = 0; c0 < valid; c0 += 16) {
-          float v[16];
+        // lane = output column, TMEM column = token: 32 tokens at a time go through the warp's staging
+        // rows so that each store is 16 bytes of one token's row
+        const int w0 = ti.m * 256 + static_cast<int>(rank) * 128 + q * 32;
+        uint16_t* o = out + rowbase * ld_out + w0;
+        uint16_t* yb = ybuf + (warp - 2) * (32 * kYPitch);
+        for (int c0 = 0; c0 < valid; c0 += 32) {
+          float v[32];
           tmem_ld16(tb + c0, v);
+          tmem_ld16(tb + c0 + 16, v + 16);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (c0 + j < valid) {
-              const __nv_bfloat16 hb = __float2bfloat16_rn(v[j]);
-              o[static_cast<size_t>(c0 + j) * ld_out] = *reinterpret_cast<const uint16_t*>(&hb);
-            }
+          for (int j = 0; j < 32; ++j) {
+            const __nv_bfloat16 hb = __float2bfloat16_rn(v[j]);
+            yb[j * kYPitch + lane] = *reinterpret_cast<const uint16_t*>(&hb);
           }
+          __syncwarp();
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int j = r * 8 + lane / 4, part = lane % 4;
+            if (c0 + j < valid)
+              *reinterpret_cast<uint4*>(o + static_cast<size_t>(c0 + j) * ld_out + part * 8) =
+                  *reinterpret_cast<const uint4*>(yb + j * kYPitch + part * 8);
+          }
+          __syncwarp();
         }
       }
       tc_fence_before();
