@@ -7,9 +7,9 @@
 // persistent CTA walks 128-token tiles: warp 0 streams x and Wr tiles with
 // TMA, warp 1 issues the MMAs into a double-buffered accumulator, and each of
 // the four epilogue warps owns 32 tokens: thread i reads its token's E logits
-// from TMEM lane i, 16 columns at a time, adds the bias and keeps the top k in
-// registers by insertion (experts visited in ascending id, so equal logits
-// keep the lower id first), then writes the softmax over the k picks.  No
+// from TMEM lane i (32 columns per wait), adds the bias and selects the top k
+// (one scan with register insertion for k = 2, 4, 6, 8; k passes otherwise),
+// then writes the softmax over the k picks.  The picks live in registers; no
 // shared-memory staging of logits, no global scratch, one launch.
 #include "ftm_gemm.cuh"
 
@@ -24,6 +24,105 @@ constexpr uint32_t kRtXBytes = kRtBM * 128;          // 128 tokens x 64 bf16
 constexpr uint32_t kRtWBytes = kRtMaxNE * 128;       // up to 256 router rows x 64 bf16
 constexpr uint32_t kRtStage = kRtXBytes + kRtWBytes;
 constexpr uint32_t kRtTmemCols = 2 * kRtMaxNE;       // two accumulators of up to 256 columns
+
+// Gates of one token from its top k (pv descending, pi ids): softmax over the
+// k picks, written at row tok.
+template <int NK>
+__device__ __forceinline__ void write_gates(const float (&pv)[NK], const int (&pi)[NK], int k, int tok, int T,
+                                            int32_t* __restrict__ topk_ids, float* __restrict__ topk_w) {
+  if (tok >= T) return;
+  float ex[NK];
+  float sum = 0.f;
+#pragma unroll
+  for (int j = 0; j < NK; ++j) {
+    ex[j] = j < k ? expf(pv[j] - pv[0]) : 0.f;
+    sum += ex[j];
+  }
+#pragma unroll
+  for (int j = 0; j < NK; ++j) {
+    if (j < k) {
+      topk_ids[static_cast<size_t>(tok) * k + j] = pi[j];
+      topk_w[static_cast<size_t>(tok) * k + j] = ex[j] / sum;
+    }
+  }
+}
+
+// Route one token (the TMEM lane of the calling thread holds its logits in
+// columns [0, NE), read 32 per wait) for a k known at compile time: one scan
+// with insertion into a sorted register list.  Experts are visited in
+// ascending id and an entry moves only for a strictly larger logit, so equal
+// logits keep the lower id first; NaN and -inf logits never enter.
+template <int K>
+__device__ __forceinline__ void route_token_k(uint32_t tb, int NE, int E, const float* s_bias, int tok, int T,
+                                              int32_t* __restrict__ topk_ids, float* __restrict__ topk_w) {
+  float pv[K];
+  int pi[K];
+#pragma unroll
+  for (int j = 0; j < K; ++j) { pv[j] = -INFINITY; pi[j] = 0x7FFFFFFF; }
+  for (int c0 = 0; c0 < NE; c0 += 32) {
+    float v[32];
+    tmem_ld16(tb + c0, v);
+    if (c0 + 16 < NE) tmem_ld16(tb + c0 + 16, v + 16);
+    tmem_ld_wait();
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj) {
+      const int e = c0 + jj;
+      const float val = v[jj] + s_bias[e < kRtMaxNE ? e : 0];
+      if (e < E && val > pv[K - 1]) {
+        // position j takes the old entry j-1 if val is above it, else val if val is above the old entry j
+#pragma unroll
+        for (int j = K - 1; j >= 0; --j) {
+          if (j > 0 && val > pv[j - 1]) {
+            pv[j] = pv[j - 1];
+            pi[j] = pi[j - 1];
+          } else if (val > pv[j]) {
+            pv[j] = val;
+            pi[j] = e;
+          }
+        }
+      }
+    }
+  }
+  write_gates<K>(pv, pi, K, tok, T, topk_ids, topk_w);
+}
+
+// Any k <= 16: k passes, each taking the largest logit (then lowest id) below
+// the previous pick.  Same order and exclusions as route_token_k.
+__device__ __forceinline__ void route_token_any(uint32_t tb, int NE, int E, int k, const float* s_bias, int tok,
+                                                int T, int32_t* __restrict__ topk_ids, float* __restrict__ topk_w) {
+  float pv[kRtMaxK];
+  int pi[kRtMaxK];
+  float prev_v = INFINITY;
+  int prev_e = -1;
+#pragma unroll
+  for (int p = 0; p < kRtMaxK; ++p) {
+    float bv = -INFINITY;
+    int be = 0x7FFFFFFF;
+    if (p < k) {
+      for (int c0 = 0; c0 < NE; c0 += 32) {
+        float v[32];
+        tmem_ld16(tb + c0, v);
+        if (c0 + 16 < NE) tmem_ld16(tb + c0 + 16, v + 16);
+        tmem_ld_wait();
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const int e = c0 + jj;
+          const float val = v[jj] + s_bias[e < kRtMaxNE ? e : 0];
+          const bool below = val < prev_v || (val == prev_v && e > prev_e);
+          if (e < E && below && val > bv) {
+            bv = val;
+            be = e;
+          }
+        }
+      }
+    }
+    pv[p] = bv;
+    pi[p] = be;
+    prev_v = bv;
+    prev_e = be;
+  }
+  write_gates<kRtMaxK>(pv, pi, k, tok, T, topk_ids, topk_w);
+}
 
 __global__ void __launch_bounds__(kTcThreads, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, int T, int d,
@@ -117,58 +216,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!epilogue_all(mbar_wait(&tfull_bar[ab], aphase))) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * kRtMaxNE;
-      float pv[kRtMaxK];
-      int pi[kRtMaxK];
-#pragma unroll
-      for (int j = 0; j < kRtMaxK; ++j) { pv[j] = -INFINITY; pi[j] = 0x7FFFFFFF; }
-      float kth = -INFINITY;                      // pv[k - 1], kept in a register
-      for (int c0 = 0; c0 < NE; c0 += 16) {
-        float v[16];
-        tmem_ld16(tb + c0, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int e = c0 + jj;
-          const float val = v[jj] + s_bias[e];
-          if (e >= E || !(val > kth)) continue;  // not among the top k so far (ties keep the lower id)
-#pragma unroll
-          for (int j = kRtMaxK - 1; j >= 0; --j) {   // insertion, from the end
-            if (j >= k) continue;
-            if (val > pv[j]) {
-              if (j > 0 && val > pv[j - 1]) {
-                pv[j] = pv[j - 1];
-                pi[j] = pi[j - 1];
-              } else {
-                pv[j] = val;
-                pi[j] = e;
-              }
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < kRtMaxK; ++j)
-            if (j == k - 1) kth = pv[j];
-        }
+      const int tok = t * kRtBM + q * 32 + lane;
+      switch (k) {
+        case 8: route_token_k<8>(tb, NE, E, s_bias, tok, T, topk_ids, topk_w); break;
+        case 6: route_token_k<6>(tb, NE, E, s_bias, tok, T, topk_ids, topk_w); break;
+        case 4: route_token_k<4>(tb, NE, E, s_bias, tok, T, topk_ids, topk_w); break;
+        case 2: route_token_k<2>(tb, NE, E, s_bias, tok, T, topk_ids, topk_w); break;
+        default: route_token_any(tb, NE, E, k, s_bias, tok, T, topk_ids, topk_w); break;
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty_bar[ab]);
-      const int tok = t * kRtBM + q * 32 + lane;
-      if (tok < T) {
-        float ex[kRtMaxK];
-        float sum = 0.f;
-#pragma unroll
-        for (int j = 0; j < kRtMaxK; ++j) {
-          ex[j] = j < k ? expf(pv[j] - pv[0]) : 0.f;
-          sum += ex[j];
-        }
-#pragma unroll
-        for (int j = 0; j < kRtMaxK; ++j) {
-          if (j < k) {
-            topk_ids[static_cast<size_t>(tok) * k + j] = pi[j];
-            topk_w[static_cast<size_t>(tok) * k + j] = ex[j] / sum;
-          }
-        }
-      }
     }
   }
   tc_fence_before();

@@ -38,13 +38,39 @@ def test_route_configs(name, T):
                                         # MMA N side padded to 16 (N = 48 .. 256), ragged last tiles, k = 16
                                         (37, 3, 128, 2049, "bf16"), (120, 4, 256, 2100, "bf16"),
                                         (200, 6, 128, 2500, "bf16"), (256, 16, 256, 3000, "bf16"),
-                                        (128, 8, 256, 10000, "bf16"), (160, 8, 256, 9601, "bf16")])
+                                        (128, 8, 256, 10000, "bf16"), (160, 8, 256, 9601, "bf16"),
+                                        (64, 2, 128, 2048, "bf16"), (96, 1, 128, 2100, "bf16")])
 def test_route_shapes(E, k, d, T, dt):
     cfg = synth.LayerConfig("route_case", d=d, E=E, k=k, I=128, wdtype=dt, has_shared=0, S=E, bias="uniform", T=(T,))
     ids, gw, rid, rg = _route_case(cfg, T)
     assert np.array_equal(ids, rid)
     assert np.allclose(gw, rg, rtol=gate_rtol(d), atol=1e-6)
     assert np.allclose(gw.sum(1), 1.0, atol=1e-5)
+
+
+@pytest.mark.parametrize("k", [1, 2, 5, 8, 16])
+def test_route_tc_ties(k):
+    """Tensor-core router on exact ties: zero tokens make every logit its bias, which repeats in threes, so
+    each pick list must order equal logits by ascending expert id like the oracle; the other tokens are
+    random.  k = 2 and 8 take the single-scan selection, 1, 5 and 16 the pass-based one."""
+    T, E, d = 2048, 64, 128
+    rng = np.random.default_rng(40 + k)
+    x = rng.standard_normal((T, d)).astype(np.float32)
+    x[: T // 2] = 0.0
+    wr = (0.02 * rng.standard_normal((E, d))).astype(np.float32)
+    bias = np.ascontiguousarray(0.5 * ((E - 1 - np.arange(E)) // 3), dtype=np.float32)   # 0 alone, then threes
+    xb = torch.from_numpy(x).to(torch.bfloat16).cuda()
+    wb = torch.from_numpy(wr).to(torch.bfloat16).cuda()
+    cfg = synth.LayerConfig("route_ties", d=d, E=E, k=k, I=128, wdtype="bf16", has_shared=0, S=E, bias="uniform",
+                            T=(T,))
+    ids = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    gw = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    ftm.ftm_route(ftm.desc_for(cfg), xb, T, wb, torch.from_numpy(bias).cuda(), ids, gw)
+    torch.cuda.synchronize()
+    rid, rg, _ = oracle.route(xb.float().cpu().numpy(), wb.float().cpu().numpy(), bias, k)
+    assert np.array_equal(ids.cpu().numpy()[: T // 2], rid[: T // 2])
+    assert (ids.cpu().numpy()[: T // 2, 0] == 0).all()
+    assert np.allclose(gw.cpu().numpy(), rg, rtol=gate_rtol(d), atol=1e-6)
 
 
 @pytest.mark.parametrize("T,k,E", [(1, 1, 1), (5, 2, 8), (64, 8, 128), (37, 3, 300), (600, 8, 128),
