@@ -517,6 +517,20 @@ def run_resident(dl, T, args, dist, local):
     return rec
 
 
+def latency_floor(cfg, args, dist, local):
+    """The same kernel chain as a T = 1 decode step of cfg, on a layer with
+    d = I = 256 (about 3 MB of weights touched): the step time left when the
+    bytes are negligible, i.e. the launch and dependency latency of the chain."""
+    fcfg = synth.scaled(cfg, name=cfg.name + "_floor", d=256, I=256)
+    dl = device_layer(fcfg, args, local, dist)
+    rec = run_resident(dl, 1, args, dist, local)
+    del dl
+    return {"workload": f"latency floor: the {cfg.name} T=1 kernel chain at d = I = 256",
+            "ms_per_step": rec["ms_per_step"], "steps": rec["steps"], "launch": rec["launch"],
+            "launches_per_step": rec["launches_per_step"], "kernels_ms_breakdown": rec["kernels_ms_breakdown"],
+            "clocks": rec["clocks"], "device_status": rec["device_status"]}
+
+
 def run_trace(cfg, T, args, dist, local):
     """The decode trace over the LRU slot cache: one step = route, permute, cache
     update with miss copies (host sync), FFN, combine.  Warm-up = the first W
@@ -845,6 +859,8 @@ def main():
             for T in Ts:
                 records.append(run_trace(cfg, T, args, dist, local))
             continue
+        if name == "35b_decode":
+            records.append(latency_floor(cfg, args, dist, local))
         dl = device_layer(cfg, args, local, dist, cache=name == head[0])
         for T in Ts:
             try:
