@@ -1,22 +1,24 @@
 // Weighted un-permute and combine (step a8):
 //   out[t] = sum_{j ascending} g[t][j] * y[inv[t*k + j]]  (+ y[P + t] for the shared expert)
-// fp32 accumulation, fixed summation order (deterministic).  One warp per
-// token (grid-strided), 16-byte loads and stores along d.
+// fp32 accumulation, fixed summation order (deterministic).  A warp takes one
+// item at a time (grid-strided): a whole token for large batches, one
+// 32-vector slice of d for small ones, so even a single token spreads over
+// d / 256 (bf16) warps; 16-byte loads and stores.
 #include "ftm_common.cuh"
 
 namespace ftm {
 
 constexpr int kMaxTerms = 17;   // k <= 16 routed picks + the shared expert
 
-// One warp per token: lane j < k fetches the token's j-th row index and gate
-// (lane k: the shared expert's row, gate 1), the warp shares them by shuffles,
-// then every lane walks its 16-byte vectors of d, issuing all of the token's
-// row loads before the fused multiply-adds.  The terms are added in ascending
-// j, so the result does not depend on the schedule.
+// Per item: lane j < k fetches the token's j-th row index and gate (lane k:
+// the shared expert's row, gate 1) into the warp's shared-memory slots, then
+// each lane issues all of the token's row loads for its 16-byte vector before
+// the fused multiply-adds.  The terms are added in ascending j, so the result
+// does not depend on the schedule.
 template <bool F32>
 __global__ void __launch_bounds__(256, 2) combine_kernel(const void* __restrict__ y, const int32_t* __restrict__ inv,
                                                       const float* __restrict__ gw, int T, int k, int d, int P,
-                                                      int has_shared, void* __restrict__ out) {
+                                                      int has_shared, int spi, void* __restrict__ out) {
   constexpr int V = F32 ? 4 : 8;   // elements per 16-byte vector
   constexpr int EB = F32 ? 4 : 2;  // bytes per element
   const int nv = d / V;
@@ -27,7 +29,13 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(const void* __restrict_
   __shared__ float s_gs[8][kMaxTerms];
   pdl_wait();
   pdl_trigger();
-  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
+  const int nch = (nv + 31) / 32;                    // 32-vector slices of a row
+  const int ipt = (nch + spi - 1) / spi;             // items per token (spi slices each)
+  const long long items = static_cast<long long>(T) * ipt;
+  for (long long item = static_cast<long long>(blockIdx.x) * wpb + (threadIdx.x >> 5); item < items;
+       item += static_cast<long long>(gridDim.x) * wpb) {
+    const int t = static_cast<int>(item / ipt);
+    const int c0 = static_cast<int>(item % ipt) * spi * 32;
     int my_row = -1;
     float my_g = 0.f;
     if (lane < nterms) {
@@ -47,7 +55,7 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(const void* __restrict_
       gs[lane] = my_g;
     }
     __syncwarp();
-    for (int c = lane; c < nv; c += 32) {
+    for (int c = c0 + lane; c < nv && c < c0 + spi * 32; c += 32) {
       uint4 u[kMaxTerms];
 #pragma unroll
       for (int j = 0; j < kMaxTerms; ++j)
@@ -91,18 +99,25 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(const void* __restrict_
       *reinterpret_cast<uint4*>(static_cast<uint8_t*>(out) +
                                 (static_cast<size_t>(t) * d + static_cast<size_t>(c) * V) * EB) = o;
     }
-    __syncwarp();   // the warp's rows and gates are rewritten for its next token
+    __syncwarp();   // the warp's rows and gates are rewritten for its next item
   }
 }
 
 cudaError_t launch_combine(bool f32, const void* y, const int32_t* inv, const float* gw, int T, int k, int d, int P,
                            int has_shared, void* out, cudaStream_t st) {
-  const int blocks = (T + 7) / 8;   // 8 tokens (warps) per block
-  const int grid = blocks < 148 * 8 ? blocks : 148 * 8;
+  // a warp takes a whole token when the batch alone fills the GPU (its rows and gates are read once), else one
+  // 32-vector slice of d at a time so that a few tokens still spread over many warps
+  const int V = f32 ? 4 : 8;
+  const int nch = (d / V + 31) / 32;
+  const int spi = T >= 148 * 8 ? nch : 1;
+  const long long items = static_cast<long long>(T) * ((nch + spi - 1) / spi);
+  const long long blocks = (items + 7) / 8;   // 8 items (warps) per block
+  const int grid = static_cast<int>(blocks < 148 * 8 ? blocks : 148 * 8);
   if (f32)
-    return launch_pdl(combine_kernel<true>, dim3(grid), dim3(256), 0, st, y, inv, gw, T, k, d, P, has_shared, out);
+    return launch_pdl(combine_kernel<true>, dim3(grid), dim3(256), 0, st, y, inv, gw, T, k, d, P, has_shared, spi, out);
   else
-    return launch_pdl(combine_kernel<false>, dim3(grid), dim3(256), 0, st, y, inv, gw, T, k, d, P, has_shared, out);
+    return launch_pdl(combine_kernel<false>, dim3(grid), dim3(256), 0, st, y, inv, gw, T, k, d, P, has_shared, spi,
+                      out);
   return cudaGetLastError();
 }
 
