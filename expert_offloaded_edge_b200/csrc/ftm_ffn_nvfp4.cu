@@ -240,12 +240,13 @@ __global__ void __launch_bounds__(256) quant_tokens_f4_kernel(const uint16_t* __
 }
 
 // ---------------------------------------------------------------------------
-// Gather of the quantised tokens into the padded activation rows: one warp
-// per padded row copies its token's d/2 packed bytes (16-byte vectors) and
-// scatters its scale words (one per chunk of four groups: d/64 for NVFP4,
-// d/128 for MXFP4) into the row's place in the scale chunks (rows past a
-// group's end are zeros).  The padded group offsets sit in
-// shared memory; lane 0 finds the row's source token.
+// Gather of the quantised tokens into the padded activation rows.  Packed
+// codes: one warp per padded row copies its token's d/2 bytes (16-byte
+// vectors).  Scale words (one per chunk of four groups: d/64 for NVFP4, d/128
+// for MXFP4): one warp per 128-row chunk block and eight chunk columns, lane l
+// collecting the words of rows l, l+32, l+64 and l+96 (the 16 bytes it owns in
+// each 512-byte chunk), so every store is a full coalesced chunk (rows past a
+// group's end are zeros).  The padded group offsets sit in shared memory.
 // ---------------------------------------------------------------------------
 template <bool MX>
 __global__ void __launch_bounds__(256) gather_f4_kernel(const uint8_t* __restrict__ xq_tok,
@@ -265,18 +266,20 @@ __global__ void __launch_bounds__(256) gather_f4_kernel(const uint8_t* __restric
   const int nkc = d / F4Fmt<MX>::kChunkK, nvec = d / 32;    // scale words, 16-byte vectors per packed row
   const int nsub = (BN + 127) / 128;               // 128-row scale chunks per BN-row block
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nwarps = blockDim.x / 32;
+  // the source token of padded row pr, or -1 past its group's end
+  auto token_of = [&](int pr) -> int {
+    int lo = 0, hi = G;  // s_prow0[lo] <= pr < s_prow0[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_prow0[mid] <= pr) lo = mid; else hi = mid;
+    }
+    const int local = pr - s_prow0[lo];
+    const int rows = lo < E ? offsets[lo + 1] - offsets[lo] : T;
+    return local >= rows ? -1 : (lo < E ? perm[offsets[lo] + local] / k : local);
+  };
   for (int pr = blockIdx.x * nwarps + warp; pr < rows_pad; pr += gridDim.x * nwarps) {
     int src = -1;
-    if (lane == 0) {
-      int lo = 0, hi = G;  // s_prow0[lo] <= pr < s_prow0[hi]
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (s_prow0[mid] <= pr) lo = mid; else hi = mid;
-      }
-      const int local = pr - s_prow0[lo];
-      const int rows = lo < E ? offsets[lo + 1] - offsets[lo] : T;
-      src = local >= rows ? -1 : (lo < E ? perm[offsets[lo] + local] / k : local);
-    }
+    if (lane == 0) src = token_of(pr);
     src = __shfl_sync(0xffffffffu, src, 0);
     const uint4* s = reinterpret_cast<const uint4*>(xq_tok + static_cast<size_t>(src < 0 ? 0 : src) * (d / 2));
     uint4* dst = reinterpret_cast<uint4*>(xq + static_cast<size_t>(pr) * (d / 2));
@@ -293,11 +296,36 @@ __global__ void __launch_bounds__(256) gather_f4_kernel(const uint8_t* __restric
         if (c < nvec) dst[c] = v[u];
       }
     }
-    const int blk = pr / BN, r = pr % BN;
-    const uint32_t* sw = reinterpret_cast<const uint32_t*>(s_tok + static_cast<size_t>(src < 0 ? 0 : src) * (4 * nkc));
-    uint8_t* chunk0 = sfx + (static_cast<size_t>(blk) * nsub + r / 128) * nkc * kSfChunk + sf_byte(r % 128, 0);
-    for (int kb = lane; kb < nkc; kb += 32)
-      *reinterpret_cast<uint32_t*>(chunk0 + static_cast<size_t>(kb) * kSfChunk) = src >= 0 ? sw[kb] : 0u;
+  }
+  const uint32_t* sw = reinterpret_cast<const uint32_t*>(s_tok);
+  const int ncb = (rows_pad / BN) * nsub;             // 128-row chunk blocks
+  const int nkg = (nkc + 7) / 8;                       // groups of eight chunk columns
+  for (long long it = static_cast<long long>(blockIdx.x) * nwarps + warp; it < static_cast<long long>(ncb) * nkg;
+       it += static_cast<long long>(gridDim.x) * nwarps) {
+    const int cb = static_cast<int>(it / nkg), kg = static_cast<int>(it % nkg);
+    const int blk = cb / nsub, sub = cb % nsub;
+    int src[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int i = sub * 128 + lane + 32 * q;          // row within the BN-row block
+      src[q] = i < BN ? token_of(blk * BN + i) : -1;
+    }
+    uint4 w[8];
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const int kb = kg * 8 + kk;
+      uint32_t v[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        v[q] = (kb < nkc && src[q] >= 0) ? sw[static_cast<size_t>(src[q]) * nkc + kb] : 0u;
+      w[kk] = make_uint4(v[0], v[1], v[2], v[3]);
+    }
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const int kb = kg * 8 + kk;
+      if (kb < nkc)
+        *reinterpret_cast<uint4*>(sfx + (static_cast<size_t>(cb) * nkc + kb) * kSfChunk + lane * 16) = w[kk];
+    }
   }
 }
 
