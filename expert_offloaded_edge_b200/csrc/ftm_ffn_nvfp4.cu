@@ -24,6 +24,9 @@ namespace ftm {
 
 constexpr int kF4StageK = 256;         // K per stage: 128 bytes of packed e2m1 = one swizzle row
 constexpr uint32_t kSfChunk = 512;     // bytes of one scale chunk (128 rows x four scale groups)
+// NVFP4 CTA-pair gate/up: the token scales of one K step for a 224-row block, the chunk of rows 0-127 four
+// times then the chunk of rows 128-255 four times (the TMEM image of two 32x128b.warpx4 copies)
+constexpr uint32_t kRepChunkBytes = 4096;
 
 // The two block-scale formats of the e2m1 kernels.  NVFP4 (MX = false): one
 // e4m3 scale per 16 elements, a chunk covers K = 64, one MMA (K = 64) reads
@@ -254,8 +257,8 @@ __global__ void __launch_bounds__(256) gather_f4_kernel(const uint8_t* __restric
                                                           const int32_t* __restrict__ perm,
                                                           const int32_t* __restrict__ offsets,
                                                           const int32_t* __restrict__ prow0, int E, int has_shared,
-                                                          int T, int k, int d, int BN, uint8_t* __restrict__ xq,
-                                                          uint8_t* __restrict__ sfx) {
+                                                          int T, int k, int d, int BN, int replicate,
+                                                          uint8_t* __restrict__ xq, uint8_t* __restrict__ sfx) {
   __shared__ int32_t s_prow0[kMaxGroups + 1];
   pdl_wait();
   pdl_trigger();
@@ -323,8 +326,14 @@ __global__ void __launch_bounds__(256) gather_f4_kernel(const uint8_t* __restric
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
       const int kb = kg * 8 + kk;
-      if (kb < nkc)
+      if (kb >= nkc) continue;
+      if (replicate) {   // the K step's 4 KB block: [chunk of rows 0-127 x 4][chunk of rows 128-255 x 4]
+        uint8_t* b = sfx + (static_cast<size_t>(blk) * nkc + kb) * kRepChunkBytes + sub * 2048 + lane * 16;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) *reinterpret_cast<uint4*>(b + r * kSfChunk) = w[kk];
+      } else {
         *reinterpret_cast<uint4*>(sfx + (static_cast<size_t>(cb) * nkc + kb) * kSfChunk + lane * 16) = w[kk];
+      }
     }
   }
 }
@@ -336,9 +345,11 @@ __global__ void __launch_bounds__(256) gather_f4_kernel(const uint8_t* __restric
 // block rb, row rr of the chunk, Nw intermediate columns.  NVFP4: e4m3 scale
 // of amax / (6 gh) times gh.  MXFP4: the 32-group is this thread's 16 values
 // and those of lane ^ 1 (all 32 lanes must call); the even lane stores the
-// code.  Padding rows are quantised too (never read back).
+// code.  Padding rows are quantised too (never read back).  REP (NVFP4 on CTA
+// pairs): rb is the 224-row block and rr the row in it, and the scale goes to
+// the block's replicated layout (each 128-row chunk four times per K step).
 // ---------------------------------------------------------------------------
-template <bool MX>
+template <bool MX, bool REP = false>
 __device__ __forceinline__ void quant_store_h(const float (&h)[16], float gh, float six_gh, uint8_t* q_dst,
                                               uint8_t* out_sf, size_t rb, int rr, int mb, int grp, int Nw) {
   float amax = 0.f;
@@ -364,7 +375,13 @@ __device__ __forceinline__ void quant_store_h(const float (&h)[16], float gh, fl
         packed[i / 8] |= static_cast<uint32_t>(f32x2_to_e2m1x2(h[i + 1] / sc, h[i] / sc)) << (4 * (i % 8));
     }
     *reinterpret_cast<uint2*>(q_dst) = make_uint2(packed[0], packed[1]);
-    out_sf[(rb * (Nw / 64) + mb) * kSfChunk + sf_byte(rr, grp)] = sq;
+    if constexpr (REP) {
+      uint8_t* b = out_sf + (rb * (Nw / 64) + mb) * kRepChunkBytes + (rr / 128) * 2048 + sf_byte(rr % 128, grp);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) b[r * kSfChunk] = sq;
+    } else {
+      out_sf[(rb * (Nw / 64) + mb) * kSfChunk + sf_byte(rr, grp)] = sq;
+    }
   }
 }
 
@@ -664,10 +681,15 @@ constexpr int kQThreads = 224;                  // warps 0 TMA, 1 MMA, 2-5 epilo
 // read through scale-factor ids 0 and 2), cycling through a ring of kRing unit
 // slots in the columns left after the accumulators, so the copies of a unit
 // overlap the MMAs of the ones before.
-template <bool MX>
+template <bool MX, bool GATED>
 struct Q2Fmt {
+  // NVFP4: the token scales (x for gate/up, H for down) arrive replicated (per K step a 4 KB block holding
+  // each of the two 128-row chunks four times, the TMEM layout of the 32x128b.warpx4 copies), so one
+  // 128x256b copy moves a K step's token scales; four stages then fit shared memory instead of five
+  static constexpr bool kRep = !MX;
+  static constexpr int kStages = kRep ? 4 : kQStages;
   static constexpr uint32_t kSfa = F4Fmt<MX>::kSfStage;
-  static constexpr uint32_t kSfb = 2 * F4Fmt<MX>::kSfStage;
+  static constexpr uint32_t kSfb = kRep ? 4 * kRepChunkBytes : 2 * F4Fmt<MX>::kSfStage;
   static constexpr uint32_t kStage = kQABytes + kQBBytes + kSfa + kSfb;
   static constexpr int kUnitK = MX ? 4 : 2;               // K steps per scale unit
   static constexpr int kUnits = 4 / kUnitK;               // scale units per stage (4 K steps)
@@ -709,6 +731,24 @@ __device__ __forceinline__ void tmem_cp_sf2(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
+// Both CTAs of the pair: copy 128 rows of 32 bytes (8 columns) from this
+// offset of each CTA's shared memory into the same columns of its own TMEM.
+__device__ __forceinline__ void tmem_cp_wide2(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Descriptor of a replicated 4 KB token-scale block: no swizzle, 128 rows of
+// two 16-byte columns, the second column 2048 bytes after the first (leading
+// byte offset), 8-row groups 128 bytes apart (stride byte offset).
+__device__ __forceinline__ uint64_t smem_desc_rep(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(2048u >> 4) << 16;
+  d |= static_cast<uint64_t>(128u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;            // version; layout type 0: no swizzle
+  return d;
+}
+
 // Arrive on this CTA's barrier once the executing thread's pair operations complete.
 __device__ __forceinline__ void umma2_commit_local(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -728,17 +768,17 @@ __global__ void __launch_bounds__(kQThreads, 1)
                          const float* __restrict__ act_scale) {
   constexpr uint32_t kTmemCols = 512;
   constexpr int kRowsPerPair = GATED ? 128 : 256;   // output rows (intermediate / hidden) per pair tile
-  using Q = Q2Fmt<MX>;
+  using Q = Q2Fmt<MX, GATED>;
   constexpr int kCh = F4Fmt<MX>::kChunks;
   constexpr uint32_t kQStage = Q::kStage;
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[kQStages], empty_bar[kQStages], tfull_bar[2], tempty_bar[2];
+  __shared__ __align__(8) uint64_t full_bar[Q::kStages], empty_bar[Q::kStages], tfull_bar[2], tempty_bar[2];
   // Scale copies and MMAs run from different threads.  Scale unit u (counted over the whole kernel) uses
   // TMEM slot u % kRing.  sf_ready[stage * kUnits + j] = unit j of the stage in that smem slot is in TMEM
   // (one barrier per stage slot and unit, so a barrier is reused only once per trip round the stages);
   // sf_free[slot] = the MMAs that read the TMEM slot are done.  The copies run up to kRing - 1 units ahead.
-  __shared__ __align__(8) uint64_t sf_ready[kQStages * Q::kUnits], sf_free[Q::kRing];
+  __shared__ __align__(8) uint64_t sf_ready[Q::kStages * Q::kUnits], sf_free[Q::kRing];
   __shared__ uint32_t tmem_holder;
   __shared__ int32_t tile_start[kMaxGroups + 1], grp_rows[kMaxGroups], grp_row0[kMaxGroups];
   __shared__ float xbuf[GATED ? 128 * 17 : 1];
@@ -759,11 +799,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
   const int Kc = K / F4Fmt<MX>::kChunkK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kQStages; ++s) {
+    for (int s = 0; s < Q::kStages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    for (int r = 0; r < kQStages * Q::kUnits; ++r) mbar_init(&sf_ready[r], 1);
+    for (int r = 0; r < Q::kStages * Q::kUnits; ++r) mbar_init(&sf_ready[r], 1);
     for (int r = 0; r < Q::kRing; ++r) mbar_init(&sf_free[r], 1);
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
@@ -834,10 +874,14 @@ __global__ void __launch_bounds__(kQThreads, 1)
           if (routed) tma2_load_3d(sfa_tile(stage), &tmSfa, lbar, 0, sfa_row, slot);
           else tma2_load_2d(sfa_tile(stage), &tmSfaSh, lbar, 0, sfa_row);
           tma2_load_2d(b_tile(stage), &tmB, lbar, kc, brow);
+          if (Q::kRep) {   // the stage's four replicated K steps: 16 KB = 64 rows of 256 bytes
+            tma2_load_2d(sfb_tile(stage), &tmSfb, lbar, 0, (blk * Kc + kCh * kb) * (kRepChunkBytes / 256));
+          } else {
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
-            tma2_load_2d(sfb_tile(stage) + h * Q::kSfa, &tmSfb, lbar, 0, ((blk * 2 + h) * Kc + kCh * kb) * 2);
-          if (++stage == kQStages) { stage = 0; phase ^= 1u; }
+            for (int h = 0; h < 2; ++h)
+              tma2_load_2d(sfb_tile(stage) + h * Q::kSfa, &tmSfb, lbar, 0, ((blk * 2 + h) * Kc + kCh * kb) * 2);
+          }
+          if (++stage == Q::kStages) { stage = 0; phase ^= 1u; }
         }
       }
     }
@@ -886,7 +930,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
           }
           if (!ok) break;
           umma2_commit_both(&empty_bar[stage]);
-          if (++stage == kQStages) { stage = 0; phase ^= 1u; }
+          if (++stage == Q::kStages) { stage = 0; phase ^= 1u; }
         }
         if (ok) umma2_commit_both(&tfull_bar[ab]);
       }
@@ -914,13 +958,18 @@ __global__ void __launch_bounds__(kQThreads, 1)
             for (int c = 0; c < Q::kUnitChunks; ++c) {   // NVFP4 one chunk per K step, MXFP4 one per two
               const uint32_t off = (j * Q::kUnitChunks + c) * kSfChunk;
               tmem_cp_sf2(sf + 4 * c, smem_desc_sf(ssa + off));                          // this CTA's weight rows
-              tmem_cp_sf2(sf + 4 * Q::kUnitChunks + 8 * c, smem_desc_sf(ssb + off));     // tokens 0-127
-              tmem_cp_sf2(sf + 4 * Q::kUnitChunks + 8 * c + 4, smem_desc_sf(ssb + Q::kSfa + off));  // 128-223
+              if (Q::kRep) {                                                             // all 224 tokens at once
+                tmem_cp_wide2(sf + 4 * Q::kUnitChunks + 8 * c,
+                              smem_desc_rep(ssb + (j * Q::kUnitChunks + c) * kRepChunkBytes));
+              } else {
+                tmem_cp_sf2(sf + 4 * Q::kUnitChunks + 8 * c, smem_desc_sf(ssb + off));   // tokens 0-127
+                tmem_cp_sf2(sf + 4 * Q::kUnitChunks + 8 * c + 4, smem_desc_sf(ssb + Q::kSfa + off));  // 128-223
+              }
             }
             umma2_commit_local(&sf_ready[stage * Q::kUnits + j]);
           }
           if (!ok) break;
-          if (++stage == kQStages) { stage = 0; phase ^= 1u; }
+          if (++stage == Q::kStages) { stage = 0; phase ^= 1u; }
         }
       }
     }
@@ -975,8 +1024,13 @@ __global__ void __launch_bounds__(kQThreads, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i) h[i] = tbuf[tok * 68 + grp * 17 + i];
           const int tr = c0 + tok;   // token row within the 224-row block
-          quant_store_h<MX>(h, gh, six_gh, out_q + static_cast<size_t>(prow + tr) * (Nw / 2) + (pb * 64 + grp * 16) / 2,
-                            out_sf, static_cast<size_t>(blk * 2 + tr / 128), tr % 128, pb, grp, Nw);
+          if constexpr (MX)
+            quant_store_h<MX>(h, gh, six_gh, out_q + static_cast<size_t>(prow + tr) * (Nw / 2) + (pb * 64 + grp * 16) / 2,
+                              out_sf, static_cast<size_t>(blk * 2 + tr / 128), tr % 128, pb, grp, Nw);
+          else
+            quant_store_h<MX, true>(h, gh, six_gh,
+                                    out_q + static_cast<size_t>(prow + tr) * (Nw / 2) + (pb * 64 + grp * 16) / 2, out_sf,
+                                    static_cast<size_t>(blk), tr, pb, grp, Nw);
         }
       } else {
         // lane = output column, TMEM column = token: 32 tokens at a time go through the warp's staging
@@ -1045,14 +1099,21 @@ static int64_t nvfp4_rows_pad(int64_t P, int T, int G, int has_shared, int BN) {
   return P + (has_shared ? T : 0) + static_cast<int64_t>(G) * (BN - 1);
 }
 
+// Bytes of the gathered token-scale region: 128-row chunks (at most rows_pad / 32 + one partial block per
+// group), or for the NVFP4 pair path one replicated 4 KB block per 224-row block and K step.
+static int64_t sfx_region_bytes(int64_t rp, int G, int d) {
+  const int64_t chunks = (rp / 32 + G + 1) * (d / 64) * kSfChunk;
+  const int64_t replicated = (rp / kQN + 1) * (d / 64) * static_cast<int64_t>(kRepChunkBytes);
+  return chunks > replicated ? chunks : replicated;
+}
+
 // Workspace: prow0 | Xq [rows_pad][d/2] | SFx chunks | Hq [rows_pad][I/2] | SFh chunks |
 //            per-token Xq [T][d/2] | per-token scales [T][d/16]
 size_t nvfp4_ffn_workspace_bytes(int64_t P, int T, int E, int has_shared, int d, int I) {
   const int G = E + (has_shared ? 1 : 0);
   const int64_t rp = nvfp4_rows_pad(P, T, G, has_shared, kQN);   // the largest tile bounds all
-  const int64_t blocks = rp / 32 + G + 1;   // 128-row scale chunks: at most rows_pad / 32 + one partial per group
-  return al256(sizeof(int32_t) * (G + 1)) + al256(rp * (d / 2)) + al256(blocks * (d / 64) * kSfChunk) +
-         al256(rp * (I / 2)) + al256(blocks * (I / 64) * kSfChunk) + al256(static_cast<int64_t>(T) * (d / 2)) +
+  return al256(sizeof(int32_t) * (G + 1)) + al256(rp * (d / 2)) + al256(sfx_region_bytes(rp, G, d)) +
+         al256(rp * (I / 2)) + al256(sfx_region_bytes(rp, G, I)) + al256(static_cast<int64_t>(T) * (d / 2)) +
          al256(static_cast<int64_t>(T) * (d / 16));
 }
 
@@ -1105,7 +1166,7 @@ template <bool GATED, bool MX>
 static cudaError_t launch_nvfp4_tc2_one(const CUtensorMap* maps, const FfnArgs& a, const int32_t* prow0, int K,
                                         int Nw, int up_row0, size_t st_off, int st_idx, uint8_t* out_q,
                                         uint8_t* out_sf, uint16_t* out_bf16, cudaStream_t st) {
-  const size_t smem = 1024 + static_cast<size_t>(kQStages) * Q2Fmt<MX>::kStage;
+  const size_t smem = 1024 + static_cast<size_t>(Q2Fmt<MX, GATED>::kStages) * Q2Fmt<MX, GATED>::kStage;
   auto kern = ffn_nvfp4_tc2_kernel<GATED, MX>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
@@ -1158,11 +1219,11 @@ static const char* launch_nvfp4_gemms_tc2(const FfnArgs& a, const int32_t* prow0
   bool ok = make_map_f4(&m1[0], a.pool + a.w_gu_off, a.d, 2ull * a.I, S, a.bank_bytes, 64) &&
             make_map_f4(&m1[2], xq, a.d, static_cast<uint64_t>(rp), 0, 0, kQH) &&
             make_map_rows256(&m1[3], a.pool + s_gu_off, s_gu_bytes, S, a.bank_bytes, kBox) &&
-            make_map_rows256(&m1[5], sfx, sfx_bytes, 0, 0, kBox) &&
+            make_map_rows256(&m1[5], sfx, sfx_bytes, 0, 0, MX ? kBox : 4 * kRepChunkBytes / 256) &&
             make_map_f4(&m2[0], a.pool + a.w_d_off, a.I, a.d, S, a.bank_bytes, 128) &&
             make_map_f4(&m2[2], hq, a.I, static_cast<uint64_t>(rp), 0, 0, kQH) &&
             make_map_rows256(&m2[3], a.pool + s_d_off, s_d_bytes, S, a.bank_bytes, kBox) &&
-            make_map_rows256(&m2[5], sfh, sfh_bytes, 0, 0, kBox);
+            make_map_rows256(&m2[5], sfh, sfh_bytes, 0, 0, MX ? kBox : 4 * kRepChunkBytes / 256);
   if (ok && a.has_shared) {
     ok = make_map_f4(&m1[1], a.shared_bank + a.w_gu_off, a.d, 2ull * a.I, 0, 0, 64) &&
          make_map_rows256(&m1[4], a.shared_bank + s_gu_off, s_gu_bytes, 0, 0, kBox) &&
@@ -1203,9 +1264,9 @@ static const char* launch_f4(const FfnArgs& a, size_t s_gu_off, size_t s_d_off, 
   uint8_t* xq = ws + al256(sizeof(int32_t) * (G + 1));
   uint8_t* sfx = xq + al256(rp * (a.d / 2));
   // regions sized for NVFP4's chunks (MXFP4 uses half of each scale region)
-  uint8_t* hq = sfx + al256(blocks * (a.d / 64) * kSfChunk);
+  uint8_t* hq = sfx + al256(sfx_region_bytes(rp, G, a.d));
   uint8_t* sfh = hq + al256(rp * (a.I / 2));
-  uint8_t* xq_tok = sfh + al256(blocks * (a.I / 64) * kSfChunk);
+  uint8_t* xq_tok = sfh + al256(sfx_region_bytes(rp, G, a.I));
   uint8_t* s_tok = xq_tok + al256(static_cast<int64_t>(a.T) * (a.d / 2));
   prof_mark(FTM_K_GATHER, st, false);
   // each token is quantised once, then its packed row is copied into every
@@ -1219,13 +1280,14 @@ static const char* launch_f4(const FfnArgs& a, size_t s_gu_off, size_t s_d_off, 
   if (*cerr == cudaSuccess) {
     const int grid = static_cast<int>(rp / 8 + 1 < 148 * 8 ? rp / 8 + 1 : 148 * 8);
     *cerr = launch_pdl(gather_f4_kernel<MX>, dim3(grid), dim3(256), 0, st, xq_tok, s_tok, a.perm, a.offsets, prow0,
-                       a.E, a.has_shared, a.T, a.k, a.d, BN, xq, sfx);
+                       a.E, a.has_shared, a.T, a.k, a.d, BN, !MX && pair ? 1 : 0, xq, sfx);
   }
   prof_mark(FTM_K_GATHER, st, true);
   if (*cerr != cudaSuccess) return "nvfp4 gather launch failed";
   if (pair)
     return launch_nvfp4_gemms_tc2<MX>(a, prow0, s_gu_off, s_d_off, s_t_off, rp, xq, sfx,
-                                      blocks * (a.d / kCK) * kSfChunk, hq, sfh, blocks * (a.I / kCK) * kSfChunk, st, cerr);
+                                      MX ? blocks * (a.d / kCK) * kSfChunk : sfx_region_bytes(rp, G, a.d), hq, sfh,
+                                      MX ? blocks * (a.I / kCK) * kSfChunk : sfx_region_bytes(rp, G, a.I), st, cerr);
   CUtensorMap mA1, mAsh1, mB1, mA2, mAsh2, mB2;
   const uint64_t S = static_cast<uint64_t>(a.S);
   // gate/up boxes are 64 rows: a tile stages 64 gate rows and the same 64 up rows
