@@ -154,8 +154,8 @@ def dtype_peak(pk: dict, src: str, wdtype: str):
     sustained bf16 figure times the nominal dense ratio for fp8 (2) and fp4 (4)."""
     bf16 = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
     ratio = {"f32": 1.0, "bf16": 1.0, "fp8": 2.0, "nvfp4": 4.0, "mxfp4": 4.0}[wdtype]
-    where = (f"{src} bf16_tflops_sustained" if ratio == 1.0 else
-             f"derived: {ratio:g} x {src} bf16_tflops_sustained (nominal dense ratio)")
+    where = (f"bf16_tflops_sustained (of {src})" if ratio == 1.0 else
+             f"derived: {ratio:g} x bf16_tflops_sustained (of {src}; nominal dense ratio)")
     return bf16 * ratio, where
 
 
@@ -268,7 +268,7 @@ def rooflines(cfg, alg, g1_ms, step_ms, decode: bool):
         lay = alg["layer_bytes"] / (step_ms * 1e-3) / 1e9
         return {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                 "kernel": "gemm1 (grouped gate/up + SwiGLU)", "algorithmic_bytes": alg["gemm1_bytes"],
-                "peak_source": f"{src} hbm_gbs (of {src})",
+                "peak_source": f"hbm_gbs (of {src})",
                 "layer": {"achieved": lay, "frac": lay / peak, "algorithmic_bytes": alg["layer_bytes"],
                           "what": "expert banks touched + router + activations, per step, over ms_per_step"}}
     peak, where = dtype_peak(pk, src, cfg.wdtype)
@@ -622,7 +622,7 @@ def run_trace(cfg, T, args, dist, local):
         "launch": "eager (one host sync per step to read the miss list)",
         "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                      "kernel": "gemm1 (fp8 grouped gate/up + SwiGLU)", "algorithmic_bytes": alg_g1,
-                     "peak_source": f"{src} hbm_gbs (of {src})",
+                     "peak_source": f"hbm_gbs (of {src})",
                      "traffic": ncu_traffic(workload_name(cfg, T), "gemm1", cfg.wdtype),
                      "layer": {"achieved": layer_bytes / (ms / K * 1e-3) / 1e9,
                                "frac": layer_bytes / (ms / K * 1e-3) / 1e9 / peak, "algorithmic_bytes": layer_bytes,
