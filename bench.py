@@ -865,7 +865,7 @@ def main():
         for T in Ts:
             try:
                 records.append(run_resident(dl, T, args, dist, local))
-            except ftm.FtmError as e:     # a workload this build has no kernel for
+            except ftm.FtmError as e:     # a workload the library has no kernel for
                 if e.status != ftm.binding.FTM_ERR_UNSUPPORTED:
                     raise
                 records.append({"workload": workload_name(cfg, T), "unsupported": str(e)})
