@@ -24,6 +24,7 @@ from .binding import (  # noqa: F401
     ftm_ffn_workspace_bytes,
     ftm_get_bank_layout,
     ftm_kernel_launches,
+    ftm_selftest_bounded_wait,
     ftm_last_error,
     ftm_moe_layer_forward,
     ftm_moe_layer_forward_noalloc,

@@ -88,6 +88,7 @@ def library() -> ctypes.CDLL:
         L.ftm_set_profile_events.restype = c_i32
         L.ftm_kernel_launches.argtypes = []
         L.ftm_kernel_launches.restype = c_u64
+        L.ftm_selftest_bounded_wait.argtypes = [P(c_i32), c_p]
         L.ftm_workspace_bytes.argtypes = [P(LayerDesc), c_i32]
         L.ftm_workspace_bytes.restype = c_sz
         for name in ("ftm_get_bank_layout", "ftm_route", "ftm_permute", "ftm_slot_lookup_update", "ftm_slot_resize",
@@ -227,6 +228,13 @@ def ftm_set_profile_events(which: int, start_event=None, stop_event=None):
 
 def ftm_kernel_launches() -> int:
     return int(library().ftm_kernel_launches())
+
+
+def ftm_selftest_bounded_wait(stream=None) -> int:
+    """Run the bounded-wait self-test kernel; returns the device status it left (1 = the wait gave up)."""
+    v = ctypes.c_int32(-1)
+    _check(library().ftm_selftest_bounded_wait(ctypes.byref(v), _stream(stream)))
+    return int(v.value)
 
 
 def ftm_workspace_bytes(desc, T_max) -> int:

@@ -22,6 +22,7 @@ cudaError_t launch_lru_restore(int E, int S, int key_base, int32_t* soe, int32_t
 cudaError_t launch_slot_resize(int E, int S_old, const int32_t* eos_old, const int64_t* lu_old, int S_new,
                                int32_t* soe_new, int32_t* eos_new, int64_t* lu_new, const void* old_pool,
                                void* new_pool, size_t bank_bytes, int32_t* ws, cudaStream_t st);
+cudaError_t launch_wait_selftest(cudaStream_t st);
 cudaError_t launch_combine(bool f32, const void* y, const int32_t* inv, const float* gw, int T, int k, int d, int P,
                            int has_shared, void* out, cudaStream_t st);
 const char* launch_expert_ffn(const FfnArgs& a, cudaStream_t st, cudaError_t* cerr);
@@ -345,6 +346,15 @@ ftm_status ftm_set_profile_events(int32_t which, void* start_event, void* stop_e
   g_prof[which][0] = static_cast<cudaEvent_t>(start_event);
   g_prof[which][1] = static_cast<cudaEvent_t>(stop_event);
   return ok();
+}
+
+ftm_status ftm_selftest_bounded_wait(int32_t* observed, void* stream) {
+  if (observed == nullptr) return fail(FTM_ERR_INVALID_ARG, "ftm_selftest_bounded_wait: observed is NULL");
+  cudaError_t e = ftm::launch_wait_selftest(S_(stream));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(S_(stream));
+  if (e != cudaSuccess) return fail(FTM_ERR_CUDA, "ftm_selftest_bounded_wait: %s", cudaGetErrorString(e));
+  *observed = ftm_device_status(1);
+  return FTM_OK;
 }
 
 int32_t ftm_device_status(int32_t reset) {

@@ -394,6 +394,16 @@ const char* ftm_last_error(void);
  * outside its range (an expert id outside [0, E)) and skipped the access. */
 int32_t ftm_device_status(int32_t reset);
 
+/* Failure-detection self-test of the bounded waits: launches one block of one
+ * thread that waits on a shared-memory mbarrier nothing ever completes, with
+ * the wait every tensor-core kernel uses.  The wait gives up after its time
+ * limit (about 2 s), sets the device status word to 1 and the kernel returns,
+ * so the context stays usable.  Synchronises `stream`, then writes the status
+ * word to *observed (1 expected) and clears it.  Allocates nothing; returns
+ * FTM_ERR_CUDA if the launch or the synchronisation failed.  Not part of the
+ * layer path: a test of the mechanism the layer kernels rely on. */
+ftm_status ftm_selftest_bounded_wait(int32_t* observed, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

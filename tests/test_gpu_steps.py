@@ -305,3 +305,15 @@ def test_combine_skips_unplaced_pairs():
     yc = y.cpu().numpy().astype(np.float64)
     want = np.stack([0.25 * yc[3], 0.5 * yc[1] + 0.5 * yc[2]])
     assert np.allclose(out.cpu().numpy(), want, rtol=1e-6)
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    """A wait on a barrier that nothing completes gives up after its limit, reports status 1 (timeout), and
+    the context stays usable: a layer computed afterwards still matches the oracle."""
+    ftm.ftm_device_status(True)
+    assert ftm.ftm_selftest_bounded_wait() == 1
+    assert ftm.ftm_device_status(True) == 0
+    cfg = synth.CONFIGS["tiny"]
+    ids, gw, rid, rg = _route_case(cfg, 16)
+    assert np.array_equal(ids, rid)
+    assert ftm.ftm_device_status(True) == 0
