@@ -400,8 +400,10 @@ __device__ __forceinline__ void quant_store_h(const float (&h)[16], float gh, fl
 // memory, applies the per-tensor scales and SwiGLU, then transposes H so each
 // thread quantises one token's 16 consecutive intermediate values.
 // ---------------------------------------------------------------------------
+constexpr int kF4Threads = 224;   // warps 0 TMA, 1 MMA, 2-5 epilogue, 6 scale copies
+
 template <int BN, bool GATED, bool MX>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kF4Threads, 1)
     ffn_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAsh,
                      const __grid_constant__ CUtensorMap tmB, const int32_t* __restrict__ offsets,
                      const int32_t* __restrict__ prow0, const int32_t* __restrict__ slot_of_expert, int E,
@@ -430,6 +432,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[8], empty_bar[8], tfull_bar[2], tempty_bar[2];
+  // the scale warp copies a stage's chunks into scale set g % kSfSets (g = stages so far), then commits
+  // sf_ready[stage]; the MMA thread commits sf_free[set] once the MMAs reading the set are done
+  __shared__ __align__(8) uint64_t sf_ready[8], sf_free[4];
   __shared__ uint32_t tmem_holder;
   __shared__ int32_t tile_start[kMaxGroups + 1], grp_rows[kMaxGroups], grp_row0[kMaxGroups];
   // gate/up epilogue: half-chunks crossing between gate and up warps, and a
@@ -446,7 +451,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int Kc = K / Fmt::kChunkK;                  // scale chunks along K of one 128-row block
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < stages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+      mbar_init(&sf_ready[s], 1);
+    }
+    for (int r = 0; r < static_cast<int>(kSfSets); ++r) mbar_init(&sf_free[r], 1);
     for (int a = 0; a < 2; ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 4); }
     fence_mbar_init();
   }
@@ -531,16 +541,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t d = tmem_base + ab * kAccCols;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase)) { ok = false; break; }
+          if (!mbar_wait(&sf_ready[stage], phase)) { ok = false; break; }   // the stage's scales are in TMEM
           tc_fence_after();
+          const uint32_t cur_set = sf_set;
           const uint32_t tmem_sf = tmem_sf0 + sf_set * kSfCols;
           if (++sf_set == kSfSets) sf_set = 0;
           const uint32_t sb = smem_u32(b_tile(stage));
-#pragma unroll
-          for (int c = 0; c < kCh; ++c) {
-#pragma unroll
-            for (int p = 0; p <= NP; ++p)
-              tmem_cp_sf(tmem_sf + 4 * kCh * p + 4 * c, smem_desc_sf(smem_u32(sf_tile(stage, p)) + c * kSfChunk));
-          }
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const int c = kk * kCh / 4;                    // the chunk of this K step
@@ -559,10 +565,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               }
             }
           }
+          umma_commit(&sf_free[cur_set]);   // the scale warp may refill this set
           umma_commit(&empty_bar[stage]);
           if (++stage == stages) { stage = 0; phase ^= 1u; }
         }
         if (ok) umma_commit(&tfull_bar[ab]);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 6) {
+    // scale warp: copies each stage's weight and token scale chunks into the next TMEM set, ahead of the MMAs
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      uint32_t g = 0;   // stages copied so far
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (int kb = 0; kb < KB; ++kb, ++g) {
+          if (!mbar_wait(&full_bar[stage], phase)) { ok = false; break; }
+          const uint32_t set = g % kSfSets;
+          // the set is free once the MMAs of the stage kSfSets earlier are done
+          if (g >= kSfSets && !mbar_wait(&sf_free[set], (g / kSfSets - 1) & 1u)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t tmem_sf = tmem_sf0 + set * kSfCols;
+#pragma unroll
+          for (int c = 0; c < kCh; ++c) {
+#pragma unroll
+            for (int p = 0; p <= NP; ++p)
+              tmem_cp_sf(tmem_sf + 4 * kCh * p + 4 * c, smem_desc_sf(smem_u32(sf_tile(stage, p)) + c * kSfChunk));
+          }
+          umma_commit(&sf_ready[stage]);
+          if (++stage == stages) { stage = 0; phase ^= 1u; }
+        }
       }
     }
     __syncwarp();
@@ -1135,7 +1169,7 @@ static cudaError_t launch_nvfp4(const CUtensorMap& mA, const CUtensorMap& mAsh, 
   const int G = a.E + (a.has_shared ? 1 : 0);
   const long max_tiles = static_cast<long>((P + BN - 1) / BN + G) * (Nw / ((GATED ? 64 : 128) * NP));
   const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
-  return launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st, mA, mAsh, mB, a.offsets, prow0, a.slot_of_expert,
+  return launch_pdl(kern, dim3(grid), dim3(kF4Threads), smem, st, mA, mAsh, mB, a.offsets, prow0, a.slot_of_expert,
                     a.E, a.has_shared, a.T, P, K, Nw, up_row0, a.pool, a.shared_bank, a.bank_bytes, wsf_off, st_off,
                     st_idx, act_sf, out_q, out_sf, out_bf16, a.act_scale, stages);
 }
