@@ -15,8 +15,8 @@ constexpr int kMaxTerms = 17;   // k <= 16 routed picks + the shared expert
 // each lane issues all of the token's row loads for its 16-byte vector before
 // the fused multiply-adds.  The terms are added in ascending j, so the result
 // does not depend on the schedule.
-template <bool F32>
-__global__ void __launch_bounds__(256, 2) combine_kernel(const void* __restrict__ y, const int32_t* __restrict__ inv,
+template <bool F32, int MAXT>
+__global__ void __launch_bounds__(256, MAXT <= 9 ? 3 : 2) combine_kernel(const void* __restrict__ y, const int32_t* __restrict__ inv,
                                                       const float* __restrict__ gw, int T, int k, int d, int P,
                                                       int has_shared, int spi, void* __restrict__ out) {
   constexpr int V = F32 ? 4 : 8;   // elements per 16-byte vector
@@ -25,8 +25,8 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(const void* __restrict_
   const int nterms = k + (has_shared ? 1 : 0);
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
-  __shared__ int s_rows[8][kMaxTerms];
-  __shared__ float s_gs[8][kMaxTerms];
+  __shared__ int s_rows[8][MAXT];
+  __shared__ float s_gs[8][MAXT];
   pdl_wait();
   pdl_trigger();
   const int nch = (nv + 31) / 32;                    // 32-vector slices of a row
@@ -50,15 +50,15 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(const void* __restrict_
     // the warp's copy of the token's rows and gates
     int* rows = s_rows[threadIdx.x >> 5];
     float* gs = s_gs[threadIdx.x >> 5];
-    if (lane < kMaxTerms) {
+    if (lane < MAXT) {
       rows[lane] = lane < nterms ? my_row : -1;
       gs[lane] = my_g;
     }
     __syncwarp();
     for (int c = c0 + lane; c < nv && c < c0 + spi * 32; c += 32) {
-      uint4 u[kMaxTerms];
+      uint4 u[MAXT];
 #pragma unroll
-      for (int j = 0; j < kMaxTerms; ++j)
+      for (int j = 0; j < MAXT; ++j)
         if (j < nterms && rows[j] >= 0)
           u[j] = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(y) +
                                                  (static_cast<size_t>(rows[j]) * d + static_cast<size_t>(c) * V) * EB);
@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(const void* __restrict_
 #pragma unroll
       for (int i = 0; i < V; ++i) acc[i] = 0.f;
 #pragma unroll
-      for (int j = 0; j < kMaxTerms; ++j) {
+      for (int j = 0; j < MAXT; ++j) {
         if (j >= nterms || rows[j] < 0) continue;
         const float g = gs[j];
         if constexpr (F32) {
@@ -113,12 +113,17 @@ cudaError_t launch_combine(bool f32, const void* y, const int32_t* inv, const fl
   const long long items = static_cast<long long>(T) * ((nch + spi - 1) / spi);
   const long long blocks = (items + 7) / 8;   // 8 items (warps) per block
   const int grid = static_cast<int>(blocks < 148 * 8 ? blocks : 148 * 8);
+  // up to 8 routed picks + the shared expert: a 9-term register file, which lets three blocks share an SM
+  const bool small = k + (has_shared ? 1 : 0) <= 9;
   if (f32)
-    return launch_pdl(combine_kernel<true>, dim3(grid), dim3(256), 0, st, y, inv, gw, T, k, d, P, has_shared, spi, out);
-  else
-    return launch_pdl(combine_kernel<false>, dim3(grid), dim3(256), 0, st, y, inv, gw, T, k, d, P, has_shared, spi,
-                      out);
-  return cudaGetLastError();
+    return small ? launch_pdl(combine_kernel<true, 9>, dim3(grid), dim3(256), 0, st, y, inv, gw, T, k, d, P, has_shared,
+                              spi, out)
+                 : launch_pdl(combine_kernel<true, kMaxTerms>, dim3(grid), dim3(256), 0, st, y, inv, gw, T, k, d, P,
+                              has_shared, spi, out);
+  return small ? launch_pdl(combine_kernel<false, 9>, dim3(grid), dim3(256), 0, st, y, inv, gw, T, k, d, P, has_shared,
+                            spi, out)
+               : launch_pdl(combine_kernel<false, kMaxTerms>, dim3(grid), dim3(256), 0, st, y, inv, gw, T, k, d, P,
+                            has_shared, spi, out);
 }
 
 }  // namespace ftm

@@ -19,10 +19,10 @@ constexpr int kRtBK = 64;             // K per stage (bf16, one 128-byte swizzle
 constexpr int kRtBM = 128;            // tokens per tile (the MMA M)
 constexpr int kRtMaxK = 16;
 constexpr int kRtMaxNE = 256;         // experts (MMA N) at most
-constexpr int kRtStages = 4;
+constexpr int kRtMaxStages = 8;
 constexpr uint32_t kRtXBytes = kRtBM * 128;          // 128 tokens x 64 bf16
-constexpr uint32_t kRtWBytes = kRtMaxNE * 128;       // up to 256 router rows x 64 bf16
-constexpr uint32_t kRtStage = kRtXBytes + kRtWBytes;
+// a stage is the x tile and NE router rows x 64 bf16 (NE a multiple of 16, so every tile stays 1024-aligned);
+// as many stages as fit 199 KB, at most 8: 6 for E = 128, 5 for E = 160, 4 for E = 256
 constexpr uint32_t kRtTmemCols = 2 * kRtMaxNE;       // two accumulators of up to 256 columns
 
 // Gates of one token from its top k (pv descending, pi ids): softmax over the
@@ -127,9 +127,9 @@ __device__ __forceinline__ void route_token_any(uint32_t tb, int NE, int E, int 
 __global__ void __launch_bounds__(kTcThreads, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, int T, int d,
                     const float* __restrict__ bias, int E, int NE, int k, int32_t* __restrict__ topk_ids,
-                    float* __restrict__ topk_w) {
+                    float* __restrict__ topk_w, int stages) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[kRtStages], empty_bar[kRtStages], tfull_bar[2], tempty_bar[2];
+  __shared__ __align__(8) uint64_t full_bar[kRtMaxStages], empty_bar[kRtMaxStages], tfull_bar[2], tempty_bar[2];
   __shared__ uint32_t tmem_holder;
   __shared__ float s_bias[kRtMaxNE];
 
@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t idesc = idesc_bf16_f32(kRtBM, NE);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kRtStages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    for (int s = 0; s < stages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 4); }
     fence_mbar_init();
   }
@@ -161,8 +161,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_holder;
-  auto x_tile = [&](int s) -> uint8_t* { return smem + static_cast<size_t>(s) * kRtStage; };
-  auto w_tile = [&](int s) -> uint8_t* { return smem + static_cast<size_t>(s) * kRtStage + kRtXBytes; };
+  const size_t stage_bytes = kRtXBytes + static_cast<size_t>(NE) * 128;
+  auto x_tile = [&](int s) -> uint8_t* { return smem + static_cast<size_t>(s) * stage_bytes; };
+  auto w_tile = [&](int s) -> uint8_t* { return smem + static_cast<size_t>(s) * stage_bytes + kRtXBytes; };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -175,7 +176,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           mbar_arrive_expect_tx(&full_bar[stage], tx);
           tma_load_2d(x_tile(stage), &tmX, &full_bar[stage], kb * kRtBK, t * kRtBM);
           tma_load_2d(w_tile(stage), &tmW, &full_bar[stage], kb * kRtBK, 0);
-          if (++stage == kRtStages) { stage = 0; phase ^= 1u; }
+          if (++stage == stages) { stage = 0; phase ^= 1u; }
         }
       }
     }
@@ -201,7 +202,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             umma_f16(dacc, smem_desc_sw128(sx + kk * 32), smem_desc_sw128(sw + kk * 32), idesc,
                      (kb | kk) != 0 ? 1u : 0u);
           umma_commit(&empty_bar[stage]);
-          if (++stage == kRtStages) { stage = 0; phase ^= 1u; }
+          if (++stage == stages) { stage = 0; phase ^= 1u; }
         }
         if (ok) umma_commit(&tfull_bar[ab]);
       }
@@ -248,11 +249,15 @@ cudaError_t launch_route_tc(const void* x, int T, int d, const void* wr, const f
     return cudaErrorInvalidValue;
   const int tiles = (T + kRtBM - 1) / kRtBM;
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  const size_t smem = 1024 + static_cast<size_t>(kRtStages) * kRtStage;
+  const size_t stage_bytes = kRtXBytes + static_cast<size_t>(NE) * 128;
+  int stages = static_cast<int>((199 * 1024) / stage_bytes);
+  if (stages > kRtMaxStages) stages = kRtMaxStages;
+  const size_t smem = 1024 + static_cast<size_t>(stages) * stage_bytes;
   cudaError_t e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  return launch_pdl(route_tc_kernel, dim3(grid), dim3(kTcThreads), smem, st, mX, mW, T, d, bias, E, NE, k, ids, w);
+  return launch_pdl(route_tc_kernel, dim3(grid), dim3(kTcThreads), smem, st, mX, mW, T, d, bias, E, NE, k, ids, w,
+                    stages);
 }
 
 }  // namespace ftm
