@@ -639,7 +639,91 @@ def run_trace(cfg, T, args, dist, local):
                           "on top of the miss copies the step already makes"},
         "gpu_launches": int(launches), "launches_per_step": launches / K, "launches_per_warmup_step": launches_warm,
         "clocks": clk, "device_status": status,
+        "hybrid": run_trace_hybrid(dl, T, xs, W, K, stream, copy_stream, ms / K),
     }
+
+
+def calibrate_bandwidths(dl, stream, reps: int = 5):
+    """The two bandwidths of the miss split, measured the way the pages' `ft bench bw`
+    calibration does: Bp = one expert bank copied from the pinned host pool to the
+    device (CUDA events), Bh = one expert's FFN computed on the host for one row
+    (wall clock), each as expert-bank bytes per second (GB/s)."""
+    bb = int(dl.bl.bank_bytes)
+    dst = torch.empty(bb, dtype=torch.uint8, device="cuda")
+    src = dl.host_pool[:bb]
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            dst.copy_(src, non_blocking=True)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            dst.copy_(src, non_blocking=True)
+        b.record(stream)
+    torch.cuda.synchronize()
+    bp = reps * bb / (a.elapsed_time(b) * 1e-3) / 1e9
+    desc = dl.desc
+    x = np.ascontiguousarray(dl.layer.hidden_storage(1, 0))
+    y = np.zeros_like(x)
+    nb = ftm.ftm_host_ffn_scratch_bytes(desc, 1)
+    scratch = torch.empty(nb + 64, dtype=torch.uint8)
+    sp = scratch.data_ptr() + (-scratch.data_ptr()) % 64
+    bank = dl.host_pool.data_ptr()
+    ftm.ftm_host_expert_ffn(desc, bank, x, 1, y, sp, nb, 0)
+    t = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        ftm.ftm_host_expert_ffn(desc, bank, x, 1, y, sp, nb, 0)
+        t.append(time.perf_counter() - t0)
+    bh = bb / statistics.median(t) / 1e9
+    return bp, bh
+
+
+def run_trace_hybrid(dl, T, xs, W, K, stream, copy_stream, plain_ms):
+    """The same trace steps through the bandwidth-adaptive miss split
+    (ftm_moe_layer_forward_hybrid), from a cold cache like the offload run: W
+    warm-up steps, then K timed with CUDA events on the layer's stream."""
+    from synth.device import Workspace
+    bp, bh = calibrate_bandwidths(dl, stream)
+    for t in (dl.slot_of_expert, dl.expert_of_slot, dl.last_use):
+        t.fill_(-1)
+    dl.cache.step = 0
+    torch.cuda.synchronize()
+    ws = Workspace(ftm.ftm_hybrid_workspace_bytes(dl.desc, T))
+    nb = ftm.ftm_hybrid_host_bytes(dl.desc, T)
+    hbuf = torch.empty(nb, dtype=torch.uint8, pin_memory=True)
+    h = ftm.Hybrid(bp, bh, 0, 0, 0, 0, 0.0, hbuf.data_ptr(), nb)
+    out = torch.empty((T, dl.cfg.d), dtype=torch.bfloat16, device="cuda")
+    w = dl.weights()
+
+    def step(s):
+        ftm.ftm_moe_layer_forward_hybrid(dl.desc, w, dl.cache, h, xs[s], T, out, ws.ptr, ws.nbytes, stream,
+                                         copy_stream)
+        return h.last_misses, h.last_host, h.last_host_ms
+
+    for s in range(W):
+        step(s)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    m = host = 0
+    host_ms = 0.0
+    t0.record(stream)
+    for i in range(K):
+        a, b, c = step(W + i)
+        m, host, host_ms = m + a, host + b, host_ms + c
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / K
+    return {"what": "the same trace steps with the bandwidth-adaptive miss split (q* policy): of each step's m "
+                    "misses, q = round(m Bp / (Bp + Bh)) are copied over PCIe and computed on the GPU, m - q are "
+                    "computed on the host CPU from the pinned host pool meanwhile; cold cache, as the offload run",
+            "pcie_gbs": bp, "host_gbs": bh,
+            "calibration": "Bp: one expert bank host->device, pinned (CUDA events); Bh: one expert's FFN for one "
+                           "row on the host threads (wall clock); both in expert-bank bytes per second",
+            "host_threads": os.cpu_count(), "steps": K, "warmup": W, "ms_per_step": ms,
+            "ms_per_step_offload": plain_ms, "speedup_vs_offload": plain_ms / ms,
+            "value": K * T / (ms * K * 1e-3), "unit": "tokens/s",
+            "misses_per_step": m / K, "host_experts_per_step": host / K, "host_ffn_ms_per_step": host_ms / K,
+            "device_status": ftm.ftm_device_status(True)}
 
 
 def run_layers_pipeline(cfg, T, n_layers, args, local):
@@ -899,6 +983,7 @@ def main():
             "kernels_ms": head_rec.get("kernels_ms"),
             "kernels_ms_breakdown": head_rec.get("kernels_ms_breakdown"),
             "device_status": head_rec["device_status"],
+            **{key: head_rec[key] for key in ("cache", "hybrid") if key in head_rec},
             "workloads": records,
         }
         print(json.dumps(line), flush=True)

@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     FTM_NVFP4,
     BankLayout,
     FtmError,
+    Hybrid,
     LayerDesc,
     LayerWeights,
     SlotCache,
@@ -23,10 +24,16 @@ from .binding import (  # noqa: F401
     ftm_expert_ffn,
     ftm_ffn_workspace_bytes,
     ftm_get_bank_layout,
+    ftm_host_expert_ffn,
+    ftm_host_ffn_scratch_bytes,
+    ftm_hybrid_host_bytes,
+    ftm_hybrid_split,
+    ftm_hybrid_workspace_bytes,
     ftm_kernel_launches,
     ftm_selftest_bounded_wait,
     ftm_last_error,
     ftm_moe_layer_forward,
+    ftm_moe_layer_forward_hybrid,
     ftm_moe_layer_forward_noalloc,
     ftm_moe_layers_forward,
     ftm_last_warning,

@@ -40,6 +40,13 @@ class LayerWeights(ctypes.Structure):
                 ("shared_bank", c_p), ("act_scale", c_p)]
 
 
+class Hybrid(ctypes.Structure):
+    """ftm_hybrid: the bandwidth-adaptive miss split's parameters, host buffer and results."""
+    _fields_ = [("pcie_gbs", ctypes.c_double), ("host_gbs", ctypes.c_double), ("threads", c_i32),
+                ("last_misses", c_i32), ("last_host", c_i32), ("last_host_rows", c_i32),
+                ("last_host_ms", ctypes.c_double), ("host_ws", c_p), ("host_ws_bytes", c_sz)]
+
+
 class FtmError(RuntimeError):
     def __init__(self, status: int, msg: str):
         super().__init__(f"ftm status {status}: {msg}")
@@ -91,9 +98,17 @@ def library() -> ctypes.CDLL:
         L.ftm_selftest_bounded_wait.argtypes = [P(c_i32), c_p]
         L.ftm_workspace_bytes.argtypes = [P(LayerDesc), c_i32]
         L.ftm_workspace_bytes.restype = c_sz
+        L.ftm_hybrid_split.argtypes = [c_i32, ctypes.c_double, ctypes.c_double]
+        L.ftm_hybrid_split.restype = c_i32
+        for name in ("ftm_hybrid_workspace_bytes", "ftm_hybrid_host_bytes", "ftm_host_ffn_scratch_bytes"):
+            getattr(L, name).argtypes = [P(LayerDesc), c_i32]
+            getattr(L, name).restype = c_sz
+        L.ftm_host_expert_ffn.argtypes = [P(LayerDesc), c_p, c_p, c_i32, c_p, c_p, c_sz, c_i32]
+        L.ftm_moe_layer_forward_hybrid.argtypes = [P(LayerDesc), P(LayerWeights), P(SlotCache), P(Hybrid), c_p,
+                                                   c_i32, c_p, c_p, c_sz, c_p, c_p]
         for name in ("ftm_get_bank_layout", "ftm_route", "ftm_permute", "ftm_slot_lookup_update", "ftm_slot_resize",
                      "ftm_slot_stage_layer", "ftm_expert_ffn", "ftm_combine", "ftm_moe_layer_forward",
-                     "ftm_moe_layers_forward"):
+                     "ftm_moe_layers_forward", "ftm_host_expert_ffn", "ftm_moe_layer_forward_hybrid"):
             getattr(L, name).restype = c_i32
         _lib = L
     return _lib
@@ -109,7 +124,9 @@ def _ptr(t) -> Optional[int]:
         return None
     if isinstance(t, int):
         return t
-    return t.data_ptr()
+    if hasattr(t, "data_ptr"):
+        return t.data_ptr()
+    return t.ctypes.data   # numpy array (host)
 
 
 def _stream(stream) -> Optional[int]:
@@ -254,3 +271,33 @@ def ftm_moe_layer_forward_noalloc(desc, weights: LayerWeights, x, T, out, stream
     (for callers that cannot allocate device memory; see include/ftm.h)."""
     _check(library().ftm_moe_layer_forward_noalloc(ctypes.byref(desc), ctypes.byref(weights), _ptr(x), T, _ptr(out),
                                                    _stream(stream)))
+
+
+def ftm_hybrid_split(m: int, pcie_gbs: float, host_gbs: float) -> int:
+    """q of the bandwidth-adaptive miss split (-1 on invalid arguments)."""
+    return int(library().ftm_hybrid_split(m, pcie_gbs, host_gbs))
+
+
+def ftm_hybrid_workspace_bytes(desc, T_max) -> int:
+    return int(library().ftm_hybrid_workspace_bytes(ctypes.byref(desc), T_max))
+
+
+def ftm_hybrid_host_bytes(desc, T_max) -> int:
+    return int(library().ftm_hybrid_host_bytes(ctypes.byref(desc), T_max))
+
+
+def ftm_host_ffn_scratch_bytes(desc, n) -> int:
+    return int(library().ftm_host_ffn_scratch_bytes(ctypes.byref(desc), n))
+
+
+def ftm_host_expert_ffn(desc, bank, x, n, y, scratch, scratch_bytes, threads: int = 0):
+    """One expert's FFN on the host (host buffers: numpy arrays, CPU tensors or addresses)."""
+    _check(library().ftm_host_expert_ffn(ctypes.byref(desc), _ptr(bank), _ptr(x), n, _ptr(y), _ptr(scratch),
+                                         scratch_bytes, threads))
+
+
+def ftm_moe_layer_forward_hybrid(desc, weights: LayerWeights, cache: SlotCache, hybrid: Hybrid, x, T, out, workspace,
+                                 ws_bytes, stream=None, copy_stream=None):
+    _check(library().ftm_moe_layer_forward_hybrid(ctypes.byref(desc), ctypes.byref(weights), ctypes.byref(cache),
+                                                  ctypes.byref(hybrid), _ptr(x), T, _ptr(out), _ptr(workspace),
+                                                  ws_bytes, _stream(stream), _stream(copy_stream)))

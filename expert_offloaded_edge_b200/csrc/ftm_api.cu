@@ -3,10 +3,15 @@
 // Every computation step runs in the kernels of the sibling .cu files.
 #include <stdarg.h>
 #include <atomic>
+#include <cmath>
+#include <vector>
 #include <stdio.h>
 #include <string.h>
 
+#include <chrono>
+
 #include "ftm_common.cuh"
+#include "ftm_host_ffn.h"
 
 namespace ftm {
 cudaError_t launch_route(bool f32, const void* x, int T, int d, const void* wr, const float* bias, int E, int k,
@@ -16,7 +21,9 @@ cudaError_t launch_permute(const int32_t* ids, int P, int E, int32_t* counts, in
 size_t permute_workspace_bytes(int E, int64_t P);
 size_t lru_workspace_bytes(int E, int S);
 cudaError_t launch_lru_step(const int32_t* ids, int P, int E, int S, int64_t step, int64_t reserve, int key_base,
-                            int32_t* soe, int32_t* eos, int64_t* lu, int32_t* ws, cudaStream_t st);
+                            int skip_id, int32_t* soe, int32_t* eos, int64_t* lu, int32_t* ws, cudaStream_t st);
+cudaError_t launch_hybrid_split(const int32_t* ids, int P, int E, const int32_t* soe, double bp, double bh,
+                                int32_t* ids2, int32_t* out, cudaStream_t st);
 cudaError_t launch_lru_restore(int E, int S, int key_base, int32_t* soe, int32_t* eos, int64_t* lu, int32_t* ws,
                                int n_dirty, cudaStream_t st);
 cudaError_t launch_slot_resize(int E, int S_old, const int32_t* eos_old, const int64_t* lu_old, int S_new,
@@ -163,6 +170,75 @@ LayerWs carve(const ftm_layer_desc* L, int32_t T, uint8_t* base) {
   return w;
 }
 
+// Workspace of the hybrid layer: the layer's own, then the remapped ids, the
+// counts / offsets of E + 1 groups (group E: the pairs of the experts computed
+// on the host), the permutation workspace for E + 1 groups and the split's
+// output.  The layer's perm / inv hold the E + 1-group permutation.
+struct HybridWs {
+  LayerWs w;
+  int32_t* ids2;
+  int32_t* counts2;
+  int32_t* offsets2;
+  void* perm_ws2;
+  int32_t* split;
+  size_t total;
+};
+
+HybridWs carve_hybrid(const ftm_layer_desc* L, int32_t T, uint8_t* base) {
+  HybridWs h;
+  h.w = carve(L, T, base);
+  const size_t P = static_cast<size_t>(T) * L->k, E = static_cast<size_t>(L->E);
+  size_t off = h.w.total;
+  auto take = [&](size_t bytes) { uint8_t* p = base ? base + off : nullptr; off += al(bytes); return p; };
+  h.ids2 = reinterpret_cast<int32_t*>(take(P * 4));
+  h.counts2 = reinterpret_cast<int32_t*>(take((E + 1) * 4));
+  h.offsets2 = reinterpret_cast<int32_t*>(take((E + 2) * 4));
+  h.perm_ws2 = take(permute_workspace_bytes(L->E + 1, static_cast<int64_t>(P)));
+  h.split = reinterpret_cast<int32_t*>(take((4 + E) * 4));
+  h.total = off;
+  return h;
+}
+
+// Pinned host workspace of the hybrid layer (64-byte aligned pieces).
+struct HybridHost {
+  int32_t* split;          // [4 + E] the split's output
+  int32_t* ids;            // [P] routed ids
+  int32_t* perm;           // [P] the E + 1-group permutation
+  int32_t* offsets;        // [E + 2]
+  uint8_t* x;              // [T][d] activations
+  uint8_t* y;              // [P][d] outputs of the host rows
+  float* scratch;          // host FFN scratch
+  const uint8_t** xrow;    // [P]
+  uint8_t** yrow;          // [P]
+  HostGroup* groups;       // [E]
+  int32_t* gidx;           // [E] host group of an expert, -1
+  int32_t* gpos;           // [E + 1] first row of each host group
+  size_t total;
+};
+
+HybridHost carve_host(const ftm_layer_desc* L, int32_t T, void* base_v) {
+  HybridHost h;
+  uint8_t* base = static_cast<uint8_t*>(base_v);
+  const size_t P = static_cast<size_t>(T) * L->k, E = static_cast<size_t>(L->E);
+  const size_t row = static_cast<size_t>(L->d) * act_elt(L);
+  size_t off = 0;
+  auto take = [&](size_t bytes) { uint8_t* p = base ? base + off : nullptr; off += (bytes + 63) & ~size_t{63}; return p; };
+  h.split = reinterpret_cast<int32_t*>(take((4 + E) * 4));
+  h.ids = reinterpret_cast<int32_t*>(take(P * 4));
+  h.perm = reinterpret_cast<int32_t*>(take(P * 4));
+  h.offsets = reinterpret_cast<int32_t*>(take((E + 2) * 4));
+  h.x = take(static_cast<size_t>(T) * row);
+  h.y = take(P * row);
+  h.scratch = reinterpret_cast<float*>(take(host_ffn_scratch_bytes(L, static_cast<int64_t>(P))));
+  h.xrow = reinterpret_cast<const uint8_t**>(take(P * sizeof(void*)));
+  h.yrow = reinterpret_cast<uint8_t**>(take(P * sizeof(void*)));
+  h.groups = reinterpret_cast<HostGroup*>(take(E * sizeof(HostGroup)));
+  h.gidx = reinterpret_cast<int32_t*>(take(E * 4));
+  h.gpos = reinterpret_cast<int32_t*>(take((E + 1) * 4));
+  h.total = off;
+  return h;
+}
+
 ftm_status check_ws(void* ws, size_t have, size_t need, const char* who) {
   if (need && !ws) return fail(FTM_ERR_INVALID_ARG, "%s: workspace is NULL (%zu bytes needed)", who, need);
   if (have < need) return fail(FTM_ERR_INVALID_ARG, "%s: workspace %zu bytes < %zu needed", who, have, need);
@@ -221,17 +297,18 @@ cudaEvent_t list_event() {
 // when given, the miss list read back (the host waits for that kernel only),
 // then one bank copy per miss on `copy_stream` (also after `after`).  Victims
 // are the slots with last_use < reserve.  On a copy failure the state is
-// rolled back (slots a copy may have written left empty).
+// rolled back (slots a copy may have written left empty).  skip_id >= 0:
+// pairs with that id are not requests (see hybrid_split_kernel).
 ftm_status cache_step(const ftm_layer_desc* L, ftm_slot_cache* C, const int32_t* ids, int P, int64_t reserve,
                       int32_t* ws, cudaStream_t lru_stream, cudaStream_t copy_stream, cudaEvent_t after,
-                      int* misses_out) {
+                      int* misses_out, int skip_id = -1) {
   *misses_out = 0;
   cudaError_t e;
   // the step rewrites the entries of the keys it evicts: the compute that
   // reads them (done when `after` completes) must be over first
   if (after && (e = cudaStreamWaitEvent(lru_stream, after, 0)) != cudaSuccess) return cuda_fail(e, "lru stream wait");
   prof_mark(FTM_K_LRU, lru_stream, false);
-  e = launch_lru_step(ids, P, L->E, L->S, C->step, reserve, C->key_base, C->slot_of_expert,
+  e = launch_lru_step(ids, P, L->E, L->S, C->step, reserve, C->key_base, skip_id, C->slot_of_expert,
                                   C->expert_of_slot, C->last_use, ws, lru_stream);
   prof_mark(FTM_K_LRU, lru_stream, true);
   if (e != cudaSuccess) return cuda_fail(e, "lru step launch");
@@ -668,5 +745,163 @@ ftm_status ftm_moe_layers_forward(const ftm_layer_desc* L, int32_t n_layers, con
 }
 
 const char* ftm_last_warning(void) { return g_warn; }
+
+int32_t ftm_hybrid_split(int32_t m, double pcie_gbs, double host_gbs) {
+  if (m < 0 || !(pcie_gbs >= 0.0) || !(host_gbs >= 0.0) || !(pcie_gbs + host_gbs > 0.0) ||
+      !std::isfinite(pcie_gbs + host_gbs))
+    return -1;
+  int q = static_cast<int>(floor(static_cast<double>(m) * pcie_gbs / (pcie_gbs + host_gbs) + 0.5));
+  return q < 0 ? 0 : q > m ? m : q;
+}
+
+size_t ftm_hybrid_workspace_bytes(const ftm_layer_desc* L, int32_t T_max) {
+  if (check_desc(L) || T_max < 0) return 0;
+  return carve_hybrid(L, T_max, nullptr).total;
+}
+
+size_t ftm_hybrid_host_bytes(const ftm_layer_desc* L, int32_t T_max) {
+  if (check_desc(L) || T_max < 0) return 0;
+  return carve_host(L, T_max, nullptr).total;
+}
+
+size_t ftm_host_ffn_scratch_bytes(const ftm_layer_desc* L, int32_t n) {
+  if (check_desc(L) || n < 0) return 0;
+  return host_ffn_scratch_bytes(L, n);
+}
+
+ftm_status ftm_host_expert_ffn(const ftm_layer_desc* L, const void* bank, const void* x, int32_t n, void* y,
+                               void* scratch, size_t scratch_bytes, int32_t threads) {
+  ftm_status s = check_desc(L);
+  if (s) return s;
+  if (!host_ffn_supported(L->wdtype))
+    return fail(FTM_ERR_UNSUPPORTED, "ftm_host_expert_ffn: the host FFN handles fp32, bf16 and FP8 banks");
+  if (n < 0) return fail(FTM_ERR_INVALID_ARG, "ftm_host_expert_ffn: n=%d is negative", n);
+  if (n == 0) return ok();
+  if (!bank || !x || !y || !scratch) return fail(FTM_ERR_INVALID_ARG, "ftm_host_expert_ffn: NULL pointer");
+  if (scratch_bytes < host_ffn_scratch_bytes(L, n))
+    return fail(FTM_ERR_INVALID_ARG, "ftm_host_expert_ffn: scratch %zu bytes < %zu needed", scratch_bytes,
+                host_ffn_scratch_bytes(L, n));
+  if (!aligned(bank, 16) || !aligned(scratch, 16))
+    return fail(FTM_ERR_INVALID_ARG, "ftm_host_expert_ffn: bank / scratch not 16-byte aligned");
+  ftm_bank_layout bl;
+  bank_layout(L, &bl);
+  const size_t row = static_cast<size_t>(L->d) * act_elt(L);
+  std::vector<const uint8_t*> xr(n);
+  std::vector<uint8_t*> yr(n);
+  for (int r = 0; r < n; ++r) {
+    xr[r] = static_cast<const uint8_t*>(x) + r * row;
+    yr[r] = static_cast<uint8_t*>(y) + r * row;
+  }
+  HostGroup g{static_cast<const uint8_t*>(bank), n, xr.data(), yr.data()};
+  host_ffn_groups(L, &bl, &g, 1, static_cast<float*>(scratch), threads);
+  return ok();
+}
+
+ftm_status ftm_moe_layer_forward_hybrid(const ftm_layer_desc* L, const ftm_layer_weights* W, ftm_slot_cache* C,
+                                        ftm_hybrid* H, const void* x, int32_t T, void* out, void* workspace,
+                                        size_t ws_bytes, void* stream, void* copy_stream) {
+  static const char* who = "ftm_moe_layer_forward_hybrid";
+  ftm_status s = check_desc(L);
+  if (s || (s = check_T(T))) return s;
+  if (!W || !W->w_router) return fail(FTM_ERR_INVALID_ARG, "%s: NULL weights", who);
+  if (!H) return fail(FTM_ERR_INVALID_ARG, "%s: NULL split parameters", who);
+  if (ftm_hybrid_split(0, H->pcie_gbs, H->host_gbs) < 0)
+    return fail(FTM_ERR_INVALID_ARG, "%s: bandwidths must be finite, >= 0 and not both 0 (Bp=%g, Bh=%g)", who,
+                H->pcie_gbs, H->host_gbs);
+  if (!host_ffn_supported(L->wdtype))
+    return fail(FTM_ERR_UNSUPPORTED, "%s: the host FFN handles fp32, bf16 and FP8 banks", who);
+  if ((s = check_cache(L, C, who))) return s;
+  if (T == 0) return ok();
+  if (!x || !out) return fail(FTM_ERR_INVALID_ARG, "%s: NULL x / out", who);
+  HybridWs hw = carve_hybrid(L, T, static_cast<uint8_t*>(workspace));
+  if ((s = check_ws(workspace, ws_bytes, hw.total, who))) return s;
+  HybridHost hh = carve_host(L, T, H->host_ws);
+  if (!H->host_ws || H->host_ws_bytes < hh.total || !aligned(H->host_ws, 64))
+    return fail(FTM_ERR_INVALID_ARG, "%s: host_ws needs %zu bytes, 64-byte aligned (have %zu)", who, hh.total,
+                H->host_ws ? H->host_ws_bytes : static_cast<size_t>(0));
+  cudaPointerAttributes pa;
+  if (cudaPointerGetAttributes(&pa, H->host_ws) != cudaSuccess || pa.type != cudaMemoryTypeHost) {
+    cudaGetLastError();
+    return fail(FTM_ERR_INVALID_ARG, "%s: host_ws is not pinned host memory", who);
+  }
+  const int E = L->E, k = L->k, d = L->d, P = T * k;
+  const size_t row = static_cast<size_t>(d) * act_elt(L);
+  cudaStream_t cs = S_(stream), ps = S_(copy_stream);
+  LayerWs& w = hw.w;
+  cudaError_t e;
+  if ((s = ftm_route(L, x, T, W->w_router, W->router_bias, w.ids, w.gates, stream))) return s;
+  // the split (against the residency before this step), then the pairs by
+  // expert with the host experts' pairs as one last group E
+  if ((e = launch_hybrid_split(w.ids, P, E, C->slot_of_expert + C->key_base, H->pcie_gbs, H->host_gbs, hw.ids2,
+                               hw.split, cs)) != cudaSuccess)
+    return cuda_fail(e, "split launch");
+  prof_mark(FTM_K_PERMUTE, cs, false);
+  e = launch_permute(hw.ids2, P, E + 1, hw.counts2, hw.offsets2, w.perm, w.inv, hw.perm_ws2, cs);
+  prof_mark(FTM_K_PERMUTE, cs, true);
+  if (e != cudaSuccess) return cuda_fail(e, "permute launch");
+  // what the host needs, read back before the lookup's own read (same stream)
+  struct { void* dst; const void* src; size_t n; } rd[5] = {
+      {hh.split, hw.split, (4 + static_cast<size_t>(E)) * 4}, {hh.ids, w.ids, static_cast<size_t>(P) * 4},
+      {hh.perm, w.perm, static_cast<size_t>(P) * 4}, {hh.offsets, hw.offsets2, (static_cast<size_t>(E) + 2) * 4},
+      {hh.x, x, static_cast<size_t>(T) * row}};
+  for (auto& c : rd)
+    if ((e = cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
+      return cuda_fail(e, "split read-back");
+  // the cache step over the GPU's share: hits and the q copied misses (the
+  // host waits here for the lookup, and with it for the reads above)
+  int misses = 0;
+  if ((s = cache_step(L, C, hw.ids2, P, C->step, w.lru_ws, cs, ps, nullptr, &misses, E))) return s;
+  if (misses > 0) {
+    cudaEvent_t ev = copy_event();
+    if (!ev) return fail(FTM_ERR_CUDA, "could not create the copy event");
+    if ((e = cudaEventRecord(ev, ps)) != cudaSuccess) return cuda_fail(e, "copy event record");
+    if ((e = cudaStreamWaitEvent(cs, ev, 0)) != cudaSuccess) return cuda_fail(e, "copy event wait");
+  }
+  // the GPU's groups (the host experts' groups 0..E-1 are empty)
+  const int32_t* soe = C->slot_of_expert + C->key_base;
+  if ((s = ftm_expert_ffn(L, x, T, hw.offsets2, w.perm, soe, C->slot_pool, W->shared_bank, W->act_scale, w.y, w.ffn_ws,
+                          ffn_ws_bytes(L, T), stream)))
+    return s;
+  // meanwhile the host experts' pairs, positions offsets2[E] .. P-1, on the host
+  const int m = hh.split[0], Hn = hh.split[2], rows = hh.split[3], p0 = hh.offsets[E];
+  if (Hn < 0 || Hn > E || p0 < 0 || p0 + rows != P)
+    return fail(FTM_ERR_CUDA, "%s: inconsistent split (H=%d, rows=%d, first host position %d, P=%d)", who, Hn, rows,
+                p0, P);
+  ftm_bank_layout bl;
+  bank_layout(L, &bl);
+  for (int i = 0; i < E; ++i) hh.gidx[i] = -1;
+  for (int h = 0; h <= Hn; ++h) hh.gpos[h] = 0;
+  for (int h = 0; h < Hn; ++h) hh.gidx[hh.split[4 + h]] = h;
+  for (int p = p0; p < P; ++p) {
+    const int q = hh.perm[p];
+    const int g = (q >= 0 && q < P && hh.ids[q] >= 0 && hh.ids[q] < E) ? hh.gidx[hh.ids[q]] : -1;
+    if (g < 0) return fail(FTM_ERR_CUDA, "%s: position %d of the host group maps to no host expert", who, p);
+    hh.gpos[g + 1] += 1;
+  }
+  for (int h = 0; h < Hn; ++h) hh.gpos[h + 1] += hh.gpos[h];
+  for (int h = 0; h < Hn; ++h) {
+    const int key = C->key_base + hh.split[4 + h];
+    hh.groups[h] = HostGroup{static_cast<const uint8_t*>(C->host_pool) + static_cast<size_t>(key) * bl.bank_bytes, 0,
+                             hh.xrow + hh.gpos[h], hh.yrow + hh.gpos[h]};
+  }
+  for (int p = p0; p < P; ++p) {   // ascending positions: each group's rows in ascending pair order
+    const int q = hh.perm[p], g = hh.gidx[hh.ids[q]];
+    HostGroup& G = hh.groups[g];
+    hh.xrow[hh.gpos[g] + G.n] = hh.x + static_cast<size_t>(q / k) * row;
+    hh.yrow[hh.gpos[g] + G.n] = hh.y + static_cast<size_t>(p - p0) * row;
+    G.n += 1;
+  }
+  const auto t0 = std::chrono::steady_clock::now();
+  host_ffn_groups(L, &bl, hh.groups, Hn, hh.scratch, H->threads);
+  const auto t1 = std::chrono::steady_clock::now();
+  if (rows > 0 && (e = cudaMemcpyAsync(static_cast<uint8_t*>(w.y) + static_cast<size_t>(p0) * row, hh.y,
+                                       static_cast<size_t>(rows) * row, cudaMemcpyHostToDevice, cs)) != cudaSuccess)
+    return cuda_fail(e, "host rows copy");
+  H->last_misses = m;
+  H->last_host = Hn;
+  H->last_host_rows = rows;
+  H->last_host_ms = std::chrono::duration<double, std::milli>(t1 - t0).count();
+  return ftm_combine(L, w.y, w.inv, w.gates, T, out, stream);
+}
 
 }  // extern "C"

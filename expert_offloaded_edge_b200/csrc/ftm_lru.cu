@@ -38,8 +38,10 @@ __device__ __forceinline__ int64_t* lru_backup_lu(int32_t* ws, int E, int S) {
   return reinterpret_cast<int64_t*>(reinterpret_cast<uint8_t*>(ws) + off);
 }
 
+// skip_id >= 0: pairs whose id equals it are not requests (the experts the
+// bandwidth-adaptive split computes on the host carry that id).
 __global__ void __launch_bounds__(kLruThreads) lru_step_kernel(const int32_t* __restrict__ ids, int P, int E, int S,
-                                                               int64_t step, int64_t reserve, int key_base,
+                                                               int64_t step, int64_t reserve, int key_base, int skip_id,
                                                                int32_t* __restrict__ slot_of_key,
                                                                int32_t* __restrict__ key_of_slot,
                                                                int64_t* __restrict__ last_use,
@@ -61,7 +63,7 @@ __global__ void __launch_bounds__(kLruThreads) lru_step_kernel(const int32_t* __
     for (int q = threadIdx.x; q < P; q += blockDim.x) {
       const int e = ids[q];
       if (e >= 0 && e < E) want[e] = 1;
-      else s_bad = 1;
+      else if (e != skip_id) s_bad = 1;
     }
   }
   __syncthreads();
@@ -152,13 +154,94 @@ __global__ void __launch_bounds__(kLruThreads) lru_step_kernel(const int32_t* __
 }
 
 cudaError_t launch_lru_step(const int32_t* ids, int P, int E, int S, int64_t step, int64_t reserve, int key_base,
-                            int32_t* soe, int32_t* eos, int64_t* lu, int32_t* ws, cudaStream_t st) {
+                            int skip_id, int32_t* soe, int32_t* eos, int64_t* lu, int32_t* ws, cudaStream_t st) {
   const size_t smem = sizeof(int32_t) * (2 * static_cast<size_t>(E) + 1 + 2 * S);
   cudaError_t err =
       cudaFuncSetAttribute(lru_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   return launch_pdl(lru_step_kernel, dim3(1), dim3(kLruThreads), smem, st, ids, P, E, S, step, reserve, key_base,
-                    soe, eos, lu, ws);
+                    skip_id, soe, eos, lu, ws);
+}
+
+// ---------------------------------------------------------------------------
+// Bandwidth-adaptive miss split (the pages' q* policy: freelamp.com FreeToken
+// article, section 2.1; chenxutan.com FreeToken article, "choosing among the
+// five MoE backends", `hybrid`).  Of the m experts a step requests that are not
+// resident, q are copied over PCIe and computed on the GPU and m - q are
+// computed on the host from host memory, the two sides overlapped.  With a
+// PCIe bandwidth Bp and a host FFN bandwidth Bh (expert bytes per second each
+// side moves), both sides finish together when q / Bp = (m - q) / Bh, i.e.
+// q = m Bp / (Bp + Bh); q is that value rounded to the nearest integer (halves
+// up), computed in fp64 as floor(m * Bp / (Bp + Bh) + 0.5).  The host takes the
+// m - q misses with the fewest pairs (ties: the lower expert id): its cost per
+// expert grows with the rows, a copy's does not.
+//   ids2[q] = E for a pair of a host expert, else ids[q] (ids outside [0, E)
+//   copied through for the lookup to reject); out (int32): [0] m, [1] q,
+//   [2] host experts H = m - q, [3] their pairs, [4 .. 4+H) the host experts
+//   in order (fewest pairs first).
+// One block; the residency read is the state before the step's lookup.
+__global__ void __launch_bounds__(kLruThreads) hybrid_split_kernel(const int32_t* __restrict__ ids, int P, int E,
+                                                                   const int32_t* __restrict__ soe, double bp,
+                                                                   double bh, int32_t* __restrict__ ids2,
+                                                                   int32_t* __restrict__ out) {
+  extern __shared__ int32_t sm[];
+  int32_t* cnt = sm;          // [E] pairs per expert
+  int32_t* host = sm + E;     // [E] 1: miss (then: host expert)
+  int32_t* rank = sm + 2 * E; // [E] rank of a miss, -1 otherwise
+  __shared__ int32_t s_m, s_h, s_rows;
+  pdl_wait();
+  pdl_trigger();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  if (threadIdx.x == 0) { s_m = 0; s_rows = 0; }
+  __syncthreads();
+  for (int q = threadIdx.x; q < P; q += blockDim.x) {
+    const int e = ids[q];
+    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    host[e] = cnt[e] > 0 && soe[e] < 0;
+    if (host[e]) atomicAdd(&s_m, 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int m = s_m;
+    int q = static_cast<int>(floor(static_cast<double>(m) * bp / (bp + bh) + 0.5));
+    q = q < 0 ? 0 : q > m ? m : q;
+    s_h = m - q;
+  }
+  __syncthreads();
+  const int H = s_h;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {   // rank among the misses by (pairs, id)
+    int r = -1;
+    if (host[e]) {
+      r = 0;
+      for (int f = 0; f < E; ++f)
+        r += (host[f] && (cnt[f] < cnt[e] || (cnt[f] == cnt[e] && f < e))) ? 1 : 0;
+    }
+    rank[e] = r;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int r = rank[e];
+    host[e] = r >= 0 && r < H;
+    if (host[e]) {
+      out[4 + r] = e;
+      atomicAdd(&s_rows, cnt[e]);
+    }
+  }
+  __syncthreads();
+  for (int q = threadIdx.x; q < P; q += blockDim.x) {
+    const int e = ids[q];
+    ids2[q] = (e >= 0 && e < E && host[e]) ? E : e;
+  }
+  if (threadIdx.x == 0) { out[0] = s_m; out[1] = s_m - H; out[2] = H; out[3] = s_rows; }
+}
+
+cudaError_t launch_hybrid_split(const int32_t* ids, int P, int E, const int32_t* soe, double bp, double bh,
+                                int32_t* ids2, int32_t* out, cudaStream_t st) {
+  const size_t smem = sizeof(int32_t) * 3 * static_cast<size_t>(E);
+  return launch_pdl(hybrid_split_kernel, dim3(1), dim3(kLruThreads), smem, st, ids, P, E, soe, bp, bh, ids2, out);
 }
 
 // Rollback of a step whose miss copies could not all be issued: the state

@@ -20,7 +20,9 @@
  *  - Pointers marked "device" are CUDA device pointers, "host" are host
  *    pointers.  The caller owns every buffer; the library never allocates device
  *    or host memory and keeps no per-call state beyond a thread-local error
- *    string and one cached CUDA event per thread for the miss-copy ordering.
+ *    string and one cached CUDA event per thread for the miss-copy ordering
+ *    (and, once the host FFN of the miss split has run, its pool of host
+ *    threads).
  *  - `stream` arguments are cudaStream_t values passed as void* (NULL = the
  *    legacy default stream).  Work is enqueued asynchronously; the entry
  *    points that synchronise the host are the cache steps
@@ -340,6 +342,79 @@ ftm_status ftm_moe_layers_forward(const ftm_layer_desc* L, int32_t n_layers, con
                                   ftm_slot_cache* C, const void* const* x, int32_t T, void* const* out,
                                   int32_t overlap, int32_t* overlapped, void* workspace, size_t ws_bytes,
                                   void* stream, void* copy_stream);
+
+/* Bandwidth-adaptive miss split (the pages' q* policy: freelamp.com FreeToken
+ * article, section 2.1 "bandwidth-adaptive execution"; chenxutan.com FreeToken
+ * article, "choosing among the five MoE backends", `hybrid`, and the bandwidth
+ * calibration `ft bench bw` that feeds it).  Of the m experts a step requests
+ * that are not in the cache, q are copied over PCIe and computed on the GPU,
+ * the other m - q are computed on the host CPU from host memory, both sides at
+ * once.  With Bp the PCIe bandwidth and Bh the host FFN's (expert bytes per
+ * second each side gets through), the two finish together when
+ * q / Bp = (m - q) / Bh:  q = m Bp / (Bp + Bh), rounded to the nearest integer
+ * (halves up), computed in fp64 as floor(m * Bp / (Bp + Bh) + 0.5).  (One page
+ * prints q* = m Bp / Bh, which does not balance the two sides; this library
+ * takes the balanced form the same pages describe in words.)  Bh = 0 gives
+ * q = m (every miss over PCIe, the plain cache step); Bp = 0 gives q = 0.
+ * Returns q, or -1 when m < 0 or the bandwidths are negative, not finite or
+ * both 0.  Host-only, no CUDA call. */
+int32_t ftm_hybrid_split(int32_t m, double pcie_gbs, double host_gbs);
+
+/* Parameters, host buffer and per-call results of ftm_moe_layer_forward_hybrid. */
+typedef struct ftm_hybrid {
+  double pcie_gbs;          /* Bp >= 0 (GB/s of bank copies host -> GPU) */
+  double host_gbs;          /* Bh >= 0 (GB/s of expert banks the host FFN gets through); Bp + Bh > 0 */
+  int32_t threads;          /* host FFN threads (0: every hardware thread) */
+  int32_t last_misses;      /* out: m, requested experts not in the cache */
+  int32_t last_host;        /* out: m - q, of which computed on the host */
+  int32_t last_host_rows;   /* out: (token, pick) pairs computed on the host */
+  double last_host_ms;      /* out: wall time of the host FFN */
+  void* host_ws;            /* host, pinned, 64-byte aligned, >= ftm_hybrid_host_bytes(L, T) bytes */
+  size_t host_ws_bytes;
+} ftm_hybrid;
+
+size_t ftm_hybrid_workspace_bytes(const ftm_layer_desc* L, int32_t T_max);
+size_t ftm_hybrid_host_bytes(const ftm_layer_desc* L, int32_t T_max);
+
+/* The layer with a cache step split by ftm_hybrid_split (fp32, bf16 and FP8
+ * layers; other dtypes return FTM_ERR_UNSUPPORTED).  Sequence:
+ *  1. route on `stream`;
+ *  2. one kernel counts each expert's pairs, finds the misses (against the
+ *     cache state before this step), sets q, and gives the host the m - q
+ *     misses with the fewest pairs (ties: the lower expert id); their pairs are
+ *     relabelled E;
+ *  3. the pairs are permuted over E + 1 groups (group E = the host's pairs, in
+ *     ascending pair order, at positions P - rows .. P - 1);
+ *  4. the cache step of ftm_slot_lookup_update over the remaining requests
+ *     (hits and the q copied misses): the LRU state changes exactly as a plain
+ *     step whose topk_ids held only those experts; the host experts are not
+ *     inserted and their last use is not updated.  The host waits here once;
+ *  5. the GPU expert FFN of every group but E, after the copies;
+ *  6. meanwhile the host computes group E's rows from the banks in
+ *     C->host_pool (the same FFN, FP8 activations quantised per 128 as on the
+ *     GPU, fp32 accumulation; ftm_host_expert_ffn) on H->threads threads, then
+ *     copies them into place on `stream`;
+ *  7. combine, as ftm_moe_layer_forward.
+ * Output rows agree with ftm_moe_layer_forward within the dtype's tolerance
+ * (bit-identical when m - q = 0).  Arguments as ftm_moe_layer_forward with a
+ * cache, plus H; workspace >= ftm_hybrid_workspace_bytes(L, T).  H->host_ws
+ * may be reused once `stream` has passed the call.  Errors as
+ * ftm_slot_lookup_update (state unchanged on capacity / id errors). */
+ftm_status ftm_moe_layer_forward_hybrid(const ftm_layer_desc* L, const ftm_layer_weights* W, ftm_slot_cache* C,
+                                        ftm_hybrid* H, const void* x, int32_t T, void* out, void* workspace,
+                                        size_t ws_bytes, void* stream, void* copy_stream);
+
+/* The host half of the split on its own: one expert's SwiGLU FFN on the CPU.
+ *   bank     host, one expert bank (layout from ftm_get_bank_layout), 16-byte aligned
+ *   x, y     host [n][d] (bf16, fp32 for FTM_F32), row-major
+ *   scratch  host, >= ftm_host_ffn_scratch_bytes(L, n) bytes, 16-byte aligned
+ *   threads  0: every hardware thread
+ * fp32, bf16 and FP8 layers; FP8 quantises x and the SwiGLU output per 128
+ * elements (scale amax / 448, E4M3 round to nearest even), as the GPU path
+ * does.  No CUDA call: runs without a GPU. */
+size_t ftm_host_ffn_scratch_bytes(const ftm_layer_desc* L, int32_t n);
+ftm_status ftm_host_expert_ffn(const ftm_layer_desc* L, const void* bank, const void* x, int32_t n, void* y,
+                               void* scratch, size_t scratch_bytes, int32_t threads);
 
 /* Thread-local warning of the last ftm_moe_layers_forward call ("" if none). */
 const char* ftm_last_warning(void);

@@ -71,6 +71,8 @@ def lib():
         L.orc_lru_step.restype = i32
         L.orc_lru_step_reserve.argtypes = [i32, i32, p, p, p, i64, i64, p, i32, p, p, p, p, p]
         L.orc_lru_step_reserve.restype = i32
+        L.orc_hybrid_split.argtypes = [i32, p, p, ctypes.c_double, ctypes.c_double, p, p, p]
+        L.orc_hybrid_split.restype = i32
         L.orc_lru_resize.argtypes = [i32, i32, p, p, p, i32, p, p, p, p]
         L.orc_lru_resize.restype = i32
         L.orc_expert_ffn.argtypes = [p, i32, i32, i32, p, p, p, i32, p]
@@ -309,6 +311,20 @@ class LRUState:
                                     _p(self.last_use), S_new, _p(n.slot_of_expert), _p(n.expert_of_slot),
                                     _p(n.last_use), _p(mf))
         return n, mf[:kept].copy()
+
+
+def hybrid_split(counts: np.ndarray, resident: np.ndarray, bp: float, bh: float):
+    """Bandwidth-adaptive miss split (see orc_hybrid_split).  counts: pairs per
+    expert; resident: nonzero where the expert is in the cache.  Returns
+    (m, q, host experts in order)."""
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    resident = np.ascontiguousarray(resident, dtype=np.int32)
+    E = counts.size
+    host = np.empty(max(1, E), dtype=np.int32)
+    m, q = np.zeros(1, dtype=np.int32), np.zeros(1, dtype=np.int32)
+    n = lib().orc_hybrid_split(E, _p(counts), _p(resident), ctypes.c_double(bp), ctypes.c_double(bh), _p(host),
+                               _p(m), _p(q))
+    return int(m[0]), int(q[0]), [int(v) for v in host[:n]]
 
 
 # ---- expert FFN / combine -----------------------------------------------------------

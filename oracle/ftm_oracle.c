@@ -415,6 +415,48 @@ int orc_lru_step(int E, int S, int32_t* slot_of_expert, int32_t* expert_of_slot,
 }
 
 /* ---------------------------------------------------------------------------
+ * Bandwidth-adaptive miss split (freelamp.com FreeToken article, section 2.1
+ * "bandwidth-adaptive execution": the machine's measured PCIe bandwidth Bp and
+ * host bandwidth Bh set how many of a step's m cache misses are copied to the
+ * GPU and how many are computed on the CPU, the two running at once;
+ * chenxutan.com FreeToken article, "choosing among the five MoE backends",
+ * `hybrid`: the misses are split by the bandwidth ratio so that both sides
+ * finish together).  Both sides move one expert bank per miss, so they finish
+ * together when q / Bp = (m - q) / Bh:  q = m Bp / (Bp + Bh), taken to the
+ * nearest integer, halves up, in fp64: floor(m * Bp / (Bp + Bh) + 0.5).  (The
+ * printed formula q* = m Bp / Bh does not balance the two sides the text
+ * describes; the balanced form is the reading.)  Which m - q misses go to the
+ * host is not said: read as those with the fewest routed pairs (the host's
+ * cost per expert grows with its rows, a copy's does not), ties to the lower
+ * expert id.
+ *   counts[E]   pairs routed to each expert this step
+ *   resident[E] nonzero: expert in the cache (a hit)
+ *   host[]      out: the host's experts, fewest pairs first (at most E)
+ * Returns m - q; *m_out = m, *q_out = q.  Selection by repeated minimum.
+ * ------------------------------------------------------------------------- */
+int orc_hybrid_split(int E, const int32_t* counts, const int32_t* resident, double bp, double bh, int32_t* host,
+                     int32_t* m_out, int32_t* q_out) {
+  int m = 0;
+  for (int e = 0; e < E; ++e)
+    if (counts[e] > 0 && !resident[e]) ++m;
+  int q = (int)floor((double)m * bp / (bp + bh) + 0.5);
+  if (q < 0) q = 0;
+  if (q > m) q = m;
+  uint8_t* taken = (uint8_t*)calloc((size_t)E + 1, 1);
+  for (int i = 0; i < m - q; ++i) {
+    int best = -1;
+    for (int e = 0; e < E; ++e)
+      if (counts[e] > 0 && !resident[e] && !taken[e] && (best < 0 || counts[e] < counts[best])) best = e;
+    taken[best] = 1;
+    host[i] = best;
+  }
+  free(taken);
+  *m_out = m;
+  *q_out = q;
+  return m - q;
+}
+
+/* ---------------------------------------------------------------------------
  * Cache step of a cache shared by several layers, with slots held back.
  * Keys: the cache holds n_keys entries; in a cache shared by several layers of
  * E experts each, layer l's expert e is key l*E + e.  Step s requests the

@@ -1,0 +1,170 @@
+"""The bandwidth-adaptive miss split (the pages' q* policy), on the CPU.
+
+Oracle pins (orc_hybrid_split), from outside the oracle:
+  - the hand-worked case of the docstring example below;
+  - q against a brute-force search over every q' in [0, m] for the one that
+    balances the two sides best (|q'(Bp + Bh) - m Bp| smallest, halves to the
+    larger q');
+  - the endpoints Bh = 0 (every miss over PCIe) and Bp = 0 (every miss on the
+    host) and the invariants of the choice: host experts are misses, the host's
+    (pairs, id) all precede the GPU misses', in that order.
+Library against the oracle, no GPU needed: ftm_hybrid_split's q, and the
+host expert FFN (ftm_host_expert_ffn) for fp32, bf16 and FP8 banks against the
+oracle's expert FFN in the same activation mode.
+"""
+import itertools
+
+import numpy as np
+import pytest
+
+import expert_offloaded_edge_b200 as ftm
+import oracle
+import synth
+from expert_offloaded_edge_b200.layout import pack_bank
+
+
+def test_split_hand_worked():
+    # experts 0..5 with 3, 0, 1, 2, 1, 5 pairs; expert 3 is cached.  Misses:
+    # 0 (3 pairs), 2 (1), 4 (1), 5 (5): m = 4.  Bp = Bh: q = floor(2 + 0.5) = 2,
+    # the host takes the two with the fewest pairs: 2 and 4 (1 pair each, the
+    # lower id first).  Bp = 52.7, Bh = 77.3 (the pages' `ft bench bw` example):
+    # 4 * 52.7 / 130 = 1.62 -> q = 2.  Bp = 3 Bh: 3 -> q = 3, host = [2].
+    counts = np.array([3, 0, 1, 2, 1, 5])
+    resident = np.array([0, 0, 0, 1, 0, 0])
+    assert oracle.hybrid_split(counts, resident, 1.0, 1.0) == (4, 2, [2, 4])
+    assert oracle.hybrid_split(counts, resident, 52.7, 77.3) == (4, 2, [2, 4])
+    assert oracle.hybrid_split(counts, resident, 3.0, 1.0) == (4, 3, [2])
+    # Bh = 0: all over PCIe; Bp = 0: all on the host, fewest pairs first
+    assert oracle.hybrid_split(counts, resident, 1.0, 0.0) == (4, 4, [])
+    assert oracle.hybrid_split(counts, resident, 0.0, 1.0) == (4, 0, [2, 4, 0, 5])
+
+
+def _brute_q(m, bp, bh):
+    best, bq = None, None
+    for q in range(m + 1):
+        dev = abs(q * (bp + bh) - m * bp)
+        if best is None or dev < best - 1e-12 or (abs(dev - best) <= 1e-12 and q > bq):
+            best, bq = dev, q
+    return bq
+
+
+def test_split_q_balances_the_two_sides_brute_force():
+    rng = np.random.default_rng(1)
+    for _ in range(400):
+        E = int(rng.integers(1, 40))
+        counts = rng.integers(0, 5, size=E)
+        resident = rng.integers(0, 2, size=E)
+        bp, bh = (float(v) for v in rng.uniform(0.0, 100.0, size=2))
+        m, q, host = oracle.hybrid_split(counts, resident, bp, bh)
+        assert m == int(np.sum((counts > 0) & (resident == 0)))
+        assert q == _brute_q(m, bp, bh), (m, bp, bh, q)
+        assert len(host) == m - q
+        # the library's split takes the same decision in the same precision
+        assert ftm.ftm_hybrid_split(m, bp, bh) == q
+
+
+def test_split_choice_invariants_and_brute_force():
+    rng = np.random.default_rng(2)
+    for _ in range(200):
+        E = int(rng.integers(1, 9))
+        counts = rng.integers(0, 4, size=E)
+        resident = rng.integers(0, 2, size=E)
+        bp, bh = (float(v) for v in rng.uniform(0.0, 10.0, size=2))
+        m, q, host = oracle.hybrid_split(counts, resident, bp, bh)
+        misses = [e for e in range(E) if counts[e] > 0 and not resident[e]]
+        assert set(host) <= set(misses) and len(set(host)) == len(host)
+        gpu = [e for e in misses if e not in host]
+        key = lambda e: (int(counts[e]), e)   # noqa: E731
+        assert [key(e) for e in host] == sorted(key(e) for e in host)
+        if host and gpu:
+            assert max(key(e) for e in host) < min(key(e) for e in gpu)
+        # brute force: of every subset of m - q misses, the host's has the fewest
+        # pairs, and among those the smallest sorted id list
+        best = min(itertools.combinations(misses, m - q), key=lambda c: (sum(int(counts[e]) for e in c), sorted(c)))
+        assert sorted(host) == sorted(best)
+
+
+def test_library_split_endpoints_and_errors():
+    assert ftm.ftm_hybrid_split(7, 1.0, 0.0) == 7
+    assert ftm.ftm_hybrid_split(7, 0.0, 1.0) == 0
+    assert ftm.ftm_hybrid_split(0, 1.0, 1.0) == 0
+    assert ftm.ftm_hybrid_split(5, 1.0, 1.0) == 3   # 2.5 rounds half up
+    for bad in ((3, 0.0, 0.0), (3, -1.0, 1.0), (3, float("nan"), 1.0), (3, float("inf"), 1.0), (-1, 1.0, 1.0)):
+        assert ftm.ftm_hybrid_split(*bad) == -1
+
+
+def _aligned(nbytes, align=64):
+    buf = np.zeros(nbytes + align, dtype=np.uint8)
+    off = (-buf.ctypes.data) % align
+    return buf[off:off + nbytes]
+
+
+HOST_CFGS = {
+    "f32": synth.scaled(synth.CONFIGS["tiny"], name="host_f32", d=128, I=128, E=4, k=2, S=4, has_shared=0),
+    "bf16": synth.scaled(synth.CONFIGS["35b_decode"], name="host_bf16", d=256, I=128, E=4, k=2, S=4, has_shared=0),
+    "fp8": synth.scaled(synth.CONFIGS["284b_trace"], name="host_fp8", d=256, I=256, E=4, k=2, S=4, has_shared=0,
+                        lru=False, bias="uniform", T=(8,), trace_steps=1),
+}
+HOST_TOL = {"f32": 1e-4, "bf16": 2e-2, "fp8": 5e-2}
+
+
+@pytest.mark.parametrize("wdtype", ["f32", "bf16", "fp8"])
+@pytest.mark.parametrize("n", [1, 5])
+def test_host_expert_ffn_matches_oracle(wdtype, n):
+    cfg = HOST_CFGS[wdtype]
+    layer = synth.Layer(cfg, 0)
+    desc = ftm.desc_for(cfg)
+    bl = ftm.ftm_get_bank_layout(desc)
+    e = 2
+    bank = _aligned(bl.bank_bytes)
+    pack_bank(desc, layer.expert(e), bl, out=bank)
+    xs = layer.hidden_storage(n, 0)                  # bf16 bits, or fp32 for f32 layers
+    x = np.ascontiguousarray(xs)
+    y = np.zeros_like(x)
+    nb = ftm.ftm_host_ffn_scratch_bytes(desc, n)
+    scratch = _aligned(nb)
+    ftm.ftm_host_expert_ffn(desc, bank, x, n, y, scratch, nb, threads=3)
+    xf = x.astype(np.float32) if wdtype == "f32" else oracle.bf16_to_f32(x)
+    yf = y.astype(np.float32) if wdtype == "f32" else oracle.bf16_to_f32(y)
+    Wg, Wu, Wd = oracle.expert_weights_f32(layer, e)
+    want = oracle.expert_ffn(xf, Wg, Wu, Wd, oracle.qa_mode(wdtype))
+    for r in range(n):
+        err = float(np.max(np.abs(yf[r] - want[r])))
+        scale = float(np.max(np.abs(want[r])))
+        assert err <= HOST_TOL[wdtype] * scale, (wdtype, r, err, scale)
+    if wdtype == "fp8":
+        # the activation quantisation is applied: without it the result moves
+        plain = oracle.expert_ffn(xf, Wg, Wu, Wd, oracle.QA_NONE)
+        assert not np.allclose(want, plain, rtol=0, atol=1e-6)
+    # the thread count does not change a value (each output element is one thread's sum)
+    y1 = np.zeros_like(x)
+    ftm.ftm_host_expert_ffn(desc, bank, x, n, y1, scratch, nb, threads=1)
+    assert np.array_equal(y, y1)
+
+
+def test_host_ffn_rejects_block_scaled_fp4_and_short_scratch():
+    cfg = synth.CONFIGS["753b_nvfp4"]
+    desc = ftm.desc_for(cfg)
+    with pytest.raises(ftm.FtmError) as ei:
+        ftm.ftm_host_expert_ffn(desc, 16, 16, 1, 16, 16, 1 << 20)
+    assert ei.value.status == ftm.binding.FTM_ERR_UNSUPPORTED
+    cfg = HOST_CFGS["bf16"]
+    desc = ftm.desc_for(cfg)
+    nb = ftm.ftm_host_ffn_scratch_bytes(desc, 2)
+    assert nb == 2 * (cfg.d + cfg.I) * 4
+    with pytest.raises(ftm.FtmError) as ei:
+        ftm.ftm_host_expert_ffn(desc, 64, 64, 2, 64, 64, nb - 1)
+    assert ei.value.status == ftm.binding.FTM_ERR_INVALID_ARG
+
+
+def test_hybrid_layer_rejects_fp4_before_any_device_call():
+    cfg = synth.CONFIGS["753b_nvfp4"]
+    desc = ftm.desc_for(cfg)
+    h = ftm.Hybrid(1.0, 1.0, 0)
+    with pytest.raises(ftm.FtmError) as ei:
+        ftm.ftm_moe_layer_forward_hybrid(desc, ftm.LayerWeights(16), ftm.SlotCache(), h, 16, 1, 16, 16, 0, 1, 1)
+    assert ei.value.status == ftm.binding.FTM_ERR_UNSUPPORTED
+    h = ftm.Hybrid(0.0, 0.0, 0)
+    with pytest.raises(ftm.FtmError) as ei:
+        ftm.ftm_moe_layer_forward_hybrid(desc, ftm.LayerWeights(16), ftm.SlotCache(), h, 16, 1, 16, 16, 0, 1, 1)
+    assert ei.value.status == ftm.binding.FTM_ERR_INVALID_ARG
