@@ -19,6 +19,7 @@
 #include <cstdint>
 #include <cstring>
 #include <functional>
+#include <immintrin.h>
 #include <mutex>
 #include <thread>
 #include <vector>
@@ -127,11 +128,85 @@ void convert_e4m3(const uint8_t* w, float* out) {
   }
 }
 
+// ---- AVX2 + FMA path (chosen at run time) ----------------------------------------
+// 8 weights per vector: E4M3 codes widened to 32 bits and rebuilt as fp32 with
+// the same bit rule as convert_e4m3 (normal codes by integer shift and add,
+// exponent field 0 as m * 2^-9 by a convert and multiply, then the sign);
+// bf16 by a 16-bit shift.
+__attribute__((target("avx2,fma"))) inline __m256 e4m3x8(const uint8_t* p) {
+  const __m256i v = _mm256_cvtepu8_epi32(_mm_loadl_epi64(reinterpret_cast<const __m128i*>(p)));
+  const __m256i em = _mm256_and_si256(v, _mm256_set1_epi32(0x7F));
+  const __m256 normal =
+      _mm256_castsi256_ps(_mm256_add_epi32(_mm256_slli_epi32(em, 20), _mm256_set1_epi32(120 << 23)));
+  const __m256 sub = _mm256_mul_ps(_mm256_cvtepi32_ps(em), _mm256_set1_ps(0x1p-9f));
+  const __m256 isn = _mm256_castsi256_ps(_mm256_cmpgt_epi32(em, _mm256_set1_epi32(7)));
+  const __m256 val = _mm256_blendv_ps(sub, normal, isn);
+  const __m256i sign = _mm256_slli_epi32(_mm256_and_si256(v, _mm256_set1_epi32(0x80)), 24);
+  return _mm256_or_ps(val, _mm256_castsi256_ps(sign));
+}
+
+__attribute__((target("avx2,fma"))) inline __m256 bf16x8(const uint8_t* p) {
+  const __m256i v = _mm256_cvtepu16_epi32(_mm_loadu_si128(reinterpret_cast<const __m128i*>(p)));
+  return _mm256_castsi256_ps(_mm256_slli_epi32(v, 16));
+}
+
+__attribute__((target("avx2,fma"))) inline float hsum8(__m256 v) {
+  const __m128 s = _mm_add_ps(_mm256_castps256_ps128(v), _mm256_extractf128_ps(v, 1));
+  const __m128 t = _mm_add_ps(s, _mm_movehl_ps(s, s));
+  return _mm_cvtss_f32(_mm_add_ss(t, _mm_shuffle_ps(t, t, 1)));
+}
+
+// NR (1..4) activation rows per pass: each block of 128 weights is decoded
+// once and multiplied into every row's accumulators in registers, two
+// independent accumulators per row so consecutive FMAs do not wait on each
+// other.
+template <bool FP8, int NR>
+__attribute__((target("avx2,fma"))) void dot_rows_avx2(const uint8_t* w, const float* sc, int K, const float* x,
+                                                       int ldx, float* out) {
+  constexpr int kEb = FP8 ? 1 : 2;   // bytes per weight
+  float tot[NR] = {};
+  for (int c0 = 0; c0 < K; c0 += 128) {
+    __m256 a0[NR], a1[NR];
+    for (int r = 0; r < NR; ++r) a0[r] = a1[r] = _mm256_setzero_ps();
+    for (int c = c0; c < c0 + 128; c += 16) {
+      const __m256 w0 = FP8 ? e4m3x8(w + c) : bf16x8(w + static_cast<size_t>(c) * kEb);
+      const __m256 w1 = FP8 ? e4m3x8(w + c + 8) : bf16x8(w + static_cast<size_t>(c + 8) * kEb);
+      for (int r = 0; r < NR; ++r) {
+        a0[r] = _mm256_fmadd_ps(w0, _mm256_loadu_ps(x + static_cast<size_t>(r) * ldx + c), a0[r]);
+        a1[r] = _mm256_fmadd_ps(w1, _mm256_loadu_ps(x + static_cast<size_t>(r) * ldx + c + 8), a1[r]);
+      }
+    }
+    const float s = FP8 ? sc[c0 / 128] : 1.0f;
+    for (int r = 0; r < NR; ++r) tot[r] += s * hsum8(_mm256_add_ps(a0[r], a1[r]));
+  }
+  for (int r = 0; r < NR; ++r) out[r] = tot[r];
+}
+
+template <bool FP8>
+void dot_row_avx2(const uint8_t* w, const float* sc, int K, const float* x, int ldx, int n, float* out) {
+  for (int r0 = 0; r0 < n; r0 += 4) {
+    const float* xr = x + static_cast<size_t>(r0) * ldx;
+    switch (n - r0 < 4 ? n - r0 : 4) {
+      case 1: dot_rows_avx2<FP8, 1>(w, sc, K, xr, ldx, out + r0); break;
+      case 2: dot_rows_avx2<FP8, 2>(w, sc, K, xr, ldx, out + r0); break;
+      case 3: dot_rows_avx2<FP8, 3>(w, sc, K, xr, ldx, out + r0); break;
+      default: dot_rows_avx2<FP8, 4>(w, sc, K, xr, ldx, out + r0); break;
+    }
+  }
+}
+
+const bool g_avx2 = __builtin_cpu_supports("avx2") && __builtin_cpu_supports("fma");
+
 // out[r] = sum_c W[row][c] * x[r][c] for one row of a weight matrix with K
 // columns.  `sc` = the row's fp32 block scales (FP8), one per 128 columns.
 void dot_row(int wdtype, const uint8_t* wrow, const float* sc, int K, const float* x, int ldx, int n, float* out) {
   if (wdtype == FTM_F32) {
     dot_f32(reinterpret_cast<const float*>(wrow), K, x, ldx, n, out);
+    return;
+  }
+  if (g_avx2) {
+    if (wdtype == FTM_FP8_E4M3_B128) dot_row_avx2<true>(wrow, sc, K, x, ldx, n, out);
+    else dot_row_avx2<false>(wrow, sc, K, x, ldx, n, out);
     return;
   }
   for (int r = 0; r < n; ++r) out[r] = 0.0f;
