@@ -103,7 +103,7 @@ def library() -> ctypes.CDLL:
         for name in ("ftm_hybrid_workspace_bytes", "ftm_hybrid_host_bytes", "ftm_host_ffn_scratch_bytes"):
             getattr(L, name).argtypes = [P(LayerDesc), c_i32]
             getattr(L, name).restype = c_sz
-        L.ftm_host_expert_ffn.argtypes = [P(LayerDesc), c_p, c_p, c_i32, c_p, c_p, c_sz, c_i32]
+        L.ftm_host_expert_ffn.argtypes = [P(LayerDesc), c_p, c_p, c_i32, c_p, c_p, c_p, c_sz, c_i32]
         L.ftm_moe_layer_forward_hybrid.argtypes = [P(LayerDesc), P(LayerWeights), P(SlotCache), P(Hybrid), c_p,
                                                    c_i32, c_p, c_p, c_sz, c_p, c_p]
         for name in ("ftm_get_bank_layout", "ftm_route", "ftm_permute", "ftm_slot_lookup_update", "ftm_slot_resize",
@@ -290,10 +290,11 @@ def ftm_host_ffn_scratch_bytes(desc, n) -> int:
     return int(library().ftm_host_ffn_scratch_bytes(ctypes.byref(desc), n))
 
 
-def ftm_host_expert_ffn(desc, bank, x, n, y, scratch, scratch_bytes, threads: int = 0):
-    """One expert's FFN on the host (host buffers: numpy arrays, CPU tensors or addresses)."""
-    _check(library().ftm_host_expert_ffn(ctypes.byref(desc), _ptr(bank), _ptr(x), n, _ptr(y), _ptr(scratch),
-                                         scratch_bytes, threads))
+def ftm_host_expert_ffn(desc, bank, x, n, y, scratch, scratch_bytes, threads: int = 0, act_scale=None):
+    """One expert's FFN on the host (host buffers: numpy arrays, CPU tensors or addresses;
+    act_scale: host fp32[2] NVFP4 activation global scales or None)."""
+    _check(library().ftm_host_expert_ffn(ctypes.byref(desc), _ptr(bank), _ptr(x), n, _ptr(y), _ptr(act_scale),
+                                         _ptr(scratch), scratch_bytes, threads))
 
 
 def ftm_moe_layer_forward_hybrid(desc, weights: LayerWeights, cache: SlotCache, hybrid: Hybrid, x, T, out, workspace,

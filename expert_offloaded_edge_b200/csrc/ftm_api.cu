@@ -213,6 +213,7 @@ struct HybridHost {
   HostGroup* groups;       // [E]
   int32_t* gidx;           // [E] host group of an expert, -1
   int32_t* gpos;           // [E + 1] first row of each host group
+  float* act;              // [2] NVFP4 activation global scales
   size_t total;
 };
 
@@ -235,6 +236,7 @@ HybridHost carve_host(const ftm_layer_desc* L, int32_t T, void* base_v) {
   h.groups = reinterpret_cast<HostGroup*>(take(E * sizeof(HostGroup)));
   h.gidx = reinterpret_cast<int32_t*>(take(E * 4));
   h.gpos = reinterpret_cast<int32_t*>(take((E + 1) * 4));
+  h.act = reinterpret_cast<float*>(take(2 * sizeof(float)));
   h.total = off;
   return h;
 }
@@ -770,11 +772,11 @@ size_t ftm_host_ffn_scratch_bytes(const ftm_layer_desc* L, int32_t n) {
 }
 
 ftm_status ftm_host_expert_ffn(const ftm_layer_desc* L, const void* bank, const void* x, int32_t n, void* y,
-                               void* scratch, size_t scratch_bytes, int32_t threads) {
+                               const float* act_scale, void* scratch, size_t scratch_bytes, int32_t threads) {
   ftm_status s = check_desc(L);
   if (s) return s;
   if (!host_ffn_supported(L->wdtype))
-    return fail(FTM_ERR_UNSUPPORTED, "ftm_host_expert_ffn: the host FFN handles fp32, bf16 and FP8 banks");
+    return fail(FTM_ERR_UNSUPPORTED, "ftm_host_expert_ffn: no host FFN for wdtype %d", L->wdtype);
   if (n < 0) return fail(FTM_ERR_INVALID_ARG, "ftm_host_expert_ffn: n=%d is negative", n);
   if (n == 0) return ok();
   if (!bank || !x || !y || !scratch) return fail(FTM_ERR_INVALID_ARG, "ftm_host_expert_ffn: NULL pointer");
@@ -793,7 +795,7 @@ ftm_status ftm_host_expert_ffn(const ftm_layer_desc* L, const void* bank, const 
     yr[r] = static_cast<uint8_t*>(y) + r * row;
   }
   HostGroup g{static_cast<const uint8_t*>(bank), n, xr.data(), yr.data()};
-  host_ffn_groups(L, &bl, &g, 1, static_cast<float*>(scratch), threads);
+  host_ffn_groups(L, &bl, &g, 1, act_scale, static_cast<float*>(scratch), threads);
   return ok();
 }
 
@@ -808,8 +810,7 @@ ftm_status ftm_moe_layer_forward_hybrid(const ftm_layer_desc* L, const ftm_layer
   if (ftm_hybrid_split(0, H->pcie_gbs, H->host_gbs) < 0)
     return fail(FTM_ERR_INVALID_ARG, "%s: bandwidths must be finite, >= 0 and not both 0 (Bp=%g, Bh=%g)", who,
                 H->pcie_gbs, H->host_gbs);
-  if (!host_ffn_supported(L->wdtype))
-    return fail(FTM_ERR_UNSUPPORTED, "%s: the host FFN handles fp32, bf16 and FP8 banks", who);
+  if (!host_ffn_supported(L->wdtype)) return fail(FTM_ERR_UNSUPPORTED, "%s: no host FFN for wdtype %d", who, L->wdtype);
   if ((s = check_cache(L, C, who))) return s;
   if (T == 0) return ok();
   if (!x || !out) return fail(FTM_ERR_INVALID_ARG, "%s: NULL x / out", who);
@@ -840,12 +841,13 @@ ftm_status ftm_moe_layer_forward_hybrid(const ftm_layer_desc* L, const ftm_layer
   prof_mark(FTM_K_PERMUTE, cs, true);
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   // what the host needs, read back before the lookup's own read (same stream)
-  struct { void* dst; const void* src; size_t n; } rd[5] = {
+  const bool gscale = L->wdtype == FTM_NVFP4 && W->act_scale;   // the NVFP4 activation global scales
+  struct { void* dst; const void* src; size_t n; } rd[6] = {
       {hh.split, hw.split, (4 + static_cast<size_t>(E)) * 4}, {hh.ids, w.ids, static_cast<size_t>(P) * 4},
       {hh.perm, w.perm, static_cast<size_t>(P) * 4}, {hh.offsets, hw.offsets2, (static_cast<size_t>(E) + 2) * 4},
-      {hh.x, x, static_cast<size_t>(T) * row}};
+      {hh.x, x, static_cast<size_t>(T) * row}, {hh.act, W->act_scale, gscale ? 2 * sizeof(float) : 0}};
   for (auto& c : rd)
-    if ((e = cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
+    if (c.n && (e = cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
       return cuda_fail(e, "split read-back");
   // the cache step over the GPU's share: hits and the q copied misses (the
   // host waits here for the lookup, and with it for the reads above)
@@ -892,7 +894,7 @@ ftm_status ftm_moe_layer_forward_hybrid(const ftm_layer_desc* L, const ftm_layer
     G.n += 1;
   }
   const auto t0 = std::chrono::steady_clock::now();
-  host_ffn_groups(L, &bl, hh.groups, Hn, hh.scratch, H->threads);
+  host_ffn_groups(L, &bl, hh.groups, Hn, gscale ? hh.act : nullptr, hh.scratch, H->threads);
   const auto t1 = std::chrono::steady_clock::now();
   if (rows > 0 && (e = cudaMemcpyAsync(static_cast<uint8_t*>(w.y) + static_cast<size_t>(p0) * row, hh.y,
                                        static_cast<size_t>(rows) * row, cudaMemcpyHostToDevice, cs)) != cudaSuccess)

@@ -82,6 +82,83 @@ void quant_fp8_row(float* v, int K) {
   }
 }
 
+// E2M1 magnitudes by code (1 sign, 2 exponent bits with bias 1, 1 mantissa bit).
+constexpr float kE2m1[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+
+// Nearest E2M1 magnitude of a >= 0, ties to the even code, saturating at 6.
+// The midpoints between neighbours are 0.25, 0.75, 1.25, 1.75, 2.5, 3.5 and 5;
+// at a midpoint the even code (0, 1, 1, 2, 2, 4, 4) wins.
+inline float e2m1_round(float a) {
+  if (a <= 0.25f) return 0.0f;
+  if (a < 0.75f) return 0.5f;
+  if (a <= 1.25f) return 1.0f;
+  if (a < 1.75f) return 1.5f;
+  if (a <= 2.5f) return 2.0f;
+  if (a < 3.5f) return 3.0f;
+  if (a <= 5.0f) return 4.0f;
+  return 6.0f;
+}
+
+// NVFP4 activation quantisation of one row, in place: groups of 16 with the
+// per-tensor global scale g: s16 = e4m3(amax / (6 g)), u = s16 * g,
+// v <- e2m1(v / u) * u (a group with u = 0 becomes zero).
+void quant_nvfp4_row(float* v, int K, float g) {
+  const float six_g = 6.0f * g;
+  for (int b = 0; b < K; b += 16) {
+    float amax = 0.0f;
+    for (int j = 0; j < 16; ++j) amax = std::fmax(amax, std::fabs(v[b + j]));
+    const float u = e4m3_round(amax / six_g) * g;
+    for (int j = 0; j < 16; ++j) {
+      if (u == 0.0f) { v[b + j] = 0.0f; continue; }
+      const float q = v[b + j] / u;
+      const float r = e2m1_round(std::fabs(q));
+      v[b + j] = (q < 0.0f ? -r : r) * u;
+    }
+  }
+}
+
+// MXFP4 activation quantisation of one row, in place (OCP MX): groups of 32
+// share X = 2^e, e = floor(log2 amax) - 2 clamped to [-127, 127] (floor(log2)
+// read exactly from frexp); v <- e2m1(v / X) * X.  An all-zero group stays zero.
+void quant_mx_row(float* v, int K) {
+  for (int b = 0; b < K; b += 32) {
+    float amax = 0.0f;
+    for (int j = 0; j < 32; ++j) amax = std::fmax(amax, std::fabs(v[b + j]));
+    if (amax == 0.0f) continue;
+    int k;
+    std::frexp(amax, &k);                 // amax in [2^(k-1), 2^k)
+    int e = (k - 1) - 2;
+    e = e < -127 ? -127 : e > 127 ? 127 : e;
+    const double X = std::ldexp(1.0, e);  // 2^-127 is below fp32's range: scale in double
+    for (int j = 0; j < 32; ++j) {
+      const float q = static_cast<float>(v[b + j] / X);
+      const float r = e2m1_round(std::fabs(q));
+      v[b + j] = static_cast<float>((q < 0.0f ? -r : r) * X);
+    }
+  }
+}
+
+// Per-group fp32 scales of one weight row of an NVFP4 / MXFP4 bank, read
+// through the 512-byte chunk layout: chunk (row block rb, column block kb) of
+// four scale groups at (rb * nkb + kb) * 512, the scale of local row r for its
+// group j at byte (r % 32) * 16 + (r / 32) * 4 + j.  `r_in_block` and `rb` are
+// the row's place in that layout (gate/up rows in paired order).  NVFP4:
+// e4m3(code) * s_t; MXFP4: 2^(code - 127).
+void fp4_row_scales(const uint8_t* chunks, int rb, int r_in_block, int K, bool mx, float s_t, float* out) {
+  const int group = mx ? 32 : 16;
+  const int ng = K / group, nkb = ng / 4;
+  const uint8_t* base = chunks + static_cast<size_t>(rb) * nkb * 512 + (r_in_block % 32) * 16 + (r_in_block / 32) * 4;
+  for (int gi = 0; gi < ng; ++gi) {
+    const uint8_t c = base[static_cast<size_t>(gi / 4) * 512 + gi % 4];
+    if (mx) out[gi] = static_cast<float>(std::ldexp(1.0, static_cast<int>(c) - 127));
+    else {
+      const uint32_t em = c & 0x7Fu;
+      const float mag = (em >> 3) ? bits_f32((em << 20) + (120u << 23)) : static_cast<float>(em) * 0x1p-9f;
+      out[gi] = ((c & 0x80u) ? -mag : mag) * s_t;
+    }
+  }
+}
+
 // ---- dot products of one weight row with n activation rows ---------------------
 // Eight partial sums per row so the compiler can keep them in one vector.
 __attribute__((target_clones("arch=haswell", "default")))
@@ -195,11 +272,77 @@ void dot_row_avx2(const uint8_t* w, const float* sc, int K, const float* x, int 
   }
 }
 
+// 8 packed E2M1 codes (4 bytes, element 2j in the low nibble of byte j): lane l
+// takes bits 4l..4l+3 of the little-endian word, the magnitude from the
+// 8-entry table, the sign from the code's top bit.
+__attribute__((target("avx2,fma"))) inline __m256 e2m1x8(const uint8_t* p) {
+  uint32_t word;
+  std::memcpy(&word, p, 4);
+  const __m256i nib = _mm256_and_si256(
+      _mm256_srlv_epi32(_mm256_set1_epi32(static_cast<int>(word)), _mm256_setr_epi32(0, 4, 8, 12, 16, 20, 24, 28)),
+      _mm256_set1_epi32(0xF));
+  const __m256 mag = _mm256_permutevar8x32_ps(_mm256_loadu_ps(kE2m1), _mm256_and_si256(nib, _mm256_set1_epi32(7)));
+  const __m256i sign = _mm256_slli_epi32(_mm256_and_si256(nib, _mm256_set1_epi32(8)), 28);
+  return _mm256_or_ps(mag, _mm256_castsi256_ps(sign));
+}
+
+// FP4 rows: each group of `group` weights (16 NVFP4, 32 MXFP4) decoded and
+// multiplied by its scale once, then into every row's accumulators.
+template <int NR>
+__attribute__((target("avx2,fma"))) void dot_rows_fp4_avx2(const uint8_t* w, const float* sc, int K, int group,
+                                                           const float* x, int ldx, float* out) {
+  __m256 a0[NR], a1[NR];
+  for (int r = 0; r < NR; ++r) a0[r] = a1[r] = _mm256_setzero_ps();
+  for (int c = 0; c < K; c += 16) {
+    const __m256 s = _mm256_set1_ps(sc[c / group]);
+    const __m256 w0 = _mm256_mul_ps(e2m1x8(w + c / 2), s);
+    const __m256 w1 = _mm256_mul_ps(e2m1x8(w + c / 2 + 4), s);
+    for (int r = 0; r < NR; ++r) {
+      a0[r] = _mm256_fmadd_ps(w0, _mm256_loadu_ps(x + static_cast<size_t>(r) * ldx + c), a0[r]);
+      a1[r] = _mm256_fmadd_ps(w1, _mm256_loadu_ps(x + static_cast<size_t>(r) * ldx + c + 8), a1[r]);
+    }
+  }
+  for (int r = 0; r < NR; ++r) out[r] = hsum8(_mm256_add_ps(a0[r], a1[r]));
+}
+
+void dot_row_fp4_avx2(const uint8_t* w, const float* sc, int K, int group, const float* x, int ldx, int n,
+                      float* out) {
+  for (int r0 = 0; r0 < n; r0 += 4) {
+    const float* xr = x + static_cast<size_t>(r0) * ldx;
+    switch (n - r0 < 4 ? n - r0 : 4) {
+      case 1: dot_rows_fp4_avx2<1>(w, sc, K, group, xr, ldx, out + r0); break;
+      case 2: dot_rows_fp4_avx2<2>(w, sc, K, group, xr, ldx, out + r0); break;
+      case 3: dot_rows_fp4_avx2<3>(w, sc, K, group, xr, ldx, out + r0); break;
+      default: dot_rows_fp4_avx2<4>(w, sc, K, group, xr, ldx, out + r0); break;
+    }
+  }
+}
+
 const bool g_avx2 = __builtin_cpu_supports("avx2") && __builtin_cpu_supports("fma");
 
 // out[r] = sum_c W[row][c] * x[r][c] for one row of a weight matrix with K
-// columns.  `sc` = the row's fp32 block scales (FP8), one per 128 columns.
+// columns.  `sc` = the row's fp32 scales: FP8 one per 128-column block, NVFP4
+// one per 16 columns (s_t included), MXFP4 one per 32.
 void dot_row(int wdtype, const uint8_t* wrow, const float* sc, int K, const float* x, int ldx, int n, float* out) {
+  if (wdtype == FTM_NVFP4 || wdtype == FTM_MXFP4) {
+    const int group = wdtype == FTM_NVFP4 ? 16 : 32;
+    if (g_avx2) {
+      dot_row_fp4_avx2(wrow, sc, K, group, x, ldx, n, out);
+      return;
+    }
+    for (int r = 0; r < n; ++r) {
+      const float* xr = x + static_cast<size_t>(r) * ldx;
+      float acc = 0.0f;
+      for (int c = 0; c < K; ++c) {
+        const uint8_t b = wrow[c / 2];
+        const uint8_t nib = (c & 1) ? (b >> 4) : (b & 15);
+        const float v = (nib & 8) ? -kE2m1[nib & 7] : kE2m1[nib & 7];
+        acc += v * sc[c / group] * xr[c];
+      }
+      out[r] = acc;
+    }
+    return;
+  }
   if (wdtype == FTM_F32) {
     dot_f32(reinterpret_cast<const float*>(wrow), K, x, ldx, n, out);
     return;
@@ -313,7 +456,7 @@ size_t host_ffn_scratch_bytes(const ftm_layer_desc* L, int64_t rows) {
 }
 
 int host_ffn_supported(int wdtype) {
-  return wdtype == FTM_F32 || wdtype == FTM_BF16 || wdtype == FTM_FP8_E4M3_B128;
+  return wdtype >= FTM_F32 && wdtype <= FTM_MXFP4;
 }
 
 int host_threads(int threads) {
@@ -323,15 +466,32 @@ int host_threads(int threads) {
 }
 
 // Every group's rows through gate/up, SwiGLU and down.  Activations are bf16
-// (fp32 for FTM_F32 layers), one row pointer per row; FP8 layers quantise x and
-// h per 128-group before each contraction, as the GPU kernels do.
+// (fp32 for FTM_F32 layers), one row pointer per row.  Quantised layers
+// quantise x and h before each contraction as the GPU kernels do: FP8 per 128
+// (amax / 448), NVFP4 per 16 with the global scales act_scale = {gx, gh}
+// (NULL: 1, 1), MXFP4 per 32 (E8M0).
 void host_ffn_groups(const ftm_layer_desc* L, const ftm_bank_layout* bl, const HostGroup* groups, int ng,
-                     float* scratch, int threads) {
+                     const float* act_scale, float* scratch, int threads) {
   const int d = L->d, I = L->I, wd = L->wdtype;
-  const bool f32 = wd == FTM_F32;
+  const bool f32 = wd == FTM_F32, fp4 = wd == FTM_NVFP4 || wd == FTM_MXFP4, mx = wd == FTM_MXFP4;
   const size_t elt = f32 ? 4 : 2;
-  const size_t wrow_gu = static_cast<size_t>(d) * (wd == FTM_F32 ? 4 : wd == FTM_BF16 ? 2 : 1);
-  const size_t wrow_d = static_cast<size_t>(I) * (wd == FTM_F32 ? 4 : wd == FTM_BF16 ? 2 : 1);
+  auto row_bytes = [&](int K) -> size_t {
+    return wd == FTM_F32 ? 4u * K : wd == FTM_BF16 ? 2u * K : fp4 ? K / 2u : static_cast<size_t>(K);
+  };
+  const size_t wrow_gu = row_bytes(d), wrow_d = row_bytes(I);
+  const float gx = act_scale ? act_scale[0] : 1.0f, gh = act_scale ? act_scale[1] : 1.0f;
+  auto quant = [&](float* v, int K, float g) {
+    if (wd == FTM_FP8_E4M3_B128) quant_fp8_row(v, K);
+    else if (wd == FTM_NVFP4) quant_nvfp4_row(v, K, g);
+    else if (wd == FTM_MXFP4) quant_mx_row(v, K);
+  };
+  // NVFP4 per-tensor weight scales {gate, up, down}
+  auto s_t = [&](const HostGroup& G, int which) -> float {
+    if (wd != FTM_NVFP4) return 1.0f;
+    float v;
+    std::memcpy(&v, G.bank + bl->s_t_off + 4 * which, 4);
+    return v;
+  };
   std::vector<int64_t> row0(ng + 1, 0);
   for (int g = 0; g < ng; ++g) row0[g + 1] = row0[g] + groups[g].n;
   const int64_t N = row0[ng];
@@ -350,7 +510,7 @@ void host_ffn_groups(const ftm_layer_desc* L, const ftm_bank_layout* bl, const H
     if (f32) std::memcpy(dst, src, sizeof(float) * d);
     else
       for (int c = 0; c < d; ++c) dst[c] = bf16_value(reinterpret_cast<const uint16_t*>(src)[c]);
-    if (wd == FTM_FP8_E4M3_B128) quant_fp8_row(dst, d);
+    quant(dst, d, gx);
   });
   // 2. gate/up + SwiGLU: items of kRowsPerItem intermediate rows of one group
   const int ib = (I + kRowsPerItem - 1) / kRowsPerItem;
@@ -362,21 +522,28 @@ void host_ffn_groups(const ftm_layer_desc* L, const ftm_bank_layout* bl, const H
     const uint8_t* wgu = G.bank + bl->w_gu_off;
     const float* sgu = reinterpret_cast<const float*>(G.bank + bl->s_gu_off);
     const float* x = xs + static_cast<size_t>(row0[g]) * d;
-    std::vector<float> gv(n), uv(n);
+    std::vector<float> gv(n), uv(n), gs(fp4 ? d / 16 : 0), us(fp4 ? d / 16 : 0);
+    const float st_g = s_t(G, 0), st_u = s_t(G, 1);
     for (int i = i0; i < i0 + kRowsPerItem && i < I; ++i) {
       const int up = I + i;
-      dot_row(wd, wgu + static_cast<size_t>(i) * wrow_gu, sgu + static_cast<size_t>(i / 128) * (d / 128), d, x, d, n,
-              gv.data());
-      dot_row(wd, wgu + static_cast<size_t>(up) * wrow_gu, sgu + static_cast<size_t>(up / 128) * (d / 128), d, x, d,
-              n, uv.data());
+      const float* sg = sgu + static_cast<size_t>(i / 128) * (d / 128);
+      const float* su = sgu + static_cast<size_t>(up / 128) * (d / 128);
+      if (fp4) {   // paired order: block i / 64 holds gate rows then the same up rows
+        fp4_row_scales(G.bank + bl->s_gu_off, i / 64, i % 64, d, mx, st_g, gs.data());
+        fp4_row_scales(G.bank + bl->s_gu_off, i / 64, 64 + i % 64, d, mx, st_u, us.data());
+        sg = gs.data();
+        su = us.data();
+      }
+      dot_row(wd, wgu + static_cast<size_t>(i) * wrow_gu, sg, d, x, d, n, gv.data());
+      dot_row(wd, wgu + static_cast<size_t>(up) * wrow_gu, su, d, x, d, n, uv.data());
       for (int r = 0; r < n; ++r) {
         const float gg = gv[r];
         hs[static_cast<size_t>(row0[g] + r) * I + i] = gg / (1.0f + std::exp(-gg)) * uv[r];
       }
     }
   });
-  if (wd == FTM_FP8_E4M3_B128)
-    pool().run(nt, N, [&](int64_t i) { quant_fp8_row(hs + static_cast<size_t>(i) * I, I); });
+  if (wd != FTM_F32 && wd != FTM_BF16)
+    pool().run(nt, N, [&](int64_t i) { quant(hs + static_cast<size_t>(i) * I, I, gh); });
   // 3. down projection, written straight to each row's output
   const int jb = (d + kRowsPerItem - 1) / kRowsPerItem;
   pool().run(nt, static_cast<int64_t>(ng) * jb, [&](int64_t it) {
@@ -387,10 +554,15 @@ void host_ffn_groups(const ftm_layer_desc* L, const ftm_bank_layout* bl, const H
     const uint8_t* wdn = G.bank + bl->w_d_off;
     const float* sd = reinterpret_cast<const float*>(G.bank + bl->s_d_off);
     const float* h = hs + static_cast<size_t>(row0[g]) * I;
-    std::vector<float> yv(n);
+    std::vector<float> yv(n), ds(fp4 ? I / 16 : 0);
+    const float st_d = s_t(G, 2);
     for (int j = j0; j < j0 + kRowsPerItem && j < d; ++j) {
-      dot_row(wd, wdn + static_cast<size_t>(j) * wrow_d, sd + static_cast<size_t>(j / 128) * (I / 128), I, h, I, n,
-              yv.data());
+      const float* sj = sd + static_cast<size_t>(j / 128) * (I / 128);
+      if (fp4) {
+        fp4_row_scales(G.bank + bl->s_d_off, j / 128, j % 128, I, mx, st_d, ds.data());
+        sj = ds.data();
+      }
+      dot_row(wd, wdn + static_cast<size_t>(j) * wrow_d, sj, I, h, I, n, yv.data());
       for (int r = 0; r < n; ++r) {
         uint8_t* dst = G.y[r] + static_cast<size_t>(j) * elt;
         if (f32) std::memcpy(dst, &yv[r], 4);

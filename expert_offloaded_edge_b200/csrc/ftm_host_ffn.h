@@ -19,11 +19,12 @@ struct HostGroup {
 
 // fp32 scratch the host FFN needs for `rows` rows in all.
 size_t host_ffn_scratch_bytes(const ftm_layer_desc* L, int64_t rows);
-// 1 if the host FFN handles this weight dtype (fp32, bf16, FP8 with 128x128 block scales).
+// 1 if the host FFN handles this weight dtype (every ftm_wdtype).
 int host_ffn_supported(int wdtype);
 // threads > 0, else the hardware thread count.
 int host_threads(int threads);
+// act_scale: host fp32[2], the NVFP4 activation global scales {gx, gh}, or NULL (1, 1).
 void host_ffn_groups(const ftm_layer_desc* L, const ftm_bank_layout* bl, const HostGroup* groups, int ng,
-                     float* scratch, int threads);
+                     const float* act_scale, float* scratch, int threads);
 
 }  // namespace ftm

@@ -376,8 +376,8 @@ typedef struct ftm_hybrid {
 size_t ftm_hybrid_workspace_bytes(const ftm_layer_desc* L, int32_t T_max);
 size_t ftm_hybrid_host_bytes(const ftm_layer_desc* L, int32_t T_max);
 
-/* The layer with a cache step split by ftm_hybrid_split (fp32, bf16 and FP8
- * layers; other dtypes return FTM_ERR_UNSUPPORTED).  Sequence:
+/* The layer with a cache step split by ftm_hybrid_split (every weight dtype).
+ * Sequence:
  *  1. route on `stream`;
  *  2. one kernel counts each expert's pairs, finds the misses (against the
  *     cache state before this step), sets q, and gives the host the m - q
@@ -391,9 +391,10 @@ size_t ftm_hybrid_host_bytes(const ftm_layer_desc* L, int32_t T_max);
  *     inserted and their last use is not updated.  The host waits here once;
  *  5. the GPU expert FFN of every group but E, after the copies;
  *  6. meanwhile the host computes group E's rows from the banks in
- *     C->host_pool (the same FFN, FP8 activations quantised per 128 as on the
- *     GPU, fp32 accumulation; ftm_host_expert_ffn) on H->threads threads, then
- *     copies them into place on `stream`;
+ *     C->host_pool (the same FFN with the GPU path's activation quantisation,
+ *     fp32 accumulation; ftm_host_expert_ffn; the NVFP4 global scales are read
+ *     from W->act_scale) on H->threads threads, then copies them into place on
+ *     `stream`;
  *  7. combine, as ftm_moe_layer_forward.
  * Output rows agree with ftm_moe_layer_forward within the dtype's tolerance
  * (bit-identical when m - q = 0).  Arguments as ftm_moe_layer_forward with a
@@ -405,16 +406,20 @@ ftm_status ftm_moe_layer_forward_hybrid(const ftm_layer_desc* L, const ftm_layer
                                         size_t ws_bytes, void* stream, void* copy_stream);
 
 /* The host half of the split on its own: one expert's SwiGLU FFN on the CPU.
- *   bank     host, one expert bank (layout from ftm_get_bank_layout), 16-byte aligned
- *   x, y     host [n][d] (bf16, fp32 for FTM_F32), row-major
- *   scratch  host, >= ftm_host_ffn_scratch_bytes(L, n) bytes, 16-byte aligned
- *   threads  0: every hardware thread
- * fp32, bf16 and FP8 layers; FP8 quantises x and the SwiGLU output per 128
- * elements (scale amax / 448, E4M3 round to nearest even), as the GPU path
- * does.  No CUDA call: runs without a GPU. */
+ *   bank      host, one expert bank (layout from ftm_get_bank_layout), 16-byte aligned
+ *   x, y      host [n][d] (bf16, fp32 for FTM_F32), row-major
+ *   act_scale host fp32[2] = {gx, gh}, the NVFP4 activation global scales (see
+ *             ftm_expert_ffn), or NULL (1, 1); ignored by other dtypes
+ *   scratch   host, >= ftm_host_ffn_scratch_bytes(L, n) bytes, 16-byte aligned
+ *   threads   0: every hardware thread
+ * Every weight dtype, with the GPU path's activation quantisation of x and of
+ * the SwiGLU output: FP8 per 128 elements (amax / 448, E4M3 nearest even),
+ * NVFP4 per 16 (e4m3(amax / (6 g)) scales, E2M1 codes), MXFP4 per 32 (E8M0
+ * scales); fp32 accumulation, outputs rounded to bf16 (fp32 for FTM_F32).  No
+ * CUDA call: runs without a GPU. */
 size_t ftm_host_ffn_scratch_bytes(const ftm_layer_desc* L, int32_t n);
 ftm_status ftm_host_expert_ffn(const ftm_layer_desc* L, const void* bank, const void* x, int32_t n, void* y,
-                               void* scratch, size_t scratch_bytes, int32_t threads);
+                               const float* act_scale, void* scratch, size_t scratch_bytes, int32_t threads);
 
 /* Thread-local warning of the last ftm_moe_layers_forward call ("" if none). */
 const char* ftm_last_warning(void);

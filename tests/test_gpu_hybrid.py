@@ -27,6 +27,10 @@ HYB = {
                         T=(16,), trace_steps=10),
     "bf16": synth.scaled(synth.CONFIGS["35b_decode"], name="hyb_bf16", d=256, I=256, E=32, k=4, S=10,
                          bias="zipf", T=(16,), trace_steps=10, lru=True),
+    "nvfp4": synth.scaled(synth.CONFIGS["753b_nvfp4"], name="hyb_nvfp4", d=256, I=256, E=32, k=4, S=10,
+                          bias="zipf", T=(16,), trace_steps=10, lru=True),
+    "mxfp4": synth.scaled(synth.CONFIGS["753b_mxfp4"], name="hyb_mxfp4", d=256, I=256, E=32, k=4, S=10,
+                          bias="zipf", T=(16,), trace_steps=10, lru=True),
 }
 
 
@@ -79,8 +83,9 @@ def _run_trace(wdtype, bp, bh):
     return totals
 
 
-@pytest.mark.parametrize("wdtype", ["fp8", "bf16"])
-@pytest.mark.parametrize("bp,bh", [(1.0, 1.0), (52.7, 77.3), (3.0, 1.0)])
+@pytest.mark.parametrize("wdtype,bp,bh", [("fp8", 1.0, 1.0), ("fp8", 52.7, 77.3), ("fp8", 3.0, 1.0),
+                                          ("bf16", 1.0, 1.0), ("bf16", 52.7, 77.3), ("nvfp4", 1.0, 1.0),
+                                          ("mxfp4", 1.0, 1.0)])
 def test_hybrid_trace_matches_oracle(wdtype, bp, bh):
     m, host = _run_trace(wdtype, bp, bh)
     assert m > 0 and host > 0     # the split really sent work both ways
