@@ -27,8 +27,11 @@
  *    legacy default stream).  Work is enqueued asynchronously; the entry
  *    points that synchronise the host are the cache steps
  *    (ftm_slot_lookup_update, ftm_slot_stage_layer, ftm_moe_layers_forward,
- *    and ftm_moe_layer_forward with a cache): each must read its miss list
- *    before it can issue the copies, and waits for that kernel alone.
+ *    ftm_moe_layer_forward with a cache, and ftm_moe_layer_forward_hybrid):
+ *    each must read its miss list before it can issue the copies, and waits
+ *    for that kernel alone.  ftm_moe_layer_forward_hybrid and
+ *    ftm_host_expert_ffn also compute on the calling thread (and the library's
+ *    host threads) before they return.
  *  - Arguments are validated before anything is enqueued; on error nothing is
  *    launched, the function returns a non-zero ftm_status and ftm_last_error()
  *    describes it.  No C++ exception crosses this boundary.
