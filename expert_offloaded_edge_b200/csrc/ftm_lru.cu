@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(kLruThreads) lru_step_kernel(const int32_t* __
     for (int q = threadIdx.x; q < P; q += blockDim.x) {
       const int e = ids[q];
       if (e >= 0 && e < E) want[e] = 1;
-      else if (e != skip_id) s_bad = 1;
+      else if (skip_id < 0 || e != skip_id) s_bad = 1;   // skip_id -1: no pair is skipped
     }
   }
   __syncthreads();
