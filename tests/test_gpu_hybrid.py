@@ -119,3 +119,69 @@ def test_hybrid_without_host_bandwidth_is_the_plain_cache_step():
             assert np.array_equal(u, v), f"step {s}"
     assert ftm.ftm_device_status(True) == 0
     del hbuf
+
+
+def _step(dl, h, ws, out, cs, s, T):
+    ftm.ftm_moe_layer_forward_hybrid(dl.desc, dl.weights(), dl.cache, h, dl.hidden(T, s), T, out, ws.ptr, ws.nbytes,
+                                     None, cs)
+    torch.cuda.synchronize()
+
+
+def test_hybrid_capacity_refused_with_state_unchanged():
+    """Two slots: a cold step whose GPU share needs more than two copies is
+    refused with the state untouched; the same step with every miss on the host
+    (Bp = 0) needs no slot and matches the oracle."""
+    cfg = synth.scaled(HYB["fp8"], name="hyb_fp8_s2", S=2)
+    T = cfg.T[0]
+    dl = screened_layer(cfg, T, steps=1)
+    ws = Workspace(ftm.ftm_hybrid_workspace_bytes(dl.desc, T))
+    out = torch.empty((T, cfg.d), dtype=torch.bfloat16, device="cuda")
+    cs = torch.cuda.Stream()
+    x, ids, g = oracle_route(dl, T, 0)
+    m, q, _ = oracle.hybrid_split(oracle.permute(ids, cfg.E)[0], np.zeros(cfg.E, np.int32), 1.0, 0.0)
+    assert q == m > cfg.S
+    h, hbuf = _hybrid(dl.desc, T, 1.0, 0.0)
+    before = _state(dl)
+    with pytest.raises(ftm.FtmError) as ei:
+        _step(dl, h, ws, out, cs, 0, T)
+    assert ei.value.status == ftm.binding.FTM_ERR_CAPACITY and dl.cache.step == 0
+    assert all(np.array_equal(u, v) for u, v in zip(before, _state(dl)))
+    h.pcie_gbs, h.host_gbs = 0.0, 1.0
+    _step(dl, h, ws, out, cs, 0, T)
+    assert (h.last_misses, h.last_host) == (m, m) and dl.cache.step == 1
+    assert all(np.array_equal(u, v) for u, v in zip(before, _state(dl)))   # nothing inserted, nothing touched
+    want = oracle.moe_rows(dl.layer, x, range(T), ids, g)
+    assert_rows_close(to_np_f32(out), want, TOL["fp8"], "all misses on the host")
+    assert ftm.ftm_device_status(True) == 0
+    del hbuf
+
+
+def test_hybrid_copy_failure_rolls_back_then_the_step_succeeds():
+    """A step whose first miss copy cannot be issued (the library's test hook)
+    fails with FTM_ERR_CUDA and leaves the cache as it was; the same step then
+    runs and matches the oracle's split, LRU state and outputs."""
+    cfg = HYB["fp8"]
+    T = cfg.T[0]
+    dl = screened_layer(cfg, T, steps=1)
+    ws = Workspace(ftm.ftm_hybrid_workspace_bytes(dl.desc, T))
+    out = torch.empty((T, cfg.d), dtype=torch.bfloat16, device="cuda")
+    cs = torch.cuda.Stream()
+    h, hbuf = _hybrid(dl.desc, T, 1.0, 1.0)
+    before = _state(dl)
+    dl.cache.fail_before_copy = 1
+    with pytest.raises(ftm.FtmError) as ei:
+        _step(dl, h, ws, out, cs, 0, T)
+    assert ei.value.status == ftm.binding.FTM_ERR_CUDA and dl.cache.step == 0 and dl.cache.fail_before_copy == 0
+    assert all(np.array_equal(u, v) for u, v in zip(before, _state(dl)))
+    _step(dl, h, ws, out, cs, 0, T)
+    x, ids, g = oracle_route(dl, T, 0)
+    counts = oracle.permute(ids, cfg.E)[0]
+    ref = oracle.LRUState(cfg.E, cfg.S)
+    m, q, host = oracle.hybrid_split(counts, ref.slot_of_expert >= 0, 1.0, 1.0)
+    assert q > 0 and (h.last_misses, h.last_host) == (m, m - q)
+    assert ref.update(ids[~np.isin(ids, host)])[0] == 0
+    for u, v in zip(_state(dl), (ref.slot_of_expert, ref.expert_of_slot, ref.last_use)):
+        assert np.array_equal(u, v)
+    assert_rows_close(to_np_f32(out), oracle.moe_rows(dl.layer, x, range(T), ids, g), TOL["fp8"], "after rollback")
+    assert ftm.ftm_device_status(True) == 0
+    del hbuf
