@@ -873,7 +873,12 @@ ftm_status ftm_moe_layer_forward_hybrid(const ftm_layer_desc* L, const ftm_layer
   bank_layout(L, &bl);
   for (int i = 0; i < E; ++i) hh.gidx[i] = -1;
   for (int h = 0; h <= Hn; ++h) hh.gpos[h] = 0;
-  for (int h = 0; h < Hn; ++h) hh.gidx[hh.split[4 + h]] = h;
+  for (int h = 0; h < Hn; ++h) {
+    const int eh = hh.split[4 + h];
+    if (eh < 0 || eh >= E || hh.gidx[eh] != -1)
+      return fail(FTM_ERR_CUDA, "%s: host expert list entry %d (%d) out of range or repeated", who, h, eh);
+    hh.gidx[eh] = h;
+  }
   for (int p = p0; p < P; ++p) {
     const int q = hh.perm[p];
     const int g = (q >= 0 && q < P && hh.ids[q] >= 0 && hh.ids[q] < E) ? hh.gidx[hh.ids[q]] : -1;
