@@ -112,7 +112,9 @@ uint8_t orc_e4m3_encode(float v) {
   return (uint8_t)((v < 0.0f ? 0x80 : 0) | best);
 }
 
-/* Round to the nearest E2M1 value, ties to the even code, saturating at 6. */
+/* Round to the nearest E2M1 value, ties to the even code, saturating at 6.
+ * Magnitudes above 6 take code 7 outright: for huge ones the distances to 4
+ * and to 6 round to the same double, and the tie rule would pick 4. */
 uint8_t orc_e2m1_encode(float v) {
   double a = fabs((double)v);
   int best = 0;
@@ -121,6 +123,7 @@ uint8_t orc_e2m1_encode(float v) {
     double dd = fabs(a - orc_e2m1_value((uint8_t)c));
     if (dd < bd || (dd == bd && (c & 1) == 0)) { bd = dd; best = c; }
   }
+  if (a > 6.0) best = 7;
   if (best == 0) return 0;
   return (uint8_t)((v < 0.0f ? 0x8 : 0) | best);
 }

@@ -55,6 +55,7 @@ def test_e4m3_ties_and_saturation():
     assert enc(3 * 2.0 ** -10) == 2.0 ** -8
     assert enc(460.0) == 448.0
     assert enc(1e6) == 448.0 and enc(-1e6) == -448.0
+    assert enc(1e30) == 448.0 and enc(-3e38) == -448.0   # every distance rounds to the same double here
 
 
 def test_e2m1_grid_and_ties():
@@ -65,7 +66,8 @@ def test_e2m1_grid_and_ties():
         assert oracle.e2m1_encode(v) == c
     enc = lambda v: oracle.e2m1_value(oracle.e2m1_encode(v))
     for v, want in [(0.25, 0.0), (0.75, 1.0), (1.25, 1.0), (1.75, 2.0), (2.5, 2.0),
-                     (3.5, 4.0), (5.0, 4.0), (7.0, 6.0), (100.0, 6.0), (-2.5, -2.0), (-5.0, -4.0),
+                     (3.5, 4.0), (5.0, 4.0), (7.0, 6.0), (100.0, 6.0), (1e30, 6.0), (-3e38, -6.0),
+                     (-2.5, -2.0), (-5.0, -4.0),
                      (0.3, 0.5), (2.6, 3.0)]:
         assert enc(v) == want, (v, enc(v), want)
 
