@@ -222,6 +222,33 @@ __attribute__((target("avx2,fma"))) inline __m256 e4m3x8(const uint8_t* p) {
   return _mm256_or_ps(val, _mm256_castsi256_ps(sign));
 }
 
+// 32 E4M3 codes to fp32 through their exact fp16 images (every E4M3 value is
+// an fp16 value).  Normal codes (exponent field 1..15): fp16 = (code & 0x7F) << 7
+// plus 8 << 10 (the exponent rebased from 7 to 15), so the fp16 high byte is
+// ((code >> 1) & 0x3F) + 0x20 and the low byte (code & 1) << 7.  Exponent field
+// 0 (m * 2^-9, m = code & 7) has a low byte of 0 and a high byte from an
+// 8-entry table: 0, 2^-9, 2^-8, 1.5 2^-8, 2^-7, 1.25 2^-7, 1.5 2^-7, 1.75 2^-7.
+// The sign bit carries over.  Bytes are interleaved into fp16 words and
+// widened with F16C; out[0..3] hold elements 0-7, 8-15, 16-23, 24-31.
+__attribute__((target("avx2,fma,f16c"))) inline void e4m3x32(const uint8_t* p, __m256 out[4]) {
+  const __m256i b = _mm256_loadu_si256(reinterpret_cast<const __m256i*>(p));
+  const __m256i sub_hi = _mm256_setr_epi8(0x00, 0x18, 0x1C, 0x1E, 0x20, 0x21, 0x22, 0x23, 0, 0, 0, 0, 0, 0, 0, 0,
+                                          0x00, 0x18, 0x1C, 0x1E, 0x20, 0x21, 0x22, 0x23, 0, 0, 0, 0, 0, 0, 0, 0);
+  const __m256i sign = _mm256_and_si256(b, _mm256_set1_epi8(static_cast<char>(0x80)));
+  const __m256i hi_n = _mm256_add_epi8(_mm256_and_si256(_mm256_srli_epi16(b, 1), _mm256_set1_epi8(0x3F)),
+                                       _mm256_set1_epi8(0x20));
+  const __m256i hi_s = _mm256_shuffle_epi8(sub_hi, _mm256_and_si256(b, _mm256_set1_epi8(0x07)));
+  const __m256i is_sub = _mm256_cmpeq_epi8(_mm256_and_si256(b, _mm256_set1_epi8(0x78)), _mm256_setzero_si256());
+  const __m256i hi = _mm256_or_si256(_mm256_blendv_epi8(hi_n, hi_s, is_sub), sign);
+  const __m256i lo = _mm256_andnot_si256(is_sub, _mm256_slli_epi16(_mm256_and_si256(b, _mm256_set1_epi8(1)), 7));
+  const __m256i w0 = _mm256_unpacklo_epi8(lo, hi);   // elements 0-7 | 16-23
+  const __m256i w1 = _mm256_unpackhi_epi8(lo, hi);   // elements 8-15 | 24-31
+  out[0] = _mm256_cvtph_ps(_mm256_castsi256_si128(w0));
+  out[1] = _mm256_cvtph_ps(_mm256_castsi256_si128(w1));
+  out[2] = _mm256_cvtph_ps(_mm256_extracti128_si256(w0, 1));
+  out[3] = _mm256_cvtph_ps(_mm256_extracti128_si256(w1, 1));
+}
+
 __attribute__((target("avx2,fma"))) inline __m256 bf16x8(const uint8_t* p) {
   const __m256i v = _mm256_cvtepu16_epi32(_mm_loadu_si128(reinterpret_cast<const __m128i*>(p)));
   return _mm256_castsi256_ps(_mm256_slli_epi32(v, 16));
@@ -231,6 +258,32 @@ __attribute__((target("avx2,fma"))) inline float hsum8(__m256 v) {
   const __m128 s = _mm_add_ps(_mm256_castps256_ps128(v), _mm256_extractf128_ps(v, 1));
   const __m128 t = _mm_add_ps(s, _mm_movehl_ps(s, s));
   return _mm_cvtss_f32(_mm_add_ss(t, _mm_shuffle_ps(t, t, 1)));
+}
+
+const bool g_f16c = __builtin_cpu_supports("avx2") && __builtin_cpu_supports("fma") &&
+                    __builtin_cpu_supports("f16c");
+
+// FP8 rows, NR (1..4) activation rows per pass: 32 weights decoded at a time,
+// four independent accumulators per row, one hsum and scale per 128-block.
+template <int NR>
+__attribute__((target("avx2,fma,f16c"))) void dot_rows_fp8_avx2(const uint8_t* w, const float* sc, int K,
+                                                                const float* x, int ldx, float* out) {
+  float tot[NR] = {};
+  for (int c0 = 0; c0 < K; c0 += 128) {
+    __m256 a[NR][4];
+    for (int r = 0; r < NR; ++r)
+      for (int v = 0; v < 4; ++v) a[r][v] = _mm256_setzero_ps();
+    for (int c = c0; c < c0 + 128; c += 32) {
+      __m256 wv[4];
+      e4m3x32(w + c, wv);
+      for (int r = 0; r < NR; ++r)
+        for (int v = 0; v < 4; ++v)
+          a[r][v] = _mm256_fmadd_ps(wv[v], _mm256_loadu_ps(x + static_cast<size_t>(r) * ldx + c + 8 * v), a[r][v]);
+    }
+    for (int r = 0; r < NR; ++r)
+      tot[r] += sc[c0 / 128] * hsum8(_mm256_add_ps(_mm256_add_ps(a[r][0], a[r][1]), _mm256_add_ps(a[r][2], a[r][3])));
+  }
+  for (int r = 0; r < NR; ++r) out[r] = tot[r];
 }
 
 // NR (1..4) activation rows per pass: each block of 128 weights is decoded
@@ -261,6 +314,18 @@ __attribute__((target("avx2,fma"))) void dot_rows_avx2(const uint8_t* w, const f
 
 template <bool FP8>
 void dot_row_avx2(const uint8_t* w, const float* sc, int K, const float* x, int ldx, int n, float* out) {
+  if (FP8 && g_f16c) {
+    for (int r0 = 0; r0 < n; r0 += 4) {
+      const float* xr = x + static_cast<size_t>(r0) * ldx;
+      switch (n - r0 < 4 ? n - r0 : 4) {
+        case 1: dot_rows_fp8_avx2<1>(w, sc, K, xr, ldx, out + r0); break;
+        case 2: dot_rows_fp8_avx2<2>(w, sc, K, xr, ldx, out + r0); break;
+        case 3: dot_rows_fp8_avx2<3>(w, sc, K, xr, ldx, out + r0); break;
+        default: dot_rows_fp8_avx2<4>(w, sc, K, xr, ldx, out + r0); break;
+      }
+    }
+    return;
+  }
   for (int r0 = 0; r0 < n; r0 += 4) {
     const float* xr = x + static_cast<size_t>(r0) * ldx;
     switch (n - r0 < 4 ? n - r0 : 4) {
