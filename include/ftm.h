@@ -376,6 +376,12 @@ typedef struct ftm_hybrid {
   size_t host_ws_bytes;
 } ftm_hybrid;
 
+/* Device workspace of ftm_moe_layer_forward_hybrid: ftm_workspace_bytes(L, T_max)
+ * plus a few int32 arrays of P = T_max * k and E + 2 entries.  Pinned host
+ * workspace: the read-back ids, permutation and activations, the host rows'
+ * outputs, and the host FFN's fp32 scratch for up to P rows, about
+ * P * (d + I) * 4 + (T_max + P) * d * 2 bytes: the split is meant for decode-sized
+ * batches. */
 size_t ftm_hybrid_workspace_bytes(const ftm_layer_desc* L, int32_t T_max);
 size_t ftm_hybrid_host_bytes(const ftm_layer_desc* L, int32_t T_max);
 
