@@ -811,6 +811,10 @@ ftm_status ftm_moe_layer_forward_hybrid(const ftm_layer_desc* L, const ftm_layer
     return fail(FTM_ERR_INVALID_ARG, "%s: bandwidths must be finite, >= 0 and not both 0 (Bp=%g, Bh=%g)", who,
                 H->pcie_gbs, H->host_gbs);
   if (!host_ffn_supported(L->wdtype)) return fail(FTM_ERR_UNSUPPORTED, "%s: no host FFN for wdtype %d", who, L->wdtype);
+  // the fp32 GPU FFN (SIMT) maps every row to a group by searching the offsets,
+  // so the host experts' rows cannot be left out of it: tensor-core dtypes only
+  if (L->wdtype == FTM_F32)
+    return fail(FTM_ERR_UNSUPPORTED, "%s: fp32 layers have no split (their GPU FFN computes every row)", who);
   if ((s = check_cache(L, C, who))) return s;
   if (T == 0) return ok();
   if (!x || !out) return fail(FTM_ERR_INVALID_ARG, "%s: NULL x / out", who);

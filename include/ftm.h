@@ -385,8 +385,9 @@ typedef struct ftm_hybrid {
 size_t ftm_hybrid_workspace_bytes(const ftm_layer_desc* L, int32_t T_max);
 size_t ftm_hybrid_host_bytes(const ftm_layer_desc* L, int32_t T_max);
 
-/* The layer with a cache step split by ftm_hybrid_split (every weight dtype).
- * Sequence:
+/* The layer with a cache step split by ftm_hybrid_split (bf16, FP8, NVFP4 and
+ * MXFP4 layers; fp32 layers return FTM_ERR_UNSUPPORTED, since their SIMT GPU FFN
+ * computes every row and cannot leave the host's rows out).  Sequence:
  *  1. route on `stream`;
  *  2. one kernel counts each expert's pairs, finds the misses (against the
  *     cache state before this step), sets q, and gives the host the m - q

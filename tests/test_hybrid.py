@@ -158,7 +158,13 @@ def test_host_ffn_rejects_short_scratch_and_bad_bandwidths():
     with pytest.raises(ftm.FtmError) as ei:
         ftm.ftm_host_expert_ffn(desc, 64, 64, 2, 64, 64, nb - 1)
     assert ei.value.status == ftm.binding.FTM_ERR_INVALID_ARG
-    # the layer entry point checks the bandwidths before any device call
+    # the layer entry point refuses fp32 layers (their SIMT GPU FFN computes
+    # every row, the host's too) and bad bandwidths before any device call
+    f32 = ftm.desc_for(HOST_CFGS["f32"])
+    with pytest.raises(ftm.FtmError) as ei:
+        ftm.ftm_moe_layer_forward_hybrid(f32, ftm.LayerWeights(16), ftm.SlotCache(), ftm.Hybrid(1.0, 1.0, 0), 16, 1,
+                                         16, 16, 0, 1, 1)
+    assert ei.value.status == ftm.binding.FTM_ERR_UNSUPPORTED
     h = ftm.Hybrid(0.0, 0.0, 0)
     with pytest.raises(ftm.FtmError) as ei:
         ftm.ftm_moe_layer_forward_hybrid(desc, ftm.LayerWeights(16), ftm.SlotCache(), h, 16, 1, 16, 16, 0, 1, 1)
