@@ -604,12 +604,15 @@ def run_trace(cfg, T, args, dist, local):
     e2e_ms, e2e_value = job_throughput(e0.elapsed_time(e1), K2 * T, dist, "cuda")
     status = ftm.ftm_device_status(True)
     pk, src = peaks()
-    # GEMM1 bytes of one step: (distinct routed experts + the shared expert) x gate/up bytes (+ scales)
+    # The GEMM1 events bracket the launch of a step's hit experts and the shared
+    # expert (the copied misses' launch follows the copies): its bytes are
+    # (hits + 1) x gate/up bytes (+ scales), plus the activations of all rows (an
+    # overcount of under 0.5%: the miss rows' activations go to the later launch)
     g1_w = 2 * cfg.I * cfg.d + bl.s_gu_bytes
     g2_w = cfg.d * cfg.I + bl.s_d_bytes
     groups = distinct / K + 1
     rows = T * cfg.k + T
-    alg_g1 = groups * g1_w + rows * (cfg.d + cfg.I) * 2
+    alg_g1 = (hits / K + 1) * g1_w + rows * (cfg.d + cfg.I) * 2
     layer_bytes = groups * (g1_w + g2_w) + rows * (cfg.d + cfg.I) * 4 + cfg.E * cfg.d * 2 + 2 * T * cfg.d * 2
     g1_ms = float(np.mean(g1))
     ach = alg_g1 / (g1_ms * 1e-3) / 1e9
@@ -619,11 +622,15 @@ def run_trace(cfg, T, args, dist, local):
         "ms_per_step": ms / K, "steps": K, "warmup": W, "dtype": cfg.wdtype,
         "config": workload_config(cfg, T, dist.get_world_size() if dist else 1),
         "l2": "inputs larger than L2: ~1.1 GB of FP8 expert banks touched per step",
-        "launch": "eager (one host sync per step to read the miss list)",
+        "launch": "eager (one host sync per step to read the miss list); the hit experts' FFN runs during the "
+                  "miss copies, the copied misses' FFN after them",
         "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-                     "kernel": "gemm1 (fp8 grouped gate/up + SwiGLU)", "algorithmic_bytes": alg_g1,
+                     "kernel": "gemm1 (fp8 grouped gate/up + SwiGLU) of the hit experts and the shared expert, "
+                               "which runs while the step's misses are copied", "algorithmic_bytes": alg_g1,
                      "peak_source": f"hbm_gbs (of {src})",
-                     "traffic": ncu_traffic(workload_name(cfg, T), "gemm1", cfg.wdtype),
+                     # the stored capture is of the single FFN launch a cache step made before
+                     # the hit experts' launch was split from the misses': none for this one yet
+                     "traffic": ncu_traffic(workload_name(cfg, T), "gemm1-hits", cfg.wdtype),
                      "layer": {"achieved": layer_bytes / (ms / K * 1e-3) / 1e9,
                                "frac": layer_bytes / (ms / K * 1e-3) / 1e9 / peak, "algorithmic_bytes": layer_bytes,
                                "what": "expert banks touched per step over the step time, which includes the "

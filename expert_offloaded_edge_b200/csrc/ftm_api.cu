@@ -21,9 +21,12 @@ cudaError_t launch_permute(const int32_t* ids, int P, int E, int32_t* counts, in
 size_t permute_workspace_bytes(int E, int64_t P);
 size_t lru_workspace_bytes(int E, int S);
 cudaError_t launch_lru_step(const int32_t* ids, int P, int E, int S, int64_t step, int64_t reserve, int key_base,
-                            int skip_id, int32_t* soe, int32_t* eos, int64_t* lu, int32_t* ws, cudaStream_t st);
+                            const int32_t* skip, int32_t* soe, int32_t* eos, int64_t* lu, int32_t* ws,
+                            cudaStream_t st);
 cudaError_t launch_hybrid_split(const int32_t* ids, int P, int E, const int32_t* soe, double bp, double bh,
-                                int32_t* ids2, int32_t* out, cudaStream_t st);
+                                int32_t* ids2, int32_t* skip, int32_t* out, cudaStream_t st);
+cudaError_t launch_miss_relabel(const int32_t* ids, int P, int E, const int32_t* soe, int32_t* ids2,
+                                cudaStream_t st);
 cudaError_t launch_lru_restore(int E, int S, int key_base, int32_t* soe, int32_t* eos, int64_t* lu, int32_t* ws,
                                int n_dirty, cudaStream_t st);
 cudaError_t launch_slot_resize(int E, int S_old, const int32_t* eos_old, const int64_t* lu_old, int S_new,
@@ -148,6 +151,12 @@ struct LayerWs {
   uint8_t* ffn_ws;
   void* y;
   int32_t* lru_ws;
+  // cache steps: group labels (hits e, misses E + e, host experts 2E), their
+  // counts / offsets over 2E + 1 groups and the permutation's workspace
+  int32_t* ids2;
+  int32_t* counts2;
+  int32_t* offsets2;
+  void* perm_ws2;
   size_t total;
 };
 
@@ -166,35 +175,33 @@ LayerWs carve(const ftm_layer_desc* L, int32_t T, uint8_t* base) {
   w.ffn_ws = take(ffn_ws_bytes(L, T));
   w.y = take(static_cast<size_t>(ffn_rows(L, T)) * L->d * act_elt(L));
   w.lru_ws = reinterpret_cast<int32_t*>(take(lru_workspace_bytes(L->E, L->S)));
+  const size_t G2 = 2 * static_cast<size_t>(L->E) + 1;
+  w.ids2 = reinterpret_cast<int32_t*>(take(P * 4));
+  w.counts2 = reinterpret_cast<int32_t*>(take(G2 * 4));
+  w.offsets2 = reinterpret_cast<int32_t*>(take((G2 + 1) * 4));
+  w.perm_ws2 = take(permute_workspace_bytes(static_cast<int>(G2), static_cast<int64_t>(P)));
   w.total = off;
   return w;
 }
 
-// Workspace of the hybrid layer: the layer's own, then the remapped ids, the
-// counts / offsets of E + 1 groups (group E: the pairs of the experts computed
-// on the host), the permutation workspace for E + 1 groups and the split's
-// output.  The layer's perm / inv hold the E + 1-group permutation.
+// Workspace of the hybrid layer: the layer's own (its perm / inv hold the
+// permutation over 2E + 1 groups), then the split's output and the lookup's
+// skip mask.
 struct HybridWs {
   LayerWs w;
-  int32_t* ids2;
-  int32_t* counts2;
-  int32_t* offsets2;
-  void* perm_ws2;
   int32_t* split;
+  int32_t* skip;
   size_t total;
 };
 
 HybridWs carve_hybrid(const ftm_layer_desc* L, int32_t T, uint8_t* base) {
   HybridWs h;
   h.w = carve(L, T, base);
-  const size_t P = static_cast<size_t>(T) * L->k, E = static_cast<size_t>(L->E);
+  const size_t E = static_cast<size_t>(L->E);
   size_t off = h.w.total;
   auto take = [&](size_t bytes) { uint8_t* p = base ? base + off : nullptr; off += al(bytes); return p; };
-  h.ids2 = reinterpret_cast<int32_t*>(take(P * 4));
-  h.counts2 = reinterpret_cast<int32_t*>(take((E + 1) * 4));
-  h.offsets2 = reinterpret_cast<int32_t*>(take((E + 2) * 4));
-  h.perm_ws2 = take(permute_workspace_bytes(L->E + 1, static_cast<int64_t>(P)));
   h.split = reinterpret_cast<int32_t*>(take((4 + E) * 4));
+  h.skip = reinterpret_cast<int32_t*>(take(E * 4));
   h.total = off;
   return h;
 }
@@ -204,7 +211,7 @@ struct HybridHost {
   int32_t* split;          // [4 + E] the split's output
   int32_t* ids;            // [P] routed ids
   int32_t* perm;           // [P] the E + 1-group permutation
-  int32_t* offsets;        // [E + 2]
+  int32_t* offsets;        // [2E + 2]
   uint8_t* x;              // [T][d] activations
   uint8_t* y;              // [P][d] outputs of the host rows
   float* scratch;          // host FFN scratch
@@ -227,7 +234,7 @@ HybridHost carve_host(const ftm_layer_desc* L, int32_t T, void* base_v) {
   h.split = reinterpret_cast<int32_t*>(take((4 + E) * 4));
   h.ids = reinterpret_cast<int32_t*>(take(P * 4));
   h.perm = reinterpret_cast<int32_t*>(take(P * 4));
-  h.offsets = reinterpret_cast<int32_t*>(take((E + 2) * 4));
+  h.offsets = reinterpret_cast<int32_t*>(take((2 * E + 2) * 4));
   h.x = take(static_cast<size_t>(T) * row);
   h.y = take(P * row);
   h.scratch = reinterpret_cast<float*>(take(host_ffn_scratch_bytes(L, static_cast<int64_t>(P))));
@@ -299,18 +306,19 @@ cudaEvent_t list_event() {
 // when given, the miss list read back (the host waits for that kernel only),
 // then one bank copy per miss on `copy_stream` (also after `after`).  Victims
 // are the slots with last_use < reserve.  On a copy failure the state is
-// rolled back (slots a copy may have written left empty).  skip_id >= 0:
-// pairs with that id are not requests (see hybrid_split_kernel).
+// rolled back (slots a copy may have written left empty).  skip (device,
+// [E], nullable): experts flagged nonzero are not requests (see
+// hybrid_split_kernel).
 ftm_status cache_step(const ftm_layer_desc* L, ftm_slot_cache* C, const int32_t* ids, int P, int64_t reserve,
                       int32_t* ws, cudaStream_t lru_stream, cudaStream_t copy_stream, cudaEvent_t after,
-                      int* misses_out, int skip_id = -1) {
+                      int* misses_out, const int32_t* skip = nullptr) {
   *misses_out = 0;
   cudaError_t e;
   // the step rewrites the entries of the keys it evicts: the compute that
   // reads them (done when `after` completes) must be over first
   if (after && (e = cudaStreamWaitEvent(lru_stream, after, 0)) != cudaSuccess) return cuda_fail(e, "lru stream wait");
   prof_mark(FTM_K_LRU, lru_stream, false);
-  e = launch_lru_step(ids, P, L->E, L->S, C->step, reserve, C->key_base, skip_id, C->slot_of_expert,
+  e = launch_lru_step(ids, P, L->E, L->S, C->step, reserve, C->key_base, skip, C->slot_of_expert,
                                   C->expert_of_slot, C->last_use, ws, lru_stream);
   prof_mark(FTM_K_LRU, lru_stream, true);
   if (e != cudaSuccess) return cuda_fail(e, "lru step launch");
@@ -365,6 +373,43 @@ ftm_status cache_step(const ftm_layer_desc* L, ftm_slot_cache* C, const int32_t*
   C->step += 1;
   *misses_out = misses;
   return FTM_OK;
+}
+
+// The expert FFN of a cache step in two launches over the permutation of 2E
+// groups (w.offsets2, labels from miss_relabel_kernel or hybrid_split_kernel):
+// groups 0..E-1, the hit experts (and the shared expert), at once, so their
+// tiles run while the misses are copied; after the copies (an event on the
+// copy stream), groups E..2E-1, the copied misses, with no shared expert.  Both
+// write Y at the pairs' positions, so the combine reads it through w.inv.  The
+// profile events of the FFN's kernels bracket the first launch only.
+ftm_status ffn_hits_then_misses(const ftm_layer_desc* L, const ftm_layer_weights* W, const ftm_slot_cache* C,
+                                const void* x, int T, const LayerWs& w, int misses, cudaStream_t cs,
+                                cudaStream_t ps) {
+  const int32_t* soe = C->slot_of_expert + C->key_base;
+  ftm_status s = ftm_expert_ffn(L, x, T, w.offsets2, w.perm, soe, C->slot_pool, W->shared_bank, W->act_scale, w.y,
+                                w.ffn_ws, ffn_ws_bytes(L, T), cs);
+  if (s || misses == 0) return s;
+  cudaError_t e;
+  cudaEvent_t ev = copy_event();
+  if (!ev) return fail(FTM_ERR_CUDA, "could not create the copy event");
+  if ((e = cudaEventRecord(ev, ps)) != cudaSuccess) return cuda_fail(e, "copy event record");
+  if ((e = cudaStreamWaitEvent(cs, ev, 0)) != cudaSuccess) return cuda_fail(e, "copy event wait");
+  ftm_layer_desc Lm = *L;
+  Lm.has_shared = 0;
+  const int hooks[3] = {FTM_K_GATHER, FTM_K_GEMM1, FTM_K_GEMM2};
+  cudaEvent_t saved[3][2];
+  for (int i = 0; i < 3; ++i) {
+    saved[i][0] = g_prof[hooks[i]][0];
+    saved[i][1] = g_prof[hooks[i]][1];
+    g_prof[hooks[i]][0] = g_prof[hooks[i]][1] = nullptr;
+  }
+  s = ftm_expert_ffn(&Lm, x, T, w.offsets2 + L->E, w.perm, soe, C->slot_pool, nullptr, W->act_scale, w.y, w.ffn_ws,
+                     ffn_ws_bytes(&Lm, T), cs);
+  for (int i = 0; i < 3; ++i) {
+    g_prof[hooks[i]][0] = saved[i][0];
+    g_prof[hooks[i]][1] = saved[i][1];
+  }
+  return s;
 }
 
 thread_local char g_warn[256] = "";
@@ -663,12 +708,31 @@ ftm_status ftm_moe_layer_forward(const ftm_layer_desc* L, const ftm_layer_weight
   LayerWs w = carve(L, T, static_cast<uint8_t*>(workspace));
   if ((s = check_ws(workspace, ws_bytes, w.total, "ftm_moe_layer_forward"))) return s;
   if ((s = ftm_route(L, x, T, W->w_router, W->router_bias, w.ids, w.gates, stream))) return s;
+  if (C && L->wdtype != FTM_F32) {
+    // cache step with the hit experts' FFN overlapping the miss copies: the
+    // pairs labelled against the residency before the lookup (misses as E + e)
+    // and permuted over 2E groups, then the lookup (the host waits for it), the
+    // copies, and the FFN in two launches (ffn_hits_then_misses)
+    if ((s = check_cache(L, C, "ftm_moe_layer_forward"))) return s;
+    cudaStream_t cs = S_(stream), ps = S_(copy_stream);
+    const int P = T * L->k, E = L->E;
+    cudaError_t e = launch_miss_relabel(w.ids, P, E, C->slot_of_expert + C->key_base, w.ids2, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "relabel launch");
+    prof_mark(FTM_K_PERMUTE, cs, false);
+    e = launch_permute(w.ids2, P, 2 * E, w.counts2, w.offsets2, w.perm, w.inv, w.perm_ws2, cs);
+    prof_mark(FTM_K_PERMUTE, cs, true);
+    if (e != cudaSuccess) return cuda_fail(e, "permute launch");
+    int misses = 0;
+    if ((s = cache_step(L, C, w.ids, P, C->step, w.lru_ws, cs, ps, nullptr, &misses))) return s;
+    if ((s = ffn_hits_then_misses(L, W, C, x, T, w, misses, cs, ps))) return s;
+    return ftm_combine(L, w.y, w.inv, w.gates, T, out, stream);
+  }
   if ((s = ftm_permute(L, w.ids, T, w.counts, w.offsets, w.perm, w.inv, w.perm_ws,
                        permute_workspace_bytes(L->E, static_cast<int64_t>(T) * L->k), stream)))
     return s;
   const void* pool = W->slot_pool;
   const int32_t* soe = W->slot_of_expert;
-  if (C) {
+  if (C) {   // fp32 layers: their SIMT FFN computes every row, so it runs once, after the copies
     if ((s = ftm_slot_lookup_update(L, C, w.ids, T, w.lru_ws, lru_workspace_bytes(L->E, L->S), stream, copy_stream)))
       return s;
     pool = C->slot_pool;
@@ -678,8 +742,7 @@ ftm_status ftm_moe_layer_forward(const ftm_layer_desc* L, const ftm_layer_weight
   if ((s = ftm_expert_ffn(L, x, T, w.offsets, w.perm, soe, pool, W->shared_bank, W->act_scale, w.y, w.ffn_ws,
                           ffn_ws_bytes(L, T),
                           stream)))
-    return s;
-  return ftm_combine(L, w.y, w.inv, w.gates, T, out, stream);
+    return s;  return ftm_combine(L, w.y, w.inv, w.gates, T, out, stream);
 }
 
 ftm_status ftm_moe_layers_forward(const ftm_layer_desc* L, int32_t n_layers, const ftm_layer_weights* W,
@@ -837,18 +900,18 @@ ftm_status ftm_moe_layer_forward_hybrid(const ftm_layer_desc* L, const ftm_layer
   if ((s = ftm_route(L, x, T, W->w_router, W->router_bias, w.ids, w.gates, stream))) return s;
   // the split (against the residency before this step), then the pairs by
   // expert with the host experts' pairs as one last group E
-  if ((e = launch_hybrid_split(w.ids, P, E, C->slot_of_expert + C->key_base, H->pcie_gbs, H->host_gbs, hw.ids2,
-                               hw.split, cs)) != cudaSuccess)
+  if ((e = launch_hybrid_split(w.ids, P, E, C->slot_of_expert + C->key_base, H->pcie_gbs, H->host_gbs, w.ids2,
+                               hw.skip, hw.split, cs)) != cudaSuccess)
     return cuda_fail(e, "split launch");
   prof_mark(FTM_K_PERMUTE, cs, false);
-  e = launch_permute(hw.ids2, P, E + 1, hw.counts2, hw.offsets2, w.perm, w.inv, hw.perm_ws2, cs);
+  e = launch_permute(w.ids2, P, 2 * E + 1, w.counts2, w.offsets2, w.perm, w.inv, w.perm_ws2, cs);
   prof_mark(FTM_K_PERMUTE, cs, true);
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   // what the host needs, read back before the lookup's own read (same stream)
   const bool gscale = L->wdtype == FTM_NVFP4 && W->act_scale;   // the NVFP4 activation global scales
   struct { void* dst; const void* src; size_t n; } rd[6] = {
       {hh.split, hw.split, (4 + static_cast<size_t>(E)) * 4}, {hh.ids, w.ids, static_cast<size_t>(P) * 4},
-      {hh.perm, w.perm, static_cast<size_t>(P) * 4}, {hh.offsets, hw.offsets2, (static_cast<size_t>(E) + 2) * 4},
+      {hh.perm, w.perm, static_cast<size_t>(P) * 4}, {hh.offsets, w.offsets2, (2 * static_cast<size_t>(E) + 2) * 4},
       {hh.x, x, static_cast<size_t>(T) * row}, {hh.act, W->act_scale, gscale ? 2 * sizeof(float) : 0}};
   for (auto& c : rd)
     if (c.n && (e = cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
@@ -856,20 +919,11 @@ ftm_status ftm_moe_layer_forward_hybrid(const ftm_layer_desc* L, const ftm_layer
   // the cache step over the GPU's share: hits and the q copied misses (the
   // host waits here for the lookup, and with it for the reads above)
   int misses = 0;
-  if ((s = cache_step(L, C, hw.ids2, P, C->step, w.lru_ws, cs, ps, nullptr, &misses, E))) return s;
-  if (misses > 0) {
-    cudaEvent_t ev = copy_event();
-    if (!ev) return fail(FTM_ERR_CUDA, "could not create the copy event");
-    if ((e = cudaEventRecord(ev, ps)) != cudaSuccess) return cuda_fail(e, "copy event record");
-    if ((e = cudaStreamWaitEvent(cs, ev, 0)) != cudaSuccess) return cuda_fail(e, "copy event wait");
-  }
-  // the GPU's groups (the host experts' groups 0..E-1 are empty)
-  const int32_t* soe = C->slot_of_expert + C->key_base;
-  if ((s = ftm_expert_ffn(L, x, T, hw.offsets2, w.perm, soe, C->slot_pool, W->shared_bank, W->act_scale, w.y, w.ffn_ws,
-                          ffn_ws_bytes(L, T), stream)))
-    return s;
-  // meanwhile the host experts' pairs, positions offsets2[E] .. P-1, on the host
-  const int m = hh.split[0], Hn = hh.split[2], rows = hh.split[3], p0 = hh.offsets[E];
+  if ((s = cache_step(L, C, w.ids, P, C->step, w.lru_ws, cs, ps, nullptr, &misses, hw.skip))) return s;
+  // the GPU's groups: hits while the copies run, the copied misses after them
+  if ((s = ffn_hits_then_misses(L, W, C, x, T, w, misses, cs, ps))) return s;
+  // meanwhile the host experts' pairs, positions offsets2[2E] .. P-1, on the host
+  const int m = hh.split[0], Hn = hh.split[2], rows = hh.split[3], p0 = hh.offsets[2 * E];
   if (Hn < 0 || Hn > E || p0 < 0 || p0 + rows != P)
     return fail(FTM_ERR_CUDA, "%s: inconsistent split (H=%d, rows=%d, first host position %d, P=%d)", who, Hn, rows,
                 p0, P);

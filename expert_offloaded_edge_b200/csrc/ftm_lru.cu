@@ -38,10 +38,11 @@ __device__ __forceinline__ int64_t* lru_backup_lu(int32_t* ws, int E, int S) {
   return reinterpret_cast<int64_t*>(reinterpret_cast<uint8_t*>(ws) + off);
 }
 
-// skip_id >= 0: pairs whose id equals it are not requests (the experts the
-// bandwidth-adaptive split computes on the host carry that id).
+// skip (nullable, [E]): experts flagged nonzero are not requests even when
+// routed (the experts the bandwidth-adaptive split computes on the host).
 __global__ void __launch_bounds__(kLruThreads) lru_step_kernel(const int32_t* __restrict__ ids, int P, int E, int S,
-                                                               int64_t step, int64_t reserve, int key_base, int skip_id,
+                                                               int64_t step, int64_t reserve, int key_base,
+                                                               const int32_t* __restrict__ skip,
                                                                int32_t* __restrict__ slot_of_key,
                                                                int32_t* __restrict__ key_of_slot,
                                                                int64_t* __restrict__ last_use,
@@ -62,8 +63,11 @@ __global__ void __launch_bounds__(kLruThreads) lru_step_kernel(const int32_t* __
   if (ids) {
     for (int q = threadIdx.x; q < P; q += blockDim.x) {
       const int e = ids[q];
-      if (e >= 0 && e < E) want[e] = 1;
-      else if (skip_id < 0 || e != skip_id) s_bad = 1;   // skip_id -1: no pair is skipped
+      if (e >= 0 && e < E) {
+        if (!skip || !skip[e]) want[e] = 1;
+      } else {
+        s_bad = 1;
+      }
     }
   }
   __syncthreads();
@@ -154,13 +158,37 @@ __global__ void __launch_bounds__(kLruThreads) lru_step_kernel(const int32_t* __
 }
 
 cudaError_t launch_lru_step(const int32_t* ids, int P, int E, int S, int64_t step, int64_t reserve, int key_base,
-                            int skip_id, int32_t* soe, int32_t* eos, int64_t* lu, int32_t* ws, cudaStream_t st) {
+                            const int32_t* skip, int32_t* soe, int32_t* eos, int64_t* lu, int32_t* ws,
+                            cudaStream_t st) {
   const size_t smem = sizeof(int32_t) * (2 * static_cast<size_t>(E) + 1 + 2 * S);
   cudaError_t err =
       cudaFuncSetAttribute(lru_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   return launch_pdl(lru_step_kernel, dim3(1), dim3(kLruThreads), smem, st, ids, P, E, S, step, reserve, key_base,
-                    skip_id, soe, eos, lu, ws);
+                    skip, soe, eos, lu, ws);
+}
+
+// Group labels of a cache step whose expert FFN runs in two launches, the hit
+// experts' while the misses are copied and the copied misses' after: a pair
+// routed to a resident expert e keeps label e, one routed to an expert not in
+// the cache (the state before this step's lookup) gets E + e.  A permutation
+// over 2E groups then holds the hits at positions 0 .. P_hit - 1 and the
+// misses, still grouped by expert, after them.  Ids outside [0, E) are copied
+// through (the lookup refuses the step before they are used).
+__global__ void miss_relabel_kernel(const int32_t* __restrict__ ids, int P, int E, const int32_t* __restrict__ soe,
+                                    int32_t* __restrict__ ids2) {
+  pdl_wait();
+  pdl_trigger();
+  for (int q = blockIdx.x * blockDim.x + threadIdx.x; q < P; q += gridDim.x * blockDim.x) {
+    const int e = ids[q];
+    ids2[q] = (e >= 0 && e < E && soe[e] < 0) ? E + e : e;
+  }
+}
+
+cudaError_t launch_miss_relabel(const int32_t* ids, int P, int E, const int32_t* soe, int32_t* ids2,
+                                cudaStream_t st) {
+  const int blocks = P > 0 ? (P + 255) / 256 < 148 ? (P + 255) / 256 : 148 : 1;
+  return launch_pdl(miss_relabel_kernel, dim3(blocks), dim3(256), 0, st, ids, P, E, soe, ids2);
 }
 
 // ---------------------------------------------------------------------------
@@ -175,14 +203,17 @@ cudaError_t launch_lru_step(const int32_t* ids, int P, int E, int S, int64_t ste
 // up), computed in fp64 as floor(m * Bp / (Bp + Bh) + 0.5).  The host takes the
 // m - q misses with the fewest pairs (ties: the lower expert id): its cost per
 // expert grows with the rows, a copy's does not.
-//   ids2[q] = E for a pair of a host expert, else ids[q] (ids outside [0, E)
-//   copied through for the lookup to reject); out (int32): [0] m, [1] q,
-//   [2] host experts H = m - q, [3] their pairs, [4 .. 4+H) the host experts
-//   in order (fewest pairs first).
+//   ids2[q] = 2E for a pair of a host expert, E + e for one of an expert
+//   copied this step, e for a resident expert (ids outside [0, E) copied
+//   through; the lookup rejects them); skip[e] = 1 for a host expert, else 0
+//   (the lookup's mask); out (int32): [0] m, [1] q, [2] host experts H = m - q,
+//   [3] their pairs, [4 .. 4+H) the host experts in order (fewest pairs
+//   first).
 // One block; the residency read is the state before the step's lookup.
 __global__ void __launch_bounds__(kLruThreads) hybrid_split_kernel(const int32_t* __restrict__ ids, int P, int E,
                                                                    const int32_t* __restrict__ soe, double bp,
                                                                    double bh, int32_t* __restrict__ ids2,
+                                                                   int32_t* __restrict__ skip,
                                                                    int32_t* __restrict__ out) {
   extern __shared__ int32_t sm[];
   int32_t* cnt = sm;          // [E] pairs per expert
@@ -225,6 +256,7 @@ __global__ void __launch_bounds__(kLruThreads) hybrid_split_kernel(const int32_t
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const int r = rank[e];
     host[e] = r >= 0 && r < H;
+    skip[e] = host[e];
     if (host[e]) {
       out[4 + r] = e;
       atomicAdd(&s_rows, cnt[e]);
@@ -233,15 +265,16 @@ __global__ void __launch_bounds__(kLruThreads) hybrid_split_kernel(const int32_t
   __syncthreads();
   for (int q = threadIdx.x; q < P; q += blockDim.x) {
     const int e = ids[q];
-    ids2[q] = (e >= 0 && e < E && host[e]) ? E : e;
+    ids2[q] = (e >= 0 && e < E) ? (host[e] ? 2 * E : rank[e] >= 0 ? E + e : e) : e;
   }
   if (threadIdx.x == 0) { out[0] = s_m; out[1] = s_m - H; out[2] = H; out[3] = s_rows; }
 }
 
 cudaError_t launch_hybrid_split(const int32_t* ids, int P, int E, const int32_t* soe, double bp, double bh,
-                                int32_t* ids2, int32_t* out, cudaStream_t st) {
+                                int32_t* ids2, int32_t* skip, int32_t* out, cudaStream_t st) {
   const size_t smem = sizeof(int32_t) * 3 * static_cast<size_t>(E);
-  return launch_pdl(hybrid_split_kernel, dim3(1), dim3(kLruThreads), smem, st, ids, P, E, soe, bp, bh, ids2, out);
+  return launch_pdl(hybrid_split_kernel, dim3(1), dim3(kLruThreads), smem, st, ids, P, E, soe, bp, bh, ids2, skip,
+                    out);
 }
 
 // Rollback of a step whose miss copies could not all be issued: the state
