@@ -310,7 +310,12 @@ typedef struct ftm_layer_weights {
  *   C          NULL for a resident layer (every expert in W->slot_pool at
  *              W->slot_of_expert[e]); otherwise the LRU cache (its slot_pool and
  *              slot_of_expert are used, and the call synchronises once, see
- *              ftm_slot_lookup_update)
+ *              ftm_slot_lookup_update).  With a cache (bf16 / FP8 / FP4
+ *              layers) the expert FFN runs in two launches: the experts that
+ *              were resident (and the shared expert) right after the lookup,
+ *              while the misses are copied on copy_stream, then the copied
+ *              misses once their copies are done; fp32 layers run one FFN
+ *              after the copies
  *   x, out     device [T][d]
  *   workspace  device, >= ftm_workspace_bytes(L, T) bytes, 256-aligned
  *   copy_stream  stream for the miss copies (only used with a cache) */
@@ -466,7 +471,9 @@ typedef enum ftm_kernel_id {
 /* While set on the calling thread, every launch of kernel `which` is bracketed
  * by cudaEventRecord(start) / cudaEventRecord(stop) on the stream it is
  * launched on (events are cudaEvent_t passed as void*, created by the caller
- * with timing enabled).  NULL events clear the hook.  Nothing else changes. */
+ * with timing enabled).  NULL events clear the hook.  Nothing else changes.
+ * In a layer call with a cache, the gather and GEMM events bracket the first
+ * of the two FFN launches (the resident experts' and the shared expert's). */
 ftm_status ftm_set_profile_events(int32_t which, void* start_event, void* stop_event);
 
 /* Number of kernel launches the library has enqueued in this process so far
