@@ -169,3 +169,41 @@ def test_host_ffn_rejects_short_scratch_and_bad_bandwidths():
     with pytest.raises(ftm.FtmError) as ei:
         ftm.ftm_moe_layer_forward_hybrid(desc, ftm.LayerWeights(16), ftm.SlotCache(), h, 16, 1, 16, 16, 0, 1, 1)
     assert ei.value.status == ftm.binding.FTM_ERR_INVALID_ARG
+
+
+def test_host_ffn_concurrent_callers_match_sequential_results():
+    """The host FFN's thread pool is shared by the process: calls from several
+    host threads at once (ctypes releases the GIL) must each get the result a
+    call on its own gets."""
+    import threading
+
+    cfg = HOST_CFGS["fp8"]
+    layer = synth.Layer(cfg, 0)
+    desc = ftm.desc_for(cfg)
+    bl = ftm.ftm_get_bank_layout(desc)
+    n = 3
+    jobs = []
+    for e in range(4):
+        bank = _aligned(bl.bank_bytes)
+        pack_bank(desc, layer.expert(e), bl, out=bank)
+        x = np.ascontiguousarray(layer.hidden_storage(n, e))
+        nb = ftm.ftm_host_ffn_scratch_bytes(desc, n)
+        want = np.zeros_like(x)
+        ftm.ftm_host_expert_ffn(desc, bank, x, n, want, _aligned(nb), nb, threads=4)
+        jobs.append((bank, x, want, nb))
+    errors = []
+
+    def worker(j):
+        bank, x, want, nb = jobs[j % 4]
+        for _ in range(5):
+            y = np.zeros_like(x)
+            ftm.ftm_host_expert_ffn(desc, bank, x, n, y, _aligned(nb), nb, threads=4)
+            if not np.array_equal(y, want):
+                errors.append(j)
+
+    threads = [threading.Thread(target=worker, args=(j,)) for j in range(8)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors
