@@ -20,9 +20,12 @@
  *  - Pointers marked "device" are CUDA device pointers, "host" are host
  *    pointers.  The caller owns every buffer; the library never allocates device
  *    or host memory and keeps no per-call state beyond a thread-local error
- *    string and one cached CUDA event per thread for the miss-copy ordering
- *    (and, once the host FFN of the miss split has run, its pool of host
- *    threads).
+ *    string and one cached CUDA event per thread for the miss-copy ordering.
+ *    The one exception is the host FFN of the miss split
+ *    (ftm_moe_layer_forward_hybrid, ftm_host_expert_ffn): it allocates small
+ *    host buffers per call (row tables, and per work item the partial sums of
+ *    its rows and one weight row's scales), and keeps a pool of host threads
+ *    from its first call to process exit.
  *  - `stream` arguments are cudaStream_t values passed as void* (NULL = the
  *    legacy default stream).  Work is enqueued asynchronously; the entry
  *    points that synchronise the host are the cache steps
