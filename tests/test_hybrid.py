@@ -207,3 +207,20 @@ def test_host_ffn_concurrent_callers_match_sequential_results():
     for t in threads:
         t.join()
     assert not errors
+
+
+def test_split_workspace_queries():
+    for name in ("284b_trace", "35b_decode", "753b_nvfp4"):
+        desc = ftm.desc_for(synth.CONFIGS[name])
+        prev_d = prev_h = 0
+        for T in (1, 16, 64, 512):
+            wd = ftm.ftm_hybrid_workspace_bytes(desc, T)
+            wh = ftm.ftm_hybrid_host_bytes(desc, T)
+            assert wd >= ftm.ftm_workspace_bytes(desc, T) > 0
+            assert wd >= prev_d and wh > prev_h
+            # the host FFN scratch for every pair is part of the host buffer
+            assert wh >= ftm.ftm_host_ffn_scratch_bytes(desc, T * desc.k)
+            prev_d, prev_h = wd, wh
+    bad = ftm.LayerDesc(100, 8, 2, 128, 0, 8, ftm.FTM_BF16, 0)   # d not a multiple of 128
+    assert ftm.ftm_hybrid_workspace_bytes(bad, 16) == 0 and ftm.ftm_hybrid_host_bytes(bad, 16) == 0
+    assert ftm.ftm_host_ffn_scratch_bytes(bad, 4) == 0
